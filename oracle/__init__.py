@@ -1,0 +1,187 @@
+"""Oracle for grouped / depthwise convolution -- TEST INFRASTRUCTURE ONLY.
+
+A plain fp64 CPU implementation (``oracle.c``, nested loops, OpenMP over the outermost
+output loop) of what the CUDA library computes. Only the tests, the package smoke check
+and the benchmark's CPU-baseline leg import this module; the product path never does,
+and the two share no code.
+
+Definitions followed (see the header of ``oracle.c`` for the full statement):
+  * grouped conv2d -- "Grouped convolutions" (neon issue #296): channels, filters and
+    outputs split into groups with no cross-group connections, group-major channel
+    order; cross-correlation with zero padding as ``F.conv2d(..., groups=g)`` in
+    "F.conv2d runs x15 slower in mixed-precision/half-precision mode";
+  * depthwise conv1d on (batch, steps, channels), forward and backward -- "Investigate
+    custom Triton kernels for depthwise-separable convolutions in Conformer".
+
+Every function takes and returns float64 numpy arrays (inputs are the exact values the
+GPU receives, widened to fp64).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+NCHW = 0
+NHWC = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` with gcc (OpenMP on)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
+                               "-Wall", "-Wno-unknown-pragmas", _SRC, "-o", tmp])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _configure(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    L, I, P = ctypes.c_long, ctypes.c_int, ctypes.c_void_p
+    lib.oracle_conv2d.argtypes = [P, P, P, P] + [L] * 11 + [I]
+    lib.oracle_conv2d.restype = I
+    lib.oracle_conv2d_points.argtypes = [P, P, P, P, P, L] + [L] * 11 + [I]
+    lib.oracle_conv2d_points.restype = I
+    for name in ("oracle_dwconv1d_fwd", "oracle_dwconv1d_bwd_data",
+                 "oracle_dwconv1d_bwd_weight"):
+        f = getattr(lib, name)
+        f.argtypes = [P, P, P] + [L] * 6
+        f.restype = I
+    lib.oracle_conv_out_extent.argtypes = [L] * 5
+    lib.oracle_conv_out_extent.restype = L
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = I
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _configure(ctypes.CDLL(build()))
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def out_extent(size: int, k: int, stride: int, pad: int, dilation: int) -> int:
+    return int(_load().oracle_conv_out_extent(size, k, stride, pad, dilation))
+
+
+def conv2d_out_shape(x_shape, w_shape, stride, pad, dilation, groups, layout):
+    if layout == NCHW:
+        N, C_in, H, W = x_shape
+        C_out, _, kH, kW = w_shape
+    else:
+        N, H, W, C_in = x_shape
+        C_out, kH, kW, _ = w_shape
+    Ho = out_extent(H, kH, stride, pad, dilation)
+    Wo = out_extent(W, kW, stride, pad, dilation)
+    return (N, C_out, Ho, Wo) if layout == NCHW else (N, Ho, Wo, C_out)
+
+
+def _conv_args(x, w, groups, layout):
+    if layout == NCHW:
+        N, C_in, H, W = x.shape
+        C_out, cpg_in, kH, kW = w.shape
+    elif layout == NHWC:
+        N, H, W, C_in = x.shape
+        C_out, kH, kW, cpg_in = w.shape
+    else:
+        raise ValueError("layout must be NCHW (0) or NHWC (1)")
+    if groups <= 0 or C_in % groups or C_out % groups or cpg_in * groups != C_in:
+        raise ValueError("inconsistent groups / channel counts")
+    return N, C_in, H, W, C_out, kH, kW
+
+
+def conv2d(x, w, bias=None, stride=1, pad=0, dilation=1, groups=1, layout=NCHW):
+    """Grouped conv2d in fp64; x, w, y in the layouts of ``layout``."""
+    x, w = _f64(x), _f64(w)
+    b = None if bias is None else _f64(bias)
+    N, C_in, H, W, C_out, kH, kW = _conv_args(x, w, groups, layout)
+    y = np.empty(conv2d_out_shape(x.shape, w.shape, stride, pad, dilation, groups, layout))
+    rc = _load().oracle_conv2d(_ptr(x), _ptr(w), _ptr(b), _ptr(y), N, C_in, H, W, C_out, kH,
+                               kW, stride, pad, dilation, groups, layout)
+    if rc != 0:
+        raise ValueError("oracle_conv2d rejected the shape")
+    return y
+
+
+def conv2d_points(x, w, idx, bias=None, stride=1, pad=0, dilation=1, groups=1, layout=NCHW):
+    """Outputs of grouped conv2d at idx[i] = (n, co, ho, wo) (logical indices)."""
+    x, w = _f64(x), _f64(w)
+    b = None if bias is None else _f64(bias)
+    idx = np.ascontiguousarray(idx, dtype=np.int64).reshape(-1, 4)
+    N, C_in, H, W, C_out, kH, kW = _conv_args(x, w, groups, layout)
+    out = np.empty(idx.shape[0])
+    rc = _load().oracle_conv2d_points(_ptr(x), _ptr(w), _ptr(b), _ptr(out), _ptr(idx),
+                                      idx.shape[0], N, C_in, H, W, C_out, kH, kW, stride, pad,
+                                      dilation, groups, layout)
+    if rc != 0:
+        raise ValueError("oracle_conv2d_points rejected the shape or an index")
+    return out
+
+
+def _conv1d_check(x_shape, w_shape):
+    B, T, C = x_shape
+    C2, K = w_shape
+    if C2 != C:
+        raise ValueError("w must be [C, K]")
+    return B, T, C, K
+
+
+def dwconv1d_fwd(x, w, pad_left, pad_right):
+    """y[b,t,c] = sum_k w[c,k] x[b,t+k-pad_left,c] on (batch, steps, channels)."""
+    x, w = _f64(x), _f64(w)
+    B, T, C, K = _conv1d_check(x.shape, w.shape)
+    T_out = T + pad_left + pad_right - K + 1
+    y = np.empty((B, T_out, C))
+    if _load().oracle_dwconv1d_fwd(_ptr(x), _ptr(w), _ptr(y), B, T, C, K, pad_left,
+                                   pad_right) != 0:
+        raise ValueError("oracle_dwconv1d_fwd rejected the shape")
+    return y
+
+
+def dwconv1d_bwd_data(dy, w, T, pad_left, pad_right):
+    """dx for dwconv1d_fwd, given dy [B, T_out, C] and the input length T."""
+    dy, w = _f64(dy), _f64(w)
+    B, T_out, C = dy.shape
+    K = w.shape[1]
+    if T_out != T + pad_left + pad_right - K + 1:
+        raise ValueError("dy has the wrong number of steps")
+    dx = np.empty((B, T, C))
+    if _load().oracle_dwconv1d_bwd_data(_ptr(dy), _ptr(w), _ptr(dx), B, T, C, K, pad_left,
+                                        pad_right) != 0:
+        raise ValueError("oracle_dwconv1d_bwd_data rejected the shape")
+    return dx
+
+
+def dwconv1d_bwd_weight(x, dy, K, pad_left, pad_right):
+    """dw [C, K] for dwconv1d_fwd, given x [B, T, C] and dy [B, T_out, C]."""
+    x, dy = _f64(x), _f64(dy)
+    B, T, C = x.shape
+    if dy.shape != (B, T + pad_left + pad_right - K + 1, C):
+        raise ValueError("dy has the wrong shape")
+    dw = np.empty((C, K))
+    if _load().oracle_dwconv1d_bwd_weight(_ptr(x), _ptr(dy), _ptr(dw), B, T, C, K, pad_left,
+                                          pad_right) != 0:
+        raise ValueError("oracle_dwconv1d_bwd_weight rejected the shape")
+    return dw

@@ -1,0 +1,225 @@
+/*
+ * Oracle for grouped / depthwise convolution -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, fp64 nested loops that state the definitions directly. Only the
+ * test-suite, the package smoke check and the benchmark's CPU-baseline leg use
+ * this file. The CUDA library shares no code, header or table with it.
+ *
+ * What is computed, and where it is defined:
+ *  - Grouped 2-D convolution: input channels, filters and output channels are
+ *    split into `groups` equal blocks with no connection between blocks
+ *    ("Grouped convolutions", neon issue #296, thestew42's first reply), in
+ *    the usual group-major channel order 1111 2222 3333 ... (same thread,
+ *    ibmua's post on output orderings). The arithmetic is cross-correlation with
+ *    zero padding, i.e. the semantics of `F.conv2d(input, weight, padding,
+ *    groups)` as called in "F.conv2d runs x15 slower in mixed-precision/
+ *    half-precision mode" (the timing script in the first post). groups == C_in
+ *    is the fully-grouped (depthwise) case of the neon thread.
+ *  - Depthwise conv1d over (batch, steps, channels) with groups = channels, as
+ *    in "Investigate custom Triton kernels for depthwise-separable convolutions
+ *    in Conformer" (speechbrain #2733, the issue text and the Oct 27 comment on
+ *    the (batch, steps, channels) layout), plus its backward pass (the Oct 30
+ *    comment): data gradient and weight gradient, written as the literal
+ *    adjoint (scatter form) of the forward sum.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  - output size  Ho = floor((H + 2*pad - dil*(kH-1) - 1)/stride) + 1 (PyTorch's
+ *    rule for F.conv2d; symmetric scalar stride/pad/dilation);
+ *  - weight layouts: NCHW uses w[C_out][C_in/g][kH][kW] (the shape printed in
+ *    the timing script), NHWC uses w[C_out][kH][kW][C_in/g];
+ *  - conv1d: T_out = T + pad_left + pad_right - K + 1, zero outside [0, T).
+ *
+ * All buffers are dense, row-major, fp64. Parallelism: OpenMP over the
+ * outermost independent output loop only; each output is one sequential sum.
+ */
+#include <stddef.h>
+#include <stdint.h>
+
+#define ORACLE_NCHW 0
+#define ORACLE_NHWC 1
+
+typedef struct {
+  long N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups, Ho, Wo;
+  int layout;
+} conv2d_shape;
+
+static long out_extent(long in, long k, long stride, long pad, long dil) {
+  long span = in + 2 * pad - dil * (k - 1) - 1;
+  if (span < 0) return 0;
+  return span / stride + 1;
+}
+
+static long x_index(const conv2d_shape* s, long n, long c, long h, long w) {
+  if (s->layout == ORACLE_NCHW) return ((n * s->C_in + c) * s->H + h) * s->W + w;
+  return ((n * s->H + h) * s->W + w) * s->C_in + c;
+}
+
+static long w_index(const conv2d_shape* s, long co, long ci, long kh, long kw) {
+  long cpg_in = s->C_in / s->groups;
+  if (s->layout == ORACLE_NCHW) return ((co * cpg_in + ci) * s->kH + kh) * s->kW + kw;
+  return ((co * s->kH + kh) * s->kW + kw) * cpg_in + ci;
+}
+
+static long y_index(const conv2d_shape* s, long n, long co, long ho, long wo) {
+  if (s->layout == ORACLE_NCHW) return ((n * s->C_out + co) * s->Ho + ho) * s->Wo + wo;
+  return ((n * s->Ho + ho) * s->Wo + wo) * s->C_out + co;
+}
+
+/* One output element of the grouped convolution: the whole definition. */
+static double conv2d_point(const conv2d_shape* s, const double* x, const double* w,
+                           const double* bias, long n, long co, long ho, long wo) {
+  long cpg_in = s->C_in / s->groups;
+  long cpg_out = s->C_out / s->groups;
+  long g = co / cpg_out;            /* group-major: output channel co is in group co / cpg_out */
+  double acc = bias ? bias[co] : 0.0;
+  for (long ci = 0; ci < cpg_in; ++ci) {
+    long c = g * cpg_in + ci;         /* the group reads only its own block of input channels */
+    for (long kh = 0; kh < s->kH; ++kh) {
+      long h = ho * s->stride - s->pad + kh * s->dil;
+      if (h < 0 || h >= s->H) continue;   /* zero padding */
+      for (long kw = 0; kw < s->kW; ++kw) {
+        long wi = wo * s->stride - s->pad + kw * s->dil;
+        if (wi < 0 || wi >= s->W) continue;
+        acc += w[w_index(s, co, ci, kh, kw)] * x[x_index(s, n, c, h, wi)];
+      }
+    }
+  }
+  return acc;
+}
+
+static int make_shape(conv2d_shape* s, long N, long C_in, long H, long W, long C_out, long kH,
+                      long kW, long stride, long pad, long dil, long groups, int layout) {
+  if (N < 0 || C_in <= 0 || H <= 0 || W <= 0 || C_out <= 0 || kH <= 0 || kW <= 0) return -1;
+  if (stride <= 0 || pad < 0 || dil <= 0 || groups <= 0) return -1;
+  if (C_in % groups != 0 || C_out % groups != 0) return -1;
+  if (layout != ORACLE_NCHW && layout != ORACLE_NHWC) return -1;
+  s->N = N; s->C_in = C_in; s->H = H; s->W = W; s->C_out = C_out; s->kH = kH; s->kW = kW;
+  s->stride = stride; s->pad = pad; s->dil = dil; s->groups = groups; s->layout = layout;
+  s->Ho = out_extent(H, kH, stride, pad, dil);
+  s->Wo = out_extent(W, kW, stride, pad, dil);
+  if (s->Ho <= 0 || s->Wo <= 0) return -1;
+  return 0;
+}
+
+/* Output spatial size for the given input size; 0 when the window does not fit. */
+long oracle_conv_out_extent(long in, long k, long stride, long pad, long dil) {
+  if (stride <= 0 || dil <= 0 || k <= 0 || pad < 0) return 0;
+  return out_extent(in, k, stride, pad, dil);
+}
+
+/* Full grouped conv2d. Returns 0 on success, -1 on an invalid shape. */
+int oracle_conv2d(const double* x, const double* w, const double* bias, double* y, long N,
+                  long C_in, long H, long W, long C_out, long kH, long kW, long stride, long pad,
+                  long dil, long groups, int layout) {
+  conv2d_shape s;
+  if (make_shape(&s, N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups, layout)) return -1;
+  long outer = N * C_out;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long nc = 0; nc < outer; ++nc) {
+    long n = nc / C_out, co = nc % C_out;
+    for (long ho = 0; ho < s.Ho; ++ho)
+      for (long wo = 0; wo < s.Wo; ++wo)
+        y[y_index(&s, n, co, ho, wo)] = conv2d_point(&s, x, w, bias, n, co, ho, wo);
+  }
+  return 0;
+}
+
+/* Selected outputs of grouped conv2d: out[i] = y at the 4-tuple idx[4i..4i+3] =
+ * (n, co, ho, wo). Used to check full-size launches on sampled outputs. */
+int oracle_conv2d_points(const double* x, const double* w, const double* bias, double* out,
+                         const int64_t* idx, long npts, long N, long C_in, long H, long W,
+                         long C_out, long kH, long kW, long stride, long pad, long dil,
+                         long groups, int layout) {
+  conv2d_shape s;
+  if (make_shape(&s, N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups, layout)) return -1;
+  for (long i = 0; i < npts; ++i) {
+    long n = idx[4 * i], co = idx[4 * i + 1], ho = idx[4 * i + 2], wo = idx[4 * i + 3];
+    if (n < 0 || n >= N || co < 0 || co >= C_out || ho < 0 || ho >= s.Ho || wo < 0 || wo >= s.Wo)
+      return -1;
+  }
+#pragma omp parallel for schedule(static)
+  for (long i = 0; i < npts; ++i)
+    out[i] = conv2d_point(&s, x, w, bias, idx[4 * i], idx[4 * i + 1], idx[4 * i + 2],
+                          idx[4 * i + 3]);
+  return 0;
+}
+
+/* ---------------- depthwise conv1d over (batch, steps, channels) ---------------- */
+
+static int conv1d_ok(long B, long T, long C, long K, long pl, long pr) {
+  if (B < 0 || T <= 0 || C <= 0 || K <= 0 || pl < 0 || pr < 0) return 0;
+  return T + pl + pr - K + 1 > 0;
+}
+
+/* y[b][t][c] = sum_k w[c][k] * x[b][t + k - pl][c], x = 0 outside [0, T). */
+int oracle_dwconv1d_fwd(const double* x, const double* w, double* y, long B, long T, long C,
+                        long K, long pl, long pr) {
+  if (!conv1d_ok(B, T, C, K, pl, pr)) return -1;
+  long T_out = T + pl + pr - K + 1;
+#pragma omp parallel for schedule(static)
+  for (long b = 0; b < B; ++b)
+    for (long t = 0; t < T_out; ++t)
+      for (long c = 0; c < C; ++c) {
+        double acc = 0.0;
+        for (long k = 0; k < K; ++k) {
+          long s = t + k - pl;
+          if (s < 0 || s >= T) continue;
+          acc += w[c * K + k] * x[(b * T + s) * C + c];
+        }
+        y[(b * T_out + t) * C + c] = acc;
+      }
+  return 0;
+}
+
+/* Data gradient: each forward term w[c][k]*x[b][s][c] (s = t + k - pl) sends
+ * w[c][k]*dy[b][t][c] back to dx[b][s][c]. Written in that scatter form; the
+ * per-batch loop keeps the scatter race-free under OpenMP. */
+int oracle_dwconv1d_bwd_data(const double* dy, const double* w, double* dx, long B, long T,
+                             long C, long K, long pl, long pr) {
+  if (!conv1d_ok(B, T, C, K, pl, pr)) return -1;
+  long T_out = T + pl + pr - K + 1;
+#pragma omp parallel for schedule(static)
+  for (long b = 0; b < B; ++b) {
+    for (long s = 0; s < T; ++s)
+      for (long c = 0; c < C; ++c) dx[(b * T + s) * C + c] = 0.0;
+    for (long t = 0; t < T_out; ++t)
+      for (long k = 0; k < K; ++k) {
+        long s = t + k - pl;
+        if (s < 0 || s >= T) continue;
+        for (long c = 0; c < C; ++c)
+          dx[(b * T + s) * C + c] += w[c * K + k] * dy[(b * T_out + t) * C + c];
+      }
+  }
+  return 0;
+}
+
+/* Weight gradient: dw[c][k] = sum over (b, t) of dy[b][t][c] * x[b][t + k - pl][c],
+ * summed in (b, t) order. */
+int oracle_dwconv1d_bwd_weight(const double* x, const double* dy, double* dw, long B, long T,
+                               long C, long K, long pl, long pr) {
+  if (!conv1d_ok(B, T, C, K, pl, pr)) return -1;
+  long T_out = T + pl + pr - K + 1;
+#pragma omp parallel for schedule(static)
+  for (long c = 0; c < C; ++c)
+    for (long k = 0; k < K; ++k) {
+      double acc = 0.0;
+      for (long b = 0; b < B; ++b)
+        for (long t = 0; t < T_out; ++t) {
+          long s = t + k - pl;
+          if (s < 0 || s >= T) continue;
+          acc += dy[(b * T_out + t) * C + c] * x[(b * T + s) * C + c];
+        }
+      dw[c * K + k] = acc;
+    }
+  return 0;
+}
+
+/* Number of OpenMP threads the oracle runs with (1 without OpenMP). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

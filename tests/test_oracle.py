@@ -1,0 +1,453 @@
+"""Pins for the fp64 oracle: it is checked against things other than itself.
+
+Each test ties the oracle to a fact the pages or the mathematics fix: an independent
+brute-force evaluator on tiny integer inputs (exact), library routines for special cases
+(numpy einsum / correlate / convolve, scipy correlate2d), closed forms (delta kernels,
+box sums by integral image), invariants (group concatenation, linearity, adjointness,
+ensemble-as-groups), finite differences, the pages' printed facts (tests/golden), and
+planted mistakes that the pins must catch. No GPU is needed.
+"""
+import ctypes
+import json
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+import scipy.signal
+
+import oracle
+from depthwise_convolution_gconv2d_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+NCHW, NHWC = oracle.NCHW, oracle.NHWC
+
+
+# ---------------------------------------------------------------- independent evaluators
+
+def n_positions(size, k, stride, pad, dil):
+    """Count window start positions by enumeration (no closed-form output-size rule)."""
+    span = dil * (k - 1) + 1
+    return len(range(0, size + 2 * pad - span + 1, stride))
+
+
+def brute_conv2d_nchw(x, w, stride, pad, dil, groups):
+    """Tap decomposition on an explicitly zero-padded int64 tensor, one group at a time."""
+    x = np.asarray(x).astype(np.int64)
+    w = np.asarray(w).astype(np.int64)
+    N, C_in, H, W = x.shape
+    C_out, cpg_in, kH, kW = w.shape
+    cpg_out = C_out // groups
+    Ho, Wo = n_positions(H, kH, stride, pad, dil), n_positions(W, kW, stride, pad, dil)
+    xp = np.zeros((N, C_in, H + 2 * pad, W + 2 * pad), np.int64)
+    xp[:, :, pad:pad + H, pad:pad + W] = x
+    y = np.zeros((N, C_out, Ho, Wo), np.int64)
+    for j in range(groups):
+        xg = xp[:, j * cpg_in:(j + 1) * cpg_in]
+        wg = w[j * cpg_out:(j + 1) * cpg_out]
+        for kh in range(kH):
+            for kw in range(kW):
+                patch = xg[:, :, kh * dil: kh * dil + stride * (Ho - 1) + 1: stride,
+                           kw * dil: kw * dil + stride * (Wo - 1) + 1: stride]
+                y[:, j * cpg_out:(j + 1) * cpg_out] += np.einsum("nchw,oc->nohw", patch,
+                                                                 wg[:, :, kh, kw])
+    return y
+
+
+def brute_dwconv1d_fwd(x, w, pl, pr):
+    """Pure-Python loops over an explicitly padded sequence (integers, exact)."""
+    B, T, C = x.shape
+    K = w.shape[1]
+    xp = np.zeros((B, T + pl + pr, C), np.int64)
+    xp[:, pl:pl + T] = x.astype(np.int64)
+    T_out = T + pl + pr - K + 1
+    y = np.zeros((B, T_out, C), np.int64)
+    for b in range(B):
+        for t in range(T_out):
+            for c in range(C):
+                y[b, t, c] = sum(int(w[c, k]) * int(xp[b, t + k, c]) for k in range(K))
+    return y
+
+
+def to_nhwc(x):
+    return np.ascontiguousarray(np.transpose(x, (0, 2, 3, 1)))
+
+
+def from_nhwc(y):
+    return np.ascontiguousarray(np.transpose(y, (0, 3, 1, 2)))
+
+
+def rng_int(seed, shape):
+    return np.random.default_rng(seed).integers(-2, 3, shape).astype(np.float64)
+
+
+# ---------------------------------------------------------------- brute force, all shapes
+
+def _tiny_cases():
+    r = np.random.default_rng(7)
+    cases = []
+    for _ in range(48):
+        groups = int(r.choice([1, 2, 3, 4]))
+        cpg_in = int(r.integers(1, 4))
+        cpg_out = int(r.integers(1, 4))
+        k = (int(r.integers(1, 4)), int(r.integers(1, 4)))
+        stride, pad, dil = int(r.choice([1, 2])), int(r.choice([0, 1, 2])), int(r.choice([1, 2]))
+        H, W = int(r.integers(1, 8)), int(r.integers(1, 8))
+        if n_positions(H, k[0], stride, pad, dil) < 1 or n_positions(W, k[1], stride, pad, dil) < 1:
+            continue
+        cases.append((int(r.integers(1, 3)), groups * cpg_in, H, W, groups * cpg_out, k, stride,
+                      pad, dil, groups))
+    return cases
+
+
+@pytest.mark.parametrize("case", _tiny_cases())
+@pytest.mark.parametrize("layout", [NCHW, NHWC])
+def test_brute_force_conv2d(case, layout):
+    N, C_in, H, W, C_out, (kH, kW), s, p, d, g = case
+    x = rng_int(1, (N, C_in, H, W))
+    w = rng_int(2, (C_out, C_in // g, kH, kW))
+    ref = brute_conv2d_nchw(x, w, s, p, d, g)
+    if layout == NCHW:
+        y = oracle.conv2d(x, w, None, s, p, d, g, NCHW)
+    else:
+        y = from_nhwc(oracle.conv2d(to_nhwc(x), to_nhwc(w), None, s, p, d, g, NHWC))
+    assert y.shape == ref.shape
+    assert np.array_equal(y, ref.astype(np.float64))
+
+
+def test_points_match_full():
+    x, w = rng_int(3, (2, 6, 7, 5)), rng_int(4, (9, 2, 3, 2))
+    b = rng_int(5, (9,))
+    y = oracle.conv2d(x, w, b, 2, 1, 1, 3, NCHW)
+    idx = np.array([(n, co, ho, wo) for n in range(2) for co in range(9)
+                    for ho in range(y.shape[2]) for wo in range(y.shape[3])])
+    pts = oracle.conv2d_points(x, w, idx, b, 2, 1, 1, 3, NCHW)
+    assert np.array_equal(pts, y[idx[:, 0], idx[:, 1], idx[:, 2], idx[:, 3]])
+
+
+# ---------------------------------------------------------------- invariants and library pins
+
+def test_group_concat_of_dense_convs():
+    g, cpg_in, cpg_out = 4, 3, 2
+    x, w = rng_int(10, (2, g * cpg_in, 6, 5)), rng_int(11, (g * cpg_out, cpg_in, 3, 3))
+    y = oracle.conv2d(x, w, None, 1, 1, 1, g, NCHW)
+    for j in range(g):
+        yj = oracle.conv2d(x[:, j * cpg_in:(j + 1) * cpg_in], w[j * cpg_out:(j + 1) * cpg_out],
+                           None, 1, 1, 1, 1, NCHW)
+        assert np.array_equal(y[:, j * cpg_out:(j + 1) * cpg_out], yj)
+
+
+def test_groups1_1x1_is_matmul():
+    x, w = rng_int(12, (3, 7, 4, 5)), rng_int(13, (6, 7, 1, 1))
+    y = oracle.conv2d(x, w, None, 1, 0, 1, 1, NCHW)
+    assert np.array_equal(y, np.einsum("nchw,oc->nohw", x, w[:, :, 0, 0]))
+
+
+def test_dense_conv_vs_scipy_correlate2d():
+    r = np.random.default_rng(14)
+    x, w = r.standard_normal((2, 3, 9, 8)), r.standard_normal((4, 3, 3, 2))
+    y = oracle.conv2d(x, w, None, 1, 1, 1, 1, NCHW)
+    xp = np.pad(x, ((0, 0), (0, 0), (1, 1), (1, 1)))
+    ref = np.zeros_like(y)
+    for n in range(2):
+        for co in range(4):
+            for ci in range(3):
+                ref[n, co] += scipy.signal.correlate2d(xp[n, ci], w[co, ci], mode="valid")
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_conv_vs_scipy_per_group():
+    r = np.random.default_rng(15)
+    g = 3
+    x, w = r.standard_normal((1, 6, 7, 7)), r.standard_normal((9, 2, 3, 3))
+    y = oracle.conv2d(x, w, None, 1, 1, 1, g, NCHW)
+    xp = np.pad(x, ((0, 0), (0, 0), (1, 1), (1, 1)))
+    for co in range(9):
+        j = co // 3
+        ref = sum(scipy.signal.correlate2d(xp[0, 2 * j + ci], w[co, ci], mode="valid")
+                  for ci in range(2))
+        np.testing.assert_allclose(y[0, co], ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("layout", [NCHW, NHWC])
+def test_centred_delta_is_identity(layout):
+    g, C = 4, 8
+    cpg = C // g
+    x = np.random.default_rng(16).standard_normal((2, C, 6, 7))
+    w = np.zeros((C, cpg, 3, 5))
+    for co in range(C):
+        w[co, co % cpg, 1, 2] = 1.0
+    if layout == NCHW:
+        y = oracle.conv2d(x, w, None, 1, 0, 1, g, NCHW)  # pad 0 -> interior only
+        assert np.array_equal(y, x[:, :, 1:-1, 2:-2])
+    xs = to_nhwc(x) if layout == NHWC else x
+    w3 = np.zeros((C, cpg, 3, 3))
+    for co in range(C):
+        w3[co, co % cpg, 1, 1] = 1.0
+    y = oracle.conv2d(xs, to_nhwc(w3) if layout == NHWC else w3, None, 1, 1, 1, g, layout)
+    assert np.array_equal(y, xs)
+
+
+def test_offcentre_delta_is_shift_with_zero_fill():
+    x = np.random.default_rng(17).standard_normal((1, 2, 5, 6))
+    w = np.zeros((2, 1, 3, 3))
+    w[:, 0, 0, 2] = 1.0          # tap (kh=0, kw=2) with pad 1: y[h, w] = x[h-1, w+1]
+    y = oracle.conv2d(x, w, None, 1, 1, 1, 2, NCHW)
+    ref = np.zeros_like(x)
+    ref[:, :, 1:, :-1] = x[:, :, :-1, 1:]
+    assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("k,pad", [(3, 1), (5, 2), (3, 0), (4, 3)])
+def test_all_ones_depthwise_is_box_sum(k, pad):
+    C, H, W = 3, 9, 11
+    x = rng_int(18, (2, C, H, W))
+    w = np.ones((C, 1, k, k))
+    y = oracle.conv2d(x, w, None, 1, pad, 1, C, NCHW)
+    # integral image over the zero-padded input
+    xp = np.pad(x, ((0, 0), (0, 0), (pad, pad), (pad, pad)))
+    S = np.zeros((2, C, xp.shape[2] + 1, xp.shape[3] + 1))
+    S[:, :, 1:, 1:] = xp.cumsum(2).cumsum(3)
+    Ho, Wo = y.shape[2], y.shape[3]
+    ref = (S[:, :, k:k + Ho, k:k + Wo] - S[:, :, :Ho, k:k + Wo] - S[:, :, k:k + Ho, :Wo]
+           + S[:, :, :Ho, :Wo])
+    assert np.array_equal(y, ref)
+
+
+def test_linearity_in_x_and_w():
+    r = np.random.default_rng(19)
+    x1, x2 = r.standard_normal((2, 4, 6, 6)), r.standard_normal((2, 4, 6, 6))
+    w1, w2 = r.standard_normal((6, 2, 3, 3)), r.standard_normal((6, 2, 3, 3))
+    a, b = 0.75, -1.5
+    f = lambda x, w: oracle.conv2d(x, w, None, 2, 1, 2, 2, NCHW)
+    np.testing.assert_allclose(f(a * x1 + b * x2, w1), a * f(x1, w1) + b * f(x2, w1),
+                               rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(f(x1, a * w1 + b * w2), a * f(x1, w1) + b * f(x1, w2),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_stride_is_subsampled_stride1():
+    x, w = rng_int(20, (2, 4, 9, 10)), rng_int(21, (4, 2, 3, 3))
+    y1 = oracle.conv2d(x, w, None, 1, 1, 1, 2, NCHW)
+    y2 = oracle.conv2d(x, w, None, 2, 1, 1, 2, NCHW)
+    assert np.array_equal(y2, y1[:, :, ::2, ::2])
+
+
+def test_dilation_is_zero_inserted_kernel():
+    x, w = rng_int(22, (1, 3, 11, 12)), rng_int(23, (3, 1, 3, 2))
+    y = oracle.conv2d(x, w, None, 1, 2, 2, 3, NCHW)
+    wd = np.zeros((3, 1, 5, 3))
+    wd[:, :, ::2, ::2] = w
+    assert np.array_equal(y, oracle.conv2d(x, wd, None, 1, 2, 1, 3, NCHW))
+
+
+def test_layouts_agree():
+    x, w = rng_int(24, (2, 6, 5, 7)), rng_int(25, (9, 2, 3, 3))
+    b = rng_int(26, (9,))
+    y = oracle.conv2d(x, w, b, 2, 1, 1, 3, NCHW)
+    y2 = oracle.conv2d(to_nhwc(x), to_nhwc(w), b, 2, 1, 1, 3, NHWC)
+    assert np.array_equal(from_nhwc(y2), y)
+
+
+def test_bias_is_broadcast_add():
+    x, w, b = rng_int(27, (2, 4, 5, 5)), rng_int(28, (4, 1, 3, 3)), rng_int(29, (4,))
+    y0 = oracle.conv2d(x, w, None, 1, 1, 1, 4, NCHW)
+    y1 = oracle.conv2d(x, w, b, 1, 1, 1, 4, NCHW)
+    assert np.array_equal(y1, y0 + b[None, :, None, None])
+
+
+def test_ensemble_equals_groups():
+    """M models each mapping cin->cout channels, stacked model-major into one groups=M conv
+    (the vmap batching rule of "Optimize convolution batching rule performance")."""
+    M, cin, cout, B = 4, 3, 5, 2
+    r = np.random.default_rng(30)
+    xs = [r.integers(-2, 3, (B, cin, 6, 6)).astype(float) for _ in range(M)]
+    ws = [r.integers(-2, 3, (cout, cin, 3, 3)).astype(float) for _ in range(M)]
+    y = oracle.conv2d(np.concatenate(xs, 1), np.concatenate(ws, 0), None, 1, 1, 1, M, NCHW)
+    for m in range(M):
+        ym = oracle.conv2d(xs[m], ws[m], None, 1, 1, 1, 1, NCHW)
+        assert np.array_equal(y[:, m * cout:(m + 1) * cout], ym)
+        assert np.array_equal(ym, brute_conv2d_nchw(xs[m], ws[m], 1, 1, 1, 1))
+
+
+def test_rejects_bad_shapes():
+    with pytest.raises(ValueError):
+        oracle.conv2d(np.zeros((1, 6, 4, 4)), np.zeros((4, 3, 3, 3)), groups=4)
+    with pytest.raises(ValueError):       # window larger than the padded input
+        oracle.conv2d(np.zeros((1, 2, 2, 2)), np.zeros((2, 2, 5, 5)), pad=0)
+
+
+# ---------------------------------------------------------------- pages' printed facts
+
+def test_group_order_golden():
+    """Output channel co of a grouped conv reads input group co // (C_out/g): the usual
+    group-major order of the neon thread."""
+    gold = json.load(open(os.path.join(GOLDEN, "group_order.json")))
+    C, g = gold["C_out"], gold["groups"]
+    cpg = C // g
+    assert gold["expected"].startswith(gold["printed"])
+    x = np.zeros((1, C, 1, 1))
+    for c in range(C):
+        x[0, c] = c // cpg + 1           # input channel carries its group label
+    w = np.ones((C, cpg, 1, 1)) / cpg    # output = mean of the inputs it is connected to
+    y = oracle.conv2d(x, w, None, 1, 0, 1, g, NCHW)
+    assert "".join(str(int(v)) for v in y[0, :, 0, 0]) == gold["expected"]
+
+
+def test_p2_layer_golden():
+    gold = json.load(open(os.path.join(GOLDEN, "p2_layer.json")))
+    xs, ws = gold["input_shape"], gold["weight_shape"]
+    assert ws[1] * gold["groups"] == xs[1]
+    shape = oracle.conv2d_out_shape(xs, ws, 1, gold["padding"], 1, gold["groups"], NCHW)
+    assert list(shape) == gold["expected_output_shape"]
+    # a few sampled outputs of the full-size layer against a per-point window sum
+    p = wl.wide_group(wl.NCHW, wl.F32)
+    r = np.random.default_rng(31)
+    x = r.integers(-2, 3, p.x_shape).astype(np.float64)
+    w = r.integers(-2, 3, p.w_shape).astype(np.float64)
+    idx = np.array([(0, 0, 0, 0), (0, 511, 255, 255), (0, 130, 17, 0), (0, 383, 255, 100)])
+    got = oracle.conv2d_points(x, w, idx, None, 1, 1, 1, 4, NCHW)
+    xp = np.pad(x, ((0, 0), (0, 0), (1, 1), (1, 1)))
+    for (n, co, ho, wo), v in zip(idx, got):
+        j = co // 128
+        win = xp[n, j * 128:(j + 1) * 128, ho:ho + 3, wo:wo + 3]
+        assert v == float((win * w[co]).sum())
+
+
+# ---------------------------------------------------------------- dwconv1d
+
+CONV1D_CASES = [(2, 9, 3, 3, 1, 1), (1, 12, 4, 5, 4, 0), (3, 7, 2, 31, 15, 15),
+                (2, 40, 5, 31, 30, 0), (1, 5, 1, 2, 0, 1), (2, 6, 3, 4, 0, 0)]
+
+
+@pytest.mark.parametrize("B,T,C,K,pl,pr", CONV1D_CASES)
+def test_dwconv1d_fwd_brute_force(B, T, C, K, pl, pr):
+    x, w = rng_int(40, (B, T, C)), rng_int(41, (C, K))
+    assert np.array_equal(oracle.dwconv1d_fwd(x, w, pl, pr),
+                          brute_dwconv1d_fwd(x, w, pl, pr).astype(float))
+
+
+@pytest.mark.parametrize("B,T,C,K,pl,pr", CONV1D_CASES)
+def test_dwconv1d_library_pins(B, T, C, K, pl, pr):
+    """fwd = numpy.correlate, dgrad = numpy.convolve ('full', cropped), wgrad =
+    numpy.correlate of the padded input with dy, per (batch, channel)."""
+    r = np.random.default_rng(42)
+    x, w = r.standard_normal((B, T, C)), r.standard_normal((C, K))
+    T_out = T + pl + pr - K + 1
+    dy = r.standard_normal((B, T_out, C))
+    y = oracle.dwconv1d_fwd(x, w, pl, pr)
+    dx = oracle.dwconv1d_bwd_data(dy, w, T, pl, pr)
+    dw = oracle.dwconv1d_bwd_weight(x, dy, K, pl, pr)
+    dw_ref = np.zeros((C, K))
+    for b in range(B):
+        for c in range(C):
+            xp = np.concatenate([np.zeros(pl), x[b, :, c], np.zeros(pr)])
+            np.testing.assert_allclose(y[b, :, c], np.correlate(xp, w[c], "valid"),
+                                       rtol=1e-12, atol=1e-12)
+            full = np.convolve(dy[b, :, c], w[c], "full")
+            np.testing.assert_allclose(dx[b, :, c], full[pl:pl + T], rtol=1e-12, atol=1e-12)
+            dw_ref[c] += np.correlate(xp, dy[b, :, c], "valid")
+    np.testing.assert_allclose(dw, dw_ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("B,T,C,K,pl,pr", CONV1D_CASES)
+def test_dwconv1d_adjoint_identity(B, T, C, K, pl, pr):
+    """<fwd(x, w), dy> = <x, dgrad(dy, w)> = <w, wgrad(x, dy)>."""
+    r = np.random.default_rng(43)
+    x, w = r.standard_normal((B, T, C)), r.standard_normal((C, K))
+    dy = r.standard_normal((B, T + pl + pr - K + 1, C))
+    a = np.vdot(oracle.dwconv1d_fwd(x, w, pl, pr), dy)
+    b = np.vdot(x, oracle.dwconv1d_bwd_data(dy, w, T, pl, pr))
+    c = np.vdot(w, oracle.dwconv1d_bwd_weight(x, dy, K, pl, pr))
+    assert abs(a - b) <= 1e-10 * max(1.0, abs(a))
+    assert abs(a - c) <= 1e-10 * max(1.0, abs(a))
+
+
+def test_dwconv1d_finite_differences():
+    """Central differences of L = <fwd(x, w), dy> (the gradcheck idea of the Conformer
+    thread) against dgrad and wgrad."""
+    B, T, C, K, pl, pr = 2, 7, 2, 4, 2, 1
+    r = np.random.default_rng(44)
+    x, w = r.standard_normal((B, T, C)), r.standard_normal((C, K))
+    dy = r.standard_normal((B, T + pl + pr - K + 1, C))
+    L = lambda xx, ww: np.vdot(oracle.dwconv1d_fwd(xx, ww, pl, pr), dy)
+    dx = oracle.dwconv1d_bwd_data(dy, w, T, pl, pr)
+    dw = oracle.dwconv1d_bwd_weight(x, dy, K, pl, pr)
+    h = 1e-6
+    for i in np.ndindex(x.shape):
+        e = np.zeros_like(x)
+        e[i] = h
+        assert abs((L(x + e, w) - L(x - e, w)) / (2 * h) - dx[i]) < 1e-6
+    for i in np.ndindex(w.shape):
+        e = np.zeros_like(w)
+        e[i] = h
+        assert abs((L(x, w + e) - L(x, w - e)) / (2 * h) - dw[i]) < 1e-6
+
+
+def test_dwconv1d_same_and_causal_relation():
+    """With equal total padding, the causal output is the 'same' output shifted by the
+    difference in left padding (here 15 steps), zero-filled where the window leaves x."""
+    x, w = rng_int(45, (2, 50, 3)), rng_int(46, (3, 31))
+    ys = oracle.dwconv1d_fwd(x, w, 15, 15)
+    yc = oracle.dwconv1d_fwd(x, w, 30, 0)
+    # yc[t] = sum_k w[k] x[t+k-30] = ys[t-15] for t >= 15
+    assert np.array_equal(yc[:, 15:], ys[:, :-15])
+
+
+def test_dwconv1d_equals_depthwise_conv2d():
+    """conv1d on (batch, steps, channels) is the depthwise conv2d with H = 1 (NHWC)."""
+    B, T, C, K = 2, 13, 4, 5
+    x, w = rng_int(47, (B, T, C)), rng_int(48, (C, K))
+    # conv2d pads H as well (scalar pad); with kH = 1 the middle row is the conv1d result
+    y2 = oracle.conv2d(x[:, None], w[:, None, :, None], None, 1, 2, 1, C, NHWC)[:, 2]
+    assert np.array_equal(y2, oracle.dwconv1d_fwd(x, w, 2, 2))
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+MUTANTS = {
+    "kh_kw_swapped_in_nchw_weight": ("((co * cpg_in + ci) * s->kH + kh) * s->kW + kw",
+                                     "((co * cpg_in + ci) * s->kH + kw) * s->kW + kh"),
+    "group_offset_dropped": ("long c = g * cpg_in + ci;", "long c = ci;"),
+    "pad_sign_flipped": ("long h = ho * s->stride - s->pad + kh * s->dil;",
+                         "long h = ho * s->stride + s->pad + kh * s->dil;"),
+    "last_tap_dropped": ("for (long kw = 0; kw < s->kW; ++kw)", "for (long kw = 0; kw < s->kW - 1; ++kw)"),
+    "conv_instead_of_correlation_1d": ("acc += w[c * K + k] * x[(b * T + s) * C + c];",
+                                       "acc += w[c * K + (K - 1 - k)] * x[(b * T + s) * C + c];"),
+    "dgrad_wrong_direction": ("dx[(b * T + s) * C + c] += w[c * K + k]",
+                              "dx[(b * T + s) * C + c] += w[c * K + (K - 1 - k)]"),
+    "wgrad_sign": ("acc += dy[(b * T_out + t) * C + c] * x[(b * T + s) * C + c];",
+                   "acc -= dy[(b * T_out + t) * C + c] * x[(b * T + s) * C + c];"),
+}
+
+
+def _pins_pass():
+    """A compact run of the pins above; returns False as soon as one fails."""
+    try:
+        for case in _tiny_cases()[:16]:
+            for layout in (NCHW, NHWC):
+                test_brute_force_conv2d(case, layout)
+        for args in CONV1D_CASES:
+            test_dwconv1d_fwd_brute_force(*args)
+            test_dwconv1d_library_pins(*args)
+        test_group_order_golden()
+    except AssertionError:
+        return False
+    return True
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistakes_are_caught(name, monkeypatch):
+    old, new = MUTANTS[name]
+    src = open(oracle._SRC).read()
+    assert src.count(old) >= 1, name
+    with tempfile.TemporaryDirectory() as d:
+        path = os.path.join(d, "oracle_mutant.c")
+        open(path, "w").write(src.replace(old, new, 1))
+        so = os.path.join(d, "liboracle_mutant.so")
+        subprocess.check_call(["gcc", "-O1", "-fPIC", "-shared", "-std=c99", path, "-o", so])
+        monkeypatch.setattr(oracle, "_lib", oracle._configure(ctypes.CDLL(so)))
+        assert not _pins_pass(), f"mutant {name} survived the pins"
+    monkeypatch.undo()
+    assert _pins_pass()
