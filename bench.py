@@ -1,0 +1,464 @@
+"""Benchmark: grouped-conv TFLOP/s and depthwise GB/s on B200, as fractions of the tensor / HBM
+roofline, with the fp64 CPU oracle timed beside it.
+
+One step = one forward of the wide-group layer x[1, 512, 256, 256] * w[512, 128, 3, 3],
+groups = 4, pad 1 (the layer timed in "F.conv2d runs x15 slower in mixed-precision/
+half-precision mode"), bf16 in / fp32 accumulate / bf16 out, NHWC by default, through the
+library's C ABI. `value` is whole-job TFLOP/s (77.31 GFLOP per step per GPU) over the K timed
+steps. Inputs are synthetic (seeded, x ~ N(0,1), w ~ N(0, 1/1152)); the timed steps rotate
+over enough x/y buffer sets that every step's working set is evicted from L2 by the next.
+
+The same JSON line carries the depthwise measurements (GB/s against the HBM roofline):
+the depthwise conv2d x[32, 56, 56, 1024] 3x3 at stride 1 and 2, and the Conformer depthwise
+conv1d x[8, 2048, 512], K = 31 (fwd, dgrad, wgrad), each kernel timed with CUDA events on its
+own stream with an L2 flush before every launch (outside the event bracket).
+
+Multi-GPU: the path does not shard (one conv runs on one GPU); with N ranks each GPU runs an
+independent replica on its own inputs, no data-path collective, and the timing is the max
+over ranks ("scaling": "weak").
+
+`--impl reference` times the fp64 CPU oracle (the only reference that exists for this path)
+on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from depthwise_convolution_gconv2d_b200 import workloads as wl  # noqa: E402
+
+METRIC = "grouped-conv TFLOP/s and depthwise GB/s on 1 B200; % of tensor / HBM roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return d, "of measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK), "of fallback"
+
+
+def kernel_source_hash(name: str) -> str:
+    path = os.path.join(ROOT, "depthwise_convolution_gconv2d_b200", "csrc", name)
+    try:
+        return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return ""
+
+
+def traffic_for(kernel: str, source: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel is unchanged."""
+    try:
+        d = json.load(open(TRAFFIC_FILE)).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not d or d.get("source_sha") != kernel_source_hash(source):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if not self.out:
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- device helpers
+
+def dev_tensor(torch, storage, dtype, device):
+    a = np.ascontiguousarray(storage)
+    if dtype == wl.F32:
+        return torch.from_numpy(a.astype(np.float32)).to(device)
+    t = torch.from_numpy(a.view(np.int16)).to(device)
+    return t.view(torch.bfloat16 if dtype == wl.BF16 else torch.float16)
+
+
+def torch_dtype(torch, dtype):
+    return {wl.F32: torch.float32, wl.F16: torch.float16, wl.BF16: torch.bfloat16}[dtype]
+
+
+def l2_flusher(torch, device):
+    buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=device)
+
+    def flush(stream):
+        with torch.cuda.stream(stream):
+            buf.fill_(1)
+    return flush
+
+
+def time_launches(torch, fn, stream, reps, flush=None):
+    """Median and mean CUDA-event time (ms) of `fn(i)` over `reps` launches on `stream`,
+    flushing L2 before each launch outside the event bracket."""
+    times = []
+    for i in range(reps):
+        if flush is not None:
+            flush(stream)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn(i)
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times), sum(times) / len(times)
+
+
+# ---------------------------------------------------------------------------- workloads
+
+def conv2d_problem(layout: str):
+    return wl.wide_group(wl.NHWC if layout == "nhwc" else wl.NCHW)
+
+
+def kernel_name(code: int) -> str:
+    return {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "igemm_tc_nchw"}.get(
+        code, str(code))
+
+
+LAUNCHES_PER_CALL = {1: 1, 2: 1, 3: 1, 4: 3}
+KERNEL_SOURCE = {1: "direct_generic.cu", 2: "depthwise_nhwc.cu", 3: "igemm_tc.cu",
+                 4: "igemm_tc.cu"}
+
+
+def depthwise_measurements(torch, gb, device, stream, pk, reps):
+    """GB/s of the depthwise kernels (config shapes), L2 flushed before each launch."""
+    flush = l2_flusher(torch, device)
+    out = {}
+    hbm = pk["hbm_gbs"]
+    for stride in (1, 2):
+        p = wl.depthwise_56(stride)
+        inp = wl.make_conv2d_inputs(p, 5)
+        x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
+        y = torch.empty(p.y_shape, dtype=torch.bfloat16, device=device)
+        fn = lambda i: gb.gconv2d_fwd(x, w, None, p.stride, p.pad, p.dilation, p.groups,
+                                      p.layout, out=y, stream=stream)
+        for _ in range(3):
+            fn(0)
+        med, mean = time_launches(torch, fn, stream, reps, flush)
+        gbs = p.bytes() / (med * 1e-3) / 1e9
+        out[f"depthwise56_s{stride}"] = {"us": round(med * 1e3, 2), "GB/s": round(gbs, 1),
+                                         "frac": round(gbs / hbm, 3), "alg_bytes": p.bytes()}
+        del x, w, y
+    for causal in (False, True):
+        p = wl.conformer_dw1d(causal)
+        inp = wl.make_dwconv1d_inputs(p, 3)
+        x, w, dy = (dev_tensor(torch, a, p.dtype, device) for a in (inp.x, inp.w, inp.dy))
+        y = torch.empty((p.B, p.T_out, p.C), dtype=torch.bfloat16, device=device)
+        dx = torch.empty((p.B, p.T, p.C), dtype=torch.bfloat16, device=device)
+        dw = torch.empty((p.C, p.K), dtype=torch.bfloat16, device=device)
+        need = gb.dwconv1d_bwd_weight_workspace_size(p.B, p.T, p.C, p.K, p.pad_left, p.pad_right,
+                                                     p.dtype)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+        ops = {
+            "fwd": lambda i: gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right, out=y, stream=stream),
+            "dgrad": lambda i: gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right, out=dx,
+                                                    stream=stream),
+            "wgrad": lambda i: gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right, out=dw,
+                                                      workspace=ws, stream=stream),
+        }
+        tag = "causal" if causal else "same"
+        for op, fn in ops.items():
+            for _ in range(3):
+                fn(0)
+            med, mean = time_launches(torch, fn, stream, reps, flush)
+            gbs = p.bytes(op) / (med * 1e-3) / 1e9
+            out[f"dw1d_{tag}_{op}"] = {"us": round(med * 1e3, 2), "GB/s": round(gbs, 1),
+                                       "frac": round(gbs / hbm, 3), "alg_bytes": p.bytes(op)}
+    return out
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(p, inp_x64, inp_w64, target_s: float):
+    """Time the fp64 oracle on the first rows of the workload, growing the sample until it
+    takes about `target_s` seconds. Returns (TFLOP/s, seconds, rows, threads)."""
+    import oracle
+    rows = 2
+    while True:
+        if p.layout == wl.NCHW:
+            xs = np.ascontiguousarray(inp_x64[:, :, :rows, :])
+        else:
+            xs = np.ascontiguousarray(inp_x64[:, :rows, :, :])
+        t0 = time.perf_counter()
+        y = oracle.conv2d(xs, inp_w64, None, p.stride, p.pad, p.dilation, p.groups, p.layout)
+        dt = time.perf_counter() - t0
+        Ho, Wo = (y.shape[2], y.shape[3]) if p.layout == wl.NCHW else (y.shape[1], y.shape[2])
+        flops = 2 * p.N * Ho * Wo * p.C_out * p.cpg_in * p.kH * p.kW
+        if dt >= target_s * 0.5 or rows >= p.H:
+            return flops / dt / 1e12, dt, rows, oracle.num_threads()
+        rows = min(p.H, max(rows + 1, int(rows * target_s / max(dt, 1e-3) * 0.8)))
+
+
+def run_reference(args):
+    """--impl reference: the fp64 oracle on host cores, same metric and unit."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    p = conv2d_problem(args.layout)
+    inp = wl.make_conv2d_inputs(p, 2)
+    x64, w64 = inp.x64(), inp.w64()
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, dt, rows, thr = oracle_sample(p, x64, w64, per_step)
+        if i >= args.warmup:
+            vals.append((v, dt, rows, thr))
+    value = statistics.median(v for v, *_ in vals)
+    rows, thr = vals[-1][2], vals[-1][3]
+    sample = (f"first {rows} of {p.H} input rows of the workload (all channels, groups, taps), "
+              f"fp64 nested loops, {thr} OpenMP threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(statistics.median(dt for _, dt, *_ in vals) * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(p, args),
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": thr,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def config_dict(p, args):
+    return {"workload": f"wide-group conv2d x[1,512,256,256] w[512,128,3,3] groups=4 pad=1 "
+                        f"bf16/fp32-acc {args.layout.upper()}",
+            "N": p.N, "C_in": p.C_in, "H": p.H, "W": p.W, "C_out": p.C_out, "kH": p.kH,
+            "kW": p.kW, "groups": p.groups, "stride": p.stride, "pad": p.pad,
+            "layout": args.layout.upper(), "global_batch": p.N * max(1, args.gpus),
+            "l2": "rotating buffer sets larger than 2x L2 between timed steps",
+            "parallelism": f"replicas x{max(1, args.gpus)}"}
+
+
+# ---------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layout", default="nhwc", choices=["nhwc", "nchw"])
+    ap.add_argument("--path", default="auto", choices=["auto", "direct", "igemm", "generic"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-depthwise", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from depthwise_convolution_gconv2d_b200 import binding as gb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    pk, peak_src = peaks()
+
+    p = conv2d_problem(args.layout)
+    path = {"auto": gb.PATH_AUTO, "direct": gb.PATH_DIRECT, "igemm": gb.PATH_IGEMM,
+            "generic": gb.PATH_GENERIC}[args.path]
+    kcode = gb.gconv2d_select_path(p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride, p.pad,
+                                   p.dilation, p.groups, p.layout, p.dtype, path)
+    inp = wl.make_conv2d_inputs(p, 2 + 100 * rank)
+    x_host = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).view(torch.bfloat16)
+    w_host = torch.from_numpy(np.ascontiguousarray(inp.w).view(np.int16)).view(torch.bfloat16)
+    step_bytes = (x_host.numel() + p.N * p.C_out * p.Ho * p.Wo) * 2
+    nsets = max(2, -(-4 * L2_BYTES // step_bytes))       # >= 2x L2 between reuses
+    xs = [x_host.to(device) for _ in range(nsets)]
+    w = w_host.to(device)
+    ys = [torch.empty(p.y_shape, dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+    ws_need = gb.gconv2d_fwd_workspace_size(p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride,
+                                            p.pad, p.dilation, p.groups, p.layout, p.dtype, path)
+    ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=device)
+
+    def step(i):
+        gb.gconv2d_fwd(xs[i % nsets], w, None, p.stride, p.pad, p.dilation, p.groups, p.layout,
+                       out=ys[i % nsets], workspace=ws, path=path, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.25)
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        time.sleep(0.25)
+    total_ms = t_start.elapsed_time(t_end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+
+    flops = p.flops()
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    avg_launch_ms = sum(launch_ms) / len(launch_ms)
+    achieved = flops / (avg_launch_ms * 1e-3) / 1e12
+    tensor_peak = pk["bf16_tflops"]
+    roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tensor_peak,
+            "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4),
+            "traffic": traffic_for(kernel_name(kcode), KERNEL_SOURCE.get(kcode, "")),
+            "kernel": kernel_name(kcode), "peak_source": f"bf16_tflops (burst) {peak_src}"}
+    if kcode in (1, 2):   # CUDA-core kernels on this workload are not tensor-bound
+        roof["note"] = "CUDA-core path selected; tensor peak used as the headline denominator"
+
+    # e2e: host (pinned) -> device copy of x and w, the call, device -> host copy of y
+    e2e = None
+    if True:
+        x_pin = x_host.pin_memory()
+        w_pin = w_host.pin_memory()
+        y_pin = torch.empty(p.y_shape, dtype=torch.bfloat16).pin_memory()
+        xd, wd, yd = xs[0], w, ys[0]
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                xd.copy_(x_pin, non_blocking=True)
+                wd.copy_(w_pin, non_blocking=True)
+            gb.gconv2d_fwd(xd, wd, None, p.stride, p.pad, p.dilation, p.groups, p.layout,
+                           out=yd, workspace=ws, path=path, stream=stream)
+            with torch.cuda.stream(stream):
+                y_pin.copy_(yd, non_blocking=True)
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 10))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": round(flops * world * n_e2e / (e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": (x_host.numel() + w_host.numel()) * 2,
+               "d2h_bytes_per_step": y_pin.numel() * 2, "steps": n_e2e}
+
+    dwm = None
+    if not args.no_depthwise and rank == 0:
+        dwm = depthwise_measurements(torch, gb, device, stream, pk, 20)
+    dev_err = gb.device_error(stream)
+
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        v, dt, rows, thr = oracle_sample(p, inp.x64(), inp.w64(), args.cpu_seconds)
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": f"first {rows} of {p.H} input rows of the workload, fp64 nested loops, "
+                         f"{dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(p, argparse.Namespace(layout=args.layout, gpus=world)),
+            "kernel": kernel_name(kcode), "roofline": roof, "e2e": e2e,
+            "gpu_launches": LAUNCHES_PER_CALL.get(kcode, 1) * args.steps,
+            "clocks": clk.summary(), "cpu_baseline": cpu, "depthwise": dwm,
+            "device_error": dev_err,
+            "peaks": {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                      "source": peak_src},
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

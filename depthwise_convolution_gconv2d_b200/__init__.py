@@ -20,8 +20,8 @@ __all__ = [
 
 
 def __getattr__(name):
-    if name in __all__ or name in ("binding", "NCHW", "NHWC", "PATH_AUTO", "PATH_DIRECT",
-                                   "PATH_IGEMM", "GconvError"):
-        from . import binding
-        return getattr(binding, name) if name != "binding" else binding
+    if name in __all__ or name in ("NCHW", "NHWC", "PATH_AUTO", "PATH_DIRECT", "PATH_IGEMM",
+                                   "PATH_GENERIC", "GconvError"):
+        import importlib
+        return getattr(importlib.import_module(".binding", __name__), name)
     raise AttributeError(name)

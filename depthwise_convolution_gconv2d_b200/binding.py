@@ -1,0 +1,259 @@
+"""ctypes binding over libgconv.so (include/gconv.h).
+
+Argument marshalling only: each function reads sizes from torch CUDA tensors, allocates
+outputs (and the workspace the library asks for) with torch, and passes raw device
+pointers, sizes and the current CUDA stream to the C ABI. Every step of the computation
+runs in the library's kernels. There is no fallback: if the library cannot be loaded,
+``load_library`` raises RuntimeError.
+
+Tensors are taken in their physical (contiguous) layout:
+  NCHW  x [N, C_in, H, W], w [C_out, C_in/g, kH, kW] -> y [N, C_out, Ho, Wo]
+  NHWC  x [N, H, W, C_in], w [C_out, kH, kW, C_in/g] -> y [N, Ho, Wo, C_out]
+  conv1d  x [B, T, C], w [C, K], dy [B, T_out, C]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libgconv.so")
+
+NCHW, NHWC = 0, 1
+F32, F16, BF16 = 0, 1, 2
+PATH_AUTO, PATH_DIRECT, PATH_IGEMM, PATH_GENERIC = 0, 1, 2, 3
+KERNEL_NAMES = {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "igemm_tc_nchw"}
+STATUS = {0: "GCONV_OK", 1: "GCONV_ERR_INVALID_ARG", 2: "GCONV_ERR_UNSUPPORTED",
+          3: "GCONV_ERR_MISALIGNED", 4: "GCONV_ERR_WORKSPACE", 5: "GCONV_ERR_CUDA",
+          6: "GCONV_ERR_DEVICE_TIMEOUT"}
+
+EXPORTS = ["gconv2d_fwd", "gconv2d_fwd_path", "gconv2d_fwd_workspace_size",
+           "gconv2d_select_path", "dwconv1d_fwd", "dwconv1d_bwd_data",
+           "dwconv1d_bwd_weight", "dwconv1d_bwd_weight_workspace_size",
+           "gconv_get_device_error", "gconv_status_string", "gconv_version"]
+
+_lib = None
+
+
+class GconvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libgconv.so once and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m depthwise_convolution_gconv2d_b200.build`")
+    try:
+        lib = ctypes.CDLL(_LIB_PATH)
+    except OSError as e:
+        raise RuntimeError(f"cannot load {_LIB_PATH}: {e}") from e
+    I, P, Z = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+    conv = [I] * 11
+    lib.gconv2d_fwd_workspace_size.argtypes = conv + [I, I, I]
+    lib.gconv2d_fwd_workspace_size.restype = Z
+    lib.gconv2d_fwd.argtypes = [P, P, P, P] + conv + [I, I, P, Z, P]
+    lib.gconv2d_fwd.restype = I
+    lib.gconv2d_fwd_path.argtypes = [P, P, P, P] + conv + [I, I, I, P, Z, P]
+    lib.gconv2d_fwd_path.restype = I
+    lib.gconv2d_select_path.argtypes = conv + [I, I, I]
+    lib.gconv2d_select_path.restype = I
+    lib.dwconv1d_fwd.argtypes = [P, P, P] + [I] * 6 + [I, P]
+    lib.dwconv1d_fwd.restype = I
+    lib.dwconv1d_bwd_data.argtypes = [P, P, P] + [I] * 6 + [I, P]
+    lib.dwconv1d_bwd_data.restype = I
+    lib.dwconv1d_bwd_weight_workspace_size.argtypes = [I] * 7
+    lib.dwconv1d_bwd_weight_workspace_size.restype = Z
+    lib.dwconv1d_bwd_weight.argtypes = [P, P, P, P, Z] + [I] * 6 + [I, P]
+    lib.dwconv1d_bwd_weight.restype = I
+    lib.gconv_get_device_error.argtypes = [P, ctypes.POINTER(I)]
+    lib.gconv_get_device_error.restype = I
+    lib.gconv_status_string.argtypes = [I]
+    lib.gconv_status_string.restype = ctypes.c_char_p
+    lib.gconv_version.argtypes = []
+    lib.gconv_version.restype = I
+    _lib = lib
+    return lib
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return F32
+    if t == torch.float16:
+        return F16
+    if t == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _layout_code(layout) -> int:
+    if isinstance(layout, str):
+        return {"NCHW": NCHW, "NHWC": NHWC}[layout.upper()]
+    return int(layout)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise GconvError(status, where)
+
+
+def _need(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous in its physical layout")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _out_extent(n, k, s, p, d):
+    span = n + 2 * p - d * (k - 1) - 1
+    return span // s + 1 if span >= 0 else 0
+
+
+def conv2d_dims(x, w, stride, padding, dilation, groups, layout):
+    lay = _layout_code(layout)
+    if lay == NCHW:
+        N, C_in, H, W = x.shape
+        C_out, cpg_in, kH, kW = w.shape
+    else:
+        N, H, W, C_in = x.shape
+        C_out, kH, kW, cpg_in = w.shape
+    if cpg_in * groups != C_in:
+        raise ValueError(f"weight has {cpg_in} input channels per group; x has {C_in} channels "
+                         f"in {groups} groups")
+    Ho = _out_extent(H, kH, stride, padding, dilation)
+    Wo = _out_extent(W, kW, stride, padding, dilation)
+    y_shape = (N, C_out, Ho, Wo) if lay == NCHW else (N, Ho, Wo, C_out)
+    return lay, (N, C_in, H, W, C_out, kH, kW), y_shape
+
+
+def gconv2d_fwd_workspace_size(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups,
+                               layout, dtype, path=PATH_AUTO) -> int:
+    return int(load_library().gconv2d_fwd_workspace_size(
+        N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups,
+        _layout_code(layout), dtype if isinstance(dtype, int) else _dtype_code(dtype), path))
+
+
+def gconv2d_select_path(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, layout,
+                        dtype, path=PATH_AUTO) -> int:
+    return int(load_library().gconv2d_select_path(
+        N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, _layout_code(layout),
+        dtype if isinstance(dtype, int) else _dtype_code(dtype), path))
+
+
+def gconv2d_fwd(x, w, bias=None, stride=1, padding=0, dilation=1, groups=1, layout="NCHW",
+                out=None, workspace=None, path=PATH_AUTO, stream=None):
+    """Grouped conv2d forward through the C ABI; returns y."""
+    lib = load_library()
+    _need(x, "x")
+    _need(w, "w", x.dtype)
+    if bias is not None:
+        _need(bias, "bias", x.dtype)
+    lay, dims, y_shape = conv2d_dims(x, w, stride, padding, dilation, groups, layout)
+    dt = _dtype_code(x.dtype)
+    y = torch.empty(y_shape, dtype=x.dtype, device=x.device) if out is None else out
+    _need(y, "out", x.dtype)
+    if tuple(y.shape) != y_shape:
+        raise ValueError(f"out has shape {tuple(y.shape)}, expected {y_shape}")
+    ws_need = lib.gconv2d_fwd_workspace_size(*dims, stride, padding, dilation, groups, lay, dt,
+                                             path)
+    if ws_need and workspace is None:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.gconv2d_fwd_path(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), *dims, stride, padding,
+                              dilation, groups, lay, dt, path, _ptr(workspace), ws_bytes,
+                              _stream(stream))
+    _check(st, "gconv2d_fwd")
+    return y
+
+
+def _conv1d_dims(x, w):
+    B, T, C = x.shape
+    C2, K = w.shape
+    if C2 != C:
+        raise ValueError("w must be [C, K] with the channel count of x")
+    return B, T, C, K
+
+
+def dwconv1d_fwd(x, w, pad_left, pad_right, out=None, stream=None):
+    lib = load_library()
+    _need(x, "x")
+    _need(w, "w", x.dtype)
+    B, T, C, K = _conv1d_dims(x, w)
+    T_out = T + pad_left + pad_right - K + 1
+    y = torch.empty((B, T_out, C), dtype=x.dtype, device=x.device) if out is None else out
+    _need(y, "out", x.dtype)
+    st = lib.dwconv1d_fwd(_ptr(x), _ptr(w), _ptr(y), B, T, C, K, pad_left, pad_right,
+                          _dtype_code(x.dtype), _stream(stream))
+    _check(st, "dwconv1d_fwd")
+    return y
+
+
+def dwconv1d_bwd_data(dy, w, T, pad_left, pad_right, out=None, stream=None):
+    lib = load_library()
+    _need(dy, "dy")
+    _need(w, "w", dy.dtype)
+    B, T_out, C = dy.shape
+    K = w.shape[1]
+    if T_out != T + pad_left + pad_right - K + 1:
+        raise ValueError("dy has the wrong number of steps for T, K and the pads")
+    dx = torch.empty((B, T, C), dtype=dy.dtype, device=dy.device) if out is None else out
+    _need(dx, "out", dy.dtype)
+    st = lib.dwconv1d_bwd_data(_ptr(dy), _ptr(w), _ptr(dx), B, T, C, K, pad_left, pad_right,
+                               _dtype_code(dy.dtype), _stream(stream))
+    _check(st, "dwconv1d_bwd_data")
+    return dx
+
+
+def dwconv1d_bwd_weight_workspace_size(B, T, C, K, pad_left, pad_right, dtype) -> int:
+    dt = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    return int(load_library().dwconv1d_bwd_weight_workspace_size(B, T, C, K, pad_left,
+                                                                 pad_right, dt))
+
+
+def dwconv1d_bwd_weight(x, dy, K, pad_left, pad_right, out=None, workspace=None, stream=None):
+    lib = load_library()
+    _need(x, "x")
+    _need(dy, "dy", x.dtype)
+    B, T, C = x.shape
+    dt = _dtype_code(x.dtype)
+    dw = torch.empty((C, K), dtype=x.dtype, device=x.device) if out is None else out
+    _need(dw, "out", x.dtype)
+    need = lib.dwconv1d_bwd_weight_workspace_size(B, T, C, K, pad_left, pad_right, dt)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.dwconv1d_bwd_weight(_ptr(x), _ptr(dy), _ptr(dw), _ptr(workspace), ws_bytes, B, T,
+                                 C, K, pad_left, pad_right, dt, _stream(stream))
+    _check(st, "dwconv1d_bwd_weight")
+    return dw
+
+
+def device_error(stream=None) -> int:
+    """Synchronise and read/clear the library's device error word (0 = none)."""
+    code = ctypes.c_int(0)
+    st = load_library().gconv_get_device_error(_stream(stream), ctypes.byref(code))
+    if st not in (0, 6):
+        raise GconvError(st, "gconv_get_device_error")
+    return code.value

@@ -1,0 +1,261 @@
+// C ABI of libgconv.so: argument validation, kernel selection and launch.
+//
+// Shape logic (all integer, checked before any launch): C_in and C_out must be multiples of
+// `groups` (the equal split of channels and filters into groups of "Grouped convolutions",
+// neon issue #296), Ho/Wo follow F.conv2d's output-size rule and must be >= 1, and a group
+// index is never stored per element -- it is derived from the output channel in every kernel,
+// so all groups run in one launch (the thread's argument against one launch per group).
+#include <limits.h>
+
+#include <atomic>
+
+#include "internal.cuh"
+
+namespace gconv {
+
+__device__ unsigned int g_device_error;   // set by kernels whose bounded waits give up
+
+unsigned int* device_error_word() {
+  static std::atomic<unsigned int*> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  unsigned int* p = cached[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_device_error) != cudaSuccess) return nullptr;
+  cached[dev].store((unsigned int*)addr, std::memory_order_release);
+  return (unsigned int*)addr;
+}
+
+cudaError_t read_and_clear_device_error(cudaStream_t s, int* code) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (v) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  }
+  *code = (int)v;
+  return e;
+}
+
+namespace {
+
+long long out_extent(long long in, long long k, long long stride, long long pad, long long dil) {
+  const long long span = in + 2 * pad - dil * (k - 1) - 1;
+  return span < 0 ? 0 : span / stride + 1;
+}
+
+// Fills `p`; returns GCONV_OK or GCONV_ERR_INVALID_ARG.
+gconv_status make_conv2d(Conv2d* p, int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                         int stride, int pad, int dil, int groups, int layout, int dtype) {
+  if (N < 0 || C_in <= 0 || H <= 0 || W <= 0 || C_out <= 0 || kH <= 0 || kW <= 0)
+    return GCONV_ERR_INVALID_ARG;
+  if (stride <= 0 || pad < 0 || dil <= 0 || groups <= 0) return GCONV_ERR_INVALID_ARG;
+  if (C_in % groups != 0 || C_out % groups != 0) return GCONV_ERR_INVALID_ARG;
+  if (layout != GCONV_NCHW && layout != GCONV_NHWC) return GCONV_ERR_INVALID_ARG;
+  if (dtype != GCONV_F32 && dtype != GCONV_F16 && dtype != GCONV_BF16) return GCONV_ERR_INVALID_ARG;
+  const long long Ho = out_extent(H, kH, stride, pad, dil);
+  const long long Wo = out_extent(W, kW, stride, pad, dil);
+  if (Ho < 1 || Wo < 1 || Ho > INT_MAX || Wo > INT_MAX) return GCONV_ERR_INVALID_ARG;
+  // element counts must be addressable with 64-bit offsets and sane grid sizes
+  const long long xs = (long long)N * C_in * H * W;
+  const long long ys = (long long)N * C_out * Ho * Wo;
+  if (xs < 0 || ys < 0 || xs > (1LL << 40) || ys > (1LL << 40)) return GCONV_ERR_INVALID_ARG;
+  p->N = N; p->C_in = C_in; p->H = H; p->W = W; p->C_out = C_out; p->kH = kH; p->kW = kW;
+  p->stride = stride; p->pad = pad; p->dil = dil; p->groups = groups;
+  p->Ho = (int)Ho; p->Wo = (int)Wo;
+  p->cpg_in = C_in / groups; p->cpg_out = C_out / groups;
+  p->layout = layout; p->dtype = dtype;
+  return GCONV_OK;
+}
+
+int depthwise_vec_bytes(const Conv2d& p) { return 2 * (p.kH <= 3 ? 8 : (p.kH <= 5 ? 4 : 2)); }
+
+bool aligned_to(const void* ptr, int bytes) {
+  return ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) % (uintptr_t)bytes) == 0;
+}
+
+// Kernel choice. `x`/`y` may be null (query mode: alignment assumed).
+int choose_kernel(const Conv2d& p, int path, const void* x, const void* y, gconv_status* why) {
+  *why = GCONV_OK;
+  const bool query = (x == nullptr && y == nullptr);
+  const bool dw_ok = depthwise_nhwc_supported(p) && p.N <= 65535;
+  const bool dw_al = query || (aligned_to(x, depthwise_vec_bytes(p)) &&
+                               aligned_to(y, depthwise_vec_bytes(p)));
+  const bool tc_ok = igemm_supported(p);
+  const bool tc_al = query || (aligned16(x) && aligned16(y));
+  const int tc_kernel = p.layout == GCONV_NHWC ? GCONV_KERNEL_IGEMM_TC : GCONV_KERNEL_IGEMM_TC_NCHW;
+  switch (path) {
+    case GCONV_PATH_GENERIC:
+      return GCONV_KERNEL_DIRECT_GENERIC;
+    case GCONV_PATH_DIRECT:
+      return (dw_ok && dw_al) ? GCONV_KERNEL_DEPTHWISE_NHWC : GCONV_KERNEL_DIRECT_GENERIC;
+    case GCONV_PATH_IGEMM:
+      if (!tc_ok) { *why = GCONV_ERR_UNSUPPORTED; return -1; }
+      if (!tc_al) { *why = GCONV_ERR_MISALIGNED; return -1; }
+      return tc_kernel;
+    case GCONV_PATH_AUTO:
+      if (p.dtype == GCONV_F32) return GCONV_KERNEL_DIRECT_GENERIC;
+      if (dw_ok && dw_al) return GCONV_KERNEL_DEPTHWISE_NHWC;
+      if (tc_ok && tc_al) return tc_kernel;
+      return GCONV_KERNEL_DIRECT_GENERIC;
+    default:
+      *why = GCONV_ERR_INVALID_ARG;
+      return -1;
+  }
+}
+
+gconv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GCONV_OK : GCONV_ERR_CUDA; }
+
+gconv_status make_conv1d(Conv1d* p, int B, int T, int C, int K, int pl, int pr, int dtype) {
+  if (B < 0 || T <= 0 || C <= 0 || K <= 0 || pl < 0 || pr < 0) return GCONV_ERR_INVALID_ARG;
+  if (dtype != GCONV_F32 && dtype != GCONV_F16 && dtype != GCONV_BF16) return GCONV_ERR_INVALID_ARG;
+  const long long T_out = (long long)T + pl + pr - K + 1;
+  if (T_out < 1 || T_out > INT_MAX) return GCONV_ERR_INVALID_ARG;
+  const long long n = (long long)B * (T > T_out ? T : T_out) * C;
+  if (n > (1LL << 40)) return GCONV_ERR_INVALID_ARG;
+  p->B = B; p->T = T; p->C = C; p->K = K; p->pad_left = pl; p->pad_right = pr;
+  p->T_out = (int)T_out; p->dtype = dtype;
+  return GCONV_OK;
+}
+
+}  // namespace
+}  // namespace gconv
+
+using namespace gconv;
+
+extern "C" {
+
+size_t gconv2d_fwd_workspace_size(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                  int stride, int pad, int dilation, int groups,
+                                  gconv_layout layout, gconv_dtype dtype, gconv_path path) {
+  Conv2d p;
+  if (make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups, layout,
+                  dtype) != GCONV_OK)
+    return 0;
+  gconv_status why;
+  const int k = choose_kernel(p, path, nullptr, nullptr, &why);
+  return k == GCONV_KERNEL_IGEMM_TC_NCHW ? igemm_nchw_workspace(p) : 0;
+}
+
+int gconv2d_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW, int stride,
+                        int pad, int dilation, int groups, gconv_layout layout,
+                        gconv_dtype dtype, gconv_path path) {
+  Conv2d p;
+  gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups,
+                                layout, dtype);
+  if (st != GCONV_OK) return -(int)st;
+  const int k = choose_kernel(p, path, nullptr, nullptr, &st);
+  return k < 0 ? -(int)st : k;
+}
+
+gconv_status gconv2d_fwd_path(const void* x, const void* w, const void* bias, void* y, int N,
+                              int C_in, int H, int W, int C_out, int kH, int kW, int stride,
+                              int pad, int dilation, int groups, gconv_layout layout,
+                              gconv_dtype dtype, gconv_path path, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  Conv2d p;
+  gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups,
+                                layout, dtype);
+  if (st != GCONV_OK) return st;
+  if (N > 0 && (x == nullptr || w == nullptr || y == nullptr)) return GCONV_ERR_INVALID_ARG;
+  const int kernel = choose_kernel(p, path, x, y, &st);
+  if (kernel < 0) return st;
+  if (N == 0) return GCONV_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  switch (kernel) {
+    case GCONV_KERNEL_DEPTHWISE_NHWC:
+      return cuda_status(launch_depthwise_nhwc(p, x, w, bias, y, s));
+    case GCONV_KERNEL_IGEMM_TC:
+      return cuda_status(launch_igemm_nhwc(p, x, w, bias, y, s));
+    case GCONV_KERNEL_IGEMM_TC_NCHW: {
+      const size_t need = igemm_nchw_workspace(p);
+      if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+        return GCONV_ERR_WORKSPACE;
+      return cuda_status(launch_igemm_nchw(p, x, w, bias, y, workspace, s));
+    }
+    default:
+      return cuda_status(launch_direct_generic(p, x, w, bias, y, s));
+  }
+}
+
+gconv_status gconv2d_fwd(const void* x, const void* w, const void* bias, void* y, int N,
+                         int C_in, int H, int W, int C_out, int kH, int kW, int stride, int pad,
+                         int dilation, int groups, gconv_layout layout, gconv_dtype dtype,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  return gconv2d_fwd_path(x, w, bias, y, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation,
+                          groups, layout, dtype, GCONV_PATH_AUTO, workspace, workspace_bytes,
+                          stream);
+}
+
+gconv_status dwconv1d_fwd(const void* x, const void* w, void* y, int B, int T, int C, int K,
+                          int pad_left, int pad_right, gconv_dtype dtype, void* stream) {
+  Conv1d p;
+  gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
+  if (st != GCONV_OK) return st;
+  if (B > 0 && (x == nullptr || w == nullptr || y == nullptr)) return GCONV_ERR_INVALID_ARG;
+  if (B == 0) return GCONV_OK;
+  return cuda_status(launch_dwconv1d_fwd(p, x, w, y, false, pad_left, T, p.T_out,
+                                         (cudaStream_t)stream));
+}
+
+gconv_status dwconv1d_bwd_data(const void* dy, const void* w, void* dx, int B, int T, int C,
+                               int K, int pad_left, int pad_right, gconv_dtype dtype,
+                               void* stream) {
+  Conv1d p;
+  gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
+  if (st != GCONV_OK) return st;
+  if (B > 0 && (dy == nullptr || w == nullptr || dx == nullptr)) return GCONV_ERR_INVALID_ARG;
+  if (B == 0) return GCONV_OK;
+  // dx = forward of dy (T_out steps) with the reversed filter and left pad K-1-pad_left
+  return cuda_status(launch_dwconv1d_fwd(p, dy, w, dx, true, K - 1 - pad_left, p.T_out, T,
+                                         (cudaStream_t)stream));
+}
+
+size_t dwconv1d_bwd_weight_workspace_size(int B, int T, int C, int K, int pad_left,
+                                          int pad_right, gconv_dtype dtype) {
+  Conv1d p;
+  if (make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype) != GCONV_OK) return 0;
+  return dwconv1d_wgrad_workspace(p);
+}
+
+gconv_status dwconv1d_bwd_weight(const void* x, const void* dy, void* dw, void* workspace,
+                                 size_t workspace_bytes, int B, int T, int C, int K,
+                                 int pad_left, int pad_right, gconv_dtype dtype, void* stream) {
+  Conv1d p;
+  gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
+  if (st != GCONV_OK) return st;
+  if (dw == nullptr || (B > 0 && (x == nullptr || dy == nullptr))) return GCONV_ERR_INVALID_ARG;
+  const size_t need = dwconv1d_wgrad_workspace(p);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return GCONV_ERR_WORKSPACE;
+  return cuda_status(launch_dwconv1d_wgrad(p, x, dy, dw, workspace, (cudaStream_t)stream));
+}
+
+gconv_status gconv_get_device_error(void* stream, int* code) {
+  if (code == nullptr) return GCONV_ERR_INVALID_ARG;
+  *code = 0;
+  const cudaError_t e = read_and_clear_device_error((cudaStream_t)stream, code);
+  if (e != cudaSuccess) return GCONV_ERR_CUDA;
+  return *code ? GCONV_ERR_DEVICE_TIMEOUT : GCONV_OK;
+}
+
+const char* gconv_status_string(gconv_status s) {
+  switch (s) {
+    case GCONV_OK: return "GCONV_OK";
+    case GCONV_ERR_INVALID_ARG: return "GCONV_ERR_INVALID_ARG";
+    case GCONV_ERR_UNSUPPORTED: return "GCONV_ERR_UNSUPPORTED";
+    case GCONV_ERR_MISALIGNED: return "GCONV_ERR_MISALIGNED";
+    case GCONV_ERR_WORKSPACE: return "GCONV_ERR_WORKSPACE";
+    case GCONV_ERR_CUDA: return "GCONV_ERR_CUDA";
+    case GCONV_ERR_DEVICE_TIMEOUT: return "GCONV_ERR_DEVICE_TIMEOUT";
+    default: return "GCONV_ERR_UNKNOWN";
+  }
+}
+
+int gconv_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,113 @@
+// Internal declarations shared by the CUDA translation units of libgconv.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "gconv.h"
+
+namespace gconv {
+
+// A validated conv2d problem (all derived sizes filled in by the host dispatcher).
+struct Conv2d {
+  int N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups;
+  int Ho, Wo, cpg_in, cpg_out;
+  int layout;  // GCONV_NCHW / GCONV_NHWC
+  int dtype;   // GCONV_F32 / GCONV_F16 / GCONV_BF16
+};
+
+// A validated depthwise conv1d problem on (batch, steps, channels).
+struct Conv1d {
+  int B, T, C, K, pad_left, pad_right, T_out;
+  int dtype;
+};
+
+// ------------------------------------------------------------------ element conversions
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f32(float v) { return v; }
+  static __device__ __forceinline__ float from_f32(float v) { return v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f32(float v) { return __float2bfloat16_rn(v); }
+};
+template <> struct Elem<__half> {
+  static __device__ __forceinline__ float to_f32(__half v) { return __half2float(v); }
+  static __device__ __forceinline__ __half from_f32(float v) { return __float2half_rn(v); }
+};
+
+// Two packed 16-bit values (low half = lower address) -> float2.
+template <typename T> __device__ __forceinline__ float2 unpack2(uint32_t u);
+template <> __device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t u) {
+  // bf16 is the upper half of an fp32 bit pattern
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+template <> __device__ __forceinline__ float2 unpack2<__half>(uint32_t u) {
+  __half2 h = *reinterpret_cast<__half2*>(&u);
+  return __half22float2(h);
+}
+
+// float2 -> two packed 16-bit values, each rounded to nearest even.
+template <typename T> __device__ __forceinline__ uint32_t pack2(float2 v);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float2 v) {
+  __nv_bfloat162 h = __float22bfloat162_rn(v);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float2 v) {
+  __half2 h = __float22half2_rn(v);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  return __ffma2_rn(a, b, c);
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Raise a kernel's dynamic shared-memory limit once per device (bit i of `mask` = device i).
+inline cudaError_t set_max_dynamic_smem(const void* func, size_t bytes,
+                                        std::atomic<unsigned int>& mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned int bit = 1u << (dev & 31);
+  if (mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) mask.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+// ------------------------------------------------------------------ launchers
+// Each returns cudaSuccess or the launch error. Host-side checks have been done.
+
+cudaError_t launch_direct_generic(const Conv2d& p, const void* x, const void* w, const void* bias,
+                                  void* y, cudaStream_t s);
+
+bool depthwise_nhwc_supported(const Conv2d& p);
+cudaError_t launch_depthwise_nhwc(const Conv2d& p, const void* x, const void* w,
+                                  const void* bias, void* y, cudaStream_t s);
+
+bool igemm_supported(const Conv2d& p);      // shape/dtype eligibility, layout-independent
+size_t igemm_nchw_workspace(const Conv2d& p);
+cudaError_t launch_igemm_nhwc(const Conv2d& p, const void* x, const void* w, const void* bias,
+                              void* y, cudaStream_t s);
+cudaError_t launch_igemm_nchw(const Conv2d& p, const void* x, const void* w, const void* bias,
+                              void* y, void* workspace, cudaStream_t s);
+
+bool conv1d_vector_supported(const Conv1d& p);
+cudaError_t launch_dwconv1d_fwd(const Conv1d& p, const void* x, const void* w, void* y,
+                                bool flip, int pad_left, int T_in, int T_out, cudaStream_t s);
+size_t dwconv1d_wgrad_workspace(const Conv1d& p);
+cudaError_t launch_dwconv1d_wgrad(const Conv1d& p, const void* x, const void* dy, void* dw,
+                                  void* workspace, cudaStream_t s);
+
+// Device error word (set by kernels whose bounded waits give up).
+cudaError_t read_and_clear_device_error(cudaStream_t s, int* code);
+unsigned int* device_error_word();
+
+}  // namespace gconv

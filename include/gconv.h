@@ -1,0 +1,166 @@
+/*
+ * gconv.h -- C ABI of libgconv.so: grouped / depthwise convolution on NVIDIA B200 (sm_100a).
+ *
+ * The operations, and the passages that define them:
+ *
+ *  gconv2d_fwd  Grouped 2-D convolution. Input channels, filters and output channels are
+ *               divided into `groups` equal blocks with no connections between blocks
+ *               ("Grouped convolutions", neon issue #296, thestew42's first reply); output
+ *               channels come out group-major, 111122223333... (same thread, ibmua's post on
+ *               output orderings). groups == C_in is the fully-grouped (depthwise) case of
+ *               that thread. The arithmetic is F.conv2d's cross-correlation with zero padding,
+ *               as called with padding and groups in "F.conv2d runs x15 slower in
+ *               mixed-precision/half-precision mode" (the timing script), where the weight is
+ *               [C_out, C_in/groups, kH, kW]:
+ *                 y[n,co,ho,wo] = bias[co] + sum_{ci<C_in/g, kh<kH, kw<kW}
+ *                     w[co,ci,kh,kw] * x[n, (co / (C_out/g))*(C_in/g) + ci,
+ *                                        ho*stride - pad + kh*dilation,
+ *                                        wo*stride - pad + kw*dilation]
+ *               with x = 0 outside the image and
+ *                 Ho = floor((H + 2*pad - dilation*(kH-1) - 1) / stride) + 1 (same for Wo).
+ *
+ *  dwconv1d_*   Depthwise conv1d over (batch, steps, channels) with groups = channels, the
+ *               Conformer convolution module's depthwise layer ("Investigate custom Triton
+ *               kernels for depthwise-separable convolutions in Conformer", speechbrain #2733:
+ *               the issue text and the Oct 27 comment on the layout), with its backward pass
+ *               (Oct 30 comment):
+ *                 fwd    y[b,t,c]  = sum_{k<K} w[c,k] * x[b, t+k-pad_left, c]
+ *                 dgrad  dx[b,s,c] = sum_{k<K} w[c,k] * dy[b, s-k+pad_left, c]
+ *                 wgrad  dw[c,k]   = sum_{b,t} dy[b,t,c] * x[b, t+k-pad_left, c]
+ *               with x = 0 outside [0, T), dy = 0 outside [0, T_out),
+ *               T_out = T + pad_left + pad_right - K + 1.
+ *
+ * Layouts (dense, row-major, no strides):
+ *   GCONV_NCHW  x[N][C_in][H][W], w[C_out][C_in/g][kH][kW], y[N][C_out][Ho][Wo]
+ *   GCONV_NHWC  x[N][H][W][C_in], w[C_out][kH][kW][C_in/g], y[N][Ho][Wo][C_out]
+ *               (PyTorch's channels_last for activations and weights)
+ *   conv1d      x, dx: [B][T][C]; y, dy: [B][T_out][C]; w, dw: [C][K]
+ *   bias        [C_out] in the data dtype, or NULL.
+ *
+ * Numerics: GCONV_F32 accumulates in fp32 FMA (no TF32); GCONV_F16 / GCONV_BF16 read 16-bit
+ * inputs, accumulate in fp32 (tensor-core TMEM accumulators or CUDA-core FMA) and round the
+ * result once to the data dtype, round-to-nearest-even. dw is written in the data dtype.
+ *
+ * Ownership and calling convention: every pointer is device memory owned by the caller. The
+ * library allocates nothing; scratch comes from the caller's workspace, sized by the
+ * *_workspace_size queries (0 means none is needed). Outputs are overwritten, never
+ * accumulated into. Inputs and outputs must not overlap. All calls validate on the host
+ * first; on any error they return a status, launch nothing and leave the outputs untouched.
+ * Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default stream)
+ * on the current device; the call returns without synchronising. There is no mutable global
+ * state apart from the device error word read by gconv_get_device_error(), so calls on
+ * different streams may be made from different threads.
+ */
+#ifndef GCONV_H_
+#define GCONV_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GCONV_OK = 0,
+  GCONV_ERR_INVALID_ARG = 1,    /* NULL pointer, non-positive size, groups not dividing C_in
+                                   and C_out, window larger than the padded input, bad enum */
+  GCONV_ERR_UNSUPPORTED = 2,    /* a forced path that cannot run this problem */
+  GCONV_ERR_MISALIGNED = 3,     /* a forced vector/tensor-core path whose pointers or channel
+                                   strides are not 16-byte aligned */
+  GCONV_ERR_WORKSPACE = 4,      /* workspace NULL or smaller than the query returned */
+  GCONV_ERR_CUDA = 5,           /* a CUDA runtime/driver call or a kernel launch failed */
+  GCONV_ERR_DEVICE_TIMEOUT = 6  /* a kernel's bounded wait gave up (see gconv_get_device_error) */
+} gconv_status;
+
+typedef enum { GCONV_NCHW = 0, GCONV_NHWC = 1 } gconv_layout;
+
+typedef enum { GCONV_F32 = 0, GCONV_F16 = 1, GCONV_BF16 = 2 } gconv_dtype;
+
+/* Which kernel family runs a gconv2d_fwd problem. AUTO picks one by shape (see
+ * gconv2d_select_path); the others force a family and fail with UNSUPPORTED / MISALIGNED
+ * if it cannot run the problem. */
+typedef enum {
+  GCONV_PATH_AUTO = 0,
+  GCONV_PATH_DIRECT = 1,   /* CUDA-core direct convolution (vectorised depthwise kernel when
+                              it applies, otherwise the generic direct kernel) */
+  GCONV_PATH_IGEMM = 2,    /* per-group implicit GEMM on tcgen05 tensor cores (F16 / BF16) */
+  GCONV_PATH_GENERIC = 3   /* the generic direct kernel (any shape, layout and dtype) */
+} gconv_path;
+
+/* Kernels reported by gconv2d_select_path. */
+typedef enum {
+  GCONV_KERNEL_DIRECT_GENERIC = 1,    /* one thread per output, fp32 FMA, any problem */
+  GCONV_KERNEL_DEPTHWISE_NHWC = 2,    /* 8-channel vectors, sliding window, 16-bit NHWC */
+  GCONV_KERNEL_IGEMM_TC = 3,          /* tcgen05 implicit GEMM, NHWC */
+  GCONV_KERNEL_IGEMM_TC_NCHW = 4      /* NCHW -> NHWC staging in the workspace + tcgen05 */
+} gconv_kernel;
+
+/* Bytes of workspace gconv2d_fwd needs for this problem under `path` (0 if none; also 0 for
+ * invalid arguments, which gconv2d_fwd then rejects). */
+size_t gconv2d_fwd_workspace_size(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                  int stride, int pad, int dilation, int groups,
+                                  gconv_layout layout, gconv_dtype dtype, gconv_path path);
+
+/* Grouped conv2d forward (definition above), kernel chosen automatically. `y` is written in
+ * full. `workspace` may be NULL when gconv2d_fwd_workspace_size(..., GCONV_PATH_AUTO) is 0.
+ * Errors: INVALID_ARG, WORKSPACE, CUDA. Never MISALIGNED: unaligned problems run on a
+ * kernel without the vector requirement. */
+gconv_status gconv2d_fwd(const void* x, const void* w, const void* bias, void* y,
+                         int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                         int stride, int pad, int dilation, int groups,
+                         gconv_layout layout, gconv_dtype dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* gconv2d_fwd with an explicit kernel family (for path sweeps and tests). */
+gconv_status gconv2d_fwd_path(const void* x, const void* w, const void* bias, void* y,
+                              int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                              int stride, int pad, int dilation, int groups,
+                              gconv_layout layout, gconv_dtype dtype, gconv_path path,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* The gconv_kernel that gconv2d_fwd_path would run for this problem, assuming 16-byte
+ * aligned pointers; a negative gconv_status (e.g. -GCONV_ERR_INVALID_ARG) if it would fail. */
+int gconv2d_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW, int stride,
+                        int pad, int dilation, int groups, gconv_layout layout,
+                        gconv_dtype dtype, gconv_path path);
+
+/* Depthwise conv1d forward: x [B][T][C], w [C][K] -> y [B][T_out][C].
+ * Errors: INVALID_ARG (incl. T_out < 1), CUDA. */
+gconv_status dwconv1d_fwd(const void* x, const void* w, void* y, int B, int T, int C, int K,
+                          int pad_left, int pad_right, gconv_dtype dtype, void* stream);
+
+/* Depthwise conv1d data gradient: dy [B][T_out][C], w [C][K] -> dx [B][T][C].
+ * Computed as the forward kernel with the filter reversed and pads (K-1-pad_left,
+ * K-1-pad_right). Errors as dwconv1d_fwd. */
+gconv_status dwconv1d_bwd_data(const void* dy, const void* w, void* dx, int B, int T, int C,
+                               int K, int pad_left, int pad_right, gconv_dtype dtype,
+                               void* stream);
+
+/* Bytes of workspace dwconv1d_bwd_weight needs (fp32 partial sums of fixed slices of B*T_out;
+ * 0 for invalid arguments). */
+size_t dwconv1d_bwd_weight_workspace_size(int B, int T, int C, int K, int pad_left,
+                                          int pad_right, gconv_dtype dtype);
+
+/* Depthwise conv1d weight gradient: x [B][T][C], dy [B][T_out][C] -> dw [C][K].
+ * Deterministic: fixed slices of B*T_out are reduced in a fixed order (no float atomics),
+ * so repeated calls give bitwise-identical dw. Errors: INVALID_ARG, WORKSPACE, CUDA. */
+gconv_status dwconv1d_bwd_weight(const void* x, const void* dy, void* dw, void* workspace,
+                                 size_t workspace_bytes, int B, int T, int C, int K,
+                                 int pad_left, int pad_right, gconv_dtype dtype, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word that kernels with
+ * bounded waits set when a wait gives up. *code receives 0 if none gave up. Returns
+ * GCONV_ERR_DEVICE_TIMEOUT if one did, GCONV_ERR_CUDA if synchronisation failed. */
+gconv_status gconv_get_device_error(void* stream, int* code);
+
+/* Human-readable name of a status. Never NULL. */
+const char* gconv_status_string(gconv_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int gconv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GCONV_H_ */

@@ -1,0 +1,117 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point include/gconv.h
+declares, and host-side validation rejects bad arguments before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from depthwise_convolution_gconv2d_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from depthwise_convolution_gconv2d_b200 import build
+    build.build()
+    return binding.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("gconv2d_fwd", "dwconv1d_fwd", "dwconv1d_bwd_data", "dwconv1d_bwd_weight"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libgconv.so does not export {name}"
+    for name in binding.EXPORTS:
+        assert name in declared_functions()
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS.items():
+        assert lib.gconv_status_string(code).decode() == name
+    assert lib.gconv_status_string(99).decode() == "GCONV_ERR_UNKNOWN"
+    assert lib.gconv_version() >= 100
+
+
+CONV = dict(N=1, C_in=8, H=16, W=16, C_out=8, kH=3, kW=3, stride=1, pad=1, dil=1, groups=4)
+
+
+def _conv_args(**over):
+    a = dict(CONV, **over)
+    return [a[k] for k in ("N", "C_in", "H", "W", "C_out", "kH", "kW", "stride", "pad", "dil",
+                           "groups")]
+
+
+@pytest.mark.parametrize("over", [dict(groups=3), dict(C_out=6), dict(groups=0), dict(kH=0),
+                                  dict(stride=0), dict(pad=-1), dict(dil=0), dict(H=1, pad=0),
+                                  dict(C_in=0), dict(N=-1), dict(W=2, kW=5, pad=1)])
+def test_invalid_conv2d_rejected_before_launch(lib, over):
+    args = _conv_args(**over)
+    # fake, never-dereferenced pointers: validation must fail before any CUDA call
+    p = ctypes.c_void_p(0x1000)
+    st = lib.gconv2d_fwd(p, p, None, p, *args, 0, 2, None, 0, None)
+    assert st == 1, binding.STATUS.get(st)
+    assert lib.gconv2d_select_path(*args, 0, 2, 0) == -1
+    assert lib.gconv2d_fwd_workspace_size(*args, 0, 2, 0) == 0
+
+
+def test_null_pointers_and_bad_enums_rejected(lib):
+    p = ctypes.c_void_p(0x1000)
+    args = _conv_args()
+    assert lib.gconv2d_fwd(None, p, None, p, *args, 0, 2, None, 0, None) == 1
+    assert lib.gconv2d_fwd(p, p, None, None, *args, 0, 2, None, 0, None) == 1
+    assert lib.gconv2d_fwd(p, p, None, p, *args, 2, 2, None, 0, None) == 1    # layout
+    assert lib.gconv2d_fwd(p, p, None, p, *args, 0, 3, None, 0, None) == 1    # dtype
+    assert lib.gconv2d_fwd_path(p, p, None, p, *args, 0, 2, 9, None, 0, None) == 1  # path
+    assert lib.dwconv1d_fwd(None, p, p, 2, 8, 4, 3, 1, 1, 2, None) == 1
+    assert lib.dwconv1d_fwd(p, p, p, 2, 8, 4, 20, 1, 1, 2, None) == 1           # T_out < 1
+    assert lib.dwconv1d_bwd_data(p, p, p, 2, 8, 4, 3, -1, 1, 2, None) == 1
+    assert lib.dwconv1d_bwd_weight(p, p, p, None, 0, 2, 8, 4, 3, 1, 1, 7, None) == 1
+    code = ctypes.c_int(0)
+    assert lib.gconv_get_device_error(None, None) == 1
+
+
+def test_empty_batch_is_a_noop(lib):
+    """N = 0 / B = 0: nothing to compute, nothing launched, OK returned."""
+    p = ctypes.c_void_p(0x1000)
+    assert lib.gconv2d_fwd(None, None, None, None, *_conv_args(N=0), 0, 2, None, 0, None) == 0
+    assert lib.dwconv1d_fwd(None, None, None, 0, 8, 4, 3, 1, 1, 2, None) == 0
+
+
+def test_path_selection(lib):
+    sel = lambda path, **over: lib.gconv2d_select_path(*_conv_args(**over), over.get("layout", 0),
+                                                       over.get("dtype", 2), path)
+    # fp32 always runs the generic direct kernel under AUTO
+    assert lib.gconv2d_select_path(*_conv_args(), 0, 0, 0) == 1
+    # depthwise NHWC bf16 -> vectorised depthwise kernel
+    assert lib.gconv2d_select_path(*_conv_args(C_in=64, C_out=64, groups=64), 1, 2, 0) == 2
+    # depthwise NCHW has no vector kernel: generic
+    assert lib.gconv2d_select_path(*_conv_args(C_in=64, C_out=64, groups=64), 0, 2, 0) == 1
+    # forced generic
+    assert lib.gconv2d_select_path(*_conv_args(C_in=64, C_out=64, groups=64), 1, 2, 3) == 1
+    # the tensor-core path refuses fp32 and narrow groups
+    assert lib.gconv2d_select_path(*_conv_args(), 1, 0, 2) == -2
+    assert lib.gconv2d_select_path(*_conv_args(C_in=32, C_out=32, groups=8), 1, 2, 2) == -2
+
+
+def test_wgrad_workspace_query(lib):
+    n = lib.dwconv1d_bwd_weight_workspace_size(8, 2048, 512, 31, 15, 15, 2)
+    assert n > 0 and n % 4 == 0
+    assert lib.dwconv1d_bwd_weight_workspace_size(8, 2048, 512, 31, 15, 15, 0) == 0   # fp32: generic
+    assert lib.dwconv1d_bwd_weight_workspace_size(8, 10, 512, 31, 0, 0, 2) == 0       # invalid

@@ -1,0 +1,118 @@
+"""GPU parity of dwconv1d_fwd / dwconv1d_bwd_data / dwconv1d_bwd_weight against the fp64
+oracle, on the Conformer workload (x[8, 2048, 512], K = 31, 'same' and causal pads) in full
+and on small ragged shapes; bit-exact on integer-valued data where sums are exact; wgrad
+bitwise reproducible."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from depthwise_convolution_gconv2d_b200 import binding as gb
+from depthwise_convolution_gconv2d_b200 import workloads as wl
+from _util import assert_close, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_all(inp):
+    p = inp.problem
+    x, w, dy = (to_dev(a, p.dtype) for a in (inp.x, inp.w, inp.dy))
+    y = gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right)
+    dx = gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right)
+    dw = gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right)
+    torch.cuda.synchronize()
+    return to_f64(y), to_f64(dx), to_f64(dw)
+
+
+def oracle_all(inp):
+    p = inp.problem
+    x, w, dy = (wl.widen(a, p.dtype) for a in (inp.x, inp.w, inp.dy))
+    return (oracle.dwconv1d_fwd(x, w, p.pad_left, p.pad_right),
+            oracle.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right),
+            oracle.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right))
+
+
+def check(p, workload, dist="normal"):
+    inp = wl.make_dwconv1d_inputs(p, workload, dist)
+    for name, got, ref in zip(("fwd", "dgrad", "wgrad"), gpu_all(inp), oracle_all(inp)):
+        assert_close(got, ref, p.dtype, f"{name} {p}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_conformer_full_size(causal):
+    check(wl.conformer_dw1d(causal), 3)
+
+
+SMALL = [
+    # B, T, C, K, pl, pr
+    (2, 300, 72, 31, 15, 15),     # ragged T and C (vector path)
+    (1, 129, 64, 31, 30, 0),
+    (3, 50, 16, 3, 1, 1),
+    (2, 77, 24, 5, 4, 0),
+    (1, 200, 136, 7, 3, 3),
+    (2, 64, 8, 9, 0, 8),
+    (1, 40, 32, 15, 7, 7),
+    (2, 100, 40, 31, 0, 0),       # T_out < T
+    (1, 20, 8, 31, 15, 15),       # T shorter than the filter
+    (2, 90, 5, 31, 15, 15),       # C not a multiple of 8: generic kernels
+    (1, 33, 16, 4, 2, 1),         # K without an unrolled kernel: generic
+    (2, 45, 24, 11, 10, 0),
+]
+
+
+@pytest.mark.parametrize("case", SMALL)
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F16, wl.F32])
+def test_small_shapes(case, dtype):
+    check(wl.Dwconv1dProblem(*case, dtype), 30)
+
+
+@pytest.mark.parametrize("case", SMALL[:8])
+def test_integer_valued_bit_exact_fwd_dgrad(case):
+    """Integers in [-2, 2]: every partial sum is exact in fp32 and the result (|.| <= 124)
+    is exact in bf16, so any summation order gives the oracle's value bit for bit."""
+    p = wl.Dwconv1dProblem(*case, wl.BF16)
+    inp = wl.make_dwconv1d_inputs(p, 31, "int")
+    inp.w = wl.to_storage(np.random.default_rng(5).integers(-2, 3, (p.C, p.K)), wl.BF16)
+    (y, dx, _), (ry, rdx, _) = gpu_all(inp), oracle_all(inp)
+    assert np.array_equal(y, ry)
+    assert np.array_equal(dx, rdx)
+
+
+def test_wgrad_deterministic():
+    p = wl.conformer_dw1d(False)
+    inp = wl.make_dwconv1d_inputs(p, 3)
+    x, dy = to_dev(inp.x, p.dtype), to_dev(inp.dy, p.dtype)
+    ref = gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right).clone()
+    for _ in range(10):
+        again = gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right)
+        assert torch.equal(again.view(torch.int16), ref.view(torch.int16))
+
+
+def test_wgrad_workspace_too_small_rejected():
+    p = wl.conformer_dw1d(False)
+    inp = wl.make_dwconv1d_inputs(p, 3)
+    x, dy = to_dev(inp.x, p.dtype), to_dev(inp.dy, p.dtype)
+    need = gb.dwconv1d_bwd_weight_workspace_size(p.B, p.T, p.C, p.K, p.pad_left, p.pad_right,
+                                                 p.dtype)
+    ws = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(gb.GconvError) as e:
+        gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right, workspace=ws)
+    assert e.value.status == 4
+
+
+def test_guard_bands_untouched():
+    p = wl.Dwconv1dProblem(2, 300, 72, 31, 15, 15, wl.BF16)
+    inp = wl.make_dwconv1d_inputs(p, 32)
+    x, w, dy = (to_dev(a, p.dtype) for a in (inp.x, inp.w, inp.dy))
+    guard = 2048
+    for shape, fn in (((p.B, p.T_out, p.C), lambda o: gb.dwconv1d_fwd(x, w, 15, 15, out=o)),
+                      ((p.B, p.T, p.C), lambda o: gb.dwconv1d_bwd_data(dy, w, p.T, 15, 15, out=o)),
+                      ((p.C, p.K), lambda o: gb.dwconv1d_bwd_weight(x, dy, p.K, 15, 15, out=o))):
+        n = int(np.prod(shape))
+        buf = torch.full((n + 2 * guard,), float("nan"), dtype=torch.bfloat16, device="cuda")
+        sent = buf[:guard].view(torch.int16).clone()
+        fn(buf[guard:guard + n].view(shape))
+        torch.cuda.synchronize()
+        assert torch.equal(buf[:guard].view(torch.int16), sent)
+        assert torch.equal(buf[guard + n:].view(torch.int16), sent)
+        assert not torch.isnan(buf[guard:guard + n]).any()
