@@ -149,6 +149,13 @@ def l2_flusher(torch, device):
     return flush
 
 
+def gpu_spin(torch, stream, us=200):
+    """Keep the stream busy for ~`us` microseconds so that the host has enqueued what follows
+    before the GPU reaches it (host launch latency stays outside event brackets)."""
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(us * 2000))
+
+
 def time_launches(torch, fn, stream, reps, flush=None):
     """Median and mean CUDA-event time (ms) of `fn(i)` over `reps` launches on `stream`,
     flushing L2 before each launch outside the event bracket."""
@@ -156,6 +163,7 @@ def time_launches(torch, fn, stream, reps, flush=None):
     for i in range(reps):
         if flush is not None:
             flush(stream)
+        gpu_spin(torch, stream)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -348,9 +356,21 @@ def main():
                                             p.pad, p.dilation, p.groups, p.layout, p.dtype, path)
     ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=device)
 
+    # the C ABI call with its arguments marshalled once (device pointers rotate per step)
+    import ctypes
+    lib = gb.load_library()
+    fixed = (p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride, p.pad, p.dilation, p.groups,
+             p.layout, p.dtype, path)
+    tail = (ctypes.c_void_p(ws.data_ptr()), ctypes.c_size_t(ws.numel()),
+            ctypes.c_void_p(stream.cuda_stream))
+    wptr = ctypes.c_void_p(w.data_ptr())
+    xptrs = [ctypes.c_void_p(t.data_ptr()) for t in xs]
+    yptrs = [ctypes.c_void_p(t.data_ptr()) for t in ys]
+
     def step(i):
-        gb.gconv2d_fwd(xs[i % nsets], w, None, p.stride, p.pad, p.dilation, p.groups, p.layout,
-                       out=ys[i % nsets], workspace=ws, path=path, stream=stream)
+        st = lib.gconv2d_fwd_path(xptrs[i % nsets], wptr, None, yptrs[i % nsets], *fixed, *tail)
+        if st != 0:
+            raise gb.GconvError(st, "gconv2d_fwd_path")
 
     for i in range(args.warmup):
         step(i)
@@ -365,6 +385,7 @@ def main():
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         time.sleep(0.25)
+        gpu_spin(torch, stream, 500)
         t_start.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
@@ -413,6 +434,7 @@ def main():
         torch.cuda.synchronize()
         n_e2e = max(3, min(args.steps, 10))
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        gpu_spin(torch, stream)
         a.record(stream)
         for _ in range(n_e2e):
             e2e_step()

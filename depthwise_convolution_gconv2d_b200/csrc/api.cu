@@ -78,15 +78,18 @@ bool aligned_to(const void* ptr, int bytes) {
   return ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) % (uintptr_t)bytes) == 0;
 }
 
-// Kernel choice. `x`/`y` may be null (query mode: alignment assumed).
-int choose_kernel(const Conv2d& p, int path, const void* x, const void* y, gconv_status* why) {
+// Kernel choice. `x`/`w`/`y` may all be null (query mode: alignment assumed).
+int choose_kernel(const Conv2d& p, int path, const void* x, const void* w, const void* y,
+                  gconv_status* why) {
   *why = GCONV_OK;
-  const bool query = (x == nullptr && y == nullptr);
+  const bool query = (x == nullptr && w == nullptr && y == nullptr);
   const bool dw_ok = depthwise_nhwc_supported(p) && p.N <= 65535;
   const bool dw_al = query || (aligned_to(x, depthwise_vec_bytes(p)) &&
                                aligned_to(y, depthwise_vec_bytes(p)));
   const bool tc_ok = igemm_supported(p);
-  const bool tc_al = query || (aligned16(x) && aligned16(y));
+  // tensor maps need 16-byte aligned bases (x, and w when it is used in place: NHWC)
+  const bool tc_al = query || (aligned16(x) && aligned16(y) &&
+                               (p.layout == GCONV_NCHW || aligned16(w)));
   const int tc_kernel = p.layout == GCONV_NHWC ? GCONV_KERNEL_IGEMM_TC : GCONV_KERNEL_IGEMM_TC_NCHW;
   switch (path) {
     case GCONV_PATH_GENERIC:
@@ -137,7 +140,7 @@ size_t gconv2d_fwd_workspace_size(int N, int C_in, int H, int W, int C_out, int 
                   dtype) != GCONV_OK)
     return 0;
   gconv_status why;
-  const int k = choose_kernel(p, path, nullptr, nullptr, &why);
+  const int k = choose_kernel(p, path, nullptr, nullptr, nullptr, &why);
   return k == GCONV_KERNEL_IGEMM_TC_NCHW ? igemm_nchw_workspace(p) : 0;
 }
 
@@ -148,7 +151,7 @@ int gconv2d_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW
   gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups,
                                 layout, dtype);
   if (st != GCONV_OK) return -(int)st;
-  const int k = choose_kernel(p, path, nullptr, nullptr, &st);
+  const int k = choose_kernel(p, path, nullptr, nullptr, nullptr, &st);
   return k < 0 ? -(int)st : k;
 }
 
@@ -162,7 +165,7 @@ gconv_status gconv2d_fwd_path(const void* x, const void* w, const void* bias, vo
                                 layout, dtype);
   if (st != GCONV_OK) return st;
   if (N > 0 && (x == nullptr || w == nullptr || y == nullptr)) return GCONV_ERR_INVALID_ARG;
-  const int kernel = choose_kernel(p, path, x, y, &st);
+  const int kernel = choose_kernel(p, path, x, w, y, &st);
   if (kernel < 0) return st;
   if (N == 0) return GCONV_OK;
   cudaStream_t s = (cudaStream_t)stream;

@@ -1,17 +1,669 @@
-// Per-group implicit GEMM on tcgen05 tensor cores (placeholder until the kernel lands).
+// Per-group implicit GEMM for grouped conv2d on tcgen05 tensor cores (sm_100a).
+//
+// For group j the convolution is a GEMM  D[M x N] = A[M x K] * B[K x N]  with
+//   M = N_img * Ho * Wo output pixels, N = C_out/g filters of the group,
+//   K = kH * kW * (C_in/g): for each filter tap, the group's input channels,
+// and A is never materialised (no im2col). Grouped convolutions fall off the fp16
+// tensor-core path in the half-precision thread ("F.conv2d runs x15 slower in mixed-precision/
+// half-precision mode", second reply); this kernel puts every group on the tensor cores in
+// one launch, with the group index taken from the tile index -- the "offset the input and
+// output by the group from the grid" idea of "Grouped convolutions" (neon issue #296).
+//
+// Data path (NHWC activations, weights [C_out][kH][kW][C_in/g]):
+//  * a tile is 128 output pixels (BH rows x BW columns of one image) x BN filters of one group;
+//  * k-block = (tap (kh, kw), block of BKC <= 64 input channels): TMA loads the 4-D box
+//    x[n, ho0-pad+kh*dil .., wo0-pad+kw*dil .., c-block] straight into a K-major,
+//    BKC*2-byte-swizzled shared tile -- the tap shift is the box origin and the tensor-map's
+//    zero fill outside the image is the padding -- and a 2-D box of the weights;
+//  * one thread issues tcgen05.mma (kind::f16, bf16/fp16 in, fp32 accumulate) from the two
+//    shared tiles into a TMEM accumulator; tcgen05.commit frees the stage;
+//  * four epilogue warps read the accumulator with tcgen05.ld, add the bias, round to the
+//    output dtype and store (NHWC vector stores, or NCHW stores coalesced along W).
+// Persistent CTAs walk the tile list; TMEM holds two accumulators so the epilogue of one tile
+// overlaps the MMAs of the next. Every mbarrier wait is bounded (globaltimer); a wait that
+// gives up sets the library's device error word and the CTA winds down cleanly.
+//
+// NCHW: the activations are first transposed to NHWC and the weights repacked to
+// [C_out][kH][kW][C_in/g] in the caller's workspace (two small kernels), and the epilogue
+// writes NCHW directly.
+#include <cuda.h>
+
 #include "internal.cuh"
 
 namespace gconv {
+namespace {
 
-bool igemm_supported(const Conv2d&) { return false; }
-size_t igemm_nchw_workspace(const Conv2d&) { return 0; }
-cudaError_t launch_igemm_nhwc(const Conv2d&, const void*, const void*, const void*, void*,
-                              cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int BM = 128;                 // output pixels per tile (UMMA M)
+constexpr int NUM_THREADS = 192;        // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
+constexpr int MAX_STAGES = 32;
+constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;   // 1 s
+constexpr size_t SMEM_BUDGET = 227 * 1024;
+
+enum : unsigned int { ERR_WAIT_PRODUCER = 1u, ERR_WAIT_MMA = 2u, ERR_WAIT_EPILOGUE = 4u,
+                      ERR_WAIT_DRAIN = 8u };
+
+struct IgemmParams {
+  int N, H, W, C_in, C_out, Ho, Wo, kW, pad, dil, cpg_in, cpg_out;
+  int BW, BH, BN, BKC, cblocks, kblocks, tiles_w, tiles_h, m_tiles, n_tiles, num_tiles;
+  int stages;
+  unsigned int tx_bytes;       // TMA bytes per stage (A box + B box)
+  unsigned int a_stage, b_stage;
+  unsigned int idesc;
+  unsigned int swz;            // smem-descriptor layout code
+  unsigned int sbo;            // bytes between 8-row core-matrix groups
+  unsigned int tmem_cols;
+  int out_nchw;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ unsigned int smem_u32(const void* p) {
+  return (unsigned int)__cvta_generic_to_shared(p);
 }
-cudaError_t launch_igemm_nchw(const Conv2d&, const void*, const void*, const void*, void*, void*,
-                              cudaStream_t) {
-  return cudaErrorNotSupported;
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, unsigned int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, unsigned int bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned int parity) {
+  unsigned int ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with `parity` to complete; gives up after WAIT_LIMIT_NS (sets the CTA's
+// abort flag and the device error word) or when another role has aborted.
+__device__ __noinline__ bool mbar_wait(unsigned long long* bar, unsigned int parity,
+                                       volatile int* abort_flag, unsigned int* err,
+                                       unsigned int code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+      *abort_flag = 1;
+      if (err) atomicOr(err, code);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* map, unsigned long long* bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, unsigned long long* bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(unsigned int* slot, unsigned int ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(unsigned int taddr, unsigned int ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D(tmem) (+)= A(smem desc) * B(smem desc), kind::f16, issued by one thread.
+__device__ __forceinline__ void umma_f16(unsigned int d_tmem, unsigned long long a_desc,
+                                         unsigned long long b_desc, unsigned int idesc,
+                                         unsigned int accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05.mma this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(unsigned long long* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// Warp-collective: lane i reads TMEM lane (base lane + i), 32 / 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld32(unsigned int taddr, unsigned int (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16(unsigned int taddr, unsigned int (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading / stride byte offsets
+// (16-byte units), descriptor version 1 at bits 46-47, layout (swizzle) code at bits 61-63.
+__device__ __forceinline__ unsigned long long smem_desc(unsigned int saddr, unsigned int sbo,
+                                                        unsigned int swz) {
+  unsigned long long d = (unsigned long long)((saddr >> 4) & 0x3FFFu);
+  d |= (unsigned long long)1u << 16;                          // LBO (unused for swizzled K-major)
+  d |= (unsigned long long)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (unsigned long long)1u << 46;
+  d |= (unsigned long long)(swz & 7u) << 61;
+  return d;
+}
+
+template <typename T>
+__device__ __forceinline__ void epilogue_store(const IgemmParams& P, T* __restrict__ y,
+                                               const T* __restrict__ bias, const unsigned int* r,
+                                               int ncols, int n, int ho, int wo, int co) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (bias) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < ncols) v[i] += Elem<T>::to_f32(bias[co + i]);
+  }
+  if (!P.out_nchw) {
+    T* dst = y + (((long long)n * P.Ho + ho) * P.Wo + wo) * P.C_out + co;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (q * 8 < ncols) {
+        uint4 u;
+        u.x = pack2<T>(make_float2(v[8 * q + 0], v[8 * q + 1]));
+        u.y = pack2<T>(make_float2(v[8 * q + 2], v[8 * q + 3]));
+        u.z = pack2<T>(make_float2(v[8 * q + 4], v[8 * q + 5]));
+        u.w = pack2<T>(make_float2(v[8 * q + 6], v[8 * q + 7]));
+        *reinterpret_cast<uint4*>(dst + 8 * q) = u;
+      }
+    }
+  } else {
+    const long long plane = (long long)P.Ho * P.Wo;
+    T* dst = y + ((long long)n * P.C_out + co) * plane + (long long)ho * P.Wo + wo;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < ncols) dst[i * plane] = Elem<T>::from_f32(v[i]);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    igemm_tc_kernel(const __grid_constant__ CUtensorMap tma_x,
+                    const __grid_constant__ CUtensorMap tma_w, const T* __restrict__ bias,
+                    T* __restrict__ y, const IgemmParams P, unsigned int* err) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* a_base = smem;
+  unsigned char* b_base = smem + (size_t)P.stages * P.a_stage;
+  unsigned long long* bars =
+      reinterpret_cast<unsigned long long*>(b_base + (size_t)P.stages * P.b_stage);
+  unsigned long long* full = bars;
+  unsigned long long* empty = bars + MAX_STAGES;
+  unsigned long long* tfull = bars + 2 * MAX_STAGES;
+  unsigned long long* tempty = tfull + 2;
+  unsigned long long* done = tempty + 2;
+  unsigned int* tmem_slot = reinterpret_cast<unsigned int*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tma_x);
+    prefetch_tmap(&tma_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, P.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const unsigned int tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int s = 0;
+      unsigned int ph = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
+        const int mt = t % P.m_tiles, rest = t / P.m_tiles;
+        const int nt = rest % P.n_tiles, j = rest / P.n_tiles;
+        const int tw = mt % P.tiles_w, r2 = mt / P.tiles_w;
+        const int th = r2 % P.tiles_h, n = r2 / P.tiles_h;
+        const int hbase = th * P.BH - P.pad, wbase = tw * P.BW - P.pad;
+        const int cbase = j * P.cpg_in, obase = j * P.cpg_out + nt * P.BN;
+        for (int kb = 0; kb < P.kblocks; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          const int tap = kb / P.cblocks, cb = kb - tap * P.cblocks;
+          const int kh = tap / P.kW, kw = tap - kh * P.kW;
+          mbar_arrive_expect_tx(&full[s], P.tx_bytes);
+          tma_load_4d(a_base + (size_t)s * P.a_stage, &tma_x, &full[s], cbase + cb * P.BKC,
+                      wbase + kw * P.dil, hbase + kh * P.dil, n);
+          tma_load_2d(b_base + (size_t)s * P.b_stage, &tma_w, &full[s],
+                      tap * P.cpg_in + cb * P.BKC, obase);
+          ++issued;
+          if (++s == P.stages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      // copies in flight must land before the CTA can exit (no-op on the normal path)
+      const long long first = issued > P.stages ? issued - P.stages : 0;
+      for (long long i = first; i < issued; ++i)
+        mbar_wait(&full[i % P.stages], (unsigned int)((i / P.stages) & 1), abort_flag, err,
+                  ERR_WAIT_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int s = 0, acc = 0;
+      unsigned int ph = 0, aph = 0;
+      bool ok = true;
+      const int ksteps = P.BKC / 16;
+      for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERR_WAIT_MMA)) break;
+        tc_fence_after();
+        const unsigned int d_tmem = tmem_base + (unsigned int)(acc * P.BN);
+        for (int kb = 0; kb < P.kblocks; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag, err, ERR_WAIT_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const unsigned int a_addr = smem_u32(a_base + (size_t)s * P.a_stage);
+          const unsigned int b_addr = smem_u32(b_base + (size_t)s * P.b_stage);
+          for (int kk = 0; kk < ksteps; ++kk) {
+            const unsigned long long ad = smem_desc(a_addr + kk * 32, P.sbo, P.swz);
+            const unsigned long long bd = smem_desc(b_addr + kk * 32, P.sbo, P.swz);
+            umma_f16(d_tmem, ad, bd, P.idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          if (++s == P.stages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          aph ^= 1u;
+        }
+      }
+      // every issued MMA must complete before TMEM is released
+      umma_commit(done);
+      mbar_wait(done, 0, abort_flag, err, ERR_WAIT_DRAIN);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5, TMEM lane quarter (warp % 4)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int hl = row / P.BW, wl = row - hl * P.BW;
+    int acc = 0;
+    unsigned int aph = 0;
+    for (int t = blockIdx.x; t < P.num_tiles; t += gridDim.x) {
+      const int mt = t % P.m_tiles, rest = t / P.m_tiles;
+      const int nt = rest % P.n_tiles, j = rest / P.n_tiles;
+      const int tw = mt % P.tiles_w, r2 = mt / P.tiles_w;
+      const int th = r2 % P.tiles_h, n = r2 / P.tiles_h;
+      const bool got = mbar_wait(&tfull[acc], aph, abort_flag, err, ERR_WAIT_EPILOGUE);
+      if (!__all_sync(0xffffffffu, got)) break;    // warp-uniform: tcgen05.ld is .aligned
+      tc_fence_after();
+      const int ho = th * P.BH + hl, wo = tw * P.BW + wl;
+      const bool valid = hl < P.BH && ho < P.Ho && wo < P.Wo;
+      const int co0 = j * P.cpg_out + nt * P.BN;
+      const unsigned int taddr =
+          tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.BN);
+      for (int c = 0; c < P.BN; c += 32) {
+        unsigned int r[32];
+        const int ncols = P.BN - c < 32 ? P.BN - c : 32;
+        if (ncols == 32)
+          tmem_ld32(taddr + c, r);
+        else
+          tmem_ld16(taddr + c, r);
+        tmem_ld_wait();
+        if (valid) epilogue_store<T>(P, y, bias, r, ncols, n, ho, wo, co0 + c);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, P.tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------------ NCHW staging kernels
+
+// x[n][c][hw] -> xt[n][hw][c], 64 x 64 tiles through shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const T* __restrict__ x,
+                                                           T* __restrict__ xt, int C, int HW) {
+  __shared__ T tile[64][66];
+  const int n = blockIdx.z;
+  const int c0 = blockIdx.y * 64, s0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const T* xn = x + (long long)n * C * HW;
+  T* tn = xt + (long long)n * C * HW;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int c = c0 + ty + 8 * r;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int s = s0 + tx + 32 * h;
+      if (c < C && s < HW) tile[ty + 8 * r][tx + 32 * h] = xn[(long long)c * HW + s];
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int s = s0 + ty + 8 * r;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = c0 + tx + 32 * h;
+      if (c < C && s < HW) tn[(long long)s * C + c] = tile[tx + 32 * h][ty + 8 * r];
+    }
+  }
+}
+
+// w[co][ci][kh][kw] -> wt[co][kh][kw][ci]
+template <typename T>
+__global__ void repack_weight_kernel(const T* __restrict__ w, T* __restrict__ wt, int C_out,
+                                     int cpg_in, int taps) {
+  const long long total = (long long)C_out * cpg_in * taps;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int ci = (int)(i % cpg_in);
+    const long long r = i / cpg_in;
+    const int tap = (int)(r % taps);
+    const int co = (int)(r / taps);
+    wt[i] = w[((long long)co * cpg_in + ci) * taps + tap];
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (f) return f;
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || p == nullptr)
+    return nullptr;
+  f = reinterpret_cast<EncodeTiledFn>(p);
+  fn.store(f, std::memory_order_release);
+  return f;
+}
+
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int v = cached[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    v = 148;
+  cached[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+int tile_bn(const Conv2d& p) {
+  if (p.cpg_out <= 256) return p.cpg_out;
+  return p.cpg_out % 128 == 0 ? 128 : 0;
+}
+
+unsigned int pow2_cols(int n) {
+  unsigned int c = 32;
+  while ((int)c < n) c <<= 1;
+  return c;
+}
+
+bool make_params(const Conv2d& p, IgemmParams* P) {
+  P->N = p.N; P->H = p.H; P->W = p.W; P->C_in = p.C_in; P->C_out = p.C_out;
+  P->Ho = p.Ho; P->Wo = p.Wo; P->kW = p.kW; P->pad = p.pad; P->dil = p.dil;
+  P->cpg_in = p.cpg_in; P->cpg_out = p.cpg_out;
+  P->BW = p.Wo < BM ? p.Wo : BM;
+  P->BH = BM / P->BW;
+  if (P->BH > p.Ho) P->BH = p.Ho;
+  P->BN = tile_bn(p);
+  P->BKC = p.cpg_in % 64 == 0 ? 64 : (p.cpg_in % 32 == 0 ? 32 : 16);
+  P->cblocks = p.cpg_in / P->BKC;
+  P->kblocks = p.kH * p.kW * P->cblocks;
+  P->tiles_w = (p.Wo + P->BW - 1) / P->BW;
+  P->tiles_h = (p.Ho + P->BH - 1) / P->BH;
+  const long long m_tiles = (long long)p.N * P->tiles_w * P->tiles_h;
+  P->n_tiles = p.cpg_out / P->BN;
+  const long long tiles = m_tiles * P->n_tiles * p.groups;
+  if (m_tiles > INT32_MAX || tiles > INT32_MAX) return false;
+  P->m_tiles = (int)m_tiles;
+  P->num_tiles = (int)tiles;
+  const unsigned int row_bytes = (unsigned int)P->BKC * 2u;
+  P->a_stage = (BM * row_bytes + 1023u) & ~1023u;
+  P->b_stage = ((unsigned int)P->BN * row_bytes + 1023u) & ~1023u;
+  P->tx_bytes = (unsigned int)(P->BW * P->BH) * row_bytes + (unsigned int)P->BN * row_bytes;
+  const size_t fixed = 1024 + (2 * MAX_STAGES + 5) * 8 + 16;
+  int stages = (int)((SMEM_BUDGET - fixed) / (P->a_stage + P->b_stage));
+  if (stages > MAX_STAGES) stages = MAX_STAGES;
+  if (stages < 2) return false;
+  P->stages = stages;
+  P->swz = row_bytes == 128 ? 2u : (row_bytes == 64 ? 4u : 6u);   // 128B / 64B / 32B swizzle
+  P->sbo = 8u * row_bytes;
+  const unsigned int fmt = p.dtype == GCONV_BF16 ? 1u : 0u;        // A/B: 0 = f16, 1 = bf16
+  P->idesc = (1u << 4)                     // D format: f32
+             | (fmt << 7) | (fmt << 10)    // A, B formats
+             | ((unsigned int)(P->BN >> 3) << 17)   // N / 8
+             | ((unsigned int)(BM >> 4) << 24);     // M / 16
+  P->tmem_cols = pow2_cols(2 * P->BN);
+  P->out_nchw = p.layout == GCONV_NCHW;
+  return true;
+}
+
+size_t smem_bytes(const IgemmParams& P) {
+  return 1024 + (size_t)P.stages * (P.a_stage + P.b_stage) + (2 * MAX_STAGES + 5) * 8 + 16;
+}
+
+CUtensorMapSwizzle swizzle_of(int BKC) {
+  return BKC == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                   : (BKC == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+// x: NHWC activations, w: [C_out][kH][kW][cpg_in] weights (both device pointers).
+template <typename T>
+cudaError_t launch_core(const Conv2d& p, const IgemmParams& P, const void* x, const void* w,
+                        const void* bias, void* y, cudaStream_t s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const CUtensorMapDataType dt =
+      p.dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tx, tw;
+  const cuuint64_t xdim[4] = {(cuuint64_t)p.C_in, (cuuint64_t)p.W, (cuuint64_t)p.H,
+                              (cuuint64_t)p.N};
+  const cuuint64_t xstr[3] = {(cuuint64_t)p.C_in * 2, (cuuint64_t)p.W * p.C_in * 2,
+                              (cuuint64_t)p.H * p.W * p.C_in * 2};
+  const cuuint32_t xbox[4] = {(cuuint32_t)P.BKC, (cuuint32_t)P.BW, (cuuint32_t)P.BH, 1};
+  const cuuint32_t ones[4] = {1, 1, 1, 1};
+  if (enc(&tx, dt, 4, const_cast<void*>(x), xdim, xstr, xbox, ones,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(P.BKC), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const cuuint64_t ktot = (cuuint64_t)p.kH * p.kW * p.cpg_in;
+  const cuuint64_t wdim[2] = {ktot, (cuuint64_t)p.C_out};
+  const cuuint64_t wstr[1] = {ktot * 2};
+  const cuuint32_t wbox[2] = {(cuuint32_t)P.BKC, (cuuint32_t)P.BN};
+  if (enc(&tw, dt, 2, const_cast<void*>(w), wdim, wstr, wbox, ones,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(P.BKC), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const size_t smem = smem_bytes(P);
+  if (smem > SMEM_BUDGET) return cudaErrorInvalidValue;
+  // the limit is raised once per device to the full budget, so every tile shape fits
+  static std::atomic<unsigned int> configured{0};
+  cudaError_t e = set_max_dynamic_smem((const void*)igemm_tc_kernel<T>, SMEM_BUDGET, configured);
+  if (e != cudaSuccess) return e;
+  int grid = sm_count();
+  if (grid > P.num_tiles) grid = P.num_tiles;
+  igemm_tc_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, tw, (const T*)bias, (T*)y, P,
+                                                     device_error_word());
+  return cudaGetLastError();
+}
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+}  // namespace
+
+// Eligibility of the tensor-core path: 16-bit data, stride 1, channels per group multiples
+// of 16 (UMMA K granularity and 16-byte TMA rows), filters per group 16..256 (UMMA N) or a
+// multiple of 128, and tile bookkeeping within int range.
+bool igemm_supported(const Conv2d& p) {
+  if (p.dtype != GCONV_BF16 && p.dtype != GCONV_F16) return false;
+  if (p.stride != 1) return false;
+  if (p.cpg_in % 16 != 0 || p.cpg_out % 16 != 0) return false;
+  if (tile_bn(p) == 0) return false;
+  if (p.N > 65535 || p.H > 65535 || p.W > 65535) return false;
+  IgemmParams P;
+  return make_params(p, &P);
+}
+
+size_t igemm_nchw_workspace(const Conv2d& p) {
+  return align256((size_t)p.N * p.H * p.W * p.C_in * 2) +
+         align256((size_t)p.C_out * p.kH * p.kW * p.cpg_in * 2);
+}
+
+cudaError_t launch_igemm_nhwc(const Conv2d& p, const void* x, const void* w, const void* bias,
+                              void* y, cudaStream_t s) {
+  IgemmParams P;
+  if (!make_params(p, &P)) return cudaErrorNotSupported;
+  if (p.dtype == GCONV_BF16) return launch_core<__nv_bfloat16>(p, P, x, w, bias, y, s);
+  return launch_core<__half>(p, P, x, w, bias, y, s);
+}
+
+template <typename T>
+cudaError_t launch_nchw_typed(const Conv2d& p, const IgemmParams& P, const void* x, const void* w,
+                              const void* bias, void* y, void* workspace, cudaStream_t s) {
+  T* xt = (T*)workspace;
+  T* wt = (T*)((char*)workspace + align256((size_t)p.N * p.H * p.W * p.C_in * 2));
+  const int taps = p.kH * p.kW;
+  const long long wtotal = (long long)p.C_out * p.cpg_in * taps;
+  long long wb = (wtotal + 255) / 256;
+  if (wb > 4096) wb = 4096;
+  repack_weight_kernel<T><<<(unsigned)wb, 256, 0, s>>>((const T*)w, wt, p.C_out, p.cpg_in, taps);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int HW = p.H * p.W;
+  dim3 grid((HW + 63) / 64, (p.C_in + 63) / 64, p.N);
+  nchw_to_nhwc_kernel<T><<<grid, 256, 0, s>>>((const T*)x, xt, p.C_in, HW);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_core<T>(p, P, xt, wt, bias, y, s);
+}
+
+cudaError_t launch_igemm_nchw(const Conv2d& p, const void* x, const void* w, const void* bias,
+                              void* y, void* workspace, cudaStream_t s) {
+  IgemmParams P;
+  if (!make_params(p, &P)) return cudaErrorNotSupported;
+  if ((long long)p.H * p.W > INT32_MAX || p.C_in > 65535 * 64) return cudaErrorNotSupported;
+  if (p.dtype == GCONV_BF16)
+    return launch_nchw_typed<__nv_bfloat16>(p, P, x, w, bias, y, workspace, s);
+  return launch_nchw_typed<__half>(p, P, x, w, bias, y, workspace, s);
 }
 
 }  // namespace gconv
