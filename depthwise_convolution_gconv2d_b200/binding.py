@@ -32,6 +32,7 @@ STATUS = {0: "GCONV_OK", 1: "GCONV_ERR_INVALID_ARG", 2: "GCONV_ERR_UNSUPPORTED",
 EXPORTS = ["gconv2d_fwd", "gconv2d_fwd_path", "gconv2d_fwd_workspace_size",
            "gconv2d_select_path", "dwconv1d_fwd", "dwconv1d_bwd_data",
            "dwconv1d_bwd_weight", "dwconv1d_bwd_weight_workspace_size",
+           "dwconv1d_bwd_weight_noalloc",
            "gconv_get_device_error", "gconv_status_string", "gconv_version"]
 
 _lib = None
@@ -77,6 +78,8 @@ def load_library():
     lib.dwconv1d_bwd_weight_workspace_size.restype = Z
     lib.dwconv1d_bwd_weight.argtypes = [P, P, P, P, Z] + [I] * 6 + [I, P]
     lib.dwconv1d_bwd_weight.restype = I
+    lib.dwconv1d_bwd_weight_noalloc.argtypes = [P, P, P] + [I] * 6 + [I, P]
+    lib.dwconv1d_bwd_weight_noalloc.restype = I
     lib.gconv_get_device_error.argtypes = [P, ctypes.POINTER(I)]
     lib.gconv_get_device_error.restype = I
     lib.gconv_status_string.argtypes = [I]
@@ -247,6 +250,21 @@ def dwconv1d_bwd_weight(x, dy, K, pad_left, pad_right, out=None, workspace=None,
     st = lib.dwconv1d_bwd_weight(_ptr(x), _ptr(dy), _ptr(dw), _ptr(workspace), ws_bytes, B, T,
                                  C, K, pad_left, pad_right, dt, _stream(stream))
     _check(st, "dwconv1d_bwd_weight")
+    return dw
+
+
+def dwconv1d_bwd_weight_noalloc(x, dy, K, pad_left, pad_right, out=None, stream=None):
+    """dwconv1d_bwd_weight with the library's fixed device scratch instead of a workspace
+    (for callers that cannot allocate device memory); see include/gconv.h."""
+    lib = load_library()
+    _need(x, "x")
+    _need(dy, "dy", x.dtype)
+    B, T, C = x.shape
+    dw = torch.empty((C, K), dtype=x.dtype, device=x.device) if out is None else out
+    _need(dw, "out", x.dtype)
+    st = lib.dwconv1d_bwd_weight_noalloc(_ptr(x), _ptr(dy), _ptr(dw), B, T, C, K, pad_left,
+                                         pad_right, _dtype_code(x.dtype), _stream(stream))
+    _check(st, "dwconv1d_bwd_weight_noalloc")
     return dw
 
 

@@ -238,6 +238,17 @@ gconv_status dwconv1d_bwd_weight(const void* x, const void* dy, void* dw, void* 
   return cuda_status(launch_dwconv1d_wgrad(p, x, dy, dw, workspace, (cudaStream_t)stream));
 }
 
+gconv_status dwconv1d_bwd_weight_noalloc(const void* x, const void* dy, void* dw, int B, int T,
+                                         int C, int K, int pad_left, int pad_right,
+                                         gconv_dtype dtype, void* stream) {
+  Conv1d p;
+  gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
+  if (st != GCONV_OK) return st;
+  if (dw == nullptr || (B > 0 && (x == nullptr || dy == nullptr))) return GCONV_ERR_INVALID_ARG;
+  if (dwconv1d_wgrad_workspace(p) > dwconv1d_wgrad_noalloc_limit()) return GCONV_ERR_WORKSPACE;
+  return cuda_status(launch_dwconv1d_wgrad_noalloc(p, x, dy, dw, (cudaStream_t)stream));
+}
+
 gconv_status gconv_get_device_error(void* stream, int* code) {
   if (code == nullptr) return GCONV_ERR_INVALID_ARG;
   *code = 0;

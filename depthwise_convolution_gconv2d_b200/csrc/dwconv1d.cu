@@ -363,3 +363,54 @@ cudaError_t launch_dwconv1d_wgrad(const Conv1d& p, const void* x, const void* dy
 }
 
 }  // namespace gconv
+
+// ---------------------------------------------------------------- allocation-free variant
+//
+// dwconv1d_bwd_weight_noalloc runs the same weight-gradient kernels with their partial-sum
+// scratch taken from the fixed device array below instead of a caller workspace, for
+// callers that cannot allocate device memory. The array is part of the library image: every
+// GPU that loads the library holds it until the process exits. Calls share it, so two such
+// calls that overlap on the GPU (different streams, no ordering) race on it. Nothing in it
+// needs to start at zero: the partial kernel writes every slot the reduction reads.
+
+namespace gconv {
+namespace {
+
+constexpr size_t kNoallocScratchBytes = GCONV_WGRAD_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) float g_wgrad_noalloc_scratch[kNoallocScratchBytes / sizeof(float)];
+
+// Device address of the scratch array for the current device, looked up (with that device
+// current) on the first call made on it and cached. The host-side symbol is only a handle.
+cudaError_t noalloc_scratch(float** out) {
+  static std::atomic<float*> cached[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  float* p = cached[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    void* addr = nullptr;
+    e = cudaGetSymbolAddress(&addr, g_wgrad_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    p = static_cast<float*>(addr);
+    cached[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t dwconv1d_wgrad_noalloc_limit() { return kNoallocScratchBytes; }
+
+cudaError_t launch_dwconv1d_wgrad_noalloc(const Conv1d& p, const void* x, const void* dy,
+                                          void* dw, cudaStream_t s) {
+  float* scratch = nullptr;
+  if (dwconv1d_wgrad_workspace(p) > 0) {
+    const cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_dwconv1d_wgrad(p, x, dy, dw, scratch, s);
+}
+
+}  // namespace gconv

@@ -105,6 +105,9 @@ cudaError_t launch_dwconv1d_fwd(const Conv1d& p, const void* x, const void* w, v
 size_t dwconv1d_wgrad_workspace(const Conv1d& p);
 cudaError_t launch_dwconv1d_wgrad(const Conv1d& p, const void* x, const void* dy, void* dw,
                                   void* workspace, cudaStream_t s);
+size_t dwconv1d_wgrad_noalloc_limit();
+cudaError_t launch_dwconv1d_wgrad_noalloc(const Conv1d& p, const void* x, const void* dy,
+                                          void* dw, cudaStream_t s);
 
 // Device error word (set by kernels whose bounded waits give up).
 cudaError_t read_and_clear_device_error(cudaStream_t s, int* code);

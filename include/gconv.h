@@ -48,8 +48,9 @@
  * first; on any error they return a status, launch nothing and leave the outputs untouched.
  * Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default stream)
  * on the current device; the call returns without synchronising. There is no mutable global
- * state apart from the device error word read by gconv_get_device_error(), so calls on
- * different streams may be made from different threads.
+ * state apart from the device error word read by gconv_get_device_error() and the fixed
+ * scratch of dwconv1d_bwd_weight_noalloc, so calls on different streams may be made from
+ * different threads (that one entry point excepted, see its comment).
  */
 #ifndef GCONV_H_
 #define GCONV_H_
@@ -147,6 +148,28 @@ size_t dwconv1d_bwd_weight_workspace_size(int B, int T, int C, int K, int pad_le
 gconv_status dwconv1d_bwd_weight(const void* x, const void* dy, void* dw, void* workspace,
                                  size_t workspace_bytes, int B, int T, int C, int K,
                                  int pad_left, int pad_right, gconv_dtype dtype, void* stream);
+
+/* Size of the fixed device scratch used by dwconv1d_bwd_weight_noalloc (4 MiB). */
+#define GCONV_WGRAD_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+
+/* dwconv1d_bwd_weight without a workspace argument, for callers that cannot allocate device
+ * memory: runtimes that forbid device allocation once they are running (fixed memory budgets
+ * in long-lived speech / streaming servers), and plugins or foreign-language callers that have
+ * no handle on the host application's device allocator. The pages have no counterpart: it is
+ * a calling convention of this library, not part of the method.
+ * Same arguments, result and errors as dwconv1d_bwd_weight, and bitwise the same dw. The
+ * partial sums go to a file-scope device array of GCONV_WGRAD_NOALLOC_SCRATCH_BYTES that is
+ * part of the library image, so every GPU that loads the library holds it until the process
+ * exits; problems whose dwconv1d_bwd_weight_workspace_size exceeds it are rejected with
+ * GCONV_ERR_WORKSPACE before any launch. Nothing is allocated: no cudaMalloc, cudaFree or
+ * allocating library call. The first call on a device looks up the array's device address
+ * with that device current (a cudaGetSymbolAddress); make that first call before any stream
+ * capture. All calls share the one array: calls that overlap on the GPU (on different
+ * streams without ordering between them) race and may return wrong dw. No part of the array
+ * has to start at zero; each call writes every slot it reads. */
+gconv_status dwconv1d_bwd_weight_noalloc(const void* x, const void* dy, void* dw, int B, int T,
+                                         int C, int K, int pad_left, int pad_right,
+                                         gconv_dtype dtype, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word that kernels with
  * bounded waits set when a wait gives up. *code receives 0 if none gave up. Returns
