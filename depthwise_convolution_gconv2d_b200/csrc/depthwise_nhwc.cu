@@ -5,14 +5,24 @@
 // thread points to ("F.conv2d runs x15 slower ...", the NHWC replies). Memory-bound: each
 // output needs kH*kW multiply-adds per channel and one read of its inputs.
 //
-// Mapping: a thread owns VEC consecutive channels (one 16-, 8- or 4-byte vector) of one
-// output column (n, wo) and walks down a chunk of output rows. Its kH x kW input window sits
-// in registers as packed 16-bit vectors; moving one output row down shifts the window by
-// `stride` input rows, so only `stride` new rows of kW vectors are loaded per output (when
-// dilation == 1), and those loads are issued one row ahead of the arithmetic. The filter of
-// the thread's VEC channels stays in fp32 registers. Consecutive threads take consecutive
-// channel vectors, so a warp's loads and stores are contiguous runs of the channel dim.
+// 3x3, dilation 1, stride 1 or 2 (the depthwise layers of the workloads) run on a TMA-staged
+// kernel: persistent CTAs stream (rows x columns x 64 channels) input boxes through a ring of
+// shared-memory stages with one TMA load per tile (the tensor map's zero fill is the padding),
+// so the bytes in flight per SM come from the copy engine rather than from thread count.
+// Each thread owns 4 channels of one output column; the three input rows it needs sit in
+// registers as fp32 pairs and rotate by renaming as the fully unrolled row loop moves down;
+// the 3x3 filter of its channels stays in registers; the multiply-adds are fp32x2 packed.
+//
+// Other shapes run the register-window kernel: a thread owns VEC consecutive channels (one 16-,
+// 8- or 4-byte vector) of one output column (n, wo) and walks down a chunk of output rows. Its
+// kH x kW input window sits in registers as packed 16-bit vectors; moving one output row down
+// shifts the window by `stride` input rows, so only `stride` new rows of kW vectors are loaded
+// per output (when dilation == 1), and those loads are issued one row ahead of the arithmetic.
+// The filter of the thread's VEC channels stays in fp32 registers. Consecutive threads take
+// consecutive channel vectors, so a warp's loads and stores are contiguous runs of the channel
+// dim.
 #include "internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace gconv {
 namespace {
@@ -132,6 +142,246 @@ __global__ void __launch_bounds__(256) depthwise_nhwc_kernel(
   }
 }
 
+// ---------------------------------------------------------------- 3x3 TMA-staged kernel
+
+constexpr int DW3_MAX_STAGES = 8;
+constexpr int DW3_CH = 64;                 // channels per tile (128-byte box rows)
+constexpr size_t DW3_SMEM_BUDGET = 200 * 1024;
+
+struct Dw3Params {
+  int N, H, W, C, Ho, Wo, pad;
+  int BW, IW, IH;                          // output tile columns; input box columns and rows
+  int n_ct, n_wt, n_ht, num_tiles, stages;
+  unsigned int stage_bytes, tx_bytes;
+};
+
+template <typename T>
+__device__ __forceinline__ void unpack_vec(const uint4& v, float2 (&o)[4]) {
+  o[0] = unpack2<T>(v.x);
+  o[1] = unpack2<T>(v.y);
+  o[2] = unpack2<T>(v.z);
+  o[3] = unpack2<T>(v.w);
+}
+template <typename T>
+__device__ __forceinline__ void unpack_vec(const uint2& v, float2 (&o)[2]) {
+  o[0] = unpack2<T>(v.x);
+  o[1] = unpack2<T>(v.y);
+}
+
+// tile t -> (channel tile, image, row tile, column tile); channel tile slowest so that a CTA
+// keeps its filter registers across consecutive tiles
+__device__ __forceinline__ void dw3_decode(const Dw3Params& P, int t, int& ct, int& n, int& th,
+                                           int& tw) {
+  tw = t % P.n_wt;
+  int r = t / P.n_wt;
+  th = r % P.n_ht;
+  r /= P.n_ht;
+  n = r % P.N;
+  ct = r / P.N;
+}
+
+constexpr int DW3_MAX_BW = 14;             // output columns per tile (16 x 14 = 224 threads)
+
+template <typename T, int S, int BH, int VEC>
+__global__ void __launch_bounds__(16 * DW3_MAX_BW, 2)
+    dw3x3_tma_kernel(const __grid_constant__ CUtensorMap tmx, const T* __restrict__ w,
+                     const T* __restrict__ bias, T* __restrict__ y, const Dw3Params P,
+                     unsigned int* err) {
+  using namespace ptx;
+  constexpr int NP = VEC / 2;                 // channel pairs per thread
+  constexpr int NV = DW3_CH / VEC;            // channel vectors per tile row
+  using Vec = typename VecT<NP>::type;        // VEC 16-bit values
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  unsigned long long* full =
+      reinterpret_cast<unsigned long long*>(smem + (size_t)P.stages * P.stage_bytes);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + DW3_MAX_STAGES);
+
+  const int tid = threadIdx.x, cv = tid % NV, wl = tid / NV;
+  if (tid == 0) {
+    for (int s = 0; s < P.stages; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmx);
+  }
+  __syncthreads();
+
+  auto issue = [&](int t, int s) {
+    int ct, n, th, tw;
+    dw3_decode(P, t, ct, n, th, tw);
+    mbar_arrive_expect_tx(&full[s], P.tx_bytes);
+    tma_load_4d(smem + (size_t)s * P.stage_bytes, &tmx, &full[s], ct * DW3_CH,
+                tw * P.BW * S - P.pad, th * BH * S - P.pad, n);
+  };
+  long long issued = 0;
+  if (tid == 0) {
+    for (int i = 0; i < P.stages; ++i) {
+      const long long t = blockIdx.x + (long long)i * gridDim.x;
+      if (t >= P.num_tiles) break;
+      issue((int)t, i);
+      ++issued;
+    }
+  }
+
+  int prev_ct = -1;
+  float2 wv[3][3][NP];
+  float2 bv[NP];
+  long long consumed = 0;
+  int i = 0;
+  for (int t = blockIdx.x; t < P.num_tiles; t += gridDim.x, ++i) {
+    const int s = i % P.stages;
+    const unsigned int par = (unsigned int)((i / P.stages) & 1);
+    int ct, n, th, tw;
+    dw3_decode(P, t, ct, n, th, tw);
+    const bool ok = mbar_wait(&full[s], par, abort_flag, err, 16u);
+    if (!__syncthreads_and(ok)) break;
+    ++consumed;
+    const int c = ct * DW3_CH + cv * VEC;
+    if (ct != prev_ct) {
+      prev_ct = ct;
+      if (c < P.C) {
+#pragma unroll
+        for (int kh = 0; kh < 3; ++kh)
+#pragma unroll
+          for (int kw = 0; kw < 3; ++kw)
+#pragma unroll
+            for (int q = 0; q < NP; ++q)
+              wv[kh][kw][q] = make_float2(Elem<T>::to_f32(w[(c + 2 * q) * 9 + kh * 3 + kw]),
+                                          Elem<T>::to_f32(w[(c + 2 * q + 1) * 9 + kh * 3 + kw]));
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+          bv[q] = bias ? make_float2(Elem<T>::to_f32(bias[c + 2 * q]),
+                                     Elem<T>::to_f32(bias[c + 2 * q + 1]))
+                       : make_float2(0.f, 0.f);
+      }
+    }
+    const int wo = tw * P.BW + wl;
+    if (wl < P.BW && c < P.C) {
+      const Vec* px = reinterpret_cast<const Vec*>(smem + (size_t)s * P.stage_bytes) +
+                      (wl * S) * NV + cv;
+      const int row_v = P.IW * NV;                      // vectors per input row of the box
+      float2 rows[3][3][NP];                            // [slot][kw][channel pair]
+      auto load_row = [&](int r, float2 (&dst)[3][NP]) {
+#pragma unroll
+        for (int kw = 0; kw < 3; ++kw) unpack_vec<T>(px[r * row_v + kw * NV], dst[kw]);
+      };
+      T* yp = y + (((long long)n * P.Ho + th * BH) * P.Wo + wo) * P.C + c;
+      const long long ystep = (long long)P.Wo * P.C;
+      load_row(0, rows[0]);
+      if (S == 1) load_row(1, rows[1]);
+#pragma unroll
+      for (int j = 0; j < BH; ++j) {
+        if (S == 1) {
+          load_row(j + 2, rows[(j + 2) % 3]);
+        } else {
+          load_row(2 * j + 1, rows[(2 * j + 1) % 3]);
+          load_row(2 * j + 2, rows[(2 * j + 2) % 3]);
+        }
+        // two partial sums per channel pair (taps split by kh parity) for more ILP
+        float2 acc[2][NP];
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+          acc[0][q] = bv[q];
+          acc[1][q] = make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int kh = 0; kh < 3; ++kh) {
+          const int slot = (j * S + kh) % 3;
+#pragma unroll
+          for (int kw = 0; kw < 3; ++kw)
+#pragma unroll
+            for (int q = 0; q < NP; ++q)
+              acc[kh & 1][q] = ffma2(wv[kh][kw][q], rows[slot][kw][q], acc[kh & 1][q]);
+        }
+        if (th * BH + j < P.Ho && wo < P.Wo) {
+          Vec o;
+          unsigned int* ou = reinterpret_cast<unsigned int*>(&o);
+#pragma unroll
+          for (int q = 0; q < NP; ++q)
+            ou[q] = pack2<T>(make_float2(acc[0][q].x + acc[1][q].x, acc[0][q].y + acc[1][q].y));
+          *reinterpret_cast<Vec*>(yp + j * ystep) = o;
+        }
+      }
+    }
+    __syncthreads();   // every thread is done with stage s
+    if (tid == 0) {
+      const long long t2 = t + (long long)P.stages * gridDim.x;
+      if (t2 < P.num_tiles) {
+        issue((int)t2, s);
+        ++issued;
+      }
+    }
+  }
+  // copies still in flight (only after an abort) must land before the CTA exits
+  if (tid == 0) {
+    for (long long q = consumed; q < issued; ++q)
+      mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr, 0u);
+  }
+}
+
+template <typename T, int S, int BH>
+cudaError_t launch_dw3_tma(const Conv2d& p, const void* x, const void* w, const void* bias,
+                           void* y, cudaStream_t s) {
+  constexpr int VEC = 4;
+  constexpr int NV = DW3_CH / VEC;
+  Dw3Params P;
+  P.N = p.N; P.H = p.H; P.W = p.W; P.C = p.C_in; P.Ho = p.Ho; P.Wo = p.Wo; P.pad = p.pad;
+  const int nw = (p.Wo + DW3_MAX_BW - 1) / DW3_MAX_BW;
+  P.BW = (p.Wo + nw - 1) / nw;
+  P.IW = (P.BW - 1) * S + 3;
+  P.IH = (BH - 1) * S + 3;
+  P.n_ct = (p.C_in + DW3_CH - 1) / DW3_CH;
+  P.n_wt = (p.Wo + P.BW - 1) / P.BW;
+  P.n_ht = (p.Ho + BH - 1) / BH;
+  const long long tiles = (long long)P.n_ct * p.N * P.n_ht * P.n_wt;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  P.num_tiles = (int)tiles;
+  P.tx_bytes = (unsigned int)(DW3_CH * P.IW * P.IH * 2);
+  P.stage_bytes = (P.tx_bytes + 127u) & ~127u;
+  int stages = (int)(DW3_SMEM_BUDGET / 3 / P.stage_bytes);   // three CTAs per SM
+  if (stages > DW3_MAX_STAGES) stages = DW3_MAX_STAGES;
+  if (stages < 2) stages = 2;
+  if ((size_t)stages * P.stage_bytes > DW3_SMEM_BUDGET) return cudaErrorInvalidValue;
+  P.stages = stages;
+  const size_t smem = 128 + (size_t)stages * P.stage_bytes + DW3_MAX_STAGES * 8 + 16;
+
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tm;
+  const cuuint64_t dims[4] = {(cuuint64_t)p.C_in, (cuuint64_t)p.W, (cuuint64_t)p.H,
+                              (cuuint64_t)p.N};
+  const cuuint64_t strides[3] = {(cuuint64_t)p.C_in * 2, (cuuint64_t)p.W * p.C_in * 2,
+                                 (cuuint64_t)p.H * p.W * p.C_in * 2};
+  const cuuint32_t box[4] = {DW3_CH, (cuuint32_t)P.IW, (cuuint32_t)P.IH, 1};
+  const cuuint32_t ones[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt =
+      p.dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  if (enc(&tm, dt, 4, const_cast<void*>(x), dims, strides, box, ones,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  static std::atomic<unsigned int> configured{0};
+  cudaError_t e = set_max_dynamic_smem((const void*)dw3x3_tma_kernel<T, S, BH, VEC>,
+                                       DW3_SMEM_BUDGET + 1024, configured);
+  if (e != cudaSuccess) return e;
+  int per_sm = 3;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+          &per_sm, dw3x3_tma_kernel<T, S, BH, VEC>, NV * P.BW, smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  long long grid = (long long)sm_count() * per_sm;
+  if (grid > P.num_tiles) grid = P.num_tiles;
+  dw3x3_tma_kernel<T, S, BH, VEC><<<(unsigned)grid, NV * P.BW, smem, s>>>(
+      tm, (const T*)w, (const T*)bias, (T*)y, P, device_error_word());
+  return cudaGetLastError();
+}
+
+bool dw3_tma_eligible(const Conv2d& p) {
+  return p.kH == 3 && p.kW == 3 && p.dil == 1 && (p.stride == 1 || p.stride == 2) &&
+         p.C_in % 8 == 0 && p.pad <= 2;
+}
+
 template <int K> constexpr int vec_for() { return K <= 3 ? 8 : (K <= 5 ? 4 : 2); }
 
 template <typename T, int K, int S>
@@ -166,6 +416,9 @@ cudaError_t launch_ks(const Conv2d& p, const void* x, const void* w, const void*
 template <typename T>
 cudaError_t launch_typed(const Conv2d& p, const void* x, const void* w, const void* bias, void* y,
                          cudaStream_t s) {
+  if (dw3_tma_eligible(p))
+    return p.stride == 1 ? launch_dw3_tma<T, 1, 8>(p, x, w, bias, y, s)
+                         : launch_dw3_tma<T, 2, 4>(p, x, w, bias, y, s);
   const int K = p.kH;
   if (p.stride == 1) {
     if (K == 3) return launch_ks<T, 3, 1>(p, x, w, bias, y, s);

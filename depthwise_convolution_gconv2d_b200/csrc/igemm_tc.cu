@@ -29,14 +29,16 @@
 #include <cuda.h>
 
 #include "internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace gconv {
 namespace {
 
+using namespace ptx;
+
 constexpr int BM = 128;                 // output pixels per tile (UMMA M)
 constexpr int NUM_THREADS = 192;        // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
 constexpr int MAX_STAGES = 32;
-constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;   // 1 s
 constexpr size_t SMEM_BUDGET = 227 * 1024;
 
 enum : unsigned int { ERR_WAIT_PRODUCER = 1u, ERR_WAIT_MMA = 2u, ERR_WAIT_EPILOGUE = 4u,
@@ -55,158 +57,9 @@ struct IgemmParams {
   int out_nchw;
 };
 
-// ------------------------------------------------------------------ PTX wrappers
-
-__device__ __forceinline__ unsigned int smem_u32(const void* p) {
-  return (unsigned int)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ unsigned long long globaltimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(unsigned long long* bar, unsigned int count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, unsigned int bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned int parity) {
-  unsigned int ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for the phase with `parity` to complete; gives up after WAIT_LIMIT_NS (sets the CTA's
-// abort flag and the device error word) or when another role has aborted.
-__device__ __noinline__ bool mbar_wait(unsigned long long* bar, unsigned int parity,
-                                       volatile int* abort_flag, unsigned int* err,
-                                       unsigned int code) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
-      *abort_flag = 1;
-      if (err) atomicOr(err, code);
-      return false;
-    }
-  }
-}
-
-__device__ __forceinline__ void prefetch_tmap(const void* map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
-}
-
-__device__ __forceinline__ void tma_load_4d(void* dst, const void* map, unsigned long long* bar,
-                                            int c0, int c1, int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, unsigned long long* bar,
-                                            int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(unsigned int* slot, unsigned int ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(slot)),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(unsigned int taddr, unsigned int ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// D(tmem) (+)= A(smem desc) * B(smem desc), kind::f16, issued by one thread.
-__device__ __forceinline__ void umma_f16(unsigned int d_tmem, unsigned long long a_desc,
-                                         unsigned long long b_desc, unsigned int idesc,
-                                         unsigned int accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once on `bar` when every tcgen05.mma this thread issued so far has completed.
-__device__ __forceinline__ void umma_commit(unsigned long long* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-
-// Warp-collective: lane i reads TMEM lane (base lane + i), 32 / 16 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_ld32(unsigned int taddr, unsigned int (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld16(unsigned int taddr, unsigned int (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_wait() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
 // Shared-memory matrix descriptor (tcgen05): start address, leading / stride byte offsets
 // (16-byte units), descriptor version 1 at bits 46-47, layout (swizzle) code at bits 61-63.
+// The base-offset field (bits 49-51) stays 0: the swizzle is taken from the absolute address.
 __device__ __forceinline__ unsigned long long smem_desc(unsigned int saddr, unsigned int sbo,
                                                         unsigned int swz) {
   unsigned long long d = (unsigned long long)((saddr >> 4) & 0x3FFFu);
@@ -217,8 +70,8 @@ __device__ __forceinline__ unsigned long long smem_desc(unsigned int saddr, unsi
   return d;
 }
 
-template <typename T>
-__device__ __forceinline__ void epilogue_store(const IgemmParams& P, T* __restrict__ y,
+template <typename T, typename PP>
+__device__ __forceinline__ void epilogue_store(const PP& P, T* __restrict__ y,
                                                const T* __restrict__ bias, const unsigned int* r,
                                                int ncols, int n, int ho, int wo, int co) {
   float v[32];
@@ -342,6 +195,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       unsigned int ph = 0, aph = 0;
       bool ok = true;
       const int ksteps = P.BKC / 16;
+      // descriptors are built once; per stage and per K step only their address field moves
+      // (a 64-bit add of a 16-byte-unit offset), which keeps the issuing thread's dependent
+      // instruction chain short enough for back-to-back MMAs
+      const unsigned long long a_desc0 = smem_desc(smem_u32(a_base), P.sbo, P.swz);
+      const unsigned long long b_desc0 = smem_desc(smem_u32(b_base), P.sbo, P.swz);
       for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERR_WAIT_MMA)) break;
         tc_fence_after();
@@ -352,13 +210,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const unsigned int a_addr = smem_u32(a_base + (size_t)s * P.a_stage);
-          const unsigned int b_addr = smem_u32(b_base + (size_t)s * P.b_stage);
-          for (int kk = 0; kk < ksteps; ++kk) {
-            const unsigned long long ad = smem_desc(a_addr + kk * 32, P.sbo, P.swz);
-            const unsigned long long bd = smem_desc(b_addr + kk * 32, P.sbo, P.swz);
-            umma_f16(d_tmem, ad, bd, P.idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
+          const unsigned long long ad = a_desc0 + (((unsigned long long)s * P.a_stage) >> 4);
+          const unsigned long long bd = b_desc0 + (((unsigned long long)s * P.b_stage) >> 4);
+          umma_f16(d_tmem, ad, bd, P.idesc, kb != 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 1; kk < 4; ++kk)
+            if (kk < ksteps) umma_f16(d_tmem, ad + 2 * kk, bd + 2 * kk, P.idesc, 1u);
           umma_commit(&empty[s]);
           if (++s == P.stages) {
             s = 0;
@@ -405,6 +262,261 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld16(taddr + c, r);
         tmem_ld_wait();
         if (valid) epilogue_store<T>(P, y, bias, r, ncols, n, ho, wo, co0 + c);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, P.tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------------ row-strip kernel
+//
+// For rows of at least 128 output pixels (Wo >= 128), a tile is NSUB consecutive 128-pixel
+// segments of one output row x BN filters. For each (channel block, kh) the TMA warp loads,
+// per segment, one strip of 128 + (kW-1)*dil input pixels; the kW taps of that kh are then
+// the same strip read from row offsets kw*dil -- a start-address shift of the K-major,
+// 128-byte-swizzled operand. The tensor cores apply the 128-byte swizzle to absolute shared-
+// memory address bits, as TMA does when it writes the strip, so a start address moved by whole
+// 128-byte rows reads exactly the rows TMA wrote there, with the descriptor's base-offset field
+// left at 0 (measured: a non-zero base offset there gives wrong sums) -- and each input strip
+// is fetched once per kh instead of once per tap. The NSUB segments share
+// every weight tile. Strips and weight tiles have their own stage rings.
+
+constexpr int ROW_MAX_A = 4;
+constexpr int ROW_MAX_B = 16;
+
+struct RowParams {
+  int N, H, W, C_in, C_out, Ho, Wo, kH, kW, pad, dil, cpg_in, cpg_out;
+  int BN, NSUB, cblocks, segs, n_tiles, num_tiles, strip_rows;
+  int a_stages, b_stages;
+  unsigned int a_stage, strip_stride, b_stage, a_tx, b_tx;
+  unsigned int idesc, tmem_cols;
+  int out_nchw;
+};
+
+__device__ __forceinline__ void row_decode(const RowParams& P, int t, int& j, int& nt, int& n,
+                                           int& ho, int& seg) {
+  seg = t % P.segs;
+  int r = t / P.segs;
+  ho = r % P.Ho;
+  r /= P.Ho;
+  n = r % P.N;
+  r /= P.N;
+  nt = r % P.n_tiles;
+  j = r / P.n_tiles;
+}
+
+template <typename T, int NSUB>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    igemm_row_kernel(const __grid_constant__ CUtensorMap tma_x,
+                     const __grid_constant__ CUtensorMap tma_w, const T* __restrict__ bias,
+                     T* __restrict__ y, const RowParams P, unsigned int* err) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* a_base = smem;
+  unsigned char* b_base = smem + (size_t)P.a_stages * P.a_stage;
+  unsigned long long* bars =
+      reinterpret_cast<unsigned long long*>(b_base + (size_t)P.b_stages * P.b_stage);
+  unsigned long long* fa = bars;
+  unsigned long long* ea = fa + ROW_MAX_A;
+  unsigned long long* fb = ea + ROW_MAX_A;
+  unsigned long long* eb = fb + ROW_MAX_B;
+  unsigned long long* tfull = eb + ROW_MAX_B;
+  unsigned long long* tempty = tfull + 2;
+  unsigned long long* done = tempty + 2;
+  unsigned int* tmem_slot = reinterpret_cast<unsigned int*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P.a_stages; ++s) {
+      mbar_init(&fa[s], 1);
+      mbar_init(&ea[s], 1);
+    }
+    for (int s = 0; s < P.b_stages; ++s) {
+      mbar_init(&fb[s], 1);
+      mbar_init(&eb[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tma_x);
+    prefetch_tmap(&tma_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, P.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const unsigned int tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int sa = 0, sb = 0;
+      unsigned int pa = 0, pb = 0;
+      long long na = 0, nb = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
+        int j, nt, n, ho, seg;
+        row_decode(P, t, j, nt, n, ho, seg);
+        const int wbase = seg * NSUB * BM - P.pad;
+        const int obase = j * P.cpg_out + nt * P.BN;
+        for (int cb = 0; cb < P.cblocks && ok; ++cb) {
+          const int cin = j * P.cpg_in + cb * 64;
+          for (int kh = 0; kh < P.kH && ok; ++kh) {
+            if (!mbar_wait(&ea[sa], pa ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&fa[sa], P.a_tx);
+            for (int sub = 0; sub < NSUB; ++sub)
+              tma_load_4d(a_base + (size_t)sa * P.a_stage + (size_t)sub * P.strip_stride, &tma_x,
+                          &fa[sa], cin, wbase + sub * BM, ho - P.pad + kh * P.dil, n);
+            ++na;
+            if (++sa == P.a_stages) {
+              sa = 0;
+              pa ^= 1u;
+            }
+            for (int kw = 0; kw < P.kW; ++kw) {
+              if (!mbar_wait(&eb[sb], pb ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_expect_tx(&fb[sb], P.b_tx);
+              tma_load_2d(b_base + (size_t)sb * P.b_stage, &tma_w, &fb[sb],
+                          (kh * P.kW + kw) * P.cpg_in + cb * 64, obase);
+              ++nb;
+              if (++sb == P.b_stages) {
+                sb = 0;
+                pb ^= 1u;
+              }
+            }
+          }
+        }
+      }
+      // copies in flight must land before the CTA exits (no-op on the normal path)
+      for (long long q = (na > P.a_stages ? na - P.a_stages : 0); q < na; ++q)
+        mbar_wait(&fa[q % P.a_stages], (unsigned int)((q / P.a_stages) & 1), abort_flag, err,
+                  ERR_WAIT_DRAIN);
+      for (long long q = (nb > P.b_stages ? nb - P.b_stages : 0); q < nb; ++q)
+        mbar_wait(&fb[q % P.b_stages], (unsigned int)((q / P.b_stages) & 1), abort_flag, err,
+                  ERR_WAIT_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int sa = 0, sb = 0, acc = 0;
+      unsigned int pa = 0, pb = 0, aph = 0;
+      bool ok = true;
+      // descriptors built once; the loop only adds 16-byte-unit offsets (see the tile kernel)
+      const unsigned long long a_desc0 = smem_desc(smem_u32(a_base), 1024u, 2u);
+      const unsigned long long b_desc0 = smem_desc(smem_u32(b_base), 1024u, 2u);
+      const unsigned long long sub_step = P.strip_stride >> 4;
+      const unsigned long long kw_step = (unsigned long long)P.dil * 8u;   // dil rows of 128 B
+      for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERR_WAIT_MMA)) break;
+        tc_fence_after();
+        const unsigned int d0 = tmem_base + (unsigned int)(acc * NSUB * P.BN);
+        for (int cb = 0; cb < P.cblocks && ok; ++cb) {
+          for (int kh = 0; kh < P.kH && ok; ++kh) {
+            if (!mbar_wait(&fa[sa], pa, abort_flag, err, ERR_WAIT_MMA)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const unsigned long long a_st = a_desc0 + (((unsigned long long)sa * P.a_stage) >> 4);
+            for (int kw = 0; kw < P.kW; ++kw) {
+              if (!mbar_wait(&fb[sb], pb, abort_flag, err, ERR_WAIT_MMA)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const unsigned long long bd = b_desc0 + (((unsigned long long)sb * P.b_stage) >> 4);
+              unsigned long long ad[NSUB];
+              unsigned int dd[NSUB];
+#pragma unroll
+              for (int sub = 0; sub < NSUB; ++sub) {
+                ad[sub] = a_st + kw * kw_step + sub * sub_step;
+                dd[sub] = d0 + (unsigned int)(sub * P.BN);
+              }
+              const unsigned int acc0 = (cb | kh | kw) == 0 ? 0u : 1u;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int sub = 0; sub < NSUB; ++sub)
+                  umma_f16(dd[sub], ad[sub] + 2 * kk, bd + 2 * kk, P.idesc, kk == 0 ? acc0 : 1u);
+              umma_commit(&eb[sb]);
+              if (++sb == P.b_stages) {
+                sb = 0;
+                pb ^= 1u;
+              }
+            }
+            if (!ok) break;
+            umma_commit(&ea[sa]);
+            if (++sa == P.a_stages) {
+              sa = 0;
+              pa ^= 1u;
+            }
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          aph ^= 1u;
+        }
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, abort_flag, err, ERR_WAIT_DRAIN);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5, TMEM lane quarter (warp % 4)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    int acc = 0;
+    unsigned int aph = 0;
+    for (int t = blockIdx.x; t < P.num_tiles; t += gridDim.x) {
+      int j, nt, n, ho, seg;
+      row_decode(P, t, j, nt, n, ho, seg);
+      const bool got = mbar_wait(&tfull[acc], aph, abort_flag, err, ERR_WAIT_EPILOGUE);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int co0 = j * P.cpg_out + nt * P.BN;
+      for (int sub = 0; sub < NSUB; ++sub) {
+        const int wo = (seg * NSUB + sub) * BM + row;
+        const bool valid = wo < P.Wo;
+        const unsigned int taddr = tmem_base + ((unsigned int)(quarter * 32) << 16) +
+                                   (unsigned int)((acc * NSUB + sub) * P.BN);
+        for (int c = 0; c < P.BN; c += 32) {
+          unsigned int r[32];
+          const int ncols = P.BN - c < 32 ? P.BN - c : 32;
+          if (ncols == 32)
+            tmem_ld32(taddr + c, r);
+          else
+            tmem_ld16(taddr + c, r);
+          tmem_ld_wait();
+          if (valid) epilogue_store<T>(P, y, bias, r, ncols, n, ho, wo, co0 + c);
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -474,38 +586,6 @@ __global__ void repack_weight_kernel(const T* __restrict__ w, T* __restrict__ wt
 
 // ------------------------------------------------------------------ host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static std::atomic<EncodeTiledFn> fn{nullptr};
-  EncodeTiledFn f = fn.load(std::memory_order_acquire);
-  if (f) return f;
-  void* p = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-          cudaSuccess ||
-      q != cudaDriverEntryPointSuccess || p == nullptr)
-    return nullptr;
-  f = reinterpret_cast<EncodeTiledFn>(p);
-  fn.store(f, std::memory_order_release);
-  return f;
-}
-
-int sm_count() {
-  static std::atomic<int> cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  int v = cached[dev].load(std::memory_order_relaxed);
-  if (v > 0) return v;
-  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
-    v = 148;
-  cached[dev].store(v, std::memory_order_relaxed);
-  return v;
-}
-
 int tile_bn(const Conv2d& p) {
   if (p.cpg_out <= 256) return p.cpg_out;
   return p.cpg_out % 128 == 0 ? 128 : 0;
@@ -566,11 +646,122 @@ CUtensorMapSwizzle swizzle_of(int BKC) {
                    : (BKC == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
+// Row-strip kernel parameters; false if the problem does not take that kernel (rows shorter
+// than 128 outputs, channel blocks narrower than 64, or the stage rings do not fit).
+bool make_row_params(const Conv2d& p, RowParams* R) {
+  if (p.Wo < BM || p.cpg_in % 64 != 0) return false;
+  const int BN = tile_bn(p);
+  if (BN == 0) return false;
+  R->N = p.N; R->H = p.H; R->W = p.W; R->C_in = p.C_in; R->C_out = p.C_out;
+  R->Ho = p.Ho; R->Wo = p.Wo; R->kH = p.kH; R->kW = p.kW; R->pad = p.pad; R->dil = p.dil;
+  R->cpg_in = p.cpg_in; R->cpg_out = p.cpg_out;
+  R->BN = BN;
+  int nsub = 256 / BN;
+  const int row_segs = (p.Wo + BM - 1) / BM;
+  if (nsub > row_segs) nsub = row_segs;
+  if (nsub >= 4) nsub = 4;
+  else if (nsub >= 2) nsub = 2;
+  else nsub = 1;
+  R->NSUB = nsub;
+  R->cblocks = p.cpg_in / 64;
+  R->segs = (p.Wo + nsub * BM - 1) / (nsub * BM);
+  R->n_tiles = p.cpg_out / BN;
+  const long long tiles = (long long)R->segs * p.Ho * p.N * R->n_tiles * p.groups;
+  if (tiles > INT32_MAX) return false;
+  R->num_tiles = (int)tiles;
+  R->strip_rows = BM + (p.kW - 1) * p.dil;
+  if (R->strip_rows > 256) return false;
+  R->strip_stride = ((unsigned int)R->strip_rows * 128u + 1023u) & ~1023u;
+  R->a_stage = (unsigned int)nsub * R->strip_stride;
+  R->b_stage = (unsigned int)BN * 128u;
+  R->a_tx = (unsigned int)nsub * (unsigned int)R->strip_rows * 128u;
+  R->b_tx = (unsigned int)BN * 128u;
+  const size_t fixed = 1024 + (2 * (ROW_MAX_A + ROW_MAX_B) + 5) * 8 + 16;
+  const size_t budget = SMEM_BUDGET - fixed;
+  int a_st = 3;
+  if ((size_t)a_st * R->a_stage > budget / 2) a_st = 2;
+  if ((size_t)a_st * R->a_stage >= budget) return false;
+  int b_st = (int)((budget - (size_t)a_st * R->a_stage) / R->b_stage);
+  if (b_st > ROW_MAX_B) b_st = ROW_MAX_B;
+  if (b_st < 2) return false;
+  R->a_stages = a_st;
+  R->b_stages = b_st;
+  const unsigned int fmt = p.dtype == GCONV_BF16 ? 1u : 0u;
+  R->idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((unsigned int)(BN >> 3) << 17) |
+             ((unsigned int)(BM >> 4) << 24);
+  R->tmem_cols = pow2_cols(2 * nsub * BN);
+  if (R->tmem_cols > 512) return false;
+  R->out_nchw = p.layout == GCONV_NCHW;
+  return true;
+}
+
+size_t row_smem_bytes(const RowParams& R) {
+  return 1024 + (size_t)R.a_stages * R.a_stage + (size_t)R.b_stages * R.b_stage +
+         (2 * (ROW_MAX_A + ROW_MAX_B) + 5) * 8 + 16;
+}
+
+template <typename T>
+cudaError_t launch_row(const Conv2d& p, const RowParams& R, const void* x, const void* w,
+                       const void* bias, void* y, cudaStream_t s) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const CUtensorMapDataType dt =
+      p.dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tx, tw;
+  const cuuint64_t xdim[4] = {(cuuint64_t)p.C_in, (cuuint64_t)p.W, (cuuint64_t)p.H,
+                              (cuuint64_t)p.N};
+  const cuuint64_t xstr[3] = {(cuuint64_t)p.C_in * 2, (cuuint64_t)p.W * p.C_in * 2,
+                              (cuuint64_t)p.H * p.W * p.C_in * 2};
+  const cuuint32_t xbox[4] = {64, (cuuint32_t)R.strip_rows, 1, 1};
+  const cuuint32_t ones[4] = {1, 1, 1, 1};
+  if (enc(&tx, dt, 4, const_cast<void*>(x), xdim, xstr, xbox, ones,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const cuuint64_t ktot = (cuuint64_t)p.kH * p.kW * p.cpg_in;
+  const cuuint64_t wdim[2] = {ktot, (cuuint64_t)p.C_out};
+  const cuuint64_t wstr[1] = {ktot * 2};
+  const cuuint32_t wbox[2] = {64, (cuuint32_t)R.BN};
+  if (enc(&tw, dt, 2, const_cast<void*>(w), wdim, wstr, wbox, ones,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const size_t smem = row_smem_bytes(R);
+  if (smem > SMEM_BUDGET) return cudaErrorInvalidValue;
+  int grid = sm_count();
+  if (grid > R.num_tiles) grid = R.num_tiles;
+  static std::atomic<unsigned int> configured[3];
+  cudaError_t e;
+  switch (R.NSUB) {
+    case 1:
+      e = set_max_dynamic_smem((const void*)igemm_row_kernel<T, 1>, SMEM_BUDGET, configured[0]);
+      if (e != cudaSuccess) return e;
+      igemm_row_kernel<T, 1><<<grid, NUM_THREADS, smem, s>>>(tx, tw, (const T*)bias, (T*)y, R,
+                                                             device_error_word());
+      break;
+    case 2:
+      e = set_max_dynamic_smem((const void*)igemm_row_kernel<T, 2>, SMEM_BUDGET, configured[1]);
+      if (e != cudaSuccess) return e;
+      igemm_row_kernel<T, 2><<<grid, NUM_THREADS, smem, s>>>(tx, tw, (const T*)bias, (T*)y, R,
+                                                             device_error_word());
+      break;
+    default:
+      e = set_max_dynamic_smem((const void*)igemm_row_kernel<T, 4>, SMEM_BUDGET, configured[2]);
+      if (e != cudaSuccess) return e;
+      igemm_row_kernel<T, 4><<<grid, NUM_THREADS, smem, s>>>(tx, tw, (const T*)bias, (T*)y, R,
+                                                             device_error_word());
+      break;
+  }
+  return cudaGetLastError();
+}
+
 // x: NHWC activations, w: [C_out][kH][kW][cpg_in] weights (both device pointers).
 template <typename T>
 cudaError_t launch_core(const Conv2d& p, const IgemmParams& P, const void* x, const void* w,
                         const void* bias, void* y, cudaStream_t s) {
-  EncodeTiledFn enc = encode_fn();
+  RowParams R;
+  if (make_row_params(p, &R)) return launch_row<T>(p, R, x, w, bias, y, s);
+  EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   const CUtensorMapDataType dt =
       p.dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;

@@ -8,6 +8,8 @@
 
 #include <atomic>
 
+#include <cuda.h>   // CUtensorMap types (the driver entry point is resolved at run time)
+
 #include "gconv.h"
 
 namespace gconv {
@@ -108,6 +110,14 @@ cudaError_t launch_dwconv1d_wgrad(const Conv1d& p, const void* x, const void* dy
 size_t dwconv1d_wgrad_noalloc_limit();
 cudaError_t launch_dwconv1d_wgrad_noalloc(const Conv1d& p, const void* x, const void* dy,
                                           void* dw, cudaStream_t s);
+
+// cuTensorMapEncodeTiled, resolved through the runtime (null if unavailable).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
+int sm_count();                       // SMs of the current device (cached)
 
 // Device error word (set by kernels whose bounded waits give up).
 cudaError_t read_and_clear_device_error(cudaStream_t s, int* code);
