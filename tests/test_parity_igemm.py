@@ -28,6 +28,10 @@ SMALL = [
     (3, 128, 7, 56, 256, 3, 1, 1, 1),        # 56-wide rows: 112-row tiles; N = 256
     (1, 64, 3, 3, 32, 3, 0, 1, 1),           # single output pixel
     (2, 48, 6, 6, 48, 3, 1, 1, 3),           # 16 / 16 with three groups
+    (1, 128, 4, 140, 192, 3, 1, 1, 2),       # row-strip kernel: Wo >= 128, 96 filters per group
+    (2, 128, 3, 300, 256, 3, 1, 1, 2),       # transposed row kernel, 2 segments per row
+    (1, 64, 6, 140, 128, 3, 2, 2, 1),        # transposed row kernel with dilation 2
+    (1, 64, 7, 131, 128, 5, 2, 1, 1),        # transposed row kernel, 5x5
 ]
 
 
@@ -46,7 +50,7 @@ def test_igemm_small_nhwc(case):
     assert_close(to_f64(y), oracle_full(inp), p.dtype, str(case))
 
 
-@pytest.mark.parametrize("case", SMALL[:6])
+@pytest.mark.parametrize("case", SMALL[:6] + SMALL[10:])
 def test_igemm_small_nchw(case):
     p = problem(case, wl.NCHW, bias=True)
     assert kernel_of(p, gb.PATH_IGEMM) == 4
