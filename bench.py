@@ -74,7 +74,7 @@ def traffic_for(kernel: str, source: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -88,7 +88,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -188,6 +188,55 @@ def kernel_name(code: int) -> str:
 LAUNCHES_PER_CALL = {1: 1, 2: 1, 3: 1, 4: 3}
 KERNEL_SOURCE = {1: "direct_generic.cu", 2: "depthwise_nhwc.cu", 3: "igemm_tc.cu",
                  4: "igemm_tc.cu"}
+
+
+def conv2d_measurement(torch, gb, device, stream, pk, p, workload, path, reps, flush):
+    inp = wl.make_conv2d_inputs(p, workload)
+    x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
+    y = torch.empty(p.y_shape, dtype=torch.bfloat16, device=device)
+    need = gb.gconv2d_fwd_workspace_size(p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride,
+                                         p.pad, p.dilation, p.groups, p.layout, p.dtype, path)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    kcode = gb.gconv2d_select_path(p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride, p.pad,
+                                   p.dilation, p.groups, p.layout, p.dtype, path)
+    fn = lambda i: gb.gconv2d_fwd(x, w, None, p.stride, p.pad, p.dilation, p.groups, p.layout,
+                                  out=y, workspace=ws, path=path, stream=stream)
+    for _ in range(2):
+        fn(0)
+    med, mean = time_launches(torch, fn, stream, reps, flush)
+    tf = p.flops() / (med * 1e-3) / 1e12
+    gbs = p.bytes() / (med * 1e-3) / 1e9
+    t_tensor = p.flops() / (pk["bf16_tflops"] * 1e12)
+    t_hbm = p.bytes() / (pk["hbm_gbs"] * 1e9)
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    frac = max(t_tensor, t_hbm) / (med * 1e-3)
+    return {"kernel": kernel_name(kcode), "us": round(med * 1e3, 2), "TFLOP/s": round(tf, 1),
+            "GB/s": round(gbs, 1), "bound": bound, "frac": round(frac, 3),
+            "alg_flops": p.flops(), "alg_bytes": p.bytes()}
+
+
+def more_conv2d_measurements(torch, gb, device, stream, pk, reps):
+    """The other conv2d workloads: ensemble-as-groups layer and the groups sweep at C = 1024."""
+    flush = l2_flusher(torch, device)
+    out = {}
+    out["ensemble_g64_nhwc"] = conv2d_measurement(torch, gb, device, stream, pk,
+                                                  wl.ensemble_groups(), 4, gb.PATH_AUTO, reps,
+                                                  flush)
+    out["wide_group_nchw"] = conv2d_measurement(torch, gb, device, stream, pk,
+                                                wl.wide_group(wl.NCHW), 2, gb.PATH_AUTO, reps,
+                                                flush)
+    for g in (1024, 256, 64, 16):
+        p = wl.depthwise_56(1, g)
+        for name, path in (("auto", gb.PATH_AUTO), ("direct", gb.PATH_DIRECT),
+                           ("igemm", gb.PATH_IGEMM)):
+            if path == gb.PATH_IGEMM and gb.gconv2d_select_path(
+                    p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride, p.pad, p.dilation,
+                    p.groups, p.layout, p.dtype, path) < 0:
+                continue
+            r = 3 if (path == gb.PATH_DIRECT and g <= 64) else reps
+            out[f"sweep56_g{g}_{name}"] = conv2d_measurement(torch, gb, device, stream, pk, p, 5,
+                                                             path, r, flush)
+    return out
 
 
 def depthwise_measurements(torch, gb, device, stream, pk, reps):
@@ -307,7 +356,7 @@ def config_dict(p, args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layout", default="nhwc", choices=["nhwc", "nchw"])
@@ -450,8 +499,10 @@ def main():
                "d2h_bytes_per_step": y_pin.numel() * 2, "steps": n_e2e}
 
     dwm = None
+    more = None
     if not args.no_depthwise and rank == 0:
         dwm = depthwise_measurements(torch, gb, device, stream, pk, 20)
+        more = more_conv2d_measurements(torch, gb, device, stream, pk, 10)
     dev_err = gb.device_error(stream)
 
     cpu = None
@@ -471,6 +522,7 @@ def main():
             "kernel": kernel_name(kcode), "roofline": roof, "e2e": e2e,
             "gpu_launches": LAUNCHES_PER_CALL.get(kcode, 1) * args.steps,
             "clocks": clk.summary(), "cpu_baseline": cpu, "depthwise": dwm,
+            "other_workloads": more,
             "device_error": dev_err,
             "peaks": {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
                       "source": peak_src},

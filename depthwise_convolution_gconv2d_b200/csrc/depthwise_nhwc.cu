@@ -168,22 +168,36 @@ __device__ __forceinline__ void unpack_vec(const uint2& v, float2 (&o)[2]) {
   o[1] = unpack2<T>(v.y);
 }
 
-// tile t -> (channel tile, image, row tile, column tile); channel tile slowest so that a CTA
-// keeps its filter registers across consecutive tiles
-__device__ __forceinline__ void dw3_decode(const Dw3Params& P, int t, int& ct, int& n, int& th,
-                                           int& tw) {
-  tw = t % P.n_wt;
-  int r = t / P.n_wt;
-  th = r % P.n_ht;
-  r /= P.n_ht;
-  n = r % P.N;
-  ct = r / P.N;
-}
+// Tile coordinates, channel tile slowest: tw -> th -> n -> ct. A CTA walks a contiguous chunk
+// of tiles, so its filter registers change only when the chunk crosses a channel tile.
+struct Dw3Coord {
+  int ct, n, th, tw;
+  __device__ __forceinline__ void set(const Dw3Params& P, long long t) {
+    tw = (int)(t % P.n_wt);
+    long long r = t / P.n_wt;
+    th = (int)(r % P.n_ht);
+    r /= P.n_ht;
+    n = (int)(r % P.N);
+    ct = (int)(r / P.N);
+  }
+  __device__ __forceinline__ void next(const Dw3Params& P) {
+    if (++tw < P.n_wt) return;
+    tw = 0;
+    if (++th < P.n_ht) return;
+    th = 0;
+    if (++n < P.N) return;
+    n = 0;
+    ++ct;
+  }
+};
 
-constexpr int DW3_MAX_BW = 14;             // output columns per tile (16 x 14 = 224 threads)
+constexpr int DW3_MAX_BW = 14;             // output columns per tile (16 x 14 = 224 compute threads)
+constexpr int DW3_THREADS = 32 + 16 * DW3_MAX_BW;
 
+// Warp 0 lane 0 is the TMA producer; warps 1.. compute. Stage s is handed over through
+// full[s] (TMA transaction bytes) and empty[s] (one arrival per compute warp).
 template <typename T, int S, int BH, int VEC>
-__global__ void __launch_bounds__(16 * DW3_MAX_BW, 2)
+__global__ void __launch_bounds__(DW3_THREADS, 2)
     dw3x3_tma_kernel(const __grid_constant__ CUtensorMap tmx, const T* __restrict__ w,
                      const T* __restrict__ bias, T* __restrict__ y, const Dw3Params P,
                      unsigned int* err) {
@@ -196,128 +210,143 @@ __global__ void __launch_bounds__(16 * DW3_MAX_BW, 2)
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
   unsigned long long* full =
       reinterpret_cast<unsigned long long*>(smem + (size_t)P.stages * P.stage_bytes);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + DW3_MAX_STAGES);
+  unsigned long long* empty = full + DW3_MAX_STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + DW3_MAX_STAGES);
 
-  const int tid = threadIdx.x, cv = tid % NV, wl = tid / NV;
-  if (tid == 0) {
-    for (int s = 0; s < P.stages; ++s) mbar_init(&full[s], 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_compute_warps = (int)(blockDim.x >> 5) - 1;
+  const long long t_begin = (long long)P.num_tiles * blockIdx.x / gridDim.x;
+  const long long t_end = (long long)P.num_tiles * (blockIdx.x + 1) / gridDim.x;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], (unsigned int)n_compute_warps);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmx);
   }
   __syncthreads();
 
-  auto issue = [&](int t, int s) {
-    int ct, n, th, tw;
-    dw3_decode(P, t, ct, n, th, tw);
-    mbar_arrive_expect_tx(&full[s], P.tx_bytes);
-    tma_load_4d(smem + (size_t)s * P.stage_bytes, &tmx, &full[s], ct * DW3_CH,
-                tw * P.BW * S - P.pad, th * BH * S - P.pad, n);
-  };
-  long long issued = 0;
-  if (tid == 0) {
-    for (int i = 0; i < P.stages; ++i) {
-      const long long t = blockIdx.x + (long long)i * gridDim.x;
-      if (t >= P.num_tiles) break;
-      issue((int)t, i);
-      ++issued;
-    }
-  }
-
-  int prev_ct = -1;
-  float2 wv[3][3][NP];
-  float2 bv[NP];
-  long long consumed = 0;
-  int i = 0;
-  for (int t = blockIdx.x; t < P.num_tiles; t += gridDim.x, ++i) {
-    const int s = i % P.stages;
-    const unsigned int par = (unsigned int)((i / P.stages) & 1);
-    int ct, n, th, tw;
-    dw3_decode(P, t, ct, n, th, tw);
-    const bool ok = mbar_wait(&full[s], par, abort_flag, err, 16u);
-    if (!__syncthreads_and(ok)) break;
-    ++consumed;
-    const int c = ct * DW3_CH + cv * VEC;
-    if (ct != prev_ct) {
-      prev_ct = ct;
-      if (c < P.C) {
-#pragma unroll
-        for (int kh = 0; kh < 3; ++kh)
-#pragma unroll
-          for (int kw = 0; kw < 3; ++kw)
-#pragma unroll
-            for (int q = 0; q < NP; ++q)
-              wv[kh][kw][q] = make_float2(Elem<T>::to_f32(w[(c + 2 * q) * 9 + kh * 3 + kw]),
-                                          Elem<T>::to_f32(w[(c + 2 * q + 1) * 9 + kh * 3 + kw]));
-#pragma unroll
-        for (int q = 0; q < NP; ++q)
-          bv[q] = bias ? make_float2(Elem<T>::to_f32(bias[c + 2 * q]),
-                                     Elem<T>::to_f32(bias[c + 2 * q + 1]))
-                       : make_float2(0.f, 0.f);
+  if (warp == 0) {
+    if (lane == 0) {
+      Dw3Coord c;
+      c.set(P, t_begin);
+      int s = 0;
+      unsigned int ph = 0;
+      long long issued = 0;
+      for (long long t = t_begin; t < t_end; ++t) {
+        if (!mbar_try_wait(&empty[s], ph ^ 1u) &&
+            !mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, 16u))
+          break;
+        mbar_arrive_expect_tx(&full[s], P.tx_bytes);
+        tma_load_4d(smem + (size_t)s * P.stage_bytes, &tmx, &full[s], c.ct * DW3_CH,
+                    c.tw * P.BW * S - P.pad, c.th * BH * S - P.pad, c.n);
+        ++issued;
+        c.next(P);
+        if (++s == P.stages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
+      // copies in flight must land before the CTA exits (instant on the normal path)
+      for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
+        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr,
+                  0u);
     }
-    const int wo = tw * P.BW + wl;
-    if (wl < P.BW && c < P.C) {
-      const Vec* px = reinterpret_cast<const Vec*>(smem + (size_t)s * P.stage_bytes) +
-                      (wl * S) * NV + cv;
-      const int row_v = P.IW * NV;                      // vectors per input row of the box
-      float2 rows[3][3][NP];                            // [slot][kw][channel pair]
-      auto load_row = [&](int r, float2 (&dst)[3][NP]) {
+  } else {
+    const int tid = threadIdx.x - 32, cv = tid % NV, wl = tid / NV;
+    Dw3Coord c;
+    c.set(P, t_begin);
+    int prev_ct = -1;
+    float2 wv[3][3][NP];
+    float2 bv[NP];
+    int s = 0;
+    unsigned int ph = 0;
+    for (long long t = t_begin; t < t_end; ++t) {
+      bool got = mbar_try_wait(&full[s], ph);
+      if (!got) got = mbar_wait(&full[s], ph, abort_flag, err, 16u);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const int ch = c.ct * DW3_CH + cv * VEC;
+      if (c.ct != prev_ct) {
+        prev_ct = c.ct;
+        if (ch < P.C) {
 #pragma unroll
-        for (int kw = 0; kw < 3; ++kw) unpack_vec<T>(px[r * row_v + kw * NV], dst[kw]);
-      };
-      T* yp = y + (((long long)n * P.Ho + th * BH) * P.Wo + wo) * P.C + c;
-      const long long ystep = (long long)P.Wo * P.C;
-      load_row(0, rows[0]);
-      if (S == 1) load_row(1, rows[1]);
+          for (int kh = 0; kh < 3; ++kh)
 #pragma unroll
-      for (int j = 0; j < BH; ++j) {
-        if (S == 1) {
-          load_row(j + 2, rows[(j + 2) % 3]);
-        } else {
-          load_row(2 * j + 1, rows[(2 * j + 1) % 3]);
-          load_row(2 * j + 2, rows[(2 * j + 2) % 3]);
-        }
-        // two partial sums per channel pair (taps split by kh parity) for more ILP
-        float2 acc[2][NP];
+            for (int kw = 0; kw < 3; ++kw)
 #pragma unroll
-        for (int q = 0; q < NP; ++q) {
-          acc[0][q] = bv[q];
-          acc[1][q] = make_float2(0.f, 0.f);
-        }
-#pragma unroll
-        for (int kh = 0; kh < 3; ++kh) {
-          const int slot = (j * S + kh) % 3;
-#pragma unroll
-          for (int kw = 0; kw < 3; ++kw)
-#pragma unroll
-            for (int q = 0; q < NP; ++q)
-              acc[kh & 1][q] = ffma2(wv[kh][kw][q], rows[slot][kw][q], acc[kh & 1][q]);
-        }
-        if (th * BH + j < P.Ho && wo < P.Wo) {
-          Vec o;
-          unsigned int* ou = reinterpret_cast<unsigned int*>(&o);
+              for (int q = 0; q < NP; ++q)
+                wv[kh][kw][q] =
+                    make_float2(Elem<T>::to_f32(w[(ch + 2 * q) * 9 + kh * 3 + kw]),
+                                Elem<T>::to_f32(w[(ch + 2 * q + 1) * 9 + kh * 3 + kw]));
 #pragma unroll
           for (int q = 0; q < NP; ++q)
-            ou[q] = pack2<T>(make_float2(acc[0][q].x + acc[1][q].x, acc[0][q].y + acc[1][q].y));
-          *reinterpret_cast<Vec*>(yp + j * ystep) = o;
+            bv[q] = bias ? make_float2(Elem<T>::to_f32(bias[ch + 2 * q]),
+                                       Elem<T>::to_f32(bias[ch + 2 * q + 1]))
+                         : make_float2(0.f, 0.f);
         }
       }
-    }
-    __syncthreads();   // every thread is done with stage s
-    if (tid == 0) {
-      const long long t2 = t + (long long)P.stages * gridDim.x;
-      if (t2 < P.num_tiles) {
-        issue((int)t2, s);
-        ++issued;
+      const int wo = c.tw * P.BW + wl;
+      if (wl < P.BW && ch < P.C && wo < P.Wo) {
+        const Vec* px = reinterpret_cast<const Vec*>(smem + (size_t)s * P.stage_bytes) +
+                        (wl * S) * NV + cv;
+        const int row_v = P.IW * NV;                    // vectors per input row of the box
+        float2 rows[3][3][NP];                          // [slot][kw][channel pair]
+        auto load_row = [&](int r, float2 (&dst)[3][NP]) {
+#pragma unroll
+          for (int kw = 0; kw < 3; ++kw) unpack_vec<T>(px[r * row_v + kw * NV], dst[kw]);
+        };
+        const int ho0 = c.th * BH;
+        T* yp = y + (((long long)c.n * P.Ho + ho0) * P.Wo + wo) * P.C + ch;
+        const long long ystep = (long long)P.Wo * P.C;
+        load_row(0, rows[0]);
+        if (S == 1) load_row(1, rows[1]);
+#pragma unroll
+        for (int j = 0; j < BH; ++j) {
+          if (S == 1) {
+            load_row(j + 2, rows[(j + 2) % 3]);
+          } else {
+            load_row(2 * j + 1, rows[(2 * j + 1) % 3]);
+            load_row(2 * j + 2, rows[(2 * j + 2) % 3]);
+          }
+          // two partial sums per channel pair (taps split by kh parity) for more ILP
+          float2 acc[2][NP];
+#pragma unroll
+          for (int q = 0; q < NP; ++q) {
+            acc[0][q] = bv[q];
+            acc[1][q] = make_float2(0.f, 0.f);
+          }
+#pragma unroll
+          for (int kh = 0; kh < 3; ++kh) {
+            const int slot = (j * S + kh) % 3;
+#pragma unroll
+            for (int kw = 0; kw < 3; ++kw)
+#pragma unroll
+              for (int q = 0; q < NP; ++q)
+                acc[kh & 1][q] = ffma2(wv[kh][kw][q], rows[slot][kw][q], acc[kh & 1][q]);
+          }
+          if (ho0 + j < P.Ho) {
+            Vec o;
+            unsigned int* ou = reinterpret_cast<unsigned int*>(&o);
+#pragma unroll
+            for (int q = 0; q < NP; ++q)
+              ou[q] = pack2<T>(make_float2(acc[0][q].x + acc[1][q].x, acc[0][q].y + acc[1][q].y));
+            // streaming store: the output is not re-read, keep L2 for the input halo
+            __stcs(reinterpret_cast<Vec*>(yp + j * ystep), o);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      c.next(P);
+      if (++s == P.stages) {
+        s = 0;
+        ph ^= 1u;
       }
     }
   }
-  // copies still in flight (only after an abort) must land before the CTA exits
-  if (tid == 0) {
-    for (long long q = consumed; q < issued; ++q)
-      mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr, 0u);
-  }
+  __syncthreads();
 }
 
 template <typename T, int S, int BH>
@@ -339,12 +368,17 @@ cudaError_t launch_dw3_tma(const Conv2d& p, const void* x, const void* w, const 
   P.num_tiles = (int)tiles;
   P.tx_bytes = (unsigned int)(DW3_CH * P.IW * P.IH * 2);
   P.stage_bytes = (P.tx_bytes + 127u) & ~127u;
-  int stages = (int)(DW3_SMEM_BUDGET / 3 / P.stage_bytes);   // three CTAs per SM
+  // two CTAs per SM when two rings of >= 2 stages fit, else one CTA with a deeper ring
+  int per_sm = 2;
+  int stages = (int)(DW3_SMEM_BUDGET / 2 / P.stage_bytes);
+  if (stages < 2) {
+    per_sm = 1;
+    stages = (int)(DW3_SMEM_BUDGET / P.stage_bytes);
+  }
   if (stages > DW3_MAX_STAGES) stages = DW3_MAX_STAGES;
-  if (stages < 2) stages = 2;
-  if ((size_t)stages * P.stage_bytes > DW3_SMEM_BUDGET) return cudaErrorInvalidValue;
+  if (stages < 2) return cudaErrorInvalidValue;
   P.stages = stages;
-  const size_t smem = 128 + (size_t)stages * P.stage_bytes + DW3_MAX_STAGES * 8 + 16;
+  const size_t smem = 128 + (size_t)stages * P.stage_bytes + 2 * DW3_MAX_STAGES * 8 + 16;
 
   EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
@@ -365,14 +399,16 @@ cudaError_t launch_dw3_tma(const Conv2d& p, const void* x, const void* w, const 
   cudaError_t e = set_max_dynamic_smem((const void*)dw3x3_tma_kernel<T, S, BH, VEC>,
                                        DW3_SMEM_BUDGET + 1024, configured);
   if (e != cudaSuccess) return e;
-  int per_sm = 3;
+  // whole warps only: the compute warps use full-mask warp collectives
+  const int threads = 32 + ((NV * P.BW + 31) / 32) * 32;
+  int fit = per_sm;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-          &per_sm, dw3x3_tma_kernel<T, S, BH, VEC>, NV * P.BW, smem) != cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
-  long long grid = (long long)sm_count() * per_sm;
+          &fit, dw3x3_tma_kernel<T, S, BH, VEC>, threads, smem) != cudaSuccess || fit < 1)
+    fit = 1;
+  if (fit > per_sm) fit = per_sm;
+  long long grid = (long long)sm_count() * fit;
   if (grid > P.num_tiles) grid = P.num_tiles;
-  dw3x3_tma_kernel<T, S, BH, VEC><<<(unsigned)grid, NV * P.BW, smem, s>>>(
+  dw3x3_tma_kernel<T, S, BH, VEC><<<(unsigned)grid, threads, smem, s>>>(
       tm, (const T*)w, (const T*)bias, (T*)y, P, device_error_word());
   return cudaGetLastError();
 }
@@ -417,8 +453,8 @@ template <typename T>
 cudaError_t launch_typed(const Conv2d& p, const void* x, const void* w, const void* bias, void* y,
                          cudaStream_t s) {
   if (dw3_tma_eligible(p))
-    return p.stride == 1 ? launch_dw3_tma<T, 1, 8>(p, x, w, bias, y, s)
-                         : launch_dw3_tma<T, 2, 4>(p, x, w, bias, y, s);
+    return p.stride == 1 ? launch_dw3_tma<T, 1, 16>(p, x, w, bias, y, s)
+                         : launch_dw3_tma<T, 2, 8>(p, x, w, bias, y, s);
   const int K = p.kH;
   if (p.stride == 1) {
     if (K == 3) return launch_ks<T, 3, 1>(p, x, w, bias, y, s);

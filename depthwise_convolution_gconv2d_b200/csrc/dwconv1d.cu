@@ -9,21 +9,27 @@
 //                    = the forward with the filter reversed and pads (K-1-pl, K-1-pr)
 //   wgrad  dw[c,k]   = sum_{b,t} dy[b,t,c] * x[b, t+k-pl, c]
 //
-// Vector kernels (16-bit data, C % 8 == 0, 16-byte aligned x / dy, K in the instantiated set):
-//  * fwd / dgrad: a block stages a [128 + K - 1 steps] x [64 channels] input tile in shared
-//    memory as fp32 pairs (16-byte global loads, zero fill outside [0, T)). A thread owns a
-//    channel pair and 16 consecutive outputs; its K filter taps stay in registers and each
-//    staged input step is read once and applied to every output it touches (packed fp32x2
-//    FMA). The loop over the kernel size is fully unrolled.
-//  * wgrad: a block owns 64 channels and a fixed slice of one batch's steps; a thread keeps K
-//    fp32-pair partial sums for its channel pair over 16-step strips; strips are summed in a
-//    fixed order in shared memory and the per-slice partials go to the caller's workspace. A
-//    second kernel sums the slices in a fixed order. No float atomics: bitwise reproducible.
+// Vector kernels (16-bit data, C % 8 == 0, 16-byte aligned x / dy, K in the instantiated set)
+// stream their inputs with TMA through shared-memory rings filled by a producer warp (the
+// tensor map's zero fill outside [0, T) is the padding), so bytes in flight come from the copy
+// engine rather than from thread count:
+//  * fwd / dgrad: persistent CTAs walk a contiguous chunk of [128 steps x 64 channels] output
+//    tiles; a box of 128 + K - 1 input steps per tile. A thread owns a channel pair and 16
+//    consecutive outputs; its K filter taps stay in registers (reloaded only when the chunk
+//    moves to the next channel tile) and each staged input step is read once from shared
+//    memory and applied to every output it touches (packed fp32x2 FMA, loop over the kernel
+//    size fully unrolled).
+//  * wgrad: a block owns 64 channels and a fixed slice of one batch's steps and streams
+//    (dy, x) box pairs of 128 steps through its ring; a thread keeps K fp32-pair partial sums
+//    for its channel pair over 16-step strips; strips are summed in a fixed order in shared
+//    memory and the per-slice partials go to the caller's workspace. A second kernel sums the
+//    slices in a fixed order. No float atomics: bitwise reproducible.
 // Generic kernels cover every other shape, one thread per output (fwd/dgrad) or one warp per
 // (c, k) with a fixed-order shuffle reduction (wgrad).
 #include <type_traits>
 
 #include "internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace gconv {
 namespace {
@@ -35,126 +41,286 @@ constexpr int CH = 2 * CP;        // channels per block
 constexpr int TB = TS * STRIPS;   // steps per block tile
 constexpr int NTHREADS = CP * STRIPS;
 
-// Stage steps [s0, s0 + rows) x channels [c0, c0 + 64) of a [.., T, C] tensor as fp32 pairs
-// dst[r * CP + pair]; zero outside [0, T) and beyond C.
-template <typename T>
-__device__ __forceinline__ void stage_rows(float2* dst, const T* src, int T_len, int C, int s0,
-                                           int rows, int c0) {
-  for (int i = threadIdx.x; i < rows * 8; i += NTHREADS) {
-    const int r = i >> 3, q = i & 7;
-    const int s = s0 + r, c = c0 + q * 8;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (s >= 0 && s < T_len && c < C) v = __ldg(reinterpret_cast<const uint4*>(src + (long long)s * C + c));
-    float2* d = dst + r * CP + q * 4;
-    d[0] = unpack2<T>(v.x);
-    d[1] = unpack2<T>(v.y);
-    d[2] = unpack2<T>(v.z);
-    d[3] = unpack2<T>(v.w);
+// Ring kernels: 1 producer warp + RSTRIPS compute warps = 8 warps, so that two CTAs share an
+// SM (the register file is split across the four SM sub-partitions; a ninth warp would put
+// three warps of each CTA on one of them)
+constexpr int RSTRIPS = 7;
+constexpr int RCOMPUTE = 32 * RSTRIPS;
+constexpr int RING_THREADS = 32 + RCOMPUTE;
+constexpr int TBF = TS * RSTRIPS;               // forward: steps per tile
+constexpr int MAX_STAGES = 6;
+
+struct Ring1d {
+  int B, T_in, C, T_out, pl;
+  int n_ct, n_tt, num_tiles, stages;
+  unsigned int stage_bytes, tx_bytes;
+};
+
+// tile t -> (step tile, batch, channel tile), channel tile slowest
+struct Coord1d {
+  int tt, b, ct;
+  __device__ __forceinline__ void set(const Ring1d& P, long long t) {
+    tt = (int)(t % P.n_tt);
+    const long long r = t / P.n_tt;
+    b = (int)(r % P.B);
+    ct = (int)(r / P.B);
   }
-}
+  __device__ __forceinline__ void next(const Ring1d& P) {
+    if (++tt < P.n_tt) return;
+    tt = 0;
+    if (++b < P.B) return;
+    b = 0;
+    ++ct;
+  }
+};
 
 template <typename T, int K, bool FLIP>
-__global__ void __launch_bounds__(NTHREADS, 2) dwconv1d_fwd_kernel(const T* __restrict__ x,
-                                                                    const T* __restrict__ w,
-                                                                    T* __restrict__ y, int T_in,
-                                                                    int C, int T_out, int pl) {
-  extern __shared__ float2 smem[];
-  constexpr int ROWS = TB + K - 1;
-  float2* xs = smem;               // [ROWS][CP]
-  float* wsm = reinterpret_cast<float*>(smem + ROWS * CP);   // [K][CH]
-  const int tid = threadIdx.x, cp = tid % CP, strip = tid / CP;
-  const int c0 = blockIdx.x * CH, t0 = blockIdx.y * TB, b = blockIdx.z;
-
-  for (int i = tid; i < CH * K; i += NTHREADS) {
-    const int cc = i / K, k = i % K;
-    const float v = (c0 + cc < C) ? Elem<T>::to_f32(w[(long long)(c0 + cc) * K + k]) : 0.0f;
-    wsm[(FLIP ? K - 1 - k : k) * CH + cc] = v;
+__global__ void __maxnreg__(104)
+    dwconv1d_fwd_kernel(const __grid_constant__ CUtensorMap tmx, const T* __restrict__ w,
+                        T* __restrict__ y, const Ring1d P, unsigned int* err) {
+  using namespace ptx;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  unsigned long long* full =
+      reinterpret_cast<unsigned long long*>(smem + (size_t)P.stages * P.stage_bytes);
+  unsigned long long* empty = full + MAX_STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + MAX_STAGES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long t_begin = (long long)P.num_tiles * blockIdx.x / gridDim.x;
+  const long long t_end = (long long)P.num_tiles * (blockIdx.x + 1) / gridDim.x;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], RSTRIPS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmx);
   }
-  stage_rows<T>(xs, x + (long long)b * T_in * C, T_in, C, t0 - pl, ROWS, c0);
   __syncthreads();
-
-  float2 wk[K];
+  if (warp == 0) {
+    if (lane == 0) {
+      Coord1d c;
+      c.set(P, t_begin);
+      int s = 0;
+      unsigned int ph = 0;
+      long long issued = 0;
+      for (long long t = t_begin; t < t_end; ++t) {
+        if (!mbar_try_wait(&empty[s], ph ^ 1u) &&
+            !mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, 32u))
+          break;
+        mbar_arrive_expect_tx(&full[s], P.tx_bytes);
+        tma_load_3d(smem + (size_t)s * P.stage_bytes, &tmx, &full[s], c.ct * CH,
+                    c.tt * TBF - P.pl, c.b);
+        ++issued;
+        c.next(P);
+        if (++s == P.stages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
+        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr,
+                  0u);
+    }
+  } else {
+    // taps of the current channel tile as fp32 pairs [K][CP] after the ring
+    float2* wsm = reinterpret_cast<float2*>(empty + MAX_STAGES + 2);
+    const int cp = lane, strip = warp - 1, ctid = threadIdx.x - 32;
+    Coord1d c;
+    c.set(P, t_begin);
+    int prev_ct = -1;
+    int s = 0;
+    unsigned int ph = 0;
+    for (long long t = t_begin; t < t_end; ++t) {
+      const int ch = c.ct * CH + 2 * cp;
+      if (c.ct != prev_ct) {
+        prev_ct = c.ct;
+        asm volatile("bar.sync 1, %0;" ::"r"(RCOMPUTE));   // compute warps only
+        for (int i = ctid; i < K * CP; i += RCOMPUTE) {
+          const int k = i / CP, pp = i % CP;
+          const int kk = FLIP ? K - 1 - k : k;
+          const int cc = c.ct * CH + 2 * pp;
+          wsm[i] = cc < P.C ? make_float2(Elem<T>::to_f32(w[(long long)cc * K + kk]),
+                                          Elem<T>::to_f32(w[(long long)(cc + 1) * K + kk]))
+                            : make_float2(0.f, 0.f);
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(RCOMPUTE));
+      }
+      bool got = mbar_try_wait(&full[s], ph);
+      if (!got) got = mbar_wait(&full[s], ph, abort_flag, err, 32u);
+      if (!__all_sync(0xffffffffu, got)) break;
+      // staged box: row r (input step tt*TB - pl + r) holds 64 channels = 32 packed pairs
+      const uint32_t* xr =
+          reinterpret_cast<const uint32_t*>(smem + (size_t)s * P.stage_bytes) + strip * TS * CP +
+          cp;
+      float2 acc[TS];
 #pragma unroll
-  for (int k = 0; k < K; ++k) wk[k] = reinterpret_cast<const float2*>(wsm + k * CH)[cp];
-  float2 acc[TS];
+      for (int i = 0; i < TS; ++i) acc[i] = make_float2(0.f, 0.f);
+      // the filter in passes of at most KC taps, so only KC taps are live in registers
+      constexpr int KC = K > 16 ? (K + 2) / 3 : K;
 #pragma unroll
-  for (int i = 0; i < TS; ++i) acc[i] = make_float2(0.f, 0.f);
-  const float2* xr = xs + strip * TS * CP + cp;
+      for (int k0 = 0; k0 < K; k0 += KC) {
+        const int kn = K - k0 < KC ? K - k0 : KC;
+        float2 wk[KC];
 #pragma unroll
-  for (int j = 0; j < TS + K - 1; ++j) {
-    const float2 xv = xr[j * CP];
+        for (int k = 0; k < KC; ++k)
+          if (k < kn) wk[k] = wsm[(k0 + k) * CP + cp];
 #pragma unroll
-    for (int i = 0; i < TS; ++i) {
-      const int k = j - i;
-      if (k >= 0 && k < K) acc[i] = ffma2(wk[k], xv, acc[i]);
+        for (int j = 0; j < TS + KC - 1; ++j) {
+          if (j < TS + kn - 1) {
+            const float2 xv = unpack2<T>(xr[(k0 + j) * CP]);
+#pragma unroll
+            for (int i = 0; i < TS; ++i) {
+              const int k = j - i;
+              if (k >= 0 && k < kn) acc[i] = ffma2(wk[k], xv, acc[i]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (ch < P.C) {
+        const int t0 = c.tt * TBF + strip * TS;
+        T* yp = y + ((long long)c.b * P.T_out + t0) * P.C + ch;
+#pragma unroll
+        for (int i = 0; i < TS; ++i)
+          if (t0 + i < P.T_out)
+            *reinterpret_cast<uint32_t*>(yp + (long long)i * P.C) = pack2<T>(acc[i]);
+      }
+      c.next(P);
+      if (++s == P.stages) {
+        s = 0;
+        ph ^= 1u;
+      }
     }
   }
-  const int c = c0 + 2 * cp;
-  if (c < C) {
-    T* yp = y + ((long long)b * T_out + t0 + strip * TS) * C + c;
-#pragma unroll
-    for (int i = 0; i < TS; ++i)
-      if (t0 + strip * TS + i < T_out)
-        *reinterpret_cast<uint32_t*>(yp + (long long)i * C) = pack2<T>(acc[i]);
-  }
+  __syncthreads();
 }
 
-template <typename T, int K>
-__global__ void __launch_bounds__(NTHREADS, 2) dwconv1d_wgrad_kernel(
-    const T* __restrict__ x, const T* __restrict__ dy, float* __restrict__ partial, int T_in,
-    int C, int T_out, int pl, int slice_len, int n_tslices) {
-  extern __shared__ float2 smem[];
-  float2* dys = smem;              // [TB][CP]
-  float2* xs = smem + TB * CP;     // [TB + K - 1][CP]
-  const int tid = threadIdx.x, cp = tid % CP, strip = tid / CP;
-  const int c0 = blockIdx.x * CH;
-  const int slice = blockIdx.y, b = slice / n_tslices, ts = slice % n_tslices;
-  const int t_begin = ts * slice_len;
-  const int t_end = min(T_out, t_begin + slice_len);
-  const T* xb = x + (long long)b * T_in * C;
-  const T* dyb = dy + (long long)b * T_out * C;
+constexpr int WTS = 8;             // weight gradient: steps per thread strip
+constexpr int WTB = WTS * RSTRIPS; // steps per sub-tile
 
+struct WgradRing {
+  int T_in, C, T_out, pl, slice_len, n_tslices, stages;
+  unsigned int stage_bytes, dy_bytes, x_bytes;
+};
+
+template <typename T, int K>
+__global__ void __maxnreg__(104)
+    dwconv1d_wgrad_kernel(const __grid_constant__ CUtensorMap tmx,
+                          const __grid_constant__ CUtensorMap tmdy, float* __restrict__ partial,
+                          const WgradRing P, unsigned int* err) {
+  using namespace ptx;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  unsigned long long* full =
+      reinterpret_cast<unsigned long long*>(smem + (size_t)P.stages * P.stage_bytes);
+  unsigned long long* empty = full + MAX_STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + MAX_STAGES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ct = blockIdx.x;
+  const int slice = blockIdx.y, b = slice / P.n_tslices, ts = slice % P.n_tslices;
+  const int t_begin = ts * P.slice_len;
+  const int t_end = min(P.T_out, t_begin + P.slice_len);
+  const int n_sub = (t_end - t_begin + WTB - 1) / WTB;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], RSTRIPS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmx);
+    prefetch_tmap(&tmdy);
+  }
+  __syncthreads();
   float2 acc[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) acc[k] = make_float2(0.f, 0.f);
-
-  for (int tb = t_begin; tb < t_end; tb += TB) {
-    stage_rows<T>(dys, dyb, t_end, C, tb, TB, c0);          // zero at and beyond t_end
-    stage_rows<T>(xs, xb, T_in, C, tb - pl, TB + K - 1, c0);
-    __syncthreads();
-    float2 dv[TS];
+  if (warp == 0) {
+    if (lane == 0) {
+      // the last sub-tile may reach into the next slice: those dy steps are masked to zero by
+      // the compute warps; past T_out the boxes read the tensor map's zero fill
+      int s = 0;
+      unsigned int ph = 0;
+      long long issued = 0;
+      for (int i = 0; i < n_sub; ++i) {
+        if (!mbar_try_wait(&empty[s], ph ^ 1u) &&
+            !mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, 64u))
+          break;
+        const int tb = t_begin + i * WTB;
+        unsigned char* st = smem + (size_t)s * P.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], P.dy_bytes + P.x_bytes);
+        tma_load_3d(st, &tmdy, &full[s], ct * CH, tb, b);
+        tma_load_3d(st + P.dy_bytes, &tmx, &full[s], ct * CH, tb - P.pl, b);
+        ++issued;
+        if (++s == P.stages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
+        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr,
+                  0u);
+    }
+  } else {
+    const int cp = lane, strip = warp - 1;
+    int s = 0;
+    unsigned int ph = 0;
+    for (int i = 0; i < n_sub; ++i) {
+      bool got = mbar_try_wait(&full[s], ph);
+      if (!got) got = mbar_wait(&full[s], ph, abort_flag, err, 64u);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const uint32_t* dyr = reinterpret_cast<const uint32_t*>(smem + (size_t)s * P.stage_bytes) +
+                            strip * WTS * CP + cp;
+      const uint32_t* xr =
+          reinterpret_cast<const uint32_t*>(smem + (size_t)s * P.stage_bytes + P.dy_bytes) +
+          strip * WTS * CP + cp;
+      const int tq0 = t_begin + i * WTB + strip * WTS;   // step of dv[0]
+      float2 dv[WTS];
 #pragma unroll
-    for (int i = 0; i < TS; ++i) dv[i] = dys[(strip * TS + i) * CP + cp];
-    const float2* xr = xs + strip * TS * CP + cp;
+      for (int q = 0; q < WTS; ++q)
+        dv[q] = tq0 + q < t_end ? unpack2<T>(dyr[q * CP]) : make_float2(0.f, 0.f);
 #pragma unroll
-    for (int j = 0; j < TS + K - 1; ++j) {
-      const float2 xv = xr[j * CP];
+      for (int j = 0; j < WTS + K - 1; ++j) {
+        const float2 xv = unpack2<T>(xr[j * CP]);
 #pragma unroll
-      for (int i = 0; i < TS; ++i) {
-        const int k = j - i;
-        if (k >= 0 && k < K) acc[k] = ffma2(dv[i], xv, acc[k]);
+        for (int q = 0; q < WTS; ++q) {
+          const int k = j - q;
+          if (k >= 0 && k < K) acc[k] = ffma2(dv[q], xv, acc[k]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == P.stages) {
+        s = 0;
+        ph ^= 1u;
       }
     }
-    __syncthreads();
   }
-  // fixed-order sum over the block's strips
-  float2* red = smem;              // [STRIPS][K][CP], fits in the staging area
+  __syncthreads();   // ring drained: reuse it for the fixed-order sum over strips
+  float2* red = reinterpret_cast<float2*>(smem);     // [RSTRIPS][K][CP]
+  if (warp > 0) {
 #pragma unroll
-  for (int k = 0; k < K; ++k) red[(strip * K + k) * CP + cp] = acc[k];
+    for (int k = 0; k < K; ++k) red[((warp - 1) * K + k) * CP + lane] = acc[k];
+  }
   __syncthreads();
-  for (int i = tid; i < K * CP; i += NTHREADS) {
+  for (int i = threadIdx.x; i < K * CP; i += blockDim.x) {
     const int k = i / CP, pp = i % CP;
-    float2 s = red[k * CP + pp];
-    for (int st = 1; st < STRIPS; ++st) {
+    float2 sum = red[k * CP + pp];
+    for (int st = 1; st < RSTRIPS; ++st) {
       const float2 v = red[(st * K + k) * CP + pp];
-      s.x += v.x;
-      s.y += v.y;
+      sum.x += v.x;
+      sum.y += v.y;
     }
-    const int c = c0 + 2 * pp;
-    if (c < C) {
-      float* dst = partial + ((long long)slice * C + c) * K + k;
-      dst[0] = s.x;
-      dst[K] = s.y;
+    const int c = ct * CH + 2 * pp;
+    if (c < P.C) {
+      float* dst = partial + ((long long)slice * P.C + c) * K + k;
+      dst[0] = sum.x;
+      dst[K] = sum.y;
     }
   }
 }
@@ -218,16 +384,51 @@ bool k_instantiated(int K) {
   return K == 3 || K == 5 || K == 7 || K == 9 || K == 15 || K == 31;
 }
 
+bool make_tensor_map_btc(CUtensorMap* m, int dtype, const void* base, int C, int T_len, int B,
+                         int rows) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const CUtensorMapDataType dt =
+      dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T_len, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)C * 2, (cuuint64_t)T_len * C * 2};
+  const cuuint32_t box[3] = {CH, (cuuint32_t)rows, 1};
+  const cuuint32_t ones[3] = {1, 1, 1};
+  return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, ones,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T, int K, bool FLIP>
-cudaError_t fwd_vec(const T* x, const T* w, T* y, int B, int T_in, int C, int T_out, int pl,
-                    cudaStream_t s) {
-  const size_t smem = (size_t)(TB + K - 1) * CP * sizeof(float2) + (size_t)K * CH * sizeof(float);
+cudaError_t fwd_vec(const Conv1d& p, const T* x, const T* w, T* y, int B, int T_in, int C,
+                    int T_out, int pl, cudaStream_t s) {
+  Ring1d P;
+  P.B = B; P.T_in = T_in; P.C = C; P.T_out = T_out; P.pl = pl;
+  P.n_ct = (C + CH - 1) / CH;
+  P.n_tt = (T_out + TBF - 1) / TBF;
+  const long long tiles = (long long)P.n_ct * B * P.n_tt;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  P.num_tiles = (int)tiles;
+  P.tx_bytes = (unsigned int)(TBF + K - 1) * CH * 2;
+  P.stage_bytes = (P.tx_bytes + 127u) & ~127u;
+  P.stages = 4;
+  const size_t smem = 128 + (size_t)P.stages * P.stage_bytes + 2 * MAX_STAGES * 8 + 16 +
+                      (size_t)K * CP * sizeof(float2);
+  CUtensorMap tm;
+  if (!make_tensor_map_btc(&tm, p.dtype, x, C, T_in, B, TBF + K - 1)) return cudaErrorInvalidValue;
   static std::atomic<unsigned int> configured{0};
   cudaError_t e = set_max_dynamic_smem((const void*)dwconv1d_fwd_kernel<T, K, FLIP>, smem,
                                        configured);
   if (e != cudaSuccess) return e;
-  dim3 grid((C + CH - 1) / CH, (T_out + TB - 1) / TB, B);
-  dwconv1d_fwd_kernel<T, K, FLIP><<<grid, NTHREADS, smem, s>>>(x, w, y, T_in, C, T_out, pl);
+  int fit = 2;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, dwconv1d_fwd_kernel<T, K, FLIP>,
+                                                    RING_THREADS, smem) != cudaSuccess ||
+      fit < 1)
+    fit = 1;
+  long long grid = (long long)sm_count() * fit;
+  if (grid > P.num_tiles) grid = P.num_tiles;
+  dwconv1d_fwd_kernel<T, K, FLIP><<<(unsigned)grid, RING_THREADS, smem, s>>>(tm, w, y, P,
+                                                                           device_error_word());
   return cudaGetLastError();
 }
 
@@ -239,12 +440,12 @@ cudaError_t fwd_dispatch(const Conv1d& p, const void* x, const void* w, void* y,
   T* yy = (T*)y;
   if constexpr (!std::is_same<T, float>::value) {
     if (vec) switch (p.K) {
-      case 3: return fwd_vec<T, 3, FLIP>(xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
-      case 5: return fwd_vec<T, 5, FLIP>(xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
-      case 7: return fwd_vec<T, 7, FLIP>(xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
-      case 9: return fwd_vec<T, 9, FLIP>(xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
-      case 15: return fwd_vec<T, 15, FLIP>(xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
-      case 31: return fwd_vec<T, 31, FLIP>(xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
+      case 3: return fwd_vec<T, 3, FLIP>(p, xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
+      case 5: return fwd_vec<T, 5, FLIP>(p, xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
+      case 7: return fwd_vec<T, 7, FLIP>(p, xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
+      case 9: return fwd_vec<T, 9, FLIP>(p, xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
+      case 15: return fwd_vec<T, 15, FLIP>(p, xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
+      case 31: return fwd_vec<T, 31, FLIP>(p, xx, ww, yy, p.B, T_in, p.C, T_out, pl, s);
       default: break;
     }
   }
@@ -282,16 +483,28 @@ cudaError_t wgrad_vec(const Conv1d& p, const T* x, const T* dy, T* dw, float* pa
                       cudaStream_t s) {
   int slice_len, n_tslices;
   wgrad_slicing(p, &slice_len, &n_tslices);
-  const size_t stage = (size_t)(2 * TB + K - 1) * CP * sizeof(float2);
-  const size_t red = (size_t)STRIPS * K * CP * sizeof(float2);
-  const size_t smem = stage > red ? stage : red;
+  WgradRing P;
+  P.T_in = p.T; P.C = p.C; P.T_out = p.T_out; P.pl = p.pad_left;
+  P.slice_len = slice_len; P.n_tslices = n_tslices;
+  P.dy_bytes = (unsigned int)WTB * CH * 2;
+  P.x_bytes = (unsigned int)(WTB + K - 1) * CH * 2;
+  P.stage_bytes = (P.dy_bytes + P.x_bytes + 127u) & ~127u;
+  P.stages = 4;
+  const size_t red = (size_t)RSTRIPS * K * CP * sizeof(float2);
+  size_t ring = (size_t)P.stages * P.stage_bytes;
+  if (ring < red) ring = red;
+  const size_t smem = 128 + ring + 2 * MAX_STAGES * 8 + 16;
+  CUtensorMap tx, tdy;
+  if (!make_tensor_map_btc(&tx, p.dtype, x, p.C, p.T, p.B, WTB + K - 1) ||
+      !make_tensor_map_btc(&tdy, p.dtype, dy, p.C, p.T_out, p.B, WTB))
+    return cudaErrorInvalidValue;
   static std::atomic<unsigned int> configured{0};
   cudaError_t e = set_max_dynamic_smem((const void*)dwconv1d_wgrad_kernel<T, K>, smem, configured);
   if (e != cudaSuccess) return e;
   const int n_slices = p.B * n_tslices;
   dim3 grid((p.C + CH - 1) / CH, n_slices);
-  dwconv1d_wgrad_kernel<T, K><<<grid, NTHREADS, smem, s>>>(x, dy, partial, p.T, p.C, p.T_out,
-                                                            p.pad_left, slice_len, n_tslices);
+  dwconv1d_wgrad_kernel<T, K><<<grid, RING_THREADS, smem, s>>>(tx, tdy, partial, P,
+                                                               device_error_word());
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int CK = p.C * p.K;

@@ -281,6 +281,223 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------ halo tile kernel
+//
+// For images narrower than 128 outputs (whole rows per tile: BW = Wo, BH = 128 / Wo rows), a
+// stage is one input-channel block and KWS filter columns: per column kw one TMA box of
+// BH + (kH-1)*dil input rows x Wo pixels, whose kH taps are the same box read from row offsets
+// kh*dil*Wo (whole 8-row swizzle atoms, since Wo % 8 == 0), plus the kH*KWS weight tiles.
+// Each stage thus feeds kH*KWS*BKC/16 MMAs to the single issuing thread between barrier waits,
+// and the input is fetched once per kw instead of once per tap.
+
+struct HaloParams {
+  int N, H, W, C_in, C_out, Ho, Wo, kH, kW, pad, dil, cpg_in, cpg_out;
+  int BW, BH, BN, BKC, cblocks, KWS, kw_groups, tiles_h, m_tiles, n_tiles, num_tiles;
+  int stages, box_rows;
+  unsigned int a_region, a_stage, b_tile, b_stage, tx_bytes;
+  unsigned int idesc, swz, sbo, row_bytes, tmem_cols;
+  int out_nchw;
+};
+
+__device__ __forceinline__ void halo_decode(const HaloParams& P, int t, int& j, int& nt, int& n,
+                                            int& th) {
+  const int mt = t % P.m_tiles, rest = t / P.m_tiles;
+  nt = rest % P.n_tiles;
+  j = rest / P.n_tiles;
+  th = mt % P.tiles_h;
+  n = mt / P.tiles_h;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    igemm_halo_kernel(const __grid_constant__ CUtensorMap tma_x,
+                      const __grid_constant__ CUtensorMap tma_w, const T* __restrict__ bias,
+                      T* __restrict__ y, const HaloParams P, unsigned int* err) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* a_base = smem;
+  unsigned char* b_base = smem + (size_t)P.stages * P.a_stage;
+  unsigned long long* bars =
+      reinterpret_cast<unsigned long long*>(b_base + (size_t)P.stages * P.b_stage);
+  unsigned long long* full = bars;
+  unsigned long long* empty = bars + MAX_STAGES;
+  unsigned long long* tfull = bars + 2 * MAX_STAGES;
+  unsigned long long* tempty = tfull + 2;
+  unsigned long long* done = tempty + 2;
+  unsigned int* tmem_slot = reinterpret_cast<unsigned int*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tma_x);
+    prefetch_tmap(&tma_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, P.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const unsigned int tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int s = 0;
+      unsigned int ph = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
+        int j, nt, n, th;
+        halo_decode(P, t, j, nt, n, th);
+        const int hbase = th * P.BH - P.pad;
+        const int obase = j * P.cpg_out + nt * P.BN;
+        for (int cb = 0; cb < P.cblocks && ok; ++cb) {
+          const int cin = j * P.cpg_in + cb * P.BKC;
+          for (int kg = 0; kg < P.kw_groups; ++kg) {
+            if (!mbar_try_wait(&empty[s], ph ^ 1u) &&
+                !mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[s], P.tx_bytes);
+            unsigned char* a_st = a_base + (size_t)s * P.a_stage;
+            unsigned char* b_st = b_base + (size_t)s * P.b_stage;
+            for (int kwi = 0; kwi < P.KWS; ++kwi) {
+              const int kw = kg * P.KWS + kwi;
+              tma_load_4d(a_st + (size_t)kwi * P.a_region, &tma_x, &full[s], cin,
+                          kw * P.dil - P.pad, hbase, n);
+              for (int kh = 0; kh < P.kH; ++kh)
+                tma_load_2d(b_st + (size_t)(kwi * P.kH + kh) * P.b_tile, &tma_w, &full[s],
+                            (kh * P.kW + kw) * P.cpg_in + cb * P.BKC, obase);
+            }
+            ++issued;
+            if (++s == P.stages) {
+              s = 0;
+              ph ^= 1u;
+            }
+          }
+        }
+      }
+      for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
+        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, err,
+                  ERR_WAIT_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer (descriptors built once, advanced by offsets)
+      int s = 0, acc = 0;
+      unsigned int ph = 0, aph = 0;
+      bool ok = true;
+      const int ksteps = P.BKC / 16;
+      const unsigned long long a_desc0 = smem_desc(smem_u32(a_base), P.sbo, P.swz);
+      const unsigned long long b_desc0 = smem_desc(smem_u32(b_base), P.sbo, P.swz);
+      const unsigned long long kh_step =
+          ((unsigned long long)P.dil * P.BW * P.row_bytes) >> 4;   // kh rows of the box
+      const unsigned long long kw_step = P.a_region >> 4;
+      const unsigned long long bt_step = P.b_tile >> 4;
+      for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERR_WAIT_MMA)) break;
+        tc_fence_after();
+        const unsigned int d = tmem_base + (unsigned int)(acc * P.BN);
+        for (int cb = 0; cb < P.cblocks && ok; ++cb) {
+          for (int kg = 0; kg < P.kw_groups; ++kg) {
+            if (!mbar_try_wait(&full[s], ph) &&
+                !mbar_wait(&full[s], ph, abort_flag, err, ERR_WAIT_MMA)) {
+              ok = false;
+              break;
+            }
+            const unsigned long long ad0 = a_desc0 + (((unsigned long long)s * P.a_stage) >> 4);
+            const unsigned long long bd0 = b_desc0 + (((unsigned long long)s * P.b_stage) >> 4);
+            for (int kwi = 0; kwi < P.KWS; ++kwi) {
+              for (int kh = 0; kh < P.kH; ++kh) {
+                const unsigned long long ad = ad0 + kwi * kw_step + kh * kh_step;
+                const unsigned long long bd = bd0 + (kwi * P.kH + kh) * bt_step;
+                const unsigned int acc0 = (cb | kg | kwi | kh) == 0 ? 0u : 1u;
+                umma_f16(d, ad, bd, P.idesc, acc0);
+                if (ksteps > 1) umma_f16(d, ad + 2, bd + 2, P.idesc, 1u);
+                if (ksteps > 2) {
+                  umma_f16(d, ad + 4, bd + 4, P.idesc, 1u);
+                  umma_f16(d, ad + 6, bd + 6, P.idesc, 1u);
+                }
+              }
+            }
+            umma_commit(&empty[s]);
+            if (++s == P.stages) {
+              s = 0;
+              ph ^= 1u;
+            }
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          aph ^= 1u;
+        }
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, abort_flag, err, ERR_WAIT_DRAIN);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5, TMEM lane quarter (warp % 4)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int hl = row / P.BW, wl = row - hl * P.BW;
+    int acc = 0;
+    unsigned int aph = 0;
+    for (int t = blockIdx.x; t < P.num_tiles; t += gridDim.x) {
+      int j, nt, n, th;
+      halo_decode(P, t, j, nt, n, th);
+      const bool got = mbar_wait(&tfull[acc], aph, abort_flag, err, ERR_WAIT_EPILOGUE);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int ho = th * P.BH + hl, wo = wl;
+      const bool valid = hl < P.BH && ho < P.Ho;
+      const int co0 = j * P.cpg_out + nt * P.BN;
+      const unsigned int taddr =
+          tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.BN);
+      for (int c = 0; c < P.BN; c += 32) {
+        unsigned int r[32];
+        const int ncols = P.BN - c < 32 ? P.BN - c : 32;
+        if (ncols == 32)
+          tmem_ld32(taddr + c, r);
+        else
+          tmem_ld16(taddr + c, r);
+        tmem_ld_wait();
+        if (valid) epilogue_store<T>(P, y, bias, r, ncols, n, ho, wo, co0 + c);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, P.tmem_cols);
+  }
+}
+
 // ------------------------------------------------------------------ row-strip kernel
 //
 // For rows of at least 128 output pixels (Wo >= 128), a tile is NSUB consecutive 128-pixel
@@ -804,33 +1021,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // ------------------------------------------------------------------ NCHW staging kernels
 
-// x[n][c][hw] -> xt[n][hw][c], 64 x 64 tiles through shared memory.
-template <typename T>
+// x[n][c][hw] -> xt[n][hw][c], 64 x 64 tiles through shared memory. When HW and C are
+// multiples of 8 both the global loads (8 consecutive hw of one channel) and the global stores
+// (8 consecutive channels of one pixel) are 16-byte vectors; the transposition itself is done
+// with 2-byte shared-memory accesses (row pitch 66 elements against bank conflicts).
+template <typename T, bool VEC>
 __global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const T* __restrict__ x,
                                                            T* __restrict__ xt, int C, int HW) {
-  __shared__ T tile[64][66];
+  __shared__ unsigned short tile[64][66];   // [c][hw]
   const int n = blockIdx.z;
   const int c0 = blockIdx.y * 64, s0 = blockIdx.x * 64;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const T* xn = x + (long long)n * C * HW;
-  T* tn = xt + (long long)n * C * HW;
+  const unsigned short* xn = reinterpret_cast<const unsigned short*>(x) + (long long)n * C * HW;
+  unsigned short* tn = reinterpret_cast<unsigned short*>(xt) + (long long)n * C * HW;
+  const int tid = threadIdx.x;
+  if (VEC) {
+    // 64 channels x 8 vectors of 8 pixels: 512 loads, 2 per thread
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int c = c0 + ty + 8 * r;
+    for (int r = 0; r < 2; ++r) {
+      const int i = tid + 256 * r;
+      const int cl = i >> 3, v = i & 7;
+      const int c = c0 + cl, sp = s0 + v * 8;
+      uint4 u = make_uint4(0u, 0u, 0u, 0u);
+      if (c < C && sp < HW) u = __ldg(reinterpret_cast<const uint4*>(xn + (long long)c * HW + sp));
+      const unsigned short* e = reinterpret_cast<const unsigned short*>(&u);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int s = s0 + tx + 32 * h;
-      if (c < C && s < HW) tile[ty + 8 * r][tx + 32 * h] = xn[(long long)c * HW + s];
+      for (int q = 0; q < 8; ++q) tile[cl][v * 8 + q] = e[q];
     }
-  }
-  __syncthreads();
+    __syncthreads();
+    // 64 pixels x 8 vectors of 8 channels
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int s = s0 + ty + 8 * r;
+    for (int r = 0; r < 2; ++r) {
+      const int i = tid + 256 * r;
+      const int sl = i >> 3, v = i & 7;
+      const int sp = s0 + sl, c = c0 + v * 8;
+      if (sp < HW && c < C) {
+        uint4 u;
+        unsigned short* e = reinterpret_cast<unsigned short*>(&u);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = c0 + tx + 32 * h;
-      if (c < C && s < HW) tn[(long long)s * C + c] = tile[tx + 32 * h][ty + 8 * r];
+        for (int q = 0; q < 8; ++q) e[q] = tile[v * 8 + q][sl];
+        *reinterpret_cast<uint4*>(tn + (long long)sp * C + c) = u;
+      }
+    }
+  } else {
+    const int tx = tid & 31, ty = tid >> 5;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int c = c0 + ty + 8 * r;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int sp = s0 + tx + 32 * h;
+        if (c < C && sp < HW) tile[ty + 8 * r][tx + 32 * h] = xn[(long long)c * HW + sp];
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int sp = s0 + ty + 8 * r;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = c0 + tx + 32 * h;
+        if (c < C && sp < HW) tn[(long long)sp * C + c] = tile[tx + 32 * h][ty + 8 * r];
+      }
     }
   }
 }
@@ -1108,6 +1359,109 @@ cudaError_t launch_rowt(const Conv2d& p, const RowTParams& R, const void* x, con
   return cudaGetLastError();
 }
 
+// Halo tile kernel parameters; false if the problem does not take it (rows wider than 128,
+// a width that is not a multiple of 8, or stages that do not fit).
+bool make_halo_params(const Conv2d& p, HaloParams* H) {
+  if (p.Wo > BM || p.Wo % 8 != 0) return false;
+  const int BN = tile_bn(p);
+  if (BN == 0) return false;
+  H->N = p.N; H->H = p.H; H->W = p.W; H->C_in = p.C_in; H->C_out = p.C_out;
+  H->Ho = p.Ho; H->Wo = p.Wo; H->kH = p.kH; H->kW = p.kW; H->pad = p.pad; H->dil = p.dil;
+  H->cpg_in = p.cpg_in; H->cpg_out = p.cpg_out;
+  H->BW = p.Wo;
+  H->BH = BM / p.Wo;
+  if (H->BH > p.Ho) H->BH = p.Ho;
+  H->BN = BN;
+  H->BKC = p.cpg_in % 64 == 0 ? 64 : (p.cpg_in % 32 == 0 ? 32 : 16);
+  H->cblocks = p.cpg_in / H->BKC;
+  H->tiles_h = (p.Ho + H->BH - 1) / H->BH;
+  const long long m_tiles = (long long)p.N * H->tiles_h;
+  H->n_tiles = p.cpg_out / BN;
+  const long long tiles = m_tiles * H->n_tiles * p.groups;
+  if (tiles > INT32_MAX) return false;
+  H->m_tiles = (int)m_tiles;
+  H->num_tiles = (int)tiles;
+  H->box_rows = H->BH + (p.kH - 1) * p.dil;
+  if (H->box_rows > 256) return false;
+  H->row_bytes = (unsigned int)H->BKC * 2u;
+  // rows an MMA may read from a box: up to (kH-1)*dil*BW + 128
+  unsigned int rows = (unsigned int)(H->box_rows * H->BW);
+  const unsigned int mma_rows = (unsigned int)((p.kH - 1) * p.dil * H->BW + BM);
+  if (mma_rows > rows) rows = mma_rows;
+  H->a_region = (rows * H->row_bytes + 1023u) & ~1023u;
+  H->b_tile = (unsigned int)BN * H->row_bytes;
+  const size_t fixed = 1024 + (2 * MAX_STAGES + 5) * 8 + 16;
+  const size_t budget = SMEM_BUDGET - fixed;
+  // all kw of a channel block per stage when three such stages fit, else one kw per stage
+  int kws = p.kW;
+  for (;;) {
+    const size_t st = (size_t)kws * H->a_region + ((size_t)kws * p.kH * H->b_tile + 1023) / 1024 * 1024;
+    const int n = (int)(budget / st);
+    if (n >= 3 || kws == 1) {
+      H->KWS = kws;
+      H->a_stage = (unsigned int)((size_t)kws * H->a_region);
+      H->b_stage = (unsigned int)(((size_t)kws * p.kH * H->b_tile + 1023) / 1024 * 1024);
+      H->stages = n > MAX_STAGES ? MAX_STAGES : n;
+      break;
+    }
+    kws = 1;
+  }
+  if (H->stages < 2) return false;
+  H->kw_groups = p.kW / H->KWS;
+  H->tx_bytes = (unsigned int)H->KWS *
+                ((unsigned int)(H->BKC * H->BW * H->box_rows * 2) + (unsigned int)p.kH * H->b_tile);
+  H->swz = H->row_bytes == 128 ? 2u : (H->row_bytes == 64 ? 4u : 6u);
+  H->sbo = 8u * H->row_bytes;
+  const unsigned int fmt = p.dtype == GCONV_BF16 ? 1u : 0u;
+  H->idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((unsigned int)(BN >> 3) << 17) |
+             ((unsigned int)(BM >> 4) << 24);
+  H->tmem_cols = pow2_cols(2 * BN);
+  H->out_nchw = p.layout == GCONV_NCHW;
+  return true;
+}
+
+size_t halo_smem_bytes(const HaloParams& H) {
+  return 1024 + (size_t)H.stages * (H.a_stage + H.b_stage) + (2 * MAX_STAGES + 5) * 8 + 16;
+}
+
+template <typename T>
+cudaError_t launch_halo(const Conv2d& p, const HaloParams& H, const void* x, const void* w,
+                        const void* bias, void* y, cudaStream_t s) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const CUtensorMapDataType dt =
+      p.dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tx, tw;
+  const cuuint64_t xdim[4] = {(cuuint64_t)p.C_in, (cuuint64_t)p.W, (cuuint64_t)p.H,
+                              (cuuint64_t)p.N};
+  const cuuint64_t xstr[3] = {(cuuint64_t)p.C_in * 2, (cuuint64_t)p.W * p.C_in * 2,
+                              (cuuint64_t)p.H * p.W * p.C_in * 2};
+  const cuuint32_t xbox[4] = {(cuuint32_t)H.BKC, (cuuint32_t)H.BW, (cuuint32_t)H.box_rows, 1};
+  const cuuint32_t ones[4] = {1, 1, 1, 1};
+  if (enc(&tx, dt, 4, const_cast<void*>(x), xdim, xstr, xbox, ones,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(H.BKC), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const cuuint64_t ktot = (cuuint64_t)p.kH * p.kW * p.cpg_in;
+  const cuuint64_t wdim[2] = {ktot, (cuuint64_t)p.C_out};
+  const cuuint64_t wstr[1] = {ktot * 2};
+  const cuuint32_t wbox[2] = {(cuuint32_t)H.BKC, (cuuint32_t)H.BN};
+  if (enc(&tw, dt, 2, const_cast<void*>(w), wdim, wstr, wbox, ones,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(H.BKC), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const size_t smem = halo_smem_bytes(H);
+  if (smem > SMEM_BUDGET) return cudaErrorInvalidValue;
+  static std::atomic<unsigned int> configured{0};
+  cudaError_t e = set_max_dynamic_smem((const void*)igemm_halo_kernel<T>, SMEM_BUDGET, configured);
+  if (e != cudaSuccess) return e;
+  int grid = sm_count();
+  if (grid > H.num_tiles) grid = H.num_tiles;
+  igemm_halo_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, tw, (const T*)bias, (T*)y, H,
+                                                       device_error_word());
+  return cudaGetLastError();
+}
+
 // x: NHWC activations, w: [C_out][kH][kW][cpg_in] weights (both device pointers).
 template <typename T>
 cudaError_t launch_core(const Conv2d& p, const IgemmParams& P, const void* x, const void* w,
@@ -1116,6 +1470,8 @@ cudaError_t launch_core(const Conv2d& p, const IgemmParams& P, const void* x, co
   if (make_rowt_params(p, &RT)) return launch_rowt<T>(p, RT, x, w, bias, y, s);
   RowParams R;
   if (make_row_params(p, &R)) return launch_row<T>(p, R, x, w, bias, y, s);
+  HaloParams HP;
+  if (make_halo_params(p, &HP)) return launch_halo<T>(p, HP, x, w, bias, y, s);
   EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   const CUtensorMapDataType dt =
@@ -1196,7 +1552,10 @@ cudaError_t launch_nchw_typed(const Conv2d& p, const IgemmParams& P, const void*
   if (e != cudaSuccess) return e;
   const int HW = p.H * p.W;
   dim3 grid((HW + 63) / 64, (p.C_in + 63) / 64, p.N);
-  nchw_to_nhwc_kernel<T><<<grid, 256, 0, s>>>((const T*)x, xt, p.C_in, HW);
+  if (HW % 8 == 0 && p.C_in % 8 == 0 && aligned16(x))
+    nchw_to_nhwc_kernel<T, true><<<grid, 256, 0, s>>>((const T*)x, xt, p.C_in, HW);
+  else
+    nchw_to_nhwc_kernel<T, false><<<grid, 256, 0, s>>>((const T*)x, xt, p.C_in, HW);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_core<T>(p, P, xt, wt, bias, y, s);

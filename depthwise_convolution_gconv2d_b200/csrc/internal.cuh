@@ -80,6 +80,11 @@ inline cudaError_t set_max_dynamic_smem(const void* func, size_t bytes,
   const unsigned int bit = 1u << (dev & 31);
   if (mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  // ask for the largest shared-memory carveout, so that occupancy is not cut by an L1/shared
+  // split sized for a single block
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) mask.fetch_or(bit, std::memory_order_acq_rel);
   return e;
 }

@@ -32,6 +32,9 @@ SMALL = [
     (2, 128, 3, 300, 256, 3, 1, 1, 2),       # transposed row kernel, 2 segments per row
     (1, 64, 6, 140, 128, 3, 2, 2, 1),        # transposed row kernel with dilation 2
     (1, 64, 7, 131, 128, 5, 2, 1, 1),        # transposed row kernel, 5x5
+    (1, 64, 12, 16, 64, 3, 2, 2, 2),         # halo tile kernel: Wo = 16, dilation 2
+    (2, 96, 9, 32, 96, 5, 2, 1, 3),          # halo tile kernel: 5x5, 32 / 32
+    (1, 128, 5, 40, 64, 3, 1, 1, 2),         # halo tile kernel: 64-channel blocks, 3-row tiles
 ]
 
 
