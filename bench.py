@@ -455,11 +455,15 @@ def main():
     value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
     avg_launch_ms = sum(launch_ms) / len(launch_ms)
     achieved = flops / (avg_launch_ms * 1e-3) / 1e12
-    tensor_peak = pk["bf16_tflops"]
+    # the timed region is a long back-to-back loop (sustained clocks under the power cap), so
+    # the denominator is the sustained bf16 figure; the burst fraction is reported beside it
+    tensor_peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tensor_peak,
             "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4),
             "traffic": traffic_for(kernel_name(kcode), KERNEL_SOURCE.get(kcode, "")),
-            "kernel": kernel_name(kcode), "peak_source": f"bf16_tflops (burst) {peak_src}"}
+            "kernel": kernel_name(kcode),
+            "peak_source": f"bf16_tflops_sustained {peak_src}",
+            "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4)}
     if kcode in (1, 2):   # CUDA-core kernels on this workload are not tensor-bound
         roof["note"] = "CUDA-core path selected; tensor peak used as the headline denominator"
 

@@ -548,8 +548,10 @@ bool conv1d_vector_supported(const Conv1d& p) {
 
 cudaError_t launch_dwconv1d_fwd(const Conv1d& p, const void* x, const void* w, void* y, bool flip,
                                 int pad_left, int T_in, int T_out, cudaStream_t s) {
-  const bool vec = conv1d_vector_supported(p) && aligned16(x) && aligned16(y);
   if (p.B == 0) return cudaSuccess;
+  if (conv1d_tc_supported(p) && aligned16(x) && aligned16(y) && aligned16(w))
+    return launch_dwconv1d_tc(p, x, w, y, flip, pad_left, T_in, T_out, s);
+  const bool vec = conv1d_vector_supported(p) && aligned16(x) && aligned16(y);
   switch (p.dtype) {
     case GCONV_F32: return fwd_any_dtype<float>(p, x, w, y, flip, pad_left, T_in, T_out, false, s);
     case GCONV_F16: return fwd_any_dtype<__half>(p, x, w, y, flip, pad_left, T_in, T_out, vec, s);

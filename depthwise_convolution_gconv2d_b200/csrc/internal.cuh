@@ -109,6 +109,10 @@ cudaError_t launch_igemm_nchw(const Conv2d& p, const void* x, const void* w, con
 bool conv1d_vector_supported(const Conv1d& p);
 cudaError_t launch_dwconv1d_fwd(const Conv1d& p, const void* x, const void* w, void* y,
                                 bool flip, int pad_left, int T_in, int T_out, cudaStream_t s);
+// Tensor-core forward / data gradient: 16-bit data, C % 8 == 0, K <= 49, 16-byte aligned x, w, y.
+bool conv1d_tc_supported(const Conv1d& p);
+cudaError_t launch_dwconv1d_tc(const Conv1d& p, const void* x, const void* w, void* y, bool flip,
+                               int pad_left, int T_in, int T_out, cudaStream_t s);
 size_t dwconv1d_wgrad_workspace(const Conv1d& p);
 cudaError_t launch_dwconv1d_wgrad(const Conv1d& p, const void* x, const void* dy, void* dw,
                                   void* workspace, cudaStream_t s);

@@ -1,7 +1,9 @@
 """GPU parity of dwconv1d_fwd / dwconv1d_bwd_data / dwconv1d_bwd_weight against the fp64
 oracle, on the Conformer workload (x[8, 2048, 512], K = 31, 'same' and causal pads) in full
-and on small ragged shapes; bit-exact on integer-valued data where sums are exact; wgrad
-bitwise reproducible."""
+and on small ragged shapes; the tensor-core forward / data gradient on its edge cases (several
+2048-step chunks, ragged chunk ends, every filter-window size up to K = 49, inputs shorter
+than a TMA box, pads wider than a box); bit-exact on integer-valued data where sums are
+exact; wgrad bitwise reproducible."""
 import numpy as np
 import pytest
 import torch
@@ -55,9 +57,32 @@ SMALL = [
     (2, 100, 40, 31, 0, 0),       # T_out < T
     (1, 20, 8, 31, 15, 15),       # T shorter than the filter
     (2, 90, 5, 31, 15, 15),       # C not a multiple of 8: generic kernels
-    (1, 33, 16, 4, 2, 1),         # K without an unrolled kernel: generic
+    (1, 33, 16, 4, 2, 1),         # K without an unrolled wgrad kernel: generic wgrad
     (2, 45, 24, 11, 10, 0),
 ]
+
+# Tensor-core forward / data gradient (16-bit data, C % 16 == 0, K <= 49): tiles of 16
+# channels x 2048 steps, MMA rows of 16-step blocks, 16*KS-step input windows with
+# KS = ceil((K + 15) / 16). C % 16 == 8 (e.g. 72, 136 above) takes the CUDA-core ring kernel.
+TC_CASES = [
+    # B, T, C, K, pl, pr
+    (1, 4100, 16, 31, 15, 15),    # three chunks, the last one ragged
+    (2, 2049, 16, 17, 8, 8),      # KS = 2 at its largest K; one step into a second chunk
+    (2, 2048, 32, 33, 16, 16),    # KS = 3 at its largest K; two channel tiles
+    (1, 500, 16, 34, 17, 16),     # KS = 4
+    (1, 300, 16, 49, 24, 24),     # K = 49, the largest filter on the tensor cores
+    (1, 300, 16, 50, 25, 24),     # K = 50: CUDA-core kernels
+    (1, 700, 16, 1, 0, 0),        # K = 1, KS = 1
+    (1, 300, 32, 31, 30, 30),     # T_out > T
+    (1, 100, 16, 5, 300, 0),      # left pad wider than a TMA box: box skipped, zeros
+    (3, 7, 48, 31, 15, 15),       # T far shorter than the window
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES)
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F16])
+def test_tensor_core_edges(case, dtype):
+    check(wl.Dwconv1dProblem(*case, dtype), 33)
 
 
 @pytest.mark.parametrize("case", SMALL)
@@ -66,7 +91,7 @@ def test_small_shapes(case, dtype):
     check(wl.Dwconv1dProblem(*case, dtype), 30)
 
 
-@pytest.mark.parametrize("case", SMALL[:8])
+@pytest.mark.parametrize("case", SMALL[:8] + TC_CASES[:3])
 def test_integer_valued_bit_exact_fwd_dgrad(case):
     """Integers in [-2, 2]: every partial sum is exact in fp32 and the result (|.| <= 124)
     is exact in bf16, so any summation order gives the oracle's value bit for bit."""
