@@ -353,6 +353,42 @@ def config_dict(p, args):
 
 # ---------------------------------------------------------------------------- main
 
+PROFILE_WORKLOADS = ("wide_group_nhwc", "wide_group_nchw", "ensemble_g64", "depthwise56_s1",
+                     "depthwise56_s2", "dw1d_same", "sweep56_g64", "sweep56_g16")
+
+
+def run_profile(name: str, reps: int) -> int:
+    """--profile: run one workload's launches `reps` times (no timing), for profiler captures."""
+    import torch
+
+    from depthwise_convolution_gconv2d_b200 import binding as gb
+    device = torch.device("cuda", 0)
+    if name == "dw1d_same":
+        p = wl.conformer_dw1d(False)
+        inp = wl.make_dwconv1d_inputs(p, 3)
+        x, w, dy = (dev_tensor(torch, a, p.dtype, device) for a in (inp.x, inp.w, inp.dy))
+        for _ in range(reps):
+            gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right)
+            gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right)
+            gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right)
+    else:
+        p = {"wide_group_nhwc": lambda: wl.wide_group(wl.NHWC),
+             "wide_group_nchw": lambda: wl.wide_group(wl.NCHW),
+             "ensemble_g64": wl.ensemble_groups,
+             "depthwise56_s1": lambda: wl.depthwise_56(1),
+             "depthwise56_s2": lambda: wl.depthwise_56(2),
+             "sweep56_g64": lambda: wl.depthwise_56(1, 64),
+             "sweep56_g16": lambda: wl.depthwise_56(1, 16)}[name]()
+        inp = wl.make_conv2d_inputs(p, 2)
+        x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
+        for _ in range(reps):
+            gb.gconv2d_fwd(x, w, None, p.stride, p.pad, p.dilation, p.groups, p.layout)
+    torch.cuda.synchronize()
+    code = gb.device_error()
+    print(json.dumps({"profile": name, "reps": reps, "device_error": code}))
+    return 0 if code == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -364,7 +400,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-depthwise", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile", choices=PROFILE_WORKLOADS,
+                    help="run this workload's launches --profile-reps times for a profiler "
+                         "capture, untimed, and exit")
+    ap.add_argument("--profile-reps", type=int, default=2)
     args = ap.parse_args()
+    if args.profile:
+        return run_profile(args.profile, args.profile_reps)
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         return run_reference(args)

@@ -9,10 +9,10 @@
 // kernel: persistent CTAs stream (rows x columns x 64 channels) input boxes through a ring of
 // shared-memory stages with one TMA load per tile (the tensor map's zero fill is the padding),
 // so the bytes in flight per SM come from the copy engine rather than from thread count.
-// Each thread owns 4 channels of one output column; the three input rows it needs sit in
-// registers as fp32 pairs and rotate by renaming as the fully unrolled row loop moves down;
-// the 3x3 filter of its channels stays in registers; the multiply-adds are fp32x2 packed.
-//
+// Each thread owns one channel pair across 4 adjacent output columns: every staged input word
+// it needs is read and widened to fp32 once and then feeds all of its outputs (3 rows of 6 or
+// 9 fp32 pairs rotate by renaming as the fully unrolled row loop moves down); the 3x3 filter
+// of its pair stays in registers; the multiply-adds are fp32x2 packed, 4 independent chains.
 // Other shapes run the register-window kernel: a thread owns VEC consecutive channels (one 16-,
 // 8- or 4-byte vector) of one output column (n, wo) and walks down a chunk of output rows. Its
 // kH x kW input window sits in registers as packed 16-bit vectors; moving one output row down
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(256) depthwise_nhwc_kernel(
 
 constexpr int DW3_MAX_STAGES = 8;
 constexpr int DW3_CH = 64;                 // channels per tile (128-byte box rows)
-constexpr size_t DW3_SMEM_BUDGET = 200 * 1024;
+constexpr size_t DW3_SMEM_BUDGET = 220 * 1024;   // per SM: two CTAs of <= 110 KB
 
 struct Dw3Params {
   int N, H, W, C, Ho, Wo, pad;
@@ -154,19 +154,6 @@ struct Dw3Params {
   int n_ct, n_wt, n_ht, num_tiles, stages;
   unsigned int stage_bytes, tx_bytes;
 };
-
-template <typename T>
-__device__ __forceinline__ void unpack_vec(const uint4& v, float2 (&o)[4]) {
-  o[0] = unpack2<T>(v.x);
-  o[1] = unpack2<T>(v.y);
-  o[2] = unpack2<T>(v.z);
-  o[3] = unpack2<T>(v.w);
-}
-template <typename T>
-__device__ __forceinline__ void unpack_vec(const uint2& v, float2 (&o)[2]) {
-  o[0] = unpack2<T>(v.x);
-  o[1] = unpack2<T>(v.y);
-}
 
 // Tile coordinates, channel tile slowest: tw -> th -> n -> ct. A CTA walks a contiguous chunk
 // of tiles, so its filter registers change only when the chunk crosses a channel tile.
@@ -191,32 +178,35 @@ struct Dw3Coord {
   }
 };
 
-constexpr int DW3_MAX_BW = 14;             // output columns per tile (16 x 14 = 224 compute threads)
-constexpr int DW3_THREADS = 32 + 16 * DW3_MAX_BW;
+constexpr int DW3_R = 4;                   // output columns per thread
+constexpr int DW3_NG = 7;                  // column groups (one compute warp each)
+constexpr int DW3_BW = DW3_R * DW3_NG;     // output columns per tile
+constexpr int DW3_THREADS = 32 + 32 * DW3_NG;
+template <int S> constexpr int DW3_IW() { return (DW3_BW - 1) * S + 3; }   // input box columns
 
 // Warp 0 lane 0 is the TMA producer; warps 1.. compute. Stage s is handed over through
 // full[s] (TMA transaction bytes) and empty[s] (one arrival per compute warp).
-template <typename T, int S, int BH, int VEC>
+template <typename T, int S, int BH>
 __global__ void __launch_bounds__(DW3_THREADS, 2)
-    dw3x3_tma_kernel(const __grid_constant__ CUtensorMap tmx, const T* __restrict__ w,
-                     const T* __restrict__ bias, T* __restrict__ y, const Dw3Params P,
-                     unsigned int* err) {
+    dw3x3_tma_kernel(const __grid_constant__ CUtensorMap tmx,
+                     const __grid_constant__ CUtensorMap tmy, const T* __restrict__ w,
+                     const T* __restrict__ bias, const Dw3Params P, unsigned int* err) {
   using namespace ptx;
-  constexpr int NP = VEC / 2;                 // channel pairs per thread
-  constexpr int NV = DW3_CH / VEC;            // channel vectors per tile row
-  using Vec = typename VecT<NP>::type;        // VEC 16-bit values
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  // output staging after the input ring: compute warp g owns [BH][DW3_R][64 ch], the box of
+  // its own TMA store
+  unsigned char* ostage = smem + (size_t)P.stages * P.stage_bytes;
   unsigned long long* full =
-      reinterpret_cast<unsigned long long*>(smem + (size_t)P.stages * P.stage_bytes);
+      reinterpret_cast<unsigned long long*>(ostage + (size_t)BH * DW3_BW * DW3_CH * 2);
   unsigned long long* empty = full + DW3_MAX_STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + DW3_MAX_STAGES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_compute_warps = (int)(blockDim.x >> 5) - 1;
-  const long long t_begin = (long long)P.num_tiles * blockIdx.x / gridDim.x;
-  const long long t_end = (long long)P.num_tiles * (blockIdx.x + 1) / gridDim.x;
+  const int t_begin = (int)((long long)P.num_tiles * blockIdx.x / gridDim.x);
+  const int t_end = (int)((long long)P.num_tiles * (blockIdx.x + 1) / gridDim.x);
   if (threadIdx.x == 0) {
     for (int s = 0; s < P.stages; ++s) {
       mbar_init(&full[s], 1);
@@ -225,6 +215,7 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmx);
+    prefetch_tmap(&tmy);
   }
   __syncthreads();
 
@@ -235,7 +226,7 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
       int s = 0;
       unsigned int ph = 0;
       long long issued = 0;
-      for (long long t = t_begin; t < t_end; ++t) {
+      for (int t = t_begin; t < t_end; ++t) {
         if (!mbar_try_wait(&empty[s], ph ^ 1u) &&
             !mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, 16u))
           break;
@@ -255,96 +246,88 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
                   0u);
     }
   } else {
-    const int tid = threadIdx.x - 32, cv = tid % NV, wl = tid / NV;
+    constexpr int NIN = (DW3_R - 1) * S + 3;        // input columns a thread reads per row
+    constexpr int row_w = DW3_IW<S>() * (DW3_CH / 2);  // 32-bit words per box row
+    const int cp = lane, g = warp - 1;
     Dw3Coord c;
     c.set(P, t_begin);
     int prev_ct = -1;
-    float2 wv[3][3][NP];
-    float2 bv[NP];
+    float2 wv[3][3];
+    float2 bv = make_float2(0.f, 0.f);
     int s = 0;
     unsigned int ph = 0;
-    for (long long t = t_begin; t < t_end; ++t) {
+    unsigned char* wstage = ostage + (size_t)g * BH * DW3_R * DW3_CH * 2;
+    unsigned int* orow = reinterpret_cast<unsigned int*>(wstage) + cp;
+    for (int t = t_begin; t < t_end; ++t) {
       bool got = mbar_try_wait(&full[s], ph);
       if (!got) got = mbar_wait(&full[s], ph, abort_flag, err, 16u);
       if (!__all_sync(0xffffffffu, got)) break;
-      const int ch = c.ct * DW3_CH + cv * VEC;
+      if (lane == 0) bulk_wait_read0();              // this warp's previous store has read it
+      __syncwarp();
+      const int ch = c.ct * DW3_CH + 2 * cp;
+      const bool ch_ok = ch < P.C;
       if (c.ct != prev_ct) {
         prev_ct = c.ct;
-        if (ch < P.C) {
 #pragma unroll
-          for (int kh = 0; kh < 3; ++kh)
+        for (int kh = 0; kh < 3; ++kh)
 #pragma unroll
-            for (int kw = 0; kw < 3; ++kw)
-#pragma unroll
-              for (int q = 0; q < NP; ++q)
-                wv[kh][kw][q] =
-                    make_float2(Elem<T>::to_f32(w[(ch + 2 * q) * 9 + kh * 3 + kw]),
-                                Elem<T>::to_f32(w[(ch + 2 * q + 1) * 9 + kh * 3 + kw]));
-#pragma unroll
-          for (int q = 0; q < NP; ++q)
-            bv[q] = bias ? make_float2(Elem<T>::to_f32(bias[ch + 2 * q]),
-                                       Elem<T>::to_f32(bias[ch + 2 * q + 1]))
-                         : make_float2(0.f, 0.f);
-        }
+          for (int kw = 0; kw < 3; ++kw)
+            wv[kh][kw] = ch_ok ? make_float2(Elem<T>::to_f32(w[ch * 9 + kh * 3 + kw]),
+                                             Elem<T>::to_f32(w[(ch + 1) * 9 + kh * 3 + kw]))
+                               : make_float2(0.f, 0.f);
+        bv = (bias && ch_ok) ? make_float2(Elem<T>::to_f32(bias[ch]), Elem<T>::to_f32(bias[ch + 1]))
+                             : make_float2(0.f, 0.f);
       }
-      const int wo = c.tw * P.BW + wl;
-      if (wl < P.BW && ch < P.C && wo < P.Wo) {
-        const Vec* px = reinterpret_cast<const Vec*>(smem + (size_t)s * P.stage_bytes) +
-                        (wl * S) * NV + cv;
-        const int row_v = P.IW * NV;                    // vectors per input row of the box
-        float2 rows[3][3][NP];                          // [slot][kw][channel pair]
-        auto load_row = [&](int r, float2 (&dst)[3][NP]) {
+      // box word (row, column, pair) = (row * IW + column) * 32 + pair
+      const uint32_t* px = reinterpret_cast<const uint32_t*>(smem + (size_t)s * P.stage_bytes) +
+                           (g * DW3_R * S) * (DW3_CH / 2) + cp;
+      float2 in[3][NIN];                               // input row r lives in slot r % 3
+      auto load_row = [&](int r, float2 (&dst)[NIN]) {
 #pragma unroll
-          for (int kw = 0; kw < 3; ++kw) unpack_vec<T>(px[r * row_v + kw * NV], dst[kw]);
-        };
-        const int ho0 = c.th * BH;
-        T* yp = y + (((long long)c.n * P.Ho + ho0) * P.Wo + wo) * P.C + ch;
-        const long long ystep = (long long)P.Wo * P.C;
-        load_row(0, rows[0]);
-        if (S == 1) load_row(1, rows[1]);
+        for (int i = 0; i < NIN; ++i) dst[i] = unpack2<T>(px[r * row_w + i * (DW3_CH / 2)]);
+      };
+      load_row(0, in[0]);
+      if (S == 1) load_row(1, in[1]);
 #pragma unroll
-        for (int j = 0; j < BH; ++j) {
-          if (S == 1) {
-            load_row(j + 2, rows[(j + 2) % 3]);
-          } else {
-            load_row(2 * j + 1, rows[(2 * j + 1) % 3]);
-            load_row(2 * j + 2, rows[(2 * j + 2) % 3]);
-          }
-          // two partial sums per channel pair (taps split by kh parity) for more ILP
-          float2 acc[2][NP];
-#pragma unroll
-          for (int q = 0; q < NP; ++q) {
-            acc[0][q] = bv[q];
-            acc[1][q] = make_float2(0.f, 0.f);
-          }
-#pragma unroll
-          for (int kh = 0; kh < 3; ++kh) {
-            const int slot = (j * S + kh) % 3;
-#pragma unroll
-            for (int kw = 0; kw < 3; ++kw)
-#pragma unroll
-              for (int q = 0; q < NP; ++q)
-                acc[kh & 1][q] = ffma2(wv[kh][kw][q], rows[slot][kw][q], acc[kh & 1][q]);
-          }
-          if (ho0 + j < P.Ho) {
-            Vec o;
-            unsigned int* ou = reinterpret_cast<unsigned int*>(&o);
-#pragma unroll
-            for (int q = 0; q < NP; ++q)
-              ou[q] = pack2<T>(make_float2(acc[0][q].x + acc[1][q].x, acc[0][q].y + acc[1][q].y));
-            // streaming store: the output is not re-read, keep L2 for the input halo
-            __stcs(reinterpret_cast<Vec*>(yp + j * ystep), o);
-          }
+      for (int j = 0; j < BH; ++j) {
+        if (S == 1) {
+          load_row(j + 2, in[(j + 2) % 3]);
+        } else {
+          load_row(2 * j + 1, in[(2 * j + 1) % 3]);
+          load_row(2 * j + 2, in[(2 * j + 2) % 3]);
         }
+        float2 acc[DW3_R];
+#pragma unroll
+        for (int r = 0; r < DW3_R; ++r) acc[r] = bv;
+#pragma unroll
+        for (int kh = 0; kh < 3; ++kh) {
+          const int slot = (j * S + kh) % 3;
+#pragma unroll
+          for (int kw = 0; kw < 3; ++kw)
+#pragma unroll
+            for (int r = 0; r < DW3_R; ++r)
+              acc[r] = ffma2(wv[kh][kw], in[slot][r * S + kw], acc[r]);
+        }
+        // staged output word (row j, column r, pair cp); the TMA store clips the box at the
+        // tensor's edges (rows past Ho, columns past Wo, channels past C)
+#pragma unroll
+        for (int r = 0; r < DW3_R; ++r)
+          orow[(j * DW3_R + r) * (DW3_CH / 2)] = pack2<T>(acc[r]);
       }
+      fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      if (lane == 0) {
+        mbar_arrive(&empty[s]);
+        tma_store_4d(&tmy, wstage, c.ct * DW3_CH, c.tw * DW3_BW + g * DW3_R, c.th * BH, c.n);
+        bulk_commit();
+      }
       c.next(P);
       if (++s == P.stages) {
         s = 0;
         ph ^= 1u;
       }
     }
+    if (lane == 0) bulk_wait0();
   }
   __syncthreads();
 }
@@ -352,13 +335,10 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
 template <typename T, int S, int BH>
 cudaError_t launch_dw3_tma(const Conv2d& p, const void* x, const void* w, const void* bias,
                            void* y, cudaStream_t s) {
-  constexpr int VEC = 4;
-  constexpr int NV = DW3_CH / VEC;
   Dw3Params P;
   P.N = p.N; P.H = p.H; P.W = p.W; P.C = p.C_in; P.Ho = p.Ho; P.Wo = p.Wo; P.pad = p.pad;
-  const int nw = (p.Wo + DW3_MAX_BW - 1) / DW3_MAX_BW;
-  P.BW = (p.Wo + nw - 1) / nw;
-  P.IW = (P.BW - 1) * S + 3;
+  P.BW = DW3_BW;
+  P.IW = DW3_IW<S>();
   P.IH = (BH - 1) * S + 3;
   P.n_ct = (p.C_in + DW3_CH - 1) / DW3_CH;
   P.n_wt = (p.Wo + P.BW - 1) / P.BW;
@@ -368,17 +348,19 @@ cudaError_t launch_dw3_tma(const Conv2d& p, const void* x, const void* w, const 
   P.num_tiles = (int)tiles;
   P.tx_bytes = (unsigned int)(DW3_CH * P.IW * P.IH * 2);
   P.stage_bytes = (P.tx_bytes + 127u) & ~127u;
-  // two CTAs per SM when two rings of >= 2 stages fit, else one CTA with a deeper ring
-  int per_sm = 2;
-  int stages = (int)(DW3_SMEM_BUDGET / 2 / P.stage_bytes);
-  if (stages < 2) {
-    per_sm = 1;
-    stages = (int)(DW3_SMEM_BUDGET / P.stage_bytes);
+  // as many CTAs per SM (up to 3) as can each hold a ring of >= 2 stages
+  const size_t ostage = (size_t)BH * DW3_BW * DW3_CH * 2;
+  int per_sm = 3, stages = 0;
+  for (; per_sm >= 1; --per_sm) {
+    const size_t share = DW3_SMEM_BUDGET / per_sm;
+    stages = share > ostage ? (int)((share - ostage) / P.stage_bytes) : 0;
+    if (stages >= 2) break;
   }
   if (stages > DW3_MAX_STAGES) stages = DW3_MAX_STAGES;
   if (stages < 2) return cudaErrorInvalidValue;
   P.stages = stages;
-  const size_t smem = 128 + (size_t)stages * P.stage_bytes + 2 * DW3_MAX_STAGES * 8 + 16;
+  const size_t smem =
+      128 + (size_t)stages * P.stage_bytes + ostage + 2 * DW3_MAX_STAGES * 8 + 16;
 
   EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
@@ -391,25 +373,36 @@ cudaError_t launch_dw3_tma(const Conv2d& p, const void* x, const void* w, const 
   const cuuint32_t ones[4] = {1, 1, 1, 1};
   const CUtensorMapDataType dt =
       p.dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  // 128-byte promotion: a box row is one pixel's 64 channels; wider promotion would pull in
+  // the next channel tile, which this CTA order reaches only much later
   if (enc(&tm, dt, 4, const_cast<void*>(x), dims, strides, box, ones,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  CUtensorMap tmy;
+  const cuuint64_t ydims[4] = {(cuuint64_t)p.C_out, (cuuint64_t)p.Wo, (cuuint64_t)p.Ho,
+                               (cuuint64_t)p.N};
+  const cuuint64_t ystrides[3] = {(cuuint64_t)p.C_out * 2, (cuuint64_t)p.Wo * p.C_out * 2,
+                                  (cuuint64_t)p.Ho * p.Wo * p.C_out * 2};
+  const cuuint32_t ybox[4] = {DW3_CH, DW3_R, BH, 1};
+  if (enc(&tmy, dt, 4, y, ydims, ystrides, ybox, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   static std::atomic<unsigned int> configured{0};
-  cudaError_t e = set_max_dynamic_smem((const void*)dw3x3_tma_kernel<T, S, BH, VEC>,
+  cudaError_t e = set_max_dynamic_smem((const void*)dw3x3_tma_kernel<T, S, BH>,
                                        DW3_SMEM_BUDGET + 1024, configured);
   if (e != cudaSuccess) return e;
-  // whole warps only: the compute warps use full-mask warp collectives
-  const int threads = 32 + ((NV * P.BW + 31) / 32) * 32;
+  const int threads = DW3_THREADS;
   int fit = per_sm;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-          &fit, dw3x3_tma_kernel<T, S, BH, VEC>, threads, smem) != cudaSuccess || fit < 1)
+          &fit, dw3x3_tma_kernel<T, S, BH>, threads, smem) != cudaSuccess || fit < 1)
     fit = 1;
   if (fit > per_sm) fit = per_sm;
   long long grid = (long long)sm_count() * fit;
   if (grid > P.num_tiles) grid = P.num_tiles;
-  dw3x3_tma_kernel<T, S, BH, VEC><<<(unsigned)grid, threads, smem, s>>>(
-      tm, (const T*)w, (const T*)bias, (T*)y, P, device_error_word());
+  dw3x3_tma_kernel<T, S, BH><<<(unsigned)grid, threads, smem, s>>>(
+      tm, tmy, (const T*)w, (const T*)bias, P, device_error_word());
   return cudaGetLastError();
 }
 
@@ -453,8 +446,8 @@ template <typename T>
 cudaError_t launch_typed(const Conv2d& p, const void* x, const void* w, const void* bias, void* y,
                          cudaStream_t s) {
   if (dw3_tma_eligible(p))
-    return p.stride == 1 ? launch_dw3_tma<T, 1, 16>(p, x, w, bias, y, s)
-                         : launch_dw3_tma<T, 2, 8>(p, x, w, bias, y, s);
+    return p.stride == 1 ? launch_dw3_tma<T, 1, 8>(p, x, w, bias, y, s)
+                         : launch_dw3_tma<T, 2, 2>(p, x, w, bias, y, s);
   const int K = p.kH;
   if (p.stride == 1) {
     if (K == 3) return launch_ks<T, 3, 1>(p, x, w, bias, y, s);

@@ -92,6 +92,9 @@ DW_CASES = [
     (2, 32, 10, 10, 3, 1, 2, 2),      # dilation: no sliding window
     (1, 8, 1, 1, 3, 1, 1, 1),         # 1x1 image, everything padding but the centre
     (1, 256, 3, 300, 3, 1, 0, 1),     # no padding, wide
+    (1, 128, 5, 29, 3, 1, 1, 1),      # one output column past a 28-column tile
+    (2, 64, 9, 59, 3, 2, 1, 1),       # stride 2: two column tiles, ragged 2-row tiles
+    (1, 72, 4, 57, 3, 2, 2, 1),       # stride 2, pad 2
 ]
 
 
