@@ -268,21 +268,31 @@ def depthwise_measurements(torch, gb, device, stream, pk, reps):
         need = gb.dwconv1d_bwd_weight_workspace_size(p.B, p.T, p.C, p.K, p.pad_left, p.pad_right,
                                                      p.dtype)
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+        sel = lambda path: gb.KERNEL_NAMES.get(gb.dwconv1d_select_path(
+            p.B, p.T, p.C, p.K, p.pad_left, p.pad_right, p.dtype, path), "?")
         ops = {
-            "fwd": lambda i: gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right, out=y, stream=stream),
-            "dgrad": lambda i: gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right, out=dx,
-                                                    stream=stream),
-            "wgrad": lambda i: gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right, out=dw,
-                                                      workspace=ws, stream=stream),
+            "fwd": (lambda i: gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right, out=y,
+                                              stream=stream), sel(gb.PATH_AUTO)),
+            "dgrad": (lambda i: gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right, out=dx,
+                                                     stream=stream), sel(gb.PATH_AUTO)),
+            "wgrad": (lambda i: gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right,
+                                                       out=dw, workspace=ws, stream=stream),
+                      "conv1d_wgrad"),
+            # the CUDA-core ring kernel on the same problem, for comparison
+            "fwd_cudacore": (lambda i: gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right, out=y,
+                                                       stream=stream, path=gb.PATH_DIRECT),
+                             "conv1d_ring"),
         }
         tag = "causal" if causal else "same"
-        for op, fn in ops.items():
+        for op, (fn, kname) in ops.items():
             for _ in range(3):
                 fn(0)
             med, mean = time_launches(torch, fn, stream, reps, flush)
-            gbs = p.bytes(op) / (med * 1e-3) / 1e9
-            out[f"dw1d_{tag}_{op}"] = {"us": round(med * 1e3, 2), "GB/s": round(gbs, 1),
-                                       "frac": round(gbs / hbm, 3), "alg_bytes": p.bytes(op)}
+            ab = p.bytes(op.split("_")[0])
+            gbs = ab / (med * 1e-3) / 1e9
+            out[f"dw1d_{tag}_{op}"] = {"kernel": kname, "us": round(med * 1e3, 2),
+                                       "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 3),
+                                       "alg_bytes": ab}
     return out
 
 

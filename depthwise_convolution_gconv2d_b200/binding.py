@@ -24,13 +24,15 @@ _LIB_PATH = os.path.join(_PKG, "libgconv.so")
 NCHW, NHWC = 0, 1
 F32, F16, BF16 = 0, 1, 2
 PATH_AUTO, PATH_DIRECT, PATH_IGEMM, PATH_GENERIC = 0, 1, 2, 3
-KERNEL_NAMES = {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "igemm_tc_nchw"}
+KERNEL_NAMES = {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "igemm_tc_nchw",
+                5: "conv1d_generic", 6: "conv1d_ring", 7: "conv1d_tc"}
 STATUS = {0: "GCONV_OK", 1: "GCONV_ERR_INVALID_ARG", 2: "GCONV_ERR_UNSUPPORTED",
           3: "GCONV_ERR_MISALIGNED", 4: "GCONV_ERR_WORKSPACE", 5: "GCONV_ERR_CUDA",
           6: "GCONV_ERR_DEVICE_TIMEOUT"}
 
 EXPORTS = ["gconv2d_fwd", "gconv2d_fwd_path", "gconv2d_fwd_workspace_size",
-           "gconv2d_select_path", "dwconv1d_fwd", "dwconv1d_bwd_data",
+           "gconv2d_select_path", "dwconv1d_fwd", "dwconv1d_bwd_data", "dwconv1d_fwd_path",
+           "dwconv1d_bwd_data_path", "dwconv1d_select_path",
            "dwconv1d_bwd_weight", "dwconv1d_bwd_weight_workspace_size",
            "dwconv1d_bwd_weight_noalloc",
            "gconv_get_device_error", "gconv_status_string", "gconv_version"]
@@ -74,6 +76,12 @@ def load_library():
     lib.dwconv1d_fwd.restype = I
     lib.dwconv1d_bwd_data.argtypes = [P, P, P] + [I] * 6 + [I, P]
     lib.dwconv1d_bwd_data.restype = I
+    lib.dwconv1d_fwd_path.argtypes = [P, P, P] + [I] * 6 + [I, I, P]
+    lib.dwconv1d_fwd_path.restype = I
+    lib.dwconv1d_bwd_data_path.argtypes = [P, P, P] + [I] * 6 + [I, I, P]
+    lib.dwconv1d_bwd_data_path.restype = I
+    lib.dwconv1d_select_path.argtypes = [I] * 8
+    lib.dwconv1d_select_path.restype = I
     lib.dwconv1d_bwd_weight_workspace_size.argtypes = [I] * 7
     lib.dwconv1d_bwd_weight_workspace_size.restype = Z
     lib.dwconv1d_bwd_weight.argtypes = [P, P, P, P, Z] + [I] * 6 + [I, P]
@@ -199,7 +207,14 @@ def _conv1d_dims(x, w):
     return B, T, C, K
 
 
-def dwconv1d_fwd(x, w, pad_left, pad_right, out=None, stream=None):
+def dwconv1d_select_path(B, T, C, K, pad_left, pad_right, dtype, path=PATH_AUTO) -> int:
+    """Kernel code (5 generic, 6 CUDA-core ring, 7 tensor cores) a conv1d fwd / dgrad call
+    would run, or a negative status."""
+    dt = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    return int(load_library().dwconv1d_select_path(B, T, C, K, pad_left, pad_right, dt, path))
+
+
+def dwconv1d_fwd(x, w, pad_left, pad_right, out=None, stream=None, path=PATH_AUTO):
     lib = load_library()
     _need(x, "x")
     _need(w, "w", x.dtype)
@@ -207,13 +222,13 @@ def dwconv1d_fwd(x, w, pad_left, pad_right, out=None, stream=None):
     T_out = T + pad_left + pad_right - K + 1
     y = torch.empty((B, T_out, C), dtype=x.dtype, device=x.device) if out is None else out
     _need(y, "out", x.dtype)
-    st = lib.dwconv1d_fwd(_ptr(x), _ptr(w), _ptr(y), B, T, C, K, pad_left, pad_right,
-                          _dtype_code(x.dtype), _stream(stream))
+    st = lib.dwconv1d_fwd_path(_ptr(x), _ptr(w), _ptr(y), B, T, C, K, pad_left, pad_right,
+                               _dtype_code(x.dtype), path, _stream(stream))
     _check(st, "dwconv1d_fwd")
     return y
 
 
-def dwconv1d_bwd_data(dy, w, T, pad_left, pad_right, out=None, stream=None):
+def dwconv1d_bwd_data(dy, w, T, pad_left, pad_right, out=None, stream=None, path=PATH_AUTO):
     lib = load_library()
     _need(dy, "dy")
     _need(w, "w", dy.dtype)
@@ -223,8 +238,8 @@ def dwconv1d_bwd_data(dy, w, T, pad_left, pad_right, out=None, stream=None):
         raise ValueError("dy has the wrong number of steps for T, K and the pads")
     dx = torch.empty((B, T, C), dtype=dy.dtype, device=dy.device) if out is None else out
     _need(dx, "out", dy.dtype)
-    st = lib.dwconv1d_bwd_data(_ptr(dy), _ptr(w), _ptr(dx), B, T, C, K, pad_left, pad_right,
-                               _dtype_code(dy.dtype), _stream(stream))
+    st = lib.dwconv1d_bwd_data_path(_ptr(dy), _ptr(w), _ptr(dx), B, T, C, K, pad_left,
+                                    pad_right, _dtype_code(dy.dtype), path, _stream(stream))
     _check(st, "dwconv1d_bwd_data")
     return dx
 

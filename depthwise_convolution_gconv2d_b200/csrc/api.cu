@@ -194,28 +194,55 @@ gconv_status gconv2d_fwd(const void* x, const void* w, const void* bias, void* y
                           stream);
 }
 
-gconv_status dwconv1d_fwd(const void* x, const void* w, void* y, int B, int T, int C, int K,
-                          int pad_left, int pad_right, gconv_dtype dtype, void* stream) {
+gconv_status dwconv1d_fwd_path(const void* x, const void* w, void* y, int B, int T, int C, int K,
+                               int pad_left, int pad_right, gconv_dtype dtype, gconv_path path,
+                               void* stream) {
   Conv1d p;
   gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
   if (st != GCONV_OK) return st;
   if (B > 0 && (x == nullptr || w == nullptr || y == nullptr)) return GCONV_ERR_INVALID_ARG;
+  const int kernel = conv1d_choose_kernel(p, path, x, w, y, &st);
+  if (kernel < 0) return st;
   if (B == 0) return GCONV_OK;
-  return cuda_status(launch_dwconv1d_fwd(p, x, w, y, false, pad_left, T, p.T_out,
+  return cuda_status(launch_dwconv1d_fwd(p, x, w, y, false, pad_left, T, p.T_out, kernel,
                                          (cudaStream_t)stream));
+}
+
+gconv_status dwconv1d_fwd(const void* x, const void* w, void* y, int B, int T, int C, int K,
+                          int pad_left, int pad_right, gconv_dtype dtype, void* stream) {
+  return dwconv1d_fwd_path(x, w, y, B, T, C, K, pad_left, pad_right, dtype, GCONV_PATH_AUTO,
+                           stream);
+}
+
+gconv_status dwconv1d_bwd_data_path(const void* dy, const void* w, void* dx, int B, int T, int C,
+                                    int K, int pad_left, int pad_right, gconv_dtype dtype,
+                                    gconv_path path, void* stream) {
+  Conv1d p;
+  gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
+  if (st != GCONV_OK) return st;
+  if (B > 0 && (dy == nullptr || w == nullptr || dx == nullptr)) return GCONV_ERR_INVALID_ARG;
+  const int kernel = conv1d_choose_kernel(p, path, dy, w, dx, &st);
+  if (kernel < 0) return st;
+  if (B == 0) return GCONV_OK;
+  // dx = forward of dy (T_out steps) with the reversed filter and left pad K-1-pad_left
+  return cuda_status(launch_dwconv1d_fwd(p, dy, w, dx, true, K - 1 - pad_left, p.T_out, T,
+                                         kernel, (cudaStream_t)stream));
 }
 
 gconv_status dwconv1d_bwd_data(const void* dy, const void* w, void* dx, int B, int T, int C,
                                int K, int pad_left, int pad_right, gconv_dtype dtype,
                                void* stream) {
+  return dwconv1d_bwd_data_path(dy, w, dx, B, T, C, K, pad_left, pad_right, dtype,
+                                GCONV_PATH_AUTO, stream);
+}
+
+int dwconv1d_select_path(int B, int T, int C, int K, int pad_left, int pad_right,
+                         gconv_dtype dtype, gconv_path path) {
   Conv1d p;
   gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
-  if (st != GCONV_OK) return st;
-  if (B > 0 && (dy == nullptr || w == nullptr || dx == nullptr)) return GCONV_ERR_INVALID_ARG;
-  if (B == 0) return GCONV_OK;
-  // dx = forward of dy (T_out steps) with the reversed filter and left pad K-1-pad_left
-  return cuda_status(launch_dwconv1d_fwd(p, dy, w, dx, true, K - 1 - pad_left, p.T_out, T,
-                                         (cudaStream_t)stream));
+  if (st != GCONV_OK) return -(int)st;
+  const int k = conv1d_choose_kernel(p, path, nullptr, nullptr, nullptr, &st);
+  return k < 0 ? -(int)st : k;
 }
 
 size_t dwconv1d_bwd_weight_workspace_size(int B, int T, int C, int K, int pad_left,

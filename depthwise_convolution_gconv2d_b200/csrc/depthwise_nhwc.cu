@@ -193,8 +193,7 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
                      const T* __restrict__ bias, const Dw3Params P, unsigned int* err) {
   using namespace ptx;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  unsigned char* smem = ptx::align_smem(smem_raw, 128u);
   // output staging after the input ring: compute warp g owns [BH][DW3_R][64 ch], the box of
   // its own TMA store
   unsigned char* ostage = smem + (size_t)P.stages * P.stage_bytes;

@@ -13,17 +13,18 @@
 // stream their inputs with TMA through shared-memory rings filled by a producer warp (the
 // tensor map's zero fill outside [0, T) is the padding), so bytes in flight come from the copy
 // engine rather than from thread count:
-//  * fwd / dgrad: persistent CTAs walk a contiguous chunk of [128 steps x 64 channels] output
-//    tiles; a box of 128 + K - 1 input steps per tile. A thread owns a channel pair and 16
-//    consecutive outputs; its K filter taps stay in registers (reloaded only when the chunk
-//    moves to the next channel tile) and each staged input step is read once from shared
-//    memory and applied to every output it touches (packed fp32x2 FMA, loop over the kernel
-//    size fully unrolled).
+//  * fwd / dgrad: persistent CTAs walk a contiguous chunk of [112 steps x 64 channels] output
+//    tiles; a box of 112 + K - 1 input steps per tile. A thread owns a channel pair and 16
+//    consecutive outputs; all K filter taps stay in registers as fp32 pairs (reloaded only when
+//    the chunk moves to the next channel tile) and each staged input step is read once from
+//    shared memory and applied to every output it touches (packed fp32x2 FMA, loop over the
+//    kernel size fully unrolled, one pass over the filter).
 //  * wgrad: a block owns 64 channels and a fixed slice of one batch's steps and streams
-//    (dy, x) box pairs of 128 steps through its ring; a thread keeps K fp32-pair partial sums
+//    (dy, x) box pairs of 112 steps through its ring; a thread keeps K fp32-pair partial sums
 //    for its channel pair over 16-step strips; strips are summed in a fixed order in shared
 //    memory and the per-slice partials go to the caller's workspace. A second kernel sums the
 //    slices in a fixed order. No float atomics: bitwise reproducible.
+// Both run 8-warp CTAs, two per SM, at up to 128 registers a thread.
 // Generic kernels cover every other shape, one thread per output (fwd/dgrad) or one warp per
 // (c, k) with a fixed-order shuffle reduction (wgrad).
 #include <type_traits>
@@ -75,13 +76,12 @@ struct Coord1d {
 };
 
 template <typename T, int K, bool FLIP>
-__global__ void __maxnreg__(104)
+__global__ void __maxnreg__(128)
     dwconv1d_fwd_kernel(const __grid_constant__ CUtensorMap tmx, const T* __restrict__ w,
                         T* __restrict__ y, const Ring1d P, unsigned int* err) {
   using namespace ptx;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  unsigned char* smem = ptx::align_smem(smem_raw, 128u);
   unsigned long long* full =
       reinterpret_cast<unsigned long long*>(smem + (size_t)P.stages * P.stage_bytes);
   unsigned long long* empty = full + MAX_STAGES;
@@ -125,9 +125,8 @@ __global__ void __maxnreg__(104)
                   0u);
     }
   } else {
-    // taps of the current channel tile as fp32 pairs [K][CP] after the ring
-    float2* wsm = reinterpret_cast<float2*>(empty + MAX_STAGES + 2);
-    const int cp = lane, strip = warp - 1, ctid = threadIdx.x - 32;
+    const int cp = lane, strip = warp - 1;
+    float2 wk[K];                                   // the pair's taps, fp32, in registers
     Coord1d c;
     c.set(P, t_begin);
     int prev_ct = -1;
@@ -137,46 +136,32 @@ __global__ void __maxnreg__(104)
       const int ch = c.ct * CH + 2 * cp;
       if (c.ct != prev_ct) {
         prev_ct = c.ct;
-        asm volatile("bar.sync 1, %0;" ::"r"(RCOMPUTE));   // compute warps only
-        for (int i = ctid; i < K * CP; i += RCOMPUTE) {
-          const int k = i / CP, pp = i % CP;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
           const int kk = FLIP ? K - 1 - k : k;
-          const int cc = c.ct * CH + 2 * pp;
-          wsm[i] = cc < P.C ? make_float2(Elem<T>::to_f32(w[(long long)cc * K + kk]),
-                                          Elem<T>::to_f32(w[(long long)(cc + 1) * K + kk]))
-                            : make_float2(0.f, 0.f);
+          wk[k] = ch < P.C ? make_float2(Elem<T>::to_f32(w[(long long)ch * K + kk]),
+                                         Elem<T>::to_f32(w[(long long)(ch + 1) * K + kk]))
+                           : make_float2(0.f, 0.f);
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(RCOMPUTE));
       }
       bool got = mbar_try_wait(&full[s], ph);
       if (!got) got = mbar_wait(&full[s], ph, abort_flag, err, 32u);
       if (!__all_sync(0xffffffffu, got)) break;
-      // staged box: row r (input step tt*TB - pl + r) holds 64 channels = 32 packed pairs
+      // staged box: row r (input step tt*TB - pl + r) holds 64 channels = 32 packed pairs;
+      // each input step is read and widened once and applied to every output it touches
       const uint32_t* xr =
           reinterpret_cast<const uint32_t*>(smem + (size_t)s * P.stage_bytes) + strip * TS * CP +
           cp;
       float2 acc[TS];
 #pragma unroll
       for (int i = 0; i < TS; ++i) acc[i] = make_float2(0.f, 0.f);
-      // the filter in passes of at most KC taps, so only KC taps are live in registers
-      constexpr int KC = K > 16 ? (K + 2) / 3 : K;
 #pragma unroll
-      for (int k0 = 0; k0 < K; k0 += KC) {
-        const int kn = K - k0 < KC ? K - k0 : KC;
-        float2 wk[KC];
+      for (int j = 0; j < TS + K - 1; ++j) {
+        const float2 xv = unpack2<T>(xr[j * CP]);
 #pragma unroll
-        for (int k = 0; k < KC; ++k)
-          if (k < kn) wk[k] = wsm[(k0 + k) * CP + cp];
-#pragma unroll
-        for (int j = 0; j < TS + KC - 1; ++j) {
-          if (j < TS + kn - 1) {
-            const float2 xv = unpack2<T>(xr[(k0 + j) * CP]);
-#pragma unroll
-            for (int i = 0; i < TS; ++i) {
-              const int k = j - i;
-              if (k >= 0 && k < kn) acc[i] = ffma2(wk[k], xv, acc[i]);
-            }
-          }
+        for (int i = 0; i < TS; ++i) {
+          const int k = j - i;
+          if (k >= 0 && k < K) acc[i] = ffma2(wk[k], xv, acc[i]);
         }
       }
       __syncwarp();
@@ -199,7 +184,7 @@ __global__ void __maxnreg__(104)
   __syncthreads();
 }
 
-constexpr int WTS = 8;             // weight gradient: steps per thread strip
+constexpr int WTS = 16;            // weight gradient: steps per thread strip
 constexpr int WTB = WTS * RSTRIPS; // steps per sub-tile
 
 struct WgradRing {
@@ -208,14 +193,13 @@ struct WgradRing {
 };
 
 template <typename T, int K>
-__global__ void __maxnreg__(104)
+__global__ void __maxnreg__(128)
     dwconv1d_wgrad_kernel(const __grid_constant__ CUtensorMap tmx,
                           const __grid_constant__ CUtensorMap tmdy, float* __restrict__ partial,
                           const WgradRing P, unsigned int* err) {
   using namespace ptx;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  unsigned char* smem = ptx::align_smem(smem_raw, 128u);
   unsigned long long* full =
       reinterpret_cast<unsigned long long*>(smem + (size_t)P.stages * P.stage_bytes);
   unsigned long long* empty = full + MAX_STAGES;
@@ -412,8 +396,7 @@ cudaError_t fwd_vec(const Conv1d& p, const T* x, const T* w, T* y, int B, int T_
   P.tx_bytes = (unsigned int)(TBF + K - 1) * CH * 2;
   P.stage_bytes = (P.tx_bytes + 127u) & ~127u;
   P.stages = 4;
-  const size_t smem = 128 + (size_t)P.stages * P.stage_bytes + 2 * MAX_STAGES * 8 + 16 +
-                      (size_t)K * CP * sizeof(float2);
+  const size_t smem = 128 + (size_t)P.stages * P.stage_bytes + 2 * MAX_STAGES * 8 + 16;
   CUtensorMap tm;
   if (!make_tensor_map_btc(&tm, p.dtype, x, C, T_in, B, TBF + K - 1)) return cudaErrorInvalidValue;
   static std::atomic<unsigned int> configured{0};
@@ -546,12 +529,41 @@ bool conv1d_vector_supported(const Conv1d& p) {
          (t_max + TB - 1) / TB <= 65535;   // grid.z = B, grid.y = step tiles
 }
 
+int conv1d_choose_kernel(const Conv1d& p, int path, const void* x, const void* w, const void* y,
+                         gconv_status* why) {
+  *why = GCONV_OK;
+  const bool query = (x == nullptr && w == nullptr && y == nullptr);
+  const bool ring_ok = conv1d_vector_supported(p);
+  const bool ring_al = query || (aligned16(x) && aligned16(y));
+  const bool tc_ok = conv1d_tc_supported(p);
+  const bool tc_al = query || (aligned16(x) && aligned16(y) && aligned16(w));
+  switch (path) {
+    case GCONV_PATH_GENERIC:
+      return GCONV_KERNEL_CONV1D_GENERIC;
+    case GCONV_PATH_DIRECT:
+      return (ring_ok && ring_al) ? GCONV_KERNEL_CONV1D_RING : GCONV_KERNEL_CONV1D_GENERIC;
+    case GCONV_PATH_IGEMM:
+      if (!tc_ok) { *why = GCONV_ERR_UNSUPPORTED; return -1; }
+      if (!tc_al) { *why = GCONV_ERR_MISALIGNED; return -1; }
+      return GCONV_KERNEL_CONV1D_TC;
+    case GCONV_PATH_AUTO:
+      // the tensor-core kernel is the faster of the two (Conformer layer: 22.5 vs 30.6 us);
+      // the CUDA-core ring kernel takes C % 16 == 8 and the generic kernel the rest
+      if (tc_ok && tc_al) return GCONV_KERNEL_CONV1D_TC;
+      if (ring_ok && ring_al) return GCONV_KERNEL_CONV1D_RING;
+      return GCONV_KERNEL_CONV1D_GENERIC;
+    default:
+      *why = GCONV_ERR_INVALID_ARG;
+      return -1;
+  }
+}
+
 cudaError_t launch_dwconv1d_fwd(const Conv1d& p, const void* x, const void* w, void* y, bool flip,
-                                int pad_left, int T_in, int T_out, cudaStream_t s) {
+                                int pad_left, int T_in, int T_out, int kernel, cudaStream_t s) {
   if (p.B == 0) return cudaSuccess;
-  if (conv1d_tc_supported(p) && aligned16(x) && aligned16(y) && aligned16(w))
+  if (kernel == GCONV_KERNEL_CONV1D_TC)
     return launch_dwconv1d_tc(p, x, w, y, flip, pad_left, T_in, T_out, s);
-  const bool vec = conv1d_vector_supported(p) && aligned16(x) && aligned16(y);
+  const bool vec = kernel == GCONV_KERNEL_CONV1D_RING;
   switch (p.dtype) {
     case GCONV_F32: return fwd_any_dtype<float>(p, x, w, y, flip, pad_left, T_in, T_out, false, s);
     case GCONV_F16: return fwd_any_dtype<__half>(p, x, w, y, flip, pad_left, T_in, T_out, vec, s);

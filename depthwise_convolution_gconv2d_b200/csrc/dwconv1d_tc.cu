@@ -130,8 +130,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   using namespace ptx;
   constexpr TcLayout L = tc_layout(KS);
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem = ptx::align_smem(smem_raw, 1024u);
   unsigned long long* bars = reinterpret_cast<unsigned long long*>(smem + L.total);
   unsigned long long* xs_full = bars;                          // producer: tx bytes
   unsigned long long* xs_empty = bars + 1;                     // 4 transposer warps

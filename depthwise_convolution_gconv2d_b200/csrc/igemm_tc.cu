@@ -110,8 +110,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const __grid_constant__ CUtensorMap tma_w, const T* __restrict__ bias,
                     T* __restrict__ y, const IgemmParams P, unsigned int* err) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem = ptx::align_smem(smem_raw, 1024u);
   unsigned char* a_base = smem;
   unsigned char* b_base = smem + (size_t)P.stages * P.a_stage;
   unsigned long long* bars =
@@ -314,8 +313,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       const __grid_constant__ CUtensorMap tma_w, const T* __restrict__ bias,
                       T* __restrict__ y, const HaloParams P, unsigned int* err) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem = ptx::align_smem(smem_raw, 1024u);
   unsigned char* a_base = smem;
   unsigned char* b_base = smem + (size_t)P.stages * P.a_stage;
   unsigned long long* bars =
@@ -541,8 +539,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      const __grid_constant__ CUtensorMap tma_w, const T* __restrict__ bias,
                      T* __restrict__ y, const RowParams P, unsigned int* err) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem = ptx::align_smem(smem_raw, 1024u);
   unsigned char* a_base = smem;
   unsigned char* b_base = smem + (size_t)P.a_stages * P.a_stage;
   unsigned long long* bars =
@@ -793,8 +790,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       const __grid_constant__ CUtensorMap tma_w, const T* __restrict__ bias,
                       T* __restrict__ y, const RowTParams P, unsigned int* err) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem = ptx::align_smem(smem_raw, 1024u);
   unsigned char* x_base = smem;
   unsigned char* w_base = smem + (size_t)P.x_stages * P.x_stage;
   unsigned long long* bars =

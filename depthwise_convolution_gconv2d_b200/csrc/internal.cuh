@@ -107,8 +107,13 @@ cudaError_t launch_igemm_nchw(const Conv2d& p, const void* x, const void* w, con
                               void* y, void* workspace, cudaStream_t s);
 
 bool conv1d_vector_supported(const Conv1d& p);
+// Kernel (GCONV_KERNEL_CONV1D_*) for a forward / data-gradient call under `path`; x, w, y null
+// = a query that assumes aligned pointers. -1 with *why set when the forced family cannot run.
+int conv1d_choose_kernel(const Conv1d& p, int path, const void* x, const void* w, const void* y,
+                         gconv_status* why);
 cudaError_t launch_dwconv1d_fwd(const Conv1d& p, const void* x, const void* w, void* y,
-                                bool flip, int pad_left, int T_in, int T_out, cudaStream_t s);
+                                bool flip, int pad_left, int T_in, int T_out, int kernel,
+                                cudaStream_t s);
 // Tensor-core forward / data gradient: 16-bit data, C % 8 == 0, K <= 49, 16-byte aligned x, w, y.
 bool conv1d_tc_supported(const Conv1d& p);
 cudaError_t launch_dwconv1d_tc(const Conv1d& p, const void* x, const void* w, void* y, bool flip,

@@ -15,6 +15,15 @@ __device__ __forceinline__ unsigned int smem_u32(const void* p) {
   return (unsigned int)__cvta_generic_to_shared(p);
 }
 
+// `base` advanced to the next multiple of `align` (a power of two) in the shared window. The
+// offset is computed from the 32-bit shared address and added to the shared-memory pointer, so
+// the result stays a shared-space pointer for the compiler (loads through it are shared loads
+// with immediate offsets).
+__device__ __forceinline__ unsigned char* align_smem(unsigned char* base, unsigned int align) {
+  const unsigned int a = smem_u32(base);
+  return base + (((a + align - 1u) & ~(align - 1u)) - a);
+}
+
 __device__ __forceinline__ unsigned long long globaltimer() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -93,7 +93,12 @@ typedef enum {
   GCONV_KERNEL_DIRECT_GENERIC = 1,    /* one thread per output, fp32 FMA, any problem */
   GCONV_KERNEL_DEPTHWISE_NHWC = 2,    /* 8-channel vectors, sliding window, 16-bit NHWC */
   GCONV_KERNEL_IGEMM_TC = 3,          /* tcgen05 implicit GEMM, NHWC */
-  GCONV_KERNEL_IGEMM_TC_NCHW = 4      /* NCHW -> NHWC staging in the workspace + tcgen05 */
+  GCONV_KERNEL_IGEMM_TC_NCHW = 4,     /* NCHW -> NHWC staging in the workspace + tcgen05 */
+  GCONV_KERNEL_CONV1D_GENERIC = 5,    /* dwconv1d: one thread per output, fp32 FMA, any problem */
+  GCONV_KERNEL_CONV1D_RING = 6,       /* dwconv1d: CUDA-core TMA-ring kernel; 16-bit, C % 8 == 0,
+                                         K in {3, 5, 7, 9, 15, 31} */
+  GCONV_KERNEL_CONV1D_TC = 7          /* dwconv1d: tcgen05 banded product; 16-bit, C % 16 == 0,
+                                         K <= 49 */
 } gconv_kernel;
 
 /* Bytes of workspace gconv2d_fwd needs for this problem under `path` (0 if none; also 0 for
@@ -136,6 +141,24 @@ gconv_status dwconv1d_fwd(const void* x, const void* w, void* y, int B, int T, i
 gconv_status dwconv1d_bwd_data(const void* dy, const void* w, void* dx, int B, int T, int C,
                                int K, int pad_left, int pad_right, gconv_dtype dtype,
                                void* stream);
+
+/* dwconv1d_fwd / dwconv1d_bwd_data with an explicit kernel family: DIRECT forces the
+ * CUDA-core ring kernel (else the generic kernel), IGEMM the tensor-core kernel, GENERIC the
+ * generic kernel; AUTO is what dwconv1d_fwd / dwconv1d_bwd_data run. The pages define one
+ * operation; the families are this library's kernels for it (for path comparisons and tests).
+ * Errors as dwconv1d_fwd, plus UNSUPPORTED (IGEMM on a problem it cannot run: 32-bit data,
+ * C % 16 != 0, K > 49) and MISALIGNED (IGEMM with x, w or y not 16-byte aligned). */
+gconv_status dwconv1d_fwd_path(const void* x, const void* w, void* y, int B, int T, int C, int K,
+                               int pad_left, int pad_right, gconv_dtype dtype, gconv_path path,
+                               void* stream);
+gconv_status dwconv1d_bwd_data_path(const void* dy, const void* w, void* dx, int B, int T, int C,
+                                    int K, int pad_left, int pad_right, gconv_dtype dtype,
+                                    gconv_path path, void* stream);
+
+/* The gconv_kernel (GCONV_KERNEL_CONV1D_*) that dwconv1d_fwd_path / dwconv1d_bwd_data_path
+ * would run, assuming 16-byte aligned pointers; a negative gconv_status if it would fail. */
+int dwconv1d_select_path(int B, int T, int C, int K, int pad_left, int pad_right,
+                         gconv_dtype dtype, gconv_path path);
 
 /* Bytes of workspace dwconv1d_bwd_weight needs (fp32 partial sums of fixed slices of B*T_out;
  * 0 for invalid arguments). */

@@ -115,3 +115,30 @@ def test_wgrad_workspace_query(lib):
     assert n > 0 and n % 4 == 0
     assert lib.dwconv1d_bwd_weight_workspace_size(8, 2048, 512, 31, 15, 15, 0) == 0   # fp32: generic
     assert lib.dwconv1d_bwd_weight_workspace_size(8, 10, 512, 31, 0, 0, 2) == 0       # invalid
+
+
+def test_conv1d_path_selection(lib):
+    """dwconv1d_select_path: the tensor-core kernel (7) for 16-bit data with C % 16 == 0 and
+    K <= 49, else the CUDA-core ring kernel (6) where it is instantiated, else the generic
+    kernel (5); a forced family that cannot run gives -UNSUPPORTED."""
+    BF16, F32 = 2, 0
+    sel = lambda B, T, C, K, pl, pr, dt, path: lib.dwconv1d_select_path(B, T, C, K, pl, pr, dt,
+                                                                        path)
+    conformer = (8, 2048, 512, 31, 15, 15, BF16)
+    assert sel(*conformer, 0) == 7
+    assert sel(*conformer, 1) == 6
+    assert sel(*conformer, 2) == 7
+    assert sel(*conformer, 3) == 5
+    assert sel(8, 2048, 512, 31, 15, 15, F32, 0) == 5
+    assert sel(8, 2048, 512, 31, 15, 15, F32, 2) == -2          # UNSUPPORTED
+    assert sel(2, 300, 72, 31, 15, 15, BF16, 0) == 6            # C % 16 == 8: ring only
+    assert sel(2, 300, 72, 31, 15, 15, BF16, 2) == -2
+    assert sel(1, 500, 16, 17, 8, 8, BF16, 0) == 7              # K = 17: no ring instantiation
+    assert sel(1, 500, 16, 17, 8, 8, BF16, 1) == 5
+    assert sel(1, 500, 16, 50, 25, 24, BF16, 0) == 5            # K = 50: beyond the TC kernel
+    assert sel(1, 500, 16, 50, 25, 24, BF16, 2) == -2
+    assert sel(1, 8, 16, 31, 0, 0, BF16, 0) == -1               # T_out < 1: INVALID_ARG
+    assert sel(*conformer, 9) == -1                             # unknown path
+    # a forced path that cannot run is rejected before anything is launched
+    assert lib.dwconv1d_fwd_path(None, None, None, 0, 8, 16, 3, 1, 1, F32, 2, None) == 2
+    assert lib.dwconv1d_bwd_data_path(None, None, None, 0, 8, 16, 3, 1, 1, BF16, 9, None) == 1

@@ -16,11 +16,11 @@ from _util import assert_close, to_dev, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def gpu_all(inp):
+def gpu_all(inp, path=gb.PATH_AUTO):
     p = inp.problem
     x, w, dy = (to_dev(a, p.dtype) for a in (inp.x, inp.w, inp.dy))
-    y = gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right)
-    dx = gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right)
+    y = gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right, path=path)
+    dx = gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right, path=path)
     dw = gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right)
     torch.cuda.synchronize()
     return to_f64(y), to_f64(dx), to_f64(dw)
@@ -34,15 +34,24 @@ def oracle_all(inp):
             oracle.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right))
 
 
-def check(p, workload, dist="normal"):
+def check(p, workload, dist="normal", path=gb.PATH_AUTO):
     inp = wl.make_dwconv1d_inputs(p, workload, dist)
-    for name, got, ref in zip(("fwd", "dgrad", "wgrad"), gpu_all(inp), oracle_all(inp)):
+    for name, got, ref in zip(("fwd", "dgrad", "wgrad"), gpu_all(inp, path), oracle_all(inp)):
         assert_close(got, ref, p.dtype, f"{name} {p}")
 
 
+def kernel_of(p, path=gb.PATH_AUTO):
+    return gb.dwconv1d_select_path(p.B, p.T, p.C, p.K, p.pad_left, p.pad_right, p.dtype, path)
+
+
 @pytest.mark.parametrize("causal", [False, True])
-def test_conformer_full_size(causal):
-    check(wl.conformer_dw1d(causal), 3)
+@pytest.mark.parametrize("path", [gb.PATH_AUTO, gb.PATH_DIRECT])
+def test_conformer_full_size(causal, path):
+    """The Conformer layer in full on the path the library picks (the tensor-core kernel) and
+    forced onto the CUDA-core ring kernel."""
+    p = wl.conformer_dw1d(causal)
+    assert kernel_of(p) == 7 and kernel_of(p, gb.PATH_DIRECT) == 6
+    check(p, 3, path=path)
 
 
 SMALL = [
@@ -82,7 +91,19 @@ TC_CASES = [
 @pytest.mark.parametrize("case", TC_CASES)
 @pytest.mark.parametrize("dtype", [wl.BF16, wl.F16])
 def test_tensor_core_edges(case, dtype):
-    check(wl.Dwconv1dProblem(*case, dtype), 33)
+    p = wl.Dwconv1dProblem(*case, dtype)
+    tc = p.K <= 49
+    assert kernel_of(p, gb.PATH_IGEMM) == (7 if tc else -2)      # -2: UNSUPPORTED
+    check(p, 33, path=gb.PATH_IGEMM if tc else gb.PATH_AUTO)
+
+
+@pytest.mark.parametrize("case", TC_CASES[:4])
+def test_ring_and_generic_paths_agree_with_oracle(case):
+    """The same problems forced onto the CUDA-core kernels (ring where instantiated, generic
+    otherwise) and onto the generic kernel."""
+    p = wl.Dwconv1dProblem(*case, wl.BF16)
+    check(p, 34, path=gb.PATH_DIRECT)
+    check(p, 34, path=gb.PATH_GENERIC)
 
 
 @pytest.mark.parametrize("case", SMALL)
@@ -92,13 +113,16 @@ def test_small_shapes(case, dtype):
 
 
 @pytest.mark.parametrize("case", SMALL[:8] + TC_CASES[:3])
-def test_integer_valued_bit_exact_fwd_dgrad(case):
-    """Integers in [-2, 2]: every partial sum is exact in fp32 and the result (|.| <= 124)
+@pytest.mark.parametrize("path", [gb.PATH_AUTO, gb.PATH_DIRECT, gb.PATH_IGEMM])
+def test_integer_valued_bit_exact_fwd_dgrad(case, path):
+    """Integers in [-2, 2]: every partial sum is exact in fp32 and the result (|.| <= 132)
     is exact in bf16, so any summation order gives the oracle's value bit for bit."""
     p = wl.Dwconv1dProblem(*case, wl.BF16)
+    if path == gb.PATH_IGEMM and kernel_of(p, path) != 7:
+        pytest.skip("not a tensor-core problem")
     inp = wl.make_dwconv1d_inputs(p, 31, "int")
     inp.w = wl.to_storage(np.random.default_rng(5).integers(-2, 3, (p.C, p.K)), wl.BF16)
-    (y, dx, _), (ry, rdx, _) = gpu_all(inp), oracle_all(inp)
+    (y, dx, _), (ry, rdx, _) = gpu_all(inp, path), oracle_all(inp)
     assert np.array_equal(y, ry)
     assert np.array_equal(dx, rdx)
 
