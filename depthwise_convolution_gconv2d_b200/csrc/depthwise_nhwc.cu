@@ -182,7 +182,7 @@ constexpr int DW3_R = 4;                   // output columns per thread
 constexpr int DW3_NG = 7;                  // column groups (one compute warp each)
 constexpr int DW3_BW = DW3_R * DW3_NG;     // output columns per tile
 constexpr int DW3_THREADS = 32 + 32 * DW3_NG;
-template <int S> constexpr int DW3_IW() { return (DW3_BW - 1) * S + 3; }   // input box columns
+template <int S> __host__ __device__ constexpr int DW3_IW() { return (DW3_BW - 1) * S + 3; }
 
 // Warp 0 lane 0 is the TMA producer; warps 1.. compute. Stage s is handed over through
 // full[s] (TMA transaction bytes) and empty[s] (one arrival per compute warp).

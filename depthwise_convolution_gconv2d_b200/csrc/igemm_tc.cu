@@ -296,6 +296,9 @@ struct HaloParams {
   unsigned int a_region, a_stage, b_tile, b_stage, tx_bytes;
   unsigned int idesc, swz, sbo, row_bytes, tmem_cols;
   int out_nchw;
+  int tma_out;                 // NHWC output through shared memory and TMA stores
+  unsigned int o_bytes;        // that staging, two buffers of BN/64 blocks of [128 rows][64 ch]
+                               // with the 128-byte swizzle
 };
 
 __device__ __forceinline__ void halo_decode(const HaloParams& P, int t, int& j, int& nt, int& n,
@@ -307,17 +310,83 @@ __device__ __forceinline__ void halo_decode(const HaloParams& P, int t, int& j, 
   n = mt / P.tiles_h;
 }
 
+// One halo stage's MMAs with every descriptor built before the first is issued, so the
+// issuing thread sends KWS*KH*KS MMAs back to back (rebuilding descriptors between MMAs costs
+// over a hundred cycles each, measured). The dispatchers below return false for shapes without
+// an instantiation (more than 18 MMAs per stage), which take the loop in the kernel.
+template <int KH, int KWS, int KS>
+__device__ __forceinline__ void halo_issue_fixed(unsigned int d, unsigned long long ad0,
+                                                 unsigned long long bd0,
+                                                 unsigned long long kh_step,
+                                                 unsigned long long kw_step,
+                                                 unsigned long long bt_step, unsigned int idesc,
+                                                 bool first) {
+  unsigned long long ad[KWS * KH * KS], bd[KWS * KH * KS];
+#pragma unroll
+  for (int kwi = 0; kwi < KWS; ++kwi)
+#pragma unroll
+    for (int kh = 0; kh < KH; ++kh)
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        const int i = (kwi * KH + kh) * KS + k;
+        ad[i] = ad0 + kwi * kw_step + kh * kh_step + 2 * k;
+        bd[i] = bd0 + (kwi * KH + kh) * bt_step + 2 * k;
+      }
+#pragma unroll
+  for (int i = 0; i < KWS * KH * KS; ++i)
+    umma_f16(d, ad[i], bd[i], idesc, (first && i == 0) ? 0u : 1u);
+}
+
+template <int KH, int KS>
+__device__ __forceinline__ bool halo_issue_kws(int kws, unsigned int d, unsigned long long ad0,
+                                               unsigned long long bd0, unsigned long long kh_step,
+                                               unsigned long long kw_step,
+                                               unsigned long long bt_step, unsigned int idesc,
+                                               bool first) {
+  // at most 18 MMAs per stage keep their descriptors in registers
+  if constexpr (KH * KS <= 18) {
+    if (kws == 1) {
+      halo_issue_fixed<KH, 1, KS>(d, ad0, bd0, kh_step, kw_step, bt_step, idesc, first);
+      return true;
+    }
+  }
+  if constexpr (KH * KH * KS <= 18) {
+    if (kws == KH) {
+      halo_issue_fixed<KH, KH, KS>(d, ad0, bd0, kh_step, kw_step, bt_step, idesc, first);
+      return true;
+    }
+  }
+  return false;
+}
+
+template <int KS>
+__device__ __forceinline__ bool halo_issue_kh(int kh, int kws, unsigned int d,
+                                              unsigned long long ad0, unsigned long long bd0,
+                                              unsigned long long kh_step,
+                                              unsigned long long kw_step,
+                                              unsigned long long bt_step, unsigned int idesc,
+                                              bool first) {
+  switch (kh) {
+    case 1: return halo_issue_kws<1, KS>(kws, d, ad0, bd0, kh_step, kw_step, bt_step, idesc, first);
+    case 3: return halo_issue_kws<3, KS>(kws, d, ad0, bd0, kh_step, kw_step, bt_step, idesc, first);
+    case 5: return halo_issue_kws<5, KS>(kws, d, ad0, bd0, kh_step, kw_step, bt_step, idesc, first);
+    case 7: return halo_issue_kws<7, KS>(kws, d, ad0, bd0, kh_step, kw_step, bt_step, idesc, first);
+    default: return false;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     igemm_halo_kernel(const __grid_constant__ CUtensorMap tma_x,
-                      const __grid_constant__ CUtensorMap tma_w, const T* __restrict__ bias,
+                      const __grid_constant__ CUtensorMap tma_w,
+                      const __grid_constant__ CUtensorMap tma_y, const T* __restrict__ bias,
                       T* __restrict__ y, const HaloParams P, unsigned int* err) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = ptx::align_smem(smem_raw, 1024u);
   unsigned char* a_base = smem;
   unsigned char* b_base = smem + (size_t)P.stages * P.a_stage;
-  unsigned long long* bars =
-      reinterpret_cast<unsigned long long*>(b_base + (size_t)P.stages * P.b_stage);
+  unsigned char* o_base = b_base + (size_t)P.stages * P.b_stage;   // output staging
+  unsigned long long* bars = reinterpret_cast<unsigned long long*>(o_base + P.o_bytes);
   unsigned long long* full = bars;
   unsigned long long* empty = bars + MAX_STAGES;
   unsigned long long* tfull = bars + 2 * MAX_STAGES;
@@ -420,16 +489,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             const unsigned long long ad0 = a_desc0 + (((unsigned long long)s * P.a_stage) >> 4);
             const unsigned long long bd0 = b_desc0 + (((unsigned long long)s * P.b_stage) >> 4);
-            for (int kwi = 0; kwi < P.KWS; ++kwi) {
-              for (int kh = 0; kh < P.kH; ++kh) {
-                const unsigned long long ad = ad0 + kwi * kw_step + kh * kh_step;
-                const unsigned long long bd = bd0 + (kwi * P.kH + kh) * bt_step;
-                const unsigned int acc0 = (cb | kg | kwi | kh) == 0 ? 0u : 1u;
-                umma_f16(d, ad, bd, P.idesc, acc0);
-                if (ksteps > 1) umma_f16(d, ad + 2, bd + 2, P.idesc, 1u);
-                if (ksteps > 2) {
-                  umma_f16(d, ad + 4, bd + 4, P.idesc, 1u);
-                  umma_f16(d, ad + 6, bd + 6, P.idesc, 1u);
+            const bool first = (cb | kg) == 0;
+            bool fixed = false;
+            if (ksteps == 1)
+              fixed = halo_issue_kh<1>(P.kH, P.KWS, d, ad0, bd0, kh_step, kw_step, bt_step,
+                                       P.idesc, first);
+            else if (ksteps == 2)
+              fixed = halo_issue_kh<2>(P.kH, P.KWS, d, ad0, bd0, kh_step, kw_step, bt_step,
+                                       P.idesc, first);
+            else if (ksteps == 4)
+              fixed = halo_issue_kh<4>(P.kH, P.KWS, d, ad0, bd0, kh_step, kw_step, bt_step,
+                                       P.idesc, first);
+            if (!fixed) {
+              for (int kwi = 0; kwi < P.KWS; ++kwi) {
+                for (int kh = 0; kh < P.kH; ++kh) {
+                  const unsigned long long ad = ad0 + kwi * kw_step + kh * kh_step;
+                  const unsigned long long bd = bd0 + (kwi * P.kH + kh) * bt_step;
+                  const unsigned int acc0 = (first && (kwi | kh) == 0) ? 0u : 1u;
+                  umma_f16(d, ad, bd, P.idesc, acc0);
+                  for (int k = 1; k < ksteps; ++k)
+                    umma_f16(d, ad + 2 * k, bd + 2 * k, P.idesc, 1u);
                 }
               }
             }
@@ -455,13 +534,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int hl = row / P.BW, wl = row - hl * P.BW;
-    int acc = 0;
+    const bool store_thread = (warp == 2 && lane == 0);
+    int acc = 0, ob = 0;
     unsigned int aph = 0;
     for (int t = blockIdx.x; t < P.num_tiles; t += gridDim.x) {
       int j, nt, n, th;
       halo_decode(P, t, j, nt, n, th);
       const bool got = mbar_wait(&tfull[acc], aph, abort_flag, err, ERR_WAIT_EPILOGUE);
-      if (!__all_sync(0xffffffffu, got)) break;
+      unsigned char* obuf = o_base + (size_t)ob * (P.o_bytes / 2);
+      if (P.tma_out) {
+        if (store_thread) bulk_wait_read1();       // the store from two tiles back has read it
+        if (!named_all(1, 128, got)) break;        // the four warps leave together
+      } else if (!__all_sync(0xffffffffu, got)) {
+        break;
+      }
       tc_fence_after();
       const int ho = th * P.BH + hl, wo = wl;
       const bool valid = hl < P.BH && ho < P.Ho;
@@ -476,15 +562,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         else
           tmem_ld16(taddr + c, r);
         tmem_ld_wait();
-        if (valid) epilogue_store<T>(P, y, bias, r, ncols, n, ho, wo, co0 + c);
+        if (P.tma_out) {
+          // 32 channels -> 4 16-byte chunks of this row's 128-byte line in 64-channel block
+          // c / 64; chunk k of row r sits at chunk k ^ (r % 8) (the 128-byte swizzle)
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          if (bias) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] += Elem<T>::to_f32(bias[co0 + c + i]);
+          }
+          unsigned char* line = obuf + (size_t)(c >> 6) * (128 * 128) + (size_t)row * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 u;
+            u.x = pack2<T>(make_float2(v[8 * q + 0], v[8 * q + 1]));
+            u.y = pack2<T>(make_float2(v[8 * q + 2], v[8 * q + 3]));
+            u.z = pack2<T>(make_float2(v[8 * q + 4], v[8 * q + 5]));
+            u.w = pack2<T>(make_float2(v[8 * q + 6], v[8 * q + 7]));
+            const int chunk = ((c & 63) >> 3) + q;
+            *reinterpret_cast<uint4*>(line + ((chunk ^ (row & 7)) << 4)) = u;
+          }
+        } else if (valid) {
+          epilogue_store<T>(P, y, bias, r, ncols, n, ho, wo, co0 + c);
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
+      if (P.tma_out) {
+        fence_async_smem();
+        named_sync(1, 128);
+        if (store_thread) {
+          for (int blk = 0; blk < P.BN / 64; ++blk)
+            tma_store_4d(&tma_y, obuf + (size_t)blk * (128 * 128), co0 + 64 * blk, 0,
+                         th * P.BH, n);
+          bulk_commit();
+        }
+        ob ^= 1;
+      }
       if (++acc == 2) {
         acc = 0;
         aph ^= 1u;
       }
     }
+    if (store_thread) bulk_wait0();
   }
 
   tc_fence_before();
@@ -1386,14 +1507,19 @@ bool make_halo_params(const Conv2d& p, HaloParams* H) {
   if (mma_rows > rows) rows = mma_rows;
   H->a_region = (rows * H->row_bytes + 1023u) & ~1023u;
   H->b_tile = (unsigned int)BN * H->row_bytes;
-  const size_t fixed = 1024 + (2 * MAX_STAGES + 5) * 8 + 16;
+  H->tma_out = p.layout == GCONV_NHWC && BN % 64 == 0;
+  H->o_bytes = H->tma_out ? 2u * (unsigned int)(BN / 64) * 128u * 128u : 0u;
+  const size_t fixed = 1024 + (2 * MAX_STAGES + 5) * 8 + 16 + H->o_bytes;
   const size_t budget = SMEM_BUDGET - fixed;
-  // all kw of a channel block per stage when three such stages fit, else one kw per stage
+  // all kw of a channel block per stage (one handshake per kH*kW*BKC/16 MMAs) when enough
+  // such stages fit -- two with the TMA-store epilogue, whose stores no longer hold the
+  // epilogue up, else three -- otherwise one kw per stage
+  const int min_stages = H->tma_out ? 2 : 3;
   int kws = p.kW;
   for (;;) {
     const size_t st = (size_t)kws * H->a_region + ((size_t)kws * p.kH * H->b_tile + 1023) / 1024 * 1024;
     const int n = (int)(budget / st);
-    if (n >= 3 || kws == 1) {
+    if (n >= min_stages || kws == 1) {
       H->KWS = kws;
       H->a_stage = (unsigned int)((size_t)kws * H->a_region);
       H->b_stage = (unsigned int)(((size_t)kws * p.kH * H->b_tile + 1023) / 1024 * 1024);
@@ -1417,7 +1543,8 @@ bool make_halo_params(const Conv2d& p, HaloParams* H) {
 }
 
 size_t halo_smem_bytes(const HaloParams& H) {
-  return 1024 + (size_t)H.stages * (H.a_stage + H.b_stage) + (2 * MAX_STAGES + 5) * 8 + 16;
+  return 1024 + (size_t)H.stages * (H.a_stage + H.b_stage) + H.o_bytes +
+         (2 * MAX_STAGES + 5) * 8 + 16;
 }
 
 template <typename T>
@@ -1446,6 +1573,20 @@ cudaError_t launch_halo(const Conv2d& p, const HaloParams& H, const void* x, con
           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(H.BKC), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  CUtensorMap ty;
+  if (H.tma_out) {
+    const cuuint64_t ydim[4] = {(cuuint64_t)p.C_out, (cuuint64_t)p.Wo, (cuuint64_t)p.Ho,
+                                (cuuint64_t)p.N};
+    const cuuint64_t ystr[3] = {(cuuint64_t)p.C_out * 2, (cuuint64_t)p.Wo * p.C_out * 2,
+                                (cuuint64_t)p.Ho * p.Wo * p.C_out * 2};
+    const cuuint32_t ybox[4] = {64, (cuuint32_t)H.BW, (cuuint32_t)H.BH, 1};
+    if (enc(&ty, dt, 4, y, ydim, ystr, ybox, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    ty = tx;                                  // unused by the kernel
+  }
   const size_t smem = halo_smem_bytes(H);
   if (smem > SMEM_BUDGET) return cudaErrorInvalidValue;
   static std::atomic<unsigned int> configured{0};
@@ -1453,7 +1594,7 @@ cudaError_t launch_halo(const Conv2d& p, const HaloParams& H, const void* x, con
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   if (grid > H.num_tiles) grid = H.num_tiles;
-  igemm_halo_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, tw, (const T*)bias, (T*)y, H,
+  igemm_halo_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, tw, ty, (const T*)bias, (T*)y, H,
                                                        device_error_word());
   return cudaGetLastError();
 }

@@ -35,6 +35,8 @@ SMALL = [
     (1, 64, 12, 16, 64, 3, 2, 2, 2),         # halo tile kernel: Wo = 16, dilation 2
     (2, 96, 9, 32, 96, 5, 2, 1, 3),          # halo tile kernel: 5x5, 32 / 32
     (1, 128, 5, 40, 64, 3, 1, 1, 2),         # halo tile kernel: 64-channel blocks, 3-row tiles
+    (2, 128, 9, 24, 128, 3, 1, 1, 2),        # halo: 64 filters a group (TMA-store epilogue), 5-row tiles, ragged
+    (1, 64, 6, 16, 256, 3, 1, 1, 2),         # halo: 128 filters a group (two 64-channel stores)
 ]
 
 
