@@ -288,6 +288,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // kh*dil*Wo (whole 8-row swizzle atoms, since Wo % 8 == 0), plus the kH*KWS weight tiles.
 // Each stage thus feeds kH*KWS*BKC/16 MMAs to the single issuing thread between barrier waits,
 // and the input is fetched once per kw instead of once per tap.
+//
+// Groups of 16 or 32 input channels are packed gp = 64 / cpg_in to a tile: the box holds their
+// 64 channels (one 128-byte row per pixel) and the filter tile is block-diagonal -- filter f of
+// packed group g has its cpg_in weights in channel slot g and zeros elsewhere -- so one MMA
+// chain computes all gp groups at N = gp*cpg_out. TMA builds the block-diagonal tile: each
+// group's filters are read through a [C_out][taps][cpg_in] view with a 64-channel box started
+// g*cpg_in channels before the row, so the other slots fall outside the row and are filled
+// with zeros.
 
 struct HaloParams {
   int N, H, W, C_in, C_out, Ho, Wo, kH, kW, pad, dil, cpg_in, cpg_out;
@@ -296,6 +304,8 @@ struct HaloParams {
   unsigned int a_region, a_stage, b_tile, b_stage, tx_bytes;
   unsigned int idesc, swz, sbo, row_bytes, tmem_cols;
   int out_nchw;
+  int gp, gin, gout;           // groups packed per tile (block-diagonal filters), their
+                               // input and output channels: gin = gp*cpg_in, gout = gp*cpg_out
   int tma_out;                 // NHWC output through shared memory and TMA stores
   unsigned int o_bytes;        // that staging, two buffers of BN/64 blocks of [128 rows][64 ch]
                                // with the 128-byte swizzle
@@ -431,9 +441,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int j, nt, n, th;
         halo_decode(P, t, j, nt, n, th);
         const int hbase = th * P.BH - P.pad;
-        const int obase = j * P.cpg_out + nt * P.BN;
+        const int obase = j * P.gout + nt * P.BN;
         for (int cb = 0; cb < P.cblocks && ok; ++cb) {
-          const int cin = j * P.cpg_in + cb * P.BKC;
+          const int cin = j * P.gin + cb * P.BKC;
           for (int kg = 0; kg < P.kw_groups; ++kg) {
             if (!mbar_try_wait(&empty[s], ph ^ 1u) &&
                 !mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
@@ -447,9 +457,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const int kw = kg * P.KWS + kwi;
               tma_load_4d(a_st + (size_t)kwi * P.a_region, &tma_x, &full[s], cin,
                           kw * P.dil - P.pad, hbase, n);
-              for (int kh = 0; kh < P.kH; ++kh)
-                tma_load_2d(b_st + (size_t)(kwi * P.kH + kh) * P.b_tile, &tma_w, &full[s],
-                            (kh * P.kW + kw) * P.cpg_in + cb * P.BKC, obase);
+              for (int kh = 0; kh < P.kH; ++kh) {
+                unsigned char* bt = b_st + (size_t)(kwi * P.kH + kh) * P.b_tile;
+                if (P.gp == 1) {
+                  tma_load_2d(bt, &tma_w, &full[s], (kh * P.kW + kw) * P.cpg_in + cb * P.BKC,
+                              obase);
+                } else {
+                  for (int g = 0; g < P.gp; ++g)
+                    tma_load_3d(bt + (size_t)g * P.cpg_out * P.row_bytes, &tma_w, &full[s],
+                                -g * P.cpg_in, kh * P.kW + kw, obase + g * P.cpg_out);
+                }
+              }
             }
             ++issued;
             if (++s == P.stages) {
@@ -551,7 +569,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int ho = th * P.BH + hl, wo = wl;
       const bool valid = hl < P.BH && ho < P.Ho;
-      const int co0 = j * P.cpg_out + nt * P.BN;
+      const int co0 = j * P.gout + nt * P.BN;
       const unsigned int taddr =
           tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.BN);
       for (int c = 0; c < P.BN; c += 32) {
@@ -1207,14 +1225,15 @@ __global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const T* __restrict__
 template <typename T>
 __global__ void repack_weight_kernel(const T* __restrict__ w, T* __restrict__ wt, int C_out,
                                      int cpg_in, int taps) {
-  const long long total = (long long)C_out * cpg_in * taps;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int ci = (int)(i % cpg_in);
-    const long long r = i / cpg_in;
-    const int tap = (int)(r % taps);
-    const int co = (int)(r / taps);
-    wt[i] = w[((long long)co * cpg_in + ci) * taps + tap];
+  // one filter per grid row: wt[co][tap][ci] = w[co][ci][tap], 32-bit index math
+  const int n = cpg_in * taps;
+  for (int co = blockIdx.y; co < C_out; co += gridDim.y) {
+    const T* src = w + (long long)co * n;
+    T* dst = wt + (long long)co * n;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+      const int tap = i / cpg_in, ci = i - tap * cpg_in;
+      dst[i] = src[ci * taps + tap];
+    }
   }
 }
 
@@ -1480,7 +1499,20 @@ cudaError_t launch_rowt(const Conv2d& p, const RowTParams& R, const void* x, con
 // a width that is not a multiple of 8, or stages that do not fit).
 bool make_halo_params(const Conv2d& p, HaloParams* H) {
   if (p.Wo > BM || p.Wo % 8 != 0) return false;
-  const int BN = tile_bn(p);
+  // groups packed per tile: 64 / cpg_in of them when that divides the group count and keeps
+  // N = gp * cpg_out within 64. The block-diagonal filter tile makes each MMA as wide as the
+  // packed N while the MMA count per group stays the same, and MMA time grows with operand
+  // bytes (measured: 128x128x16 ~130 cycles against ~100 for 128x64x16), so packing pays only
+  // where it lifts a narrow N (g = 64 of the sweep: 16 -> 64, 504 -> 364 us) -- not for
+  // 64-filter groups (ensemble layer: 317 -> 377 us when packed in pairs).
+  int gp = 1;
+  if ((p.cpg_in == 16 || p.cpg_in == 32) && p.groups % (64 / p.cpg_in) == 0 &&
+      (64 / p.cpg_in) * p.cpg_out <= 64 && ((64 / p.cpg_in) * p.cpg_out) % 16 == 0)
+    gp = 64 / p.cpg_in;
+  H->gp = gp;
+  H->gin = gp * p.cpg_in;
+  H->gout = gp * p.cpg_out;
+  const int BN = gp > 1 ? H->gout : tile_bn(p);
   if (BN == 0) return false;
   H->N = p.N; H->H = p.H; H->W = p.W; H->C_in = p.C_in; H->C_out = p.C_out;
   H->Ho = p.Ho; H->Wo = p.Wo; H->kH = p.kH; H->kW = p.kW; H->pad = p.pad; H->dil = p.dil;
@@ -1489,12 +1521,12 @@ bool make_halo_params(const Conv2d& p, HaloParams* H) {
   H->BH = BM / p.Wo;
   if (H->BH > p.Ho) H->BH = p.Ho;
   H->BN = BN;
-  H->BKC = p.cpg_in % 64 == 0 ? 64 : (p.cpg_in % 32 == 0 ? 32 : 16);
-  H->cblocks = p.cpg_in / H->BKC;
+  H->BKC = H->gin % 64 == 0 ? 64 : (H->gin % 32 == 0 ? 32 : 16);
+  H->cblocks = H->gin / H->BKC;
   H->tiles_h = (p.Ho + H->BH - 1) / H->BH;
   const long long m_tiles = (long long)p.N * H->tiles_h;
-  H->n_tiles = p.cpg_out / BN;
-  const long long tiles = m_tiles * H->n_tiles * p.groups;
+  H->n_tiles = H->gout / BN;
+  const long long tiles = m_tiles * H->n_tiles * (p.groups / gp);
   if (tiles > INT32_MAX) return false;
   H->m_tiles = (int)m_tiles;
   H->num_tiles = (int)tiles;
@@ -1566,13 +1598,25 @@ cudaError_t launch_halo(const Conv2d& p, const HaloParams& H, const void* x, con
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   const cuuint64_t ktot = (cuuint64_t)p.kH * p.kW * p.cpg_in;
-  const cuuint64_t wdim[2] = {ktot, (cuuint64_t)p.C_out};
-  const cuuint64_t wstr[1] = {ktot * 2};
-  const cuuint32_t wbox[2] = {(cuuint32_t)H.BKC, (cuuint32_t)H.BN};
-  if (enc(&tw, dt, 2, const_cast<void*>(w), wdim, wstr, wbox, ones,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(H.BKC), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  if (H.gp == 1) {
+    const cuuint64_t wdim[2] = {ktot, (cuuint64_t)p.C_out};
+    const cuuint64_t wstr[1] = {ktot * 2};
+    const cuuint32_t wbox[2] = {(cuuint32_t)H.BKC, (cuuint32_t)H.BN};
+    if (enc(&tw, dt, 2, const_cast<void*>(w), wdim, wstr, wbox, ones,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(H.BKC), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    // [C_out][taps][cpg_in] view; a 64-channel box over a cpg_in-channel row reads zeros
+    // outside it (block-diagonal filter tiles, see the kernel's comment)
+    const cuuint64_t wdim[3] = {(cuuint64_t)p.cpg_in, (cuuint64_t)p.kH * p.kW, (cuuint64_t)p.C_out};
+    const cuuint64_t wstr[2] = {(cuuint64_t)p.cpg_in * 2, ktot * 2};
+    const cuuint32_t wbox[3] = {(cuuint32_t)H.BKC, 1, (cuuint32_t)p.cpg_out};
+    if (enc(&tw, dt, 3, const_cast<void*>(w), wdim, wstr, wbox, ones,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(H.BKC), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   CUtensorMap ty;
   if (H.tma_out) {
     const cuuint64_t ydim[4] = {(cuuint64_t)p.C_out, (cuuint64_t)p.Wo, (cuuint64_t)p.Ho,
@@ -1681,10 +1725,9 @@ cudaError_t launch_nchw_typed(const Conv2d& p, const IgemmParams& P, const void*
   T* xt = (T*)workspace;
   T* wt = (T*)((char*)workspace + align256((size_t)p.N * p.H * p.W * p.C_in * 2));
   const int taps = p.kH * p.kW;
-  const long long wtotal = (long long)p.C_out * p.cpg_in * taps;
-  long long wb = (wtotal + 255) / 256;
-  if (wb > 4096) wb = 4096;
-  repack_weight_kernel<T><<<(unsigned)wb, 256, 0, s>>>((const T*)w, wt, p.C_out, p.cpg_in, taps);
+  const int per_filter = p.cpg_in * taps;
+  dim3 wgrid((unsigned)((per_filter + 255) / 256), (unsigned)(p.C_out < 65535 ? p.C_out : 65535));
+  repack_weight_kernel<T><<<wgrid, 256, 0, s>>>((const T*)w, wt, p.C_out, p.cpg_in, taps);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int HW = p.H * p.W;

@@ -37,6 +37,9 @@ SMALL = [
     (1, 128, 5, 40, 64, 3, 1, 1, 2),         # halo tile kernel: 64-channel blocks, 3-row tiles
     (2, 128, 9, 24, 128, 3, 1, 1, 2),        # halo: 64 filters a group (TMA-store epilogue), 5-row tiles, ragged
     (1, 64, 6, 16, 256, 3, 1, 1, 2),         # halo: 128 filters a group (two 64-channel stores)
+    (2, 64, 8, 16, 64, 3, 1, 1, 2),          # halo, 2 groups packed (32 -> 32 ch): N = 64
+    (1, 64, 6, 24, 64, 3, 1, 1, 4),          # halo, 4 groups packed (16 -> 16 ch): N = 64
+    (1, 128, 5, 8, 64, 5, 2, 1, 4),          # halo, 2 groups packed, N = 32, 5x5
 ]
 
 
