@@ -385,7 +385,7 @@ __device__ __forceinline__ bool halo_issue_kh(int kh, int kws, unsigned int d,
   }
 }
 
-template <typename T>
+template <typename T, bool PACK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     igemm_halo_kernel(const __grid_constant__ CUtensorMap tma_x,
                       const __grid_constant__ CUtensorMap tma_w,
@@ -441,9 +441,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int j, nt, n, th;
         halo_decode(P, t, j, nt, n, th);
         const int hbase = th * P.BH - P.pad;
-        const int obase = j * P.gout + nt * P.BN;
+        const int obase = j * (PACK ? P.gout : P.cpg_out) + nt * P.BN;
         for (int cb = 0; cb < P.cblocks && ok; ++cb) {
-          const int cin = j * P.gin + cb * P.BKC;
+          const int cin = j * (PACK ? P.gin : P.cpg_in) + cb * P.BKC;
           for (int kg = 0; kg < P.kw_groups; ++kg) {
             if (!mbar_try_wait(&empty[s], ph ^ 1u) &&
                 !mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                           kw * P.dil - P.pad, hbase, n);
               for (int kh = 0; kh < P.kH; ++kh) {
                 unsigned char* bt = b_st + (size_t)(kwi * P.kH + kh) * P.b_tile;
-                if (P.gp == 1) {
+                if constexpr (!PACK) {
                   tma_load_2d(bt, &tma_w, &full[s], (kh * P.kW + kw) * P.cpg_in + cb * P.BKC,
                               obase);
                 } else {
@@ -569,7 +569,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int ho = th * P.BH + hl, wo = wl;
       const bool valid = hl < P.BH && ho < P.Ho;
-      const int co0 = j * P.gout + nt * P.BN;
+      const int co0 = j * (PACK ? P.gout : P.cpg_out) + nt * P.BN;
       const unsigned int taddr =
           tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.BN);
       for (int c = 0; c < P.BN; c += 32) {
@@ -1633,13 +1633,20 @@ cudaError_t launch_halo(const Conv2d& p, const HaloParams& H, const void* x, con
   }
   const size_t smem = halo_smem_bytes(H);
   if (smem > SMEM_BUDGET) return cudaErrorInvalidValue;
-  static std::atomic<unsigned int> configured{0};
-  cudaError_t e = set_max_dynamic_smem((const void*)igemm_halo_kernel<T>, SMEM_BUDGET, configured);
+  // packing is a separate instantiation, so the unpacked kernel carries none of its code
+  static std::atomic<unsigned int> configured[2];
+  const void* fn = H.gp > 1 ? (const void*)igemm_halo_kernel<T, true>
+                            : (const void*)igemm_halo_kernel<T, false>;
+  cudaError_t e = set_max_dynamic_smem(fn, SMEM_BUDGET, configured[H.gp > 1 ? 1 : 0]);
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   if (grid > H.num_tiles) grid = H.num_tiles;
-  igemm_halo_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, tw, ty, (const T*)bias, (T*)y, H,
-                                                       device_error_word());
+  if (H.gp > 1)
+    igemm_halo_kernel<T, true><<<grid, NUM_THREADS, smem, s>>>(tx, tw, ty, (const T*)bias,
+                                                               (T*)y, H, device_error_word());
+  else
+    igemm_halo_kernel<T, false><<<grid, NUM_THREADS, smem, s>>>(tx, tw, ty, (const T*)bias,
+                                                                (T*)y, H, device_error_word());
   return cudaGetLastError();
 }
 
