@@ -472,7 +472,10 @@ cudaError_t wgrad_vec(const Conv1d& p, const T* x, const T* dy, T* dw, float* pa
   P.dy_bytes = (unsigned int)WTB * CH * 2;
   P.x_bytes = (unsigned int)(WTB + K - 1) * CH * 2;
   P.stage_bytes = (P.dy_bytes + P.x_bytes + 127u) & ~127u;
-  P.stages = 4;
+  // as deep a ring as lets two CTAs share an SM (<= 110 KB each), 2 to 4 stages
+  P.stages = (int)((110u * 1024u) / P.stage_bytes);
+  if (P.stages > 4) P.stages = 4;
+  if (P.stages < 2) P.stages = 2;
   const size_t red = (size_t)RSTRIPS * K * CP * sizeof(float2);
   size_t ring = (size_t)P.stages * P.stage_bytes;
   if (ring < red) ring = red;
