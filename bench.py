@@ -156,6 +156,16 @@ def gpu_spin(torch, stream, us=200):
         torch.cuda._sleep(int(us * 2000))
 
 
+def max_over_ranks(torch, dist, value: float, device) -> float:
+    """The maximum of `value` over all ranks of the default process group (the job's time is
+    its slowest rank's); `value` itself when no group is initialised."""
+    if dist is None or not dist.is_available() or not dist.is_initialized():
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def time_launches(torch, fn, stream, reps, flush=None):
     """Median and mean CUDA-event time (ms) of `fn(i)` over `reps` launches on `stream`,
     flushing L2 before each launch outside the event bracket."""
@@ -498,9 +508,7 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(torch, dist, total_ms, device)
         dist.barrier()
 
     flops = p.flops()
@@ -547,9 +555,7 @@ def main():
         torch.cuda.synchronize()
         e_ms = a.elapsed_time(b)
         if world > 1:
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+            e_ms = max_over_ranks(torch, dist, e_ms, device)
         e2e = {"value": round(flops * world * n_e2e / (e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                "h2d_bytes_per_step": (x_host.numel() + w_host.numel()) * 2,
                "d2h_bytes_per_step": y_pin.numel() * 2, "steps": n_e2e}
