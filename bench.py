@@ -191,13 +191,13 @@ def conv2d_problem(layout: str):
 
 
 def kernel_name(code: int) -> str:
-    return {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "igemm_tc_nchw"}.get(
-        code, str(code))
+    return {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "igemm_tc_nchw",
+            8: "grouped_nhwc"}.get(code, str(code))
 
 
-LAUNCHES_PER_CALL = {1: 1, 2: 1, 3: 1, 4: 3}
+LAUNCHES_PER_CALL = {1: 1, 2: 1, 3: 1, 4: 3, 8: 1}
 KERNEL_SOURCE = {1: "direct_generic.cu", 2: "depthwise_nhwc.cu", 3: "igemm_tc.cu",
-                 4: "igemm_tc.cu"}
+                 4: "igemm_tc.cu", 8: "grouped_nhwc.cu"}
 
 
 def conv2d_measurement(torch, gb, device, stream, pk, p, workload, path, reps, flush):

@@ -86,6 +86,8 @@ int choose_kernel(const Conv2d& p, int path, const void* x, const void* w, const
   const bool dw_ok = depthwise_nhwc_supported(p) && p.N <= 65535;
   const bool dw_al = query || (aligned_to(x, depthwise_vec_bytes(p)) &&
                                aligned_to(y, depthwise_vec_bytes(p)));
+  // narrow groups: TMA boxes and stores need 16-byte aligned x and y
+  const bool ng_ok = grouped_nhwc_supported(p) && (query || (aligned16(x) && aligned16(y)));
   const bool tc_ok = igemm_supported(p);
   // tensor maps need 16-byte aligned bases (x, and w when it is used in place: NHWC)
   const bool tc_al = query || (aligned16(x) && aligned16(y) &&
@@ -95,7 +97,8 @@ int choose_kernel(const Conv2d& p, int path, const void* x, const void* w, const
     case GCONV_PATH_GENERIC:
       return GCONV_KERNEL_DIRECT_GENERIC;
     case GCONV_PATH_DIRECT:
-      return (dw_ok && dw_al) ? GCONV_KERNEL_DEPTHWISE_NHWC : GCONV_KERNEL_DIRECT_GENERIC;
+      if (dw_ok && dw_al) return GCONV_KERNEL_DEPTHWISE_NHWC;
+      return ng_ok ? GCONV_KERNEL_GROUPED_NHWC : GCONV_KERNEL_DIRECT_GENERIC;
     case GCONV_PATH_IGEMM:
       if (!tc_ok) { *why = GCONV_ERR_UNSUPPORTED; return -1; }
       if (!tc_al) { *why = GCONV_ERR_MISALIGNED; return -1; }
@@ -103,6 +106,7 @@ int choose_kernel(const Conv2d& p, int path, const void* x, const void* w, const
     case GCONV_PATH_AUTO:
       if (p.dtype == GCONV_F32) return GCONV_KERNEL_DIRECT_GENERIC;
       if (dw_ok && dw_al) return GCONV_KERNEL_DEPTHWISE_NHWC;
+      if (ng_ok) return GCONV_KERNEL_GROUPED_NHWC;
       if (tc_ok && tc_al) return tc_kernel;
       return GCONV_KERNEL_DIRECT_GENERIC;
     default:
@@ -172,6 +176,8 @@ gconv_status gconv2d_fwd_path(const void* x, const void* w, const void* bias, vo
   switch (kernel) {
     case GCONV_KERNEL_DEPTHWISE_NHWC:
       return cuda_status(launch_depthwise_nhwc(p, x, w, bias, y, s));
+    case GCONV_KERNEL_GROUPED_NHWC:
+      return cuda_status(launch_grouped_nhwc(p, x, w, bias, y, s));
     case GCONV_KERNEL_IGEMM_TC:
       return cuda_status(launch_igemm_nhwc(p, x, w, bias, y, s));
     case GCONV_KERNEL_IGEMM_TC_NCHW: {

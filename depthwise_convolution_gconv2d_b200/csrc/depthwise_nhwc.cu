@@ -317,8 +317,10 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&empty[s]);
-        tma_store_4d(&tmy, wstage, c.ct * DW3_CH, c.tw * DW3_BW + g * DW3_R, c.th * BH, c.n);
-        bulk_commit();
+        if (c.tw * DW3_BW + g * DW3_R < P.Wo) {   // a box wholly right of the image is skipped
+          tma_store_4d(&tmy, wstage, c.ct * DW3_CH, c.tw * DW3_BW + g * DW3_R, c.th * BH, c.n);
+          bulk_commit();
+        }
       }
       c.next(P);
       if (++s == P.stages) {

@@ -99,6 +99,11 @@ bool depthwise_nhwc_supported(const Conv2d& p);
 cudaError_t launch_depthwise_nhwc(const Conv2d& p, const void* x, const void* w,
                                   const void* bias, void* y, cudaStream_t s);
 
+// Narrow groups (2 / 4 / 8 channels per group), 3x3, NHWC, 16-bit, C % 8 == 0, aligned x, y.
+bool grouped_nhwc_supported(const Conv2d& p);
+cudaError_t launch_grouped_nhwc(const Conv2d& p, const void* x, const void* w,
+                                const void* bias, void* y, cudaStream_t s);
+
 bool igemm_supported(const Conv2d& p);      // shape/dtype eligibility, layout-independent
 size_t igemm_nchw_workspace(const Conv2d& p);
 cudaError_t launch_igemm_nhwc(const Conv2d& p, const void* x, const void* w, const void* bias,

@@ -82,8 +82,8 @@ typedef enum { GCONV_F32 = 0, GCONV_F16 = 1, GCONV_BF16 = 2 } gconv_dtype;
  * if it cannot run the problem. */
 typedef enum {
   GCONV_PATH_AUTO = 0,
-  GCONV_PATH_DIRECT = 1,   /* CUDA-core direct convolution (vectorised depthwise kernel when
-                              it applies, otherwise the generic direct kernel) */
+  GCONV_PATH_DIRECT = 1,   /* CUDA-core direct convolution (the depthwise or narrow-group
+                              kernel when one applies, otherwise the generic direct kernel) */
   GCONV_PATH_IGEMM = 2,    /* per-group implicit GEMM on tcgen05 tensor cores (F16 / BF16) */
   GCONV_PATH_GENERIC = 3   /* the generic direct kernel (any shape, layout and dtype) */
 } gconv_path;
@@ -97,8 +97,10 @@ typedef enum {
   GCONV_KERNEL_CONV1D_GENERIC = 5,    /* dwconv1d: one thread per output, fp32 FMA, any problem */
   GCONV_KERNEL_CONV1D_RING = 6,       /* dwconv1d: CUDA-core TMA-ring kernel; 16-bit, C % 8 == 0,
                                          K in {3, 5, 7, 9, 15, 31} */
-  GCONV_KERNEL_CONV1D_TC = 7          /* dwconv1d: tcgen05 banded product; 16-bit, C % 16 == 0,
+  GCONV_KERNEL_CONV1D_TC = 7,         /* dwconv1d: tcgen05 banded product; 16-bit, C % 16 == 0,
                                          K <= 49 */
+  GCONV_KERNEL_GROUPED_NHWC = 8       /* conv2d, 2 / 4 / 8 channels per group in and out, 3x3,
+                                         dilation 1, stride 1 or 2, 16-bit NHWC: CUDA cores */
 } gconv_kernel;
 
 /* Bytes of workspace gconv2d_fwd needs for this problem under `path` (0 if none; also 0 for

@@ -142,3 +142,22 @@ def test_conv1d_path_selection(lib):
     # a forced path that cannot run is rejected before anything is launched
     assert lib.dwconv1d_fwd_path(None, None, None, 0, 8, 16, 3, 1, 1, F32, 2, None) == 2
     assert lib.dwconv1d_bwd_data_path(None, None, None, 0, 8, 16, 3, 1, 1, BF16, 9, None) == 1
+
+
+def test_narrow_group_selection(lib):
+    """2 / 4 / 8 channels per group, 3x3, stride 1 or 2, 16-bit NHWC -> the narrow-group
+    CUDA-core kernel (8) under AUTO and DIRECT; anything else keeps its previous kernel."""
+    NHWC, NCHW, BF16, F16, F32 = 1, 0, 2, 1, 0
+    sel = lambda path, layout=NHWC, dtype=BF16, **over: lib.gconv2d_select_path(
+        *_conv_args(**over), layout, dtype, path)
+    for cpg in (2, 4, 8):
+        kw = dict(C_in=64, C_out=64, groups=64 // cpg)
+        assert sel(0, **kw) == 8 and sel(1, **kw) == 8
+        assert sel(0, dtype=F16, **kw) == 8
+        assert sel(0, stride=2, **kw) == 8
+        assert sel(0, layout=NCHW, **kw) == 1             # NCHW: generic
+        assert sel(0, dtype=F32, **kw) == 1               # fp32: generic
+        assert sel(0, kH=5, kW=5, pad=2, **kw) == 1       # 5x5: generic
+        assert sel(0, dil=2, pad=2, **kw) == 1            # dilation: generic
+    assert sel(0, C_in=64, C_out=64, groups=4) == 3       # 16 per group: tensor cores
+    assert sel(0, C_in=64, C_out=128, groups=16) != 8     # 4 in / 8 out: not narrow-group

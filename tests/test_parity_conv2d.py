@@ -116,6 +116,43 @@ def test_depthwise_nhwc_integer_bit_exact(case):
     assert np.array_equal(to_f64(run_gpu(inp)), oracle_full(inp))
 
 
+# ------------------------------------------------------------ narrow groups (2 / 4 / 8 channels)
+
+NG_CASES = [
+    # N, C, H, W, stride, pad, groups          (channels per group = C / groups)
+    (2, 64, 9, 30, 1, 1, 16),       # 4 per group, two column tiles (28 + 2)
+    (1, 64, 7, 29, 1, 1, 32),       # 2 per group
+    (2, 128, 6, 12, 1, 1, 16),      # 8 per group, two channel tiles
+    (1, 64, 9, 59, 2, 1, 16),       # stride 2, ragged 2-row tiles
+    (1, 72, 5, 9, 1, 1, 18),        # C = 72: the second channel tile holds 8 channels
+    (1, 64, 8, 10, 2, 2, 16),       # stride 2, pad 2
+    (3, 32, 5, 5, 1, 0, 8),         # no padding, tiny image
+]
+
+
+@pytest.mark.parametrize("case", NG_CASES)
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F16])
+def test_narrow_groups_nhwc(case, dtype):
+    N, C, H, W, st, pd, g = case
+    p = wl.Conv2dProblem(N, C, H, W, C, 3, 3, st, pd, 1, g, wl.NHWC, dtype, bias=True)
+    assert kernel_of(p) == 8
+    inp = wl.make_conv2d_inputs(p, 15)
+    assert_close(to_f64(run_gpu(inp)), oracle_full(inp), dtype, str(case))
+
+
+@pytest.mark.parametrize("case", NG_CASES[:4])
+def test_narrow_groups_integer_bit_exact(case):
+    """x, w in {-1, 0, 1}: at most 72 terms per output, every partial sum exact in fp32 and the
+    result exact in bf16, so any order of the sum gives the oracle's value bit for bit."""
+    N, C, H, W, st, pd, g = case
+    p = wl.Conv2dProblem(N, C, H, W, C, 3, 3, st, pd, 1, g, wl.NHWC, wl.BF16)
+    r = np.random.default_rng(16)
+    inp = wl.make_conv2d_inputs(p, 16)
+    inp.x = wl.to_storage(r.integers(-1, 2, p.x_shape), wl.BF16)
+    inp.w = wl.to_storage(r.integers(-1, 2, p.w_shape), wl.BF16)
+    assert np.array_equal(to_f64(run_gpu(inp)), oracle_full(inp))
+
+
 @pytest.mark.parametrize("kh,kw", [(1, 1), (0, 2), (2, 0), (2, 2)])
 def test_depthwise_delta_kernel_is_exact_shift(kh, kw):
     """A delta tap at (kh, kw) with pad 1 gives y[h, w] = x[h + kh - 1, w + kw - 1] with zero

@@ -130,7 +130,7 @@ def test_auto_picks_tensor_cores_for_wide_groups():
     assert kernel_of(wl.ensemble_groups()) == 3
     assert kernel_of(wl.depthwise_56(1, 64)) == 3
     assert kernel_of(wl.depthwise_56(1, 16)) == 3
-    assert kernel_of(wl.depthwise_56(1, 256)) == 1   # 4 channels per group: CUDA cores
+    assert kernel_of(wl.depthwise_56(1, 256)) == 8   # 4 channels per group: CUDA cores
     assert kernel_of(wl.depthwise_56(1, 1024)) == 2
 
 
