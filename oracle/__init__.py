@@ -10,6 +10,8 @@ Definitions followed (see the header of ``oracle.c`` for the full statement):
     outputs split into groups with no cross-group connections, group-major channel
     order; cross-correlation with zero padding as ``F.conv2d(..., groups=g)`` in
     "F.conv2d runs x15 slower in mixed-precision/half-precision mode";
+  * the data and weight gradients of grouped conv2d (scatter / direct-sum forms of the
+    forward sum's adjoint), for the training uses of grouped layers on the pages;
   * depthwise conv1d on (batch, steps, channels), forward and backward -- "Investigate
     custom Triton kernels for depthwise-separable convolutions in Conformer".
 
@@ -51,6 +53,14 @@ def _configure(lib):
     lib.oracle_conv2d.restype = I
     lib.oracle_conv2d_points.argtypes = [P, P, P, P, P, L] + [L] * 11 + [I]
     lib.oracle_conv2d_points.restype = I
+    for name in ("oracle_conv2d_bwd_data", "oracle_conv2d_bwd_weight"):
+        f = getattr(lib, name)
+        f.argtypes = [P, P, P] + [L] * 11 + [I]
+        f.restype = I
+    for name in ("oracle_conv2d_bwd_data_points", "oracle_conv2d_bwd_weight_points"):
+        f = getattr(lib, name)
+        f.argtypes = [P, P, P, P, L] + [L] * 11 + [I]
+        f.restype = I
     for name in ("oracle_dwconv1d_fwd", "oracle_dwconv1d_bwd_data",
                  "oracle_dwconv1d_bwd_weight"):
         f = getattr(lib, name)
@@ -138,6 +148,96 @@ def conv2d_points(x, w, idx, bias=None, stride=1, pad=0, dilation=1, groups=1, l
     if rc != 0:
         raise ValueError("oracle_conv2d_points rejected the shape or an index")
     return out
+
+
+def _bwd_dims(dy_shape, w_shape, in_hw, stride, pad, dilation, groups, layout):
+    """(N, C_in, H, W, C_out, kH, kW) of the forward problem behind a backward call, checking
+    that dy has that problem's output shape."""
+    H, W = in_hw
+    if layout == NCHW:
+        N, C_out = dy_shape[0], dy_shape[1]
+        C_out2, cpg_in, kH, kW = w_shape
+    elif layout == NHWC:
+        N, C_out = dy_shape[0], dy_shape[3]
+        C_out2, kH, kW, cpg_in = w_shape
+    else:
+        raise ValueError("layout must be NCHW (0) or NHWC (1)")
+    C_in = cpg_in * groups
+    if C_out2 != C_out or groups <= 0 or C_out % groups:
+        raise ValueError("inconsistent groups / channel counts")
+    x_shape = (N, C_in, H, W) if layout == NCHW else (N, H, W, C_in)
+    if tuple(dy_shape) != conv2d_out_shape(x_shape, w_shape, stride, pad, dilation, groups,
+                                           layout):
+        raise ValueError("dy does not have the forward output's shape")
+    return (N, C_in, H, W, C_out, kH, kW), x_shape
+
+
+def conv2d_bwd_data(dy, w, in_hw, stride=1, pad=0, dilation=1, groups=1, layout=NCHW):
+    """dx of grouped conv2d (input spatial size ``in_hw`` = (H, W)), in x's layout."""
+    dy, w = _f64(dy), _f64(w)
+    dims, x_shape = _bwd_dims(dy.shape, w.shape, in_hw, stride, pad, dilation, groups, layout)
+    dx = np.empty(x_shape)
+    if _load().oracle_conv2d_bwd_data(_ptr(dy), _ptr(w), _ptr(dx), *dims, stride, pad,
+                                      dilation, groups, layout) != 0:
+        raise ValueError("oracle_conv2d_bwd_data rejected the shape")
+    return dx
+
+
+def conv2d_bwd_data_points(dy, w, in_hw, idx, stride=1, pad=0, dilation=1, groups=1,
+                           layout=NCHW):
+    """dx at idx[i] = (n, c, h, w) (logical indices)."""
+    dy, w = _f64(dy), _f64(w)
+    dims, _ = _bwd_dims(dy.shape, w.shape, in_hw, stride, pad, dilation, groups, layout)
+    idx = np.ascontiguousarray(idx, dtype=np.int64).reshape(-1, 4)
+    out = np.empty(idx.shape[0])
+    if _load().oracle_conv2d_bwd_data_points(_ptr(dy), _ptr(w), _ptr(out), _ptr(idx),
+                                             idx.shape[0], *dims, stride, pad, dilation, groups,
+                                             layout) != 0:
+        raise ValueError("oracle_conv2d_bwd_data_points rejected the shape or an index")
+    return out
+
+
+def conv2d_bwd_weight(x, dy, kernel_hw, stride=1, pad=0, dilation=1, groups=1, layout=NCHW):
+    """dw of grouped conv2d (kernel size ``kernel_hw`` = (kH, kW)), in w's layout."""
+    x, dy = _f64(x), _f64(dy)
+    w_shape = _wgrad_w_shape(x.shape, dy.shape, kernel_hw, groups, layout)
+    dims, _ = _bwd_dims(dy.shape, w_shape, _hw(x.shape, layout), stride, pad, dilation, groups,
+                        layout)
+    dw = np.empty(w_shape)
+    if _load().oracle_conv2d_bwd_weight(_ptr(x), _ptr(dy), _ptr(dw), *dims, stride, pad,
+                                        dilation, groups, layout) != 0:
+        raise ValueError("oracle_conv2d_bwd_weight rejected the shape")
+    return dw
+
+
+def conv2d_bwd_weight_points(x, dy, kernel_hw, idx, stride=1, pad=0, dilation=1, groups=1,
+                             layout=NCHW):
+    """dw at idx[i] = (co, ci, kh, kw) (logical indices, ci within the group)."""
+    x, dy = _f64(x), _f64(dy)
+    w_shape = _wgrad_w_shape(x.shape, dy.shape, kernel_hw, groups, layout)
+    dims, _ = _bwd_dims(dy.shape, w_shape, _hw(x.shape, layout), stride, pad, dilation, groups,
+                        layout)
+    idx = np.ascontiguousarray(idx, dtype=np.int64).reshape(-1, 4)
+    out = np.empty(idx.shape[0])
+    if _load().oracle_conv2d_bwd_weight_points(_ptr(x), _ptr(dy), _ptr(out), _ptr(idx),
+                                               idx.shape[0], *dims, stride, pad, dilation,
+                                               groups, layout) != 0:
+        raise ValueError("oracle_conv2d_bwd_weight_points rejected the shape or an index")
+    return out
+
+
+def _hw(x_shape, layout):
+    return (x_shape[2], x_shape[3]) if layout == NCHW else (x_shape[1], x_shape[2])
+
+
+def _wgrad_w_shape(x_shape, dy_shape, kernel_hw, groups, layout):
+    kH, kW = kernel_hw
+    C_in = x_shape[1] if layout == NCHW else x_shape[3]
+    C_out = dy_shape[1] if layout == NCHW else dy_shape[3]
+    if groups <= 0 or C_in % groups:
+        raise ValueError("inconsistent groups / channel counts")
+    cpg_in = C_in // groups
+    return (C_out, cpg_in, kH, kW) if layout == NCHW else (C_out, kH, kW, cpg_in)
 
 
 def _conv1d_check(x_shape, w_shape):

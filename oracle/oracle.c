@@ -21,6 +21,8 @@
  *    the (batch, steps, channels) layout), plus its backward pass (the Oct 30
  *    comment): data gradient and weight gradient, written as the literal
  *    adjoint (scatter form) of the forward sum.
+ *  - The grouped conv2d's own data and weight gradients, in the same scatter /
+ *    direct-sum forms, for the training uses of grouped layers on the pages.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *  - output size  Ho = floor((H + 2*pad - dil*(kH-1) - 1)/stride) + 1 (PyTorch's
@@ -141,6 +143,138 @@ int oracle_conv2d_points(const double* x, const double* w, const double* bias, d
   for (long i = 0; i < npts; ++i)
     out[i] = conv2d_point(&s, x, w, bias, idx[4 * i], idx[4 * i + 1], idx[4 * i + 2],
                           idx[4 * i + 3]);
+  return 0;
+}
+
+/* ---------------- grouped conv2d backward ---------------- */
+/* The gradients of L = sum over outputs of dy * y for the forward sum of conv2d_point (the
+ * training use of grouped layers on the pages: the Adam-trained ensemble of "Optimize
+ * convolution batching rule performance" and the backward passes timed in the Conformer
+ * thread). dy has the forward output's shape and layout, dx the input's, dw the weight's. */
+
+/* Data gradient, scatter form: each forward term w[co,ci,kh,kw] * x[n,c,h,wi] of output
+ * (n,co,ho,wo) sends w[co,ci,kh,kw] * dy[n,co,ho,wo] back to dx[n,c,h,wi]. Parallel over n,
+ * so the scatter is race-free. */
+int oracle_conv2d_bwd_data(const double* dy, const double* w, double* dx, long N, long C_in,
+                           long H, long W, long C_out, long kH, long kW, long stride, long pad,
+                           long dil, long groups, int layout) {
+  conv2d_shape s;
+  if (make_shape(&s, N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups, layout)) return -1;
+  long cpg_in = C_in / groups, cpg_out = C_out / groups;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long n = 0; n < N; ++n) {
+    for (long c = 0; c < C_in; ++c)
+      for (long h = 0; h < H; ++h)
+        for (long wi = 0; wi < W; ++wi) dx[x_index(&s, n, c, h, wi)] = 0.0;
+    for (long co = 0; co < C_out; ++co) {
+      long g = co / cpg_out;
+      for (long ho = 0; ho < s.Ho; ++ho)
+        for (long wo = 0; wo < s.Wo; ++wo) {
+          double d = dy[y_index(&s, n, co, ho, wo)];
+          for (long ci = 0; ci < cpg_in; ++ci)
+            for (long kh = 0; kh < kH; ++kh) {
+              long h = ho * stride - pad + kh * dil;
+              if (h < 0 || h >= H) continue;
+              for (long kw = 0; kw < kW; ++kw) {
+                long wi = wo * stride - pad + kw * dil;
+                if (wi < 0 || wi >= W) continue;
+                dx[x_index(&s, n, g * cpg_in + ci, h, wi)] += w[w_index(&s, co, ci, kh, kw)] * d;
+              }
+            }
+        }
+    }
+  }
+  return 0;
+}
+
+/* dx at selected input positions idx[4i..4i+3] = (n, c, h, w), gathered: the sum over the
+ * outputs (co in c's group, ho, wo) and taps (kh, kw) whose window reads x[n,c,h,w], i.e.
+ * ho*stride - pad + kh*dil == h and wo*stride - pad + kw*dil == w. */
+int oracle_conv2d_bwd_data_points(const double* dy, const double* w, double* out,
+                                  const int64_t* idx, long npts, long N, long C_in, long H,
+                                  long W, long C_out, long kH, long kW, long stride, long pad,
+                                  long dil, long groups, int layout) {
+  conv2d_shape s;
+  if (make_shape(&s, N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups, layout)) return -1;
+  for (long i = 0; i < npts; ++i) {
+    long n = idx[4 * i], c = idx[4 * i + 1], h = idx[4 * i + 2], wi = idx[4 * i + 3];
+    if (n < 0 || n >= N || c < 0 || c >= C_in || h < 0 || h >= H || wi < 0 || wi >= W) return -1;
+  }
+  long cpg_in = C_in / groups, cpg_out = C_out / groups;
+#pragma omp parallel for schedule(static)
+  for (long i = 0; i < npts; ++i) {
+    long n = idx[4 * i], c = idx[4 * i + 1], h = idx[4 * i + 2], wi = idx[4 * i + 3];
+    long g = c / cpg_in, ci = c % cpg_in;
+    double acc = 0.0;
+    for (long co = g * cpg_out; co < (g + 1) * cpg_out; ++co)
+      for (long kh = 0; kh < kH; ++kh) {
+        long th = h + pad - kh * dil;          /* = ho * stride */
+        if (th < 0 || th % stride != 0 || th / stride >= s.Ho) continue;
+        for (long kw = 0; kw < kW; ++kw) {
+          long tw = wi + pad - kw * dil;       /* = wo * stride */
+          if (tw < 0 || tw % stride != 0 || tw / stride >= s.Wo) continue;
+          acc += w[w_index(&s, co, ci, kh, kw)] * dy[y_index(&s, n, co, th / stride, tw / stride)];
+        }
+      }
+    out[i] = acc;
+  }
+  return 0;
+}
+
+/* One weight-gradient entry: dw[co,ci,kh,kw] = sum over (n, ho, wo) of
+ * dy[n,co,ho,wo] * x[n, g*cpg_in + ci, ho*stride - pad + kh*dil, wo*stride - pad + kw*dil],
+ * summed in (n, ho, wo) order; taps that fall in the padding contribute nothing. */
+static double conv2d_wgrad_entry(const conv2d_shape* s, const double* x, const double* dy,
+                                 long co, long ci, long kh, long kw) {
+  long cpg_in = s->C_in / s->groups, cpg_out = s->C_out / s->groups;
+  long c = (co / cpg_out) * cpg_in + ci;
+  double acc = 0.0;
+  for (long n = 0; n < s->N; ++n)
+    for (long ho = 0; ho < s->Ho; ++ho) {
+      long h = ho * s->stride - s->pad + kh * s->dil;
+      if (h < 0 || h >= s->H) continue;
+      for (long wo = 0; wo < s->Wo; ++wo) {
+        long wi = wo * s->stride - s->pad + kw * s->dil;
+        if (wi < 0 || wi >= s->W) continue;
+        acc += dy[y_index(s, n, co, ho, wo)] * x[x_index(s, n, c, h, wi)];
+      }
+    }
+  return acc;
+}
+
+/* Full weight gradient, dw in the weight layout of `layout`. */
+int oracle_conv2d_bwd_weight(const double* x, const double* dy, double* dw, long N, long C_in,
+                             long H, long W, long C_out, long kH, long kW, long stride, long pad,
+                             long dil, long groups, int layout) {
+  conv2d_shape s;
+  if (make_shape(&s, N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups, layout)) return -1;
+  long cpg_in = C_in / groups;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long co = 0; co < C_out; ++co)
+    for (long ci = 0; ci < cpg_in; ++ci)
+      for (long kh = 0; kh < kH; ++kh)
+        for (long kw = 0; kw < kW; ++kw)
+          dw[w_index(&s, co, ci, kh, kw)] = conv2d_wgrad_entry(&s, x, dy, co, ci, kh, kw);
+  return 0;
+}
+
+/* Selected weight-gradient entries idx[4i..4i+3] = (co, ci, kh, kw). */
+int oracle_conv2d_bwd_weight_points(const double* x, const double* dy, double* out,
+                                    const int64_t* idx, long npts, long N, long C_in, long H,
+                                    long W, long C_out, long kH, long kW, long stride, long pad,
+                                    long dil, long groups, int layout) {
+  conv2d_shape s;
+  if (make_shape(&s, N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups, layout)) return -1;
+  long cpg_in = C_in / groups;
+  for (long i = 0; i < npts; ++i) {
+    long co = idx[4 * i], ci = idx[4 * i + 1], kh = idx[4 * i + 2], kw = idx[4 * i + 3];
+    if (co < 0 || co >= C_out || ci < 0 || ci >= cpg_in || kh < 0 || kh >= kH || kw < 0 || kw >= kW)
+      return -1;
+  }
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long i = 0; i < npts; ++i)
+    out[i] = conv2d_wgrad_entry(&s, x, dy, idx[4 * i], idx[4 * i + 1], idx[4 * i + 2],
+                                idx[4 * i + 3]);
   return 0;
 }
 

@@ -404,6 +404,158 @@ def test_dwconv1d_equals_depthwise_conv2d():
     assert np.array_equal(y2, oracle.dwconv1d_fwd(x, w, 2, 2))
 
 
+# ---------------------------------------------------------------- grouped conv2d backward
+
+def brute_bwd_nchw(x, w, dy, stride, pad, dil, groups):
+    """dx and dw from the independent forward evaluator alone, by linearity: the forward is
+    linear in x and in w, so dx[i] = <brute(e_i, w), dy> and dw[j] = <brute(x, e_j), dy> for
+    the unit tensors e_i, e_j (integers, exact)."""
+    dyi = np.asarray(dy).astype(np.int64)
+    dx = np.zeros(x.shape, np.int64)
+    for i in np.ndindex(x.shape):
+        e = np.zeros(x.shape)
+        e[i] = 1
+        dx[i] = np.sum(brute_conv2d_nchw(e, w, stride, pad, dil, groups) * dyi)
+    dw = np.zeros(w.shape, np.int64)
+    for j in np.ndindex(w.shape):
+        e = np.zeros(w.shape)
+        e[j] = 1
+        dw[j] = np.sum(brute_conv2d_nchw(x, e, stride, pad, dil, groups) * dyi)
+    return dx, dw
+
+
+def _bwd_grads(x, w, dy, s, p, d, g, layout):
+    """Oracle dx, dw for NCHW tensors, run in `layout` and returned as NCHW."""
+    H, W = x.shape[2], x.shape[3]
+    k = (w.shape[2], w.shape[3])
+    if layout == NCHW:
+        return (oracle.conv2d_bwd_data(dy, w, (H, W), s, p, d, g, NCHW),
+                oracle.conv2d_bwd_weight(x, dy, k, s, p, d, g, NCHW))
+    dx = oracle.conv2d_bwd_data(to_nhwc(dy), to_nhwc(w), (H, W), s, p, d, g, NHWC)
+    dw = oracle.conv2d_bwd_weight(to_nhwc(x), to_nhwc(dy), k, s, p, d, g, NHWC)
+    return from_nhwc(dx), from_nhwc(dw)
+
+
+@pytest.mark.parametrize("case", _tiny_cases()[:20])
+@pytest.mark.parametrize("layout", [NCHW, NHWC])
+def test_conv2d_bwd_brute_force(case, layout):
+    N, C_in, H, W, C_out, (kH, kW), s, p, d, g = case
+    x = rng_int(60, (N, C_in, H, W))
+    w = rng_int(61, (C_out, C_in // g, kH, kW))
+    dy = rng_int(62, brute_conv2d_nchw(x, w, s, p, d, g).shape)
+    dx_ref, dw_ref = brute_bwd_nchw(x, w, dy, s, p, d, g)
+    dx, dw = _bwd_grads(x, w, dy, s, p, d, g, layout)
+    assert np.array_equal(dx, dx_ref.astype(float))
+    assert np.array_equal(dw, dw_ref.astype(float))
+
+
+BWD_CASES = [
+    # N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups
+    (2, 6, 9, 8, 9, 3, 3, 1, 1, 1, 3),      # cpg_in 2 != cpg_out 3
+    (1, 8, 11, 10, 8, 3, 3, 2, 1, 1, 8),    # depthwise, stride 2, ragged
+    (2, 4, 7, 9, 8, 3, 2, 3, 2, 1, 2),      # stride 3, pad larger than needed
+    (1, 6, 12, 12, 6, 3, 3, 1, 2, 2, 2),    # dilation 2
+    (1, 12, 6, 7, 12, 5, 5, 1, 2, 1, 4),    # 5x5
+    (2, 8, 5, 5, 4, 1, 1, 2, 0, 1, 4),      # 1x1 stride 2: rows / columns nobody reads
+    (1, 4, 4, 4, 4, 3, 3, 1, 3, 1, 1),      # pad 3 > dil*(k-1): border outputs read only padding
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES)
+def test_conv2d_bwd_vs_torch(case):
+    """Library pin: torch's own conv2d input / weight gradients in float64 on the CPU."""
+    import torch
+    N, C_in, H, W, C_out, kH, kW, s, p, d, g = case
+    r = np.random.default_rng(63)
+    x = r.standard_normal((N, C_in, H, W))
+    w = r.standard_normal((C_out, C_in // g, kH, kW))
+    Ho, Wo = n_positions(H, kH, s, p, d), n_positions(W, kW, s, p, d)
+    dy = r.standard_normal((N, C_out, Ho, Wo))
+    tx, tw, tdy = (torch.from_numpy(a) for a in (x, w, dy))
+    dx_ref = torch.nn.grad.conv2d_input(tx.shape, tw, tdy, s, p, d, g).numpy()
+    dw_ref = torch.nn.grad.conv2d_weight(tx, tw.shape, tdy, s, p, d, g).numpy()
+    for layout in (NCHW, NHWC):
+        dx, dw = _bwd_grads(x, w, dy, s, p, d, g, layout)
+        np.testing.assert_allclose(dx, dx_ref, rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(dw, dw_ref, rtol=1e-11, atol=1e-11)
+
+
+@pytest.mark.parametrize("case", BWD_CASES)
+def test_conv2d_bwd_adjoint_identity(case):
+    """<conv2d(x, w), dy> = <x, dx> = <w, dw> against the (separately pinned) forward."""
+    N, C_in, H, W, C_out, kH, kW, s, p, d, g = case
+    r = np.random.default_rng(64)
+    x = r.standard_normal((N, H, W, C_in))
+    w = r.standard_normal((C_out, kH, kW, C_in // g))
+    y = oracle.conv2d(x, w, None, s, p, d, g, NHWC)
+    dy = r.standard_normal(y.shape)
+    a = np.vdot(y, dy)
+    b = np.vdot(x, oracle.conv2d_bwd_data(dy, w, (H, W), s, p, d, g, NHWC))
+    c = np.vdot(w, oracle.conv2d_bwd_weight(x, dy, (kH, kW), s, p, d, g, NHWC))
+    assert abs(a - b) <= 1e-10 * max(1.0, abs(a))
+    assert abs(a - c) <= 1e-10 * max(1.0, abs(a))
+
+
+def test_conv2d_bwd_1x1_is_matmul():
+    """Closed form: for a 1x1, stride-1, unpadded layer, per group dx = W_g^T dy_g and
+    dw_g = sum over pixels of dy_g x_g^T (numpy matmul)."""
+    N, H, W, g, ci, co = 2, 5, 4, 3, 4, 2
+    r = np.random.default_rng(65)
+    x = r.standard_normal((N, H, W, g * ci))
+    w = r.standard_normal((g * co, 1, 1, ci))
+    dy = r.standard_normal((N, H, W, g * co))
+    dx = oracle.conv2d_bwd_data(dy, w, (H, W), 1, 0, 1, g, NHWC)
+    dw = oracle.conv2d_bwd_weight(x, dy, (1, 1), 1, 0, 1, g, NHWC)
+    for j in range(g):
+        Wg = w[j * co:(j + 1) * co, 0, 0, :]                      # [co, ci]
+        dyg = dy[..., j * co:(j + 1) * co].reshape(-1, co)        # [pixels, co]
+        xg = x[..., j * ci:(j + 1) * ci].reshape(-1, ci)          # [pixels, ci]
+        np.testing.assert_allclose(dx[..., j * ci:(j + 1) * ci].reshape(-1, ci), dyg @ Wg,
+                                   rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dw[j * co:(j + 1) * co, 0, 0, :], dyg.T @ xg,
+                                   rtol=1e-12, atol=1e-12)
+
+
+def test_conv2d_bwd_finite_differences():
+    """Central differences of L = <conv2d(x, w), dy> against dx and dw."""
+    N, C_in, H, W, C_out, k, s, p, d, g = 1, 4, 5, 4, 6, 3, 2, 1, 1, 2
+    r = np.random.default_rng(66)
+    x = r.standard_normal((N, C_in, H, W))
+    w = r.standard_normal((C_out, C_in // g, k, k))
+    dy = r.standard_normal(oracle.conv2d(x, w, None, s, p, d, g, NCHW).shape)
+    L = lambda xx, ww: np.vdot(oracle.conv2d(xx, ww, None, s, p, d, g, NCHW), dy)
+    dx = oracle.conv2d_bwd_data(dy, w, (H, W), s, p, d, g, NCHW)
+    dw = oracle.conv2d_bwd_weight(x, dy, (k, k), s, p, d, g, NCHW)
+    h = 1e-6
+    for a, grad, is_x in ((x, dx, True), (w, dw, False)):
+        for i in np.ndindex(a.shape):
+            e = np.zeros_like(a)
+            e[i] = h
+            fd = (L(x + e, w) - L(x - e, w)) if is_x else (L(x, w + e) - L(x, w - e))
+            assert abs(fd / (2 * h) - grad[i]) < 1e-6
+
+
+@pytest.mark.parametrize("case", BWD_CASES)
+@pytest.mark.parametrize("layout", [NCHW, NHWC])
+def test_conv2d_bwd_points_match_full(case, layout):
+    N, C_in, H, W, C_out, kH, kW, s, p, d, g = case
+    x = rng_int(67, (N, C_in, H, W))
+    w = rng_int(68, (C_out, C_in // g, kH, kW))
+    dy = rng_int(69, (N, C_out, n_positions(H, kH, s, p, d), n_positions(W, kW, s, p, d)))
+    dx, dw = _bwd_grads(x, w, dy, s, p, d, g, layout)
+    xi = np.array(list(np.ndindex(dx.shape)))
+    wi = np.array(list(np.ndindex(dw.shape)))
+    if layout == NCHW:
+        px = oracle.conv2d_bwd_data_points(dy, w, (H, W), xi, s, p, d, g, NCHW)
+        pw = oracle.conv2d_bwd_weight_points(x, dy, (kH, kW), wi, s, p, d, g, NCHW)
+    else:
+        px = oracle.conv2d_bwd_data_points(to_nhwc(dy), to_nhwc(w), (H, W), xi, s, p, d, g, NHWC)
+        pw = oracle.conv2d_bwd_weight_points(to_nhwc(x), to_nhwc(dy), (kH, kW), wi, s, p, d, g,
+                                             NHWC)
+    assert np.array_equal(px, dx[tuple(xi.T)])
+    assert np.array_equal(pw, dw[tuple(wi.T)])
+
+
 # ---------------------------------------------------------------- planted mistakes
 
 MUTANTS = {
@@ -419,6 +571,16 @@ MUTANTS = {
                               "dx[(b * T + s) * C + c] += w[c * K + (K - 1 - k)]"),
     "wgrad_sign": ("acc += dy[(b * T_out + t) * C + c] * x[(b * T + s) * C + c];",
                    "acc -= dy[(b * T_out + t) * C + c] * x[(b * T + s) * C + c];"),
+    "conv2d_dgrad_group_offset_dropped": ("dx[x_index(&s, n, g * cpg_in + ci, h, wi)]",
+                                          "dx[x_index(&s, n, ci, h, wi)]"),
+    "conv2d_dgrad_tap_flipped": ("+= w[w_index(&s, co, ci, kh, kw)] * d;",
+                                 "+= w[w_index(&s, co, ci, kH - 1 - kh, kw)] * d;"),
+    "conv2d_wgrad_group_stride": ("long c = (co / cpg_out) * cpg_in + ci;",
+                                  "long c = (co / cpg_out) * cpg_out + ci;"),
+    "conv2d_wgrad_dilation_dropped": ("long wi = wo * s->stride - s->pad + kw * s->dil;\n        if (wi < 0 || wi >= s->W) continue;\n        acc += dy",
+                                      "long wi = wo * s->stride - s->pad + kw;\n        if (wi < 0 || wi >= s->W) continue;\n        acc += dy"),
+    "conv2d_dgrad_points_stride_check": ("if (th < 0 || th % stride != 0 || th / stride >= s.Ho)",
+                                         "if (th < 0 || th / stride >= s.Ho)"),
 }
 
 
@@ -432,6 +594,10 @@ def _pins_pass():
             test_dwconv1d_fwd_brute_force(*args)
             test_dwconv1d_library_pins(*args)
         test_group_order_golden()
+        for case in _tiny_cases()[:20]:
+            test_conv2d_bwd_brute_force(case, NHWC)
+        for case in BWD_CASES:
+            test_conv2d_bwd_points_match_full(case, NCHW)
     except AssertionError:
         return False
     return True
