@@ -306,6 +306,57 @@ def depthwise_measurements(torch, gb, device, stream, pk, reps):
     return out
 
 
+def backward_measurements(torch, gb, device, stream, pk, reps):
+    """The grouped conv2d's data and weight gradients on the depthwise 56x56x1024 layer
+    (strides 1 and 2) and the wide-group layer, L2 flushed before each launch. Algorithmic
+    bytes: dgrad dy + w + dx, wgrad x + dy + dw (the workspace partials are reported apart);
+    FLOPs as the forward."""
+    flush = l2_flusher(torch, device)
+    out = {}
+    cases = [("depthwise56_s1", wl.depthwise_56(1), reps), ("depthwise56_s2", wl.depthwise_56(2), reps),
+             ("wide_group_nhwc", wl.wide_group(wl.NHWC), reps)]
+    for tag, p, r in cases:
+        inp = wl.make_conv2d_inputs(p, 5)
+        x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
+        dy = dev_tensor(torch, wl.make_conv2d_dy(p, 5), p.dtype, device)
+        dx = torch.empty(p.x_shape, dtype=torch.bfloat16, device=device)
+        dw = torch.empty(p.w_shape, dtype=torch.bfloat16, device=device)
+        dims = (p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride, p.pad, p.dilation,
+                p.groups, p.layout, p.dtype, gb.PATH_AUTO)
+        wsd = torch.empty(max(gb.gconv2d_bwd_data_workspace_size(*dims), 16), dtype=torch.uint8,
+                          device=device)
+        wsw_n = gb.gconv2d_bwd_weight_workspace_size(*dims)
+        wsw = torch.empty(max(wsw_n, 16), dtype=torch.uint8, device=device)
+        ops = {
+            "dgrad": (lambda i: gb.gconv2d_bwd_data(dy, w, (p.H, p.W), p.stride, p.pad,
+                                                    p.dilation, p.groups, p.layout, out=dx,
+                                                    workspace=wsd, stream=stream),
+                      gb.KERNEL_NAMES.get(gb.gconv2d_bwd_data_select_path(*dims))),
+            "wgrad": (lambda i: gb.gconv2d_bwd_weight(x, dy, (p.kH, p.kW), p.stride, p.pad,
+                                                      p.dilation, p.groups, p.layout, out=dw,
+                                                      workspace=wsw, stream=stream),
+                      gb.KERNEL_NAMES.get(gb.gconv2d_bwd_weight_select_path(*dims))),
+        }
+        for op, (fn, kname) in ops.items():
+            fn(0)
+            torch.cuda.synchronize()
+            n = r if not (tag.startswith("wide") and op == "wgrad") else 3
+            med, mean = time_launches(torch, fn, stream, n, flush)
+            t_tensor = p.flops() / (pk["bf16_tflops"] * 1e12)
+            t_hbm = p.bytes() / (pk["hbm_gbs"] * 1e9)
+            bound = "tensor" if t_tensor >= t_hbm else "hbm"
+            rec = {"kernel": kname, "us": round(med * 1e3, 2),
+                   "TFLOP/s": round(p.flops() / (med * 1e-3) / 1e12, 1),
+                   "GB/s": round(p.bytes() / (med * 1e-3) / 1e9, 1), "bound": bound,
+                   "frac": round(max(t_tensor, t_hbm) / (med * 1e-3), 3),
+                   "alg_bytes": p.bytes(), "alg_flops": p.flops()}
+            if op == "wgrad":
+                rec["workspace_bytes"] = wsw_n
+            out[f"{tag}_{op}"] = rec
+        del x, w, dy, dx, dw, wsd, wsw
+    return out
+
+
 # ---------------------------------------------------------------------------- CPU oracle
 
 def oracle_sample(p, inp_x64, inp_w64, target_s: float):
@@ -374,7 +425,8 @@ def config_dict(p, args):
 # ---------------------------------------------------------------------------- main
 
 PROFILE_WORKLOADS = ("wide_group_nhwc", "wide_group_nchw", "ensemble_g64", "depthwise56_s1",
-                     "depthwise56_s2", "dw1d_same", "sweep56_g64", "sweep56_g16")
+                     "depthwise56_s2", "dw1d_same", "sweep56_g64", "sweep56_g16",
+                     "depthwise56_bwd", "wide_group_dgrad")
 
 
 def run_profile(name: str, reps: int) -> int:
@@ -391,6 +443,17 @@ def run_profile(name: str, reps: int) -> int:
             gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right)
             gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right)
             gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right)
+    elif name in ("depthwise56_bwd", "wide_group_dgrad"):
+        p = wl.depthwise_56(1) if name == "depthwise56_bwd" else wl.wide_group(wl.NHWC)
+        inp = wl.make_conv2d_inputs(p, 5)
+        x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
+        dy = dev_tensor(torch, wl.make_conv2d_dy(p, 5), p.dtype, device)
+        for _ in range(reps):
+            gb.gconv2d_bwd_data(dy, w, (p.H, p.W), p.stride, p.pad, p.dilation, p.groups,
+                                p.layout)
+            if name == "depthwise56_bwd":
+                gb.gconv2d_bwd_weight(x, dy, (p.kH, p.kW), p.stride, p.pad, p.dilation,
+                                      p.groups, p.layout)
     else:
         p = {"wide_group_nhwc": lambda: wl.wide_group(wl.NHWC),
              "wide_group_nchw": lambda: wl.wide_group(wl.NCHW),
@@ -562,9 +625,11 @@ def main():
 
     dwm = None
     more = None
+    bwd = None
     if not args.no_depthwise and rank == 0:
         dwm = depthwise_measurements(torch, gb, device, stream, pk, 20)
         more = more_conv2d_measurements(torch, gb, device, stream, pk, 10)
+        bwd = backward_measurements(torch, gb, device, stream, pk, 10)
     dev_err = gb.device_error(stream)
 
     cpu = None
@@ -584,7 +649,7 @@ def main():
             "kernel": kernel_name(kcode), "roofline": roof, "e2e": e2e,
             "gpu_launches": LAUNCHES_PER_CALL.get(kcode, 1) * args.steps,
             "clocks": clk.summary(), "cpu_baseline": cpu, "depthwise": dwm,
-            "other_workloads": more,
+            "other_workloads": more, "backward": bwd,
             "device_error": dev_err,
             "peaks": {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
                       "source": peak_src},

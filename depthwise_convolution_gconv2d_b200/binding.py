@@ -25,13 +25,17 @@ NCHW, NHWC = 0, 1
 F32, F16, BF16 = 0, 1, 2
 PATH_AUTO, PATH_DIRECT, PATH_IGEMM, PATH_GENERIC = 0, 1, 2, 3
 KERNEL_NAMES = {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "igemm_tc_nchw",
-                5: "conv1d_generic", 6: "conv1d_ring", 7: "conv1d_tc", 8: "grouped_nhwc"}
+                5: "conv1d_generic", 6: "conv1d_ring", 7: "conv1d_tc", 8: "grouped_nhwc",
+                9: "dgrad_generic", 10: "wgrad_generic", 11: "wgrad_depthwise_nhwc"}
 STATUS = {0: "GCONV_OK", 1: "GCONV_ERR_INVALID_ARG", 2: "GCONV_ERR_UNSUPPORTED",
           3: "GCONV_ERR_MISALIGNED", 4: "GCONV_ERR_WORKSPACE", 5: "GCONV_ERR_CUDA",
           6: "GCONV_ERR_DEVICE_TIMEOUT"}
 
 EXPORTS = ["gconv2d_fwd", "gconv2d_fwd_path", "gconv2d_fwd_workspace_size",
-           "gconv2d_select_path", "dwconv1d_fwd", "dwconv1d_bwd_data", "dwconv1d_fwd_path",
+           "gconv2d_select_path", "gconv2d_bwd_data", "gconv2d_bwd_data_path",
+           "gconv2d_bwd_data_workspace_size", "gconv2d_bwd_data_select_path",
+           "gconv2d_bwd_weight", "gconv2d_bwd_weight_path", "gconv2d_bwd_weight_workspace_size",
+           "gconv2d_bwd_weight_select_path", "dwconv1d_fwd", "dwconv1d_bwd_data", "dwconv1d_fwd_path",
            "dwconv1d_bwd_data_path", "dwconv1d_select_path",
            "dwconv1d_bwd_weight", "dwconv1d_bwd_weight_workspace_size",
            "dwconv1d_bwd_weight_noalloc",
@@ -72,6 +76,18 @@ def load_library():
     lib.gconv2d_fwd_path.restype = I
     lib.gconv2d_select_path.argtypes = conv + [I, I, I]
     lib.gconv2d_select_path.restype = I
+    for name in ("gconv2d_bwd_data", "gconv2d_bwd_weight"):
+        getattr(lib, name).argtypes = [P, P, P] + conv + [I, I, P, Z, P]
+        getattr(lib, name).restype = I
+    for name in ("gconv2d_bwd_data_path", "gconv2d_bwd_weight_path"):
+        getattr(lib, name).argtypes = [P, P, P] + conv + [I, I, I, P, Z, P]
+        getattr(lib, name).restype = I
+    for name in ("gconv2d_bwd_data_workspace_size", "gconv2d_bwd_weight_workspace_size"):
+        getattr(lib, name).argtypes = conv + [I, I, I]
+        getattr(lib, name).restype = Z
+    for name in ("gconv2d_bwd_data_select_path", "gconv2d_bwd_weight_select_path"):
+        getattr(lib, name).argtypes = conv + [I, I, I]
+        getattr(lib, name).restype = I
     lib.dwconv1d_fwd.argtypes = [P, P, P] + [I] * 6 + [I, P]
     lib.dwconv1d_fwd.restype = I
     lib.dwconv1d_bwd_data.argtypes = [P, P, P] + [I] * 6 + [I, P]
@@ -197,6 +213,118 @@ def gconv2d_fwd(x, w, bias=None, stride=1, padding=0, dilation=1, groups=1, layo
                               _stream(stream))
     _check(st, "gconv2d_fwd")
     return y
+
+
+def _bwd_dims(dy, w, in_hw, stride, padding, dilation, groups, layout):
+    """(layout code, forward dims, x shape) for a backward call; checks dy's shape."""
+    lay = _layout_code(layout)
+    H, W = in_hw
+    if lay == NCHW:
+        N, C_out = dy.shape[0], dy.shape[1]
+        C_out2, cpg_in, kH, kW = w.shape
+    else:
+        N, C_out = dy.shape[0], dy.shape[3]
+        C_out2, kH, kW, cpg_in = w.shape
+    if C_out2 != C_out:
+        raise ValueError(f"w has {C_out2} filters; dy has {C_out} channels")
+    C_in = cpg_in * groups
+    Ho = _out_extent(H, kH, stride, padding, dilation)
+    Wo = _out_extent(W, kW, stride, padding, dilation)
+    want = (N, C_out, Ho, Wo) if lay == NCHW else (N, Ho, Wo, C_out)
+    if tuple(dy.shape) != want:
+        raise ValueError(f"dy has shape {tuple(dy.shape)}, expected {want}")
+    x_shape = (N, C_in, H, W) if lay == NCHW else (N, H, W, C_in)
+    return lay, (N, C_in, H, W, C_out, kH, kW), x_shape
+
+
+def _workspace(need, workspace, device):
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    return workspace, 0 if workspace is None else workspace.numel() * workspace.element_size()
+
+
+def gconv2d_bwd_data_workspace_size(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation,
+                                    groups, layout, dtype, path=PATH_AUTO) -> int:
+    return int(load_library().gconv2d_bwd_data_workspace_size(
+        N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, _layout_code(layout),
+        dtype if isinstance(dtype, int) else _dtype_code(dtype), path))
+
+
+def gconv2d_bwd_data_select_path(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation,
+                                 groups, layout, dtype, path=PATH_AUTO) -> int:
+    return int(load_library().gconv2d_bwd_data_select_path(
+        N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, _layout_code(layout),
+        dtype if isinstance(dtype, int) else _dtype_code(dtype), path))
+
+
+def gconv2d_bwd_weight_workspace_size(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation,
+                                      groups, layout, dtype, path=PATH_AUTO) -> int:
+    return int(load_library().gconv2d_bwd_weight_workspace_size(
+        N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, _layout_code(layout),
+        dtype if isinstance(dtype, int) else _dtype_code(dtype), path))
+
+
+def gconv2d_bwd_weight_select_path(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation,
+                                   groups, layout, dtype, path=PATH_AUTO) -> int:
+    return int(load_library().gconv2d_bwd_weight_select_path(
+        N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, _layout_code(layout),
+        dtype if isinstance(dtype, int) else _dtype_code(dtype), path))
+
+
+def gconv2d_bwd_data(dy, w, in_hw, stride=1, padding=0, dilation=1, groups=1, layout="NCHW",
+                     out=None, workspace=None, path=PATH_AUTO, stream=None):
+    """Data gradient of grouped conv2d through the C ABI: dy, w -> dx (input size in_hw)."""
+    lib = load_library()
+    _need(dy, "dy")
+    _need(w, "w", dy.dtype)
+    lay, dims, x_shape = _bwd_dims(dy, w, in_hw, stride, padding, dilation, groups, layout)
+    dt = _dtype_code(dy.dtype)
+    dx = torch.empty(x_shape, dtype=dy.dtype, device=dy.device) if out is None else out
+    _need(dx, "out", dy.dtype)
+    if tuple(dx.shape) != x_shape:
+        raise ValueError(f"out has shape {tuple(dx.shape)}, expected {x_shape}")
+    need = lib.gconv2d_bwd_data_workspace_size(*dims, stride, padding, dilation, groups, lay, dt,
+                                               path)
+    workspace, ws_bytes = _workspace(need, workspace, dy.device)
+    st = lib.gconv2d_bwd_data_path(_ptr(dy), _ptr(w), _ptr(dx), *dims, stride, padding,
+                                   dilation, groups, lay, dt, path, _ptr(workspace), ws_bytes,
+                                   _stream(stream))
+    _check(st, "gconv2d_bwd_data")
+    return dx
+
+
+def gconv2d_bwd_weight(x, dy, kernel_hw, stride=1, padding=0, dilation=1, groups=1,
+                       layout="NCHW", out=None, workspace=None, path=PATH_AUTO, stream=None):
+    """Weight gradient of grouped conv2d through the C ABI: x, dy -> dw (kernel kernel_hw)."""
+    lib = load_library()
+    _need(x, "x")
+    _need(dy, "dy", x.dtype)
+    lay = _layout_code(layout)
+    kH, kW = kernel_hw
+    C_in = x.shape[1] if lay == NCHW else x.shape[3]
+    C_out = dy.shape[1] if lay == NCHW else dy.shape[3]
+    if groups <= 0 or C_in % groups:
+        raise ValueError(f"{C_in} input channels do not split into {groups} groups")
+    cpg_in = C_in // groups
+    w_shape = (C_out, cpg_in, kH, kW) if lay == NCHW else (C_out, kH, kW, cpg_in)
+    in_hw = (x.shape[2], x.shape[3]) if lay == NCHW else (x.shape[1], x.shape[2])
+    _, dims, x_shape = _bwd_dims(dy, torch.empty(w_shape, device="meta"), in_hw, stride,
+                                 padding, dilation, groups, lay)
+    if tuple(x.shape) != x_shape:
+        raise ValueError(f"x has shape {tuple(x.shape)}, expected {x_shape}")
+    dt = _dtype_code(x.dtype)
+    dw = torch.empty(w_shape, dtype=x.dtype, device=x.device) if out is None else out
+    _need(dw, "out", x.dtype)
+    if tuple(dw.shape) != w_shape:
+        raise ValueError(f"out has shape {tuple(dw.shape)}, expected {w_shape}")
+    need = lib.gconv2d_bwd_weight_workspace_size(*dims, stride, padding, dilation, groups, lay,
+                                                 dt, path)
+    workspace, ws_bytes = _workspace(need, workspace, x.device)
+    st = lib.gconv2d_bwd_weight_path(_ptr(x), _ptr(dy), _ptr(dw), *dims, stride, padding,
+                                     dilation, groups, lay, dt, path, _ptr(workspace), ws_bytes,
+                                     _stream(stream))
+    _check(st, "gconv2d_bwd_weight")
+    return dw
 
 
 def _conv1d_dims(x, w):

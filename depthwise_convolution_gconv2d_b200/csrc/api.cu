@@ -117,6 +117,100 @@ int choose_kernel(const Conv2d& p, int path, const void* x, const void* w, const
 
 gconv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GCONV_OK : GCONV_ERR_CUDA; }
 
+// Launches forward kernel `kernel` on a validated problem (workspace checked here for NCHW
+// tensor-core staging).
+gconv_status launch_forward(int kernel, const Conv2d& p, const void* x, const void* w,
+                            const void* bias, void* y, void* workspace, size_t workspace_bytes,
+                            cudaStream_t s) {
+  switch (kernel) {
+    case GCONV_KERNEL_DEPTHWISE_NHWC:
+      return cuda_status(launch_depthwise_nhwc(p, x, w, bias, y, s));
+    case GCONV_KERNEL_GROUPED_NHWC:
+      return cuda_status(launch_grouped_nhwc(p, x, w, bias, y, s));
+    case GCONV_KERNEL_IGEMM_TC:
+      return cuda_status(launch_igemm_nhwc(p, x, w, bias, y, s));
+    case GCONV_KERNEL_IGEMM_TC_NCHW: {
+      const size_t need = igemm_nchw_workspace(p);
+      if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+        return GCONV_ERR_WORKSPACE;
+      return cuda_status(launch_igemm_nchw(p, x, w, bias, y, workspace, s));
+    }
+    default:
+      return cuda_status(launch_direct_generic(p, x, w, bias, y, s));
+  }
+}
+
+// ------------------------------------------------------------------ conv2d backward dispatch
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t weight_bytes(const Conv2d& p) {
+  return (size_t)p.C_out * p.cpg_in * p.kH * p.kW * (p.dtype == GCONV_F32 ? 4 : 2);
+}
+
+// The forward problem whose output is the data gradient (valid when dgrad_as_forward(p)):
+// input dy (C_out channels, Ho x Wo), output dx (C_in channels, H x W), stride 1,
+// pad' = dil*(k-1) - pad.
+gconv_status exchanged_problem(const Conv2d& p, Conv2d* q) {
+  return make_conv2d(q, p.N, p.C_out, p.Ho, p.Wo, p.C_in, p.kH, p.kW, 1,
+                     p.dil * (p.kH - 1) - p.pad, p.dil, p.groups, p.layout, p.dtype);
+}
+
+// Kernel for a data-gradient call: a forward kernel code (run on the exchanged problem with
+// the flipped, transposed filter) or GCONV_KERNEL_DGRAD_GENERIC. `wt` is where that filter
+// will be (the workspace); all of dy, wt, dx null = query mode.
+int dgrad_choose(const Conv2d& p, int path, const void* dy, const void* wt, const void* dx,
+                 gconv_status* why, Conv2d* q) {
+  *why = GCONV_OK;
+  const bool via = dgrad_as_forward(p) && exchanged_problem(p, q) == GCONV_OK;
+  switch (path) {
+    case GCONV_PATH_GENERIC:
+      return GCONV_KERNEL_DGRAD_GENERIC;
+    case GCONV_PATH_AUTO:
+    case GCONV_PATH_DIRECT: {
+      if (!via || (path == GCONV_PATH_AUTO && p.dtype == GCONV_F32))
+        return GCONV_KERNEL_DGRAD_GENERIC;
+      const int k = choose_kernel(*q, path, dy, wt, dx, why);
+      return (k < 0 || k == GCONV_KERNEL_DIRECT_GENERIC) ? GCONV_KERNEL_DGRAD_GENERIC : k;
+    }
+    case GCONV_PATH_IGEMM:
+      if (!via) { *why = GCONV_ERR_UNSUPPORTED; return -1; }
+      return choose_kernel(*q, path, dy, wt, dx, why);
+    default:
+      *why = GCONV_ERR_INVALID_ARG;
+      return -1;
+  }
+}
+
+size_t dgrad_workspace(const Conv2d& p, const Conv2d& q, int kernel) {
+  if (kernel == GCONV_KERNEL_DGRAD_GENERIC) return 0;
+  const size_t fwd = kernel == GCONV_KERNEL_IGEMM_TC_NCHW ? igemm_nchw_workspace(q) : 0;
+  return round_up(weight_bytes(p), 256) + fwd;
+}
+
+bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
+
+int wgrad_choose(const Conv2d& p, int path, const void* x, const void* dy, gconv_status* why) {
+  *why = GCONV_OK;
+  const bool query = x == nullptr && dy == nullptr;
+  const bool dw_ok = wgrad_depthwise_supported(p) && (query || (aligned4(x) && aligned4(dy)));
+  switch (path) {
+    case GCONV_PATH_GENERIC:
+      return GCONV_KERNEL_WGRAD_GENERIC;
+    case GCONV_PATH_AUTO:
+    case GCONV_PATH_DIRECT:
+      return dw_ok ? GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC : GCONV_KERNEL_WGRAD_GENERIC;
+    case GCONV_PATH_IGEMM:
+      *why = GCONV_ERR_UNSUPPORTED;   // no tensor-core weight gradient
+      return -1;
+    default:
+      *why = GCONV_ERR_INVALID_ARG;
+      return -1;
+  }
+}
+
+// The weight gradient's row slices are ints on the device.
+bool wgrad_rows_ok(const Conv2d& p) { return (long long)p.N * p.Ho <= (1LL << 30); }
+
 gconv_status make_conv1d(Conv1d* p, int B, int T, int C, int K, int pl, int pr, int dtype) {
   if (B < 0 || T <= 0 || C <= 0 || K <= 0 || pl < 0 || pr < 0) return GCONV_ERR_INVALID_ARG;
   if (dtype != GCONV_F32 && dtype != GCONV_F16 && dtype != GCONV_BF16) return GCONV_ERR_INVALID_ARG;
@@ -172,23 +266,8 @@ gconv_status gconv2d_fwd_path(const void* x, const void* w, const void* bias, vo
   const int kernel = choose_kernel(p, path, x, w, y, &st);
   if (kernel < 0) return st;
   if (N == 0) return GCONV_OK;
-  cudaStream_t s = (cudaStream_t)stream;
-  switch (kernel) {
-    case GCONV_KERNEL_DEPTHWISE_NHWC:
-      return cuda_status(launch_depthwise_nhwc(p, x, w, bias, y, s));
-    case GCONV_KERNEL_GROUPED_NHWC:
-      return cuda_status(launch_grouped_nhwc(p, x, w, bias, y, s));
-    case GCONV_KERNEL_IGEMM_TC:
-      return cuda_status(launch_igemm_nhwc(p, x, w, bias, y, s));
-    case GCONV_KERNEL_IGEMM_TC_NCHW: {
-      const size_t need = igemm_nchw_workspace(p);
-      if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
-        return GCONV_ERR_WORKSPACE;
-      return cuda_status(launch_igemm_nchw(p, x, w, bias, y, workspace, s));
-    }
-    default:
-      return cuda_status(launch_direct_generic(p, x, w, bias, y, s));
-  }
+  return launch_forward(kernel, p, x, w, bias, y, workspace, workspace_bytes,
+                        (cudaStream_t)stream);
 }
 
 gconv_status gconv2d_fwd(const void* x, const void* w, const void* bias, void* y, int N,
@@ -198,6 +277,121 @@ gconv_status gconv2d_fwd(const void* x, const void* w, const void* bias, void* y
   return gconv2d_fwd_path(x, w, bias, y, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation,
                           groups, layout, dtype, GCONV_PATH_AUTO, workspace, workspace_bytes,
                           stream);
+}
+
+size_t gconv2d_bwd_data_workspace_size(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                       int stride, int pad, int dilation, int groups,
+                                       gconv_layout layout, gconv_dtype dtype, gconv_path path) {
+  Conv2d p, q;
+  if (make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups, layout,
+                  dtype) != GCONV_OK)
+    return 0;
+  gconv_status why;
+  const int k = dgrad_choose(p, path, nullptr, nullptr, nullptr, &why, &q);
+  return k < 0 ? 0 : dgrad_workspace(p, q, k);
+}
+
+int gconv2d_bwd_data_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                 int stride, int pad, int dilation, int groups,
+                                 gconv_layout layout, gconv_dtype dtype, gconv_path path) {
+  Conv2d p, q;
+  gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups,
+                                layout, dtype);
+  if (st != GCONV_OK) return -(int)st;
+  const int k = dgrad_choose(p, path, nullptr, nullptr, nullptr, &st, &q);
+  return k < 0 ? -(int)st : k;
+}
+
+gconv_status gconv2d_bwd_data_path(const void* dy, const void* w, void* dx, int N, int C_in,
+                                   int H, int W, int C_out, int kH, int kW, int stride, int pad,
+                                   int dilation, int groups, gconv_layout layout,
+                                   gconv_dtype dtype, gconv_path path, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  Conv2d p, q;
+  gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups,
+                                layout, dtype);
+  if (st != GCONV_OK) return st;
+  if (N > 0 && (dy == nullptr || w == nullptr || dx == nullptr)) return GCONV_ERR_INVALID_ARG;
+  // the flipped filter goes to the start of the workspace; a forward staging area follows it
+  const bool ws_al = workspace != nullptr && aligned16(workspace);
+  const void* wt = ws_al ? workspace : nullptr;
+  const int kernel = N > 0 ? dgrad_choose(p, path, dy, wt, dx, &st, &q)
+                           : dgrad_choose(p, path, nullptr, nullptr, nullptr, &st, &q);
+  if (kernel < 0) return st;
+  if (N == 0) return GCONV_OK;
+  const size_t need = dgrad_workspace(p, q, kernel);
+  if (need > 0 && (!ws_al || workspace_bytes < need)) return GCONV_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (kernel == GCONV_KERNEL_DGRAD_GENERIC)
+    return cuda_status(launch_dgrad_generic(p, dy, w, dx, s));
+  st = cuda_status(launch_flip_transpose_weight(p, w, workspace, s));
+  if (st != GCONV_OK) return st;
+  const size_t off = round_up(weight_bytes(p), 256);
+  return launch_forward(kernel, q, dy, workspace, nullptr, dx, (char*)workspace + off,
+                        workspace_bytes - off, s);
+}
+
+gconv_status gconv2d_bwd_data(const void* dy, const void* w, void* dx, int N, int C_in, int H,
+                              int W, int C_out, int kH, int kW, int stride, int pad,
+                              int dilation, int groups, gconv_layout layout, gconv_dtype dtype,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  return gconv2d_bwd_data_path(dy, w, dx, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation,
+                               groups, layout, dtype, GCONV_PATH_AUTO, workspace,
+                               workspace_bytes, stream);
+}
+
+size_t gconv2d_bwd_weight_workspace_size(int N, int C_in, int H, int W, int C_out, int kH,
+                                         int kW, int stride, int pad, int dilation, int groups,
+                                         gconv_layout layout, gconv_dtype dtype,
+                                         gconv_path path) {
+  Conv2d p;
+  if (make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups, layout,
+                  dtype) != GCONV_OK || !wgrad_rows_ok(p))
+    return 0;
+  gconv_status why;
+  const int k = wgrad_choose(p, path, nullptr, nullptr, &why);
+  return k < 0 ? 0 : wgrad_workspace(p, k);
+}
+
+int gconv2d_bwd_weight_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                   int stride, int pad, int dilation, int groups,
+                                   gconv_layout layout, gconv_dtype dtype, gconv_path path) {
+  Conv2d p;
+  gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups,
+                                layout, dtype);
+  if (st != GCONV_OK) return -(int)st;
+  if (!wgrad_rows_ok(p)) return -(int)GCONV_ERR_UNSUPPORTED;
+  const int k = wgrad_choose(p, path, nullptr, nullptr, &st);
+  return k < 0 ? -(int)st : k;
+}
+
+gconv_status gconv2d_bwd_weight_path(const void* x, const void* dy, void* dw, int N, int C_in,
+                                     int H, int W, int C_out, int kH, int kW, int stride,
+                                     int pad, int dilation, int groups, gconv_layout layout,
+                                     gconv_dtype dtype, gconv_path path, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  Conv2d p;
+  gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups,
+                                layout, dtype);
+  if (st != GCONV_OK) return st;
+  if (dw == nullptr || (N > 0 && (x == nullptr || dy == nullptr))) return GCONV_ERR_INVALID_ARG;
+  if (!wgrad_rows_ok(p)) return GCONV_ERR_UNSUPPORTED;
+  const int kernel = N > 0 ? wgrad_choose(p, path, x, dy, &st)
+                           : wgrad_choose(p, path, nullptr, nullptr, &st);
+  if (kernel < 0) return st;
+  const size_t need = wgrad_workspace(p, kernel);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return GCONV_ERR_WORKSPACE;
+  return cuda_status(launch_wgrad(p, x, dy, dw, workspace, kernel, (cudaStream_t)stream));
+}
+
+gconv_status gconv2d_bwd_weight(const void* x, const void* dy, void* dw, int N, int C_in, int H,
+                                int W, int C_out, int kH, int kW, int stride, int pad,
+                                int dilation, int groups, gconv_layout layout, gconv_dtype dtype,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return gconv2d_bwd_weight_path(x, dy, dw, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation,
+                                 groups, layout, dtype, GCONV_PATH_AUTO, workspace,
+                                 workspace_bytes, stream);
 }
 
 gconv_status dwconv1d_fwd_path(const void* x, const void* w, void* y, int B, int T, int C, int K,

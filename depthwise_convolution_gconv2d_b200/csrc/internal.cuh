@@ -111,6 +111,19 @@ cudaError_t launch_igemm_nhwc(const Conv2d& p, const void* x, const void* w, con
 cudaError_t launch_igemm_nchw(const Conv2d& p, const void* x, const void* w, const void* bias,
                               void* y, void* workspace, cudaStream_t s);
 
+// Grouped conv2d backward. dgrad_as_forward: stride 1, square kernel, pad <= dil*(k-1), so the
+// data gradient is the forward conv of the exchanged problem with the flipped, transposed
+// filter that launch_flip_transpose_weight writes (C_out * C_in/g * kH * kW elements).
+bool dgrad_as_forward(const Conv2d& p);
+cudaError_t launch_flip_transpose_weight(const Conv2d& p, const void* w, void* wt,
+                                         cudaStream_t s);
+cudaError_t launch_dgrad_generic(const Conv2d& p, const void* dy, const void* w, void* dx,
+                                 cudaStream_t s);
+bool wgrad_depthwise_supported(const Conv2d& p);
+size_t wgrad_workspace(const Conv2d& p, int kernel);
+cudaError_t launch_wgrad(const Conv2d& p, const void* x, const void* dy, void* dw, void* ws,
+                         int kernel, cudaStream_t s);
+
 bool conv1d_vector_supported(const Conv1d& p);
 // Kernel (GCONV_KERNEL_CONV1D_*) for a forward / data-gradient call under `path`; x, w, y null
 // = a query that assumes aligned pointers. -1 with *why set when the forced family cannot run.

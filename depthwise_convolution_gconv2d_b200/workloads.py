@@ -198,6 +198,15 @@ def make_conv2d_inputs(p: Conv2dProblem, workload: int, x_dist="normal", x_scale
     return Conv2dInputs(p, x, w, b)
 
 
+def make_conv2d_dy(p: Conv2dProblem, workload: int, dist="normal", scale=1.0) -> np.ndarray:
+    """Seeded output gradient dy ~ N(0, scale^2) (or `dist`), storage array in p's y layout."""
+    dy = to_storage(draw(np.random.default_rng(seed_for(workload, "dy")),
+                         (p.N, p.C_out, p.Ho, p.Wo), dist, scale), p.dtype)
+    if p.layout == NHWC:
+        dy = np.ascontiguousarray(dy.transpose(0, 2, 3, 1))
+    return dy
+
+
 @dataclasses.dataclass(frozen=True)
 class Dwconv1dProblem:
     B: int

@@ -19,6 +19,9 @@
  *               with x = 0 outside the image and
  *                 Ho = floor((H + 2*pad - dilation*(kH-1) - 1) / stride) + 1 (same for Wo).
  *
+ *  gconv2d_bwd_*  The grouped conv2d's data and weight gradients (declared below with their
+ *               sums).
+ *
  *  dwconv1d_*   Depthwise conv1d over (batch, steps, channels) with groups = channels, the
  *               Conformer convolution module's depthwise layer ("Investigate custom Triton
  *               kernels for depthwise-separable convolutions in Conformer", speechbrain #2733:
@@ -99,8 +102,14 @@ typedef enum {
                                          K in {3, 5, 7, 9, 15, 31} */
   GCONV_KERNEL_CONV1D_TC = 7,         /* dwconv1d: tcgen05 banded product; 16-bit, C % 16 == 0,
                                          K <= 49 */
-  GCONV_KERNEL_GROUPED_NHWC = 8       /* conv2d, 2 / 4 / 8 channels per group in and out, 3x3,
+  GCONV_KERNEL_GROUPED_NHWC = 8,      /* conv2d, 2 / 4 / 8 channels per group in and out, 3x3,
                                          dilation 1, stride 1 or 2, 16-bit NHWC: CUDA cores */
+  GCONV_KERNEL_DGRAD_GENERIC = 9,     /* conv2d data gradient: one thread per dx element, fp32
+                                         FMA, any problem */
+  GCONV_KERNEL_WGRAD_GENERIC = 10,    /* conv2d weight gradient: one thread per (dw entry,
+                                         slice), fp32 FMA, any problem */
+  GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC = 11  /* conv2d weight gradient, depthwise 3x3 / 5x5,
+                                         dilation 1, stride 1 or 2, 16-bit NHWC, C even */
 } gconv_kernel;
 
 /* Bytes of workspace gconv2d_fwd needs for this problem under `path` (0 if none; also 0 for
@@ -131,6 +140,82 @@ gconv_status gconv2d_fwd_path(const void* x, const void* w, const void* bias, vo
 int gconv2d_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW, int stride,
                         int pad, int dilation, int groups, gconv_layout layout,
                         gconv_dtype dtype, gconv_path path);
+
+/* ---- grouped conv2d backward. Sizes and layouts are those of the forward problem: x
+ * [N][C_in][H][W] / [N][H][W][C_in], w as for gconv2d_fwd, dy with y's shape and layout.
+ * These are the gradients of the forward sum above (the grouped layers on the pages are
+ * trained: the Adam-trained ensemble of "Optimize convolution batching rule performance",
+ * the backward passes timed in the Conformer thread):
+ *   dx[n,c,h,w]      = sum over co in c's group and taps (kh, kw) with
+ *                      h + pad - kh*dilation = ho*stride, w + pad - kw*dilation = wo*stride
+ *                      (0 <= ho < Ho, 0 <= wo < Wo) of w[co, c mod (C_in/g), kh, kw]*dy[n,co,ho,wo]
+ *   dw[co,ci,kh,kw]  = sum over (n, ho, wo) of dy[n,co,ho,wo] *
+ *                      x[n, (co / (C_out/g))*(C_in/g) + ci, ho*stride-pad+kh*dilation,
+ *                        wo*stride-pad+kw*dilation]
+ * with x = 0 outside the image. No bias gradient (it is a plain sum of dy). */
+
+/* Bytes of workspace gconv2d_bwd_data_path needs under `path` (0 if none or invalid). When
+ * the data gradient runs as a forward convolution, this holds the flipped, transposed filter
+ * (C_out * C_in/g * kH * kW elements, rounded up to 256 bytes) followed by the forward
+ * kernel's own workspace. */
+size_t gconv2d_bwd_data_workspace_size(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                       int stride, int pad, int dilation, int groups,
+                                       gconv_layout layout, gconv_dtype dtype, gconv_path path);
+
+/* Data gradient dy, w -> dx (written in full). With stride 1, a square kernel and
+ * pad <= dilation*(k-1) it is computed as the forward convolution of dy with the per-group
+ * transposed, 180-degree-rotated filter and pad' = dilation*(k-1) - pad, on the forward
+ * kernels (AUTO / DIRECT / IGEMM choose among them as gconv2d_fwd_path does, F32 under AUTO
+ * excepted); other problems, fp32 under AUTO and GENERIC run the one-thread-per-element
+ * gather kernel. IGEMM on a problem that cannot run as a forward convolution on the tensor
+ * cores is UNSUPPORTED (or MISALIGNED). The workspace must be 16-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
+gconv_status gconv2d_bwd_data(const void* dy, const void* w, void* dx, int N, int C_in, int H,
+                              int W, int C_out, int kH, int kW, int stride, int pad,
+                              int dilation, int groups, gconv_layout layout, gconv_dtype dtype,
+                              void* workspace, size_t workspace_bytes, void* stream);
+gconv_status gconv2d_bwd_data_path(const void* dy, const void* w, void* dx, int N, int C_in,
+                                   int H, int W, int C_out, int kH, int kW, int stride, int pad,
+                                   int dilation, int groups, gconv_layout layout,
+                                   gconv_dtype dtype, gconv_path path, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/* The gconv_kernel gconv2d_bwd_data_path would run (a forward kernel code, run on the
+ * exchanged problem, or GCONV_KERNEL_DGRAD_GENERIC), assuming aligned pointers; a negative
+ * gconv_status if it would fail. */
+int gconv2d_bwd_data_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                 int stride, int pad, int dilation, int groups,
+                                 gconv_layout layout, gconv_dtype dtype, gconv_path path);
+
+/* Bytes of workspace gconv2d_bwd_weight_path needs: fp32 partial sums, one per dw entry and
+ * slice of the N*Ho output rows (0 if none or invalid). */
+size_t gconv2d_bwd_weight_workspace_size(int N, int C_in, int H, int W, int C_out, int kH,
+                                         int kW, int stride, int pad, int dilation, int groups,
+                                         gconv_layout layout, gconv_dtype dtype,
+                                         gconv_path path);
+
+/* Weight gradient x, dy -> dw (w's shape, layout and dtype; written in full, zeros when
+ * N == 0). Deterministic: the N*Ho output rows are cut into slices fixed by the problem's
+ * sizes alone, each slice's partial sums are added in a fixed order and the slices are added
+ * in slice order (no float atomics), so repeated calls -- on any GPU -- give bitwise-identical
+ * dw. AUTO and DIRECT run the depthwise kernel where it applies (GCONV_KERNEL_WGRAD_DEPTHWISE_
+ * NHWC; x and dy 4-byte aligned), else the generic kernel; GENERIC forces the generic kernel;
+ * IGEMM is UNSUPPORTED (there is no tensor-core weight gradient). N*Ho > 2^30 is UNSUPPORTED.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+gconv_status gconv2d_bwd_weight(const void* x, const void* dy, void* dw, int N, int C_in, int H,
+                                int W, int C_out, int kH, int kW, int stride, int pad,
+                                int dilation, int groups, gconv_layout layout, gconv_dtype dtype,
+                                void* workspace, size_t workspace_bytes, void* stream);
+gconv_status gconv2d_bwd_weight_path(const void* x, const void* dy, void* dw, int N, int C_in,
+                                     int H, int W, int C_out, int kH, int kW, int stride,
+                                     int pad, int dilation, int groups, gconv_layout layout,
+                                     gconv_dtype dtype, gconv_path path, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* The gconv_kernel gconv2d_bwd_weight_path would run, or a negative gconv_status. */
+int gconv2d_bwd_weight_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                   int stride, int pad, int dilation, int groups,
+                                   gconv_layout layout, gconv_dtype dtype, gconv_path path);
 
 /* Depthwise conv1d forward: x [B][T][C], w [C][K] -> y [B][T_out][C].
  * Errors: INVALID_ARG (incl. T_out < 1), CUDA. */

@@ -161,3 +161,73 @@ def test_narrow_group_selection(lib):
         assert sel(0, dil=2, pad=2, **kw) == 1            # dilation: generic
     assert sel(0, C_in=64, C_out=64, groups=4) == 3       # 16 per group: tensor cores
     assert sel(0, C_in=64, C_out=128, groups=16) != 8     # 4 in / 8 out: not narrow-group
+
+
+# ------------------------------------------------------------ conv2d backward (host logic)
+
+def test_bwd_invalid_and_workspace_rejected_before_launch(lib):
+    p = ctypes.c_void_p(0x1000)
+    for over in (dict(groups=3), dict(C_out=6), dict(stride=0), dict(H=1, pad=0)):
+        args = _conv_args(**over)
+        assert lib.gconv2d_bwd_data(p, p, p, *args, 1, 2, None, 0, None) == 1
+        assert lib.gconv2d_bwd_weight(p, p, p, *args, 1, 2, None, 0, None) == 1
+        assert lib.gconv2d_bwd_data_select_path(*args, 1, 2, 0) == -1
+        assert lib.gconv2d_bwd_weight_workspace_size(*args, 1, 2, 0) == 0
+    args = _conv_args(C_in=64, C_out=64, groups=64)
+    assert lib.gconv2d_bwd_data(None, p, p, *args, 1, 2, None, 0, None) == 1
+    assert lib.gconv2d_bwd_weight(p, p, None, *args, 1, 2, None, 0, None) == 1
+    # a kernel that needs workspace, given none (or too little, or unaligned): WORKSPACE
+    need = lib.gconv2d_bwd_data_workspace_size(*args, 1, 2, 0)
+    assert need == 256 * ((64 * 9 * 2 + 255) // 256)
+    assert lib.gconv2d_bwd_data(p, p, p, *args, 1, 2, None, 0, None) == 4
+    assert lib.gconv2d_bwd_data(p, p, p, *args, 1, 2, p, need - 1, None) == 4
+    assert lib.gconv2d_bwd_data(p, p, p, *args, 1, 2, ctypes.c_void_p(0x1004), need, None) == 4
+    assert lib.gconv2d_bwd_weight(p, p, p, *args, 1, 2, None, 0, None) == 4
+    # empty batch: the data gradient has nothing to write
+    assert lib.gconv2d_bwd_data(None, None, None, *_conv_args(N=0), 1, 2, None, 0, None) == 0
+
+
+def test_bwd_path_selection(lib):
+    def sel(fn, N, C_in, H, W, C_out, k, s, pad, d, g, layout=1, dtype=2, path=0):
+        return fn(N, C_in, H, W, C_out, k, k, s, pad, d, g, layout, dtype, path)
+    dg, wg = lib.gconv2d_bwd_data_select_path, lib.gconv2d_bwd_weight_select_path
+    # depthwise 56x56x1024: stride 1 runs the depthwise forward kernel on the flipped filter,
+    # stride 2 the gather kernel; the weight gradient has its own depthwise kernel
+    assert sel(dg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 1024) == 2
+    assert sel(dg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 9
+    assert sel(wg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 1024) == 11
+    assert sel(wg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 11
+    # wide groups: tensor cores (NHWC, NCHW staging); weight gradient generic
+    assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 3
+    assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 4
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 10
+    # narrow groups (4 channels): the narrow-group forward kernel
+    assert sel(dg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 256) == 8
+    # pad beyond dil*(k-1), fp32 under AUTO, and GENERIC: the gather kernel
+    assert sel(dg, 1, 64, 16, 16, 64, 3, 1, 3, 1, 64) == 9
+    assert sel(dg, 1, 64, 16, 16, 64, 3, 1, 1, 1, 64, dtype=0) == 9
+    assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, path=3) == 9
+    # forced IGEMM where the data gradient is not a stride-1 convolution, or on the weight
+    # gradient: UNSUPPORTED
+    assert sel(dg, 1, 512, 64, 64, 512, 3, 2, 1, 1, 4, path=2) == -2
+    assert sel(wg, 1, 512, 64, 64, 512, 3, 1, 1, 1, 4, path=2) == -2
+
+
+def test_bwd_workspace_queries(lib):
+    # the flipped filter (rounded to 256 bytes), plus the NCHW staging of the exchanged problem
+    wt = 512 * 128 * 9 * 2
+    assert lib.gconv2d_bwd_data_workspace_size(1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 1, 2,
+                                               0) == wt
+    assert lib.gconv2d_bwd_data_workspace_size(1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 0, 2,
+                                               0) == wt + lib.gconv2d_fwd_workspace_size(
+        1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 0, 2, 0)
+    # the gather kernel needs none
+    assert lib.gconv2d_bwd_data_workspace_size(32, 1024, 56, 56, 1024, 3, 3, 2, 1, 1, 1024, 1,
+                                               2, 0) == 0
+    # weight gradient: fp32 partials, a whole number of slices of every dw entry
+    for args in [(32, 1024, 56, 56, 1024, 3, 3, 1, 1, 1, 1024, 1, 2, 0),
+                 (1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 1, 2, 0),
+                 (2, 12, 9, 8, 18, 3, 2, 1, 1, 1, 3, 0, 0, 0)]:
+        n = lib.gconv2d_bwd_weight_workspace_size(*args)
+        E = args[4] * (args[1] // args[10]) * args[5] * args[6]
+        assert n > 0 and n % (4 * E) == 0
