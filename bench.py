@@ -23,6 +23,7 @@ on a bounded sample of the same workload, on the host cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -426,11 +427,12 @@ def config_dict(p, args):
 
 PROFILE_WORKLOADS = ("wide_group_nhwc", "wide_group_nchw", "ensemble_g64", "depthwise56_s1",
                      "depthwise56_s2", "dw1d_same", "sweep56_g64", "sweep56_g16",
-                     "depthwise56_bwd", "wide_group_dgrad")
+                     "depthwise56_bwd", "depthwise56_s2_bwd", "wide_group_dgrad")
 
 
-def run_profile(name: str, reps: int) -> int:
-    """--profile: run one workload's launches `reps` times (no timing), for profiler captures."""
+def run_profile(name: str, reps: int, batch: int = 0) -> int:
+    """--profile: run one workload's launches `reps` times (no timing), for profiler captures;
+    `batch` > 0 replaces the conv2d workload's batch size (a smaller capture)."""
     import torch
 
     from depthwise_convolution_gconv2d_b200 import binding as gb
@@ -443,15 +445,19 @@ def run_profile(name: str, reps: int) -> int:
             gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right)
             gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right)
             gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right)
-    elif name in ("depthwise56_bwd", "wide_group_dgrad"):
-        p = wl.depthwise_56(1) if name == "depthwise56_bwd" else wl.wide_group(wl.NHWC)
+    elif name in ("depthwise56_bwd", "depthwise56_s2_bwd", "wide_group_dgrad"):
+        p = {"depthwise56_bwd": lambda: wl.depthwise_56(1),
+             "depthwise56_s2_bwd": lambda: wl.depthwise_56(2),
+             "wide_group_dgrad": lambda: wl.wide_group(wl.NHWC)}[name]()
+        if batch > 0:
+            p = dataclasses.replace(p, N=batch)
         inp = wl.make_conv2d_inputs(p, 5)
         x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
         dy = dev_tensor(torch, wl.make_conv2d_dy(p, 5), p.dtype, device)
         for _ in range(reps):
             gb.gconv2d_bwd_data(dy, w, (p.H, p.W), p.stride, p.pad, p.dilation, p.groups,
                                 p.layout)
-            if name == "depthwise56_bwd":
+            if name != "wide_group_dgrad":
                 gb.gconv2d_bwd_weight(x, dy, (p.kH, p.kW), p.stride, p.pad, p.dilation,
                                       p.groups, p.layout)
     else:
@@ -462,6 +468,8 @@ def run_profile(name: str, reps: int) -> int:
              "depthwise56_s2": lambda: wl.depthwise_56(2),
              "sweep56_g64": lambda: wl.depthwise_56(1, 64),
              "sweep56_g16": lambda: wl.depthwise_56(1, 16)}[name]()
+        if batch > 0:
+            p = dataclasses.replace(p, N=batch)
         inp = wl.make_conv2d_inputs(p, 2)
         x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
         for _ in range(reps):
@@ -487,9 +495,11 @@ def main():
                     help="run this workload's launches --profile-reps times for a profiler "
                          "capture, untimed, and exit")
     ap.add_argument("--profile-reps", type=int, default=2)
+    ap.add_argument("--profile-batch", type=int, default=0,
+                    help="batch size of the --profile conv2d workload (0: the workload's own)")
     args = ap.parse_args()
     if args.profile:
-        return run_profile(args.profile, args.profile_reps)
+        return run_profile(args.profile, args.profile_reps, args.profile_batch)
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         return run_reference(args)

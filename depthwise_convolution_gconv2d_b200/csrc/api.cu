@@ -162,15 +162,21 @@ int dgrad_choose(const Conv2d& p, int path, const void* dy, const void* wt, cons
                  gconv_status* why, Conv2d* q) {
   *why = GCONV_OK;
   const bool via = dgrad_as_forward(p) && exchanged_problem(p, q) == GCONV_OK;
+  const bool query = dy == nullptr && wt == nullptr && dx == nullptr;
+  const int vb = dgrad_depthwise_vec_bytes(p);
+  const bool dwk = dgrad_depthwise_supported(p) &&
+                   (query || (aligned_to(dy, vb) && aligned_to(dx, vb)));
   switch (path) {
     case GCONV_PATH_GENERIC:
       return GCONV_KERNEL_DGRAD_GENERIC;
     case GCONV_PATH_AUTO:
     case GCONV_PATH_DIRECT: {
-      if (!via || (path == GCONV_PATH_AUTO && p.dtype == GCONV_F32))
-        return GCONV_KERNEL_DGRAD_GENERIC;
-      const int k = choose_kernel(*q, path, dy, wt, dx, why);
-      return (k < 0 || k == GCONV_KERNEL_DIRECT_GENERIC) ? GCONV_KERNEL_DGRAD_GENERIC : k;
+      int k = -1;
+      if (via && !(path == GCONV_PATH_AUTO && p.dtype == GCONV_F32))
+        k = choose_kernel(*q, path, dy, wt, dx, why);
+      *why = GCONV_OK;
+      if (k >= 0 && k != GCONV_KERNEL_DIRECT_GENERIC) return k;
+      return dwk ? GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC : GCONV_KERNEL_DGRAD_GENERIC;
     }
     case GCONV_PATH_IGEMM:
       if (!via) { *why = GCONV_ERR_UNSUPPORTED; return -1; }
@@ -182,7 +188,8 @@ int dgrad_choose(const Conv2d& p, int path, const void* dy, const void* wt, cons
 }
 
 size_t dgrad_workspace(const Conv2d& p, const Conv2d& q, int kernel) {
-  if (kernel == GCONV_KERNEL_DGRAD_GENERIC) return 0;
+  if (kernel == GCONV_KERNEL_DGRAD_GENERIC || kernel == GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC)
+    return 0;
   const size_t fwd = kernel == GCONV_KERNEL_IGEMM_TC_NCHW ? igemm_nchw_workspace(q) : 0;
   return round_up(weight_bytes(p), 256) + fwd;
 }
@@ -193,12 +200,14 @@ int wgrad_choose(const Conv2d& p, int path, const void* x, const void* dy, gconv
   *why = GCONV_OK;
   const bool query = x == nullptr && dy == nullptr;
   const bool dw_ok = wgrad_depthwise_supported(p) && (query || (aligned4(x) && aligned4(dy)));
+  const bool tl_ok = wgrad_tiled_supported(p) && (query || (aligned16(x) && aligned16(dy)));
   switch (path) {
     case GCONV_PATH_GENERIC:
       return GCONV_KERNEL_WGRAD_GENERIC;
     case GCONV_PATH_AUTO:
     case GCONV_PATH_DIRECT:
-      return dw_ok ? GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC : GCONV_KERNEL_WGRAD_GENERIC;
+      if (dw_ok) return GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC;
+      return tl_ok ? GCONV_KERNEL_WGRAD_TILED_NHWC : GCONV_KERNEL_WGRAD_GENERIC;
     case GCONV_PATH_IGEMM:
       *why = GCONV_ERR_UNSUPPORTED;   // no tensor-core weight gradient
       return -1;
@@ -324,6 +333,8 @@ gconv_status gconv2d_bwd_data_path(const void* dy, const void* w, void* dx, int 
   cudaStream_t s = (cudaStream_t)stream;
   if (kernel == GCONV_KERNEL_DGRAD_GENERIC)
     return cuda_status(launch_dgrad_generic(p, dy, w, dx, s));
+  if (kernel == GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC)
+    return cuda_status(launch_dgrad_depthwise(p, dy, w, dx, s));
   st = cuda_status(launch_flip_transpose_weight(p, w, workspace, s));
   if (st != GCONV_OK) return st;
   const size_t off = round_up(weight_bytes(p), 256);

@@ -164,17 +164,17 @@ __global__ void __launch_bounds__(256) wgrad_generic_kernel(const T* __restrict_
 
 // ------------------------------------------------------------------ depthwise weight gradient
 // NHWC, 16-bit, K x K (K = 3 or 5), dilation 1, stride S = 1 or 2. A thread owns one channel
-// pair and one slice of (n, ho) rows; its K x K fp32-pair accumulators and the K x K window of
-// input pairs live in registers. Walking along an output row, the window moves S columns:
-// K - S columns are kept and S new ones loaded (one 4-byte load per input row and column, a
-// warp reading 128 contiguous bytes), and one dy pair feeds K*K packed multiply-adds.
-// Partials go to ws[slice][tap][C] (coalesced float2 stores).
-template <typename T, int K, int S>
+// pair and one slice of (n, ho) rows, with its K x K fp32-pair accumulators in registers. It
+// walks each output row in chunks of U columns: first every load of the chunk is issued -- the
+// U dy pairs and the K x ((U-1)*S + K) input pairs they meet (4 bytes a lane, a warp reading
+// 128 contiguous bytes) -- so that a warp has ~40 independent loads in flight, then the chunk's
+// U*K*K packed multiply-adds run. Partials go to ws[slice][tap][C] (coalesced float2 stores).
+template <typename T, int K, int S, int U>
 __global__ void __launch_bounds__(128) wgrad_depthwise_nhwc_kernel(const T* __restrict__ x,
                                                                     const T* __restrict__ dy,
                                                                     float* __restrict__ ws,
                                                                     Conv2d p, int rows) {
-  static_assert(S < K, "the window keeps K - S columns");
+  constexpr int NC = (U - 1) * S + K;         // input columns a chunk reads
   const int CW = p.C_in / 2;                  // channel pairs = 32-bit words per pixel
   const int cp = blockIdx.x * blockDim.x + threadIdx.x;
   if (cp >= CW) return;
@@ -198,32 +198,31 @@ __global__ void __launch_bounds__(128) wgrad_depthwise_nhwc_kernel(const T* __re
       const int h = h0 + kh;
       rb[kh] = (h >= 0 && h < p.H) ? ((long long)n * p.H + h) * p.W * CW + cp : -1;
     }
-    auto load = [&](int kh, int col) -> float2 {
-      if (rb[kh] < 0 || col < 0 || col >= p.W) return make_float2(0.0f, 0.0f);
-      return unpack2<T>(__ldg(xw + rb[kh] + (long long)col * CW));
-    };
-    float2 win[K][K];
-#pragma unroll
-    for (int kh = 0; kh < K; ++kh)
-#pragma unroll
-      for (int kw = 0; kw < K; ++kw) win[kh][kw] = load(kh, kw - p.pad);
     const unsigned int* drow = dyw + ((long long)n * p.Ho + ho) * p.Wo * CW + cp;
-    for (int wo = 0; wo < p.Wo; ++wo) {
-      if (wo > 0) {
-        const int w0 = wo * S - p.pad;
+    for (int wo0 = 0; wo0 < p.Wo; wo0 += U) {
+      const int c0 = wo0 * S - p.pad;
+      float2 d[U];
 #pragma unroll
-        for (int kh = 0; kh < K; ++kh) {
-#pragma unroll
-          for (int kw = 0; kw < K - S; ++kw) win[kh][kw] = win[kh][kw + S];
-#pragma unroll
-          for (int kw = K - S; kw < K; ++kw) win[kh][kw] = load(kh, w0 + kw);
-        }
-      }
-      const float2 d = unpack2<T>(__ldg(drow + (long long)wo * CW));
+      for (int u = 0; u < U; ++u)
+        d[u] = wo0 + u < p.Wo ? unpack2<T>(__ldg(drow + (long long)(wo0 + u) * CW))
+                              : make_float2(0.0f, 0.0f);
+      float2 xv[K][NC];
 #pragma unroll
       for (int kh = 0; kh < K; ++kh)
 #pragma unroll
-        for (int kw = 0; kw < K; ++kw) acc[kh][kw] = ffma2(d, win[kh][kw], acc[kh][kw]);
+        for (int j = 0; j < NC; ++j) {
+          const int col = c0 + j;
+          xv[kh][j] = (rb[kh] >= 0 && col >= 0 && col < p.W)
+                          ? unpack2<T>(__ldg(xw + rb[kh] + (long long)col * CW))
+                          : make_float2(0.0f, 0.0f);
+        }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int kh = 0; kh < K; ++kh)
+#pragma unroll
+          for (int kw = 0; kw < K; ++kw)
+            acc[kh][kw] = ffma2(d[u], xv[kh][u * S + kw], acc[kh][kw]);
     }
   }
   float2* out = reinterpret_cast<float2*>(ws + (long long)blockIdx.y * K * K * p.C_in) + cp;
@@ -233,23 +232,228 @@ __global__ void __launch_bounds__(128) wgrad_depthwise_nhwc_kernel(const T* __re
     for (int kw = 0; kw < K; ++kw) out[(long long)(kh * K + kw) * CW] = acc[kh][kw];
 }
 
-// dw[e] = sum over slices s (in order) of the partial of entry e. TAP_MAJOR: partials are laid
-// out [s][tap][C] and e = c * taps + tap (the depthwise kernel); otherwise [s][e].
+// ------------------------------------------------------------------ depthwise data gradient
+// NHWC, 16-bit, groups == C_in == C_out, C % VEC == 0, dilation 1, K x K, any stride and pad
+// (the shapes that are not a stride-1 forward convolution). A thread owns VEC channels (one
+// 16-, 8- or 4-byte vector) and keeps their K x K filter in fp32 registers; it walks dx pixels
+// (n, h, w) and for each adds the taps (kh, kw) with h + pad - kh and w + pad - kw multiples of
+// the stride -- on average K*K/S^2 of them -- as vector loads of dy, then stores one vector.
+// Consecutive threads take consecutive channel vectors (contiguous loads and stores).
+template <int VEC> struct DVec;
+template <> struct DVec<8> { using type = uint4; };
+template <> struct DVec<4> { using type = uint2; };
+template <> struct DVec<2> { using type = unsigned int; };
+
+template <typename T, int K, int S, int VEC>
+__global__ void __launch_bounds__(256) dgrad_depthwise_nhwc_kernel(const T* __restrict__ dy,
+                                                                    const T* __restrict__ w,
+                                                                    T* __restrict__ dx,
+                                                                    Conv2d p) {
+  using V = typename DVec<VEC>::type;
+  constexpr int NW = VEC / 2;
+  const int CV = p.C_in / VEC;
+  const int cv = blockIdx.x * blockDim.x + threadIdx.x;
+  if (cv >= CV) return;
+  const int c = cv * VEC;
+  float wr[K * K][VEC];
+#pragma unroll
+  for (int t = 0; t < K * K; ++t)
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) wr[t][v] = Elem<T>::to_f32(w[(long long)(c + v) * K * K + t]);
+  const int rows = p.N * p.H;
+  for (int r = blockIdx.y; r < rows; r += gridDim.y) {      // dx rows (n, h)
+    const int n = r / p.H, h = r - n * p.H;
+    const T* drow[K];                                       // dy row of tap kh, or null
+#pragma unroll
+    for (int kh = 0; kh < K; ++kh) {
+      const int th = h + p.pad - kh;
+      drow[kh] = (th >= 0 && th % S == 0 && th / S < p.Ho)
+                     ? dy + ((long long)n * p.Ho + th / S) * p.Wo * p.C_out + c
+                     : nullptr;
+    }
+    T* xrow = dx + (long long)r * p.W * p.C_in + c;
+    for (int wi = threadIdx.y; wi < p.W; wi += blockDim.y) {
+      float2 acc[NW];
+#pragma unroll
+      for (int i = 0; i < NW; ++i) acc[i] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int kw = 0; kw < K; ++kw) {
+        const int tw = wi + p.pad - kw;
+        if (tw < 0 || tw % S != 0 || tw / S >= p.Wo) continue;
+        const int col = tw / S;
+#pragma unroll
+        for (int kh = 0; kh < K; ++kh) {
+          if (drow[kh] == nullptr) continue;
+          const V d = __ldg(reinterpret_cast<const V*>(drow[kh] + (long long)col * p.C_out));
+          const unsigned int* du = reinterpret_cast<const unsigned int*>(&d);
+#pragma unroll
+          for (int i = 0; i < NW; ++i)
+            acc[i] = ffma2(unpack2<T>(du[i]),
+                           make_float2(wr[kh * K + kw][2 * i], wr[kh * K + kw][2 * i + 1]),
+                           acc[i]);
+        }
+      }
+      V o;
+      unsigned int* ou = reinterpret_cast<unsigned int*>(&o);
+#pragma unroll
+      for (int i = 0; i < NW; ++i) ou[i] = pack2<T>(acc[i]);
+      *reinterpret_cast<V*>(xrow + (long long)wi * p.C_in) = o;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ wide-group weight gradient
+// NHWC, 16-bit, C_in/g and C_out/g multiples of 8 and at least 32. Per group and tap (kh, kw),
+// dw[co][kh][kw][ci] over the group's filters and channels is a sum over output positions p of
+// the outer product dy[p][co] * x[tap-shifted p][ci]. A CTA owns one 128 x 128 (co, ci) tile of
+// one (group, tap) and one fixed slice of positions; its 256 threads own 8 x 8 fp32
+// accumulators each. Each step stages 16 positions' dy row segment ([16][128 co]) and their
+// tap-shifted input segment ([16][128 ci], zero where the tap falls in the padding) in shared
+// memory as fp32 -- one 16-byte load per thread per operand, issued before the previous step's
+// multiply-adds -- and every thread then reads two 4-float vectors of each per position.
+constexpr int WT_TILE = 128;
+constexpr int WT_K = 16;
+
+template <typename T>
+__global__ void __launch_bounds__(256) wgrad_tiled_nhwc_kernel(const T* __restrict__ x,
+                                                                const T* __restrict__ dy,
+                                                                float* __restrict__ ws,
+                                                                Conv2d p, int n_mt, int n_nt,
+                                                                long long E, int per_slice) {
+  __shared__ __align__(16) float sA[2][WT_K][WT_TILE + 4];   // dy: [position][co]
+  __shared__ __align__(16) float sB[2][WT_K][WT_TILE + 4];   // x:  [position][ci]
+  const int taps = p.kH * p.kW;
+  int t = blockIdx.x;
+  const int nt = t % n_nt; t /= n_nt;
+  const int mt = t % n_mt; t /= n_mt;
+  const int tap = t % taps;
+  const int g = t / taps;
+  const int kh = tap / p.kW, kw = tap - kh * p.kW;
+  const long long P = (long long)p.N * p.Ho * p.Wo;
+  const long long p0 = (long long)blockIdx.y * per_slice;
+  const long long p1 = min(P, p0 + per_slice);
+
+  const int tid = threadIdx.x;
+  const int lk = tid / 16, lv = tid % 16;          // loader: position lk, 8-channel vector lv
+  const int co_l = mt * WT_TILE + lv * 8;          // within the group
+  const int ci_l = nt * WT_TILE + lv * 8;
+  const bool co_ok = co_l < p.cpg_out, ci_ok = ci_l < p.cpg_in;
+  const T* dyg = dy + (long long)g * p.cpg_out + co_l;
+  const T* xg = x + (long long)g * p.cpg_in + ci_l;
+
+  auto fetch = [&](long long pos, uint4& va, uint4& vb) {
+    va = make_uint4(0, 0, 0, 0);
+    vb = make_uint4(0, 0, 0, 0);
+    if (pos >= p1) return;
+    if (co_ok) va = __ldg(reinterpret_cast<const uint4*>(dyg + pos * p.C_out));
+    if (!ci_ok) return;
+    const int pi = (int)pos;                       // N*Ho*Wo < 2^31 (checked on the host)
+    const int wo = pi % p.Wo;
+    const int r = pi / p.Wo;
+    const int ho = r % p.Ho, n = r / p.Ho;
+    const int h = ho * p.stride - p.pad + kh * p.dil;
+    const int w = wo * p.stride - p.pad + kw * p.dil;
+    if (h < 0 || h >= p.H || w < 0 || w >= p.W) return;
+    vb = __ldg(reinterpret_cast<const uint4*>(xg + (((long long)n * p.H + h) * p.W + w) * p.C_in));
+  };
+  auto stage = [&](int buf, const uint4& va, const uint4& vb) {
+    const unsigned int* ua = reinterpret_cast<const unsigned int*>(&va);
+    const unsigned int* ub = reinterpret_cast<const unsigned int*>(&vb);
+    float4* da = reinterpret_cast<float4*>(&sA[buf][lk][lv * 8]);
+    float4* db = reinterpret_cast<float4*>(&sB[buf][lk][lv * 8]);
+    float2 a0 = unpack2<T>(ua[0]), a1 = unpack2<T>(ua[1]), a2 = unpack2<T>(ua[2]),
+           a3 = unpack2<T>(ua[3]);
+    float2 b0 = unpack2<T>(ub[0]), b1 = unpack2<T>(ub[1]), b2 = unpack2<T>(ub[2]),
+           b3 = unpack2<T>(ub[3]);
+    da[0] = make_float4(a0.x, a0.y, a1.x, a1.y);
+    da[1] = make_float4(a2.x, a2.y, a3.x, a3.y);
+    db[0] = make_float4(b0.x, b0.y, b1.x, b1.y);
+    db[1] = make_float4(b2.x, b2.y, b3.x, b3.y);
+  };
+
+  const int ty = tid / 16, tx = tid % 16;          // compute: rows ty*4 (+64), cols tx*4 (+64)
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+
+  uint4 va, vb;
+  fetch(p0 + lk, va, vb);
+  stage(0, va, vb);
+  __syncthreads();
+  int buf = 0;
+  for (long long base = p0; base < p1; base += WT_K) {
+    const bool more = base + WT_K < p1;
+    if (more) fetch(base + WT_K + lk, va, vb);     // next step's loads fly during the math
+#pragma unroll
+    for (int k = 0; k < WT_K; ++k) {
+      const float4 a_lo = *reinterpret_cast<const float4*>(&sA[buf][k][ty * 4]);
+      const float4 a_hi = *reinterpret_cast<const float4*>(&sA[buf][k][64 + ty * 4]);
+      const float4 b_lo = *reinterpret_cast<const float4*>(&sB[buf][k][tx * 4]);
+      const float4 b_hi = *reinterpret_cast<const float4*>(&sB[buf][k][64 + tx * 4]);
+      const float a[8] = {a_lo.x, a_lo.y, a_lo.z, a_lo.w, a_hi.x, a_hi.y, a_hi.z, a_hi.w};
+      const float b[8] = {b_lo.x, b_lo.y, b_lo.z, b_lo.w, b_hi.x, b_hi.y, b_hi.z, b_hi.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    if (more) {
+      stage(buf ^ 1, va, vb);
+      __syncthreads();
+      buf ^= 1;
+    }
+  }
+  // partial of this slice for dw[g*cpg_out + co][kh][kw][ci]
+  float* out = ws + (long long)blockIdx.y * E;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int co = mt * WT_TILE + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+    if (co >= p.cpg_out) continue;
+    float* row = out + (((long long)(g * p.cpg_out + co) * p.kH + kh) * p.kW + kw) * p.cpg_in;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int ci = nt * WT_TILE + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
+      if (ci < p.cpg_in) row[ci] = acc[i][j];
+    }
+  }
+}
+
+// dw from the slice partials: dw[e(q)] = sum over slices s of ws[s][q], q the partial index.
+// A CTA takes 32 consecutive q (one per lane, so each warp load is 128 contiguous bytes) and its
+// 8 warps split the slices: warp j adds slices j, j+8, j+16, ... in that order, then the 8 warp
+// sums are added in warp order -- a fixed order, so the result is bitwise reproducible.
+// TAP_MAJOR: partials are [s][tap][C] and e = c * taps + tap (the depthwise kernel); otherwise
+// e = q.
 template <typename T, bool TAP_MAJOR>
 __global__ void __launch_bounds__(256) wgrad_sum_kernel(const float* __restrict__ ws,
                                                          T* __restrict__ dw, long long E,
                                                          int S, int taps) {
-  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= E) return;
-  long long src = e;
-  if (TAP_MAJOR) {
-    const long long C = E / taps;
-    src = (e % taps) * C + e / taps;
-  }
+  __shared__ float part[8][33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long q = (long long)blockIdx.x * 32 + lane;
   float acc = 0.0f;
-  for (int s = 0; s < S; ++s) acc += ws[(long long)s * E + src];
-  dw[e] = Elem<T>::from_f32(acc);
+  if (q < E) {
+#pragma unroll 4
+    for (int s = warp; s < S; s += 8) acc += ws[(long long)s * E + q];
+  }
+  part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && q < E) {
+    float t = part[0][lane];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) t += part[j][lane];
+    long long e = q;
+    if (TAP_MAJOR) {
+      const long long C = E / taps;
+      e = (q % C) * taps + q / C;
+    }
+    dw[e] = Elem<T>::from_f32(t);
+  }
 }
+
+unsigned sum_grid(long long E) { return (unsigned)((E + 31) / 32); }
 
 unsigned grid_for(long long total, int threads) {
   long long blocks = (total + threads - 1) / threads;
@@ -283,6 +487,37 @@ cudaError_t dgrad_typed(const Conv2d& p, const void* dy, const void* w, void* dx
   return cudaGetLastError();
 }
 
+int dgrad_depthwise_vec(const Conv2d& p) { return p.kH <= 3 ? 8 : (p.kH <= 5 ? 4 : 2); }
+
+template <typename T, int K, int VEC>
+cudaError_t dgrad_dw_k(const Conv2d& p, const void* dy, const void* w, void* dx,
+                       cudaStream_t s) {
+  const int CV = p.C_in / VEC;
+  const dim3 block(32, 8);
+  const unsigned gx = (unsigned)((CV + 31) / 32);
+  long long gy = (long long)p.N * p.H;                       // one dx row per CTA row step
+  const long long cap = (WGRAD_TARGET_CTAS + gx - 1) / gx;   // ~8 CTAs per SM in all
+  if (gy > cap) gy = cap;
+  const dim3 grid(gx, (unsigned)gy);
+  if (p.stride == 1)
+    dgrad_depthwise_nhwc_kernel<T, K, 1, VEC><<<grid, block, 0, s>>>((const T*)dy, (const T*)w,
+                                                                     (T*)dx, p);
+  else
+    dgrad_depthwise_nhwc_kernel<T, K, 2, VEC><<<grid, block, 0, s>>>((const T*)dy, (const T*)w,
+                                                                     (T*)dx, p);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dgrad_dw_typed(const Conv2d& p, const void* dy, const void* w, void* dx,
+                           cudaStream_t s) {
+  switch (p.kH) {
+    case 3: return dgrad_dw_k<T, 3, 8>(p, dy, w, dx, s);
+    case 5: return dgrad_dw_k<T, 5, 4>(p, dy, w, dx, s);
+    default: return dgrad_dw_k<T, 7, 2>(p, dy, w, dx, s);
+  }
+}
+
 // Slices of the N*Ho rows for a weight-gradient launch with `blocks_x` CTAs per slice.
 void wgrad_slices(const Conv2d& p, long long blocks_x, int* S, int* rows) {
   const long long R = (long long)p.N * p.Ho;
@@ -295,6 +530,32 @@ void wgrad_slices(const Conv2d& p, long long blocks_x, int* S, int* rows) {
   *S = (int)((R + per - 1) / per);
 }
 
+void tiled_tiles(const Conv2d& p, int* n_mt, int* n_nt) {
+  *n_mt = (p.cpg_out + WT_TILE - 1) / WT_TILE;
+  *n_nt = (p.cpg_in + WT_TILE - 1) / WT_TILE;
+}
+
+// Position slices of the tiled weight gradient: a multiple of WT_K positions each, enough
+// slices for ~WGRAD_TARGET_CTAS CTAs in all (a function of the shape only).
+void tiled_slices(const Conv2d& p, long long tiles, int* S, int* per) {
+  const long long P = (long long)p.N * p.Ho * p.Wo;
+  long long want = (WGRAD_TARGET_CTAS + tiles - 1) / tiles;
+  const long long max_s = (P + WT_K - 1) / WT_K;
+  if (want > max_s) want = max_s;
+  if (want > 65535) want = 65535;
+  if (want < 1) want = 1;
+  long long q = (P + want - 1) / want;
+  q = (q + WT_K - 1) / WT_K * WT_K;
+  *per = (int)q;
+  *S = (int)((P + q - 1) / q);
+}
+
+long long tiled_count(const Conv2d& p) {
+  int n_mt, n_nt;
+  tiled_tiles(p, &n_mt, &n_nt);
+  return (long long)p.groups * p.kH * p.kW * n_mt * n_nt;
+}
+
 long long wgrad_blocks_x(const Conv2d& p, int kernel) {
   if (kernel == GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC) return (p.C_in / 2 + 127) / 128;
   const long long E = (long long)p.C_out * p.cpg_in * p.kH * p.kW;
@@ -305,6 +566,21 @@ template <typename T>
 cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw, void* ws,
                         int kernel, cudaStream_t s) {
   const long long E = (long long)p.C_out * p.cpg_in * p.kH * p.kW;
+  if constexpr (sizeof(T) == 2) {
+    if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC) {
+      int n_mt, n_nt, S, per;
+      tiled_tiles(p, &n_mt, &n_nt);
+      const long long tiles = tiled_count(p);
+      tiled_slices(p, tiles, &S, &per);
+      wgrad_tiled_nhwc_kernel<T><<<dim3((unsigned)tiles, (unsigned)S), 256, 0, s>>>(
+          (const T*)x, (const T*)dy, (float*)ws, p, n_mt, n_nt, E, per);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      wgrad_sum_kernel<T, false><<<sum_grid(E), 256, 0, s>>>((const float*)ws,
+                                                                            (T*)dw, E, S, 1);
+      return cudaGetLastError();
+    }
+  }
   int S, rows;
   const long long bx = wgrad_blocks_x(p, kernel);
   wgrad_slices(p, bx, &S, &rows);
@@ -314,13 +590,17 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
    if (kernel == GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC) {
     const T* xt = (const T*)x;
     const T* dt = (const T*)dy;
-    if (p.kH == 3 && p.stride == 1) wgrad_depthwise_nhwc_kernel<T, 3, 1><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
-    else if (p.kH == 3) wgrad_depthwise_nhwc_kernel<T, 3, 2><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
-    else if (p.stride == 1) wgrad_depthwise_nhwc_kernel<T, 5, 1><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
-    else wgrad_depthwise_nhwc_kernel<T, 5, 2><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
+    if (p.kH == 3 && p.stride == 1)
+      wgrad_depthwise_nhwc_kernel<T, 3, 1, 8><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
+    else if (p.kH == 3)
+      wgrad_depthwise_nhwc_kernel<T, 3, 2, 4><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
+    else if (p.stride == 1)
+      wgrad_depthwise_nhwc_kernel<T, 5, 1, 4><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
+    else
+      wgrad_depthwise_nhwc_kernel<T, 5, 2, 2><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wgrad_sum_kernel<T, true><<<(unsigned)((E + 255) / 256), 256, 0, s>>>(part, (T*)dw, E, S,
+    wgrad_sum_kernel<T, true><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S,
                                                                           p.kH * p.kW);
     return cudaGetLastError();
    }
@@ -333,7 +613,7 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
                                                             E, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  wgrad_sum_kernel<T, false><<<(unsigned)((E + 255) / 256), 256, 0, s>>>(part, (T*)dw, E, S, 1);
+  wgrad_sum_kernel<T, false><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S, 1);
   return cudaGetLastError();
 }
 
@@ -361,14 +641,41 @@ cudaError_t launch_dgrad_generic(const Conv2d& p, const void* dy, const void* w,
   }
 }
 
+bool dgrad_depthwise_supported(const Conv2d& p) {
+  return p.layout == GCONV_NHWC && p.dtype != GCONV_F32 && p.groups == p.C_in &&
+         p.C_out == p.C_in && p.kH == p.kW && (p.kH == 3 || p.kH == 5 || p.kH == 7) &&
+         p.dil == 1 && (p.stride == 1 || p.stride == 2) && p.C_in % dgrad_depthwise_vec(p) == 0 &&
+         (long long)p.N * p.H <= 0x7fffffffLL;
+}
+
+int dgrad_depthwise_vec_bytes(const Conv2d& p) { return 2 * dgrad_depthwise_vec(p); }
+
+cudaError_t launch_dgrad_depthwise(const Conv2d& p, const void* dy, const void* w, void* dx,
+                                   cudaStream_t s) {
+  if ((long long)p.N * p.H * p.W == 0) return cudaSuccess;
+  if (p.dtype == GCONV_F16) return dgrad_dw_typed<__half>(p, dy, w, dx, s);
+  return dgrad_dw_typed<__nv_bfloat16>(p, dy, w, dx, s);
+}
+
 bool wgrad_depthwise_supported(const Conv2d& p) {
   return p.layout == GCONV_NHWC && p.dtype != GCONV_F32 && p.groups == p.C_in &&
          p.C_out == p.C_in && p.C_in % 2 == 0 && p.kH == p.kW && (p.kH == 3 || p.kH == 5) &&
          p.dil == 1 && (p.stride == 1 || p.stride == 2);
 }
 
+bool wgrad_tiled_supported(const Conv2d& p) {
+  return p.layout == GCONV_NHWC && p.dtype != GCONV_F32 && p.cpg_in >= 32 && p.cpg_out >= 32 &&
+         p.cpg_in % 8 == 0 && p.cpg_out % 8 == 0 && tiled_count(p) <= 0x7fffffffLL &&
+         (long long)p.N * p.Ho * p.Wo <= 0x7fffffffLL;
+}
+
 size_t wgrad_workspace(const Conv2d& p, int kernel) {
   if ((long long)p.N * p.Ho == 0) return 0;
+  if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC) {
+    int S, per;
+    tiled_slices(p, tiled_count(p), &S, &per);
+    return (size_t)S * (size_t)p.C_out * p.cpg_in * p.kH * p.kW * sizeof(float);
+  }
   int S, rows;
   wgrad_slices(p, wgrad_blocks_x(p, kernel), &S, &rows);
   const long long E = (long long)p.C_out * p.cpg_in * p.kH * p.kW;

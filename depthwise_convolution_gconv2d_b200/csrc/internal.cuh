@@ -119,7 +119,16 @@ cudaError_t launch_flip_transpose_weight(const Conv2d& p, const void* w, void* w
                                          cudaStream_t s);
 cudaError_t launch_dgrad_generic(const Conv2d& p, const void* dy, const void* w, void* dx,
                                  cudaStream_t s);
+// Depthwise NHWC data gradient (16-bit, dilation 1, 3x3 / 5x5 / 7x7, stride 1 or 2); dy and dx
+// aligned to dgrad_depthwise_vec_bytes.
+bool dgrad_depthwise_supported(const Conv2d& p);
+int dgrad_depthwise_vec_bytes(const Conv2d& p);
+cudaError_t launch_dgrad_depthwise(const Conv2d& p, const void* dy, const void* w, void* dx,
+                                   cudaStream_t s);
 bool wgrad_depthwise_supported(const Conv2d& p);
+// Wide-group NHWC weight gradient (16-bit, C_in/g and C_out/g >= 32 and multiples of 8; x and
+// dy 16-byte aligned).
+bool wgrad_tiled_supported(const Conv2d& p);
 size_t wgrad_workspace(const Conv2d& p, int kernel);
 cudaError_t launch_wgrad(const Conv2d& p, const void* x, const void* dy, void* dw, void* ws,
                          int kernel, cudaStream_t s);

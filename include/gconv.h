@@ -108,8 +108,14 @@ typedef enum {
                                          FMA, any problem */
   GCONV_KERNEL_WGRAD_GENERIC = 10,    /* conv2d weight gradient: one thread per (dw entry,
                                          slice), fp32 FMA, any problem */
-  GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC = 11  /* conv2d weight gradient, depthwise 3x3 / 5x5,
+  GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC = 11, /* conv2d weight gradient, depthwise 3x3 / 5x5,
                                          dilation 1, stride 1 or 2, 16-bit NHWC, C even */
+  GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC = 12, /* conv2d data gradient, depthwise 3x3 / 5x5 / 7x7,
+                                         dilation 1, stride 1 or 2, 16-bit NHWC, C a multiple
+                                         of 8 / 4 / 2: 16- / 8- / 4-byte channel vectors */
+  GCONV_KERNEL_WGRAD_TILED_NHWC = 13  /* conv2d weight gradient, 16-bit NHWC, C_in/g and
+                                         C_out/g >= 32 and multiples of 8: shared-memory tiled
+                                         outer products on the CUDA cores */
 } gconv_kernel;
 
 /* Bytes of workspace gconv2d_fwd needs for this problem under `path` (0 if none; also 0 for
@@ -166,8 +172,9 @@ size_t gconv2d_bwd_data_workspace_size(int N, int C_in, int H, int W, int C_out,
  * pad <= dilation*(k-1) it is computed as the forward convolution of dy with the per-group
  * transposed, 180-degree-rotated filter and pad' = dilation*(k-1) - pad, on the forward
  * kernels (AUTO / DIRECT / IGEMM choose among them as gconv2d_fwd_path does, F32 under AUTO
- * excepted); other problems, fp32 under AUTO and GENERIC run the one-thread-per-element
- * gather kernel. IGEMM on a problem that cannot run as a forward convolution on the tensor
+ * excepted). Under AUTO / DIRECT, depthwise NHWC problems that do not run that way (stride 2,
+ * larger pads) take a vectorised depthwise gather kernel (GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC);
+ * other problems, fp32 under AUTO and GENERIC run the one-thread-per-element gather kernel. IGEMM on a problem that cannot run as a forward convolution on the tensor
  * cores is UNSUPPORTED (or MISALIGNED). The workspace must be 16-byte aligned.
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
 gconv_status gconv2d_bwd_data(const void* dy, const void* w, void* dx, int N, int C_in, int H,
@@ -199,7 +206,8 @@ size_t gconv2d_bwd_weight_workspace_size(int N, int C_in, int H, int W, int C_ou
  * sizes alone, each slice's partial sums are added in a fixed order and the slices are added
  * in slice order (no float atomics), so repeated calls -- on any GPU -- give bitwise-identical
  * dw. AUTO and DIRECT run the depthwise kernel where it applies (GCONV_KERNEL_WGRAD_DEPTHWISE_
- * NHWC; x and dy 4-byte aligned), else the generic kernel; GENERIC forces the generic kernel;
+ * NHWC; x and dy 4-byte aligned), else the tiled kernel for wide groups
+ * (GCONV_KERNEL_WGRAD_TILED_NHWC; x and dy 16-byte aligned), else the generic kernel; GENERIC forces the generic kernel;
  * IGEMM is UNSUPPORTED (there is no tensor-core weight gradient). N*Ho > 2^30 is UNSUPPORTED.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 gconv_status gconv2d_bwd_weight(const void* x, const void* dy, void* dw, int N, int C_in, int H,

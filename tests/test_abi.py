@@ -194,17 +194,22 @@ def test_bwd_path_selection(lib):
     # depthwise 56x56x1024: stride 1 runs the depthwise forward kernel on the flipped filter,
     # stride 2 the gather kernel; the weight gradient has its own depthwise kernel
     assert sel(dg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 1024) == 2
-    assert sel(dg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 9
+    assert sel(dg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 12
     assert sel(wg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 1024) == 11
     assert sel(wg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 11
     # wide groups: tensor cores (NHWC, NCHW staging); weight gradient generic
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 3
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 4
-    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 10
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 13
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 10
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, path=3) == 10
+    assert sel(wg, 1, 64, 56, 56, 64, 3, 1, 1, 1, 4) == 10          # 16 channels a group
     # narrow groups (4 channels): the narrow-group forward kernel
     assert sel(dg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 256) == 8
-    # pad beyond dil*(k-1), fp32 under AUTO, and GENERIC: the gather kernel
-    assert sel(dg, 1, 64, 16, 16, 64, 3, 1, 3, 1, 64) == 9
+    # depthwise with pad beyond dil*(k-1): the depthwise gather kernel; grouped: the generic
+    # one, as for fp32 under AUTO and for GENERIC
+    assert sel(dg, 1, 64, 16, 16, 64, 3, 1, 3, 1, 64) == 12
+    assert sel(dg, 1, 64, 16, 16, 64, 3, 1, 3, 1, 16) == 9
     assert sel(dg, 1, 64, 16, 16, 64, 3, 1, 1, 1, 64, dtype=0) == 9
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, path=3) == 9
     # forced IGEMM where the data gradient is not a stride-1 convolution, or on the weight
@@ -221,9 +226,10 @@ def test_bwd_workspace_queries(lib):
     assert lib.gconv2d_bwd_data_workspace_size(1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 0, 2,
                                                0) == wt + lib.gconv2d_fwd_workspace_size(
         1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 0, 2, 0)
-    # the gather kernel needs none
+    # the gather kernels need none
     assert lib.gconv2d_bwd_data_workspace_size(32, 1024, 56, 56, 1024, 3, 3, 2, 1, 1, 1024, 1,
                                                2, 0) == 0
+    assert lib.gconv2d_bwd_data_workspace_size(2, 12, 9, 8, 18, 3, 2, 1, 1, 1, 3, 1, 2, 0) == 0
     # weight gradient: fp32 partials, a whole number of slices of every dw entry
     for args in [(32, 1024, 56, 56, 1024, 3, 3, 1, 1, 1, 1024, 1, 2, 0),
                  (1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 1, 2, 0),

@@ -66,18 +66,24 @@ def oracle_wgrad(p, inp, dy):
 CASES = [
     # N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups
     ((2, 64, 12, 12, 64, 3, 3, 1, 1, 1, 64), 2, 11),       # depthwise 3x3 s1
-    ((2, 64, 13, 11, 64, 3, 3, 2, 1, 1, 64), 9, 11),       # depthwise 3x3 s2, ragged
+    ((2, 64, 13, 11, 64, 3, 3, 2, 1, 1, 64), 12, 11),      # depthwise 3x3 s2, ragged
     ((1, 32, 14, 9, 32, 5, 5, 1, 2, 1, 32), 2, 11),        # depthwise 5x5
-    ((1, 32, 15, 16, 32, 5, 5, 2, 2, 1, 32), 9, 11),       # depthwise 5x5 s2
+    ((1, 32, 15, 16, 32, 5, 5, 2, 2, 1, 32), 12, 11),      # depthwise 5x5 s2
     ((2, 48, 10, 9, 48, 3, 3, 1, 0, 1, 48), 2, 11),        # depthwise, no padding (pad' = 2)
     ((2, 64, 9, 10, 64, 3, 3, 1, 1, 1, 16), 8, 10),        # narrow groups (4 ch)
-    ((2, 128, 9, 24, 128, 3, 3, 1, 1, 1, 2), 3, 10),       # wide groups: tensor cores
-    ((1, 64, 12, 16, 128, 3, 3, 1, 2, 2, 2), 3, 10),       # dilation 2, cpg_in != cpg_out
-    ((1, 64, 7, 140, 64, 3, 3, 1, 1, 1, 1), 3, 10),        # W >= 128 (row kernels)
+    ((2, 128, 9, 24, 128, 3, 3, 1, 1, 1, 2), 3, 13),       # wide groups: tensor cores
+    ((1, 64, 12, 16, 128, 3, 3, 1, 2, 2, 2), 3, 13),       # dilation 2, cpg_in != cpg_out
+    ((1, 64, 7, 140, 64, 3, 3, 1, 1, 1, 1), 3, 13),        # W >= 128 (row kernels)
     ((2, 12, 9, 8, 18, 3, 2, 1, 1, 1, 3), 9, 10),          # rectangular kernel
     ((1, 16, 11, 10, 8, 3, 3, 3, 1, 1, 4), 9, 10),         # stride 3
     ((1, 8, 6, 7, 8, 3, 3, 1, 3, 1, 2), 9, 10),            # pad 3 > dil*(k-1)
     ((2, 16, 5, 6, 32, 1, 1, 2, 0, 1, 16), 9, 10),         # 1x1 stride 2, channel multiplier 2
+    ((1, 16, 12, 13, 16, 7, 7, 2, 3, 1, 16), 12, 10),      # depthwise 7x7 s2 (4-byte vectors)
+    ((2, 24, 9, 9, 24, 3, 3, 1, 3, 1, 24), 12, 11),        # depthwise, pad 3 > k-1
+    ((1, 40, 11, 9, 40, 5, 5, 1, 5, 1, 40), 12, 11),       # depthwise 5x5, pad 5
+    ((1, 80, 10, 11, 96, 3, 3, 1, 1, 1, 2), 9, 13),        # 40 -> 48 per group: ragged tiles
+    ((2, 64, 11, 13, 64, 3, 3, 2, 1, 1, 1), 9, 13),        # tiled weight gradient, stride 2
+    ((1, 160, 6, 7, 320, 3, 3, 1, 1, 1, 1), 3, 13),        # 160 -> 320: 3 x 2 tiles, ragged
 ]
 
 
@@ -130,7 +136,7 @@ def test_bwd_tiny_fp32(groups, layout):
     assert_close(to_f64(gpu_wgrad(p, inp, dy)), oracle_wgrad(p, inp, dy), p.dtype, "dw")
 
 
-@pytest.mark.parametrize("case,kd,kw", [CASES[0], CASES[1], CASES[5], CASES[6]])
+@pytest.mark.parametrize("case,kd,kw", [CASES[0], CASES[1], CASES[5], CASES[6], CASES[13]])
 @pytest.mark.parametrize("path", [gb.PATH_AUTO, gb.PATH_GENERIC])
 def test_bwd_integer_bit_exact(case, kd, kw, path):
     """x, w, dy in {-2..2}: every product and partial sum is an integer below 2^24, exact in
