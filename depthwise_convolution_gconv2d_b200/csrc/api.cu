@@ -201,11 +201,13 @@ int wgrad_choose(const Conv2d& p, int path, const void* x, const void* dy, gconv
   const bool query = x == nullptr && dy == nullptr;
   const bool dw_ok = wgrad_depthwise_supported(p) && (query || (aligned4(x) && aligned4(dy)));
   const bool tl_ok = wgrad_tiled_supported(p) && (query || (aligned16(x) && aligned16(dy)));
+  const bool tma_ok = wgrad_dw3_tma_supported(p) && (query || (aligned16(x) && aligned16(dy)));
   switch (path) {
     case GCONV_PATH_GENERIC:
       return GCONV_KERNEL_WGRAD_GENERIC;
     case GCONV_PATH_AUTO:
     case GCONV_PATH_DIRECT:
+      if (tma_ok) return GCONV_KERNEL_WGRAD_DW3_TMA;
       if (dw_ok) return GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC;
       return tl_ok ? GCONV_KERNEL_WGRAD_TILED_NHWC : GCONV_KERNEL_WGRAD_GENERIC;
     case GCONV_PATH_IGEMM:

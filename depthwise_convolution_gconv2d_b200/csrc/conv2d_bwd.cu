@@ -22,6 +22,7 @@
 // second kernel adds the slices in slice order and rounds once to the data type. No float
 // atomics, so repeated calls give bitwise-identical dw on any GPU.
 #include "internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace gconv {
 namespace {
@@ -230,6 +231,252 @@ __global__ void __launch_bounds__(128) wgrad_depthwise_nhwc_kernel(const T* __re
   for (int kh = 0; kh < K; ++kh)
 #pragma unroll
     for (int kw = 0; kw < K; ++kw) out[(long long)(kh * K + kw) * CW] = acc[kh][kw];
+}
+
+// ------------------------------------------------------------------ depthwise 3x3 weight gradient, TMA-staged
+// NHWC, 16-bit, 3x3, dilation 1, stride S = 1 or 2, pad <= 2, C % 8 == 0. The data path of the
+// forward 3x3 kernel with the roles of filter and output exchanged: a producer thread streams,
+// per tile of BH output rows x 28 output columns x 64 channels, the input box
+// ((BH-1)*S+3 rows x 27*S+3 columns, zero fill as the padding) and the matching dy box (zero
+// fill past Ho / Wo) through a shared-memory ring; seven compute warps each take 4 output
+// columns, a thread one channel pair, and add dy(pair) * x(pair) into 9 fp32-pair accumulators
+// with the input rows rolling through registers as in the forward. A CTA owns one channel tile
+// and a fixed slice of that tile's spatial tiles (a function of the shape only); at the end the
+// seven warps' accumulators are added in warp order in shared memory and written as the CTA's
+// partial ws[slice][tap][C]. Every wait is bounded (1 s); on expiry the CTA sets the device
+// error word, drains its copies and writes nothing.
+constexpr int DWW_CH = 64;                  // channels per tile (128-byte box rows)
+constexpr int DWW_R = 4;                    // output columns per thread
+constexpr int DWW_NG = 7;                   // compute warps (column groups)
+constexpr int DWW_BW = DWW_R * DWW_NG;      // output columns per tile
+constexpr int DWW_THREADS = 32 + 32 * DWW_NG;
+constexpr int DWW_MAX_STAGES = 4;
+constexpr int DWW_CTAS = 296;               // two CTAs on each of 148 SMs; a fixed constant
+                                            // so the summation order never depends on the device
+constexpr size_t DWW_SMEM_CTA = 110 * 1024; // two CTAs per SM
+
+template <int S> __host__ __device__ constexpr int dww_iw() { return (DWW_BW - 1) * S + 3; }
+template <int S> __host__ __device__ constexpr int dww_bh() { return S == 1 ? 4 : 2; }
+
+struct DwwParams {
+  int N, C, Ho, Wo, pad;
+  int n_ct, n_ht, n_wt, tiles_per_ct, slices, stages;
+  unsigned int x_bytes, stage_bytes, tx_bytes;
+};
+
+template <typename T, int S>
+__global__ void __launch_bounds__(DWW_THREADS, 2)
+    wgrad_dw3_tma_kernel(const __grid_constant__ CUtensorMap tmx,
+                         const __grid_constant__ CUtensorMap tmd, float* __restrict__ ws,
+                         const DwwParams P, unsigned int* err) {
+  using namespace ptx;
+  constexpr int BH = dww_bh<S>();
+  constexpr int IW = dww_iw<S>();
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = ptx::align_smem(smem_raw, 128u);
+  unsigned long long* full =
+      reinterpret_cast<unsigned long long*>(smem + (size_t)P.stages * P.stage_bytes);
+  unsigned long long* empty = full + DWW_MAX_STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + DWW_MAX_STAGES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ct = blockIdx.x / P.slices, sl = blockIdx.x - ct * P.slices;
+  const int t_begin = (int)((long long)P.tiles_per_ct * sl / P.slices);
+  const int t_end = (int)((long long)P.tiles_per_ct * (sl + 1) / P.slices);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < P.stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], (unsigned int)DWW_NG);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmx);
+    prefetch_tmap(&tmd);
+  }
+  __syncthreads();
+
+  float2 acc[3][3];
+#pragma unroll
+  for (int kh = 0; kh < 3; ++kh)
+#pragma unroll
+    for (int kw = 0; kw < 3; ++kw) acc[kh][kw] = make_float2(0.0f, 0.0f);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int st = 0;
+      unsigned int ph = 0;
+      long long issued = 0;
+      for (int t = t_begin; t < t_end; ++t) {
+        const int tw = t % P.n_wt;
+        const int r = t / P.n_wt;
+        const int th = r % P.n_ht, n = r / P.n_ht;
+        if (!mbar_try_wait(&empty[st], ph ^ 1u) &&
+            !mbar_wait(&empty[st], ph ^ 1u, abort_flag, err, 32u))
+          break;
+        unsigned char* dst = smem + (size_t)st * P.stage_bytes;
+        mbar_arrive_expect_tx(&full[st], P.tx_bytes);
+        tma_load_4d(dst, &tmx, &full[st], ct * DWW_CH, tw * DWW_BW * S - P.pad,
+                    th * BH * S - P.pad, n);
+        tma_load_4d(dst + P.x_bytes, &tmd, &full[st], ct * DWW_CH, tw * DWW_BW, th * BH, n);
+        ++issued;
+        if (++st == P.stages) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+      // copies in flight land before the ring is reused below (instant on the normal path)
+      for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
+        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr,
+                  0u);
+    }
+  } else {
+    constexpr int NIN = (DWW_R - 1) * S + 3;     // input columns a thread reads per row
+    constexpr int row_w = IW * (DWW_CH / 2);     // 32-bit words per input box row
+    constexpr int drow_w = DWW_BW * (DWW_CH / 2);
+    const int g = warp - 1;
+    int st = 0;
+    unsigned int ph = 0;
+    for (int t = t_begin; t < t_end; ++t) {
+      bool got = mbar_try_wait(&full[st], ph);
+      if (!got) got = mbar_wait(&full[st], ph, abort_flag, err, 32u);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const uint32_t* px = reinterpret_cast<const uint32_t*>(smem + (size_t)st * P.stage_bytes) +
+                           (g * DWW_R * S) * (DWW_CH / 2) + lane;
+      const uint32_t* pd =
+          reinterpret_cast<const uint32_t*>(smem + (size_t)st * P.stage_bytes + P.x_bytes) +
+          (g * DWW_R) * (DWW_CH / 2) + lane;
+      float2 in[3][NIN];                         // input row r lives in slot r % 3
+      auto load_row = [&](int r, float2 (&dst)[NIN]) {
+#pragma unroll
+        for (int i = 0; i < NIN; ++i) dst[i] = unpack2<T>(px[r * row_w + i * (DWW_CH / 2)]);
+      };
+      load_row(0, in[0]);
+      if (S == 1) load_row(1, in[1]);
+#pragma unroll
+      for (int j = 0; j < BH; ++j) {
+        if (S == 1) {
+          load_row(j + 2, in[(j + 2) % 3]);
+        } else {
+          load_row(2 * j + 1, in[(2 * j + 1) % 3]);
+          load_row(2 * j + 2, in[(2 * j + 2) % 3]);
+        }
+        float2 d[DWW_R];
+#pragma unroll
+        for (int r = 0; r < DWW_R; ++r) d[r] = unpack2<T>(pd[j * drow_w + r * (DWW_CH / 2)]);
+#pragma unroll
+        for (int kh = 0; kh < 3; ++kh) {
+          const int slot = (j * S + kh) % 3;
+#pragma unroll
+          for (int kw = 0; kw < 3; ++kw)
+#pragma unroll
+            for (int r = 0; r < DWW_R; ++r)
+              acc[kh][kw] = ffma2(d[r], in[slot][r * S + kw], acc[kh][kw]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      if (++st == P.stages) {
+        st = 0;
+        ph ^= 1u;
+      }
+    }
+  }
+  __syncthreads();
+  if (*abort_flag) return;
+  // the ring is idle (every copy has landed and been read): add the warps' sums in warp order
+  float2* red = reinterpret_cast<float2*>(smem);   // [warp][tap][lane]
+  if (warp >= 1) {
+#pragma unroll
+    for (int kh = 0; kh < 3; ++kh)
+#pragma unroll
+      for (int kw = 0; kw < 3; ++kw) red[((warp - 1) * 9 + kh * 3 + kw) * 32 + lane] = acc[kh][kw];
+  }
+  __syncthreads();
+  if (warp == 1) {
+    const int ch = ct * DWW_CH + 2 * lane;
+    if (ch < P.C) {
+      float2* out = reinterpret_cast<float2*>(ws + (long long)sl * 9 * P.C) + ch / 2;
+#pragma unroll
+      for (int tap = 0; tap < 9; ++tap) {
+        float2 v = red[tap * 32 + lane];
+#pragma unroll
+        for (int gg = 1; gg < DWW_NG; ++gg) {
+          const float2 u = red[(gg * 9 + tap) * 32 + lane];
+          v.x += u.x;
+          v.y += u.y;
+        }
+        out[(long long)tap * (P.C / 2)] = v;
+      }
+    }
+  }
+}
+
+DwwParams dww_params(const Conv2d& p) {
+  DwwParams P{};
+  const int S = p.stride;
+  const int BH = S == 1 ? dww_bh<1>() : dww_bh<2>();
+  const int IW = S == 1 ? dww_iw<1>() : dww_iw<2>();
+  const int IH = (BH - 1) * S + 3;
+  P.N = p.N; P.C = p.C_in; P.Ho = p.Ho; P.Wo = p.Wo; P.pad = p.pad;
+  P.n_ct = (p.C_in + DWW_CH - 1) / DWW_CH;
+  P.n_ht = (p.Ho + BH - 1) / BH;
+  P.n_wt = (p.Wo + DWW_BW - 1) / DWW_BW;
+  const long long tpc = (long long)p.N * P.n_ht * P.n_wt;
+  P.tiles_per_ct = tpc > 0x7fffffffLL ? 0x7fffffff : (int)tpc;
+  int sl = DWW_CTAS / P.n_ct;
+  if (sl < 1) sl = 1;
+  P.slices = sl;
+  P.x_bytes = (unsigned int)((DWW_CH * IW * IH * 2 + 127) & ~127);
+  const unsigned int d_bytes = (unsigned int)(DWW_CH * DWW_BW * BH * 2);
+  P.tx_bytes = (unsigned int)(DWW_CH * IW * IH * 2) + d_bytes;
+  P.stage_bytes = (P.x_bytes + d_bytes + 127u) & ~127u;
+  int stages = (int)((DWW_SMEM_CTA - 1024) / P.stage_bytes);
+  if (stages > DWW_MAX_STAGES) stages = DWW_MAX_STAGES;
+  P.stages = stages;
+  return P;
+}
+
+size_t dww_smem(const DwwParams& P) {
+  return 128 + (size_t)P.stages * P.stage_bytes + 2 * DWW_MAX_STAGES * 8 + 16;
+}
+
+template <typename T, int S>
+cudaError_t launch_dww(const Conv2d& p, const void* x, const void* dy, float* ws,
+                       const DwwParams& P, cudaStream_t s) {
+  constexpr int BH = dww_bh<S>();
+  constexpr int IW = dww_iw<S>();
+  if (P.stages < 2 || (long long)P.n_ct * P.slices > 0x7fffffffLL) return cudaErrorInvalidValue;
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const CUtensorMapDataType dt =
+      p.dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint32_t ones[4] = {1, 1, 1, 1};
+  CUtensorMap tmx, tmd;
+  const cuuint64_t xd[4] = {(cuuint64_t)p.C_in, (cuuint64_t)p.W, (cuuint64_t)p.H,
+                            (cuuint64_t)p.N};
+  const cuuint64_t xs[3] = {(cuuint64_t)p.C_in * 2, (cuuint64_t)p.W * p.C_in * 2,
+                            (cuuint64_t)p.H * p.W * p.C_in * 2};
+  const cuuint32_t xb[4] = {DWW_CH, (cuuint32_t)IW, (cuuint32_t)((BH - 1) * S + 3), 1};
+  if (enc(&tmx, dt, 4, const_cast<void*>(x), xd, xs, xb, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const cuuint64_t dd[4] = {(cuuint64_t)p.C_out, (cuuint64_t)p.Wo, (cuuint64_t)p.Ho,
+                            (cuuint64_t)p.N};
+  const cuuint64_t ds[3] = {(cuuint64_t)p.C_out * 2, (cuuint64_t)p.Wo * p.C_out * 2,
+                            (cuuint64_t)p.Ho * p.Wo * p.C_out * 2};
+  const cuuint32_t db[4] = {DWW_CH, DWW_BW, BH, 1};
+  if (enc(&tmd, dt, 4, const_cast<void*>(dy), dd, ds, db, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  static std::atomic<unsigned int> configured{0};
+  const size_t smem = dww_smem(P);
+  cudaError_t e = set_max_dynamic_smem((const void*)wgrad_dw3_tma_kernel<T, S>, smem, configured);
+  if (e != cudaSuccess) return e;
+  wgrad_dw3_tma_kernel<T, S><<<(unsigned)(P.n_ct * P.slices), DWW_THREADS, smem, s>>>(
+      tmx, tmd, ws, P, device_error_word());
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ depthwise data gradient
@@ -567,6 +814,15 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
                         int kernel, cudaStream_t s) {
   const long long E = (long long)p.C_out * p.cpg_in * p.kH * p.kW;
   if constexpr (sizeof(T) == 2) {
+    if (kernel == GCONV_KERNEL_WGRAD_DW3_TMA) {
+      const DwwParams P = dww_params(p);
+      cudaError_t e = p.stride == 1 ? launch_dww<T, 1>(p, x, dy, (float*)ws, P, s)
+                                    : launch_dww<T, 2>(p, x, dy, (float*)ws, P, s);
+      if (e != cudaSuccess) return e;
+      wgrad_sum_kernel<T, true><<<sum_grid(E), 256, 0, s>>>((const float*)ws, (T*)dw, E,
+                                                            P.slices, 9);
+      return cudaGetLastError();
+    }
     if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC) {
       int n_mt, n_nt, S, per;
       tiled_tiles(p, &n_mt, &n_nt);
@@ -657,6 +913,12 @@ cudaError_t launch_dgrad_depthwise(const Conv2d& p, const void* dy, const void* 
   return dgrad_dw_typed<__nv_bfloat16>(p, dy, w, dx, s);
 }
 
+bool wgrad_dw3_tma_supported(const Conv2d& p) {
+  return p.layout == GCONV_NHWC && p.dtype != GCONV_F32 && p.groups == p.C_in &&
+         p.C_out == p.C_in && p.kH == 3 && p.kW == 3 && p.dil == 1 &&
+         (p.stride == 1 || p.stride == 2) && p.pad <= 2 && p.C_in % 8 == 0;
+}
+
 bool wgrad_depthwise_supported(const Conv2d& p) {
   return p.layout == GCONV_NHWC && p.dtype != GCONV_F32 && p.groups == p.C_in &&
          p.C_out == p.C_in && p.C_in % 2 == 0 && p.kH == p.kW && (p.kH == 3 || p.kH == 5) &&
@@ -671,6 +933,8 @@ bool wgrad_tiled_supported(const Conv2d& p) {
 
 size_t wgrad_workspace(const Conv2d& p, int kernel) {
   if ((long long)p.N * p.Ho == 0) return 0;
+  if (kernel == GCONV_KERNEL_WGRAD_DW3_TMA)
+    return (size_t)dww_params(p).slices * 9 * (size_t)p.C_in * sizeof(float);
   if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC) {
     int S, per;
     tiled_slices(p, tiled_count(p), &S, &per);

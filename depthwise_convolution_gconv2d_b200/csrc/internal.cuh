@@ -126,6 +126,9 @@ int dgrad_depthwise_vec_bytes(const Conv2d& p);
 cudaError_t launch_dgrad_depthwise(const Conv2d& p, const void* dy, const void* w, void* dx,
                                    cudaStream_t s);
 bool wgrad_depthwise_supported(const Conv2d& p);
+// Depthwise 3x3 weight gradient on a TMA ring (16-bit NHWC, dilation 1, stride 1 or 2, pad <= 2,
+// C % 8 == 0; x and dy 16-byte aligned).
+bool wgrad_dw3_tma_supported(const Conv2d& p);
 // Wide-group NHWC weight gradient (16-bit, C_in/g and C_out/g >= 32 and multiples of 8; x and
 // dy 16-byte aligned).
 bool wgrad_tiled_supported(const Conv2d& p);

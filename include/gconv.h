@@ -113,9 +113,12 @@ typedef enum {
   GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC = 12, /* conv2d data gradient, depthwise 3x3 / 5x5 / 7x7,
                                          dilation 1, stride 1 or 2, 16-bit NHWC, C a multiple
                                          of 8 / 4 / 2: 16- / 8- / 4-byte channel vectors */
-  GCONV_KERNEL_WGRAD_TILED_NHWC = 13  /* conv2d weight gradient, 16-bit NHWC, C_in/g and
+  GCONV_KERNEL_WGRAD_TILED_NHWC = 13, /* conv2d weight gradient, 16-bit NHWC, C_in/g and
                                          C_out/g >= 32 and multiples of 8: shared-memory tiled
                                          outer products on the CUDA cores */
+  GCONV_KERNEL_WGRAD_DW3_TMA = 14     /* conv2d weight gradient, depthwise 3x3, dilation 1,
+                                         stride 1 or 2, pad <= 2, 16-bit NHWC, C % 8 == 0:
+                                         x and dy staged by TMA */
 } gconv_kernel;
 
 /* Bytes of workspace gconv2d_fwd needs for this problem under `path` (0 if none; also 0 for
@@ -195,7 +198,9 @@ int gconv2d_bwd_data_select_path(int N, int C_in, int H, int W, int C_out, int k
                                  gconv_layout layout, gconv_dtype dtype, gconv_path path);
 
 /* Bytes of workspace gconv2d_bwd_weight_path needs: fp32 partial sums, one per dw entry and
- * slice of the N*Ho output rows (0 if none or invalid). */
+ * slice of the work (0 if none or invalid). The size is that of the kernel chosen for
+ * 16-byte aligned x and dy; a call whose pointers select another kernel may need more (and
+ * then returns GCONV_ERR_WORKSPACE). */
 size_t gconv2d_bwd_weight_workspace_size(int N, int C_in, int H, int W, int C_out, int kH,
                                          int kW, int stride, int pad, int dilation, int groups,
                                          gconv_layout layout, gconv_dtype dtype,
@@ -205,8 +210,9 @@ size_t gconv2d_bwd_weight_workspace_size(int N, int C_in, int H, int W, int C_ou
  * N == 0). Deterministic: the N*Ho output rows are cut into slices fixed by the problem's
  * sizes alone, each slice's partial sums are added in a fixed order and the slices are added
  * in slice order (no float atomics), so repeated calls -- on any GPU -- give bitwise-identical
- * dw. AUTO and DIRECT run the depthwise kernel where it applies (GCONV_KERNEL_WGRAD_DEPTHWISE_
- * NHWC; x and dy 4-byte aligned), else the tiled kernel for wide groups
+ * dw. AUTO and DIRECT run the TMA-staged depthwise 3x3 kernel where it applies
+ * (GCONV_KERNEL_WGRAD_DW3_TMA; x and dy 16-byte aligned), else the depthwise kernel
+ * (GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC; x and dy 4-byte aligned), else the tiled kernel for wide groups
  * (GCONV_KERNEL_WGRAD_TILED_NHWC; x and dy 16-byte aligned), else the generic kernel; GENERIC forces the generic kernel;
  * IGEMM is UNSUPPORTED (there is no tensor-core weight gradient). N*Ho > 2^30 is UNSUPPORTED.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */

@@ -195,8 +195,10 @@ def test_bwd_path_selection(lib):
     # stride 2 the gather kernel; the weight gradient has its own depthwise kernel
     assert sel(dg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 1024) == 2
     assert sel(dg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 12
-    assert sel(wg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 1024) == 11
-    assert sel(wg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 11
+    assert sel(wg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 1024) == 14
+    assert sel(wg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 14
+    assert sel(wg, 32, 1024, 56, 56, 1024, 3, 1, 3, 1, 1024) == 11   # pad 3: LDG kernel
+    assert sel(wg, 32, 1024, 56, 56, 1024, 5, 1, 2, 1, 1024) == 11   # 5x5: LDG kernel
     # wide groups: tensor cores (NHWC, NCHW staging); weight gradient generic
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 3
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 4

@@ -65,11 +65,11 @@ def oracle_wgrad(p, inp, dy):
 # (case, expected AUTO dgrad kernel, expected AUTO wgrad kernel) for NHWC bf16
 CASES = [
     # N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups
-    ((2, 64, 12, 12, 64, 3, 3, 1, 1, 1, 64), 2, 11),       # depthwise 3x3 s1
-    ((2, 64, 13, 11, 64, 3, 3, 2, 1, 1, 64), 12, 11),      # depthwise 3x3 s2, ragged
+    ((2, 64, 12, 12, 64, 3, 3, 1, 1, 1, 64), 2, 14),       # depthwise 3x3 s1
+    ((2, 64, 13, 11, 64, 3, 3, 2, 1, 1, 64), 12, 14),      # depthwise 3x3 s2, ragged
     ((1, 32, 14, 9, 32, 5, 5, 1, 2, 1, 32), 2, 11),        # depthwise 5x5
     ((1, 32, 15, 16, 32, 5, 5, 2, 2, 1, 32), 12, 11),      # depthwise 5x5 s2
-    ((2, 48, 10, 9, 48, 3, 3, 1, 0, 1, 48), 2, 11),        # depthwise, no padding (pad' = 2)
+    ((2, 48, 10, 9, 48, 3, 3, 1, 0, 1, 48), 2, 14),        # depthwise, no padding (pad' = 2)
     ((2, 64, 9, 10, 64, 3, 3, 1, 1, 1, 16), 8, 10),        # narrow groups (4 ch)
     ((2, 128, 9, 24, 128, 3, 3, 1, 1, 1, 2), 3, 13),       # wide groups: tensor cores
     ((1, 64, 12, 16, 128, 3, 3, 1, 2, 2, 2), 3, 13),       # dilation 2, cpg_in != cpg_out
@@ -84,6 +84,9 @@ CASES = [
     ((1, 80, 10, 11, 96, 3, 3, 1, 1, 1, 2), 9, 13),        # 40 -> 48 per group: ragged tiles
     ((2, 64, 11, 13, 64, 3, 3, 2, 1, 1, 1), 9, 13),        # tiled weight gradient, stride 2
     ((1, 160, 6, 7, 320, 3, 3, 1, 1, 1, 1), 3, 13),        # 160 -> 320: 3 x 2 tiles, ragged
+    ((2, 72, 30, 31, 72, 3, 3, 1, 1, 1, 72), 2, 14),       # C % 64 != 0, Wo > 28 (2 column tiles)
+    ((1, 40, 31, 30, 40, 3, 3, 2, 1, 1, 40), 12, 14),      # s2, odd sizes, ragged tiles
+    ((1, 16, 10, 10, 16, 3, 3, 1, 2, 1, 16), 2, 14),       # pad 2 (dgrad pad' = 0)
 ]
 
 
@@ -226,7 +229,7 @@ def test_dgrad_full_size_sampled(p):
 def test_wgrad_depthwise56_full(stride):
     """All 1024 x 9 entries of the 56x56x1024 depthwise layer's weight gradient."""
     p = wl.depthwise_56(stride)
-    assert wgrad_kernel(p) == 11
+    assert wgrad_kernel(p) == 14
     inp, dy = inputs(p, 42)
     got = to_f64(gpu_wgrad(p, inp, dy))
     assert_close(got, oracle_wgrad(p, inp, dy), p.dtype, str(p))
