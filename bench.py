@@ -315,7 +315,8 @@ def backward_measurements(torch, gb, device, stream, pk, reps):
     flush = l2_flusher(torch, device)
     out = {}
     cases = [("depthwise56_s1", wl.depthwise_56(1), reps), ("depthwise56_s2", wl.depthwise_56(2), reps),
-             ("wide_group_nhwc", wl.wide_group(wl.NHWC), reps)]
+             ("wide_group_nhwc", wl.wide_group(wl.NHWC), reps),
+             ("wide_group_nchw", wl.wide_group(wl.NCHW), reps)]
     for tag, p, r in cases:
         inp = wl.make_conv2d_inputs(p, 5)
         x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)

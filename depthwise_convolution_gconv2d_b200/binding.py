@@ -27,7 +27,8 @@ PATH_AUTO, PATH_DIRECT, PATH_IGEMM, PATH_GENERIC = 0, 1, 2, 3
 KERNEL_NAMES = {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "igemm_tc_nchw",
                 5: "conv1d_generic", 6: "conv1d_ring", 7: "conv1d_tc", 8: "grouped_nhwc",
                 9: "dgrad_generic", 10: "wgrad_generic", 11: "wgrad_depthwise_nhwc",
-                12: "dgrad_depthwise_nhwc", 13: "wgrad_tiled_nhwc", 14: "wgrad_dw3_tma"}
+                12: "dgrad_depthwise_nhwc", 13: "wgrad_tiled_nhwc", 14: "wgrad_dw3_tma",
+                15: "wgrad_tiled_nchw"}
 STATUS = {0: "GCONV_OK", 1: "GCONV_ERR_INVALID_ARG", 2: "GCONV_ERR_UNSUPPORTED",
           3: "GCONV_ERR_MISALIGNED", 4: "GCONV_ERR_WORKSPACE", 5: "GCONV_ERR_CUDA",
           6: "GCONV_ERR_DEVICE_TIMEOUT"}

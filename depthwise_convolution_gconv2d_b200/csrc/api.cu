@@ -200,7 +200,11 @@ int wgrad_choose(const Conv2d& p, int path, const void* x, const void* dy, gconv
   *why = GCONV_OK;
   const bool query = x == nullptr && dy == nullptr;
   const bool dw_ok = wgrad_depthwise_supported(p) && (query || (aligned4(x) && aligned4(dy)));
-  const bool tl_ok = wgrad_tiled_supported(p) && (query || (aligned16(x) && aligned16(dy)));
+  // wide groups: NHWC reads x and dy in place (16-byte vectors); NCHW stages them as NHWC
+  const bool tl_ok = wgrad_tiled_supported(p) &&
+                     (p.layout == GCONV_NCHW || query || (aligned16(x) && aligned16(dy)));
+  const int tl_kernel = p.layout == GCONV_NHWC ? GCONV_KERNEL_WGRAD_TILED_NHWC
+                                               : GCONV_KERNEL_WGRAD_TILED_NCHW;
   const bool tma_ok = wgrad_dw3_tma_supported(p) && (query || (aligned16(x) && aligned16(dy)));
   switch (path) {
     case GCONV_PATH_GENERIC:
@@ -209,7 +213,7 @@ int wgrad_choose(const Conv2d& p, int path, const void* x, const void* dy, gconv
     case GCONV_PATH_DIRECT:
       if (tma_ok) return GCONV_KERNEL_WGRAD_DW3_TMA;
       if (dw_ok) return GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC;
-      return tl_ok ? GCONV_KERNEL_WGRAD_TILED_NHWC : GCONV_KERNEL_WGRAD_GENERIC;
+      return tl_ok ? tl_kernel : GCONV_KERNEL_WGRAD_GENERIC;
     case GCONV_PATH_IGEMM:
       *why = GCONV_ERR_UNSUPPORTED;   // no tensor-core weight gradient
       return -1;

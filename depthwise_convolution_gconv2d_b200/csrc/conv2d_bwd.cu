@@ -667,16 +667,52 @@ __global__ void __launch_bounds__(256) wgrad_tiled_nhwc_kernel(const T* __restri
   }
 }
 
+// [N][C][P] -> [N][P][C] for 16-bit elements (NCHW -> NHWC staging of the tiled weight
+// gradient), through 32 x 32 shared-memory tiles: reads run along P, writes along C.
+__global__ void __launch_bounds__(256) to_nhwc16_kernel(const unsigned short* __restrict__ src,
+                                                         unsigned short* __restrict__ dst,
+                                                         int C, long long P) {
+  __shared__ unsigned short tile[32][34];
+  const long long n = blockIdx.z;
+  const long long p0 = (long long)blockIdx.x * 32;
+  const int c0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + i;
+    const long long pp = p0 + tx;
+    if (c < C && pp < P) tile[i][tx] = src[(n * C + c) * P + pp];
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const long long pp = p0 + i;
+    const int c = c0 + tx;
+    if (c < C && pp < P) dst[(n * P + pp) * C + c] = tile[tx][i];
+  }
+}
+
+size_t staged_bytes(long long elems) { return ((size_t)elems * 2 + 255) / 256 * 256; }
+
+cudaError_t launch_to_nhwc16(const void* src, void* dst, int N, int C, long long P,
+                             cudaStream_t s) {
+  const dim3 grid((unsigned)((P + 31) / 32), (unsigned)((C + 31) / 32), (unsigned)N);
+  to_nhwc16_kernel<<<grid, dim3(32, 8), 0, s>>>((const unsigned short*)src,
+                                               (unsigned short*)dst, C, P);
+  return cudaGetLastError();
+}
+
 // dw from the slice partials: dw[e(q)] = sum over slices s of ws[s][q], q the partial index.
 // A CTA takes 32 consecutive q (one per lane, so each warp load is 128 contiguous bytes) and its
 // 8 warps split the slices: warp j adds slices j, j+8, j+16, ... in that order, then the 8 warp
 // sums are added in warp order -- a fixed order, so the result is bitwise reproducible.
-// TAP_MAJOR: partials are [s][tap][C] and e = c * taps + tap (the depthwise kernel); otherwise
-// e = q.
-template <typename T, bool TAP_MAJOR>
+// Partial order -> dw index e: SUM_SAME e = q; SUM_TAP_MAJOR partials are [s][tap][C] and
+// e = c * taps + tap (the depthwise kernels); SUM_TO_NCHW partials are in the NHWC weight order
+// (co, kh, kw, ci) and e is the NCHW weight order (co, ci, kh, kw).
+enum { SUM_SAME = 0, SUM_TAP_MAJOR = 1, SUM_TO_NCHW = 2 };
+
+template <typename T, int MODE>
 __global__ void __launch_bounds__(256) wgrad_sum_kernel(const float* __restrict__ ws,
                                                          T* __restrict__ dw, long long E,
-                                                         int S, int taps) {
+                                                         int S, int taps, int cpg_in, int kW) {
   __shared__ float part[8][33];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long q = (long long)blockIdx.x * 32 + lane;
@@ -692,9 +728,14 @@ __global__ void __launch_bounds__(256) wgrad_sum_kernel(const float* __restrict_
 #pragma unroll
     for (int j = 1; j < 8; ++j) t += part[j][lane];
     long long e = q;
-    if (TAP_MAJOR) {
+    if (MODE == SUM_TAP_MAJOR) {
       const long long C = E / taps;
       e = (q % C) * taps + q / C;
+    } else if (MODE == SUM_TO_NCHW) {
+      const long long ci = q % cpg_in, r = q / cpg_in;   // r = (co * kH + kh) * kW + kw
+      const long long tap = r % taps, co = r / taps;     // tap = kh * kW + kw
+      e = (co * cpg_in + ci) * taps + tap;
+      (void)kW;
     }
     dw[e] = Elem<T>::from_f32(t);
   }
@@ -819,21 +860,42 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
       cudaError_t e = p.stride == 1 ? launch_dww<T, 1>(p, x, dy, (float*)ws, P, s)
                                     : launch_dww<T, 2>(p, x, dy, (float*)ws, P, s);
       if (e != cudaSuccess) return e;
-      wgrad_sum_kernel<T, true><<<sum_grid(E), 256, 0, s>>>((const float*)ws, (T*)dw, E,
-                                                            P.slices, 9);
+      wgrad_sum_kernel<T, SUM_TAP_MAJOR><<<sum_grid(E), 256, 0, s>>>((const float*)ws, (T*)dw,
+                                                                     E, P.slices, 9, 1, 3);
       return cudaGetLastError();
     }
-    if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC) {
+    if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC || kernel == GCONV_KERNEL_WGRAD_TILED_NCHW) {
+      Conv2d q = p;
+      q.layout = GCONV_NHWC;
+      const T* xt = (const T*)x;
+      const T* dt = (const T*)dy;
+      float* part = (float*)ws;
+      if (kernel == GCONV_KERNEL_WGRAD_TILED_NCHW) {
+        // stage x and dy as NHWC at the front of the workspace, partials after them
+        const size_t xb = staged_bytes((long long)p.N * p.C_in * p.H * p.W);
+        const size_t db = staged_bytes((long long)p.N * p.C_out * p.Ho * p.Wo);
+        T* xs = (T*)ws;
+        T* ds = (T*)((char*)ws + xb);
+        part = (float*)((char*)ws + xb + db);
+        cudaError_t e = launch_to_nhwc16(x, xs, p.N, p.C_in, (long long)p.H * p.W, s);
+        if (e == cudaSuccess) e = launch_to_nhwc16(dy, ds, p.N, p.C_out, (long long)p.Ho * p.Wo, s);
+        if (e != cudaSuccess) return e;
+        xt = xs;
+        dt = ds;
+      }
       int n_mt, n_nt, S, per;
-      tiled_tiles(p, &n_mt, &n_nt);
-      const long long tiles = tiled_count(p);
-      tiled_slices(p, tiles, &S, &per);
+      tiled_tiles(q, &n_mt, &n_nt);
+      const long long tiles = tiled_count(q);
+      tiled_slices(q, tiles, &S, &per);
       wgrad_tiled_nhwc_kernel<T><<<dim3((unsigned)tiles, (unsigned)S), 256, 0, s>>>(
-          (const T*)x, (const T*)dy, (float*)ws, p, n_mt, n_nt, E, per);
+          xt, dt, part, q, n_mt, n_nt, E, per);
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
-      wgrad_sum_kernel<T, false><<<sum_grid(E), 256, 0, s>>>((const float*)ws,
-                                                                            (T*)dw, E, S, 1);
+      if (kernel == GCONV_KERNEL_WGRAD_TILED_NCHW)
+        wgrad_sum_kernel<T, SUM_TO_NCHW><<<sum_grid(E), 256, 0, s>>>(
+            part, (T*)dw, E, S, p.kH * p.kW, p.cpg_in, p.kW);
+      else
+        wgrad_sum_kernel<T, SUM_SAME><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S, 1, 1, 1);
       return cudaGetLastError();
     }
   }
@@ -856,8 +918,8 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
       wgrad_depthwise_nhwc_kernel<T, 5, 2, 2><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wgrad_sum_kernel<T, true><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S,
-                                                                          p.kH * p.kW);
+    wgrad_sum_kernel<T, SUM_TAP_MAJOR><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S,
+                                                                   p.kH * p.kW, 1, p.kW);
     return cudaGetLastError();
    }
   }
@@ -869,7 +931,7 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
                                                             E, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  wgrad_sum_kernel<T, false><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S, 1);
+  wgrad_sum_kernel<T, SUM_SAME><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S, 1, 1, 1);
   return cudaGetLastError();
 }
 
@@ -926,7 +988,10 @@ bool wgrad_depthwise_supported(const Conv2d& p) {
 }
 
 bool wgrad_tiled_supported(const Conv2d& p) {
-  return p.layout == GCONV_NHWC && p.dtype != GCONV_F32 && p.cpg_in >= 32 && p.cpg_out >= 32 &&
+  const bool staging_ok = p.layout == GCONV_NHWC ||
+                          (p.N <= 65535 && (p.H * (long long)p.W + 31) / 32 <= 0x7fffffffLL &&
+                           (p.C_in + 31) / 32 <= 65535 && (p.C_out + 31) / 32 <= 65535);
+  return staging_ok && p.dtype != GCONV_F32 && p.cpg_in >= 32 && p.cpg_out >= 32 &&
          p.cpg_in % 8 == 0 && p.cpg_out % 8 == 0 && tiled_count(p) <= 0x7fffffffLL &&
          (long long)p.N * p.Ho * p.Wo <= 0x7fffffffLL;
 }
@@ -935,10 +1000,14 @@ size_t wgrad_workspace(const Conv2d& p, int kernel) {
   if ((long long)p.N * p.Ho == 0) return 0;
   if (kernel == GCONV_KERNEL_WGRAD_DW3_TMA)
     return (size_t)dww_params(p).slices * 9 * (size_t)p.C_in * sizeof(float);
-  if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC) {
+  if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC || kernel == GCONV_KERNEL_WGRAD_TILED_NCHW) {
     int S, per;
     tiled_slices(p, tiled_count(p), &S, &per);
-    return (size_t)S * (size_t)p.C_out * p.cpg_in * p.kH * p.kW * sizeof(float);
+    size_t b = (size_t)S * (size_t)p.C_out * p.cpg_in * p.kH * p.kW * sizeof(float);
+    if (kernel == GCONV_KERNEL_WGRAD_TILED_NCHW)
+      b += staged_bytes((long long)p.N * p.C_in * p.H * p.W) +
+           staged_bytes((long long)p.N * p.C_out * p.Ho * p.Wo);
+    return b;
   }
   int S, rows;
   wgrad_slices(p, wgrad_blocks_x(p, kernel), &S, &rows);

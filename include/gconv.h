@@ -116,9 +116,11 @@ typedef enum {
   GCONV_KERNEL_WGRAD_TILED_NHWC = 13, /* conv2d weight gradient, 16-bit NHWC, C_in/g and
                                          C_out/g >= 32 and multiples of 8: shared-memory tiled
                                          outer products on the CUDA cores */
-  GCONV_KERNEL_WGRAD_DW3_TMA = 14     /* conv2d weight gradient, depthwise 3x3, dilation 1,
+  GCONV_KERNEL_WGRAD_DW3_TMA = 14,    /* conv2d weight gradient, depthwise 3x3, dilation 1,
                                          stride 1 or 2, pad <= 2, 16-bit NHWC, C % 8 == 0:
                                          x and dy staged by TMA */
+  GCONV_KERNEL_WGRAD_TILED_NCHW = 15  /* GCONV_KERNEL_WGRAD_TILED_NHWC for NCHW tensors: x and
+                                         dy transposed to NHWC in the workspace first */
 } gconv_kernel;
 
 /* Bytes of workspace gconv2d_fwd needs for this problem under `path` (0 if none; also 0 for
@@ -212,9 +214,11 @@ size_t gconv2d_bwd_weight_workspace_size(int N, int C_in, int H, int W, int C_ou
  * in slice order (no float atomics), so repeated calls -- on any GPU -- give bitwise-identical
  * dw. AUTO and DIRECT run the TMA-staged depthwise 3x3 kernel where it applies
  * (GCONV_KERNEL_WGRAD_DW3_TMA; x and dy 16-byte aligned), else the depthwise kernel
- * (GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC; x and dy 4-byte aligned), else the tiled kernel for wide groups
- * (GCONV_KERNEL_WGRAD_TILED_NHWC; x and dy 16-byte aligned), else the generic kernel; GENERIC forces the generic kernel;
- * IGEMM is UNSUPPORTED (there is no tensor-core weight gradient). N*Ho > 2^30 is UNSUPPORTED.
+ * (GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC; x and dy 4-byte aligned), else the tiled kernel for
+ * wide groups (GCONV_KERNEL_WGRAD_TILED_NHWC with x and dy 16-byte aligned, or
+ * GCONV_KERNEL_WGRAD_TILED_NCHW, which stages NCHW x and dy as NHWC in the workspace), else
+ * the generic kernel; GENERIC forces the generic kernel; IGEMM is UNSUPPORTED (there is no
+ * tensor-core weight gradient). N*Ho > 2^30 is UNSUPPORTED.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 gconv_status gconv2d_bwd_weight(const void* x, const void* dy, void* dw, int N, int C_in, int H,
                                 int W, int C_out, int kH, int kW, int stride, int pad,

@@ -203,7 +203,7 @@ def test_bwd_path_selection(lib):
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 3
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 4
     assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 13
-    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 10
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 15   # NCHW: staged
     assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, path=3) == 10
     assert sel(wg, 1, 64, 56, 56, 64, 3, 1, 1, 1, 4) == 10          # 16 channels a group
     # narrow groups (4 channels): the narrow-group forward kernel
@@ -239,3 +239,8 @@ def test_bwd_workspace_queries(lib):
         n = lib.gconv2d_bwd_weight_workspace_size(*args)
         E = args[4] * (args[1] // args[10]) * args[5] * args[6]
         assert n > 0 and n % (4 * E) == 0
+    # NCHW wide groups: x and dy staged as NHWC (256-byte rounded) ahead of the partials
+    nchw = (1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 0, 2, 0)
+    n = lib.gconv2d_bwd_weight_workspace_size(*nchw)
+    staged = 2 * (512 * 256 * 256 * 2)
+    assert n > staged and (n - staged) % (4 * 512 * 128 * 9) == 0
