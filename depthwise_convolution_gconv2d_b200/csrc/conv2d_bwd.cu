@@ -14,13 +14,18 @@
 // roles of C_in and C_out exchanged, input dy (Ho x Wo), pad' = dil*(k-1) - pad, and per group
 // the filter transposed (ci <-> co) and rotated by 180 degrees. `flip_transpose_weight_kernel`
 // writes that filter into the caller's workspace and the forward kernels (tensor cores,
-// depthwise, narrow groups) run the rest. Other shapes take the gather kernel below.
+// depthwise, narrow groups) run the rest. Other depthwise shapes (stride 2, larger pads) take a
+// gather kernel on 16-byte channel vectors, everything else a one-thread-per-element gather.
 //
 // The weight gradient is a reduction over N*Ho*Wo positions per filter tap. It is
-// deterministic: the (n, ho) rows are cut into fixed slices (a function of the shape only),
-// each slice's partial sums are accumulated in a fixed order into fp32 workspace slots, and a
+// deterministic: the work is cut into fixed slices (a function of the shape only), each
+// slice's partial sums are accumulated in a fixed order into fp32 workspace slots, and a
 // second kernel adds the slices in slice order and rounds once to the data type. No float
-// atomics, so repeated calls give bitwise-identical dw on any GPU.
+// atomics, so repeated calls give bitwise-identical dw on any GPU. Kernels, most specific
+// first: depthwise 3x3 on a TMA ring (the forward 3x3 kernel's data path with filter and
+// output exchanged), depthwise 3x3 / 5x5 with register chunks, wide groups as shared-memory
+// tiled outer products per (group, tap) on the CUDA cores (NCHW through an NHWC staging copy),
+// and a one-thread-per-entry generic kernel.
 #include "internal.cuh"
 #include "sm100_ptx.cuh"
 
