@@ -426,8 +426,7 @@ DwwParams dww_params(const Conv2d& p) {
   P.n_ct = (p.C_in + DWW_CH - 1) / DWW_CH;
   P.n_ht = (p.Ho + BH - 1) / BH;
   P.n_wt = (p.Wo + DWW_BW - 1) / DWW_BW;
-  const long long tpc = (long long)p.N * P.n_ht * P.n_wt;
-  P.tiles_per_ct = tpc > 0x7fffffffLL ? 0x7fffffff : (int)tpc;
+  P.tiles_per_ct = (int)((long long)p.N * P.n_ht * P.n_wt);   // < 2^31: checked on support
   int sl = DWW_CTAS / P.n_ct;
   if (sl < 1) sl = 1;
   P.slices = sl;
@@ -983,7 +982,9 @@ cudaError_t launch_dgrad_depthwise(const Conv2d& p, const void* dy, const void* 
 bool wgrad_dw3_tma_supported(const Conv2d& p) {
   return p.layout == GCONV_NHWC && p.dtype != GCONV_F32 && p.groups == p.C_in &&
          p.C_out == p.C_in && p.kH == 3 && p.kW == 3 && p.dil == 1 &&
-         (p.stride == 1 || p.stride == 2) && p.pad <= 2 && p.C_in % 8 == 0;
+         (p.stride == 1 || p.stride == 2) && p.pad <= 2 && p.C_in % 8 == 0 &&
+         (long long)p.N * ((p.Ho + dww_bh<2>() - 1) / dww_bh<2>()) *
+                 ((p.Wo + DWW_BW - 1) / DWW_BW) <= 0x7fffffffLL;   // tiles of a channel tile
 }
 
 bool wgrad_depthwise_supported(const Conv2d& p) {
