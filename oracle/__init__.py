@@ -12,6 +12,8 @@ Definitions followed (see the header of ``oracle.c`` for the full statement):
     "F.conv2d runs x15 slower in mixed-precision/half-precision mode";
   * the data and weight gradients of grouped conv2d (scatter / direct-sum forms of the
     forward sum's adjoint), for the training uses of grouped layers on the pages;
+  * the depthwise-separable block (depthwise conv, then a pointwise 1x1 conv over channels)
+    of the same Conformer thread, 1-D and 2-D;
   * depthwise conv1d on (batch, steps, channels), forward and backward -- "Investigate
     custom Triton kernels for depthwise-separable convolutions in Conformer".
 
@@ -66,6 +68,12 @@ def _configure(lib):
         f = getattr(lib, name)
         f.argtypes = [P, P, P] + [L] * 6
         f.restype = I
+    lib.oracle_dwsep1d_fwd.argtypes = [P] * 6 + [L] * 7
+    lib.oracle_dwsep1d_fwd.restype = I
+    lib.oracle_dwsep1d_points.argtypes = [P] * 6 + [L] * 8
+    lib.oracle_dwsep1d_points.restype = I
+    lib.oracle_dwsep2d_fwd.argtypes = [P] * 6 + [L] * 10 + [I]
+    lib.oracle_dwsep2d_fwd.restype = I
     lib.oracle_conv_out_extent.argtypes = [L] * 5
     lib.oracle_conv_out_extent.restype = L
     lib.oracle_num_threads.argtypes = []
@@ -285,3 +293,67 @@ def dwconv1d_bwd_weight(x, dy, K, pad_left, pad_right):
                                           pad_right) != 0:
         raise ValueError("oracle_dwconv1d_bwd_weight rejected the shape")
     return dw
+
+
+def _dwsep_pw(w_pw, bias, C):
+    w_pw = _f64(w_pw)
+    if w_pw.ndim != 2 or w_pw.shape[1] != C:
+        raise ValueError("w_pw must be [C_out, C]")
+    b = None if bias is None else _f64(bias)
+    if b is not None and b.shape != (w_pw.shape[0],):
+        raise ValueError("bias must be [C_out]")
+    return w_pw, b
+
+
+def dwsep1d_fwd(x, w_dw, w_pw, bias, pad_left, pad_right):
+    """Depthwise-separable block on (batch, steps, channels): z = pointwise(dwconv1d(x)),
+    z[b,t,o] = bias[o] + sum_c w_pw[o,c] * dwconv1d_fwd(x, w_dw)[b,t,c]."""
+    x, w_dw = _f64(x), _f64(w_dw)
+    B, T, C, K = _conv1d_check(x.shape, w_dw.shape)
+    w_pw, b = _dwsep_pw(w_pw, bias, C)
+    T_out = T + pad_left + pad_right - K + 1
+    y = np.empty((B, max(T_out, 0), C))
+    z = np.empty((B, max(T_out, 0), w_pw.shape[0]))
+    if _load().oracle_dwsep1d_fwd(_ptr(x), _ptr(w_dw), _ptr(w_pw), _ptr(b), _ptr(y), _ptr(z), B,
+                                  T, C, K, pad_left, pad_right, w_pw.shape[0]) != 0:
+        raise ValueError("oracle_dwsep1d_fwd rejected the shape")
+    return z
+
+
+def dwsep1d_points(x, w_dw, w_pw, bias, idx, pad_left, pad_right):
+    """Outputs of the 1-D depthwise-separable block at idx[i] = (b, t, o)."""
+    x, w_dw = _f64(x), _f64(w_dw)
+    B, T, C, K = _conv1d_check(x.shape, w_dw.shape)
+    w_pw, b = _dwsep_pw(w_pw, bias, C)
+    idx = np.ascontiguousarray(idx, dtype=np.int64).reshape(-1, 3)
+    out = np.empty(idx.shape[0])
+    if _load().oracle_dwsep1d_points(_ptr(x), _ptr(w_dw), _ptr(w_pw), _ptr(b), _ptr(out),
+                                     _ptr(idx), idx.shape[0], B, T, C, K, pad_left, pad_right,
+                                     w_pw.shape[0]) != 0:
+        raise ValueError("oracle_dwsep1d_points rejected the shape or an index")
+    return out
+
+
+def dwsep2d_fwd(x, w_dw, w_pw, bias=None, stride=1, pad=0, dilation=1, layout=NCHW):
+    """2-D depthwise-separable block: z = pointwise(depthwise conv2d(x)); x and z in `layout`,
+    w_dw the depthwise weight of that layout ([C,1,kH,kW] / [C,kH,kW,1]), w_pw [C_out, C]."""
+    x, w_dw = _f64(x), _f64(w_dw)
+    if layout == NCHW:
+        N, C, H, W = x.shape
+        C2, one, kH, kW = w_dw.shape
+    else:
+        N, H, W, C = x.shape
+        C2, kH, kW, one = w_dw.shape
+    if C2 != C or one != 1:
+        raise ValueError("w_dw must be the depthwise weight of x's channels")
+    w_pw, b = _dwsep_pw(w_pw, bias, C)
+    y_shape = conv2d_out_shape(x.shape, w_dw.shape, stride, pad, dilation, C, layout)
+    y = np.empty(y_shape)
+    C_out = w_pw.shape[0]
+    z_shape = (y_shape[0], C_out, y_shape[2], y_shape[3]) if layout == NCHW else (
+        y_shape[0], y_shape[1], y_shape[2], C_out)
+    z = np.empty(z_shape)
+    if _load().oracle_dwsep2d_fwd(_ptr(x), _ptr(w_dw), _ptr(w_pw), _ptr(b), _ptr(y), _ptr(z), N,
+                                  C, H, W, kH, kW, stride, pad, dilation, C_out, layout) != 0:
+        raise ValueError("oracle_dwsep2d_fwd rejected the shape")
+    return z

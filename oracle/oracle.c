@@ -23,6 +23,8 @@
  *    adjoint (scatter form) of the forward sum.
  *  - The grouped conv2d's own data and weight gradients, in the same scatter /
  *    direct-sum forms, for the training uses of grouped layers on the pages.
+ *  - The depthwise-separable block of the Conformer thread: a depthwise
+ *    convolution followed by a pointwise (1x1) convolution over channels.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *  - output size  Ho = floor((H + 2*pad - dil*(kH-1) - 1)/stride) + 1 (PyTorch's
@@ -345,6 +347,95 @@ int oracle_dwconv1d_bwd_weight(const double* x, const double* dy, double* dw, lo
         }
       dw[c * K + k] = acc;
     }
+  return 0;
+}
+
+/* ---------------- depthwise-separable block ---------------- */
+/* A depthwise convolution followed by a pointwise (1x1, dense) convolution over channels: the
+ * "depthwise-separable convolutions in Conformer" of the Conformer thread (the convolution
+ * module's depthwise conv1d on (batch, steps, channels), and the strided depthwise-separable
+ * Conv2D of Fast Conformer's downsampler named in its Oct 30 comment):
+ *   y[..., c] = depthwise(x)[..., c]        (the dwconv1d / depthwise conv2d above)
+ *   z[..., o] = bpw[o] + sum_c wpw[o][c] * y[..., c]
+ * computed as that composition in fp64 (no rounding of y). wpw is [C_out][C]. */
+
+/* 1-D: x [B][T][C], wdw [C][K], wpw [C_out][C], z [B][T_out][C_out]; y is caller scratch
+ * [B][T_out][C]. */
+int oracle_dwsep1d_fwd(const double* x, const double* wdw, const double* wpw, const double* bpw,
+                       double* y, double* z, long B, long T, long C, long K, long pl, long pr,
+                       long C_out) {
+  if (C_out <= 0) return -1;
+  if (oracle_dwconv1d_fwd(x, wdw, y, B, T, C, K, pl, pr)) return -1;
+  long rows = B * (T + pl + pr - K + 1);
+#pragma omp parallel for schedule(static)
+  for (long r = 0; r < rows; ++r)
+    for (long o = 0; o < C_out; ++o) {
+      double acc = bpw ? bpw[o] : 0.0;
+      for (long c = 0; c < C; ++c) acc += wpw[o * C + c] * y[r * C + c];
+      z[r * C_out + o] = acc;
+    }
+  return 0;
+}
+
+/* One output z[b][t][o] of the 1-D block, summed directly over (c, k). */
+static double dwsep1d_point(const double* x, const double* wdw, const double* wpw,
+                            const double* bpw, long T, long C, long K, long pl, long b, long t,
+                            long o) {
+  double acc = bpw ? bpw[o] : 0.0;
+  for (long c = 0; c < C; ++c) {
+    double yc = 0.0;
+    for (long k = 0; k < K; ++k) {
+      long s = t + k - pl;
+      if (s < 0 || s >= T) continue;
+      yc += wdw[c * K + k] * x[(b * T + s) * C + c];
+    }
+    acc += wpw[o * C + c] * yc;
+  }
+  return acc;
+}
+
+/* Selected outputs idx[3i..3i+2] = (b, t, o) of the 1-D block. */
+int oracle_dwsep1d_points(const double* x, const double* wdw, const double* wpw,
+                          const double* bpw, double* out, const int64_t* idx, long npts, long B,
+                          long T, long C, long K, long pl, long pr, long C_out) {
+  if (!conv1d_ok(B, T, C, K, pl, pr) || C_out <= 0) return -1;
+  long T_out = T + pl + pr - K + 1;
+  for (long i = 0; i < npts; ++i) {
+    long b = idx[3 * i], t = idx[3 * i + 1], o = idx[3 * i + 2];
+    if (b < 0 || b >= B || t < 0 || t >= T_out || o < 0 || o >= C_out) return -1;
+  }
+#pragma omp parallel for schedule(static)
+  for (long i = 0; i < npts; ++i)
+    out[i] = dwsep1d_point(x, wdw, wpw, bpw, T, C, K, pl, idx[3 * i], idx[3 * i + 1],
+                           idx[3 * i + 2]);
+  return 0;
+}
+
+/* 2-D: x in `layout` with C channels, wdw the depthwise weight ([C][1][kH][kW] or
+ * [C][kH][kW][1]), wpw [C_out][C], z in `layout` with C_out channels; y is caller scratch with
+ * the depthwise output's shape. */
+int oracle_dwsep2d_fwd(const double* x, const double* wdw, const double* wpw, const double* bpw,
+                       double* y, double* z, long N, long C, long H, long W, long kH, long kW,
+                       long stride, long pad, long dil, long C_out, int layout) {
+  conv2d_shape s;
+  if (C_out <= 0) return -1;
+  if (make_shape(&s, N, C, H, W, C, kH, kW, stride, pad, dil, C, layout)) return -1;
+  if (oracle_conv2d(x, wdw, NULL, y, N, C, H, W, C, kH, kW, stride, pad, dil, C, layout))
+    return -1;
+  long HW = s.Ho * s.Wo;
+#pragma omp parallel for schedule(static)
+  for (long np = 0; np < N * HW; ++np) {
+    long n = np / HW, hw = np % HW;
+    for (long o = 0; o < C_out; ++o) {
+      double acc = bpw ? bpw[o] : 0.0;
+      for (long c = 0; c < C; ++c) {
+        long yi = layout == ORACLE_NCHW ? (n * C + c) * HW + hw : (n * HW + hw) * C + c;
+        acc += wpw[o * C + c] * y[yi];
+      }
+      long zi = layout == ORACLE_NCHW ? (n * C_out + o) * HW + hw : (n * HW + hw) * C_out + o;
+      z[zi] = acc;
+    }
+  }
   return 0;
 }
 

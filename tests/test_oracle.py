@@ -556,6 +556,104 @@ def test_conv2d_bwd_points_match_full(case, layout):
     assert np.array_equal(pw, dw[tuple(wi.T)])
 
 
+# ---------------------------------------------------------------- depthwise-separable block
+
+def brute_dwsep1d(x, wd, wp, b, pl, pr):
+    """Pure-Python loops on integers: depthwise over an explicitly padded sequence, then the
+    channel mix."""
+    B, T, C = x.shape
+    K = wd.shape[1]
+    O = wp.shape[0]
+    T_out = T + pl + pr - K + 1
+    xp = [[[0] * C for _ in range(T + pl + pr)] for _ in range(B)]
+    for bb in range(B):
+        for t in range(T):
+            for c in range(C):
+                xp[bb][t + pl][c] = int(x[bb, t, c])
+    z = np.zeros((B, T_out, O), np.int64)
+    for bb in range(B):
+        for t in range(T_out):
+            y = [sum(int(wd[c, k]) * xp[bb][t + k][c] for k in range(K)) for c in range(C)]
+            for o in range(O):
+                z[bb, t, o] = int(b[o]) + sum(int(wp[o, c]) * y[c] for c in range(C))
+    return z
+
+
+DWSEP1D_CASES = [(2, 9, 3, 4, 3, 1, 1), (1, 12, 5, 2, 5, 4, 0), (2, 40, 4, 6, 31, 15, 15),
+                 (1, 33, 3, 3, 31, 30, 0)]
+
+
+@pytest.mark.parametrize("B,T,C,O,K,pl,pr", DWSEP1D_CASES)
+def test_dwsep1d_brute_force(B, T, C, O, K, pl, pr):
+    x, wd = rng_int(70, (B, T, C)), rng_int(71, (C, K))
+    wp, b = rng_int(72, (O, C)), rng_int(73, (O,))
+    assert np.array_equal(oracle.dwsep1d_fwd(x, wd, wp, b, pl, pr),
+                          brute_dwsep1d(x, wd, wp, b, pl, pr).astype(float))
+
+
+@pytest.mark.parametrize("B,T,C,O,K,pl,pr", DWSEP1D_CASES)
+def test_dwsep1d_vs_torch(B, T, C, O, K, pl, pr):
+    """Library pin: torch's conv1d (groups = C) then a 1x1 conv1d, float64 on the CPU."""
+    import torch
+    import torch.nn.functional as F
+    r = np.random.default_rng(74)
+    x, wd = r.standard_normal((B, T, C)), r.standard_normal((C, K))
+    wp, b = r.standard_normal((O, C)), r.standard_normal(O)
+    tx = F.pad(torch.from_numpy(x).permute(0, 2, 1), (pl, pr))
+    y = F.conv1d(tx, torch.from_numpy(wd)[:, None, :], groups=C)
+    z = F.conv1d(y, torch.from_numpy(wp)[:, :, None], torch.from_numpy(b))
+    np.testing.assert_allclose(oracle.dwsep1d_fwd(x, wd, wp, b, pl, pr),
+                               z.permute(0, 2, 1).numpy(), rtol=1e-11, atol=1e-11)
+
+
+@pytest.mark.parametrize("stride,pad,dil", [(1, 1, 1), (2, 1, 1), (1, 2, 2), (2, 0, 1)])
+@pytest.mark.parametrize("layout", [NCHW, NHWC])
+def test_dwsep2d_vs_torch(stride, pad, dil, layout):
+    """Library pin: torch's conv2d (groups = C) then a 1x1 conv2d, float64 on the CPU."""
+    import torch
+    import torch.nn.functional as F
+    N, C, H, W, O = 2, 6, 9, 8, 5
+    r = np.random.default_rng(75)
+    x, wd = r.standard_normal((N, C, H, W)), r.standard_normal((C, 1, 3, 3))
+    wp, b = r.standard_normal((O, C)), r.standard_normal(O)
+    y = F.conv2d(torch.from_numpy(x), torch.from_numpy(wd), None, stride, pad, dil, C)
+    ref = F.conv2d(y, torch.from_numpy(wp)[:, :, None, None], torch.from_numpy(b)).numpy()
+    if layout == NCHW:
+        got = oracle.dwsep2d_fwd(x, wd, wp, b, stride, pad, dil, NCHW)
+    else:
+        got = from_nhwc(oracle.dwsep2d_fwd(to_nhwc(x), to_nhwc(wd), wp, b, stride, pad, dil,
+                                           NHWC))
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-11)
+
+
+def test_dwsep_closed_forms():
+    """An identity channel mix leaves the (separately pinned) depthwise result; a depthwise
+    filter with one unit tap at k = pad_left leaves the channel mix x @ w_pw^T + b (numpy)."""
+    r = np.random.default_rng(76)
+    B, T, C, K, pl, pr = 2, 11, 5, 7, 3, 3
+    x, wd = r.standard_normal((B, T, C)), r.standard_normal((C, K))
+    np.testing.assert_allclose(oracle.dwsep1d_fwd(x, wd, np.eye(C), None, pl, pr),
+                               oracle.dwconv1d_fwd(x, wd, pl, pr), rtol=1e-13, atol=1e-13)
+    delta = np.zeros((C, K))
+    delta[:, pl] = 1.0
+    wp, b = r.standard_normal((4, C)), r.standard_normal(4)
+    np.testing.assert_allclose(oracle.dwsep1d_fwd(x, delta, wp, b, pl, pr), x @ wp.T + b,
+                               rtol=1e-12, atol=1e-12)
+    x2 = r.standard_normal((2, 6, 5, C))
+    d2 = np.zeros((C, 3, 3, 1))
+    d2[:, 1, 1, 0] = 1.0
+    np.testing.assert_allclose(oracle.dwsep2d_fwd(x2, d2, wp, b, 1, 1, 1, NHWC), x2 @ wp.T + b,
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_dwsep1d_points_match_full():
+    x, wd = rng_int(77, (2, 20, 6)), rng_int(78, (6, 9))
+    wp, b = rng_int(79, (5, 6)), rng_int(80, (5,))
+    z = oracle.dwsep1d_fwd(x, wd, wp, b, 4, 4)
+    idx = np.array(list(np.ndindex(z.shape)))
+    assert np.array_equal(oracle.dwsep1d_points(x, wd, wp, b, idx, 4, 4), z[tuple(idx.T)])
+
+
 # ---------------------------------------------------------------- planted mistakes
 
 MUTANTS = {
@@ -581,6 +679,9 @@ MUTANTS = {
                                       "long wi = wo * s->stride - s->pad + kw;\n        if (wi < 0 || wi >= s->W) continue;\n        acc += dy"),
     "conv2d_dgrad_points_stride_check": ("if (th < 0 || th % stride != 0 || th / stride >= s.Ho)",
                                          "if (th < 0 || th / stride >= s.Ho)"),
+    "dwsep1d_bias_dropped": ("      double acc = bpw ? bpw[o] : 0.0;\n      for (long c = 0; c < C; ++c) acc += wpw[o * C + c] * y[r * C + c];",
+                             "      double acc = 0.0;\n      for (long c = 0; c < C; ++c) acc += wpw[o * C + c] * y[r * C + c];"),
+    "dwsep2d_channel_reversed": ("(n * HW + hw) * C + c;", "(n * HW + hw) * C + (C - 1 - c);"),
 }
 
 
@@ -598,6 +699,9 @@ def _pins_pass():
             test_conv2d_bwd_brute_force(case, NHWC)
         for case in BWD_CASES:
             test_conv2d_bwd_points_match_full(case, NCHW)
+        for args in DWSEP1D_CASES:
+            test_dwsep1d_brute_force(*args)
+        test_dwsep2d_vs_torch(2, 1, 1, NHWC)
     except AssertionError:
         return False
     return True
