@@ -12,6 +12,8 @@ Definitions followed (see the header of ``oracle.c`` for the full statement):
     "F.conv2d runs x15 slower in mixed-precision/half-precision mode";
   * the data and weight gradients of grouped conv2d (scatter / direct-sum forms of the
     forward sum's adjoint), for the training uses of grouped layers on the pages;
+  * the neon thread's output variants: interleaved (1234...) output order and average / max
+    merges across groups;
   * the depthwise-separable block (depthwise conv, then a pointwise 1x1 conv over channels)
     of the same Conformer thread, 1-D and 2-D;
   * depthwise conv1d on (batch, steps, channels), forward and backward -- "Investigate
@@ -68,6 +70,10 @@ def _configure(lib):
         f = getattr(lib, name)
         f.argtypes = [P, P, P] + [L] * 6
         f.restype = I
+    lib.oracle_conv2d_interleaved.argtypes = [P, P, P, P] + [L] * 11 + [I]
+    lib.oracle_conv2d_interleaved.restype = I
+    lib.oracle_conv2d_group_merge.argtypes = [P, P, P, P] + [L] * 11 + [I, I]
+    lib.oracle_conv2d_group_merge.restype = I
     lib.oracle_dwsep1d_fwd.argtypes = [P] * 6 + [L] * 7
     lib.oracle_dwsep1d_fwd.restype = I
     lib.oracle_dwsep1d_points.argtypes = [P] * 6 + [L] * 8
@@ -156,6 +162,40 @@ def conv2d_points(x, w, idx, bias=None, stride=1, pad=0, dilation=1, groups=1, l
     if rc != 0:
         raise ValueError("oracle_conv2d_points rejected the shape or an index")
     return out
+
+
+def conv2d_interleaved(x, w, bias=None, stride=1, pad=0, dilation=1, groups=1, layout=NCHW):
+    """Grouped conv2d with the interleaved output order: position j*groups + i holds filter j
+    of group i (group-major channel i*cpg_out + j)."""
+    x, w = _f64(x), _f64(w)
+    b = None if bias is None else _f64(bias)
+    N, C_in, H, W, C_out, kH, kW = _conv_args(x, w, groups, layout)
+    y = np.empty(conv2d_out_shape(x.shape, w.shape, stride, pad, dilation, groups, layout))
+    if _load().oracle_conv2d_interleaved(_ptr(x), _ptr(w), _ptr(b), _ptr(y), N, C_in, H, W,
+                                         C_out, kH, kW, stride, pad, dilation, groups,
+                                         layout) != 0:
+        raise ValueError("oracle_conv2d_interleaved rejected the shape")
+    return y
+
+
+def conv2d_group_merge(x, w, bias=None, stride=1, pad=0, dilation=1, groups=1, layout=NCHW,
+                       mode="avg"):
+    """Grouped conv2d merged across groups: channel j = mean ('avg') or max ('max') over
+    groups i of group-major channel i*cpg_out + j; cpg_out output channels."""
+    x, w = _f64(x), _f64(w)
+    b = None if bias is None else _f64(bias)
+    N, C_in, H, W, C_out, kH, kW = _conv_args(x, w, groups, layout)
+    full = conv2d_out_shape(x.shape, w.shape, stride, pad, dilation, groups, layout)
+    cpg_out = C_out // groups
+    shape = (full[0], cpg_out, full[2], full[3]) if layout == NCHW else (
+        full[0], full[1], full[2], cpg_out)
+    y = np.empty(shape)
+    code = {"avg": 0, "max": 1}[mode]
+    if _load().oracle_conv2d_group_merge(_ptr(x), _ptr(w), _ptr(b), _ptr(y), N, C_in, H, W,
+                                         C_out, kH, kW, stride, pad, dilation, groups, layout,
+                                         code) != 0:
+        raise ValueError("oracle_conv2d_group_merge rejected the shape")
+    return y
 
 
 def _bwd_dims(dy_shape, w_shape, in_hw, stride, pad, dilation, groups, layout):

@@ -25,6 +25,8 @@
  *    direct-sum forms, for the training uses of grouped layers on the pages.
  *  - The depthwise-separable block of the Conformer thread: a depthwise
  *    convolution followed by a pointwise (1x1) convolution over channels.
+ *  - The neon thread's output variants: interleaved (1234...) output order and
+ *    average / max merges across groups.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *  - output size  Ho = floor((H + 2*pad - dil*(kH-1) - 1)/stride) + 1 (PyTorch's
@@ -277,6 +279,62 @@ int oracle_conv2d_bwd_weight_points(const double* x, const double* dy, double* o
   for (long i = 0; i < npts; ++i)
     out[i] = conv2d_wgrad_entry(&s, x, dy, idx[4 * i], idx[4 * i + 1], idx[4 * i + 2],
                                 idx[4 * i + 3]);
+  return 0;
+}
+
+/* ---------------- output orderings and merges across groups ---------------- */
+/* Interleaved output order: ibmua's post on output orderings in "Grouped convolutions" (neon
+ * issue #296) asks for the feature maps as 1234123412341234 instead of the usual group-major
+ * 111122223333444. Output position p = j * groups + i holds filter j of group i, i.e. the
+ * group-major output channel i * cpg_out + j. y has the forward output's shape. */
+int oracle_conv2d_interleaved(const double* x, const double* w, const double* bias, double* y,
+                              long N, long C_in, long H, long W, long C_out, long kH, long kW,
+                              long stride, long pad, long dil, long groups, int layout) {
+  conv2d_shape s;
+  if (make_shape(&s, N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups, layout)) return -1;
+  long cpg_out = C_out / groups;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long np = 0; np < N * C_out; ++np) {
+    long n = np / C_out, pos = np % C_out;
+    long i = pos % groups, j = pos / groups;
+    long co = i * cpg_out + j;
+    for (long ho = 0; ho < s.Ho; ++ho)
+      for (long wo = 0; wo < s.Wo; ++wo)
+        y[y_index(&s, n, pos, ho, wo)] = conv2d_point(&s, x, w, bias, n, co, ho, wo);
+  }
+  return 0;
+}
+
+/* Merge across groups: the same post wants the groups' results pulled together by average or
+ * max pooling across groups (volumetric pooling over the interleaved order), and the next
+ * post combines groups through a 1x1 layer for want of Avg / Max. Output channel j < cpg_out
+ * is the mean (mode 0) or the maximum (mode 1) over groups i of group-major channel
+ * i * cpg_out + j; y is [N][cpg_out][Ho][Wo] (NCHW) or [N][Ho][Wo][cpg_out] (NHWC). */
+int oracle_conv2d_group_merge(const double* x, const double* w, const double* bias, double* y,
+                              long N, long C_in, long H, long W, long C_out, long kH, long kW,
+                              long stride, long pad, long dil, long groups, int layout,
+                              int mode) {
+  conv2d_shape s;
+  if (mode != 0 && mode != 1) return -1;
+  if (make_shape(&s, N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups, layout)) return -1;
+  long cpg_out = C_out / groups;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long nj = 0; nj < N * cpg_out; ++nj) {
+    long n = nj / cpg_out, j = nj % cpg_out;
+    for (long ho = 0; ho < s.Ho; ++ho)
+      for (long wo = 0; wo < s.Wo; ++wo) {
+        double m = 0.0;
+        for (long i = 0; i < groups; ++i) {
+          double v = conv2d_point(&s, x, w, bias, n, i * cpg_out + j, ho, wo);
+          if (mode == 0) m += v;
+          else if (i == 0 || v > m) m = v;
+        }
+        if (mode == 0) m /= (double)groups;
+        long yi = layout == ORACLE_NCHW ? ((n * cpg_out + j) * s.Ho + ho) * s.Wo + wo
+                                        : ((n * s.Ho + ho) * s.Wo + wo) * cpg_out + j;
+        y[yi] = m;
+      }
+  }
   return 0;
 }
 

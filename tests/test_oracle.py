@@ -556,6 +556,109 @@ def test_conv2d_bwd_points_match_full(case, layout):
     assert np.array_equal(pw, dw[tuple(wi.T)])
 
 
+# ---------------------------------------------------------------- output order and group merges
+
+def test_interleaved_order_golden():
+    """The neon thread's alternative output order, 1234123412341234: each output position
+    reads the input group printed at its place."""
+    gold = json.load(open(os.path.join(GOLDEN, "interleaved_order.json")))
+    C, g = gold["C_out"], gold["groups"]
+    cpg = C // g
+    assert gold["expected"] == gold["printed"]
+    x = np.zeros((1, C, 1, 1))
+    for c in range(C):
+        x[0, c] = c // cpg + 1           # input channel carries its group label
+    w = np.ones((C, cpg, 1, 1)) / cpg
+    y = oracle.conv2d_interleaved(x, w, None, 1, 0, 1, g, NCHW)
+    assert "".join(str(int(v)) for v in y[0, :, 0, 0]) == gold["expected"]
+
+
+MERGE_CASES = [(2, 8, 7, 6, 12, 3, 1, 1, 1, 4), (1, 6, 9, 8, 9, 3, 2, 1, 1, 3),
+               (2, 4, 5, 5, 8, 1, 1, 0, 1, 2), (1, 16, 6, 7, 16, 3, 1, 2, 2, 16)]
+
+
+@pytest.mark.parametrize("case", MERGE_CASES)
+@pytest.mark.parametrize("layout", [NCHW, NHWC])
+def test_interleaved_is_reshape_transpose(case, layout):
+    """Interleaved output = the group-major output with its (group, filter) channel axes
+    swapped (numpy reshape / transpose)."""
+    N, C_in, H, W, C_out, k, s, p, d, g = case
+    r = np.random.default_rng(81)
+    x, w = r.standard_normal((N, C_in, H, W)), r.standard_normal((C_out, C_in // g, k, k))
+    b = r.standard_normal(C_out)
+    y = oracle.conv2d(x, w, b, s, p, d, g, NCHW)
+    n, _, Ho, Wo = y.shape
+    ref = y.reshape(n, g, C_out // g, Ho, Wo).transpose(0, 2, 1, 3, 4).reshape(y.shape)
+    if layout == NCHW:
+        got = oracle.conv2d_interleaved(x, w, b, s, p, d, g, NCHW)
+    else:
+        got = from_nhwc(oracle.conv2d_interleaved(to_nhwc(x), to_nhwc(w), b, s, p, d, g, NHWC))
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("case", MERGE_CASES)
+@pytest.mark.parametrize("mode", ["avg", "max"])
+@pytest.mark.parametrize("layout", [NCHW, NHWC])
+def test_group_merge_vs_numpy(case, mode, layout):
+    """Merge across groups = numpy mean / max over the group axis of the group-major output."""
+    N, C_in, H, W, C_out, k, s, p, d, g = case
+    r = np.random.default_rng(82)
+    x, w = r.standard_normal((N, C_in, H, W)), r.standard_normal((C_out, C_in // g, k, k))
+    y = oracle.conv2d(x, w, None, s, p, d, g, NCHW)
+    n, _, Ho, Wo = y.shape
+    yg = y.reshape(n, g, C_out // g, Ho, Wo)
+    ref = yg.mean(axis=1) if mode == "avg" else yg.max(axis=1)
+    if layout == NCHW:
+        got = oracle.conv2d_group_merge(x, w, None, s, p, d, g, NCHW, mode)
+    else:
+        got = from_nhwc(oracle.conv2d_group_merge(to_nhwc(x), to_nhwc(w), None, s, p, d, g,
+                                                  NHWC, mode))
+    np.testing.assert_allclose(got, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_group_merge_is_pooling_over_interleaved_order():
+    """Average / max pooling over windows of `groups` consecutive channels of the interleaved
+    output (the volumetric pooling the thread has in mind) is the merge across groups."""
+    N, C_in, H, W, C_out, k, s, p, d, g = MERGE_CASES[0]
+    r = np.random.default_rng(83)
+    x, w = r.standard_normal((N, C_in, H, W)), r.standard_normal((C_out, C_in // g, k, k))
+    yi = oracle.conv2d_interleaved(x, w, None, s, p, d, g, NCHW)
+    n, _, Ho, Wo = yi.shape
+    win = yi.reshape(n, C_out // g, g, Ho, Wo)
+    np.testing.assert_allclose(oracle.conv2d_group_merge(x, w, None, s, p, d, g, NCHW, "avg"),
+                               win.mean(axis=2), rtol=1e-13, atol=1e-13)
+    assert np.array_equal(oracle.conv2d_group_merge(x, w, None, s, p, d, g, NCHW, "max"),
+                          win.max(axis=2))
+
+
+def test_group_merge_averages_an_ensemble():
+    """The ensemble-as-groups layer merged with 'avg' is the mean of the models' own dense
+    convolutions (P1's ensemble, averaged)."""
+    models, cin, cout = 4, 3, 5
+    r = np.random.default_rng(84)
+    x = r.standard_normal((2, models * cin, 6, 7))
+    w = r.standard_normal((models * cout, cin, 3, 3))
+    got = oracle.conv2d_group_merge(x, w, None, 1, 1, 1, models, NCHW, "avg")
+    ref = np.mean([oracle.conv2d(x[:, m * cin:(m + 1) * cin], w[m * cout:(m + 1) * cout], None,
+                                 1, 1, 1, 1, NCHW) for m in range(models)], axis=0)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_linear_is_per_group_matmul():
+    """A grouped linear layer (the neon thread's gemmBatched use) is the grouped conv2d with
+    H = W = 1 and a 1x1 kernel: per group, y_g = x_g W_g^T + b_g (numpy matmul)."""
+    B, g, i_, o_ = 7, 5, 6, 4
+    r = np.random.default_rng(85)
+    x = r.standard_normal((B, g * i_))
+    w = r.standard_normal((g * o_, i_))
+    b = r.standard_normal(g * o_)
+    y = oracle.conv2d(x[:, :, None, None], w[:, :, None, None], b, 1, 0, 1, g, NCHW)[:, :, 0, 0]
+    for j in range(g):
+        np.testing.assert_allclose(y[:, j * o_:(j + 1) * o_],
+                                   x[:, j * i_:(j + 1) * i_] @ w[j * o_:(j + 1) * o_].T +
+                                   b[j * o_:(j + 1) * o_], rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------- depthwise-separable block
 
 def brute_dwsep1d(x, wd, wp, b, pl, pr):
@@ -682,6 +785,8 @@ MUTANTS = {
     "dwsep1d_bias_dropped": ("      double acc = bpw ? bpw[o] : 0.0;\n      for (long c = 0; c < C; ++c) acc += wpw[o * C + c] * y[r * C + c];",
                              "      double acc = 0.0;\n      for (long c = 0; c < C; ++c) acc += wpw[o * C + c] * y[r * C + c];"),
     "dwsep2d_channel_reversed": ("(n * HW + hw) * C + c;", "(n * HW + hw) * C + (C - 1 - c);"),
+    "interleave_index_swapped": ("long co = i * cpg_out + j;", "long co = j * groups + i;"),
+    "merge_max_is_min": ("else if (i == 0 || v > m) m = v;", "else if (i == 0 || v < m) m = v;"),
 }
 
 
@@ -702,6 +807,10 @@ def _pins_pass():
         for args in DWSEP1D_CASES:
             test_dwsep1d_brute_force(*args)
         test_dwsep2d_vs_torch(2, 1, 1, NHWC)
+        test_interleaved_order_golden()
+        for case in MERGE_CASES:
+            test_interleaved_is_reshape_transpose(case, NCHW)
+            test_group_merge_vs_numpy(case, "max", NCHW)
     except AssertionError:
         return False
     return True
