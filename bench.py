@@ -64,14 +64,56 @@ def kernel_source_hash(name: str) -> str:
 
 
 def traffic_for(kernel: str, source: str):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel is unchanged."""
+    """DRAM read and write bytes per launch from a committed ncu capture, if the kernel's
+    source is unchanged since (None otherwise)."""
     try:
         d = json.load(open(TRAFFIC_FILE)).get(kernel)
     except (OSError, ValueError):
         return None
     if not d or d.get("source_sha") != kernel_source_hash(source):
         return None
-    return d.get("dram_bytes_per_launch")
+    return d
+
+
+# Timed regions shorter than this run at burst clocks (the power cap needs seconds of
+# sustained load to pull the SM clock down), so their roofline uses the burst GEMM peak.
+SUSTAINED_MIN_S = 2.0
+
+
+def tensor_peak_for(pk, timed_s: float, clocks):
+    """(peak TFLOP/s, which) for a kernel timed over `timed_s` seconds: the sustained bf16
+    figure only when the region lasted seconds AND the sampled clocks show the power cap (or
+    a median SM clock under 90 % of max); the burst figure otherwise."""
+    sustained = pk.get("bf16_tflops_sustained")
+    if sustained and timed_s >= SUSTAINED_MIN_S and clocks:
+        capped = "sw_power_cap" in clocks.get("reasons", [])
+        slow = (clocks.get("sm_max_mhz") or 0) > 0 and \
+            clocks["sm_mhz"] < 0.9 * clocks["sm_max_mhz"]
+        if capped or slow:
+            return sustained, "bf16_tflops_sustained"
+    return pk["bf16_tflops"], "bf16_tflops"
+
+
+def compact_rooflines(dwm, more, bwd, extra=None):
+    """One flat map of roofline fractions, named workload_bound, for every secondary
+    workload (the headline has its own roofline object)."""
+    out = {}
+    names = {"depthwise56_s1": "dw56_s1", "depthwise56_s2": "dw56_s2"}
+    for k, v in (dwm or {}).items():
+        if k.startswith("dw1d_") and k.endswith("_cudacore"):
+            continue
+        out[f"{names.get(k, k)}_hbm"] = v["frac"]
+    for k, v in (more or {}).items():
+        if "_direct" in k and v.get("us", 0) > 5000:
+            continue
+        out[f"{k}_{v['bound']}"] = v["frac"]
+        if "ffma_frac" in v:
+            out[f"{k}_ffma"] = v["ffma_frac"]
+    for k, v in (bwd or {}).items():
+        out[f"bwd_{k}_{v['bound']}"] = v["frac"]
+    for k, v in (extra or {}).items():
+        out[f"{k}_{v['bound']}"] = v["frac"]
+    return out
 
 
 class ClockSampler:
@@ -197,6 +239,13 @@ def kernel_name(code: int) -> str:
 
 
 LAUNCHES_PER_CALL = {1: 1, 2: 1, 3: 1, 4: 3, 8: 1}
+CUDA_CORE_KERNELS = (1, 2, 8)
+SM_MAX_MHZ = 1965.0     # B200 clocks.max.sm
+
+
+def ffma_peak_tflops(sms: int = 148, mhz: float = SM_MAX_MHZ) -> float:
+    """FP32 FMA roofline of the CUDA cores: 128 FMA lanes per SM, 2 FLOP per FMA."""
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
 KERNEL_SOURCE = {1: "direct_generic.cu", 2: "depthwise_nhwc.cu", 3: "igemm_tc.cu",
                  4: "igemm_tc.cu", 8: "grouped_nhwc.cu"}
 
@@ -217,13 +266,20 @@ def conv2d_measurement(torch, gb, device, stream, pk, p, workload, path, reps, f
     med, mean = time_launches(torch, fn, stream, reps, flush)
     tf = p.flops() / (med * 1e-3) / 1e12
     gbs = p.bytes() / (med * 1e-3) / 1e9
-    t_tensor = p.flops() / (pk["bf16_tflops"] * 1e12)
     t_hbm = p.bytes() / (pk["hbm_gbs"] * 1e9)
-    bound = "tensor" if t_tensor >= t_hbm else "hbm"
-    frac = max(t_tensor, t_hbm) / (med * 1e-3)
-    return {"kernel": kernel_name(kcode), "us": round(med * 1e3, 2), "TFLOP/s": round(tf, 1),
-            "GB/s": round(gbs, 1), "bound": bound, "frac": round(frac, 3),
-            "alg_flops": p.flops(), "alg_bytes": p.bytes()}
+    rec = {"kernel": kernel_name(kcode), "us": round(med * 1e3, 2), "TFLOP/s": round(tf, 1),
+           "GB/s": round(gbs, 1)}
+    if kcode in CUDA_CORE_KERNELS:
+        # fp32 FMAs on the CUDA cores: the arithmetic roofline is the FFMA rate
+        t_alu = p.flops() / (ffma_peak_tflops() * 1e12)
+        rec["ffma_frac"] = round(tf / ffma_peak_tflops(), 3)
+        bound, t_roof = ("alu", t_alu) if t_alu >= t_hbm else ("hbm", t_hbm)
+    else:
+        t_tensor = p.flops() / (pk["bf16_tflops"] * 1e12)
+        bound, t_roof = ("tensor", t_tensor) if t_tensor >= t_hbm else ("hbm", t_hbm)
+    rec.update({"bound": bound, "frac": round(t_roof / (med * 1e-3), 3),
+                "alg_flops": p.flops(), "alg_bytes": p.bytes()})
+    return rec
 
 
 def more_conv2d_measurements(torch, gb, device, stream, pk, reps):
@@ -589,15 +645,25 @@ def main():
     value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
     avg_launch_ms = sum(launch_ms) / len(launch_ms)
     achieved = flops / (avg_launch_ms * 1e-3) / 1e12
-    # the timed region is a long back-to-back loop (sustained clocks under the power cap), so
-    # the denominator is the sustained bf16 figure; the burst fraction is reported beside it
-    tensor_peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    clocks = clk.summary()
+    tensor_peak, which = tensor_peak_for(pk, total_ms * 1e-3, clocks)
+    tr = traffic_for(kernel_name(kcode), KERNEL_SOURCE.get(kcode, ""))
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tensor_peak,
             "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4),
-            "traffic": traffic_for(kernel_name(kcode), KERNEL_SOURCE.get(kcode, "")),
+            "traffic": tr.get("dram_bytes_per_launch") if tr else None,
             "kernel": kernel_name(kcode),
-            "peak_source": f"bf16_tflops_sustained {peak_src}",
+            "peak_source": f"{which} {peak_src} (timed region {total_ms:.2f} ms)",
             "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4)}
+    if pk.get("bf16_tflops_sustained"):
+        roof["frac_of_sustained_peak"] = round(achieved / pk["bf16_tflops_sustained"], 4)
+    if tr:
+        # reads compare with x + w; the writes of one cold launch miss the part of y that is
+        # still dirty in L2 when the kernel ends (written back after it)
+        roof["traffic_read"] = tr.get("dram_read_bytes")
+        roof["traffic_write"] = tr.get("dram_write_bytes")
+        roof["alg_read"] = p.bytes() - p.N * p.C_out * p.Ho * p.Wo * 2
+        roof["alg_write"] = p.N * p.C_out * p.Ho * p.Wo * 2
+        roof["traffic_scope"] = tr.get("note", "")
     if kcode in (1, 2):   # CUDA-core kernels on this workload are not tensor-bound
         roof["note"] = "CUDA-core path selected; tensor peak used as the headline denominator"
 
@@ -650,6 +716,10 @@ def main():
                "sample": f"first {rows} of {p.H} input rows of the workload, fp64 nested loops, "
                          f"{dt:.1f} s"}
 
+    rooflines = compact_rooflines(dwm, more, bwd)
+    if rooflines:
+        # the secondary workloads' fractions travel inside the headline roofline object too
+        roof["others"] = rooflines
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -659,7 +729,7 @@ def main():
             "config": config_dict(p, argparse.Namespace(layout=args.layout, gpus=world)),
             "kernel": kernel_name(kcode), "roofline": roof, "e2e": e2e,
             "gpu_launches": LAUNCHES_PER_CALL.get(kcode, 1) * args.steps,
-            "clocks": clk.summary(), "cpu_baseline": cpu, "depthwise": dwm,
+            "clocks": clocks, "cpu_baseline": cpu, "rooflines": rooflines, "depthwise": dwm,
             "other_workloads": more, "backward": bwd,
             "device_error": dev_err,
             "peaks": {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],

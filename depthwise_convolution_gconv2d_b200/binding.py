@@ -40,7 +40,7 @@ EXPORTS = ["gconv2d_fwd", "gconv2d_fwd_path", "gconv2d_fwd_workspace_size",
            "gconv2d_bwd_weight_select_path", "dwconv1d_fwd", "dwconv1d_bwd_data", "dwconv1d_fwd_path",
            "dwconv1d_bwd_data_path", "dwconv1d_select_path",
            "dwconv1d_bwd_weight", "dwconv1d_bwd_weight_workspace_size",
-           "dwconv1d_bwd_weight_noalloc",
+           "dwconv1d_bwd_weight_noalloc", "gconv2d_out_shape", "dwconv1d_out_steps",
            "gconv_get_device_error", "gconv_status_string", "gconv_version"]
 
 _lib = None
@@ -106,6 +106,10 @@ def load_library():
     lib.dwconv1d_bwd_weight.restype = I
     lib.dwconv1d_bwd_weight_noalloc.argtypes = [P, P, P] + [I] * 6 + [I, P]
     lib.dwconv1d_bwd_weight_noalloc.restype = I
+    lib.gconv2d_out_shape.argtypes = conv + [I, I, ctypes.POINTER(I), ctypes.POINTER(I)]
+    lib.gconv2d_out_shape.restype = I
+    lib.dwconv1d_out_steps.argtypes = [I] * 7 + [ctypes.POINTER(I)]
+    lib.dwconv1d_out_steps.restype = I
     lib.gconv_get_device_error.argtypes = [P, ctypes.POINTER(I)]
     lib.gconv_get_device_error.restype = I
     lib.gconv_status_string.argtypes = [I]
@@ -155,9 +159,28 @@ def _need(t, name, dtype=None):
         raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
 
 
-def _out_extent(n, k, s, p, d):
-    span = n + 2 * p - d * (k - 1) - 1
-    return span // s + 1 if span >= 0 else 0
+def out_shape(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, layout,
+              dtype):
+    """(Ho, Wo) of a conv2d problem from the library's own shape logic (gconv2d_out_shape);
+    raises GconvError(GCONV_ERR_INVALID_ARG) for a problem the library rejects."""
+    Ho, Wo = ctypes.c_int(0), ctypes.c_int(0)
+    dt = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    st = load_library().gconv2d_out_shape(N, C_in, H, W, C_out, kH, kW, stride, padding,
+                                          dilation, groups, _layout_code(layout), dt,
+                                          ctypes.byref(Ho), ctypes.byref(Wo))
+    _check(st, "gconv2d_out_shape")
+    return Ho.value, Wo.value
+
+
+def out_steps(B, T, C, K, pad_left, pad_right, dtype):
+    """T_out of a depthwise conv1d problem (dwconv1d_out_steps); raises GconvError for a
+    problem the library rejects."""
+    T_out = ctypes.c_int(0)
+    dt = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    st = load_library().dwconv1d_out_steps(B, T, C, K, pad_left, pad_right, dt,
+                                           ctypes.byref(T_out))
+    _check(st, "dwconv1d_out_steps")
+    return T_out.value
 
 
 def conv2d_dims(x, w, stride, padding, dilation, groups, layout):
@@ -171,8 +194,8 @@ def conv2d_dims(x, w, stride, padding, dilation, groups, layout):
     if cpg_in * groups != C_in:
         raise ValueError(f"weight has {cpg_in} input channels per group; x has {C_in} channels "
                          f"in {groups} groups")
-    Ho = _out_extent(H, kH, stride, padding, dilation)
-    Wo = _out_extent(W, kW, stride, padding, dilation)
+    Ho, Wo = out_shape(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, lay,
+                       _dtype_code(x.dtype))
     y_shape = (N, C_out, Ho, Wo) if lay == NCHW else (N, Ho, Wo, C_out)
     return lay, (N, C_in, H, W, C_out, kH, kW), y_shape
 
@@ -230,8 +253,8 @@ def _bwd_dims(dy, w, in_hw, stride, padding, dilation, groups, layout):
     if C_out2 != C_out:
         raise ValueError(f"w has {C_out2} filters; dy has {C_out} channels")
     C_in = cpg_in * groups
-    Ho = _out_extent(H, kH, stride, padding, dilation)
-    Wo = _out_extent(W, kW, stride, padding, dilation)
+    Ho, Wo = out_shape(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, lay,
+                       _dtype_code(dy.dtype))
     want = (N, C_out, Ho, Wo) if lay == NCHW else (N, Ho, Wo, C_out)
     if tuple(dy.shape) != want:
         raise ValueError(f"dy has shape {tuple(dy.shape)}, expected {want}")
@@ -349,7 +372,7 @@ def dwconv1d_fwd(x, w, pad_left, pad_right, out=None, stream=None, path=PATH_AUT
     _need(x, "x")
     _need(w, "w", x.dtype)
     B, T, C, K = _conv1d_dims(x, w)
-    T_out = T + pad_left + pad_right - K + 1
+    T_out = out_steps(B, T, C, K, pad_left, pad_right, _dtype_code(x.dtype))
     y = torch.empty((B, T_out, C), dtype=x.dtype, device=x.device) if out is None else out
     _need(y, "out", x.dtype)
     st = lib.dwconv1d_fwd_path(_ptr(x), _ptr(w), _ptr(y), B, T, C, K, pad_left, pad_right,
@@ -364,7 +387,7 @@ def dwconv1d_bwd_data(dy, w, T, pad_left, pad_right, out=None, stream=None, path
     _need(w, "w", dy.dtype)
     B, T_out, C = dy.shape
     K = w.shape[1]
-    if T_out != T + pad_left + pad_right - K + 1:
+    if T_out != out_steps(B, T, C, K, pad_left, pad_right, _dtype_code(dy.dtype)):
         raise ValueError("dy has the wrong number of steps for T, K and the pads")
     dx = torch.empty((B, T, C), dtype=dy.dtype, device=dy.device) if out is None else out
     _need(dx, "out", dy.dtype)

@@ -245,6 +245,29 @@ using namespace gconv;
 
 extern "C" {
 
+gconv_status gconv2d_out_shape(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                               int stride, int pad, int dilation, int groups,
+                               gconv_layout layout, gconv_dtype dtype, int* Ho, int* Wo) {
+  if (Ho == nullptr || Wo == nullptr) return GCONV_ERR_INVALID_ARG;
+  Conv2d p;
+  const gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation,
+                                      groups, layout, dtype);
+  if (st != GCONV_OK) return st;
+  *Ho = p.Ho;
+  *Wo = p.Wo;
+  return GCONV_OK;
+}
+
+gconv_status dwconv1d_out_steps(int B, int T, int C, int K, int pad_left, int pad_right,
+                                gconv_dtype dtype, int* T_out) {
+  if (T_out == nullptr) return GCONV_ERR_INVALID_ARG;
+  Conv1d p;
+  const gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
+  if (st != GCONV_OK) return st;
+  *T_out = p.T_out;
+  return GCONV_OK;
+}
+
 size_t gconv2d_fwd_workspace_size(int N, int C_in, int H, int W, int C_out, int kH, int kW,
                                   int stride, int pad, int dilation, int groups,
                                   gconv_layout layout, gconv_dtype dtype, gconv_path path) {

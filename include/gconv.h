@@ -123,6 +123,16 @@ typedef enum {
                                          dy transposed to NHWC in the workspace first */
 } gconv_kernel;
 
+/* Output extent of a gconv2d problem: validates the arguments exactly as gconv2d_fwd does and
+ * writes *Ho, *Wo by F.conv2d's rule (Ho = floor((H + 2*pad - dilation*(kH-1) - 1) / stride)
+ * + 1, same for Wo; the output-size rule of the timing script in "F.conv2d runs x15 slower in
+ * mixed-precision/half-precision mode"). y is [N][C_out][Ho][Wo] (NCHW) or [N][Ho][Wo][C_out]
+ * (NHWC); dy of the backward calls has the same shape. Host-only, launches nothing.
+ * Errors: INVALID_ARG (also for NULL Ho / Wo, or Ho / Wo < 1); *Ho, *Wo untouched then. */
+gconv_status gconv2d_out_shape(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                               int stride, int pad, int dilation, int groups,
+                               gconv_layout layout, gconv_dtype dtype, int* Ho, int* Wo);
+
 /* Bytes of workspace gconv2d_fwd needs for this problem under `path` (0 if none; also 0 for
  * invalid arguments, which gconv2d_fwd then rejects). */
 size_t gconv2d_fwd_workspace_size(int N, int C_in, int H, int W, int C_out, int kH, int kW,
@@ -234,6 +244,12 @@ gconv_status gconv2d_bwd_weight_path(const void* x, const void* dy, void* dw, in
 int gconv2d_bwd_weight_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW,
                                    int stride, int pad, int dilation, int groups,
                                    gconv_layout layout, gconv_dtype dtype, gconv_path path);
+
+/* Output steps of a depthwise conv1d problem: validates the arguments as dwconv1d_fwd does
+ * and writes *T_out = T + pad_left + pad_right - K + 1 (the steps of y and dy; x and dx have
+ * T). Host-only. Errors: INVALID_ARG (also for NULL T_out, or T_out < 1). */
+gconv_status dwconv1d_out_steps(int B, int T, int C, int K, int pad_left, int pad_right,
+                                gconv_dtype dtype, int* T_out);
 
 /* Depthwise conv1d forward: x [B][T][C], w [C][K] -> y [B][T_out][C].
  * Errors: INVALID_ARG (incl. T_out < 1), CUDA. */

@@ -244,3 +244,60 @@ def test_bwd_workspace_queries(lib):
     n = lib.gconv2d_bwd_weight_workspace_size(*nchw)
     staged = 2 * (512 * 256 * 256 * 2)
     assert n > staged and (n - staged) % (4 * 512 * 128 * 9) == 0
+
+
+def _enumerated_extent(size, k, stride, pad, dil):
+    """Output positions counted one by one: o is an output when its whole window
+    o*stride - pad + [0, dil*(k-1)] lies inside the zero-padded input [-pad, size + pad)."""
+    n = 0
+    while n * stride - pad + dil * (k - 1) <= size - 1 + pad:
+        n += 1
+    return n
+
+
+def test_out_shape_query_matches_oracle_and_enumeration(lib):
+    """gconv2d_out_shape / dwconv1d_out_steps (the binding allocates y and checks dy with
+    them) agree with the oracle's output size and with counting window positions."""
+    import oracle
+    Ho, Wo = ctypes.c_int(-7), ctypes.c_int(-7)
+    for size in (1, 2, 5, 7, 16, 57):
+        for k in (1, 2, 3, 5):
+            for s in (1, 2, 3):
+                for p in (0, 1, 2):
+                    for d in (1, 2):
+                        want = _enumerated_extent(size, k, s, p, d)
+                        assert oracle.out_extent(size, k, s, p, d) == want
+                        st = lib.gconv2d_out_shape(2, 4, size, size + 1, 8, k, k, s, p, d, 2, 1, 2,
+                                                   ctypes.byref(Ho), ctypes.byref(Wo))
+                        if want < 1:
+                            assert st == 1
+                            continue
+                        assert st == 0
+                        assert Ho.value == want
+                        assert Wo.value == _enumerated_extent(size + 1, k, s, p, d)
+    # argument errors reach the query too
+    assert lib.gconv2d_out_shape(1, 6, 8, 8, 8, 3, 3, 1, 1, 1, 4, 1, 2, ctypes.byref(Ho),
+                                 ctypes.byref(Wo)) == 1          # 6 channels in 4 groups
+    assert lib.gconv2d_out_shape(1, 8, 8, 8, 8, 3, 3, 1, 1, 1, 4, 1, 2, None, None) == 1
+    T_out = ctypes.c_int(0)
+    for T, K, pl, pr in ((2048, 31, 15, 15), (2048, 31, 30, 0), (10, 3, 0, 0), (5, 9, 4, 4),
+                         (3, 31, 15, 15)):
+        st = lib.dwconv1d_out_steps(2, T, 8, K, pl, pr, 2, ctypes.byref(T_out))
+        want = T + pl + pr - K + 1
+        if want < 1:
+            assert st == 1
+        else:
+            assert st == 0 and T_out.value == want
+    assert binding.out_shape(1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, "NHWC", 2) == (256, 256)
+    assert binding.out_steps(8, 2048, 512, 31, 30, 0, 2) == 2048
+    with pytest.raises(binding.GconvError):
+        binding.out_shape(1, 8, 2, 2, 8, 5, 5, 1, 0, 1, 1, "NCHW", 2)
+
+
+def test_binding_restates_no_shape_rule():
+    """The binding is argument marshalling: output sizes come from the library's query, so
+    the output-size formula appears nowhere in the package's Python code."""
+    src = open(os.path.join(ROOT, "depthwise_convolution_gconv2d_b200", "binding.py")).read()
+    assert "_out_extent" not in src
+    assert "pad_left + pad_right - K" not in src
+    assert "dilation * (k" not in src
