@@ -109,6 +109,8 @@ def compact_rooflines(dwm, more, bwd, extra=None):
         out[f"{k}_{v['bound']}"] = v["frac"]
         if "ffma_frac" in v:
             out[f"{k}_ffma"] = v["ffma_frac"]
+        if "tensor_frac" in v:
+            out[f"{k}_tensor"] = v["tensor_frac"]
     for k, v in (bwd or {}).items():
         out[f"bwd_{k}_{v['bound']}"] = v["frac"]
     for k, v in (extra or {}).items():
@@ -282,6 +284,30 @@ def conv2d_measurement(torch, gb, device, stream, pk, p, workload, path, reps, f
     return rec
 
 
+def variant_measurement(torch, gb, device, stream, pk, p, workload, mode, reps, flush):
+    """The wide-group layer with its output in another channel order or merged across groups
+    (gconv2d_fwd_out): same FLOPs as the layer; bytes x + w + y, y with C_out / groups channels
+    for the merges."""
+    inp = wl.make_conv2d_inputs(p, workload)
+    x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
+    y = gb.gconv2d_fwd_out(x, w, None, p.stride, p.pad, p.dilation, p.groups, p.layout, mode)
+    kcode = gb.gconv2d_fwd_out_select_path(p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride,
+                                           p.pad, p.dilation, p.groups, p.layout, p.dtype, mode)
+    fn = lambda i: gb.gconv2d_fwd_out(x, w, None, p.stride, p.pad, p.dilation, p.groups,
+                                      p.layout, mode, out=y, stream=stream)
+    for _ in range(2):
+        fn(0)
+    med, mean = time_launches(torch, fn, stream, reps, flush)
+    nbytes = (x.numel() + w.numel() + y.numel()) * 2
+    t_tensor = p.flops() / (pk["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    bound, t_roof = ("tensor", t_tensor) if t_tensor >= t_hbm else ("hbm", t_hbm)
+    return {"kernel": kernel_name(kcode), "us": round(med * 1e3, 2),
+            "TFLOP/s": round(p.flops() / (med * 1e-3) / 1e12, 1),
+            "GB/s": round(nbytes / (med * 1e-3) / 1e9, 1), "bound": bound,
+            "frac": round(t_roof / (med * 1e-3), 3), "alg_flops": p.flops(), "alg_bytes": nbytes}
+
+
 def more_conv2d_measurements(torch, gb, device, stream, pk, reps):
     """The other conv2d workloads: ensemble-as-groups layer and the groups sweep at C = 1024."""
     flush = l2_flusher(torch, device)
@@ -292,6 +318,13 @@ def more_conv2d_measurements(torch, gb, device, stream, pk, reps):
     out["wide_group_nchw"] = conv2d_measurement(torch, gb, device, stream, pk,
                                                 wl.wide_group(wl.NCHW), 2, gb.PATH_AUTO, reps,
                                                 flush)
+    # grouped linear x[16384, 4096] -> [16384, 4096] in 4 groups (1x1 conv of 1x1 images)
+    out["grouped_linear"] = conv2d_measurement(torch, gb, device, stream, pk,
+                                               wl.grouped_linear(), 6, gb.PATH_AUTO, reps, flush)
+    for mode in ("interleaved", "avg", "max"):
+        out[f"wide_group_{mode}"] = variant_measurement(torch, gb, device, stream, pk,
+                                                        wl.wide_group(wl.NHWC), 2, mode, reps,
+                                                        flush)
     for g in (1024, 256, 64, 16):
         p = wl.depthwise_56(1, g)
         for name, path in (("auto", gb.PATH_AUTO), ("direct", gb.PATH_DIRECT),
@@ -360,6 +393,45 @@ def depthwise_measurements(torch, gb, device, stream, pk, reps):
             out[f"dw1d_{tag}_{op}"] = {"kernel": kname, "us": round(med * 1e3, 2),
                                        "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 3),
                                        "alg_bytes": ab}
+    return out
+
+
+def dwsep_measurements(torch, gb, device, stream, pk, reps):
+    """The depthwise-separable block of the Conformer convolution module: x[8, 2048, 512],
+    depthwise K = 31 'same', then pointwise 512 -> 512 (+ bias), fused in one kernel, and the
+    same block as two launches (depthwise into a workspace, then the pointwise GEMM) for
+    comparison. Algorithmic bytes x + w_dw + w_pw + bias + z; FLOPs 2*B*T*C*(K + C_out);
+    L2 flushed before each launch."""
+    flush = l2_flusher(torch, device)
+    p = wl.conformer_dw1d(False)
+    C_out = 512
+    inp = wl.make_dwsep1d_inputs(p, C_out, 7)
+    x, wdw, wpw, b = (dev_tensor(torch, a, p.dtype, device)
+                      for a in (inp.x, inp.w_dw, inp.w_pw, inp.bias))
+    z = torch.empty((p.B, p.T_out, C_out), dtype=torch.bfloat16, device=device)
+    nbytes = (x.numel() + wdw.numel() + wpw.numel() + b.numel() + z.numel()) * 2
+    flops = 2 * p.B * p.T_out * p.C * (p.K + C_out)
+    out = {}
+    for name, path in (("dwsep1d_fused", gb.PATH_AUTO), ("dwsep1d_two_launches", gb.PATH_DIRECT)):
+        need = gb.load_library().dwsep1d_fwd_workspace_size(p.B, p.T, p.C, p.K, p.pad_left,
+                                                            p.pad_right, C_out, p.dtype, path)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+        kname = gb.KERNEL_NAMES.get(gb.dwsep1d_select_path(p.B, p.T, p.C, p.K, p.pad_left,
+                                                           p.pad_right, C_out, p.dtype, path))
+        fn = lambda i: gb.dwsep1d_fwd(x, wdw, wpw, b, p.pad_left, p.pad_right, out=z,
+                                      workspace=ws, path=path, stream=stream)
+        for _ in range(3):
+            fn(0)
+        med, mean = time_launches(torch, fn, stream, reps, flush)
+        t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+        out[name] = {"kernel": kname, "us": round(med * 1e3, 2),
+                     "TFLOP/s": round(flops / (med * 1e-3) / 1e12, 1),
+                     "GB/s": round(nbytes / (med * 1e-3) / 1e9, 1), "bound": "hbm",
+                     "frac": round(t_hbm / (med * 1e-3), 3),
+                     "tensor_frac": round(2 * p.B * p.T_out * p.C * C_out / (med * 1e-3) /
+                                          (pk["bf16_tflops"] * 1e12), 3),
+                     "alg_bytes": nbytes, "alg_flops": flops}
+        del ws
     return out
 
 
@@ -484,7 +556,8 @@ def config_dict(p, args):
 
 PROFILE_WORKLOADS = ("wide_group_nhwc", "wide_group_nchw", "ensemble_g64", "depthwise56_s1",
                      "depthwise56_s2", "dw1d_same", "sweep56_g64", "sweep56_g16",
-                     "depthwise56_bwd", "depthwise56_s2_bwd", "wide_group_dgrad")
+                     "depthwise56_bwd", "depthwise56_s2_bwd", "wide_group_dgrad",
+                     "wide_group_wgrad", "dwsep1d", "grouped_linear", "wide_group_avg")
 
 
 def run_profile(name: str, reps: int, batch: int = 0) -> int:
@@ -502,6 +575,29 @@ def run_profile(name: str, reps: int, batch: int = 0) -> int:
             gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right)
             gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right)
             gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right)
+    elif name == "dwsep1d":
+        p = wl.conformer_dw1d(False)
+        inp = wl.make_dwsep1d_inputs(p, 512, 7)
+        x, wdw, wpw, b = (dev_tensor(torch, a, p.dtype, device)
+                          for a in (inp.x, inp.w_dw, inp.w_pw, inp.bias))
+        for _ in range(reps):
+            gb.dwsep1d_fwd(x, wdw, wpw, b, p.pad_left, p.pad_right)
+    elif name == "wide_group_wgrad":
+        p = wl.wide_group(wl.NHWC)
+        if batch > 0:
+            p = dataclasses.replace(p, N=batch)
+        inp = wl.make_conv2d_inputs(p, 5)
+        x = dev_tensor(torch, inp.x, p.dtype, device)
+        dy = dev_tensor(torch, wl.make_conv2d_dy(p, 5), p.dtype, device)
+        for _ in range(reps):
+            gb.gconv2d_bwd_weight(x, dy, (p.kH, p.kW), p.stride, p.pad, p.dilation, p.groups,
+                                  p.layout)
+    elif name == "wide_group_avg":
+        p = wl.wide_group(wl.NHWC)
+        inp = wl.make_conv2d_inputs(p, 2)
+        x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
+        for _ in range(reps):
+            gb.gconv2d_fwd_out(x, w, None, p.stride, p.pad, p.dilation, p.groups, p.layout, "avg")
     elif name in ("depthwise56_bwd", "depthwise56_s2_bwd", "wide_group_dgrad"):
         p = {"depthwise56_bwd": lambda: wl.depthwise_56(1),
              "depthwise56_s2_bwd": lambda: wl.depthwise_56(2),
@@ -524,7 +620,8 @@ def run_profile(name: str, reps: int, batch: int = 0) -> int:
              "depthwise56_s1": lambda: wl.depthwise_56(1),
              "depthwise56_s2": lambda: wl.depthwise_56(2),
              "sweep56_g64": lambda: wl.depthwise_56(1, 64),
-             "sweep56_g16": lambda: wl.depthwise_56(1, 16)}[name]()
+             "sweep56_g16": lambda: wl.depthwise_56(1, 16),
+             "grouped_linear": wl.grouped_linear}[name]()
         if batch > 0:
             p = dataclasses.replace(p, N=batch)
         inp = wl.make_conv2d_inputs(p, 2)
@@ -707,6 +804,7 @@ def main():
         dwm = depthwise_measurements(torch, gb, device, stream, pk, 20)
         more = more_conv2d_measurements(torch, gb, device, stream, pk, 10)
         bwd = backward_measurements(torch, gb, device, stream, pk, 10)
+        more.update(dwsep_measurements(torch, gb, device, stream, pk, 20))
     dev_err = gb.device_error(stream)
 
     cpu = None

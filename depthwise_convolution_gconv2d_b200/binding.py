@@ -28,7 +28,9 @@ KERNEL_NAMES = {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "ige
                 5: "conv1d_generic", 6: "conv1d_ring", 7: "conv1d_tc", 8: "grouped_nhwc",
                 9: "dgrad_generic", 10: "wgrad_generic", 11: "wgrad_depthwise_nhwc",
                 12: "dgrad_depthwise_nhwc", 13: "wgrad_tiled_nhwc", 14: "wgrad_dw3_tma",
-                15: "wgrad_tiled_nchw"}
+                15: "wgrad_tiled_nchw", 16: "dwsep1d_fused", 17: "dwsep_unfused",
+                18: "wgrad_tc_nhwc", 19: "wgrad_tc_nchw", 20: "conv1d_strip",
+                21: "dwsep2d_fused"}
 STATUS = {0: "GCONV_OK", 1: "GCONV_ERR_INVALID_ARG", 2: "GCONV_ERR_UNSUPPORTED",
           3: "GCONV_ERR_MISALIGNED", 4: "GCONV_ERR_WORKSPACE", 5: "GCONV_ERR_CUDA",
           6: "GCONV_ERR_DEVICE_TIMEOUT"}
@@ -41,6 +43,10 @@ EXPORTS = ["gconv2d_fwd", "gconv2d_fwd_path", "gconv2d_fwd_workspace_size",
            "dwconv1d_bwd_data_path", "dwconv1d_select_path",
            "dwconv1d_bwd_weight", "dwconv1d_bwd_weight_workspace_size",
            "dwconv1d_bwd_weight_noalloc", "gconv2d_out_shape", "dwconv1d_out_steps",
+           "gconv_debug_set_tx_surplus", "gconv2d_fwd_out", "gconv2d_fwd_out_workspace_size",
+           "gconv2d_fwd_out_select_path", "dwsep1d_fwd", "dwsep1d_fwd_workspace_size",
+           "dwsep1d_select_path", "dwsep2d_fwd", "dwsep2d_fwd_workspace_size",
+           "dwsep2d_select_path",
            "gconv_get_device_error", "gconv_status_string", "gconv_version"]
 
 _lib = None
@@ -106,10 +112,30 @@ def load_library():
     lib.dwconv1d_bwd_weight.restype = I
     lib.dwconv1d_bwd_weight_noalloc.argtypes = [P, P, P] + [I] * 6 + [I, P]
     lib.dwconv1d_bwd_weight_noalloc.restype = I
-    lib.gconv2d_out_shape.argtypes = conv + [I, I, ctypes.POINTER(I), ctypes.POINTER(I)]
+    lib.gconv2d_out_shape.argtypes = conv + [I, I, I] + [ctypes.POINTER(I)] * 3
     lib.gconv2d_out_shape.restype = I
+    lib.gconv2d_fwd_out.argtypes = [P, P, P, P] + conv + [I, I, I, I, P, Z, P]
+    lib.gconv2d_fwd_out.restype = I
+    lib.gconv2d_fwd_out_workspace_size.argtypes = conv + [I, I, I, I]
+    lib.gconv2d_fwd_out_workspace_size.restype = Z
+    lib.gconv2d_fwd_out_select_path.argtypes = conv + [I, I, I, I]
+    lib.gconv2d_fwd_out_select_path.restype = I
     lib.dwconv1d_out_steps.argtypes = [I] * 7 + [ctypes.POINTER(I)]
     lib.dwconv1d_out_steps.restype = I
+    lib.gconv_debug_set_tx_surplus.argtypes = [ctypes.c_uint]
+    lib.gconv_debug_set_tx_surplus.restype = I
+    lib.dwsep1d_fwd_workspace_size.argtypes = [I] * 9
+    lib.dwsep1d_fwd_workspace_size.restype = Z
+    lib.dwsep1d_select_path.argtypes = [I] * 9
+    lib.dwsep1d_select_path.restype = I
+    lib.dwsep1d_fwd.argtypes = [P] * 5 + [I] * 9 + [P, Z, P]
+    lib.dwsep1d_fwd.restype = I
+    lib.dwsep2d_fwd_workspace_size.argtypes = [I] * 13
+    lib.dwsep2d_fwd_workspace_size.restype = Z
+    lib.dwsep2d_select_path.argtypes = [I] * 13
+    lib.dwsep2d_select_path.restype = I
+    lib.dwsep2d_fwd.argtypes = [P] * 5 + [I] * 13 + [P, Z, P]
+    lib.dwsep2d_fwd.restype = I
     lib.gconv_get_device_error.argtypes = [P, ctypes.POINTER(I)]
     lib.gconv_get_device_error.restype = I
     lib.gconv_status_string.argtypes = [I]
@@ -159,17 +185,28 @@ def _need(t, name, dtype=None):
         raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
 
 
+OUT_GROUP_MAJOR, OUT_INTERLEAVED, OUT_MERGE_AVG, OUT_MERGE_MAX = 0, 1, 2, 3
+OUT_MODES = {"group_major": OUT_GROUP_MAJOR, "interleaved": OUT_INTERLEAVED,
+             "avg": OUT_MERGE_AVG, "max": OUT_MERGE_MAX}
+
+
+def _out_mode(mode) -> int:
+    return OUT_MODES[mode] if isinstance(mode, str) else int(mode)
+
+
 def out_shape(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, layout,
-              dtype):
-    """(Ho, Wo) of a conv2d problem from the library's own shape logic (gconv2d_out_shape);
-    raises GconvError(GCONV_ERR_INVALID_ARG) for a problem the library rejects."""
-    Ho, Wo = ctypes.c_int(0), ctypes.c_int(0)
+              dtype, out_mode=OUT_GROUP_MAJOR, channels=False):
+    """(Ho, Wo) -- or (C_y, Ho, Wo) with channels=True -- of a conv2d problem from the
+    library's own shape logic (gconv2d_out_shape); raises GconvError(GCONV_ERR_INVALID_ARG)
+    for a problem the library rejects."""
+    Cy, Ho, Wo = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
     dt = dtype if isinstance(dtype, int) else _dtype_code(dtype)
     st = load_library().gconv2d_out_shape(N, C_in, H, W, C_out, kH, kW, stride, padding,
                                           dilation, groups, _layout_code(layout), dt,
+                                          _out_mode(out_mode), ctypes.byref(Cy),
                                           ctypes.byref(Ho), ctypes.byref(Wo))
     _check(st, "gconv2d_out_shape")
-    return Ho.value, Wo.value
+    return (Cy.value, Ho.value, Wo.value) if channels else (Ho.value, Wo.value)
 
 
 def out_steps(B, T, C, K, pad_left, pad_right, dtype):
@@ -237,6 +274,42 @@ def gconv2d_fwd(x, w, bias=None, stride=1, padding=0, dilation=1, groups=1, layo
                               dilation, groups, lay, dt, path, _ptr(workspace), ws_bytes,
                               _stream(stream))
     _check(st, "gconv2d_fwd")
+    return y
+
+
+def gconv2d_fwd_out_select_path(N, C_in, H, W, C_out, kH, kW, stride, padding, dilation,
+                                groups, layout, dtype, out_mode, path=PATH_AUTO) -> int:
+    return int(load_library().gconv2d_fwd_out_select_path(
+        N, C_in, H, W, C_out, kH, kW, stride, padding, dilation, groups, _layout_code(layout),
+        dtype if isinstance(dtype, int) else _dtype_code(dtype), _out_mode(out_mode), path))
+
+
+def gconv2d_fwd_out(x, w, bias=None, stride=1, padding=0, dilation=1, groups=1, layout="NCHW",
+                    out_mode="interleaved", out=None, workspace=None, path=PATH_AUTO,
+                    stream=None):
+    """Grouped conv2d forward with the output in another channel order or merged across
+    groups (out_mode: 'group_major', 'interleaved', 'avg', 'max'); returns y."""
+    lib = load_library()
+    _need(x, "x")
+    _need(w, "w", x.dtype)
+    if bias is not None:
+        _need(bias, "bias", x.dtype)
+    lay, dims, _ = conv2d_dims(x, w, stride, padding, dilation, groups, layout)
+    dt = _dtype_code(x.dtype)
+    mode = _out_mode(out_mode)
+    Cy, Ho, Wo = out_shape(*dims, stride, padding, dilation, groups, lay, dt, mode, True)
+    y_shape = (dims[0], Cy, Ho, Wo) if lay == NCHW else (dims[0], Ho, Wo, Cy)
+    y = torch.empty(y_shape, dtype=x.dtype, device=x.device) if out is None else out
+    _need(y, "out", x.dtype)
+    if tuple(y.shape) != y_shape:
+        raise ValueError(f"out has shape {tuple(y.shape)}, expected {y_shape}")
+    need = lib.gconv2d_fwd_out_workspace_size(*dims, stride, padding, dilation, groups, lay, dt,
+                                              mode, path)
+    workspace, ws_bytes = _workspace(need, workspace, x.device)
+    st = lib.gconv2d_fwd_out(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), *dims, stride, padding,
+                             dilation, groups, lay, dt, mode, path, _ptr(workspace), ws_bytes,
+                             _stream(stream))
+    _check(st, "gconv2d_fwd_out")
     return y
 
 
@@ -434,6 +507,83 @@ def dwconv1d_bwd_weight_noalloc(x, dy, K, pad_left, pad_right, out=None, stream=
                                          pad_right, _dtype_code(x.dtype), _stream(stream))
     _check(st, "dwconv1d_bwd_weight_noalloc")
     return dw
+
+
+def dwsep1d_select_path(B, T, C, K, pad_left, pad_right, C_out, dtype, path=PATH_AUTO) -> int:
+    """Kernel code (16 fused, 17 two launches) of a dwsep1d_fwd call, or a negative status."""
+    dt = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    return int(load_library().dwsep1d_select_path(B, T, C, K, pad_left, pad_right, C_out, dt,
+                                                   path))
+
+
+def dwsep1d_fwd(x, w_dw, w_pw, bias, pad_left, pad_right, out=None, workspace=None,
+                path=PATH_AUTO, stream=None):
+    """Depthwise-separable block on (batch, steps, channels): x [B, T, C], w_dw [C, K],
+    w_pw [C_out, C], bias [C_out] or None -> z [B, T_out, C_out]."""
+    lib = load_library()
+    _need(x, "x")
+    _need(w_dw, "w_dw", x.dtype)
+    _need(w_pw, "w_pw", x.dtype)
+    if bias is not None:
+        _need(bias, "bias", x.dtype)
+    B, T, C, K = _conv1d_dims(x, w_dw)
+    C_out = w_pw.shape[0]
+    if w_pw.dim() != 2 or w_pw.shape[1] != C:
+        raise ValueError("w_pw must be [C_out, C] with the channel count of x")
+    dt = _dtype_code(x.dtype)
+    T_out = out_steps(B, T, C, K, pad_left, pad_right, dt)
+    z = torch.empty((B, T_out, C_out), dtype=x.dtype, device=x.device) if out is None else out
+    _need(z, "out", x.dtype)
+    if tuple(z.shape) != (B, T_out, C_out):
+        raise ValueError(f"out has shape {tuple(z.shape)}, expected {(B, T_out, C_out)}")
+    need = lib.dwsep1d_fwd_workspace_size(B, T, C, K, pad_left, pad_right, C_out, dt, path)
+    workspace, ws_bytes = _workspace(need, workspace, x.device)
+    st = lib.dwsep1d_fwd(_ptr(x), _ptr(w_dw), _ptr(w_pw), _ptr(bias), _ptr(z), B, T, C, K,
+                         pad_left, pad_right, C_out, dt, path, _ptr(workspace), ws_bytes,
+                         _stream(stream))
+    _check(st, "dwsep1d_fwd")
+    return z
+
+
+def dwsep2d_select_path(N, C, H, W, kH, kW, stride, padding, dilation, C_out, layout, dtype,
+                        path=PATH_AUTO) -> int:
+    """Kernel code (21 fused, 17 two launches) of a dwsep2d_fwd call, or a negative status."""
+    dt = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    return int(load_library().dwsep2d_select_path(N, C, H, W, kH, kW, stride, padding, dilation,
+                                                   C_out, _layout_code(layout), dt, path))
+
+
+def dwsep2d_fwd(x, w_dw, w_pw, bias=None, stride=1, padding=0, dilation=1, layout="NHWC",
+                out=None, workspace=None, path=PATH_AUTO, stream=None):
+    """2-D depthwise-separable block: x (NCHW or NHWC, C channels), w_dw the depthwise weight
+    of that layout, w_pw [C_out, C], bias [C_out] or None -> z (C_out channels)."""
+    lib = load_library()
+    _need(x, "x")
+    _need(w_dw, "w_dw", x.dtype)
+    _need(w_pw, "w_pw", x.dtype)
+    if bias is not None:
+        _need(bias, "bias", x.dtype)
+    lay, dims, y_shape = conv2d_dims(x, w_dw, stride, padding, dilation, x.shape[1 if
+                                     _layout_code(layout) == NCHW else 3], layout)
+    N, C, H, W, C2, kH, kW = dims
+    C_out = w_pw.shape[0]
+    if C2 != C or w_pw.dim() != 2 or w_pw.shape[1] != C:
+        raise ValueError("w_dw must be the depthwise weight of x and w_pw [C_out, C]")
+    dt = _dtype_code(x.dtype)
+    z_shape = (N, C_out, y_shape[2], y_shape[3]) if lay == NCHW else (N, y_shape[1],
+                                                                        y_shape[2], C_out)
+    z = torch.empty(z_shape, dtype=x.dtype, device=x.device) if out is None else out
+    _need(z, "out", x.dtype)
+    if tuple(z.shape) != z_shape:
+        raise ValueError(f"out has shape {tuple(z.shape)}, expected {z_shape}")
+    need = lib.dwsep2d_fwd_workspace_size(N, C, H, W, kH, kW, stride, padding, dilation, C_out,
+                                          lay, dt, path)
+    workspace, ws_bytes = _workspace(need, workspace, x.device)
+    st = lib.dwsep2d_fwd(_ptr(x), _ptr(w_dw), _ptr(w_pw), _ptr(bias), _ptr(z), N, C, H, W, kH,
+                         kW, stride, padding, dilation, C_out, lay, dt, path, _ptr(workspace),
+                         ws_bytes, _stream(stream))
+    _check(st, "dwsep2d_fwd")
+    return z
 
 
 def device_error(stream=None) -> int:

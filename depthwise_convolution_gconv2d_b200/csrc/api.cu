@@ -27,6 +27,12 @@ unsigned int* device_error_word() {
   return (unsigned int*)addr;
 }
 
+// Test hook: bytes the generic tensor-core tile kernel's producer declares per stage on top of
+// what its copies deliver (0 on every normal run).
+static std::atomic<unsigned int> g_tx_surplus{0};
+
+unsigned int debug_tx_surplus() { return g_tx_surplus.load(std::memory_order_relaxed); }
+
 cudaError_t read_and_clear_device_error(cudaStream_t s, int* code) {
   cudaError_t e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return e;
@@ -50,7 +56,10 @@ long long out_extent(long long in, long long k, long long stride, long long pad,
 
 // Fills `p`; returns GCONV_OK or GCONV_ERR_INVALID_ARG.
 gconv_status make_conv2d(Conv2d* p, int N, int C_in, int H, int W, int C_out, int kH, int kW,
-                         int stride, int pad, int dil, int groups, int layout, int dtype) {
+                         int stride, int pad, int dil, int groups, int layout, int dtype,
+                         int out_mode = GCONV_OUT_GROUP_MAJOR) {
+  if (out_mode < GCONV_OUT_GROUP_MAJOR || out_mode > GCONV_OUT_MERGE_MAX)
+    return GCONV_ERR_INVALID_ARG;
   if (N < 0 || C_in <= 0 || H <= 0 || W <= 0 || C_out <= 0 || kH <= 0 || kW <= 0)
     return GCONV_ERR_INVALID_ARG;
   if (stride <= 0 || pad < 0 || dil <= 0 || groups <= 0) return GCONV_ERR_INVALID_ARG;
@@ -69,6 +78,7 @@ gconv_status make_conv2d(Conv2d* p, int N, int C_in, int H, int W, int C_out, in
   p->Ho = (int)Ho; p->Wo = (int)Wo;
   p->cpg_in = C_in / groups; p->cpg_out = C_out / groups;
   p->layout = layout; p->dtype = dtype;
+  p->out_mode = out_mode;
   return GCONV_OK;
 }
 
@@ -108,6 +118,45 @@ int choose_kernel(const Conv2d& p, int path, const void* x, const void* w, const
       if (dw_ok && dw_al) return GCONV_KERNEL_DEPTHWISE_NHWC;
       if (ng_ok) return GCONV_KERNEL_GROUPED_NHWC;
       if (tc_ok && tc_al) return tc_kernel;
+      return GCONV_KERNEL_DIRECT_GENERIC;
+    default:
+      *why = GCONV_ERR_INVALID_ARG;
+      return -1;
+  }
+}
+
+// Output variants. The interleaved order equals the group-major one when each group has one
+// filter or there is one group, and a merge over one group is the plain output: those run on
+// the ordinary kernels. Otherwise the variant runs in the epilogue of the tensor-core tile
+// kernels (16-bit data the implicit GEMM takes) or in the generic direct kernel.
+bool out_mode_is_plain(const Conv2d& p) {
+  if (p.out_mode == GCONV_OUT_GROUP_MAJOR || p.groups == 1) return true;
+  return p.out_mode == GCONV_OUT_INTERLEAVED && p.cpg_out == 1;
+}
+
+int choose_kernel_out(const Conv2d& p, int path, const void* x, const void* w, const void* y,
+                      gconv_status* why) {
+  if (out_mode_is_plain(p)) {
+    Conv2d q = p;
+    q.out_mode = GCONV_OUT_GROUP_MAJOR;
+    return choose_kernel(q, path, x, w, y, why);
+  }
+  *why = GCONV_OK;
+  const bool query = (x == nullptr && w == nullptr && y == nullptr);
+  const bool tc_ok = igemm_supported(p);
+  const bool tc_al = query || (aligned16(x) && aligned16(y) &&
+                               (p.layout == GCONV_NCHW || aligned16(w)));
+  const int tc_kernel = p.layout == GCONV_NHWC ? GCONV_KERNEL_IGEMM_TC : GCONV_KERNEL_IGEMM_TC_NCHW;
+  switch (path) {
+    case GCONV_PATH_GENERIC:
+    case GCONV_PATH_DIRECT:
+      return GCONV_KERNEL_DIRECT_GENERIC;
+    case GCONV_PATH_IGEMM:
+      if (!tc_ok) { *why = GCONV_ERR_UNSUPPORTED; return -1; }
+      if (!tc_al) { *why = GCONV_ERR_MISALIGNED; return -1; }
+      return tc_kernel;
+    case GCONV_PATH_AUTO:
+      if (p.dtype != GCONV_F32 && tc_ok && tc_al) return tc_kernel;
       return GCONV_KERNEL_DIRECT_GENERIC;
     default:
       *why = GCONV_ERR_INVALID_ARG;
@@ -206,17 +255,33 @@ int wgrad_choose(const Conv2d& p, int path, const void* x, const void* dy, gconv
   const int tl_kernel = p.layout == GCONV_NHWC ? GCONV_KERNEL_WGRAD_TILED_NHWC
                                                : GCONV_KERNEL_WGRAD_TILED_NCHW;
   const bool tma_ok = wgrad_dw3_tma_supported(p) && (query || (aligned16(x) && aligned16(dy)));
+  // tensor cores: NHWC operands read by TMA in place (16-byte aligned), NCHW staged as NHWC
+  const bool tc_ok = wgrad_tc_supported(p) && wgrad_tiled_supported(p) &&
+                     (p.layout == GCONV_NCHW || query || (aligned16(x) && aligned16(dy)));
+  const int tc_kernel = p.layout == GCONV_NHWC ? GCONV_KERNEL_WGRAD_TC_NHWC
+                                               : GCONV_KERNEL_WGRAD_TC_NCHW;
   switch (path) {
     case GCONV_PATH_GENERIC:
       return GCONV_KERNEL_WGRAD_GENERIC;
     case GCONV_PATH_AUTO:
+      if (tma_ok) return GCONV_KERNEL_WGRAD_DW3_TMA;
+      if (dw_ok) return GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC;
+      if (tc_ok) return tc_kernel;
+      return tl_ok ? tl_kernel : GCONV_KERNEL_WGRAD_GENERIC;
     case GCONV_PATH_DIRECT:
       if (tma_ok) return GCONV_KERNEL_WGRAD_DW3_TMA;
       if (dw_ok) return GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC;
       return tl_ok ? tl_kernel : GCONV_KERNEL_WGRAD_GENERIC;
     case GCONV_PATH_IGEMM:
-      *why = GCONV_ERR_UNSUPPORTED;   // no tensor-core weight gradient
-      return -1;
+      if (!wgrad_tc_supported(p) || !wgrad_tiled_supported(p)) {
+        *why = GCONV_ERR_UNSUPPORTED;
+        return -1;
+      }
+      if (!tc_ok) {
+        *why = GCONV_ERR_MISALIGNED;
+        return -1;
+      }
+      return tc_kernel;
     default:
       *why = GCONV_ERR_INVALID_ARG;
       return -1;
@@ -238,6 +303,82 @@ gconv_status make_conv1d(Conv1d* p, int B, int T, int C, int K, int pl, int pr, 
   return GCONV_OK;
 }
 
+// ------------------------------------------------------------------ depthwise-separable block
+size_t elem_bytes(int dtype) { return dtype == GCONV_F32 ? 4 : 2; }
+
+// Kernel for a dwsep1d_fwd call: the fused kernel, or the two-kernel composition (depthwise
+// into the workspace, then the pointwise GEMM). x / wdw / wpw / z null = query mode.
+int dwsep1d_choose(const Conv1d& p, int C_out, int path, const void* x, const void* wdw,
+                   const void* wpw, const void* z, gconv_status* why) {
+  *why = GCONV_OK;
+  const bool query = x == nullptr && wdw == nullptr && wpw == nullptr && z == nullptr;
+  const bool fused_ok = dwsep1d_fused_supported(p, C_out);
+  const bool fused_al = query || (aligned16(x) && aligned16(wdw) && aligned16(wpw) &&
+                                  aligned16(z));
+  switch (path) {
+    case GCONV_PATH_AUTO:
+      return fused_ok && fused_al ? GCONV_KERNEL_DWSEP1D_FUSED : GCONV_KERNEL_DWSEP_UNFUSED;
+    case GCONV_PATH_IGEMM:
+      if (!fused_ok) { *why = GCONV_ERR_UNSUPPORTED; return -1; }
+      if (!fused_al) { *why = GCONV_ERR_MISALIGNED; return -1; }
+      return GCONV_KERNEL_DWSEP1D_FUSED;
+    case GCONV_PATH_DIRECT:
+    case GCONV_PATH_GENERIC:
+      return GCONV_KERNEL_DWSEP_UNFUSED;
+    default:
+      *why = GCONV_ERR_INVALID_ARG;
+      return -1;
+  }
+}
+
+// The 2-D block: `p` is its depthwise problem (groups = C_in = C_out = C).
+int dwsep2d_choose(const Conv2d& p, int C_out, int path, const void* x, const void* wdw,
+                   const void* wpw, const void* z, gconv_status* why) {
+  *why = GCONV_OK;
+  const bool query = x == nullptr && wdw == nullptr && wpw == nullptr && z == nullptr;
+  const bool fused_ok = dwsep2d_fused_supported(p, C_out);
+  const bool fused_al = query || (aligned16(x) && aligned16(wdw) && aligned16(wpw) &&
+                                  aligned16(z));
+  switch (path) {
+    case GCONV_PATH_AUTO:
+      return fused_ok && fused_al ? GCONV_KERNEL_DWSEP2D_FUSED : GCONV_KERNEL_DWSEP_UNFUSED;
+    case GCONV_PATH_IGEMM:
+      if (!fused_ok) { *why = GCONV_ERR_UNSUPPORTED; return -1; }
+      if (!fused_al) { *why = GCONV_ERR_MISALIGNED; return -1; }
+      return GCONV_KERNEL_DWSEP2D_FUSED;
+    case GCONV_PATH_DIRECT:
+    case GCONV_PATH_GENERIC:
+      return GCONV_KERNEL_DWSEP_UNFUSED;
+    default:
+      *why = GCONV_ERR_INVALID_ARG;
+      return -1;
+  }
+}
+
+// Composition workspace of the 2-D block: the depthwise output, then the depthwise call's and
+// the pointwise call's own workspaces (NCHW tensor-core staging).
+struct Dwsep2dWs {
+  size_t d_bytes, dw_ws, pw_ws, total;
+};
+
+Dwsep2dWs dwsep2d_ws(const Conv2d& p, const Conv2d& q, int path) {
+  Dwsep2dWs w{};
+  w.d_bytes = round_up((size_t)p.N * p.C_out * p.Ho * p.Wo * elem_bytes(p.dtype), 256);
+  gconv_status why;
+  const int part = path == GCONV_PATH_GENERIC ? GCONV_PATH_GENERIC : GCONV_PATH_AUTO;
+  const int k1 = choose_kernel(p, part, nullptr, nullptr, nullptr, &why);
+  const int k2 = choose_kernel(q, part, nullptr, nullptr, nullptr, &why);
+  w.dw_ws = k1 == GCONV_KERNEL_IGEMM_TC_NCHW ? round_up(igemm_nchw_workspace(p), 256) : 0;
+  w.pw_ws = k2 == GCONV_KERNEL_IGEMM_TC_NCHW ? round_up(igemm_nchw_workspace(q), 256) : 0;
+  w.total = w.d_bytes + (w.dw_ws > w.pw_ws ? w.dw_ws : w.pw_ws);
+  return w;
+}
+
+size_t dwsep1d_workspace(const Conv1d& p, int kernel) {
+  if (kernel != GCONV_KERNEL_DWSEP_UNFUSED) return 0;
+  return round_up((size_t)p.B * p.T_out * p.C * elem_bytes(p.dtype), 256);
+}
+
 }  // namespace
 }  // namespace gconv
 
@@ -247,15 +388,60 @@ extern "C" {
 
 gconv_status gconv2d_out_shape(int N, int C_in, int H, int W, int C_out, int kH, int kW,
                                int stride, int pad, int dilation, int groups,
-                               gconv_layout layout, gconv_dtype dtype, int* Ho, int* Wo) {
-  if (Ho == nullptr || Wo == nullptr) return GCONV_ERR_INVALID_ARG;
+                               gconv_layout layout, gconv_dtype dtype, gconv_out_mode out_mode,
+                               int* C_y, int* Ho, int* Wo) {
+  if (C_y == nullptr || Ho == nullptr || Wo == nullptr) return GCONV_ERR_INVALID_ARG;
   Conv2d p;
   const gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation,
-                                      groups, layout, dtype);
+                                      groups, layout, dtype, out_mode);
   if (st != GCONV_OK) return st;
+  *C_y = out_channels(p);
   *Ho = p.Ho;
   *Wo = p.Wo;
   return GCONV_OK;
+}
+
+size_t gconv2d_fwd_out_workspace_size(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                      int stride, int pad, int dilation, int groups,
+                                      gconv_layout layout, gconv_dtype dtype,
+                                      gconv_out_mode out_mode, gconv_path path) {
+  Conv2d p;
+  if (make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups, layout,
+                  dtype, out_mode) != GCONV_OK)
+    return 0;
+  gconv_status why;
+  const int k = choose_kernel_out(p, path, nullptr, nullptr, nullptr, &why);
+  return k == GCONV_KERNEL_IGEMM_TC_NCHW ? igemm_nchw_workspace(p) : 0;
+}
+
+int gconv2d_fwd_out_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                int stride, int pad, int dilation, int groups,
+                                gconv_layout layout, gconv_dtype dtype, gconv_out_mode out_mode,
+                                gconv_path path) {
+  Conv2d p;
+  gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups,
+                                layout, dtype, out_mode);
+  if (st != GCONV_OK) return -(int)st;
+  const int k = choose_kernel_out(p, path, nullptr, nullptr, nullptr, &st);
+  return k < 0 ? -(int)st : k;
+}
+
+gconv_status gconv2d_fwd_out(const void* x, const void* w, const void* bias, void* y, int N,
+                             int C_in, int H, int W, int C_out, int kH, int kW, int stride,
+                             int pad, int dilation, int groups, gconv_layout layout,
+                             gconv_dtype dtype, gconv_out_mode out_mode, gconv_path path,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  Conv2d p;
+  gconv_status st = make_conv2d(&p, N, C_in, H, W, C_out, kH, kW, stride, pad, dilation, groups,
+                                layout, dtype, out_mode);
+  if (st != GCONV_OK) return st;
+  if (N > 0 && (x == nullptr || w == nullptr || y == nullptr)) return GCONV_ERR_INVALID_ARG;
+  const int kernel = choose_kernel_out(p, path, x, w, y, &st);
+  if (kernel < 0) return st;
+  if (N == 0) return GCONV_OK;
+  if (out_mode_is_plain(p)) p.out_mode = GCONV_OUT_GROUP_MAJOR;
+  return launch_forward(kernel, p, x, w, bias, y, workspace, workspace_bytes,
+                        (cudaStream_t)stream);
 }
 
 gconv_status dwconv1d_out_steps(int B, int T, int C, int K, int pad_left, int pad_right,
@@ -514,6 +700,137 @@ gconv_status dwconv1d_bwd_weight_noalloc(const void* x, const void* dy, void* dw
   if (dw == nullptr || (B > 0 && (x == nullptr || dy == nullptr))) return GCONV_ERR_INVALID_ARG;
   if (dwconv1d_wgrad_workspace(p) > dwconv1d_wgrad_noalloc_limit()) return GCONV_ERR_WORKSPACE;
   return cuda_status(launch_dwconv1d_wgrad_noalloc(p, x, dy, dw, (cudaStream_t)stream));
+}
+
+size_t dwsep1d_fwd_workspace_size(int B, int T, int C, int K, int pad_left, int pad_right,
+                                  int C_out, gconv_dtype dtype, gconv_path path) {
+  Conv1d p;
+  if (C_out <= 0 || make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype) != GCONV_OK) return 0;
+  gconv_status why;
+  const int k = dwsep1d_choose(p, C_out, path, nullptr, nullptr, nullptr, nullptr, &why);
+  return k < 0 ? 0 : dwsep1d_workspace(p, k);
+}
+
+int dwsep1d_select_path(int B, int T, int C, int K, int pad_left, int pad_right, int C_out,
+                        gconv_dtype dtype, gconv_path path) {
+  Conv1d p;
+  if (C_out <= 0) return -(int)GCONV_ERR_INVALID_ARG;
+  gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
+  if (st != GCONV_OK) return -(int)st;
+  const int k = dwsep1d_choose(p, C_out, path, nullptr, nullptr, nullptr, nullptr, &st);
+  return k < 0 ? -(int)st : k;
+}
+
+gconv_status dwsep1d_fwd(const void* x, const void* w_dw, const void* w_pw, const void* bias,
+                         void* z, int B, int T, int C, int K, int pad_left, int pad_right,
+                         int C_out, gconv_dtype dtype, gconv_path path, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  Conv1d p;
+  if (C_out <= 0) return GCONV_ERR_INVALID_ARG;
+  gconv_status st = make_conv1d(&p, B, T, C, K, pad_left, pad_right, dtype);
+  if (st != GCONV_OK) return st;
+  if ((long long)B * p.T_out * C_out > (1LL << 40)) return GCONV_ERR_INVALID_ARG;
+  if (B > 0 && (x == nullptr || w_dw == nullptr || w_pw == nullptr || z == nullptr))
+    return GCONV_ERR_INVALID_ARG;
+  const int kernel = B > 0 ? dwsep1d_choose(p, C_out, path, x, w_dw, w_pw, z, &st)
+                           : dwsep1d_choose(p, C_out, path, nullptr, nullptr, nullptr, nullptr,
+                                            &st);
+  if (kernel < 0) return st;
+  const size_t need = dwsep1d_workspace(p, kernel);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return GCONV_ERR_WORKSPACE;
+  if (B == 0) return GCONV_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (kernel == GCONV_KERNEL_DWSEP1D_FUSED)
+    return cuda_status(launch_dwsep1d_fused(p, C_out, x, w_dw, w_pw, bias, z, s));
+  // composition: the depthwise output d [B][T_out][C] in the workspace, then z = the pointwise
+  // convolution of d as B images of 1 x T_out pixels (NHWC), weights [C_out][1][1][C]
+  const int part = path == GCONV_PATH_GENERIC ? GCONV_PATH_GENERIC : GCONV_PATH_AUTO;
+  st = dwconv1d_fwd_path(x, w_dw, workspace, B, T, C, K, pad_left, pad_right, dtype,
+                         (gconv_path)part, stream);
+  if (st != GCONV_OK) return st;
+  Conv2d q;
+  st = make_conv2d(&q, B, C, 1, p.T_out, C_out, 1, 1, 1, 0, 1, 1, GCONV_NHWC, dtype);
+  if (st != GCONV_OK) return st;
+  const int k2 = choose_kernel(q, part, workspace, w_pw, z, &st);
+  if (k2 < 0) return st;
+  if (k2 == GCONV_KERNEL_IGEMM_TC_NCHW) return GCONV_ERR_UNSUPPORTED;   // NHWC only here
+  return launch_forward(k2, q, workspace, w_pw, bias, z, nullptr, 0, s);
+}
+
+namespace {
+// Depthwise problem p and pointwise problem q of a 2-D block.
+gconv_status make_dwsep2d(Conv2d* p, Conv2d* q, int N, int C, int H, int W, int kH, int kW,
+                          int stride, int pad, int dilation, int C_out, int layout, int dtype) {
+  if (C_out <= 0) return GCONV_ERR_INVALID_ARG;
+  gconv_status st = make_conv2d(p, N, C, H, W, C, kH, kW, stride, pad, dilation, C, layout,
+                                dtype);
+  if (st != GCONV_OK) return st;
+  return make_conv2d(q, N, C, p->Ho, p->Wo, C_out, 1, 1, 1, 0, 1, 1, layout, dtype);
+}
+}  // namespace
+
+size_t dwsep2d_fwd_workspace_size(int N, int C, int H, int W, int kH, int kW, int stride,
+                                  int pad, int dilation, int C_out, gconv_layout layout,
+                                  gconv_dtype dtype, gconv_path path) {
+  Conv2d p, q;
+  if (make_dwsep2d(&p, &q, N, C, H, W, kH, kW, stride, pad, dilation, C_out, layout, dtype) !=
+      GCONV_OK)
+    return 0;
+  gconv_status why;
+  const int k = dwsep2d_choose(p, C_out, path, nullptr, nullptr, nullptr, nullptr, &why);
+  return k == GCONV_KERNEL_DWSEP_UNFUSED ? dwsep2d_ws(p, q, path).total : 0;
+}
+
+int dwsep2d_select_path(int N, int C, int H, int W, int kH, int kW, int stride, int pad,
+                        int dilation, int C_out, gconv_layout layout, gconv_dtype dtype,
+                        gconv_path path) {
+  Conv2d p, q;
+  gconv_status st =
+      make_dwsep2d(&p, &q, N, C, H, W, kH, kW, stride, pad, dilation, C_out, layout, dtype);
+  if (st != GCONV_OK) return -(int)st;
+  const int k = dwsep2d_choose(p, C_out, path, nullptr, nullptr, nullptr, nullptr, &st);
+  return k < 0 ? -(int)st : k;
+}
+
+gconv_status dwsep2d_fwd(const void* x, const void* w_dw, const void* w_pw, const void* bias,
+                         void* z, int N, int C, int H, int W, int kH, int kW, int stride,
+                         int pad, int dilation, int C_out, gconv_layout layout,
+                         gconv_dtype dtype, gconv_path path, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  Conv2d p, q;
+  gconv_status st =
+      make_dwsep2d(&p, &q, N, C, H, W, kH, kW, stride, pad, dilation, C_out, layout, dtype);
+  if (st != GCONV_OK) return st;
+  if (N > 0 && (x == nullptr || w_dw == nullptr || w_pw == nullptr || z == nullptr))
+    return GCONV_ERR_INVALID_ARG;
+  const int kernel = N > 0 ? dwsep2d_choose(p, C_out, path, x, w_dw, w_pw, z, &st)
+                           : dwsep2d_choose(p, C_out, path, nullptr, nullptr, nullptr, nullptr,
+                                            &st);
+  if (kernel < 0) return st;
+  const Dwsep2dWs ws = dwsep2d_ws(p, q, path);
+  if (kernel == GCONV_KERNEL_DWSEP_UNFUSED &&
+      (workspace == nullptr || workspace_bytes < ws.total || !aligned16(workspace)))
+    return GCONV_ERR_WORKSPACE;
+  if (N == 0) return GCONV_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (kernel == GCONV_KERNEL_DWSEP2D_FUSED)
+    return cuda_status(launch_dwsep2d_fused(p, C_out, x, w_dw, w_pw, bias, z, s));
+  const int part = path == GCONV_PATH_GENERIC ? GCONV_PATH_GENERIC : GCONV_PATH_AUTO;
+  void* d = workspace;
+  void* rest = (char*)workspace + ws.d_bytes;
+  const size_t rest_bytes = workspace_bytes - ws.d_bytes;
+  st = gconv2d_fwd_path(x, w_dw, nullptr, d, N, C, H, W, C, kH, kW, stride, pad, dilation, C,
+                        layout, dtype, (gconv_path)part, rest, rest_bytes, stream);
+  if (st != GCONV_OK) return st;
+  return gconv2d_fwd_path(d, w_pw, bias, z, N, C, p.Ho, p.Wo, C_out, 1, 1, 1, 0, 1, 1, layout,
+                          dtype, (gconv_path)part, rest, rest_bytes, stream);
+}
+
+gconv_status gconv_debug_set_tx_surplus(unsigned int bytes) {
+  if (bytes % 16u != 0 || bytes > (1u << 16)) return GCONV_ERR_INVALID_ARG;
+  g_tx_surplus.store(bytes, std::memory_order_relaxed);
+  return GCONV_OK;
 }
 
 gconv_status gconv_get_device_error(void* stream, int* code) {

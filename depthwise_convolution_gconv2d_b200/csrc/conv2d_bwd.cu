@@ -330,9 +330,10 @@ __global__ void __launch_bounds__(DWW_THREADS, 2)
         }
       }
       // copies in flight land before the ring is reused below (instant on the normal path)
+      const unsigned long long dl = drain_deadline();
       for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
-        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr,
-                  0u);
+        mbar_wait_until(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), dl, err,
+                        ERR_DRAIN);
     }
   } else {
     constexpr int NIN = (DWW_R - 1) * S + 3;     // input columns a thread reads per row
@@ -868,13 +869,16 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
                                                                      E, P.slices, 9, 1, 3);
       return cudaGetLastError();
     }
-    if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC || kernel == GCONV_KERNEL_WGRAD_TILED_NCHW) {
+    const bool tc = kernel == GCONV_KERNEL_WGRAD_TC_NHWC || kernel == GCONV_KERNEL_WGRAD_TC_NCHW;
+    const bool to_nchw = kernel == GCONV_KERNEL_WGRAD_TILED_NCHW ||
+                         kernel == GCONV_KERNEL_WGRAD_TC_NCHW;
+    if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC || kernel == GCONV_KERNEL_WGRAD_TILED_NCHW || tc) {
       Conv2d q = p;
       q.layout = GCONV_NHWC;
       const T* xt = (const T*)x;
       const T* dt = (const T*)dy;
       float* part = (float*)ws;
-      if (kernel == GCONV_KERNEL_WGRAD_TILED_NCHW) {
+      if (to_nchw) {
         // stage x and dy as NHWC at the front of the workspace, partials after them
         const size_t xb = staged_bytes((long long)p.N * p.C_in * p.H * p.W);
         const size_t db = staged_bytes((long long)p.N * p.C_out * p.Ho * p.Wo);
@@ -887,15 +891,22 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
         xt = xs;
         dt = ds;
       }
-      int n_mt, n_nt, S, per;
-      tiled_tiles(q, &n_mt, &n_nt);
-      const long long tiles = tiled_count(q);
-      tiled_slices(q, tiles, &S, &per);
-      wgrad_tiled_nhwc_kernel<T><<<dim3((unsigned)tiles, (unsigned)S), 256, 0, s>>>(
-          xt, dt, part, q, n_mt, n_nt, E, per);
-      cudaError_t e = cudaGetLastError();
+      int S;
+      cudaError_t e;
+      if (tc) {
+        S = wgrad_tc_slices(q);
+        e = launch_wgrad_tc(q, xt, dt, part, s);
+      } else {
+        int n_mt, n_nt, per;
+        tiled_tiles(q, &n_mt, &n_nt);
+        const long long tiles = tiled_count(q);
+        tiled_slices(q, tiles, &S, &per);
+        wgrad_tiled_nhwc_kernel<T><<<dim3((unsigned)tiles, (unsigned)S), 256, 0, s>>>(
+            xt, dt, part, q, n_mt, n_nt, E, per);
+        e = cudaGetLastError();
+      }
       if (e != cudaSuccess) return e;
-      if (kernel == GCONV_KERNEL_WGRAD_TILED_NCHW)
+      if (to_nchw)
         wgrad_sum_kernel<T, SUM_TO_NCHW><<<sum_grid(E), 256, 0, s>>>(
             part, (T*)dw, E, S, p.kH * p.kW, p.cpg_in, p.kW);
       else
@@ -1006,11 +1017,15 @@ size_t wgrad_workspace(const Conv2d& p, int kernel) {
   if ((long long)p.N * p.Ho == 0) return 0;
   if (kernel == GCONV_KERNEL_WGRAD_DW3_TMA)
     return (size_t)dww_params(p).slices * 9 * (size_t)p.C_in * sizeof(float);
-  if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC || kernel == GCONV_KERNEL_WGRAD_TILED_NCHW) {
+  if (kernel == GCONV_KERNEL_WGRAD_TILED_NHWC || kernel == GCONV_KERNEL_WGRAD_TILED_NCHW ||
+      kernel == GCONV_KERNEL_WGRAD_TC_NHWC || kernel == GCONV_KERNEL_WGRAD_TC_NCHW) {
     int S, per;
-    tiled_slices(p, tiled_count(p), &S, &per);
+    if (kernel == GCONV_KERNEL_WGRAD_TC_NHWC || kernel == GCONV_KERNEL_WGRAD_TC_NCHW)
+      S = wgrad_tc_slices(p);
+    else
+      tiled_slices(p, tiled_count(p), &S, &per);
     size_t b = (size_t)S * (size_t)p.C_out * p.cpg_in * p.kH * p.kW * sizeof(float);
-    if (kernel == GCONV_KERNEL_WGRAD_TILED_NCHW)
+    if (kernel == GCONV_KERNEL_WGRAD_TILED_NCHW || kernel == GCONV_KERNEL_WGRAD_TC_NCHW)
       b += staged_bytes((long long)p.N * p.C_in * p.H * p.W) +
            staged_bytes((long long)p.N * p.C_out * p.Ho * p.Wo);
     return b;

@@ -240,9 +240,10 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
         }
       }
       // copies in flight must land before the CTA exits (instant on the normal path)
+      const unsigned long long dl = drain_deadline();
       for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
-        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr,
-                  0u);
+        mbar_wait_until(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), dl, err,
+                        ERR_DRAIN);
     }
   } else {
     constexpr int NIN = (DW3_R - 1) * S + 3;        // input columns a thread reads per row

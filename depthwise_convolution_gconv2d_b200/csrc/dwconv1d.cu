@@ -120,9 +120,10 @@ __global__ void __maxnreg__(128)
           ph ^= 1u;
         }
       }
+      const unsigned long long dl = drain_deadline();
       for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
-        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr,
-                  0u);
+        mbar_wait_until(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), dl, err,
+                        ERR_DRAIN);
     }
   } else {
     const int cp = lane, strip = warp - 1;
@@ -246,9 +247,10 @@ __global__ void __maxnreg__(128)
           ph ^= 1u;
         }
       }
+      const unsigned long long dl = drain_deadline();
       for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
-        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr,
-                  0u);
+        mbar_wait_until(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), dl, err,
+                        ERR_DRAIN);
     }
   } else {
     const int cp = lane, strip = warp - 1;
@@ -540,18 +542,21 @@ int conv1d_choose_kernel(const Conv1d& p, int path, const void* x, const void* w
   const bool ring_al = query || (aligned16(x) && aligned16(y));
   const bool tc_ok = conv1d_tc_supported(p);
   const bool tc_al = query || (aligned16(x) && aligned16(y) && aligned16(w));
+  const bool strip_ok = conv1d_strip_supported(p) && (query || (aligned16(x) && aligned16(y)));
   switch (path) {
     case GCONV_PATH_GENERIC:
       return GCONV_KERNEL_CONV1D_GENERIC;
     case GCONV_PATH_DIRECT:
+      if (strip_ok) return GCONV_KERNEL_CONV1D_STRIP;
       return (ring_ok && ring_al) ? GCONV_KERNEL_CONV1D_RING : GCONV_KERNEL_CONV1D_GENERIC;
     case GCONV_PATH_IGEMM:
       if (!tc_ok) { *why = GCONV_ERR_UNSUPPORTED; return -1; }
       if (!tc_al) { *why = GCONV_ERR_MISALIGNED; return -1; }
       return GCONV_KERNEL_CONV1D_TC;
     case GCONV_PATH_AUTO:
-      // the tensor-core kernel is the faster of the two (Conformer layer: 22.5 vs 30.6 us);
-      // the CUDA-core ring kernel takes C % 16 == 8 and the generic kernel the rest
+      // 128-byte-row CUDA-core kernel where it applies (64-channel blocks), else the
+      // tensor-core kernel, the 16-byte-vector ring kernel, the generic kernel
+      if (strip_ok) return GCONV_KERNEL_CONV1D_STRIP;
       if (tc_ok && tc_al) return GCONV_KERNEL_CONV1D_TC;
       if (ring_ok && ring_al) return GCONV_KERNEL_CONV1D_RING;
       return GCONV_KERNEL_CONV1D_GENERIC;
@@ -566,6 +571,8 @@ cudaError_t launch_dwconv1d_fwd(const Conv1d& p, const void* x, const void* w, v
   if (p.B == 0) return cudaSuccess;
   if (kernel == GCONV_KERNEL_CONV1D_TC)
     return launch_dwconv1d_tc(p, x, w, y, flip, pad_left, T_in, T_out, s);
+  if (kernel == GCONV_KERNEL_CONV1D_STRIP)
+    return launch_dwconv1d_strip(p, x, w, y, flip, pad_left, T_in, T_out, s);
   const bool vec = kernel == GCONV_KERNEL_CONV1D_RING;
   switch (p.dtype) {
     case GCONV_F32: return fwd_any_dtype<float>(p, x, w, y, flip, pad_left, T_in, T_out, false, s);
@@ -574,15 +581,26 @@ cudaError_t launch_dwconv1d_fwd(const Conv1d& p, const void* x, const void* w, v
   }
 }
 
+// The 128-byte-row weight gradient where it applies (its partials: one fp32 value per
+// channel, tap and run of tiles), else the ring kernel's slices.
+bool wgrad_strip_ok(const Conv1d& p) { return conv1d_strip_supported(p); }
+
 size_t dwconv1d_wgrad_workspace(const Conv1d& p) {
-  if (!conv1d_vector_supported(p) || p.B == 0) return 0;
+  if (p.B == 0) return 0;
+  // the strip kernel's size, or the ring kernel's, whichever the call's pointers select: the
+  // larger of the two when both apply
+  const size_t strip = wgrad_strip_ok(p) ? dwconv1d_wgrad_strip_workspace(p) : 0;
+  if (!conv1d_vector_supported(p)) return strip;
   int slice_len, n_tslices;
   wgrad_slicing(p, &slice_len, &n_tslices);
-  return (size_t)p.B * n_tslices * p.C * p.K * sizeof(float);
+  const size_t ring = (size_t)p.B * n_tslices * p.C * p.K * sizeof(float);
+  return ring > strip ? ring : strip;
 }
 
 cudaError_t launch_dwconv1d_wgrad(const Conv1d& p, const void* x, const void* dy, void* dw,
                                   void* workspace, cudaStream_t s) {
+  if (p.B > 0 && wgrad_strip_ok(p) && aligned16(x) && aligned16(dy) && workspace != nullptr)
+    return launch_dwconv1d_wgrad_strip(p, x, dy, dw, workspace, s);
   const bool vec = conv1d_vector_supported(p) && aligned16(x) && aligned16(dy) &&
                    workspace != nullptr && p.B > 0;
   switch (p.dtype) {

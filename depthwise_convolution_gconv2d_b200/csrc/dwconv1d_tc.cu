@@ -193,7 +193,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         r0 + L.box_h * i, c.b);
       }
       // copies in flight must land before the CTA exits
-      if (n > 0) mbar_wait(xs_full, (unsigned int)(n - 1) & 1u, abort_flag, nullptr, 0u);
+      if (n > 0)
+        mbar_wait_until(xs_full, (unsigned int)(n - 1) & 1u, drain_deadline(), err, ERR_DRAIN);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -222,8 +223,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       // the last chain must finish before TMEM is released (already true on the normal path)
       if (u > 0)
-        mbar_wait(&tm_full[(u - 1) % TC_ASTAGES], (unsigned int)((u - 1) / TC_ASTAGES) & 1u,
-                  abort_flag, nullptr, 0u);
+        mbar_wait_until(&tm_full[(u - 1) % TC_ASTAGES], (unsigned int)((u - 1) / TC_ASTAGES) & 1u,
+                        drain_deadline(), err, ERR_DRAIN);
     }
   } else if (warp >= 6) {
     // ------------------------------------------------------------ transposes + filter copies

@@ -116,9 +116,10 @@ __global__ void __launch_bounds__(NG_THREADS, 2)
         }
       }
       // copies in flight must land before the CTA exits
+      const unsigned long long dl = drain_deadline();
       for (int q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
-        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, nullptr,
-                  0u);
+        mbar_wait_until(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), dl, err,
+                        ERR_DRAIN);
     }
   } else {
     // ------------------------------------------------------------ compute warps

@@ -55,6 +55,9 @@ struct IgemmParams {
   unsigned int sbo;            // bytes between 8-row core-matrix groups
   unsigned int tmem_cols;
   int out_nchw;
+  // output variants: out_mode (gconv_out_mode), channels of y, groups merged per tile (1 unless
+  // the groups are merged: then a tile covers every group, one accumulator per group)
+  int groups, out_mode, out_c, nsub;
 };
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading / stride byte offsets
@@ -101,6 +104,41 @@ __device__ __forceinline__ void epilogue_store(const PP& P, T* __restrict__ y,
 #pragma unroll
     for (int i = 0; i < 32; ++i)
       if (i < ncols) dst[i * plane] = Elem<T>::from_f32(v[i]);
+  }
+}
+
+// Stores `ncols` fp32 values (bias already added) of one output pixel: value i goes to channel
+// ch0 + i * chs of y's out_c channels -- chs = 1 for the group-major order and for merged
+// groups (16-byte NHWC vectors), chs = groups for the interleaved order (scalar stores).
+template <typename T>
+__device__ __forceinline__ void epilogue_store_mapped(const IgemmParams& P, T* __restrict__ y,
+                                                      const float* v, int ncols, int n, int ho,
+                                                      int wo, int ch0, int chs) {
+  if (!P.out_nchw) {
+    T* dst = y + (((long long)n * P.Ho + ho) * P.Wo + wo) * P.out_c + ch0;
+    if (chs == 1) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q * 8 < ncols) {
+          uint4 u;
+          u.x = pack2<T>(make_float2(v[8 * q + 0], v[8 * q + 1]));
+          u.y = pack2<T>(make_float2(v[8 * q + 2], v[8 * q + 3]));
+          u.z = pack2<T>(make_float2(v[8 * q + 4], v[8 * q + 5]));
+          u.w = pack2<T>(make_float2(v[8 * q + 6], v[8 * q + 7]));
+          *reinterpret_cast<uint4*>(dst + 8 * q) = u;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < ncols) dst[(long long)i * chs] = Elem<T>::from_f32(v[i]);
+    }
+  } else {
+    const long long plane = (long long)P.Ho * P.Wo;
+    T* dst = y + ((long long)n * P.out_c + ch0) * plane + (long long)ho * P.Wo + wo;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < ncols) dst[(long long)i * chs * plane] = Elem<T>::from_f32(v[i]);
   }
 }
 
@@ -157,35 +195,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
         const int mt = t % P.m_tiles, rest = t / P.m_tiles;
-        const int nt = rest % P.n_tiles, j = rest / P.n_tiles;
+        const int nt = rest % P.n_tiles, jt = rest / P.n_tiles;
         const int tw = mt % P.tiles_w, r2 = mt / P.tiles_w;
         const int th = r2 % P.tiles_h, n = r2 / P.tiles_h;
         const int hbase = th * P.BH - P.pad, wbase = tw * P.BW - P.pad;
-        const int cbase = j * P.cpg_in, obase = j * P.cpg_out + nt * P.BN;
-        for (int kb = 0; kb < P.kblocks; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
-            ok = false;
-            break;
-          }
-          const int tap = kb / P.cblocks, cb = kb - tap * P.cblocks;
-          const int kh = tap / P.kW, kw = tap - kh * P.kW;
-          mbar_arrive_expect_tx(&full[s], P.tx_bytes);
-          tma_load_4d(a_base + (size_t)s * P.a_stage, &tma_x, &full[s], cbase + cb * P.BKC,
-                      wbase + kw * P.dil, hbase + kh * P.dil, n);
-          tma_load_2d(b_base + (size_t)s * P.b_stage, &tma_w, &full[s],
-                      tap * P.cpg_in + cb * P.BKC, obase);
-          ++issued;
-          if (++s == P.stages) {
-            s = 0;
-            ph ^= 1u;
+        for (int sub = 0; sub < P.nsub && ok; ++sub) {
+          const int j = P.nsub > 1 ? sub : jt;
+          const int cbase = j * P.cpg_in, obase = j * P.cpg_out + nt * P.BN;
+          for (int kb = 0; kb < P.kblocks; ++kb) {
+            if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
+              ok = false;
+              break;
+            }
+            const int tap = kb / P.cblocks, cb = kb - tap * P.cblocks;
+            const int kh = tap / P.kW, kw = tap - kh * P.kW;
+            mbar_arrive_expect_tx(&full[s], P.tx_bytes);
+            tma_load_4d(a_base + (size_t)s * P.a_stage, &tma_x, &full[s], cbase + cb * P.BKC,
+                        wbase + kw * P.dil, hbase + kh * P.dil, n);
+            tma_load_2d(b_base + (size_t)s * P.b_stage, &tma_w, &full[s],
+                        tap * P.cpg_in + cb * P.BKC, obase);
+            ++issued;
+            if (++s == P.stages) {
+              s = 0;
+              ph ^= 1u;
+            }
           }
         }
       }
       // copies in flight must land before the CTA can exit (no-op on the normal path)
       const long long first = issued > P.stages ? issued - P.stages : 0;
+      const unsigned long long dl = drain_deadline();
       for (long long i = first; i < issued; ++i)
-        mbar_wait(&full[i % P.stages], (unsigned int)((i / P.stages) & 1), abort_flag, err,
-                  ERR_WAIT_DRAIN);
+        mbar_wait_until(&full[i % P.stages], (unsigned int)((i / P.stages) & 1), dl, err,
+                        ERR_WAIT_DRAIN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -199,7 +241,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // instruction chain short enough for back-to-back MMAs
       const unsigned long long a_desc0 = smem_desc(smem_u32(a_base), P.sbo, P.swz);
       const unsigned long long b_desc0 = smem_desc(smem_u32(b_base), P.sbo, P.swz);
-      for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
+      const int subs = (P.num_tiles > (int)blockIdx.x
+                            ? (P.num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0) *
+                       P.nsub;
+      for (int u = 0; u < subs && ok; ++u) {
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERR_WAIT_MMA)) break;
         tc_fence_after();
         const unsigned int d_tmem = tmem_base + (unsigned int)(acc * P.BN);
@@ -230,7 +275,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // every issued MMA must complete before TMEM is released
       umma_commit(done);
-      mbar_wait(done, 0, abort_flag, err, ERR_WAIT_DRAIN);
+      mbar_wait_until(done, 0, drain_deadline(), err, ERR_WAIT_DRAIN);
     }
   } else {
     // ---------------- epilogue: warps 2..5, TMEM lane quarter (warp % 4)
@@ -239,34 +284,91 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int hl = row / P.BW, wl = row - hl * P.BW;
     int acc = 0;
     unsigned int aph = 0;
-    for (int t = blockIdx.x; t < P.num_tiles; t += gridDim.x) {
+    const bool merge = P.nsub > 1;
+    const bool interleave = P.out_mode == GCONV_OUT_INTERLEAVED;
+    bool ok = true;
+    for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
       const int mt = t % P.m_tiles, rest = t / P.m_tiles;
-      const int nt = rest % P.n_tiles, j = rest / P.n_tiles;
+      const int nt = rest % P.n_tiles, jt = rest / P.n_tiles;
       const int tw = mt % P.tiles_w, r2 = mt / P.tiles_w;
       const int th = r2 % P.tiles_h, n = r2 / P.tiles_h;
-      const bool got = mbar_wait(&tfull[acc], aph, abort_flag, err, ERR_WAIT_EPILOGUE);
-      if (!__all_sync(0xffffffffu, got)) break;    // warp-uniform: tcgen05.ld is .aligned
-      tc_fence_after();
       const int ho = th * P.BH + hl, wo = tw * P.BW + wl;
       const bool valid = hl < P.BH && ho < P.Ho && wo < P.Wo;
-      const int co0 = j * P.cpg_out + nt * P.BN;
-      const unsigned int taddr =
-          tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.BN);
-      for (int c = 0; c < P.BN; c += 32) {
-        unsigned int r[32];
-        const int ncols = P.BN - c < 32 ? P.BN - c : 32;
-        if (ncols == 32)
-          tmem_ld32(taddr + c, r);
-        else
-          tmem_ld16(taddr + c, r);
-        tmem_ld_wait();
-        if (valid) epilogue_store<T>(P, y, bias, r, ncols, n, ho, wo, co0 + c);
+      float run[64];   // merged groups: running sum / maximum over the tile's sub-tiles
+      for (int sub = 0; sub < P.nsub; ++sub) {
+        const bool got = mbar_wait(&tfull[acc], aph, abort_flag, err, ERR_WAIT_EPILOGUE);
+        if (!__all_sync(0xffffffffu, got)) {     // warp-uniform: tcgen05.ld is .aligned
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int j = merge ? sub : jt;
+        const int co0 = j * P.cpg_out + nt * P.BN;
+        const unsigned int taddr =
+            tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.BN);
+        if (!merge) {
+          for (int c = 0; c < P.BN; c += 32) {
+            unsigned int r[32];
+            const int ncols = P.BN - c < 32 ? P.BN - c : 32;
+            if (ncols == 32)
+              tmem_ld32(taddr + c, r);
+            else
+              tmem_ld16(taddr + c, r);
+            tmem_ld_wait();
+            if (!valid) continue;
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              v[i] = __uint_as_float(r[i]) +
+                     (bias && i < ncols ? Elem<T>::to_f32(bias[co0 + c + i]) : 0.0f);
+            if (interleave)
+              epilogue_store_mapped<T>(P, y, v, ncols, n, ho, wo,
+                                       (nt * P.BN + c) * P.groups + j, P.groups);
+            else
+              epilogue_store_mapped<T>(P, y, v, ncols, n, ho, wo, co0 + c, 1);
+          }
+        } else {
+          // BN <= 64: both 32-column halves unrolled so that `run` stays in registers
+#pragma unroll
+          for (int c = 0; c < 64; c += 32) {
+            if (c < P.BN) {
+              unsigned int r[32];
+              const int ncols = P.BN - c < 32 ? P.BN - c : 32;
+              if (ncols == 32)
+                tmem_ld32(taddr + c, r);
+              else
+                tmem_ld16(taddr + c, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float v = __uint_as_float(r[i]) +
+                                (bias && i < ncols ? Elem<T>::to_f32(bias[co0 + c + i]) : 0.0f);
+                run[c + i] = sub == 0 ? v
+                             : (P.out_mode == GCONV_OUT_MERGE_MAX ? fmaxf(run[c + i], v)
+                                                                  : run[c + i] + v);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          aph ^= 1u;
+        }
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        aph ^= 1u;
+      if (ok && merge && valid) {
+        const float scale = P.out_mode == GCONV_OUT_MERGE_AVG ? 1.0f / (float)P.groups : 1.0f;
+#pragma unroll
+        for (int c = 0; c < 64; c += 32) {
+          if (c < P.BN) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = run[c + i] * scale;
+            epilogue_store_mapped<T>(P, y, v, P.BN - c < 32 ? P.BN - c : 32, n, ho, wo,
+                                     nt * P.BN + c, 1);
+          }
+        }
       }
     }
   }
@@ -477,9 +579,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      const unsigned long long dl = drain_deadline();
       for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
-        mbar_wait(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), abort_flag, err,
-                  ERR_WAIT_DRAIN);
+        mbar_wait_until(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), dl, err,
+                        ERR_WAIT_DRAIN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -545,7 +648,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       umma_commit(done);
-      mbar_wait(done, 0, abort_flag, err, ERR_WAIT_DRAIN);
+      mbar_wait_until(done, 0, drain_deadline(), err, ERR_WAIT_DRAIN);
     }
   } else {
     // ---------------- epilogue: warps 2..5, TMEM lane quarter (warp % 4)
@@ -768,12 +871,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       // copies in flight must land before the CTA exits (no-op on the normal path)
+      const unsigned long long dl = drain_deadline();
       for (long long q = (na > P.a_stages ? na - P.a_stages : 0); q < na; ++q)
-        mbar_wait(&fa[q % P.a_stages], (unsigned int)((q / P.a_stages) & 1), abort_flag, err,
-                  ERR_WAIT_DRAIN);
+        mbar_wait_until(&fa[q % P.a_stages], (unsigned int)((q / P.a_stages) & 1), dl, err,
+                        ERR_WAIT_DRAIN);
       for (long long q = (nb > P.b_stages ? nb - P.b_stages : 0); q < nb; ++q)
-        mbar_wait(&fb[q % P.b_stages], (unsigned int)((q / P.b_stages) & 1), abort_flag, err,
-                  ERR_WAIT_DRAIN);
+        mbar_wait_until(&fb[q % P.b_stages], (unsigned int)((q / P.b_stages) & 1), dl, err,
+                        ERR_WAIT_DRAIN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -840,7 +944,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       umma_commit(done);
-      mbar_wait(done, 0, abort_flag, err, ERR_WAIT_DRAIN);
+      mbar_wait_until(done, 0, drain_deadline(), err, ERR_WAIT_DRAIN);
     }
   } else {
     // ---------------- epilogue: warps 2..5, TMEM lane quarter (warp % 4)
@@ -908,6 +1012,7 @@ struct RowTParams {
   unsigned int x_stage, w_stage, x_tx, w_tx, box1_bytes;
   unsigned int idesc, tmem_cols;
   int out_nchw, nchw_vec;
+  int groups, interleave;   // interleaved output order: filter f of group j -> f * groups + j
 };
 
 __device__ __forceinline__ void rowt_decode(const RowTParams& P, int t, int& j, int& nt, int& n,
@@ -1020,12 +1125,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      const unsigned long long dl = drain_deadline();
       for (long long q = (nx > P.x_stages ? nx - P.x_stages : 0); q < nx; ++q)
-        mbar_wait(&fx[q % P.x_stages], (unsigned int)((q / P.x_stages) & 1), abort_flag, err,
-                  ERR_WAIT_DRAIN);
+        mbar_wait_until(&fx[q % P.x_stages], (unsigned int)((q / P.x_stages) & 1), dl, err,
+                        ERR_WAIT_DRAIN);
       for (long long q = (nw > P.w_stages ? nw - P.w_stages : 0); q < nw; ++q)
-        mbar_wait(&fw[q % P.w_stages], (unsigned int)((q / P.w_stages) & 1), abort_flag, err,
-                  ERR_WAIT_DRAIN);
+        mbar_wait_until(&fw[q % P.w_stages], (unsigned int)((q / P.w_stages) & 1), dl, err,
+                        ERR_WAIT_DRAIN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -1083,7 +1189,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       umma_commit(done);
-      mbar_wait(done, 0, abort_flag, err, ERR_WAIT_DRAIN);
+      mbar_wait_until(done, 0, drain_deadline(), err, ERR_WAIT_DRAIN);
     }
   } else {
     // ---------------- epilogue: warps 2..5; TMEM lane = output channel of the tile
@@ -1097,8 +1203,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool got = mbar_wait(&tfull[acc], aph, abort_flag, err, ERR_WAIT_EPILOGUE);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const int co = j * P.cpg_out + nt * BM + co_l;
-      const float bv = bias ? Elem<T>::to_f32(bias[co]) : 0.0f;
+      const int co_g = j * P.cpg_out + nt * BM + co_l;       // group-major channel
+      const int co = P.interleave ? (nt * BM + co_l) * P.groups + j : co_g;   // y's channel
+      const float bv = bias ? Elem<T>::to_f32(bias[co_g]) : 0.0f;
       const unsigned int taddr =
           tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.NPIX);
       for (int c = 0; c < P.NPIX; c += 32) {
@@ -1257,7 +1364,16 @@ bool make_params(const Conv2d& p, IgemmParams* P) {
   P->BW = p.Wo < BM ? p.Wo : BM;
   P->BH = BM / P->BW;
   if (P->BH > p.Ho) P->BH = p.Ho;
-  P->BN = tile_bn(p);
+  P->groups = p.groups;
+  P->out_mode = p.out_mode;
+  P->out_c = out_channels(p);
+  const bool merge = p.out_mode == GCONV_OUT_MERGE_AVG || p.out_mode == GCONV_OUT_MERGE_MAX;
+  P->nsub = merge ? p.groups : 1;
+  // merged groups keep a running value per accumulator column in the epilogue's registers,
+  // so their tiles are at most 64 filters wide
+  P->BN = !merge ? tile_bn(p)
+                 : (p.cpg_out <= 64 ? p.cpg_out
+                                    : (p.cpg_out % 64 == 0 ? 64 : (p.cpg_out % 32 == 0 ? 32 : 16)));
   P->BKC = p.cpg_in % 64 == 0 ? 64 : (p.cpg_in % 32 == 0 ? 32 : 16);
   P->cblocks = p.cpg_in / P->BKC;
   P->kblocks = p.kH * p.kW * P->cblocks;
@@ -1265,7 +1381,7 @@ bool make_params(const Conv2d& p, IgemmParams* P) {
   P->tiles_h = (p.Ho + P->BH - 1) / P->BH;
   const long long m_tiles = (long long)p.N * P->tiles_w * P->tiles_h;
   P->n_tiles = p.cpg_out / P->BN;
-  const long long tiles = m_tiles * P->n_tiles * p.groups;
+  const long long tiles = m_tiles * P->n_tiles * (merge ? 1 : p.groups);
   if (m_tiles > INT32_MAX || tiles > INT32_MAX) return false;
   P->m_tiles = (int)m_tiles;
   P->num_tiles = (int)tiles;
@@ -1302,6 +1418,7 @@ CUtensorMapSwizzle swizzle_of(int BKC) {
 // Row-strip kernel parameters; false if the problem does not take that kernel (rows shorter
 // than 128 outputs, channel blocks narrower than 64, or the stage rings do not fit).
 bool make_row_params(const Conv2d& p, RowParams* R) {
+  if (p.out_mode != GCONV_OUT_GROUP_MAJOR) return false;
   if (p.Wo < BM || p.cpg_in % 64 != 0) return false;
   const int BN = tile_bn(p);
   if (BN == 0) return false;
@@ -1410,6 +1527,7 @@ cudaError_t launch_row(const Conv2d& p, const RowParams& R, const void* x, const
 
 // Transposed row kernel parameters; false if the problem does not take it.
 bool make_rowt_params(const Conv2d& p, RowTParams* R) {
+  if (p.out_mode != GCONV_OUT_GROUP_MAJOR && p.out_mode != GCONV_OUT_INTERLEAVED) return false;
   if (p.Wo < BM || p.cpg_in % 64 != 0 || p.cpg_out % BM != 0) return false;
   if ((p.kW - 1) * p.dil > 8) return false;            // halo fits the 8-row second box
   R->N = p.N; R->H = p.H; R->W = p.W; R->C_in = p.C_in; R->C_out = p.C_out;
@@ -1444,6 +1562,8 @@ bool make_rowt_params(const Conv2d& p, RowTParams* R) {
   if (R->tmem_cols > 512) return false;
   R->out_nchw = p.layout == GCONV_NCHW;
   R->nchw_vec = (p.Wo % 8 == 0) ? 1 : 0;
+  R->groups = p.groups;
+  R->interleave = p.out_mode == GCONV_OUT_INTERLEAVED;
   return true;
 }
 
@@ -1498,6 +1618,7 @@ cudaError_t launch_rowt(const Conv2d& p, const RowTParams& R, const void* x, con
 // Halo tile kernel parameters; false if the problem does not take it (rows wider than 128,
 // a width that is not a multiple of 8, or stages that do not fit).
 bool make_halo_params(const Conv2d& p, HaloParams* H) {
+  if (p.out_mode != GCONV_OUT_GROUP_MAJOR) return false;
   if (p.Wo > BM || p.Wo % 8 != 0) return false;
   // groups packed per tile: 64 / cpg_in of them when that divides the group count and keeps
   // N = gp * cpg_out within 64. The block-diagonal filter tile makes each MMA as wide as the
@@ -1650,10 +1771,40 @@ cudaError_t launch_halo(const Conv2d& p, const HaloParams& H, const void* x, con
   return cudaGetLastError();
 }
 
+// A 1x1, stride-1, unpadded convolution is one GEMM over all pixels. With NHWC pixels (or one
+// NCHW image, whose output plane is the same pixel sequence) it is run as an image of
+// H' x W' = N*H*W pixels, W' as wide as the kernels take, so that tiles run across image
+// rows and images: grouped linear layers (H = W = 1, the per-group GEMMs of a batched-GEMM
+// formulation) then fill whole 128 / 256-pixel MMA tiles instead of one pixel each.
+// False if the problem is not pointwise, is already one row, or has no such factorisation.
+bool flatten_pointwise(const Conv2d& p, Conv2d* q) {
+  if (p.kH != 1 || p.kW != 1 || p.stride != 1 || p.pad != 0) return false;
+  if (p.layout == GCONV_NCHW && p.N != 1) return false;
+  if (p.N == 1 && p.H == 1) return false;
+  const long long M = (long long)p.N * p.H * p.W;
+  long long Wq = 0;
+  if (M <= 65535) {
+    Wq = M;
+  } else {
+    for (long long c = 65535; c >= 128; --c)
+      if (M % c == 0 && M / c <= 65535) {
+        Wq = c;
+        break;
+      }
+  }
+  if (Wq == 0) return false;
+  *q = p;
+  q->N = 1;
+  q->H = q->Ho = (int)(M / Wq);
+  q->W = q->Wo = (int)Wq;
+  q->dil = 1;
+  return true;
+}
+
 // x: NHWC activations, w: [C_out][kH][kW][cpg_in] weights (both device pointers).
 template <typename T>
-cudaError_t launch_core(const Conv2d& p, const IgemmParams& P, const void* x, const void* w,
-                        const void* bias, void* y, cudaStream_t s) {
+cudaError_t launch_tiles(const Conv2d& p, const IgemmParams& P, const void* x, const void* w,
+                         const void* bias, void* y, cudaStream_t s) {
   RowTParams RT;
   if (make_rowt_params(p, &RT)) return launch_rowt<T>(p, RT, x, w, bias, y, s);
   RowParams R;
@@ -1691,9 +1842,21 @@ cudaError_t launch_core(const Conv2d& p, const IgemmParams& P, const void* x, co
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   if (grid > P.num_tiles) grid = P.num_tiles;
-  igemm_tc_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, tw, (const T*)bias, (T*)y, P,
+  IgemmParams PL = P;
+  PL.tx_bytes += debug_tx_surplus();   // 0 except under the bounded-wait test hook
+  igemm_tc_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, tw, (const T*)bias, (T*)y, PL,
                                                      device_error_word());
   return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_core(const Conv2d& p, const IgemmParams& P, const void* x, const void* w,
+                        const void* bias, void* y, cudaStream_t s) {
+  Conv2d q;
+  IgemmParams Q;
+  if (flatten_pointwise(p, &q) && make_params(q, &Q))
+    return launch_tiles<T>(q, Q, x, w, bias, y, s);
+  return launch_tiles<T>(p, P, x, w, bias, y, s);
 }
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -1708,8 +1871,10 @@ bool igemm_supported(const Conv2d& p) {
   if (p.stride != 1) return false;
   if (p.cpg_in % 16 != 0 || p.cpg_out % 16 != 0) return false;
   if (tile_bn(p) == 0) return false;
-  if (p.N > 65535 || p.H > 65535 || p.W > 65535) return false;
   IgemmParams P;
+  Conv2d q;
+  if (flatten_pointwise(p, &q)) return make_params(q, &P);   // the shape that is launched
+  if (p.N > 65535 || p.H > 65535 || p.W > 65535) return false;
   return make_params(p, &P);
 }
 

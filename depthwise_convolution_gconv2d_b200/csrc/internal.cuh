@@ -20,7 +20,14 @@ struct Conv2d {
   int Ho, Wo, cpg_in, cpg_out;
   int layout;  // GCONV_NCHW / GCONV_NHWC
   int dtype;   // GCONV_F32 / GCONV_F16 / GCONV_BF16
+  int out_mode = GCONV_OUT_GROUP_MAJOR;   // gconv_out_mode of the output
 };
+
+// Channels of y: C_out, or C_out / groups when the groups are merged.
+__host__ __device__ __forceinline__ int out_channels(const Conv2d& p) {
+  return (p.out_mode == GCONV_OUT_MERGE_AVG || p.out_mode == GCONV_OUT_MERGE_MAX) ? p.cpg_out
+                                                                                  : p.C_out;
+}
 
 // A validated depthwise conv1d problem on (batch, steps, channels).
 struct Conv1d {
@@ -132,6 +139,12 @@ bool wgrad_dw3_tma_supported(const Conv2d& p);
 // Wide-group NHWC weight gradient (16-bit, C_in/g and C_out/g >= 32 and multiples of 8; x and
 // dy 16-byte aligned).
 bool wgrad_tiled_supported(const Conv2d& p);
+// Wide-group weight gradient on the tensor cores (16-bit, stride 1, C_out/g % 128 == 0,
+// C_in/g % 64 == 0, (kW-1)*dil <= 8, Wo >= 32); NHWC operands, fp32 partials [S][E].
+bool wgrad_tc_supported(const Conv2d& p);
+int wgrad_tc_slices(const Conv2d& p);
+cudaError_t launch_wgrad_tc(const Conv2d& p, const void* x, const void* dy, float* part,
+                            cudaStream_t s);
 size_t wgrad_workspace(const Conv2d& p, int kernel);
 cudaError_t launch_wgrad(const Conv2d& p, const void* x, const void* dy, void* dw, void* ws,
                          int kernel, cudaStream_t s);
@@ -148,12 +161,33 @@ cudaError_t launch_dwconv1d_fwd(const Conv1d& p, const void* x, const void* w, v
 bool conv1d_tc_supported(const Conv1d& p);
 cudaError_t launch_dwconv1d_tc(const Conv1d& p, const void* x, const void* w, void* y, bool flip,
                                int pad_left, int T_in, int T_out, cudaStream_t s);
+// Conv1d with 128-byte input rows on the CUDA cores (16-bit, C % 64 == 0, K in {3, 5, 7, 9,
+// 15, 31}): forward / data gradient, and the weight gradient with its fixed-order partials.
+bool conv1d_strip_supported(const Conv1d& p);
+cudaError_t launch_dwconv1d_strip(const Conv1d& p, const void* x, const void* w, void* y,
+                                  bool flip, int pad_left, int T_in, int T_out, cudaStream_t s);
+size_t dwconv1d_wgrad_strip_workspace(const Conv1d& p);
+cudaError_t launch_dwconv1d_wgrad_strip(const Conv1d& p, const void* x, const void* dy, void* dw,
+                                        void* workspace, cudaStream_t s);
 size_t dwconv1d_wgrad_workspace(const Conv1d& p);
 cudaError_t launch_dwconv1d_wgrad(const Conv1d& p, const void* x, const void* dy, void* dw,
                                   void* workspace, cudaStream_t s);
 size_t dwconv1d_wgrad_noalloc_limit();
 cudaError_t launch_dwconv1d_wgrad_noalloc(const Conv1d& p, const void* x, const void* dy,
                                           void* dw, cudaStream_t s);
+
+// Fused depthwise-separable block (dwconv1d then pointwise 1x1): 16-bit, C % 64 == 0,
+// C_out % 16 == 0 and <= 512, K in {3, 5, 7, 9, 15, 31}; x, w_pw, z 16-byte aligned.
+bool dwsep1d_fused_supported(const Conv1d& p, int C_out);
+cudaError_t launch_dwsep1d_fused(const Conv1d& p, int C_out, const void* x, const void* wdw,
+                                 const void* wpw, const void* bias, void* z, cudaStream_t s);
+
+// Fused 2-D depthwise-separable block (depthwise KxK, K in {3, 5}, stride 1 or 2, then
+// pointwise): 16-bit NHWC, C % 64 == 0, C_out % 16 == 0 and <= 512; `p` is the depthwise
+// problem (groups = C_in = C_out); x, w_pw, z 16-byte aligned.
+bool dwsep2d_fused_supported(const Conv2d& p, int C_out);
+cudaError_t launch_dwsep2d_fused(const Conv2d& p, int C_out, const void* x, const void* wdw,
+                                 const void* wpw, const void* bias, void* z, cudaStream_t s);
 
 // cuTensorMapEncodeTiled, resolved through the runtime (null if unavailable).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -162,6 +196,10 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn tensor_map_encoder();
 int sm_count();                       // SMs of the current device (cached)
+
+// Test hook (gconv_debug_set_tx_surplus): extra bytes per stage that the generic tensor-core
+// tile kernel's producer declares to its barrier; 0 unless a test set it.
+unsigned int debug_tx_surplus();
 
 // Device error word (set by kernels whose bounded waits give up).
 cudaError_t read_and_clear_device_error(cudaStream_t s, int* code);

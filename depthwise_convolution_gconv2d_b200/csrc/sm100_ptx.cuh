@@ -9,6 +9,7 @@ namespace gconv {
 namespace ptx {
 
 constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;   // 1 s per bounded wait
+constexpr unsigned int ERR_DRAIN = 1u << 30;   // error-word bit: a wind-down wait gave up
 
 
 __device__ __forceinline__ unsigned int smem_u32(const void* p) {
@@ -77,6 +78,28 @@ __device__ __noinline__ inline bool mbar_wait(unsigned long long* bar, unsigned 
       return false;
     }
   }
+}
+
+// Deadline for a wind-down sequence (draining copies or MMAs still in flight): one time budget
+// of WAIT_LIMIT_NS for the whole sequence.
+__device__ __forceinline__ unsigned long long drain_deadline() {
+  return globaltimer() + WAIT_LIMIT_NS;
+}
+
+// Wait for the phase with `parity` to complete, whatever the abort flag says (a CTA that
+// winds down must still let its own copies and MMAs land), until `deadline`; false if the
+// deadline passed first (the phase may never complete, e.g. when a wait elsewhere gave up
+// because a copy delivered fewer bytes than its barrier expects).
+__device__ __noinline__ inline bool mbar_wait_until(unsigned long long* bar, unsigned int parity,
+                                                    unsigned long long deadline,
+                                                    unsigned int* err, unsigned int code) {
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() > deadline) {
+      if (err) atomicOr(err, code);
+      return false;
+    }
+  }
+  return true;
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* map) {

@@ -24,6 +24,8 @@ from __future__ import annotations
 
 import dataclasses
 
+from typing import Optional
+
 import numpy as np
 
 NCHW = 0
@@ -253,6 +255,46 @@ def make_dwconv1d_inputs(p: Dwconv1dProblem, workload: int, dist="normal") -> Dw
     return Dwconv1dInputs(p, x, w, dy)
 
 
+@dataclasses.dataclass
+class DwsepInputs:
+    """Depthwise-separable block (depthwise conv1d, then pointwise 1x1 over channels)."""
+    problem: Dwconv1dProblem
+    C_out: int
+    x: np.ndarray      # [B, T, C] storage
+    w_dw: np.ndarray   # [C, K]
+    w_pw: np.ndarray   # [C_out, C]
+    bias: Optional[np.ndarray]   # [C_out] or None
+
+    def x64(self):
+        return widen(self.x, self.problem.dtype)
+
+    def w_dw64(self):
+        return widen(self.w_dw, self.problem.dtype)
+
+    def w_pw64(self):
+        return widen(self.w_pw, self.problem.dtype)
+
+    def bias64(self):
+        return None if self.bias is None else widen(self.bias, self.problem.dtype)
+
+
+def make_dwsep1d_inputs(p: Dwconv1dProblem, C_out: int, workload: int, bias: bool = True,
+                        dist="normal") -> DwsepInputs:
+    """x ~ N(0,1), w_dw ~ N(0, 1/K), w_pw ~ N(0, 1/C), bias ~ N(0,1) (integer-valued for
+    dist='int'); the same seeds roles as the other workloads (w_pw takes the 'dy' role)."""
+    x = to_storage(draw(np.random.default_rng(seed_for(workload, "x")), (p.B, p.T, p.C), dist),
+                   p.dtype)
+    w_dw = to_storage(draw(np.random.default_rng(seed_for(workload, "w")), (p.C, p.K), dist,
+                           1.0 / np.sqrt(p.K)), p.dtype)
+    w_pw = to_storage(draw(np.random.default_rng(seed_for(workload, "dy")), (C_out, p.C), dist,
+                           1.0 / np.sqrt(p.C)), p.dtype)
+    b = None
+    if bias:
+        b = to_storage(draw(np.random.default_rng(seed_for(workload, "bias")), (C_out,), dist),
+                       p.dtype)
+    return DwsepInputs(p, C_out, x, w_dw, w_pw, b)
+
+
 # ----------------------------------------------------------------------------- workloads
 
 def tiny_grouped(groups: int, layout=NCHW, dtype=F32, bias=False) -> Conv2dProblem:
@@ -275,6 +317,13 @@ def depthwise_56(stride: int = 1, groups: int = 1024, layout=NHWC, dtype=BF16) -
     return Conv2dProblem(32, 1024, 56, 56, 1024, 3, 3, stride, 1, 1, groups, layout, dtype)
 
 
+def grouped_linear(tokens: int = 16384, features: int = 4096, groups: int = 4, layout=NHWC,
+                   dtype=BF16) -> Conv2dProblem:
+    """Grouped linear layer y_g = x_g W_g^T: the grouped conv2d with H = W = 1 and a 1x1
+    kernel, one image per token (the batched-GEMM form of grouping)."""
+    return Conv2dProblem(tokens, features, 1, 1, features, 1, 1, 1, 0, 1, groups, layout, dtype)
+
+
 WORKLOADS = {
     "tiny_grouped_g4": (1, lambda: tiny_grouped(4)),
     "tiny_grouped_g8": (1, lambda: tiny_grouped(8)),
@@ -289,4 +338,6 @@ WORKLOADS = {
     "sweep56_g256": (5, lambda: depthwise_56(1, 256)),
     "sweep56_g64": (5, lambda: depthwise_56(1, 64)),
     "sweep56_g16": (5, lambda: depthwise_56(1, 16)),
+    "grouped_linear": (6, lambda: grouped_linear()),
+    "conformer_dwsep1d": (7, lambda: conformer_dw1d(False)),
 }

@@ -119,19 +119,88 @@ typedef enum {
   GCONV_KERNEL_WGRAD_DW3_TMA = 14,    /* conv2d weight gradient, depthwise 3x3, dilation 1,
                                          stride 1 or 2, pad <= 2, 16-bit NHWC, C % 8 == 0:
                                          x and dy staged by TMA */
-  GCONV_KERNEL_WGRAD_TILED_NCHW = 15  /* GCONV_KERNEL_WGRAD_TILED_NHWC for NCHW tensors: x and
+  GCONV_KERNEL_WGRAD_TILED_NCHW = 15, /* GCONV_KERNEL_WGRAD_TILED_NHWC for NCHW tensors: x and
                                          dy transposed to NHWC in the workspace first */
+  GCONV_KERNEL_DWSEP1D_FUSED = 16,    /* depthwise-separable block in one kernel: depthwise
+                                         conv1d on the CUDA cores into shared memory, pointwise
+                                         GEMM on tcgen05; 16-bit, C % 64 == 0, C_out % 16 == 0
+                                         and <= 512, K in {3, 5, 7, 9, 15, 31} */
+  GCONV_KERNEL_DWSEP_UNFUSED = 17,    /* depthwise-separable block as two launches: the
+                                         depthwise output in the workspace, then the pointwise
+                                         convolution */
+  GCONV_KERNEL_WGRAD_TC_NHWC = 18,    /* conv2d weight gradient on tcgen05 tensor cores: per
+                                         group and tap a GEMM over output positions, dy and x
+                                         read as MN-major TMA tiles; 16-bit NHWC, stride 1,
+                                         C_out/g % 128 == 0, C_in/g % 64 == 0,
+                                         (kW-1)*dilation <= 8, Wo >= 32 */
+  GCONV_KERNEL_WGRAD_TC_NCHW = 19,    /* GCONV_KERNEL_WGRAD_TC_NHWC for NCHW tensors: x and dy
+                                         transposed to NHWC in the workspace first */
+  GCONV_KERNEL_CONV1D_STRIP = 20,     /* dwconv1d: CUDA-core kernel on 128-byte input rows
+                                         (64-channel tiles, taps in registers); 16-bit,
+                                         C % 64 == 0, K in {3, 5, 7, 9, 15, 31} */
+  GCONV_KERNEL_DWSEP2D_FUSED = 21     /* 2-D depthwise-separable block in one kernel: 16-bit
+                                         NHWC, depthwise 3x3 / 5x5, stride 1 / 2, dilation 1,
+                                         C % 64 == 0, C_out % 16 == 0 and <= 512 */
 } gconv_kernel;
 
-/* Output extent of a gconv2d problem: validates the arguments exactly as gconv2d_fwd does and
- * writes *Ho, *Wo by F.conv2d's rule (Ho = floor((H + 2*pad - dilation*(kH-1) - 1) / stride)
- * + 1, same for Wo; the output-size rule of the timing script in "F.conv2d runs x15 slower in
- * mixed-precision/half-precision mode"). y is [N][C_out][Ho][Wo] (NCHW) or [N][Ho][Wo][C_out]
- * (NHWC); dy of the backward calls has the same shape. Host-only, launches nothing.
- * Errors: INVALID_ARG (also for NULL Ho / Wo, or Ho / Wo < 1); *Ho, *Wo untouched then. */
+/* Order and merging of the output channels ("Grouped convolutions", neon issue #296, ibmua's
+ * post on output orderings: the group-major order 111122223333..., the interleaved order
+ * 1234123412341234, and pulling the groups' results together by average or max pooling
+ * across groups). With cpg_out = C_out / groups, filter j of group i is group-major channel
+ * i*cpg_out + j:
+ *   GROUP_MAJOR  y has C_out channels; channel i*cpg_out + j = filter j of group i (bias
+ *                [i*cpg_out + j] added); what gconv2d_fwd writes.
+ *   INTERLEAVED  y has C_out channels; channel j*groups + i = filter j of group i.
+ *   MERGE_AVG    y has cpg_out channels; channel j = mean over groups i of group-major channel
+ *                i*cpg_out + j (each with its bias).
+ *   MERGE_MAX    y has cpg_out channels; channel j = maximum over i of the same. */
+typedef enum {
+  GCONV_OUT_GROUP_MAJOR = 0,
+  GCONV_OUT_INTERLEAVED = 1,
+  GCONV_OUT_MERGE_AVG = 2,
+  GCONV_OUT_MERGE_MAX = 3
+} gconv_out_mode;
+
+/* Output shape of a gconv2d problem: validates the arguments exactly as gconv2d_fwd_out does
+ * and writes *C_y (C_out, or C_out/groups for the merges), *Ho, *Wo by F.conv2d's rule
+ * (Ho = floor((H + 2*pad - dilation*(kH-1) - 1) / stride) + 1, same for Wo; the output-size
+ * rule of the timing script in "F.conv2d runs x15 slower in mixed-precision/half-precision
+ * mode"). y is [N][C_y][Ho][Wo] (NCHW) or [N][Ho][Wo][C_y] (NHWC); dy of the backward calls
+ * has the GROUP_MAJOR shape. Host-only, launches nothing.
+ * Errors: INVALID_ARG (also for NULL outputs, a bad out_mode, or Ho / Wo < 1); the outputs are
+ * untouched then. */
 gconv_status gconv2d_out_shape(int N, int C_in, int H, int W, int C_out, int kH, int kW,
                                int stride, int pad, int dilation, int groups,
-                               gconv_layout layout, gconv_dtype dtype, int* Ho, int* Wo);
+                               gconv_layout layout, gconv_dtype dtype, gconv_out_mode out_mode,
+                               int* C_y, int* Ho, int* Wo);
+
+/* gconv2d_fwd_path writing the output in `out_mode` (above); y has the shape
+ * gconv2d_out_shape reports. The order or the merge is applied in the kernel's epilogue, on
+ * the fp32 accumulators (a merge adds or compares the groups' fp32 values, then rounds once),
+ * so no second pass over y is made. GROUP_MAJOR, and the modes that equal it (one filter per
+ * group for INTERLEAVED, one group for the merges), run exactly as gconv2d_fwd_path. Other
+ * variants: AUTO runs the tensor-core implicit GEMM for 16-bit problems it takes (the
+ * transposed row-strip kernel for INTERLEAVED where that tiling applies, otherwise the tile
+ * kernel; a merge covers all groups of a 16..64-filter block in one tile) and the generic
+ * direct kernel otherwise; DIRECT and GENERIC run the generic direct kernel; IGEMM forces
+ * the tensor cores (UNSUPPORTED / MISALIGNED as for gconv2d_fwd_path).
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
+gconv_status gconv2d_fwd_out(const void* x, const void* w, const void* bias, void* y, int N,
+                             int C_in, int H, int W, int C_out, int kH, int kW, int stride,
+                             int pad, int dilation, int groups, gconv_layout layout,
+                             gconv_dtype dtype, gconv_out_mode out_mode, gconv_path path,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes gconv2d_fwd_out needs (0 if none or invalid), and the gconv_kernel it would
+ * run for 16-byte aligned pointers (a negative gconv_status if it would fail). */
+size_t gconv2d_fwd_out_workspace_size(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                      int stride, int pad, int dilation, int groups,
+                                      gconv_layout layout, gconv_dtype dtype,
+                                      gconv_out_mode out_mode, gconv_path path);
+int gconv2d_fwd_out_select_path(int N, int C_in, int H, int W, int C_out, int kH, int kW,
+                                int stride, int pad, int dilation, int groups,
+                                gconv_layout layout, gconv_dtype dtype, gconv_out_mode out_mode,
+                                gconv_path path);
 
 /* Bytes of workspace gconv2d_fwd needs for this problem under `path` (0 if none; also 0 for
  * invalid arguments, which gconv2d_fwd then rejects). */
@@ -222,13 +291,15 @@ size_t gconv2d_bwd_weight_workspace_size(int N, int C_in, int H, int W, int C_ou
  * N == 0). Deterministic: the N*Ho output rows are cut into slices fixed by the problem's
  * sizes alone, each slice's partial sums are added in a fixed order and the slices are added
  * in slice order (no float atomics), so repeated calls -- on any GPU -- give bitwise-identical
- * dw. AUTO and DIRECT run the TMA-staged depthwise 3x3 kernel where it applies
+ * dw. AUTO runs the TMA-staged depthwise 3x3 kernel where it applies
  * (GCONV_KERNEL_WGRAD_DW3_TMA; x and dy 16-byte aligned), else the depthwise kernel
- * (GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC; x and dy 4-byte aligned), else the tiled kernel for
- * wide groups (GCONV_KERNEL_WGRAD_TILED_NHWC with x and dy 16-byte aligned, or
- * GCONV_KERNEL_WGRAD_TILED_NCHW, which stages NCHW x and dy as NHWC in the workspace), else
- * the generic kernel; GENERIC forces the generic kernel; IGEMM is UNSUPPORTED (there is no
- * tensor-core weight gradient). N*Ho > 2^30 is UNSUPPORTED.
+ * (GCONV_KERNEL_WGRAD_DEPTHWISE_NHWC; x and dy 4-byte aligned), else the tensor-core kernel
+ * for wide groups (GCONV_KERNEL_WGRAD_TC_NHWC with x and dy 16-byte aligned, or
+ * GCONV_KERNEL_WGRAD_TC_NCHW, which stages NCHW x and dy as NHWC in the workspace), else the
+ * CUDA-core tiled kernel (GCONV_KERNEL_WGRAD_TILED_NHWC / _NCHW, same staging), else the
+ * generic kernel. DIRECT runs the same list without the tensor-core kernel; IGEMM forces the
+ * tensor-core kernel (UNSUPPORTED where it does not apply, MISALIGNED for unaligned NHWC x or
+ * dy); GENERIC forces the generic kernel. N*Ho > 2^30 is UNSUPPORTED.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 gconv_status gconv2d_bwd_weight(const void* x, const void* dy, void* dw, int N, int C_in, int H,
                                 int W, int C_out, int kH, int kW, int stride, int pad,
@@ -315,10 +386,74 @@ gconv_status dwconv1d_bwd_weight_noalloc(const void* x, const void* dy, void* dw
                                          int C, int K, int pad_left, int pad_right,
                                          gconv_dtype dtype, void* stream);
 
+/* ---- depthwise-separable block on (batch, steps, channels): a depthwise conv1d followed by a
+ * pointwise (1x1) convolution over channels, the block of the Conformer convolution module
+ * ("Investigate custom Triton kernels for depthwise-separable convolutions in Conformer",
+ * speechbrain #2733: the issue text; the Oct 30 comment on the Fast Conformer downsampler,
+ * built the same way):
+ *   d[b,t,c] = sum_{k<K} w_dw[c,k] * x[b, t+k-pad_left, c]      (dwconv1d_fwd)
+ *   z[b,t,o] = bias[o] + sum_{c<C} w_pw[o,c] * d[b,t,c]
+ * x [B][T][C], w_dw [C][K], w_pw [C_out][C], bias [C_out] or NULL, z [B][T_out][C_out],
+ * T_out = T + pad_left + pad_right - K + 1. Nothing sits between the two convolutions
+ * (normalisation and activation are separate layers). For 16-bit data the intermediate d is
+ * rounded once to the data type (the tensor-core operand); the accumulations are fp32.
+ * AUTO runs the fused kernel (GCONV_KERNEL_DWSEP1D_FUSED: d never leaves the SM) where it
+ * applies, otherwise the composition (GCONV_KERNEL_DWSEP_UNFUSED: d in the workspace, then
+ * the pointwise convolution on the library's own kernels); IGEMM forces the fused kernel
+ * (UNSUPPORTED / MISALIGNED if it cannot run), DIRECT forces the composition, GENERIC the
+ * composition on the generic kernels. The workspace (16-byte aligned) holds d for the
+ * composition; 0 bytes for the fused kernel.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
+size_t dwsep1d_fwd_workspace_size(int B, int T, int C, int K, int pad_left, int pad_right,
+                                  int C_out, gconv_dtype dtype, gconv_path path);
+int dwsep1d_select_path(int B, int T, int C, int K, int pad_left, int pad_right, int C_out,
+                        gconv_dtype dtype, gconv_path path);
+gconv_status dwsep1d_fwd(const void* x, const void* w_dw, const void* w_pw, const void* bias,
+                         void* z, int B, int T, int C, int K, int pad_left, int pad_right,
+                         int C_out, gconv_dtype dtype, gconv_path path, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* ---- 2-D depthwise-separable block: a depthwise conv2d (groups = C, kernel kH x kW, stride,
+ * pad, dilation as for gconv2d_fwd) followed by a pointwise 1x1 convolution C -> C_out, the
+ * strided layers of the Fast Conformer downsampler (same thread, Oct 30 comment):
+ *   z[n,o,ho,wo] = bias[o] + sum_c w_pw[o,c] * d[n,c,ho,wo],  d = gconv2d_fwd(x, w_dw, groups=C)
+ * x in `layout` with C channels; w_dw the depthwise weight of that layout ([C][1][kH][kW] or
+ * [C][kH][kW][1], the same bytes); w_pw [C_out][C]; bias [C_out] or NULL; z in `layout`
+ * with C_out channels and the depthwise output's Ho x Wo. AUTO runs the fused kernel
+ * (GCONV_KERNEL_DWSEP2D_FUSED) where it applies, otherwise the composition
+ * (GCONV_KERNEL_DWSEP_UNFUSED: d in the workspace, then the pointwise convolution, each on
+ * the kernel gconv2d_fwd would pick); IGEMM / DIRECT / GENERIC as for dwsep1d_fwd. The 16-bit
+ * intermediate is rounded once to the data type. The workspace (16-byte aligned) holds d and
+ * the two convolutions' own workspaces for the composition; 0 bytes for the fused kernel.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
+size_t dwsep2d_fwd_workspace_size(int N, int C, int H, int W, int kH, int kW, int stride,
+                                  int pad, int dilation, int C_out, gconv_layout layout,
+                                  gconv_dtype dtype, gconv_path path);
+int dwsep2d_select_path(int N, int C, int H, int W, int kH, int kW, int stride, int pad,
+                        int dilation, int C_out, gconv_layout layout, gconv_dtype dtype,
+                        gconv_path path);
+gconv_status dwsep2d_fwd(const void* x, const void* w_dw, const void* w_pw, const void* bias,
+                         void* z, int N, int C, int H, int W, int kH, int kW, int stride,
+                         int pad, int dilation, int C_out, gconv_layout layout,
+                         gconv_dtype dtype, gconv_path path, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word that kernels with
  * bounded waits set when a wait gives up. *code receives 0 if none gave up. Returns
  * GCONV_ERR_DEVICE_TIMEOUT if one did, GCONV_ERR_CUDA if synchronisation failed. */
 gconv_status gconv_get_device_error(void* stream, int* code);
+
+/* Test hook for the bounded waits. From the next call on, the generic tensor-core tile kernel
+ * (GCONV_KERNEL_IGEMM_TC on shapes that no specialised tiling takes, e.g. output rows narrower
+ * than 128 pixels and not a multiple of 8) declares `bytes` more per pipeline stage to its
+ * mbarrier than its TMA copies deliver, so that stage never completes: its waits give up after
+ * their 1 s limit, the CTA drains its copies and MMAs (each drain bounded by the same limit),
+ * frees its tensor memory and exits, and gconv_get_device_error then returns
+ * GCONV_ERR_DEVICE_TIMEOUT. No fault, trap or unbounded wait is involved; the context stays
+ * usable, and outputs of such a call are undefined. 0 (the default) restores normal
+ * operation. Process-wide, not thread-safe against concurrent launches; for tests only.
+ * Errors: INVALID_ARG unless bytes is a multiple of 16 and at most 65536. */
+gconv_status gconv_debug_set_tx_surplus(unsigned int bytes);
 
 /* Human-readable name of a status. Never NULL. */
 const char* gconv_status_string(gconv_status status);

@@ -118,17 +118,20 @@ def test_wgrad_workspace_query(lib):
 
 
 def test_conv1d_path_selection(lib):
-    """dwconv1d_select_path: the tensor-core kernel (7) for 16-bit data with C % 16 == 0 and
+    """dwconv1d_select_path: the 128-byte-row CUDA-core kernel (20) for 16-bit data with
+    C % 64 == 0 and an instantiated K, else the tensor-core kernel (7) for C % 16 == 0 and
     K <= 49, else the CUDA-core ring kernel (6) where it is instantiated, else the generic
     kernel (5); a forced family that cannot run gives -UNSUPPORTED."""
     BF16, F32 = 2, 0
     sel = lambda B, T, C, K, pl, pr, dt, path: lib.dwconv1d_select_path(B, T, C, K, pl, pr, dt,
                                                                         path)
     conformer = (8, 2048, 512, 31, 15, 15, BF16)
-    assert sel(*conformer, 0) == 7
-    assert sel(*conformer, 1) == 6
+    assert sel(*conformer, 0) == 20
+    assert sel(*conformer, 1) == 20
     assert sel(*conformer, 2) == 7
     assert sel(*conformer, 3) == 5
+    assert sel(8, 2048, 512, 33, 16, 16, BF16, 0) == 7          # K = 33: no strip instantiation
+    assert sel(8, 2048, 96, 31, 15, 15, BF16, 0) == 7           # C % 64 != 0
     assert sel(8, 2048, 512, 31, 15, 15, F32, 0) == 5
     assert sel(8, 2048, 512, 31, 15, 15, F32, 2) == -2          # UNSUPPORTED
     assert sel(2, 300, 72, 31, 15, 15, BF16, 0) == 6            # C % 16 == 8: ring only
@@ -199,12 +202,17 @@ def test_bwd_path_selection(lib):
     assert sel(wg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 14
     assert sel(wg, 32, 1024, 56, 56, 1024, 3, 1, 3, 1, 1024) == 11   # pad 3: LDG kernel
     assert sel(wg, 32, 1024, 56, 56, 1024, 5, 1, 2, 1, 1024) == 11   # 5x5: LDG kernel
-    # wide groups: tensor cores (NHWC, NCHW staging); weight gradient generic
+    # wide groups: tensor cores for both gradients (NHWC, NCHW staging); DIRECT keeps the
+    # CUDA-core tiled weight gradient
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 3
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 4
-    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 13
-    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 15   # NCHW: staged
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4) == 18
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0) == 19   # NCHW: staged
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, path=2) == 18
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, path=1) == 13
+    assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, layout=0, path=1) == 15
     assert sel(wg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, path=3) == 10
+    assert sel(wg, 1, 256, 64, 64, 128, 3, 1, 1, 1, 4) == 13          # 32 filters a group
     assert sel(wg, 1, 64, 56, 56, 64, 3, 1, 1, 1, 4) == 10          # 16 channels a group
     # narrow groups (4 channels): the narrow-group forward kernel
     assert sel(dg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 256) == 8
@@ -214,10 +222,11 @@ def test_bwd_path_selection(lib):
     assert sel(dg, 1, 64, 16, 16, 64, 3, 1, 3, 1, 16) == 9
     assert sel(dg, 1, 64, 16, 16, 64, 3, 1, 1, 1, 64, dtype=0) == 9
     assert sel(dg, 1, 512, 256, 256, 512, 3, 1, 1, 1, 4, path=3) == 9
-    # forced IGEMM where the data gradient is not a stride-1 convolution, or on the weight
-    # gradient: UNSUPPORTED
+    # forced IGEMM where the data gradient is not a stride-1 convolution, or on a weight
+    # gradient the tensor-core kernel does not take (stride 2, 32 filters a group): UNSUPPORTED
     assert sel(dg, 1, 512, 64, 64, 512, 3, 2, 1, 1, 4, path=2) == -2
-    assert sel(wg, 1, 512, 64, 64, 512, 3, 1, 1, 1, 4, path=2) == -2
+    assert sel(wg, 1, 512, 64, 64, 512, 3, 2, 1, 1, 4, path=2) == -2
+    assert sel(wg, 1, 256, 64, 64, 128, 3, 1, 1, 1, 4, path=2) == -2
 
 
 def test_bwd_workspace_queries(lib):
@@ -259,7 +268,7 @@ def test_out_shape_query_matches_oracle_and_enumeration(lib):
     """gconv2d_out_shape / dwconv1d_out_steps (the binding allocates y and checks dy with
     them) agree with the oracle's output size and with counting window positions."""
     import oracle
-    Ho, Wo = ctypes.c_int(-7), ctypes.c_int(-7)
+    Cy, Ho, Wo = ctypes.c_int(-7), ctypes.c_int(-7), ctypes.c_int(-7)
     for size in (1, 2, 5, 7, 16, 57):
         for k in (1, 2, 3, 5):
             for s in (1, 2, 3):
@@ -268,7 +277,8 @@ def test_out_shape_query_matches_oracle_and_enumeration(lib):
                         want = _enumerated_extent(size, k, s, p, d)
                         assert oracle.out_extent(size, k, s, p, d) == want
                         st = lib.gconv2d_out_shape(2, 4, size, size + 1, 8, k, k, s, p, d, 2, 1, 2,
-                                                   ctypes.byref(Ho), ctypes.byref(Wo))
+                                                   0, ctypes.byref(Cy), ctypes.byref(Ho),
+                                                   ctypes.byref(Wo))
                         if want < 1:
                             assert st == 1
                             continue
@@ -276,9 +286,17 @@ def test_out_shape_query_matches_oracle_and_enumeration(lib):
                         assert Ho.value == want
                         assert Wo.value == _enumerated_extent(size + 1, k, s, p, d)
     # argument errors reach the query too
-    assert lib.gconv2d_out_shape(1, 6, 8, 8, 8, 3, 3, 1, 1, 1, 4, 1, 2, ctypes.byref(Ho),
-                                 ctypes.byref(Wo)) == 1          # 6 channels in 4 groups
-    assert lib.gconv2d_out_shape(1, 8, 8, 8, 8, 3, 3, 1, 1, 1, 4, 1, 2, None, None) == 1
+    assert lib.gconv2d_out_shape(1, 6, 8, 8, 8, 3, 3, 1, 1, 1, 4, 1, 2, 0, ctypes.byref(Cy),
+                                 ctypes.byref(Ho), ctypes.byref(Wo)) == 1   # 6 ch in 4 groups
+    assert lib.gconv2d_out_shape(1, 8, 8, 8, 8, 3, 3, 1, 1, 1, 4, 1, 2, 0, None, None,
+                                 None) == 1
+    assert lib.gconv2d_out_shape(1, 8, 8, 8, 8, 3, 3, 1, 1, 1, 4, 1, 2, 4, ctypes.byref(Cy),
+                                 ctypes.byref(Ho), ctypes.byref(Wo)) == 1   # no mode 4
+    # channels of y: C_out for the orders, C_out / groups for the merges
+    for mode, want in ((0, 12), (1, 12), (2, 3), (3, 3)):
+        assert lib.gconv2d_out_shape(2, 8, 9, 9, 12, 3, 3, 2, 1, 1, 4, 1, 2, mode,
+                                     ctypes.byref(Cy), ctypes.byref(Ho), ctypes.byref(Wo)) == 0
+        assert (Cy.value, Ho.value, Wo.value) == (want, 5, 5)
     T_out = ctypes.c_int(0)
     for T, K, pl, pr in ((2048, 31, 15, 15), (2048, 31, 30, 0), (10, 3, 0, 0), (5, 9, 4, 4),
                          (3, 31, 15, 15)):
@@ -301,3 +319,27 @@ def test_binding_restates_no_shape_rule():
     assert "_out_extent" not in src
     assert "pad_left + pad_right - K" not in src
     assert "dilation * (k" not in src
+
+
+def _declared_param_counts():
+    counts = {}
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(([^)]*)\)\s*;", text,
+                             flags=re.M | re.S):
+            params = m.group(2).strip()
+            counts[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return counts
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every function the binding declares to ctypes takes as many arguments as the header
+    says (a miscount would shift arguments at call time)."""
+    counts = _declared_param_counts()
+    for name in binding.EXPORTS:
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None, f"{name} has no argtypes"
+        assert len(argtypes) == counts[name], (name, len(argtypes), counts[name])

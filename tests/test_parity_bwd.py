@@ -249,3 +249,67 @@ def test_wgrad_wide_group_sampled():
     t = [torch.from_numpy(idx[:, i]).to(dw.device) for i in range(4)]
     got = to_f64(dw[t[0], t[2], t[3], t[1]])
     assert_close(got, ref, p.dtype, "wide-group dw")
+
+
+# ------------------------------------------------------------ tensor-core weight gradient
+
+TC_WGRAD_CASES = [
+    # N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups
+    (2, 256, 10, 40, 256, 3, 3, 1, 1, 1, 2),      # 128 / 128, one partial 128-pixel segment
+    (1, 128, 6, 130, 256, 3, 3, 1, 1, 1, 1),      # 256 filters: two filter blocks; ragged rows
+    (1, 192, 5, 64, 128, 5, 5, 1, 2, 1, 1),       # 5x5: 64-channel blocks (3 of them)
+    (2, 128, 8, 36, 128, 3, 3, 1, 2, 2, 1),       # dilation 2
+    (1, 64, 9, 48, 128, 1, 1, 1, 0, 1, 1),        # 1x1
+    (1, 128, 7, 33, 128, 3, 1, 1, 1, 1, 1),       # 3x1
+    (3, 256, 4, 32, 512, 3, 3, 1, 0, 1, 4),       # 4 groups, no padding
+]
+
+
+@pytest.mark.parametrize("case", TC_WGRAD_CASES)
+@pytest.mark.parametrize("layout", [wl.NHWC, wl.NCHW])
+def test_wgrad_tensor_cores(case, layout):
+    p = wl.Conv2dProblem(*case, layout=layout, dtype=wl.BF16)
+    assert wgrad_kernel(p) == (18 if layout == wl.NHWC else 19)
+    inp, dy = inputs(p, 45)
+    assert_close(to_f64(gpu_wgrad(p, inp, dy)), oracle_wgrad(p, inp, dy), p.dtype, f"dw {case}")
+    assert gb.device_error() == 0
+
+
+def test_wgrad_tensor_cores_fp16_and_forced_paths():
+    p = wl.Conv2dProblem(2, 256, 10, 40, 256, 3, 3, 1, 1, 1, 2, wl.NHWC, wl.F16)
+    inp, dy = inputs(p, 46)
+    ref = oracle_wgrad(p, inp, dy)
+    assert_close(to_f64(gpu_wgrad(p, inp, dy)), ref, p.dtype, "fp16")
+    assert wgrad_kernel(p, gb.PATH_IGEMM) == 18 and wgrad_kernel(p, gb.PATH_DIRECT) == 13
+    assert_close(to_f64(gpu_wgrad(p, inp, dy, gb.PATH_IGEMM)), ref, p.dtype, "forced IGEMM")
+    assert_close(to_f64(gpu_wgrad(p, inp, dy, gb.PATH_DIRECT)), ref, p.dtype, "CUDA cores")
+
+
+def test_wgrad_tensor_cores_integer_exact_and_deterministic():
+    """Integer-valued data: every partial sum is an exact integer in fp32, so the slices'
+    fixed-order sum is exact and dw equals the oracle's value rounded to bf16; two calls give
+    the same bits."""
+    p = wl.Conv2dProblem(2, 256, 10, 40, 256, 3, 3, 1, 1, 1, 2, wl.NHWC, wl.BF16)
+    inp, dy = inputs(p, 47, "int")
+    assert wgrad_kernel(p) == 18
+    a = gpu_wgrad(p, inp, dy)
+    b = gpu_wgrad(p, inp, dy)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    rnd = lambda v: wl.widen(wl.to_storage(v, wl.BF16), wl.BF16)
+    assert np.array_equal(to_f64(a), rnd(oracle_wgrad(p, inp, dy)))
+
+
+def test_wgrad_wide_group_sampled_nchw():
+    p = wl.wide_group(wl.NCHW)
+    assert wgrad_kernel(p) == 19
+    inp, dy = inputs(p, 48)
+    dw = gpu_wgrad(p, inp, dy)
+    r = np.random.default_rng(49)
+    n = 400
+    idx = np.stack([r.integers(0, p.C_out, n), r.integers(0, p.cpg_in, n),
+                    r.integers(0, 3, n), r.integers(0, 3, n)], 1)
+    ref = oracle.conv2d_bwd_weight_points(inp.x64(), wl.widen(dy, p.dtype), (3, 3), idx,
+                                          p.stride, p.pad, p.dilation, p.groups, p.layout)
+    t = [torch.from_numpy(idx[:, i]).to(dw.device) for i in range(4)]
+    got = to_f64(dw[t[0], t[1], t[2], t[3]])
+    assert_close(got, ref, p.dtype, "wide-group dw, NCHW")

@@ -45,13 +45,47 @@ def kernel_of(p, path=gb.PATH_AUTO):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("path", [gb.PATH_AUTO, gb.PATH_DIRECT])
+@pytest.mark.parametrize("path", [gb.PATH_AUTO, gb.PATH_IGEMM])
 def test_conformer_full_size(causal, path):
-    """The Conformer layer in full on the path the library picks (the tensor-core kernel) and
-    forced onto the CUDA-core ring kernel."""
+    """The Conformer layer in full on the path the library picks (the 128-byte-row CUDA-core
+    kernel) and forced onto the tensor-core kernel."""
     p = wl.conformer_dw1d(causal)
-    assert kernel_of(p) == 7 and kernel_of(p, gb.PATH_DIRECT) == 6
+    assert kernel_of(p) == 20 and kernel_of(p, gb.PATH_DIRECT) == 20
+    assert kernel_of(p, gb.PATH_IGEMM) == 7
     check(p, 3, path=path)
+
+
+# The 128-byte-row kernels (16-bit, C % 64 == 0, K in {3, 5, 7, 9, 15, 31}): tiles of 64
+# channels x 112 steps, a run of tiles per CTA; weight gradient partials per run.
+STRIP_CASES = [
+    # B, T, C, K, pl, pr
+    (2, 300, 64, 31, 15, 15),     # ragged last tile (300 = 2 * 112 + 76)
+    (1, 1000, 128, 3, 1, 1),      # two channel blocks
+    (3, 117, 192, 5, 4, 0),       # causal-style pads, three channel blocks
+    (1, 40, 64, 15, 7, 7),        # fewer steps than a tile
+    (2, 500, 64, 7, 0, 0),        # T_out < T
+    (1, 300, 64, 31, 30, 30),     # T_out > T
+    (1, 100, 64, 9, 200, 0),      # left pad wider than a tile: whole tiles of zero input
+    (4, 2048, 128, 31, 15, 15),   # many tiles a run
+]
+
+
+@pytest.mark.parametrize("case", STRIP_CASES)
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F16])
+def test_strip_kernels(case, dtype):
+    p = wl.Dwconv1dProblem(*case, dtype)
+    assert kernel_of(p) == 20
+    check(p, 35)
+
+
+def test_strip_integer_bit_exact_and_wgrad_deterministic():
+    p = wl.Dwconv1dProblem(3, 700, 128, 31, 15, 15, wl.BF16)
+    inp = wl.make_dwconv1d_inputs(p, 36, "int")
+    inp.w = wl.to_storage(np.random.default_rng(6).integers(-2, 3, (p.C, p.K)), wl.BF16)
+    (y, dx, dw), (ry, rdx, rdw) = gpu_all(inp), oracle_all(inp)
+    assert np.array_equal(y, ry) and np.array_equal(dx, rdx)
+    rnd = lambda v: wl.widen(wl.to_storage(v, wl.BF16), wl.BF16)
+    assert np.array_equal(dw, rnd(rdw))
 
 
 SMALL = [
