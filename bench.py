@@ -432,6 +432,35 @@ def dwsep_measurements(torch, gb, device, stream, pk, reps):
                                           (pk["bf16_tflops"] * 1e12), 3),
                      "alg_bytes": nbytes, "alg_flops": flops}
         del ws
+    # the strided 2-D block of a Fast Conformer downsampler: x[8, 512, 40, 256] NHWC
+    # (frames x frequency bins), depthwise 3x3 stride 2 pad 1, then pointwise 256 -> 256
+    N, H, W, C, k, st, pad, Co = 8, 512, 40, 256, 3, 2, 1, 256
+    p2 = wl.Dwconv1dProblem(N, H * W, C, k * k, 0, 0, wl.BF16)
+    inp2 = wl.make_dwsep1d_inputs(p2, Co, 8)
+    x2 = dev_tensor(torch, inp2.x.reshape(N, H, W, C), wl.BF16, device)
+    wdw2 = dev_tensor(torch, inp2.w_dw.reshape(C, k, k, 1), wl.BF16, device)
+    wpw2, b2 = (dev_tensor(torch, a, wl.BF16, device) for a in (inp2.w_pw, inp2.bias))
+    Ho, Wo = gb.out_shape(N, C, H, W, C, k, k, st, pad, 1, C, "NHWC", wl.BF16)
+    z2 = torch.empty((N, Ho, Wo, Co), dtype=torch.bfloat16, device=device)
+    nbytes2 = (x2.numel() + wdw2.numel() + wpw2.numel() + b2.numel() + z2.numel()) * 2
+    flops2 = 2 * N * Ho * Wo * C * (k * k + Co)
+    for name, path in (("dwsep2d_fused", gb.PATH_AUTO), ("dwsep2d_two_launches", gb.PATH_DIRECT)):
+        kname = gb.KERNEL_NAMES.get(gb.dwsep2d_select_path(N, C, H, W, k, k, st, pad, 1, Co,
+                                                           "NHWC", wl.BF16, path))
+        need = gb.load_library().dwsep2d_fwd_workspace_size(N, C, H, W, k, k, st, pad, 1, Co,
+                                                            wl.NHWC, wl.BF16, path)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+        fn = lambda i: gb.dwsep2d_fwd(x2, wdw2, wpw2, b2, st, pad, 1, "NHWC", out=z2,
+                                      workspace=ws, path=path, stream=stream)
+        for _ in range(3):
+            fn(0)
+        med, mean = time_launches(torch, fn, stream, reps, flush)
+        out[name] = {"kernel": kname, "us": round(med * 1e3, 2),
+                     "TFLOP/s": round(flops2 / (med * 1e-3) / 1e12, 1),
+                     "GB/s": round(nbytes2 / (med * 1e-3) / 1e9, 1), "bound": "hbm",
+                     "frac": round(nbytes2 / (pk["hbm_gbs"] * 1e9) / (med * 1e-3), 3),
+                     "alg_bytes": nbytes2, "alg_flops": flops2}
+        del ws
     return out
 
 

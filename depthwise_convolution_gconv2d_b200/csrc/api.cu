@@ -215,6 +215,7 @@ int dgrad_choose(const Conv2d& p, int path, const void* dy, const void* wt, cons
   const int vb = dgrad_depthwise_vec_bytes(p);
   const bool dwk = dgrad_depthwise_supported(p) &&
                    (query || (aligned_to(dy, vb) && aligned_to(dx, vb)));
+  const bool dgs = dgrad_dw3s2_tma_supported(p) && (query || (aligned16(dy) && aligned16(dx)));
   switch (path) {
     case GCONV_PATH_GENERIC:
       return GCONV_KERNEL_DGRAD_GENERIC;
@@ -225,6 +226,7 @@ int dgrad_choose(const Conv2d& p, int path, const void* dy, const void* wt, cons
         k = choose_kernel(*q, path, dy, wt, dx, why);
       *why = GCONV_OK;
       if (k >= 0 && k != GCONV_KERNEL_DIRECT_GENERIC) return k;
+      if (dgs) return GCONV_KERNEL_DGRAD_DW3S2_TMA;
       return dwk ? GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC : GCONV_KERNEL_DGRAD_GENERIC;
     }
     case GCONV_PATH_IGEMM:
@@ -237,7 +239,8 @@ int dgrad_choose(const Conv2d& p, int path, const void* dy, const void* wt, cons
 }
 
 size_t dgrad_workspace(const Conv2d& p, const Conv2d& q, int kernel) {
-  if (kernel == GCONV_KERNEL_DGRAD_GENERIC || kernel == GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC)
+  if (kernel == GCONV_KERNEL_DGRAD_GENERIC || kernel == GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC ||
+      kernel == GCONV_KERNEL_DGRAD_DW3S2_TMA)
     return 0;
   const size_t fwd = kernel == GCONV_KERNEL_IGEMM_TC_NCHW ? igemm_nchw_workspace(q) : 0;
   return round_up(weight_bytes(p), 256) + fwd;
@@ -550,6 +553,8 @@ gconv_status gconv2d_bwd_data_path(const void* dy, const void* w, void* dx, int 
     return cuda_status(launch_dgrad_generic(p, dy, w, dx, s));
   if (kernel == GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC)
     return cuda_status(launch_dgrad_depthwise(p, dy, w, dx, s));
+  if (kernel == GCONV_KERNEL_DGRAD_DW3S2_TMA)
+    return cuda_status(launch_dgrad_dw3s2_tma(p, dy, w, dx, s));
   st = cuda_status(launch_flip_transpose_weight(p, w, workspace, s));
   if (st != GCONV_OK) return st;
   const size_t off = round_up(weight_bytes(p), 256);

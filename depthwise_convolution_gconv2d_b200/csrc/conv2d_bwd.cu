@@ -554,6 +554,178 @@ __global__ void __launch_bounds__(256) dgrad_depthwise_nhwc_kernel(const T* __re
   }
 }
 
+// ------------------------------------------------------------------ stride-2 depthwise 3x3 dgrad
+// The data gradient of a depthwise 3x3, stride 2, pad 1 layer is an upsampling: dx pixel (h, w)
+// collects w[kh][kw] * dy[(h + 1 - kh) / 2][(w + 1 - kw) / 2] over the taps whose numerators are
+// even -- one tap at (even h, even w), two at mixed parities, four at (odd, odd). A tile is
+// DGS_BH dx rows x 28 dx columns x 64 channels (h0, w0 even); its dy box is rows
+// [h0/2, h0/2 + BH/2] x columns [w0/2, w0/2 + 14] x 64 channels (TMA, zero fill past the
+// edges), in a ring of stages filled by a producer warp. Seven compute warps own 4 dx columns
+// each for all 32 channel pairs: a thread's 4 columns read dy columns 2g .. 2g+2 of the box,
+// so each dy word it needs is read once per tile, and the 9 taps of its channel pair stay in
+// registers. Each warp stages its [BH][4][64] dx box in shared memory and writes it with one
+// TMA store (clipped at the image's edges), as in the forward 3x3 kernel.
+constexpr int DGS_R = 4;                    // dx columns per thread
+constexpr int DGS_NG = 7;                   // compute warps
+constexpr int DGS_BW = DGS_R * DGS_NG;      // dx columns per tile (even)
+constexpr int DGS_BH = 8;                   // dx rows per tile (even)
+constexpr int DGS_IW = DGS_BW / 2 + 1;      // dy box columns
+constexpr int DGS_IH = DGS_BH / 2 + 1;      // dy box rows
+constexpr int DGS_CH = 64;
+constexpr int DGS_THREADS = 32 + 32 * DGS_NG;
+constexpr int DGS_MAX_STAGES = 6;
+constexpr size_t DGS_SMEM_CTA = 72 * 1024;  // three CTAs per SM
+
+struct DgsParams {
+  int N, H, W, C, Ho, Wo;
+  int n_ct, n_wt, n_ht, num_tiles, stages;
+  unsigned int stage_bytes, tx_bytes;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(DGS_THREADS, 3)
+    dgrad_dw3s2_tma_kernel(const __grid_constant__ CUtensorMap tmd,
+                           const __grid_constant__ CUtensorMap tmx, const T* __restrict__ w,
+                           const DgsParams P, unsigned int* err) {
+  using namespace ptx;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = ptx::align_smem(smem_raw, 128u);
+  unsigned char* ostage = smem + (size_t)P.stages * P.stage_bytes;
+  unsigned long long* full =
+      reinterpret_cast<unsigned long long*>(ostage + (size_t)DGS_BH * DGS_BW * DGS_CH * 2);
+  unsigned long long* empty = full + DGS_MAX_STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + DGS_MAX_STAGES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t_begin = (int)((long long)P.num_tiles * blockIdx.x / gridDim.x);
+  const int t_end = (int)((long long)P.num_tiles * (blockIdx.x + 1) / gridDim.x);
+  // tile t: tw fastest, then th, n, channel tile
+  auto decode = [&](int t, int& ct, int& n, int& th, int& tw) {
+    tw = t % P.n_wt;
+    int r = t / P.n_wt;
+    th = r % P.n_ht;
+    r /= P.n_ht;
+    n = r % P.N;
+    ct = r / P.N;
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], DGS_NG);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmd);
+    prefetch_tmap(&tmx);
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      unsigned int ph = 0;
+      long long issued = 0;
+      for (int t = t_begin; t < t_end; ++t) {
+        if (!mbar_try_wait(&empty[s], ph ^ 1u) &&
+            !mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, 128u))
+          break;
+        int ct, n, th, tw;
+        decode(t, ct, n, th, tw);
+        mbar_arrive_expect_tx(&full[s], P.tx_bytes);
+        tma_load_4d(smem + (size_t)s * P.stage_bytes, &tmd, &full[s], ct * DGS_CH,
+                    tw * (DGS_BW / 2), th * (DGS_BH / 2), n);
+        ++issued;
+        if (++s == P.stages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      const unsigned long long dl = drain_deadline();
+      for (long long q = (issued > P.stages ? issued - P.stages : 0); q < issued; ++q)
+        mbar_wait_until(&full[q % P.stages], (unsigned int)((q / P.stages) & 1), dl, err,
+                        ERR_DRAIN);
+    }
+  } else {
+    const int cp = lane, g = warp - 1;
+    int prev_ct = -1;
+    float2 wv[3][3];
+    int s = 0;
+    unsigned int ph = 0;
+    unsigned char* wstage = ostage + (size_t)g * DGS_BH * DGS_R * DGS_CH * 2;
+    unsigned int* orow = reinterpret_cast<unsigned int*>(wstage) + cp;
+    for (int t = t_begin; t < t_end; ++t) {
+      bool got = mbar_try_wait(&full[s], ph);
+      if (!got) got = mbar_wait(&full[s], ph, abort_flag, err, 128u);
+      if (!__all_sync(0xffffffffu, got)) break;
+      if (lane == 0) bulk_wait_read0();              // this warp's previous store has read it
+      __syncwarp();
+      int ct, n, th, tw;
+      decode(t, ct, n, th, tw);
+      const int ch = ct * DGS_CH + 2 * cp;
+      const bool ch_ok = ch < P.C;
+      if (ct != prev_ct) {
+        prev_ct = ct;
+#pragma unroll
+        for (int kh = 0; kh < 3; ++kh)
+#pragma unroll
+          for (int kw = 0; kw < 3; ++kw)
+            wv[kh][kw] = ch_ok ? make_float2(Elem<T>::to_f32(w[ch * 9 + kh * 3 + kw]),
+                                             Elem<T>::to_f32(w[(ch + 1) * 9 + kh * 3 + kw]))
+                               : make_float2(0.f, 0.f);
+      }
+      // box word (row, column, pair) = (row * IW + column) * 32 + pair; this thread's dy
+      // columns are 2g .. 2g + 2
+      const uint32_t* pd = reinterpret_cast<const uint32_t*>(smem + (size_t)s * P.stage_bytes) +
+                           (2 * g) * (DGS_CH / 2) + cp;
+      float2 d[DGS_IH][3];
+#pragma unroll
+      for (int r = 0; r < DGS_IH; ++r)
+#pragma unroll
+        for (int m = 0; m < 3; ++m) d[r][m] = unpack2<T>(pd[(r * DGS_IW + m) * (DGS_CH / 2)]);
+#pragma unroll
+      for (int j = 0; j < DGS_BH; ++j) {
+        float2 acc[DGS_R];
+#pragma unroll
+        for (int r = 0; r < DGS_R; ++r) acc[r] = make_float2(0.f, 0.f);
+        // (kh, dy box row) pairs of dx row j: kh = 1 from row j/2 (even j); kh = 0 from row
+        // (j+1)/2 and kh = 2 from row (j-1)/2 (odd j)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int kh = (j % 2 == 0) ? 1 : (q == 0 ? 0 : 2);
+          if (j % 2 == 0 && q == 1) continue;
+          const int row = (j % 2 == 0) ? j / 2 : (q == 0 ? (j + 1) / 2 : (j - 1) / 2);
+          // dx column 4g + r: even r: kw = 1 from dy column r/2; odd r: kw = 0 from
+          // (r+1)/2 and kw = 2 from (r-1)/2
+          acc[0] = ffma2(wv[kh][1], d[row][0], acc[0]);
+          acc[1] = ffma2(wv[kh][0], d[row][1], acc[1]);
+          acc[1] = ffma2(wv[kh][2], d[row][0], acc[1]);
+          acc[2] = ffma2(wv[kh][1], d[row][1], acc[2]);
+          acc[3] = ffma2(wv[kh][0], d[row][2], acc[3]);
+          acc[3] = ffma2(wv[kh][2], d[row][1], acc[3]);
+        }
+#pragma unroll
+        for (int r = 0; r < DGS_R; ++r)
+          orow[(j * DGS_R + r) * (DGS_CH / 2)] = pack2<T>(acc[r]);
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty[s]);
+        if (tw * DGS_BW + g * DGS_R < P.W) {   // a box wholly right of the image is skipped
+          tma_store_4d(&tmx, wstage, ct * DGS_CH, tw * DGS_BW + g * DGS_R, th * DGS_BH, n);
+          bulk_commit();
+        }
+      }
+      if (++s == P.stages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    if (lane == 0) bulk_wait0();
+  }
+  __syncthreads();
+}
+
 // ------------------------------------------------------------------ wide-group weight gradient
 // NHWC, 16-bit, C_in/g and C_out/g multiples of 8 and at least 32. Per group and tap (kh, kw),
 // dw[co][kh][kw][ci] over the group's filters and channels is a sum over output positions p of
@@ -802,6 +974,60 @@ cudaError_t dgrad_dw_k(const Conv2d& p, const void* dy, const void* w, void* dx,
 }
 
 template <typename T>
+cudaError_t launch_dgs(const Conv2d& p, const void* dy, const void* w, void* dx, cudaStream_t s) {
+  DgsParams P;
+  P.N = p.N; P.H = p.H; P.W = p.W; P.C = p.C_in; P.Ho = p.Ho; P.Wo = p.Wo;
+  P.n_ct = (p.C_in + DGS_CH - 1) / DGS_CH;
+  P.n_wt = (p.W + DGS_BW - 1) / DGS_BW;
+  P.n_ht = (p.H + DGS_BH - 1) / DGS_BH;
+  const long long tiles = (long long)P.n_ct * p.N * P.n_ht * P.n_wt;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  P.num_tiles = (int)tiles;
+  P.tx_bytes = (unsigned int)(DGS_CH * DGS_IW * DGS_IH * 2);
+  P.stage_bytes = (P.tx_bytes + 127u) & ~127u;
+  const size_t ostage = (size_t)DGS_BH * DGS_BW * DGS_CH * 2;
+  const size_t fixed = 128 + ostage + 2 * DGS_MAX_STAGES * 8 + 16;
+  int stages = (int)((DGS_SMEM_CTA - fixed) / P.stage_bytes);
+  if (stages > DGS_MAX_STAGES) stages = DGS_MAX_STAGES;
+  if (stages < 2) return cudaErrorInvalidValue;
+  P.stages = stages;
+  const size_t smem = fixed + (size_t)stages * P.stage_bytes;
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const CUtensorMapDataType dt =
+      p.dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint32_t ones[4] = {1, 1, 1, 1};
+  CUtensorMap tmd, tmx;
+  const cuuint64_t ddim[4] = {(cuuint64_t)p.C_out, (cuuint64_t)p.Wo, (cuuint64_t)p.Ho,
+                              (cuuint64_t)p.N};
+  const cuuint64_t dstr[3] = {(cuuint64_t)p.C_out * 2, (cuuint64_t)p.Wo * p.C_out * 2,
+                              (cuuint64_t)p.Ho * p.Wo * p.C_out * 2};
+  const cuuint32_t dbox[4] = {DGS_CH, DGS_IW, DGS_IH, 1};
+  if (enc(&tmd, dt, 4, const_cast<void*>(dy), ddim, dstr, dbox, ones,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const cuuint64_t xdim[4] = {(cuuint64_t)p.C_in, (cuuint64_t)p.W, (cuuint64_t)p.H,
+                              (cuuint64_t)p.N};
+  const cuuint64_t xstr[3] = {(cuuint64_t)p.C_in * 2, (cuuint64_t)p.W * p.C_in * 2,
+                              (cuuint64_t)p.H * p.W * p.C_in * 2};
+  const cuuint32_t xbox[4] = {DGS_CH, DGS_R, DGS_BH, 1};
+  if (enc(&tmx, dt, 4, dx, xdim, xstr, xbox, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  static std::atomic<unsigned int> configured{0};
+  cudaError_t e = set_max_dynamic_smem((const void*)dgrad_dw3s2_tma_kernel<T>, DGS_SMEM_CTA,
+                                       configured);
+  if (e != cudaSuccess) return e;
+  long long grid = (long long)sm_count() * 3;
+  if (grid > P.num_tiles) grid = P.num_tiles;
+  dgrad_dw3s2_tma_kernel<T><<<(unsigned)grid, DGS_THREADS, smem, s>>>(
+      tmd, tmx, (const T*)w, P, device_error_word());
+  return cudaGetLastError();
+}
+
+template <typename T>
 cudaError_t dgrad_dw_typed(const Conv2d& p, const void* dy, const void* w, void* dx,
                            cudaStream_t s) {
   switch (p.kH) {
@@ -982,6 +1208,21 @@ bool dgrad_depthwise_supported(const Conv2d& p) {
 }
 
 int dgrad_depthwise_vec_bytes(const Conv2d& p) { return 2 * dgrad_depthwise_vec(p); }
+
+bool dgrad_dw3s2_tma_supported(const Conv2d& p) {
+  return p.layout == GCONV_NHWC && p.dtype != GCONV_F32 && p.groups == p.C_in &&
+         p.C_out == p.C_in && p.kH == 3 && p.kW == 3 && p.dil == 1 && p.stride == 2 &&
+         p.pad == 1 && p.C_in % 8 == 0 && p.N <= 65535 &&
+         (long long)((p.C_in + DGS_CH - 1) / DGS_CH) * p.N * ((p.H + DGS_BH - 1) / DGS_BH) *
+                 ((p.W + DGS_BW - 1) / DGS_BW) <= 0x7fffffffLL;
+}
+
+cudaError_t launch_dgrad_dw3s2_tma(const Conv2d& p, const void* dy, const void* w, void* dx,
+                                   cudaStream_t s) {
+  if ((long long)p.N * p.H * p.W == 0) return cudaSuccess;
+  if (p.dtype == GCONV_F16) return launch_dgs<__half>(p, dy, w, dx, s);
+  return launch_dgs<__nv_bfloat16>(p, dy, w, dx, s);
+}
 
 cudaError_t launch_dgrad_depthwise(const Conv2d& p, const void* dy, const void* w, void* dx,
                                    cudaStream_t s) {

@@ -132,6 +132,11 @@ bool dgrad_depthwise_supported(const Conv2d& p);
 int dgrad_depthwise_vec_bytes(const Conv2d& p);
 cudaError_t launch_dgrad_depthwise(const Conv2d& p, const void* dy, const void* w, void* dx,
                                    cudaStream_t s);
+// Depthwise 3x3, stride 2, pad 1 data gradient on a TMA ring (16-bit NHWC, C % 8 == 0; dy and
+// dx 16-byte aligned).
+bool dgrad_dw3s2_tma_supported(const Conv2d& p);
+cudaError_t launch_dgrad_dw3s2_tma(const Conv2d& p, const void* dy, const void* w, void* dx,
+                                   cudaStream_t s);
 bool wgrad_depthwise_supported(const Conv2d& p);
 // Depthwise 3x3 weight gradient on a TMA ring (16-bit NHWC, dilation 1, stride 1 or 2, pad <= 2,
 // C % 8 == 0; x and dy 16-byte aligned).

@@ -319,10 +319,12 @@ cudaError_t launch_wgrad_tc(const Conv2d& p, const void* x, const void* dy, floa
     return cudaErrorInvalidValue;
   const size_t smem = wt_smem(P);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  static std::atomic<unsigned int> configured{0};
-  const void* fn = p.dtype == GCONV_BF16 ? (const void*)wgrad_tc_kernel<__nv_bfloat16>
-                                         : (const void*)wgrad_tc_kernel<__half>;
-  cudaError_t e = set_max_dynamic_smem(fn, 227 * 1024, configured);
+  // one flag per instantiation: each kernel's shared-memory limit is raised separately
+  static std::atomic<unsigned int> configured_bf16{0}, configured_f16{0};
+  const bool bf16 = p.dtype == GCONV_BF16;
+  const void* fn = bf16 ? (const void*)wgrad_tc_kernel<__nv_bfloat16>
+                        : (const void*)wgrad_tc_kernel<__half>;
+  cudaError_t e = set_max_dynamic_smem(fn, 227 * 1024, bf16 ? configured_bf16 : configured_f16);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)(P.units * P.S);
   if (p.dtype == GCONV_BF16)

@@ -138,9 +138,12 @@ typedef enum {
   GCONV_KERNEL_CONV1D_STRIP = 20,     /* dwconv1d: CUDA-core kernel on 128-byte input rows
                                          (64-channel tiles, taps in registers); 16-bit,
                                          C % 64 == 0, K in {3, 5, 7, 9, 15, 31} */
-  GCONV_KERNEL_DWSEP2D_FUSED = 21     /* 2-D depthwise-separable block in one kernel: 16-bit
+  GCONV_KERNEL_DWSEP2D_FUSED = 21,    /* 2-D depthwise-separable block in one kernel: 16-bit
                                          NHWC, depthwise 3x3 / 5x5, stride 1 / 2, dilation 1,
                                          C % 64 == 0, C_out % 16 == 0 and <= 512 */
+  GCONV_KERNEL_DGRAD_DW3S2_TMA = 22   /* conv2d data gradient, depthwise 3x3, stride 2, pad 1,
+                                         dilation 1, 16-bit NHWC, C % 8 == 0: dy staged by TMA,
+                                         dx written by TMA stores */
 } gconv_kernel;
 
 /* Order and merging of the output channels ("Grouped convolutions", neon issue #296, ibmua's
@@ -256,8 +259,9 @@ size_t gconv2d_bwd_data_workspace_size(int N, int C_in, int H, int W, int C_out,
  * pad <= dilation*(k-1) it is computed as the forward convolution of dy with the per-group
  * transposed, 180-degree-rotated filter and pad' = dilation*(k-1) - pad, on the forward
  * kernels (AUTO / DIRECT / IGEMM choose among them as gconv2d_fwd_path does, F32 under AUTO
- * excepted). Under AUTO / DIRECT, depthwise NHWC problems that do not run that way (stride 2,
- * larger pads) take a vectorised depthwise gather kernel (GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC);
+ * excepted). Under AUTO / DIRECT, depthwise NHWC problems that do not run that way take the
+ * TMA-staged kernel for 3x3, stride 2, pad 1 (GCONV_KERNEL_DGRAD_DW3S2_TMA; dy and dx 16-byte
+ * aligned), else a vectorised depthwise gather kernel (GCONV_KERNEL_DGRAD_DEPTHWISE_NHWC);
  * other problems, fp32 under AUTO and GENERIC run the one-thread-per-element gather kernel. IGEMM on a problem that cannot run as a forward convolution on the tensor
  * cores is UNSUPPORTED (or MISALIGNED). The workspace must be 16-byte aligned.
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */

@@ -195,9 +195,11 @@ def test_bwd_path_selection(lib):
         return fn(N, C_in, H, W, C_out, k, k, s, pad, d, g, layout, dtype, path)
     dg, wg = lib.gconv2d_bwd_data_select_path, lib.gconv2d_bwd_weight_select_path
     # depthwise 56x56x1024: stride 1 runs the depthwise forward kernel on the flipped filter,
-    # stride 2 the gather kernel; the weight gradient has its own depthwise kernel
+    # stride 2 (pad 1) the TMA-staged upsampling kernel, stride 2 with pad 2 the gather
+    # kernel; the weight gradient has its own depthwise kernel
     assert sel(dg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 1024) == 2
-    assert sel(dg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 12
+    assert sel(dg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 22
+    assert sel(dg, 32, 1024, 56, 56, 1024, 3, 2, 2, 1, 1024) == 12
     assert sel(wg, 32, 1024, 56, 56, 1024, 3, 1, 1, 1, 1024) == 14
     assert sel(wg, 32, 1024, 56, 56, 1024, 3, 2, 1, 1, 1024) == 14
     assert sel(wg, 32, 1024, 56, 56, 1024, 3, 1, 3, 1, 1024) == 11   # pad 3: LDG kernel
@@ -343,3 +345,48 @@ def test_binding_signatures_match_the_header(lib):
         argtypes = getattr(lib, name).argtypes
         assert argtypes is not None, f"{name} has no argtypes"
         assert len(argtypes) == counts[name], (name, len(argtypes), counts[name])
+
+
+def test_new_entry_points_validate_before_launch(lib):
+    """The output-variant, depthwise-separable and test-hook entry points reject bad
+    arguments on the host, with nothing launched (no GPU is touched here)."""
+    P = None
+    # gconv2d_fwd_out: bad mode, null pointers with N > 0, groups not dividing C
+    assert lib.gconv2d_fwd_out(P, P, P, P, 1, 8, 8, 8, 8, 3, 3, 1, 1, 1, 2, 1, 2, 4, 0, P, 0,
+                               P) == 1
+    assert lib.gconv2d_fwd_out(P, P, P, P, 1, 8, 8, 8, 8, 3, 3, 1, 1, 1, 2, 1, 2, 1, 0, P, 0,
+                               P) == 1
+    assert lib.gconv2d_fwd_out(P, P, P, P, 0, 8, 8, 8, 8, 3, 3, 1, 1, 1, 2, 1, 2, 2, 0, P, 0,
+                               P) == 0   # empty batch: a no-op
+    assert lib.gconv2d_fwd_out(P, P, P, P, 1, 6, 8, 8, 8, 3, 3, 1, 1, 1, 4, 1, 2, 2, 0, P, 0,
+                               P) == 1
+    # variant selection: tensor cores for 16-bit problems the implicit GEMM takes, the generic
+    # kernel otherwise; modes equal to the plain output take the ordinary kernels
+    sel = lib.gconv2d_fwd_out_select_path
+    assert sel(1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 1, 2, 1, 0) == 3
+    assert sel(1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 0, 2, 2, 0) == 4
+    assert sel(1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 1, 0, 3, 0) == 1    # fp32
+    assert sel(1, 512, 256, 256, 512, 3, 3, 1, 1, 1, 4, 1, 2, 2, 1) == 1    # DIRECT: generic
+    assert sel(32, 1024, 56, 56, 1024, 3, 3, 1, 1, 1, 1024, 1, 2, 1, 0) == 2  # depthwise
+    assert sel(1, 12, 9, 9, 12, 3, 3, 1, 1, 1, 4, 1, 2, 2, 2) == -2         # IGEMM: 3 ch/group
+    # depthwise-separable blocks
+    assert lib.dwsep1d_select_path(8, 2048, 512, 31, 15, 15, 512, 2, 0) == 16
+    assert lib.dwsep1d_select_path(8, 2048, 512, 31, 15, 15, 1024, 2, 0) == 17  # C_out > 512
+    assert lib.dwsep1d_select_path(8, 2048, 512, 31, 15, 15, 1024, 2, 2) == -2
+    assert lib.dwsep1d_select_path(8, 2048, 512, 31, 15, 15, 0, 2, 0) == -1     # C_out < 1
+    assert lib.dwsep1d_fwd_workspace_size(8, 2048, 512, 31, 15, 15, 512, 2, 0) == 0
+    assert lib.dwsep1d_fwd_workspace_size(8, 2048, 512, 31, 15, 15, 512, 2, 1) == \
+        8 * 2048 * 512 * 2
+    assert lib.dwsep1d_fwd(P, P, P, P, P, 2, 64, 64, 31, 15, 15, 64, 2, 0, P, 0, P) == 1
+    assert lib.dwsep1d_fwd(P, P, P, P, P, 0, 64, 64, 31, 15, 15, 64, 2, 1, P, 0, P) == 0
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the missing workspace is found first
+    assert lib.dwsep1d_fwd(fake, fake, fake, P, fake, 2, 64, 64, 31, 15, 15, 64, 2, 1, P, 0,
+                           P) == 4
+    assert lib.dwsep2d_select_path(8, 256, 512, 40, 3, 3, 2, 1, 1, 256, 1, 2, 0) == 21
+    assert lib.dwsep2d_select_path(8, 256, 512, 40, 3, 3, 2, 1, 1, 256, 0, 2, 0) == 17   # NCHW
+    assert lib.dwsep2d_select_path(8, 256, 512, 40, 7, 7, 2, 3, 1, 256, 1, 2, 2) == -2
+    assert lib.dwsep2d_fwd(P, P, P, P, P, 1, 64, 8, 8, 3, 3, 1, 1, 1, 64, 1, 2, 0, P, 0, P) == 1
+    # the bounded-wait test hook takes 16-byte multiples up to 64 KiB, and 0 restores
+    assert lib.gconv_debug_set_tx_surplus(24) == 1
+    assert lib.gconv_debug_set_tx_surplus(1 << 20) == 1
+    assert lib.gconv_debug_set_tx_surplus(0) == 0

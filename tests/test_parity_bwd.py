@@ -66,7 +66,7 @@ def oracle_wgrad(p, inp, dy):
 CASES = [
     # N, C_in, H, W, C_out, kH, kW, stride, pad, dil, groups
     ((2, 64, 12, 12, 64, 3, 3, 1, 1, 1, 64), 2, 14),       # depthwise 3x3 s1
-    ((2, 64, 13, 11, 64, 3, 3, 2, 1, 1, 64), 12, 14),      # depthwise 3x3 s2, ragged
+    ((2, 64, 13, 11, 64, 3, 3, 2, 1, 1, 64), 22, 14),      # depthwise 3x3 s2, ragged
     ((1, 32, 14, 9, 32, 5, 5, 1, 2, 1, 32), 2, 11),        # depthwise 5x5
     ((1, 32, 15, 16, 32, 5, 5, 2, 2, 1, 32), 12, 11),      # depthwise 5x5 s2
     ((2, 48, 10, 9, 48, 3, 3, 1, 0, 1, 48), 2, 14),        # depthwise, no padding (pad' = 2)
@@ -85,7 +85,9 @@ CASES = [
     ((2, 64, 11, 13, 64, 3, 3, 2, 1, 1, 1), 9, 13),        # tiled weight gradient, stride 2
     ((1, 160, 6, 7, 320, 3, 3, 1, 1, 1, 1), 3, 13),        # 160 -> 320: 3 x 2 tiles, ragged
     ((2, 72, 30, 31, 72, 3, 3, 1, 1, 1, 72), 2, 14),       # C % 64 != 0, Wo > 28 (2 column tiles)
-    ((1, 40, 31, 30, 40, 3, 3, 2, 1, 1, 40), 12, 14),      # s2, odd sizes, ragged tiles
+    ((1, 40, 31, 30, 40, 3, 3, 2, 1, 1, 40), 22, 14),      # s2, odd sizes, ragged tiles
+    ((2, 72, 18, 60, 72, 3, 3, 2, 1, 1, 72), 22, 14),      # s2: 3 column tiles, 2 channel tiles
+    ((1, 64, 16, 16, 64, 3, 3, 2, 2, 1, 64), 12, 14),      # s2 with pad 2: gather kernel
     ((1, 16, 10, 10, 16, 3, 3, 1, 2, 1, 16), 2, 14),       # pad 2 (dgrad pad' = 0)
 ]
 
@@ -261,7 +263,7 @@ TC_WGRAD_CASES = [
     (2, 128, 8, 36, 128, 3, 3, 1, 2, 2, 1),       # dilation 2
     (1, 64, 9, 48, 128, 1, 1, 1, 0, 1, 1),        # 1x1
     (1, 128, 7, 33, 128, 3, 1, 1, 1, 1, 1),       # 3x1
-    (3, 256, 4, 32, 512, 3, 3, 1, 0, 1, 4),       # 4 groups, no padding
+    (3, 256, 4, 34, 512, 3, 3, 1, 0, 1, 4),       # 4 groups, no padding (Wo = 32)
 ]
 
 
