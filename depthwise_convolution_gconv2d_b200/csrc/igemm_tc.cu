@@ -1013,6 +1013,11 @@ struct RowTParams {
   unsigned int idesc, tmem_cols;
   int out_nchw, nchw_vec;
   int groups, interleave;   // interleaved output order: filter f of group j -> f * groups + j
+  // average merge across groups: every group's K loop accumulates into one tile (jgroups =
+  // groups, tiles have no group index), the epilogue scales by 1/groups and writes out_c =
+  // C_out/groups channels; otherwise jgroups = 1, out_c = C_out, scale = 1
+  int jgroups, out_c;
+  float scale;
 };
 
 __device__ __forceinline__ void rowt_decode(const RowTParams& P, int t, int& j, int& nt, int& n,
@@ -1090,9 +1095,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int j, nt, n, ho, seg;
         rowt_decode(P, t, j, nt, n, ho, seg);
         const int wbase = seg * P.NPIX - P.pad;
-        const int obase = j * P.cpg_out + nt * BM;
+        for (int jj = 0; jj < P.jgroups && ok; ++jj) {
+        const int jx = P.jgroups > 1 ? jj : j;
+        const int obase = jx * P.cpg_out + nt * BM;
         for (int cb = 0; cb < P.cblocks && ok; ++cb) {
-          const int cin = j * P.cpg_in + cb * 64;
+          const int cin = jx * P.cpg_in + cb * 64;
           for (int kh = 0; kh < P.kH && ok; ++kh) {
             if (!mbar_wait(&ex[sx], px ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
               ok = false;
@@ -1124,6 +1131,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
+        }
       }
       const unsigned long long dl = drain_deadline();
       for (long long q = (nx > P.x_stages ? nx - P.x_stages : 0); q < nx; ++q)
@@ -1146,6 +1154,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERR_WAIT_MMA)) break;
         tc_fence_after();
         const unsigned int d = tmem_base + (unsigned int)(acc * P.NPIX);
+        for (int jj = 0; jj < P.jgroups && ok; ++jj) {
         for (int cb = 0; cb < P.cblocks && ok; ++cb) {
           for (int kh = 0; kh < P.kH && ok; ++kh) {
             if (!mbar_try_wait(&fx[sx], px) &&
@@ -1162,7 +1171,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
               const unsigned long long wd = w_desc0 + (((unsigned long long)sw * P.w_stage) >> 4);
               const unsigned long long xd = xs + kw * kw_step;
-              const unsigned int acc0 = (cb | kh | kw) == 0 ? 0u : 1u;
+              const unsigned int acc0 = (jj | cb | kh | kw) == 0 ? 0u : 1u;
               umma_f16(d, wd, xd, P.idesc, acc0);
               umma_f16(d, wd + 2, xd + 2, P.idesc, 1u);
               umma_f16(d, wd + 4, xd + 4, P.idesc, 1u);
@@ -1180,6 +1189,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               px ^= 1u;
             }
           }
+        }
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
@@ -1204,8 +1214,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const int co_g = j * P.cpg_out + nt * BM + co_l;       // group-major channel
-      const int co = P.interleave ? (nt * BM + co_l) * P.groups + j : co_g;   // y's channel
-      const float bv = bias ? Elem<T>::to_f32(bias[co_g]) : 0.0f;
+      // y's channel: interleaved position, merged channel, or the group-major one
+      const int co = P.interleave ? (nt * BM + co_l) * P.groups + j
+                                  : (P.jgroups > 1 ? nt * BM + co_l : co_g);
+      float bv = 0.0f;
+      if (bias) {
+        if (P.jgroups > 1) {
+          for (int i = 0; i < P.jgroups; ++i)
+            bv += Elem<T>::to_f32(bias[i * P.cpg_out + nt * BM + co_l]);
+          bv *= P.scale;
+        } else {
+          bv = Elem<T>::to_f32(bias[co_g]);
+        }
+      }
+      const float sc = P.scale;
       const unsigned int taddr =
           tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.NPIX);
       for (int c = 0; c < P.NPIX; c += 32) {
@@ -1215,31 +1237,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int wo0 = seg * P.NPIX + c;
         if (wo0 >= P.Wo) continue;
         if (!P.out_nchw) {
-          T* dst = y + (((long long)n * P.Ho + ho) * P.Wo + wo0) * P.C_out + co;
+          T* dst = y + (((long long)n * P.Ho + ho) * P.Wo + wo0) * P.out_c + co;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (wo0 + i < P.Wo)
-              dst[(long long)i * P.C_out] = Elem<T>::from_f32(__uint_as_float(r[i]) + bv);
+              dst[(long long)i * P.out_c] = Elem<T>::from_f32(fmaf(__uint_as_float(r[i]), sc, bv));
         } else {
-          T* dst = y + (((long long)n * P.C_out + co) * P.Ho + ho) * P.Wo + wo0;
+          T* dst = y + (((long long)n * P.out_c + co) * P.Ho + ho) * P.Wo + wo0;
           if (P.nchw_vec && wo0 + 32 <= P.Wo) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               uint4 u;
-              u.x = pack2<T>(make_float2(__uint_as_float(r[8 * q + 0]) + bv,
-                                         __uint_as_float(r[8 * q + 1]) + bv));
-              u.y = pack2<T>(make_float2(__uint_as_float(r[8 * q + 2]) + bv,
-                                         __uint_as_float(r[8 * q + 3]) + bv));
-              u.z = pack2<T>(make_float2(__uint_as_float(r[8 * q + 4]) + bv,
-                                         __uint_as_float(r[8 * q + 5]) + bv));
-              u.w = pack2<T>(make_float2(__uint_as_float(r[8 * q + 6]) + bv,
-                                         __uint_as_float(r[8 * q + 7]) + bv));
+              u.x = pack2<T>(make_float2(fmaf(__uint_as_float(r[8 * q + 0]), sc, bv),
+                                         fmaf(__uint_as_float(r[8 * q + 1]), sc, bv)));
+              u.y = pack2<T>(make_float2(fmaf(__uint_as_float(r[8 * q + 2]), sc, bv),
+                                         fmaf(__uint_as_float(r[8 * q + 3]), sc, bv)));
+              u.z = pack2<T>(make_float2(fmaf(__uint_as_float(r[8 * q + 4]), sc, bv),
+                                         fmaf(__uint_as_float(r[8 * q + 5]), sc, bv)));
+              u.w = pack2<T>(make_float2(fmaf(__uint_as_float(r[8 * q + 6]), sc, bv),
+                                         fmaf(__uint_as_float(r[8 * q + 7]), sc, bv)));
               reinterpret_cast<uint4*>(dst)[q] = u;
             }
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if (wo0 + i < P.Wo) dst[i] = Elem<T>::from_f32(__uint_as_float(r[i]) + bv);
+              if (wo0 + i < P.Wo) dst[i] = Elem<T>::from_f32(fmaf(__uint_as_float(r[i]), sc, bv));
           }
         }
       }
@@ -1325,6 +1347,25 @@ __global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const T* __restrict__
         if (c < C && sp < HW) tn[(long long)sp * C + c] = tile[tx + 32 * h][ty + 8 * r];
       }
     }
+  }
+}
+
+// w[co][ci][kh][kw] -> wt[co][kh][kw][ci] for filters of at most 8192 elements: one CTA per
+// filter reads it with coalesced loads into shared memory and writes it back tap-major with
+// coalesced stores.
+template <typename T>
+__global__ void __launch_bounds__(256) repack_weight_smem_kernel(const T* __restrict__ w,
+                                                                 T* __restrict__ wt, int cpg_in,
+                                                                 int taps) {
+  __shared__ unsigned short buf[8192];
+  const int n = cpg_in * taps;
+  const unsigned short* src = reinterpret_cast<const unsigned short*>(w) + (long long)blockIdx.x * n;
+  unsigned short* dst = reinterpret_cast<unsigned short*>(wt) + (long long)blockIdx.x * n;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) buf[i] = src[i];
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int tap = i / cpg_in, ci = i - tap * cpg_in;
+    dst[i] = buf[ci * taps + tap];
   }
 }
 
@@ -1527,7 +1568,7 @@ cudaError_t launch_row(const Conv2d& p, const RowParams& R, const void* x, const
 
 // Transposed row kernel parameters; false if the problem does not take it.
 bool make_rowt_params(const Conv2d& p, RowTParams* R) {
-  if (p.out_mode != GCONV_OUT_GROUP_MAJOR && p.out_mode != GCONV_OUT_INTERLEAVED) return false;
+  if (p.out_mode == GCONV_OUT_MERGE_MAX) return false;
   if (p.Wo < BM || p.cpg_in % 64 != 0 || p.cpg_out % BM != 0) return false;
   if ((p.kW - 1) * p.dil > 8) return false;            // halo fits the 8-row second box
   R->N = p.N; R->H = p.H; R->W = p.W; R->C_in = p.C_in; R->C_out = p.C_out;
@@ -1564,6 +1605,11 @@ bool make_rowt_params(const Conv2d& p, RowTParams* R) {
   R->nchw_vec = (p.Wo % 8 == 0) ? 1 : 0;
   R->groups = p.groups;
   R->interleave = p.out_mode == GCONV_OUT_INTERLEAVED;
+  const bool avg = p.out_mode == GCONV_OUT_MERGE_AVG;
+  R->jgroups = avg ? p.groups : 1;
+  R->out_c = out_channels(p);
+  R->scale = avg ? 1.0f / (float)p.groups : 1.0f;
+  if (avg) R->num_tiles /= p.groups;   // one tile covers every group's K loop
   return true;
 }
 
@@ -1898,8 +1944,14 @@ cudaError_t launch_nchw_typed(const Conv2d& p, const IgemmParams& P, const void*
   T* wt = (T*)((char*)workspace + align256((size_t)p.N * p.H * p.W * p.C_in * 2));
   const int taps = p.kH * p.kW;
   const int per_filter = p.cpg_in * taps;
-  dim3 wgrid((unsigned)((per_filter + 255) / 256), (unsigned)(p.C_out < 65535 ? p.C_out : 65535));
-  repack_weight_kernel<T><<<wgrid, 256, 0, s>>>((const T*)w, wt, p.C_out, p.cpg_in, taps);
+  if (per_filter <= 8192) {
+    repack_weight_smem_kernel<T><<<(unsigned)p.C_out, 256, 0, s>>>((const T*)w, wt, p.cpg_in,
+                                                                   taps);
+  } else {
+    dim3 wgrid((unsigned)((per_filter + 255) / 256),
+               (unsigned)(p.C_out < 65535 ? p.C_out : 65535));
+    repack_weight_kernel<T><<<wgrid, 256, 0, s>>>((const T*)w, wt, p.C_out, p.cpg_in, taps);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int HW = p.H * p.W;

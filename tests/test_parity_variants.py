@@ -76,14 +76,18 @@ def test_variants_fp16(mode):
     assert_close(to_f64(run_out(inp, mode)), oracle_out(inp, mode), p.dtype, mode)
 
 
-def test_interleaved_row_strip_kernel():
+@pytest.mark.parametrize("mode", ["interleaved", "avg"])
+def test_row_strip_kernel_variants(mode):
     """Rows of >= 128 outputs with 128k filters per group take the transposed row-strip
-    kernel, whose epilogue writes each filter to its interleaved channel."""
+    kernel: its epilogue writes each filter to its interleaved channel, and for the average
+    merge one tile runs every group's K loop into one accumulator and scales it by 1/groups."""
     for layout in (wl.NHWC, wl.NCHW):
-        p = wl.Conv2dProblem(1, 256, 4, 160, 256, 3, 3, 1, 1, 1, 2, layout, wl.BF16, bias=True)
-        inp = wl.make_conv2d_inputs(p, 33)
-        assert_close(to_f64(run_out(inp, "interleaved")), oracle_out(inp, "interleaved"),
-                     p.dtype, f"layout {layout}")
+        for g in (2, 4):
+            p = wl.Conv2dProblem(1, 128 * g, 4, 160, 128 * g, 3, 3, 1, 1, 1, g, layout, wl.BF16,
+                                 bias=True)
+            inp = wl.make_conv2d_inputs(p, 33)
+            assert_close(to_f64(run_out(inp, mode)), oracle_out(inp, mode), p.dtype,
+                         f"layout {layout} groups {g}")
 
 
 GENERIC_CASES = [
