@@ -432,9 +432,17 @@ def dwsep_measurements(torch, gb, device, stream, pk, reps):
                                           (pk["bf16_tflops"] * 1e12), 3),
                      "alg_bytes": nbytes, "alg_flops": flops}
         del ws
-    # the strided 2-D block of a Fast Conformer downsampler: x[8, 512, 40, 256] NHWC
-    # (frames x frequency bins), depthwise 3x3 stride 2 pad 1, then pointwise 256 -> 256
-    N, H, W, C, k, st, pad, Co = 8, 512, 40, 256, 3, 2, 1, 256
+    # strided 2-D blocks: a Fast Conformer downsampler layer, x[8, 512, 40, 256] NHWC (frames x
+    # frequency bins; 20 output columns, narrower than the fused kernel's 32-column tiles, so
+    # AUTO runs the two launches there), and the same layer on 128 bins (64 output columns)
+    for tag, W in (("", 40), ("_w128", 128)):
+        out.update(dwsep2d_measurement(torch, gb, device, stream, pk, reps, flush, W, tag))
+    return out
+
+
+def dwsep2d_measurement(torch, gb, device, stream, pk, reps, flush, W, tag):
+    out = {}
+    N, H, C, k, st, pad, Co = 8, 512, 256, 3, 2, 1, 256
     p2 = wl.Dwconv1dProblem(N, H * W, C, k * k, 0, 0, wl.BF16)
     inp2 = wl.make_dwsep1d_inputs(p2, Co, 8)
     x2 = dev_tensor(torch, inp2.x.reshape(N, H, W, C), wl.BF16, device)
@@ -444,7 +452,8 @@ def dwsep_measurements(torch, gb, device, stream, pk, reps):
     z2 = torch.empty((N, Ho, Wo, Co), dtype=torch.bfloat16, device=device)
     nbytes2 = (x2.numel() + wdw2.numel() + wpw2.numel() + b2.numel() + z2.numel()) * 2
     flops2 = 2 * N * Ho * Wo * C * (k * k + Co)
-    for name, path in (("dwsep2d_fused", gb.PATH_AUTO), ("dwsep2d_two_launches", gb.PATH_DIRECT)):
+    for name, path in ((f"dwsep2d{tag}_auto", gb.PATH_AUTO),
+                       (f"dwsep2d{tag}_two_launches", gb.PATH_DIRECT)):
         kname = gb.KERNEL_NAMES.get(gb.dwsep2d_select_path(N, C, H, W, k, k, st, pad, 1, Co,
                                                            "NHWC", wl.BF16, path))
         need = gb.load_library().dwsep2d_fwd_workspace_size(N, C, H, W, k, k, st, pad, 1, Co,

@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(SP_THREADS, 2)
   unsigned char* smem = align_smem(smem_raw, 1024u);
   unsigned char* ring = smem;
   unsigned char* slabs = smem + SP_STAGES * P.stage_bytes;        // 7 warps x 2 x 2 KB
-  unsigned long long* bars = reinterpret_cast<unsigned long long*>(slabs + SP_WARPS * 4096);
+  float2* wsm = reinterpret_cast<float2*>(slabs + SP_WARPS * 4096);  // taps [K][32 pairs]
+  unsigned long long* bars = reinterpret_cast<unsigned long long*>(wsm + K * 32);
   unsigned long long* full = bars;
   unsigned long long* empty = full + SP_STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + SP_STAGES);
@@ -94,6 +95,17 @@ __global__ void __launch_bounds__(SP_THREADS, 2)
     fence_mbar_init();
     prefetch_tmap(&tmx);
     prefetch_tmap(&tmy);
+  }
+  // the block's taps, read once with coalesced loads and kept as fp32 pairs [tap][pair]
+  // (reversed for the data gradient), so a lane's K pairs are conflict-free 8-byte loads
+  {
+    const T* wb = w + (long long)run.cb * SP_CB * K;
+    float* wf = reinterpret_cast<float*>(wsm);
+    for (int e = threadIdx.x; e < SP_CB * K; e += SP_THREADS) {
+      const int c = e / K, k = e - c * K;
+      const int kk = FLIP ? K - 1 - k : k;
+      wf[(kk * 32 + (c >> 1)) * 2 + (c & 1)] = Elem<T>::to_f32(wb[e]);
+    }
   }
   __syncthreads();
 
@@ -123,14 +135,8 @@ __global__ void __launch_bounds__(SP_THREADS, 2)
     const int w2 = warp - 1;
     // the taps of this lane's channel pair, fp32 pairs (reversed for the data gradient)
     float2 wk[K];
-    {
-      const T* w0 = w + (long long)(run.cb * SP_CB + 2 * lane) * K;
 #pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int kk = FLIP ? K - 1 - k : k;
-        wk[k] = make_float2(Elem<T>::to_f32(w0[kk]), Elem<T>::to_f32(w0[K + kk]));
-      }
-    }
+    for (int k = 0; k < K; ++k) wk[k] = wsm[k * 32 + lane];
     unsigned char* slab0 = slabs + w2 * 4096;
     int s = 0;
     unsigned int ph = 0;
@@ -301,19 +307,32 @@ __global__ void __launch_bounds__(SP_THREADS, 2)
   }
 }
 
-// dw[c][k] = sum over runs r (in order) of part[cb][r][c - 64 cb][k], rounded once.
+// dw[c][k] = sum over runs r of part[cb][r][c - 64 cb][k], rounded once. A CTA takes 32
+// consecutive dw entries (one per lane: coalesced loads) and its 8 warps split the runs (warp
+// j adds runs j, j+8, ... in that order); the 8 warp sums are then added in warp order -- a
+// fixed order, so the result is bitwise reproducible.
 template <typename T>
 __global__ void __launch_bounds__(256) dwconv1d_wgrad_strip_sum(const float* __restrict__ part,
                                                                 T* __restrict__ dw, int C, int K,
                                                                 int runs) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= C * K) return;
-  const int c = e / K, k = e - c * K;
-  const int cb = c / SP_CB, cl = c - cb * SP_CB;
-  const float* p = part + ((long long)cb * runs * SP_CB + cl) * K + k;
+  __shared__ float acc8[8][33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
   float v = 0.0f;
-  for (int r = 0; r < runs; ++r) v += p[(long long)r * SP_CB * K];
-  dw[e] = Elem<T>::from_f32(v);
+  if (e < C * K) {
+    const int c = e / K, k = e - c * K;
+    const int cb = c / SP_CB, cl = c - cb * SP_CB;
+    const float* p = part + ((long long)cb * runs * SP_CB + cl) * K + k;
+    for (int r = warp; r < runs; r += 8) v += p[(long long)r * SP_CB * K];
+  }
+  acc8[warp][lane] = v;
+  __syncthreads();
+  if (warp == 0 && e < C * K) {
+    float t = acc8[0][lane];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) t += acc8[j][lane];
+    dw[e] = Elem<T>::from_f32(t);
+  }
 }
 
 bool sp_k_supported(int K) {
@@ -340,8 +359,9 @@ bool make_sp_params(const Conv1d& p, int T_in, int T_out, int pl, bool wgrad, Sp
   return true;
 }
 
-size_t sp_smem(const SpParams& P, bool wgrad) {
-  return 1024 + SP_STAGES * (size_t)P.stage_bytes + (wgrad ? 0 : SP_WARPS * 4096) + 64;
+size_t sp_smem(const SpParams& P, int K, bool wgrad) {
+  return 1024 + SP_STAGES * (size_t)P.stage_bytes +
+         (wgrad ? 0 : SP_WARPS * 4096 + (size_t)K * 32 * 8) + 64;
 }
 
 bool encode_rows(EncodeTiledFn enc, CUtensorMap* m, int dtype, const void* base, int C, int T,
@@ -363,7 +383,7 @@ template <typename T, int K>
 cudaError_t launch_fwd_k(const SpParams& P, const CUtensorMap& tx, const CUtensorMap& ty,
                          const void* w, bool flip, cudaStream_t s) {
   static std::atomic<unsigned int> conf0{0}, conf1{0};
-  const size_t smem = sp_smem(P, false);
+  const size_t smem = sp_smem(P, K, false);
   const void* fn = flip ? (const void*)dwconv1d_strip_kernel<T, K, true>
                         : (const void*)dwconv1d_strip_kernel<T, K, false>;
   cudaError_t e = set_max_dynamic_smem(fn, smem, flip ? conf1 : conf0);
@@ -382,7 +402,7 @@ template <typename T, int K>
 cudaError_t launch_wgrad_k(const SpParams& P, const CUtensorMap& tx, const CUtensorMap& td,
                            float* part, void* dw, cudaStream_t s) {
   static std::atomic<unsigned int> conf{0};
-  const size_t smem = sp_smem(P, true);
+  const size_t smem = sp_smem(P, K, true);
   cudaError_t e = set_max_dynamic_smem((const void*)dwconv1d_wgrad_strip_kernel<T, K>, smem, conf);
   if (e != cudaSuccess) return e;
   dwconv1d_wgrad_strip_kernel<T, K><<<(unsigned)(P.n_cb * P.runs), SP_THREADS, smem, s>>>(
@@ -390,7 +410,7 @@ cudaError_t launch_wgrad_k(const SpParams& P, const CUtensorMap& tx, const CUten
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int E = P.C * K;
-  dwconv1d_wgrad_strip_sum<T><<<(E + 255) / 256, 256, 0, s>>>(part, (T*)dw, P.C, K, P.runs);
+  dwconv1d_wgrad_strip_sum<T><<<(E + 31) / 32, 256, 0, s>>>(part, (T*)dw, P.C, K, P.runs);
   return cudaGetLastError();
 }
 

@@ -34,7 +34,9 @@ using namespace ptx;
 
 constexpr int DS_M = 128;            // output steps per CTA (MMA M)
 constexpr int DS_CB = 64;            // input channels per block (MMA K per block)
-constexpr int DS_THREADS = 320;      // warp 0 TMA, warp 1 MMA, warps 2-9 depthwise (+2-5 epilogue)
+// warp 0 TMA, warp 1 MMA, warps 2-17 depthwise in two groups of 8 that take alternate channel
+// blocks (two blocks' depthwise in flight), warps 2-5 also the epilogue
+constexpr int DS_THREADS = 576;
 constexpr int DS_XS = 2;             // input-block stages
 constexpr int DS_AS = 2;             // A-operand stages
 constexpr int DS_BS = 2;             // B-operand stages
@@ -202,11 +204,12 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
       mbar_wait_until(done, 0, drain_deadline(), err, ERR_DRAIN);
     }
   } else {
-    // ---------------- depthwise: warp w2 = warp - 2 owns output steps [16 w2, 16 w2 + 16) of
-    // the tile, lane = channel pair (channels 2 lane, 2 lane + 1 of the block)
-    const int w2 = warp - 2;
+    // ---------------- depthwise: group dg takes channel blocks dg, dg + 2, ...; its warp w2
+    // owns output steps [16 w2, 16 w2 + 16) of the tile, lane = channel pair (channels
+    // 2 lane, 2 lane + 1 of the block)
+    const int dg = (warp - 2) >> 3, w2 = (warp - 2) & 7;
     bool ok = true;
-    for (int cb = 0; cb < P.cblocks; ++cb) {
+    for (int cb = dg; cb < P.cblocks; cb += 2) {
       const int xs = cb % DS_XS, as = cb % DS_AS;
       const bool gx = mbar_wait(&x_full[xs], (unsigned int)(cb / DS_XS) & 1u, abort_flag, err,
                                 ERR_DS | 8u);
@@ -473,13 +476,14 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
       mbar_wait_until(done, 0, drain_deadline(), err, ERR_DRAIN);
     }
   } else {
-    // ---------------- depthwise: warp w2 owns tile pixels 16 w2 .. 16 w2 + 15, i.e. tile row
-    // r = w2 / 2, columns 16 (w2 % 2) .. + 15; lane = channel pair
-    const int w2 = warp - 2;
+    // ---------------- depthwise: group dg takes channel blocks dg, dg + 2, ...; its warp w2
+    // owns tile pixels 16 w2 .. 16 w2 + 15, i.e. tile row r = w2 / 2, columns
+    // 16 (w2 % 2) .. + 15; lane = channel pair
+    const int dg = (warp - 2) >> 3, w2 = (warp - 2) & 7;
     const int r = w2 >> 1, c0 = (w2 & 1) * 16;
     const bool row_live = r < P.BH && oh0 + r < P.Ho;
     bool ok = true;
-    for (int cb = 0; cb < P.cblocks; ++cb) {
+    for (int cb = dg; cb < P.cblocks; cb += 2) {
       const int xs = cb % DS_XS, as = cb % DS_AS;
       const bool gx = mbar_wait(&x_full[xs], (unsigned int)(cb / DS_XS) & 1u, abort_flag, err,
                                 ERR_DS | 8u);
@@ -708,6 +712,9 @@ bool make_ds2_params(const Conv2d& p, int C_out, Ds2Params* P) {
   if ((p.kH != 3 && p.kH != 5) || (p.stride != 1 && p.stride != 2)) return false;
   if (p.C_in % DS_CB != 0 || C_out % 16 != 0 || C_out > DS_MAX_COUT || C_out < 16) return false;
   if (p.N > 65535 || p.H > 65535 || p.W > 65535) return false;
+  // tiles are 32 output columns wide: narrower images would leave most MMA rows and depthwise
+  // warps idle (the two-launch composition is faster there)
+  if (p.Wo < 32) return false;
   P->N = p.N; P->H = p.H; P->W = p.W; P->C = p.C_in; P->pad = p.pad; P->Ho = p.Ho;
   P->Wo = p.Wo; P->C_out = C_out;
   P->box_w = 31 * p.stride + p.kW;

@@ -1032,7 +1032,7 @@ __device__ __forceinline__ void rowt_decode(const RowTParams& P, int t, int& j, 
   j = r / P.n_tiles;
 }
 
-template <typename T>
+template <typename T, bool MERGE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     igemm_rowt_kernel(const __grid_constant__ CUtensorMap tma_x,
                       const __grid_constant__ CUtensorMap tma_xh,
@@ -1095,10 +1095,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int j, nt, n, ho, seg;
         rowt_decode(P, t, j, nt, n, ho, seg);
         const int wbase = seg * P.NPIX - P.pad;
-        for (int jj = 0; jj < P.jgroups && ok; ++jj) {
-        const int jx = P.jgroups > 1 ? jj : j;
-        const int obase = jx * P.cpg_out + nt * BM;
-        for (int cb = 0; cb < P.cblocks && ok; ++cb) {
+        // channel blocks of the tile's group; MERGE: of every group in turn (jgroups * cblocks)
+        const int nblocks = MERGE ? P.jgroups * P.cblocks : P.cblocks;
+        for (int cbg = 0; cbg < nblocks && ok; ++cbg) {
+          const int jx = MERGE ? cbg / P.cblocks : j;
+          const int cb = MERGE ? cbg - jx * P.cblocks : cbg;
+          const int obase = jx * P.cpg_out + nt * BM;
           const int cin = jx * P.cpg_in + cb * 64;
           for (int kh = 0; kh < P.kH && ok; ++kh) {
             if (!mbar_wait(&ex[sx], px ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
@@ -1131,7 +1133,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        }
       }
       const unsigned long long dl = drain_deadline();
       for (long long q = (nx > P.x_stages ? nx - P.x_stages : 0); q < nx; ++q)
@@ -1154,8 +1155,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERR_WAIT_MMA)) break;
         tc_fence_after();
         const unsigned int d = tmem_base + (unsigned int)(acc * P.NPIX);
-        for (int jj = 0; jj < P.jgroups && ok; ++jj) {
-        for (int cb = 0; cb < P.cblocks && ok; ++cb) {
+        const int nblocks = MERGE ? P.jgroups * P.cblocks : P.cblocks;
+        for (int cb = 0; cb < nblocks && ok; ++cb) {
           for (int kh = 0; kh < P.kH && ok; ++kh) {
             if (!mbar_try_wait(&fx[sx], px) &&
                 !mbar_wait(&fx[sx], px, abort_flag, err, ERR_WAIT_MMA)) {
@@ -1171,7 +1172,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
               const unsigned long long wd = w_desc0 + (((unsigned long long)sw * P.w_stage) >> 4);
               const unsigned long long xd = xs + kw * kw_step;
-              const unsigned int acc0 = (jj | cb | kh | kw) == 0 ? 0u : 1u;
+              const unsigned int acc0 = (cb | kh | kw) == 0 ? 0u : 1u;
               umma_f16(d, wd, xd, P.idesc, acc0);
               umma_f16(d, wd + 2, xd + 2, P.idesc, 1u);
               umma_f16(d, wd + 4, xd + 4, P.idesc, 1u);
@@ -1189,7 +1190,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               px ^= 1u;
             }
           }
-        }
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
@@ -1216,10 +1216,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int co_g = j * P.cpg_out + nt * BM + co_l;       // group-major channel
       // y's channel: interleaved position, merged channel, or the group-major one
       const int co = P.interleave ? (nt * BM + co_l) * P.groups + j
-                                  : (P.jgroups > 1 ? nt * BM + co_l : co_g);
+                                  : (MERGE ? nt * BM + co_l : co_g);
       float bv = 0.0f;
       if (bias) {
-        if (P.jgroups > 1) {
+        if (MERGE) {
           for (int i = 0; i < P.jgroups; ++i)
             bv += Elem<T>::to_f32(bias[i * P.cpg_out + nt * BM + co_l]);
           bv *= P.scale;
@@ -1227,7 +1227,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           bv = Elem<T>::to_f32(bias[co_g]);
         }
       }
-      const float sc = P.scale;
+      const float sc = P.scale;   // 1 unless MERGE
+      const int oc = MERGE ? P.out_c : P.C_out;
+      // accumulator -> output value (the merge scales by 1/groups; the plain kernel adds bias)
+      auto outv = [&](unsigned int u) {
+        return MERGE ? fmaf(__uint_as_float(u), sc, bv) : __uint_as_float(u) + bv;
+      };
       const unsigned int taddr =
           tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.NPIX);
       for (int c = 0; c < P.NPIX; c += 32) {
@@ -1237,31 +1242,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int wo0 = seg * P.NPIX + c;
         if (wo0 >= P.Wo) continue;
         if (!P.out_nchw) {
-          T* dst = y + (((long long)n * P.Ho + ho) * P.Wo + wo0) * P.out_c + co;
+          T* dst = y + (((long long)n * P.Ho + ho) * P.Wo + wo0) * oc + co;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (wo0 + i < P.Wo)
-              dst[(long long)i * P.out_c] = Elem<T>::from_f32(fmaf(__uint_as_float(r[i]), sc, bv));
+              dst[(long long)i * oc] = Elem<T>::from_f32(outv(r[i]));
         } else {
-          T* dst = y + (((long long)n * P.out_c + co) * P.Ho + ho) * P.Wo + wo0;
+          T* dst = y + (((long long)n * oc + co) * P.Ho + ho) * P.Wo + wo0;
           if (P.nchw_vec && wo0 + 32 <= P.Wo) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               uint4 u;
-              u.x = pack2<T>(make_float2(fmaf(__uint_as_float(r[8 * q + 0]), sc, bv),
-                                         fmaf(__uint_as_float(r[8 * q + 1]), sc, bv)));
-              u.y = pack2<T>(make_float2(fmaf(__uint_as_float(r[8 * q + 2]), sc, bv),
-                                         fmaf(__uint_as_float(r[8 * q + 3]), sc, bv)));
-              u.z = pack2<T>(make_float2(fmaf(__uint_as_float(r[8 * q + 4]), sc, bv),
-                                         fmaf(__uint_as_float(r[8 * q + 5]), sc, bv)));
-              u.w = pack2<T>(make_float2(fmaf(__uint_as_float(r[8 * q + 6]), sc, bv),
-                                         fmaf(__uint_as_float(r[8 * q + 7]), sc, bv)));
+              u.x = pack2<T>(make_float2(outv(r[8 * q + 0]), outv(r[8 * q + 1])));
+              u.y = pack2<T>(make_float2(outv(r[8 * q + 2]), outv(r[8 * q + 3])));
+              u.z = pack2<T>(make_float2(outv(r[8 * q + 4]), outv(r[8 * q + 5])));
+              u.w = pack2<T>(make_float2(outv(r[8 * q + 6]), outv(r[8 * q + 7])));
               reinterpret_cast<uint4*>(dst)[q] = u;
             }
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if (wo0 + i < P.Wo) dst[i] = Elem<T>::from_f32(fmaf(__uint_as_float(r[i]), sc, bv));
+              if (wo0 + i < P.Wo) dst[i] = Elem<T>::from_f32(outv(r[i]));
           }
         }
       }
@@ -1651,13 +1652,22 @@ cudaError_t launch_rowt(const Conv2d& p, const RowTParams& R, const void* x, con
     return cudaErrorInvalidValue;
   const size_t smem = rowt_smem_bytes(R);
   if (smem > SMEM_BUDGET) return cudaErrorInvalidValue;
-  static std::atomic<unsigned int> configured{0};
-  cudaError_t e = set_max_dynamic_smem((const void*)igemm_rowt_kernel<T>, SMEM_BUDGET, configured);
+  // the average merge is its own instantiation, so the plain kernel's loops stay as they were
+  static std::atomic<unsigned int> configured{0}, configured_merge{0};
+  const bool merge = R.jgroups > 1;
+  cudaError_t e = merge ? set_max_dynamic_smem((const void*)igemm_rowt_kernel<T, true>,
+                                               SMEM_BUDGET, configured_merge)
+                        : set_max_dynamic_smem((const void*)igemm_rowt_kernel<T, false>,
+                                               SMEM_BUDGET, configured);
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   if (grid > R.num_tiles) grid = R.num_tiles;
-  igemm_rowt_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, txh, tw, (const T*)bias, (T*)y, R,
-                                                       device_error_word());
+  if (merge)
+    igemm_rowt_kernel<T, true><<<grid, NUM_THREADS, smem, s>>>(tx, txh, tw, (const T*)bias,
+                                                               (T*)y, R, device_error_word());
+  else
+    igemm_rowt_kernel<T, false><<<grid, NUM_THREADS, smem, s>>>(tx, txh, tw, (const T*)bias,
+                                                                (T*)y, R, device_error_word());
   return cudaGetLastError();
 }
 

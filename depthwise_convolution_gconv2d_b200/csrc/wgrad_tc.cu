@@ -239,7 +239,9 @@ bool make_wt_params(const Conv2d& p, WtParams* P) {
   if (blocks > INT32_MAX || units > INT32_MAX) return false;
   P->blocks = (int)blocks;
   P->units = (int)units;
-  long long S = (WT_TARGET_CTAS + units - 1) / units;
+  // as many slices as fill one wave of 148 CTAs without starting a second (a partial second
+  // wave would double the time of the slowest CTA)
+  long long S = WT_TARGET_CTAS / units;
   if (S > blocks) S = blocks;
   if (S < 1) S = 1;
   if (units * S > INT32_MAX) return false;

@@ -118,20 +118,21 @@ def test_wgrad_workspace_query(lib):
 
 
 def test_conv1d_path_selection(lib):
-    """dwconv1d_select_path: the 128-byte-row CUDA-core kernel (20) for 16-bit data with
-    C % 64 == 0 and an instantiated K, else the tensor-core kernel (7) for C % 16 == 0 and
-    K <= 49, else the CUDA-core ring kernel (6) where it is instantiated, else the generic
-    kernel (5); a forced family that cannot run gives -UNSUPPORTED."""
+    """dwconv1d_select_path: the tensor-core kernel (7) for 16-bit data with C % 16 == 0 and
+    K <= 49, else the 128-byte-row CUDA-core kernel (20) for C % 64 == 0 and an instantiated
+    K, else the CUDA-core ring kernel (6) where it is instantiated, else the generic kernel
+    (5); DIRECT takes the 128-byte-row kernel first; a forced family that cannot run gives
+    -UNSUPPORTED."""
     BF16, F32 = 2, 0
     sel = lambda B, T, C, K, pl, pr, dt, path: lib.dwconv1d_select_path(B, T, C, K, pl, pr, dt,
                                                                         path)
     conformer = (8, 2048, 512, 31, 15, 15, BF16)
-    assert sel(*conformer, 0) == 20
+    assert sel(*conformer, 0) == 7
     assert sel(*conformer, 1) == 20
     assert sel(*conformer, 2) == 7
     assert sel(*conformer, 3) == 5
-    assert sel(8, 2048, 512, 33, 16, 16, BF16, 0) == 7          # K = 33: no strip instantiation
-    assert sel(8, 2048, 96, 31, 15, 15, BF16, 0) == 7           # C % 64 != 0
+    assert sel(8, 2048, 512, 33, 16, 16, BF16, 1) == 5          # K = 33: no strip instantiation
+    assert sel(8, 2048, 96, 31, 15, 15, BF16, 1) == 6           # C % 64 != 0: ring kernel
     assert sel(8, 2048, 512, 31, 15, 15, F32, 0) == 5
     assert sel(8, 2048, 512, 31, 15, 15, F32, 2) == -2          # UNSUPPORTED
     assert sel(2, 300, 72, 31, 15, 15, BF16, 0) == 6            # C % 16 == 8: ring only
@@ -382,7 +383,8 @@ def test_new_entry_points_validate_before_launch(lib):
     fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the missing workspace is found first
     assert lib.dwsep1d_fwd(fake, fake, fake, P, fake, 2, 64, 64, 31, 15, 15, 64, 2, 1, P, 0,
                            P) == 4
-    assert lib.dwsep2d_select_path(8, 256, 512, 40, 3, 3, 2, 1, 1, 256, 1, 2, 0) == 21
+    assert lib.dwsep2d_select_path(8, 256, 512, 80, 3, 3, 2, 1, 1, 256, 1, 2, 0) == 21
+    assert lib.dwsep2d_select_path(8, 256, 512, 40, 3, 3, 2, 1, 1, 256, 1, 2, 0) == 17  # Wo 20
     assert lib.dwsep2d_select_path(8, 256, 512, 40, 3, 3, 2, 1, 1, 256, 0, 2, 0) == 17   # NCHW
     assert lib.dwsep2d_select_path(8, 256, 512, 40, 7, 7, 2, 3, 1, 256, 1, 2, 2) == -2
     assert lib.dwsep2d_fwd(P, P, P, P, P, 1, 64, 8, 8, 3, 3, 1, 1, 1, 64, 1, 2, 0, P, 0, P) == 1

@@ -45,13 +45,12 @@ def kernel_of(p, path=gb.PATH_AUTO):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("path", [gb.PATH_AUTO, gb.PATH_IGEMM])
+@pytest.mark.parametrize("path", [gb.PATH_AUTO, gb.PATH_DIRECT])
 def test_conformer_full_size(causal, path):
-    """The Conformer layer in full on the path the library picks (the 128-byte-row CUDA-core
-    kernel) and forced onto the tensor-core kernel."""
+    """The Conformer layer in full on the path the library picks (the tensor-core kernel)
+    and forced onto the 128-byte-row CUDA-core kernel."""
     p = wl.conformer_dw1d(causal)
-    assert kernel_of(p) == 20 and kernel_of(p, gb.PATH_DIRECT) == 20
-    assert kernel_of(p, gb.PATH_IGEMM) == 7
+    assert kernel_of(p) == 7 and kernel_of(p, gb.PATH_DIRECT) == 20
     check(p, 3, path=path)
 
 
@@ -74,15 +73,15 @@ STRIP_CASES = [
 @pytest.mark.parametrize("dtype", [wl.BF16, wl.F16])
 def test_strip_kernels(case, dtype):
     p = wl.Dwconv1dProblem(*case, dtype)
-    assert kernel_of(p) == 20
-    check(p, 35)
+    assert kernel_of(p, gb.PATH_DIRECT) == 20
+    check(p, 35, path=gb.PATH_DIRECT)
 
 
 def test_strip_integer_bit_exact_and_wgrad_deterministic():
     p = wl.Dwconv1dProblem(3, 700, 128, 31, 15, 15, wl.BF16)
     inp = wl.make_dwconv1d_inputs(p, 36, "int")
     inp.w = wl.to_storage(np.random.default_rng(6).integers(-2, 3, (p.C, p.K)), wl.BF16)
-    (y, dx, dw), (ry, rdx, rdw) = gpu_all(inp), oracle_all(inp)
+    (y, dx, dw), (ry, rdx, rdw) = gpu_all(inp, gb.PATH_DIRECT), oracle_all(inp)
     assert np.array_equal(y, ry) and np.array_equal(dx, rdx)
     rnd = lambda v: wl.widen(wl.to_storage(v, wl.BF16), wl.BF16)
     assert np.array_equal(dw, rnd(rdw))

@@ -150,10 +150,10 @@ def ref_2d(x, w_dw, w_pw, bias, k, stride, pad, dtype, layout=wl.NHWC):
 FUSED_2D = [
     # N, C, H, W, k, stride, pad, C_out
     (2, 64, 12, 40, 3, 1, 1, 64),
-    (1, 128, 20, 40, 3, 2, 1, 256),        # the Fast Conformer downsampler's strided layer
+    (1, 128, 20, 80, 3, 2, 1, 256),        # a strided downsampler layer (40 output columns)
     (2, 64, 9, 70, 5, 1, 2, 128),
-    (1, 64, 11, 33, 5, 2, 2, 96),
-    (1, 192, 7, 20, 3, 2, 1, 320),          # two MMA chunks, narrow rows (20 columns)
+    (1, 64, 11, 70, 5, 2, 2, 96),
+    (1, 192, 7, 70, 3, 2, 1, 320),          # two MMA chunks, a partial column tile
     (1, 64, 5, 150, 3, 1, 0, 512),          # 512 outputs: one tile row per CTA
 ]
 
@@ -180,10 +180,17 @@ def test_dwsep2d_composition(layout, path):
 
 
 def test_dwsep2d_fp16_no_bias_and_fallbacks():
-    x, w_dw, w_pw, b = make_2d(1, 64, 10, 36, 3, 2, 1, 64, 77, dtype=wl.F16, bias=False)
+    x, w_dw, w_pw, b = make_2d(1, 64, 10, 72, 3, 2, 1, 64, 77, dtype=wl.F16, bias=False)
+    assert gb.dwsep2d_select_path(1, 64, 10, 72, 3, 3, 2, 1, 1, 64, "NHWC", wl.F16) == 21
     assert_close(to_f64(run_2d(x, w_dw, w_pw, None, 3, 2, 1, wl.F16)),
                  ref_2d(x, w_dw, w_pw, None, 3, 2, 1, wl.F16), wl.F16, "fp16")
-    # C % 64 != 0 and a 7x7 kernel take the composition under AUTO
+    # C % 64 != 0, a 7x7 kernel and outputs narrower than a 32-column tile take the
+    # composition under AUTO
+    x, w_dw, w_pw, b = make_2d(1, 64, 12, 40, 3, 2, 1, 64, 79)
+    assert gb.dwsep2d_select_path(1, 64, 12, 40, 3, 3, 2, 1, 1, 64, "NHWC", wl.BF16) == 17
+    assert gb.dwsep2d_select_path(1, 64, 12, 40, 3, 3, 2, 1, 1, 64, "NHWC", wl.BF16, 2) == -2
+    assert_close(to_f64(run_2d(x, w_dw, w_pw, b, 3, 2, 1, wl.BF16)),
+                 ref_2d(x, w_dw, w_pw, b, 3, 2, 1, wl.BF16), wl.BF16, "Wo = 20")
     for (C, k) in ((40, 3), (64, 7)):
         x, w_dw, w_pw, b = make_2d(1, C, 12, 12, k, 1, k // 2, 32, 78)
         assert gb.dwsep2d_select_path(1, C, 12, 12, k, k, 1, k // 2, 1, 32, "NHWC",
