@@ -844,38 +844,7 @@ __global__ void __launch_bounds__(256) wgrad_tiled_nhwc_kernel(const T* __restri
   }
 }
 
-// [N][C][P] -> [N][P][C] for 16-bit elements (NCHW -> NHWC staging of the tiled weight
-// gradient), through 32 x 32 shared-memory tiles: reads run along P, writes along C.
-__global__ void __launch_bounds__(256) to_nhwc16_kernel(const unsigned short* __restrict__ src,
-                                                         unsigned short* __restrict__ dst,
-                                                         int C, long long P) {
-  __shared__ unsigned short tile[32][34];
-  const long long n = blockIdx.z;
-  const long long p0 = (long long)blockIdx.x * 32;
-  const int c0 = blockIdx.y * 32;
-  const int tx = threadIdx.x, ty = threadIdx.y;
-  for (int i = ty; i < 32; i += 8) {
-    const int c = c0 + i;
-    const long long pp = p0 + tx;
-    if (c < C && pp < P) tile[i][tx] = src[(n * C + c) * P + pp];
-  }
-  __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const long long pp = p0 + i;
-    const int c = c0 + tx;
-    if (c < C && pp < P) dst[(n * P + pp) * C + c] = tile[tx][i];
-  }
-}
-
 size_t staged_bytes(long long elems) { return ((size_t)elems * 2 + 255) / 256 * 256; }
-
-cudaError_t launch_to_nhwc16(const void* src, void* dst, int N, int C, long long P,
-                             cudaStream_t s) {
-  const dim3 grid((unsigned)((P + 31) / 32), (unsigned)((C + 31) / 32), (unsigned)N);
-  to_nhwc16_kernel<<<grid, dim3(32, 8), 0, s>>>((const unsigned short*)src,
-                                               (unsigned short*)dst, C, P);
-  return cudaGetLastError();
-}
 
 // dw from the slice partials: dw[e(q)] = sum over slices s of ws[s][q], q the partial index.
 // A CTA takes 32 consecutive q (one per lane, so each warp load is 128 contiguous bytes) and its
@@ -1111,8 +1080,9 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
         T* xs = (T*)ws;
         T* ds = (T*)((char*)ws + xb);
         part = (float*)((char*)ws + xb + db);
-        cudaError_t e = launch_to_nhwc16(x, xs, p.N, p.C_in, (long long)p.H * p.W, s);
-        if (e == cudaSuccess) e = launch_to_nhwc16(dy, ds, p.N, p.C_out, (long long)p.Ho * p.Wo, s);
+        cudaError_t e = launch_nchw_to_nhwc16(x, xs, p.N, p.C_in, (long long)p.H * p.W, s);
+        if (e == cudaSuccess)
+          e = launch_nchw_to_nhwc16(dy, ds, p.N, p.C_out, (long long)p.Ho * p.Wo, s);
         if (e != cudaSuccess) return e;
         xt = xs;
         dt = ds;
@@ -1246,9 +1216,11 @@ bool wgrad_depthwise_supported(const Conv2d& p) {
 }
 
 bool wgrad_tiled_supported(const Conv2d& p) {
+  // NCHW is staged as NHWC by launch_nchw_to_nhwc16 (grid: HW / 64 x C / 64 x N)
   const bool staging_ok = p.layout == GCONV_NHWC ||
-                          (p.N <= 65535 && (p.H * (long long)p.W + 31) / 32 <= 0x7fffffffLL &&
-                           (p.C_in + 31) / 32 <= 65535 && (p.C_out + 31) / 32 <= 65535);
+                          (p.N <= 65535 && (long long)p.H * p.W <= 0x7fffffffLL &&
+                           (long long)p.Ho * p.Wo <= 0x7fffffffLL &&
+                           (p.C_in + 63) / 64 <= 65535 && (p.C_out + 63) / 64 <= 65535);
   return staging_ok && p.dtype != GCONV_F32 && p.cpg_in >= 32 && p.cpg_out >= 32 &&
          p.cpg_in % 8 == 0 && p.cpg_out % 8 == 0 && tiled_count(p) <= 0x7fffffffLL &&
          (long long)p.N * p.Ho * p.Wo <= 0x7fffffffLL;

@@ -1975,6 +1975,19 @@ cudaError_t launch_nchw_typed(const Conv2d& p, const IgemmParams& P, const void*
   return launch_core<T>(p, P, xt, wt, bias, y, s);
 }
 
+cudaError_t launch_nchw_to_nhwc16(const void* x, void* xt, int N, int C, long long HW,
+                                  cudaStream_t s) {
+  if (HW > INT32_MAX || N > 65535 || (C + 63) / 64 > 65535) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)((HW + 63) / 64), (unsigned)((C + 63) / 64), (unsigned)N);
+  if (HW % 8 == 0 && C % 8 == 0 && aligned16(x) && aligned16(xt))
+    nchw_to_nhwc_kernel<unsigned short, true><<<grid, 256, 0, s>>>(
+        (const unsigned short*)x, (unsigned short*)xt, C, (int)HW);
+  else
+    nchw_to_nhwc_kernel<unsigned short, false><<<grid, 256, 0, s>>>(
+        (const unsigned short*)x, (unsigned short*)xt, C, (int)HW);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_igemm_nchw(const Conv2d& p, const void* x, const void* w, const void* bias,
                               void* y, void* workspace, cudaStream_t s) {
   IgemmParams P;

@@ -154,6 +154,11 @@ size_t wgrad_workspace(const Conv2d& p, int kernel);
 cudaError_t launch_wgrad(const Conv2d& p, const void* x, const void* dy, void* dw, void* ws,
                          int kernel, cudaStream_t s);
 
+// [N][C][HW] -> [N][HW][C] for 16-bit elements (NCHW -> NHWC staging): 64 x 64 tiles through
+// shared memory, 16-byte loads and stores when HW and C are multiples of 8.
+cudaError_t launch_nchw_to_nhwc16(const void* x, void* xt, int N, int C, long long HW,
+                                  cudaStream_t s);
+
 bool conv1d_vector_supported(const Conv1d& p);
 // Kernel (GCONV_KERNEL_CONV1D_*) for a forward / data-gradient call under `path`; x, w, y null
 // = a query that assumes aligned pointers. -1 with *why set when the forced family cannot run.
