@@ -28,24 +28,18 @@
 // writes NCHW directly.
 #include <cuda.h>
 
-#include "internal.cuh"
-#include "sm100_ptx.cuh"
+#include "igemm_common.cuh"
 
 namespace gconv {
 namespace {
 
 using namespace ptx;
 
-constexpr int BM = 128;                 // output pixels per tile (UMMA M)
-constexpr int NUM_THREADS = 192;        // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
-constexpr int MAX_STAGES = 32;
-constexpr size_t SMEM_BUDGET = 227 * 1024;
-
-enum : unsigned int { ERR_WAIT_PRODUCER = 1u, ERR_WAIT_MMA = 2u, ERR_WAIT_EPILOGUE = 4u,
-                      ERR_WAIT_DRAIN = 8u };
-
+// Kernel parameters of the tile kernel; like every parameter struct of the tcgen05 kernels it
+// is kept at 128 bytes or less (fields only the host needs stay in Conv2d): a larger struct
+// changed the code generated for the same kernel source and cost the row-strip kernel 25 %.
 struct IgemmParams {
-  int N, H, W, C_in, C_out, Ho, Wo, kW, pad, dil, cpg_in, cpg_out;
+  int C_out, Ho, Wo, kW, pad, dil, cpg_in, cpg_out;
   int BW, BH, BN, BKC, cblocks, kblocks, tiles_w, tiles_h, m_tiles, n_tiles, num_tiles;
   int stages;
   unsigned int tx_bytes;       // TMA bytes per stage (A box + B box)
@@ -60,18 +54,6 @@ struct IgemmParams {
   int groups, out_mode, out_c, nsub;
 };
 
-// Shared-memory matrix descriptor (tcgen05): start address, leading / stride byte offsets
-// (16-byte units), descriptor version 1 at bits 46-47, layout (swizzle) code at bits 61-63.
-// The base-offset field (bits 49-51) stays 0: the swizzle is taken from the absolute address.
-__device__ __forceinline__ unsigned long long smem_desc(unsigned int saddr, unsigned int sbo,
-                                                        unsigned int swz) {
-  unsigned long long d = (unsigned long long)((saddr >> 4) & 0x3FFFu);
-  d |= (unsigned long long)1u << 16;                          // LBO (unused for swizzled K-major)
-  d |= (unsigned long long)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (unsigned long long)1u << 46;
-  d |= (unsigned long long)(swz & 7u) << 61;
-  return d;
-}
 
 template <typename T, typename PP>
 __device__ __forceinline__ void epilogue_store(const PP& P, T* __restrict__ y,
@@ -399,19 +381,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // g*cpg_in channels before the row, so the other slots fall outside the row and are filled
 // with zeros.
 
-struct HaloParams {
-  int N, H, W, C_in, C_out, Ho, Wo, kH, kW, pad, dil, cpg_in, cpg_out;
+struct HaloParams {   // at most 128 bytes, as IgemmParams
+  int C_out, Ho, Wo, kH, kW, pad, dil, cpg_in, cpg_out;
   int BW, BH, BN, BKC, cblocks, KWS, kw_groups, tiles_h, m_tiles, n_tiles, num_tiles;
-  int stages, box_rows;
+  int stages;
   unsigned int a_region, a_stage, b_tile, b_stage, tx_bytes;
-  unsigned int idesc, swz, sbo, row_bytes, tmem_cols;
+  unsigned int idesc, tmem_cols;   // swizzle, SBO and row bytes follow from BKC
   int out_nchw;
-  int gp, gin, gout;           // groups packed per tile (block-diagonal filters), their
-                               // input and output channels: gin = gp*cpg_in, gout = gp*cpg_out
+  int gp;                      // groups packed per tile (block-diagonal filters)
   int tma_out;                 // NHWC output through shared memory and TMA stores
   unsigned int o_bytes;        // that staging, two buffers of BN/64 blocks of [128 rows][64 ch]
                                // with the 128-byte swizzle
 };
+
+// Bytes per box row (BKC 16-bit channels) and the matching swizzle code of the smem
+// descriptors (128 / 64 / 32-byte swizzle); the stride between 8-row groups is 8 rows.
+__host__ __device__ __forceinline__ unsigned int halo_row_bytes(const HaloParams& P) {
+  return (unsigned int)P.BKC * 2u;
+}
+__host__ __device__ __forceinline__ unsigned int halo_swz(unsigned int row_bytes) {
+  return row_bytes == 128 ? 2u : (row_bytes == 64 ? 4u : 6u);
+}
 
 __device__ __forceinline__ void halo_decode(const HaloParams& P, int t, int& j, int& nt, int& n,
                                             int& th) {
@@ -543,9 +533,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int j, nt, n, th;
         halo_decode(P, t, j, nt, n, th);
         const int hbase = th * P.BH - P.pad;
-        const int obase = j * (PACK ? P.gout : P.cpg_out) + nt * P.BN;
+        const int obase = j * (PACK ? P.gp * P.cpg_out : P.cpg_out) + nt * P.BN;
         for (int cb = 0; cb < P.cblocks && ok; ++cb) {
-          const int cin = j * (PACK ? P.gin : P.cpg_in) + cb * P.BKC;
+          const int cin = j * (PACK ? P.gp * P.cpg_in : P.cpg_in) + cb * P.BKC;
           for (int kg = 0; kg < P.kw_groups; ++kg) {
             if (!mbar_try_wait(&empty[s], ph ^ 1u) &&
                 !mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
@@ -566,7 +556,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                               obase);
                 } else {
                   for (int g = 0; g < P.gp; ++g)
-                    tma_load_3d(bt + (size_t)g * P.cpg_out * P.row_bytes, &tma_w, &full[s],
+                    tma_load_3d(bt + (size_t)g * P.cpg_out * halo_row_bytes(P), &tma_w, &full[s],
                                 -g * P.cpg_in, kh * P.kW + kw, obase + g * P.cpg_out);
                 }
               }
@@ -591,10 +581,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       unsigned int ph = 0, aph = 0;
       bool ok = true;
       const int ksteps = P.BKC / 16;
-      const unsigned long long a_desc0 = smem_desc(smem_u32(a_base), P.sbo, P.swz);
-      const unsigned long long b_desc0 = smem_desc(smem_u32(b_base), P.sbo, P.swz);
+      const unsigned int rb = halo_row_bytes(P);
+      const unsigned long long a_desc0 = smem_desc(smem_u32(a_base), 8u * rb, halo_swz(rb));
+      const unsigned long long b_desc0 = smem_desc(smem_u32(b_base), 8u * rb, halo_swz(rb));
       const unsigned long long kh_step =
-          ((unsigned long long)P.dil * P.BW * P.row_bytes) >> 4;   // kh rows of the box
+          ((unsigned long long)P.dil * P.BW * rb) >> 4;   // kh rows of the box
       const unsigned long long kw_step = P.a_region >> 4;
       const unsigned long long bt_step = P.b_tile >> 4;
       for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
@@ -672,7 +663,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int ho = th * P.BH + hl, wo = wl;
       const bool valid = hl < P.BH && ho < P.Ho;
-      const int co0 = j * (PACK ? P.gout : P.cpg_out) + nt * P.BN;
+      const int co0 = j * (PACK ? P.gp * P.cpg_out : P.cpg_out) + nt * P.BN;
       const unsigned int taddr =
           tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.BN);
       for (int c = 0; c < P.BN; c += 32) {
@@ -751,8 +742,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // is fetched once per kh instead of once per tap. The NSUB segments share
 // every weight tile. Strips and weight tiles have their own stage rings.
 
-constexpr int ROW_MAX_A = 4;
-constexpr int ROW_MAX_B = 16;
 
 struct RowParams {
   int N, H, W, C_in, C_out, Ho, Wo, kH, kW, pad, dil, cpg_in, cpg_out;
@@ -993,296 +982,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// ------------------------------------------------------------------ transposed row kernel
-//
-// When the filters per group are a multiple of 128, the row tile is computed transposed:
-// D^T[co x px] = W[co x k] * X^T[k x px] with M = 128 filters and N = 256 (or 128) output
-// pixels of one row per MMA. Each tcgen05.mma then carries twice the work of the 128 x 128
-// form, which halves the instructions and barrier waits the single issuing thread spends per
-// unit of tensor work. The pixel operand is the same input strip as in the row kernel
-// (one TMA box of NPIX rows plus an 8-row box for the halo), read at row offsets kw*dil for
-// the kW taps; the weight operand is one [128 x 64] tile per tap. In the epilogue each thread
-// owns one output channel (its TMEM lane): NHWC stores of a warp cover 32 consecutive
-// channels of a pixel, NCHW stores of a thread cover 32 consecutive pixels.
-
-struct RowTParams {
-  int N, H, W, C_in, C_out, Ho, Wo, kH, kW, pad, dil, cpg_in, cpg_out;
-  int NPIX, cblocks, segs, n_tiles, num_tiles, strip_rows;
-  int x_stages, w_stages;
-  unsigned int x_stage, w_stage, x_tx, w_tx, box1_bytes;
-  unsigned int idesc, tmem_cols;
-  int out_nchw, nchw_vec;
-  int groups, interleave;   // interleaved output order: filter f of group j -> f * groups + j
-  // average merge across groups: every group's K loop accumulates into one tile (jgroups =
-  // groups, tiles have no group index), the epilogue scales by 1/groups and writes out_c =
-  // C_out/groups channels; otherwise jgroups = 1, out_c = C_out, scale = 1
-  int jgroups, out_c;
-  float scale;
-};
-
-__device__ __forceinline__ void rowt_decode(const RowTParams& P, int t, int& j, int& nt, int& n,
-                                            int& ho, int& seg) {
-  seg = t % P.segs;
-  int r = t / P.segs;
-  ho = r % P.Ho;
-  r /= P.Ho;
-  n = r % P.N;
-  r /= P.N;
-  nt = r % P.n_tiles;
-  j = r / P.n_tiles;
-}
-
-template <typename T, bool MERGE>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    igemm_rowt_kernel(const __grid_constant__ CUtensorMap tma_x,
-                      const __grid_constant__ CUtensorMap tma_xh,
-                      const __grid_constant__ CUtensorMap tma_w, const T* __restrict__ bias,
-                      T* __restrict__ y, const RowTParams P, unsigned int* err) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = ptx::align_smem(smem_raw, 1024u);
-  unsigned char* x_base = smem;
-  unsigned char* w_base = smem + (size_t)P.x_stages * P.x_stage;
-  unsigned long long* bars =
-      reinterpret_cast<unsigned long long*>(w_base + (size_t)P.w_stages * P.w_stage);
-  unsigned long long* fx = bars;
-  unsigned long long* ex = fx + ROW_MAX_A;
-  unsigned long long* fw = ex + ROW_MAX_A;
-  unsigned long long* ew = fw + ROW_MAX_B;
-  unsigned long long* tfull = ew + ROW_MAX_B;
-  unsigned long long* tempty = tfull + 2;
-  unsigned long long* done = tempty + 2;
-  unsigned int* tmem_slot = reinterpret_cast<unsigned int*>(done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < P.x_stages; ++s) {
-      mbar_init(&fx[s], 1);
-      mbar_init(&ex[s], 1);
-    }
-    for (int s = 0; s < P.w_stages; ++s) {
-      mbar_init(&fw[s], 1);
-      mbar_init(&ew[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
-    }
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-    prefetch_tmap(&tma_x);
-    prefetch_tmap(&tma_xh);
-    prefetch_tmap(&tma_w);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, P.tmem_cols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const unsigned int tmem_base = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer
-      int sx = 0, sw = 0;
-      unsigned int px = 0, pw = 0;
-      long long nx = 0, nw = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
-        int j, nt, n, ho, seg;
-        rowt_decode(P, t, j, nt, n, ho, seg);
-        const int wbase = seg * P.NPIX - P.pad;
-        // channel blocks of the tile's group; MERGE: of every group in turn (jgroups * cblocks)
-        const int nblocks = MERGE ? P.jgroups * P.cblocks : P.cblocks;
-        for (int cbg = 0; cbg < nblocks && ok; ++cbg) {
-          const int jx = MERGE ? cbg / P.cblocks : j;
-          const int cb = MERGE ? cbg - jx * P.cblocks : cbg;
-          const int obase = jx * P.cpg_out + nt * BM;
-          const int cin = jx * P.cpg_in + cb * 64;
-          for (int kh = 0; kh < P.kH && ok; ++kh) {
-            if (!mbar_wait(&ex[sx], px ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
-              ok = false;
-              break;
-            }
-            unsigned char* dst = x_base + (size_t)sx * P.x_stage;
-            const int hrow = ho - P.pad + kh * P.dil;
-            mbar_arrive_expect_tx(&fx[sx], P.x_tx);
-            tma_load_4d(dst, &tma_x, &fx[sx], cin, wbase, hrow, n);
-            tma_load_4d(dst + P.box1_bytes, &tma_xh, &fx[sx], cin, wbase + P.NPIX, hrow, n);
-            ++nx;
-            if (++sx == P.x_stages) {
-              sx = 0;
-              px ^= 1u;
-            }
-            for (int kw = 0; kw < P.kW; ++kw) {
-              if (!mbar_wait(&ew[sw], pw ^ 1u, abort_flag, err, ERR_WAIT_PRODUCER)) {
-                ok = false;
-                break;
-              }
-              mbar_arrive_expect_tx(&fw[sw], P.w_tx);
-              tma_load_2d(w_base + (size_t)sw * P.w_stage, &tma_w, &fw[sw],
-                          (kh * P.kW + kw) * P.cpg_in + cb * 64, obase);
-              ++nw;
-              if (++sw == P.w_stages) {
-                sw = 0;
-                pw ^= 1u;
-              }
-            }
-          }
-        }
-      }
-      const unsigned long long dl = drain_deadline();
-      for (long long q = (nx > P.x_stages ? nx - P.x_stages : 0); q < nx; ++q)
-        mbar_wait_until(&fx[q % P.x_stages], (unsigned int)((q / P.x_stages) & 1), dl, err,
-                        ERR_WAIT_DRAIN);
-      for (long long q = (nw > P.w_stages ? nw - P.w_stages : 0); q < nw; ++q)
-        mbar_wait_until(&fw[q % P.w_stages], (unsigned int)((q / P.w_stages) & 1), dl, err,
-                        ERR_WAIT_DRAIN);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer: descriptors built once, advanced by constant offsets
-      int sx = 0, sw = 0, acc = 0;
-      unsigned int px = 0, pw = 0, aph = 0;
-      bool ok = true;
-      const unsigned long long x_desc0 = smem_desc(smem_u32(x_base), 1024u, 2u);
-      const unsigned long long w_desc0 = smem_desc(smem_u32(w_base), 1024u, 2u);
-      const unsigned long long kw_step = (unsigned long long)P.dil * 8u;   // dil rows of 128 B
-      for (int t = blockIdx.x; t < P.num_tiles && ok; t += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERR_WAIT_MMA)) break;
-        tc_fence_after();
-        const unsigned int d = tmem_base + (unsigned int)(acc * P.NPIX);
-        const int nblocks = MERGE ? P.jgroups * P.cblocks : P.cblocks;
-        for (int cb = 0; cb < nblocks && ok; ++cb) {
-          for (int kh = 0; kh < P.kH && ok; ++kh) {
-            if (!mbar_try_wait(&fx[sx], px) &&
-                !mbar_wait(&fx[sx], px, abort_flag, err, ERR_WAIT_MMA)) {
-              ok = false;
-              break;
-            }
-            const unsigned long long xs = x_desc0 + (((unsigned long long)sx * P.x_stage) >> 4);
-            for (int kw = 0; kw < P.kW; ++kw) {
-              if (!mbar_try_wait(&fw[sw], pw) &&
-                  !mbar_wait(&fw[sw], pw, abort_flag, err, ERR_WAIT_MMA)) {
-                ok = false;
-                break;
-              }
-              const unsigned long long wd = w_desc0 + (((unsigned long long)sw * P.w_stage) >> 4);
-              const unsigned long long xd = xs + kw * kw_step;
-              const unsigned int acc0 = (cb | kh | kw) == 0 ? 0u : 1u;
-              umma_f16(d, wd, xd, P.idesc, acc0);
-              umma_f16(d, wd + 2, xd + 2, P.idesc, 1u);
-              umma_f16(d, wd + 4, xd + 4, P.idesc, 1u);
-              umma_f16(d, wd + 6, xd + 6, P.idesc, 1u);
-              umma_commit(&ew[sw]);
-              if (++sw == P.w_stages) {
-                sw = 0;
-                pw ^= 1u;
-              }
-            }
-            if (!ok) break;
-            umma_commit(&ex[sx]);
-            if (++sx == P.x_stages) {
-              sx = 0;
-              px ^= 1u;
-            }
-          }
-        }
-        if (!ok) break;
-        umma_commit(&tfull[acc]);
-        if (++acc == 2) {
-          acc = 0;
-          aph ^= 1u;
-        }
-      }
-      umma_commit(done);
-      mbar_wait_until(done, 0, drain_deadline(), err, ERR_WAIT_DRAIN);
-    }
-  } else {
-    // ---------------- epilogue: warps 2..5; TMEM lane = output channel of the tile
-    const int quarter = warp & 3;
-    const int co_l = quarter * 32 + lane;
-    int acc = 0;
-    unsigned int aph = 0;
-    for (int t = blockIdx.x; t < P.num_tiles; t += gridDim.x) {
-      int j, nt, n, ho, seg;
-      rowt_decode(P, t, j, nt, n, ho, seg);
-      const bool got = mbar_wait(&tfull[acc], aph, abort_flag, err, ERR_WAIT_EPILOGUE);
-      if (!__all_sync(0xffffffffu, got)) break;
-      tc_fence_after();
-      const int co_g = j * P.cpg_out + nt * BM + co_l;       // group-major channel
-      // y's channel: interleaved position, merged channel, or the group-major one
-      const int co = P.interleave ? (nt * BM + co_l) * P.groups + j
-                                  : (MERGE ? nt * BM + co_l : co_g);
-      float bv = 0.0f;
-      if (bias) {
-        if (MERGE) {
-          for (int i = 0; i < P.jgroups; ++i)
-            bv += Elem<T>::to_f32(bias[i * P.cpg_out + nt * BM + co_l]);
-          bv *= P.scale;
-        } else {
-          bv = Elem<T>::to_f32(bias[co_g]);
-        }
-      }
-      const float sc = P.scale;   // 1 unless MERGE
-      const int oc = MERGE ? P.out_c : P.C_out;
-      // accumulator -> output value (the merge scales by 1/groups; the plain kernel adds bias)
-      auto outv = [&](unsigned int u) {
-        return MERGE ? fmaf(__uint_as_float(u), sc, bv) : __uint_as_float(u) + bv;
-      };
-      const unsigned int taddr =
-          tmem_base + ((unsigned int)(quarter * 32) << 16) + (unsigned int)(acc * P.NPIX);
-      for (int c = 0; c < P.NPIX; c += 32) {
-        unsigned int r[32];
-        tmem_ld32(taddr + c, r);
-        tmem_ld_wait();
-        const int wo0 = seg * P.NPIX + c;
-        if (wo0 >= P.Wo) continue;
-        if (!P.out_nchw) {
-          T* dst = y + (((long long)n * P.Ho + ho) * P.Wo + wo0) * oc + co;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (wo0 + i < P.Wo)
-              dst[(long long)i * oc] = Elem<T>::from_f32(outv(r[i]));
-        } else {
-          T* dst = y + (((long long)n * oc + co) * P.Ho + ho) * P.Wo + wo0;
-          if (P.nchw_vec && wo0 + 32 <= P.Wo) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 u;
-              u.x = pack2<T>(make_float2(outv(r[8 * q + 0]), outv(r[8 * q + 1])));
-              u.y = pack2<T>(make_float2(outv(r[8 * q + 2]), outv(r[8 * q + 3])));
-              u.z = pack2<T>(make_float2(outv(r[8 * q + 4]), outv(r[8 * q + 5])));
-              u.w = pack2<T>(make_float2(outv(r[8 * q + 6]), outv(r[8 * q + 7])));
-              reinterpret_cast<uint4*>(dst)[q] = u;
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (wo0 + i < P.Wo) dst[i] = Elem<T>::from_f32(outv(r[i]));
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        aph ^= 1u;
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem_base, P.tmem_cols);
-  }
-}
 
 // ------------------------------------------------------------------ NCHW staging kernels
 
@@ -1393,14 +1092,9 @@ int tile_bn(const Conv2d& p) {
   return p.cpg_out % 128 == 0 ? 128 : 0;
 }
 
-unsigned int pow2_cols(int n) {
-  unsigned int c = 32;
-  while ((int)c < n) c <<= 1;
-  return c;
-}
 
 bool make_params(const Conv2d& p, IgemmParams* P) {
-  P->N = p.N; P->H = p.H; P->W = p.W; P->C_in = p.C_in; P->C_out = p.C_out;
+  P->C_out = p.C_out;
   P->Ho = p.Ho; P->Wo = p.Wo; P->kW = p.kW; P->pad = p.pad; P->dil = p.dil;
   P->cpg_in = p.cpg_in; P->cpg_out = p.cpg_out;
   P->BW = p.Wo < BM ? p.Wo : BM;
@@ -1567,109 +1261,8 @@ cudaError_t launch_row(const Conv2d& p, const RowParams& R, const void* x, const
   return cudaGetLastError();
 }
 
-// Transposed row kernel parameters; false if the problem does not take it.
-bool make_rowt_params(const Conv2d& p, RowTParams* R) {
-  if (p.out_mode == GCONV_OUT_MERGE_MAX) return false;
-  if (p.Wo < BM || p.cpg_in % 64 != 0 || p.cpg_out % BM != 0) return false;
-  if ((p.kW - 1) * p.dil > 8) return false;            // halo fits the 8-row second box
-  R->N = p.N; R->H = p.H; R->W = p.W; R->C_in = p.C_in; R->C_out = p.C_out;
-  R->Ho = p.Ho; R->Wo = p.Wo; R->kH = p.kH; R->kW = p.kW; R->pad = p.pad; R->dil = p.dil;
-  R->cpg_in = p.cpg_in; R->cpg_out = p.cpg_out;
-  R->NPIX = p.Wo > BM ? 256 : 128;
-  R->cblocks = p.cpg_in / 64;
-  R->segs = (p.Wo + R->NPIX - 1) / R->NPIX;
-  R->n_tiles = p.cpg_out / BM;
-  const long long tiles = (long long)R->segs * p.Ho * p.N * R->n_tiles * p.groups;
-  if (tiles > INT32_MAX) return false;
-  R->num_tiles = (int)tiles;
-  R->strip_rows = R->NPIX + 8;
-  R->box1_bytes = (unsigned int)R->NPIX * 128u;
-  R->x_tx = (unsigned int)R->strip_rows * 128u;
-  R->x_stage = (R->x_tx + 1023u) & ~1023u;
-  R->w_tx = (unsigned int)BM * 128u;
-  R->w_stage = R->w_tx;
-  const size_t fixed = 1024 + (2 * (ROW_MAX_A + ROW_MAX_B) + 5) * 8 + 16;
-  const size_t budget = SMEM_BUDGET - fixed;
-  int xs = 3;
-  if ((size_t)xs * R->x_stage > budget / 2) xs = 2;
-  int ws = (int)((budget - (size_t)xs * R->x_stage) / R->w_stage);
-  if (ws > ROW_MAX_B) ws = ROW_MAX_B;
-  if (ws < 2) return false;
-  R->x_stages = xs;
-  R->w_stages = ws;
-  const unsigned int fmt = p.dtype == GCONV_BF16 ? 1u : 0u;
-  R->idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((unsigned int)(R->NPIX >> 3) << 17) |
-             ((unsigned int)(BM >> 4) << 24);
-  R->tmem_cols = pow2_cols(2 * R->NPIX);
-  if (R->tmem_cols > 512) return false;
-  R->out_nchw = p.layout == GCONV_NCHW;
-  R->nchw_vec = (p.Wo % 8 == 0) ? 1 : 0;
-  R->groups = p.groups;
-  R->interleave = p.out_mode == GCONV_OUT_INTERLEAVED;
-  const bool avg = p.out_mode == GCONV_OUT_MERGE_AVG;
-  R->jgroups = avg ? p.groups : 1;
-  R->out_c = out_channels(p);
-  R->scale = avg ? 1.0f / (float)p.groups : 1.0f;
-  if (avg) R->num_tiles /= p.groups;   // one tile covers every group's K loop
-  return true;
-}
-
-size_t rowt_smem_bytes(const RowTParams& R) {
-  return 1024 + (size_t)R.x_stages * R.x_stage + (size_t)R.w_stages * R.w_stage +
-         (2 * (ROW_MAX_A + ROW_MAX_B) + 5) * 8 + 16;
-}
-
-template <typename T>
-cudaError_t launch_rowt(const Conv2d& p, const RowTParams& R, const void* x, const void* w,
-                        const void* bias, void* y, cudaStream_t s) {
-  EncodeTiledFn enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
-  const CUtensorMapDataType dt =
-      p.dtype == GCONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUtensorMap tx, txh, tw;
-  const cuuint64_t xdim[4] = {(cuuint64_t)p.C_in, (cuuint64_t)p.W, (cuuint64_t)p.H,
-                              (cuuint64_t)p.N};
-  const cuuint64_t xstr[3] = {(cuuint64_t)p.C_in * 2, (cuuint64_t)p.W * p.C_in * 2,
-                              (cuuint64_t)p.H * p.W * p.C_in * 2};
-  const cuuint32_t ones[4] = {1, 1, 1, 1};
-  const cuuint32_t xbox[4] = {64, (cuuint32_t)R.NPIX, 1, 1};
-  const cuuint32_t hbox[4] = {64, 8, 1, 1};
-  if (enc(&tx, dt, 4, const_cast<void*>(x), xdim, xstr, xbox, ones,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  if (enc(&txh, dt, 4, const_cast<void*>(x), xdim, xstr, hbox, ones,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  const cuuint64_t ktot = (cuuint64_t)p.kH * p.kW * p.cpg_in;
-  const cuuint64_t wdim[2] = {ktot, (cuuint64_t)p.C_out};
-  const cuuint64_t wstr[1] = {ktot * 2};
-  const cuuint32_t wbox[2] = {64, (cuuint32_t)BM};
-  if (enc(&tw, dt, 2, const_cast<void*>(w), wdim, wstr, wbox, ones,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  const size_t smem = rowt_smem_bytes(R);
-  if (smem > SMEM_BUDGET) return cudaErrorInvalidValue;
-  // the average merge is its own instantiation, so the plain kernel's loops stay as they were
-  static std::atomic<unsigned int> configured{0}, configured_merge{0};
-  const bool merge = R.jgroups > 1;
-  cudaError_t e = merge ? set_max_dynamic_smem((const void*)igemm_rowt_kernel<T, true>,
-                                               SMEM_BUDGET, configured_merge)
-                        : set_max_dynamic_smem((const void*)igemm_rowt_kernel<T, false>,
-                                               SMEM_BUDGET, configured);
-  if (e != cudaSuccess) return e;
-  int grid = sm_count();
-  if (grid > R.num_tiles) grid = R.num_tiles;
-  if (merge)
-    igemm_rowt_kernel<T, true><<<grid, NUM_THREADS, smem, s>>>(tx, txh, tw, (const T*)bias,
-                                                               (T*)y, R, device_error_word());
-  else
-    igemm_rowt_kernel<T, false><<<grid, NUM_THREADS, smem, s>>>(tx, txh, tw, (const T*)bias,
-                                                                (T*)y, R, device_error_word());
-  return cudaGetLastError();
-}
+// Input rows of a halo tile's TMA box: the tile's output rows plus the kH halo.
+int halo_box_rows(const Conv2d& p, const HaloParams& H) { return H.BH + (p.kH - 1) * p.dil; }
 
 // Halo tile kernel parameters; false if the problem does not take it (rows wider than 128,
 // a width that is not a multiple of 8, or stages that do not fit).
@@ -1687,35 +1280,34 @@ bool make_halo_params(const Conv2d& p, HaloParams* H) {
       (64 / p.cpg_in) * p.cpg_out <= 64 && ((64 / p.cpg_in) * p.cpg_out) % 16 == 0)
     gp = 64 / p.cpg_in;
   H->gp = gp;
-  H->gin = gp * p.cpg_in;
-  H->gout = gp * p.cpg_out;
-  const int BN = gp > 1 ? H->gout : tile_bn(p);
+  const int gin = gp * p.cpg_in, gout = gp * p.cpg_out;   // channels of a packed tile
+  const int BN = gp > 1 ? gout : tile_bn(p);
   if (BN == 0) return false;
-  H->N = p.N; H->H = p.H; H->W = p.W; H->C_in = p.C_in; H->C_out = p.C_out;
-  H->Ho = p.Ho; H->Wo = p.Wo; H->kH = p.kH; H->kW = p.kW; H->pad = p.pad; H->dil = p.dil;
+  H->C_out = p.C_out; H->Ho = p.Ho; H->Wo = p.Wo; H->kH = p.kH; H->kW = p.kW; H->pad = p.pad; H->dil = p.dil;
   H->cpg_in = p.cpg_in; H->cpg_out = p.cpg_out;
   H->BW = p.Wo;
   H->BH = BM / p.Wo;
   if (H->BH > p.Ho) H->BH = p.Ho;
   H->BN = BN;
-  H->BKC = H->gin % 64 == 0 ? 64 : (H->gin % 32 == 0 ? 32 : 16);
-  H->cblocks = H->gin / H->BKC;
+  H->BKC = gin % 64 == 0 ? 64 : (gin % 32 == 0 ? 32 : 16);
+  H->cblocks = gin / H->BKC;
   H->tiles_h = (p.Ho + H->BH - 1) / H->BH;
   const long long m_tiles = (long long)p.N * H->tiles_h;
-  H->n_tiles = H->gout / BN;
+  H->n_tiles = gout / BN;
   const long long tiles = m_tiles * H->n_tiles * (p.groups / gp);
   if (tiles > INT32_MAX) return false;
   H->m_tiles = (int)m_tiles;
   H->num_tiles = (int)tiles;
-  H->box_rows = H->BH + (p.kH - 1) * p.dil;
-  if (H->box_rows > 256) return false;
-  H->row_bytes = (unsigned int)H->BKC * 2u;
+  const int box_rows = halo_box_rows(p, *H);
+  if (box_rows > 256) return false;
+  const unsigned int row_bytes = halo_row_bytes(*H);
   // rows an MMA may read from a box: up to (kH-1)*dil*BW + 128
-  unsigned int rows = (unsigned int)(H->box_rows * H->BW);
+  unsigned int rows = (unsigned int)(box_rows * H->BW);
   const unsigned int mma_rows = (unsigned int)((p.kH - 1) * p.dil * H->BW + BM);
   if (mma_rows > rows) rows = mma_rows;
-  H->a_region = (rows * H->row_bytes + 1023u) & ~1023u;
-  H->b_tile = (unsigned int)BN * H->row_bytes;
+  H->a_region = (rows * row_bytes + 1023u) & ~1023u;
+  H->b_tile = (unsigned int)BN * row_bytes;
+  H->out_nchw = p.layout == GCONV_NCHW;
   H->tma_out = p.layout == GCONV_NHWC && BN % 64 == 0;
   H->o_bytes = H->tma_out ? 2u * (unsigned int)(BN / 64) * 128u * 128u : 0u;
   const size_t fixed = 1024 + (2 * MAX_STAGES + 5) * 8 + 16 + H->o_bytes;
@@ -1740,14 +1332,11 @@ bool make_halo_params(const Conv2d& p, HaloParams* H) {
   if (H->stages < 2) return false;
   H->kw_groups = p.kW / H->KWS;
   H->tx_bytes = (unsigned int)H->KWS *
-                ((unsigned int)(H->BKC * H->BW * H->box_rows * 2) + (unsigned int)p.kH * H->b_tile);
-  H->swz = H->row_bytes == 128 ? 2u : (H->row_bytes == 64 ? 4u : 6u);
-  H->sbo = 8u * H->row_bytes;
+                ((unsigned int)(H->BKC * H->BW * box_rows * 2) + (unsigned int)p.kH * H->b_tile);
   const unsigned int fmt = p.dtype == GCONV_BF16 ? 1u : 0u;
   H->idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((unsigned int)(BN >> 3) << 17) |
              ((unsigned int)(BM >> 4) << 24);
   H->tmem_cols = pow2_cols(2 * BN);
-  H->out_nchw = p.layout == GCONV_NCHW;
   return true;
 }
 
@@ -1768,7 +1357,8 @@ cudaError_t launch_halo(const Conv2d& p, const HaloParams& H, const void* x, con
                               (cuuint64_t)p.N};
   const cuuint64_t xstr[3] = {(cuuint64_t)p.C_in * 2, (cuuint64_t)p.W * p.C_in * 2,
                               (cuuint64_t)p.H * p.W * p.C_in * 2};
-  const cuuint32_t xbox[4] = {(cuuint32_t)H.BKC, (cuuint32_t)H.BW, (cuuint32_t)H.box_rows, 1};
+  const cuuint32_t xbox[4] = {(cuuint32_t)H.BKC, (cuuint32_t)H.BW, (cuuint32_t)halo_box_rows(p, H),
+                              1};
   const cuuint32_t ones[4] = {1, 1, 1, 1};
   if (enc(&tx, dt, 4, const_cast<void*>(x), xdim, xstr, xbox, ones,
           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(H.BKC), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1861,8 +1451,7 @@ bool flatten_pointwise(const Conv2d& p, Conv2d* q) {
 template <typename T>
 cudaError_t launch_tiles(const Conv2d& p, const IgemmParams& P, const void* x, const void* w,
                          const void* bias, void* y, cudaStream_t s) {
-  RowTParams RT;
-  if (make_rowt_params(p, &RT)) return launch_rowt<T>(p, RT, x, w, bias, y, s);
+  if (igemm_rowt_supported(p)) return launch_igemm_rowt(p, x, w, bias, y, s);
   RowParams R;
   if (make_row_params(p, &R)) return launch_row<T>(p, R, x, w, bias, y, s);
   HaloParams HP;

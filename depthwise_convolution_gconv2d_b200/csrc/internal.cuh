@@ -117,6 +117,12 @@ cudaError_t launch_igemm_nhwc(const Conv2d& p, const void* x, const void* w, con
                               void* y, cudaStream_t s);
 cudaError_t launch_igemm_nchw(const Conv2d& p, const void* x, const void* w, const void* bias,
                               void* y, void* workspace, cudaStream_t s);
+// Transposed row-strip kernel (igemm_rowt.cu): NHWC x, [C_out][kH][kW][C_in/g] weights,
+// 16-bit data; y in p.layout. Supported: outputs >= 128 wide, 64-channel input blocks,
+// filters per group a multiple of 128, kW halo <= 8 rows, any output mode but the max merge.
+bool igemm_rowt_supported(const Conv2d& p);
+cudaError_t launch_igemm_rowt(const Conv2d& p, const void* x, const void* w, const void* bias,
+                              void* y, cudaStream_t s);
 
 // Grouped conv2d backward. dgrad_as_forward: stride 1, square kernel, pad <= dil*(k-1), so the
 // data gradient is the forward conv of the exchanged problem with the flipped, transposed
