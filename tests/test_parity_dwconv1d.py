@@ -130,6 +130,43 @@ def test_tensor_core_edges(case, dtype):
     check(p, 33, path=gb.PATH_IGEMM if tc else gb.PATH_AUTO)
 
 
+# Tensor-core forward / data gradient with C a multiple of 64 (several channel tiles per
+# step chunk, as in the Conformer layer) at every KS, on short inputs whose boxes lie outside
+# the sequence, pads wider than a box and T_out > T.
+TC64_CASES = [
+    # B, T, C, K, pl, pr
+    (1, 4100, 64, 31, 15, 15),    # three step chunks, the last one ragged
+    (2, 2049, 128, 17, 8, 8),     # KS = 2 at its largest K; one step into a second chunk
+    (1, 600, 64, 33, 16, 16),     # KS = 3 at its largest K
+    (1, 300, 64, 1, 0, 0),        # K = 1, KS = 1
+    (2, 700, 64, 3, 1, 1),        # KS = 1
+    (3, 7, 64, 31, 15, 15),       # T far shorter than a box
+    (1, 100, 64, 5, 300, 0),      # left pad wider than a box
+    (1, 300, 64, 31, 30, 30),     # T_out > T
+    (2, 1030, 192, 31, 30, 0),    # causal, three channel blocks
+]
+
+
+@pytest.mark.parametrize("case", TC64_CASES)
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F16])
+def test_tensor_core_64ch_edges(case, dtype):
+    p = wl.Dwconv1dProblem(*case, dtype)
+    assert kernel_of(p, gb.PATH_IGEMM) == 7
+    check(p, 35, path=gb.PATH_IGEMM)
+
+
+@pytest.mark.parametrize("case", TC64_CASES[:3] + TC64_CASES[5:7])
+def test_tensor_core_64ch_integer_bit_exact(case):
+    """Integer-valued data: the tensor-core path gives the oracle's value bit for bit (fwd and
+    dgrad) with several channel tiles, so every index, shift and pad is exact."""
+    p = wl.Dwconv1dProblem(*case, wl.BF16)
+    inp = wl.make_dwconv1d_inputs(p, 36, "int")
+    inp.w = wl.to_storage(np.random.default_rng(6).integers(-2, 3, (p.C, p.K)), wl.BF16)
+    (y, dx, _), (ry, rdx, _) = gpu_all(inp, gb.PATH_IGEMM), oracle_all(inp)
+    assert np.array_equal(y, ry)
+    assert np.array_equal(dx, rdx)
+
+
 @pytest.mark.parametrize("case", TC_CASES[:4])
 def test_ring_and_generic_paths_agree_with_oracle(case):
     """The same problems forced onto the CUDA-core kernels (ring where instantiated, generic
