@@ -67,6 +67,46 @@ def test_igemm_small_nchw(case):
     assert_close(to_f64(y), oracle_full(inp), p.dtype, str(case))
 
 
+# NCHW problems on the transposed row-strip kernel (through the NHWC staging copy): several
+# images and groups, two row segments, dilation, 5x5 with rows outside a 3-row image, the
+# wide-group layer's channels on two rows.
+NCHW_ROWT = [
+    # N, C_in, H, W, C_out, k, pad, dil, groups
+    (2, 128, 5, 136, 256, 3, 1, 1, 2),
+    (1, 256, 4, 264, 256, 3, 1, 1, 2),
+    (1, 128, 6, 128, 128, 3, 2, 2, 1),
+    (3, 64, 3, 200, 128, 5, 2, 1, 1),
+    (1, 512, 2, 256, 512, 3, 1, 1, 4),
+]
+
+
+@pytest.mark.parametrize("case", NCHW_ROWT)
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F16])
+def test_igemm_nchw_rowt(case, dtype):
+    p = problem(case, wl.NCHW, dtype=dtype, bias=True)
+    assert kernel_of(p, gb.PATH_IGEMM) == 4
+    inp = wl.make_conv2d_inputs(p, 23)
+    y = run_gpu(inp, gb.PATH_IGEMM)
+    assert gb.device_error() == 0
+    assert_close(to_f64(y), oracle_full(inp), p.dtype, str(case))
+
+
+@pytest.mark.parametrize("case", NCHW_ROWT[::2])
+def test_igemm_nchw_rowt_integer_bit_exact(case):
+    """x in {-1, 0, 1}, sparse filters in {-1, 0, 1} with at most 255 non-zero taps each: every
+    sum is an exact integer below 256, exact in bf16, so the NCHW -> NHWC staging and every tap
+    must give the oracle's value bit for bit."""
+    p = problem(case, wl.NCHW)
+    r = np.random.default_rng(25)
+    inp = wl.make_conv2d_inputs(p, 24)
+    w = r.integers(-1, 2, p.w_shape) * (r.random(p.w_shape) < 1 / 16)
+    assert np.abs(w).reshape(p.C_out, -1).sum(axis=1).max() <= 255
+    inp.x = wl.to_storage(r.integers(-1, 2, p.x_shape), wl.BF16)
+    inp.w = wl.to_storage(w, wl.BF16)
+    y = run_gpu(inp, gb.PATH_IGEMM)
+    assert np.array_equal(to_f64(y), oracle_full(inp))
+
+
 @pytest.mark.parametrize("case", SMALL[:4])
 def test_igemm_fp16(case):
     p = problem(case, dtype=wl.F16)
