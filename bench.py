@@ -248,8 +248,10 @@ SM_MAX_MHZ = 1965.0     # B200 clocks.max.sm
 def ffma_peak_tflops(sms: int = 148, mhz: float = SM_MAX_MHZ) -> float:
     """FP32 FMA roofline of the CUDA cores: 128 FMA lanes per SM, 2 FLOP per FMA."""
     return sms * 128 * 2 * mhz * 1e6 / 1e12
-KERNEL_SOURCE = {1: "direct_generic.cu", 2: "depthwise_nhwc.cu", 3: "igemm_tc.cu",
-                 4: "igemm_tc.cu", 8: "grouped_nhwc.cu"}
+# source file of the kernel that runs the headline layer for each kernel code (the wide-group
+# layer takes the transposed row-strip kernel, igemm_rowt.cu)
+KERNEL_SOURCE = {1: "direct_generic.cu", 2: "depthwise_nhwc.cu", 3: "igemm_rowt.cu",
+                 4: "igemm_rowt.cu", 8: "grouped_nhwc.cu"}
 
 
 def conv2d_measurement(torch, gb, device, stream, pk, p, workload, path, reps, flush):
@@ -664,8 +666,12 @@ def run_profile(name: str, reps: int, batch: int = 0) -> int:
             p = dataclasses.replace(p, N=batch)
         inp = wl.make_conv2d_inputs(p, 2)
         x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
+        # every launch writes its own y: the outputs are kept, so a capture of launch k > 1
+        # with --cache-control none sees launch k-1's dirty y lines written back to DRAM
+        ys = []
         for _ in range(reps):
-            gb.gconv2d_fwd(x, w, None, p.stride, p.pad, p.dilation, p.groups, p.layout)
+            ys.append(gb.gconv2d_fwd(x, w, None, p.stride, p.pad, p.dilation, p.groups,
+                                     p.layout))
     torch.cuda.synchronize()
     code = gb.device_error()
     print(json.dumps({"profile": name, "reps": reps, "device_error": code}))
@@ -792,8 +798,8 @@ def main():
     if pk.get("bf16_tflops_sustained"):
         roof["frac_of_sustained_peak"] = round(achieved / pk["bf16_tflops_sustained"], 4)
     if tr:
-        # reads compare with x + w; the writes of one cold launch miss the part of y that is
-        # still dirty in L2 when the kernel ends (written back after it)
+        # reads compare with x + w, writes with y: one launch of a back-to-back sequence, each
+        # launch with its own y, so the previous launch's y is written back inside it
         roof["traffic_read"] = tr.get("dram_read_bytes")
         roof["traffic_write"] = tr.get("dram_write_bytes")
         roof["alg_read"] = p.bytes() - p.N * p.C_out * p.Ho * p.Wo * 2
