@@ -383,7 +383,11 @@ def test_new_entry_points_validate_before_launch(lib):
     fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the missing workspace is found first
     assert lib.dwsep1d_fwd(fake, fake, fake, P, fake, 2, 64, 64, 31, 15, 15, 64, 2, 1, P, 0,
                            P) == 4
-    assert lib.dwsep2d_select_path(8, 256, 512, 80, 3, 3, 2, 1, 1, 256, 1, 2, 0) == 21
+    # AUTO: the fused kernel only when the depthwise output (N*Ho*Wo*C*2 bytes) exceeds 96 MB,
+    # the composition when it stays in L2 between its two launches; IGEMM forces the kernel
+    assert lib.dwsep2d_select_path(8, 256, 512, 80, 3, 3, 2, 1, 1, 256, 1, 2, 0) == 17   # 42 MB
+    assert lib.dwsep2d_select_path(8, 256, 512, 80, 3, 3, 2, 1, 1, 256, 1, 2, 2) == 21
+    assert lib.dwsep2d_select_path(8, 256, 1024, 256, 3, 3, 2, 1, 1, 256, 1, 2, 0) == 21  # 268 MB
     assert lib.dwsep2d_select_path(8, 256, 512, 40, 3, 3, 2, 1, 1, 256, 1, 2, 0) == 17  # Wo 20
     assert lib.dwsep2d_select_path(8, 256, 512, 40, 3, 3, 2, 1, 1, 256, 0, 2, 0) == 17   # NCHW
     assert lib.dwsep2d_select_path(8, 256, 512, 40, 7, 7, 2, 3, 1, 256, 1, 2, 2) == -2

@@ -162,8 +162,9 @@ FUSED_2D = [
 def test_dwsep2d_fused(case):
     N, C, H, W, k, s, pad, Co = case
     x, w_dw, w_pw, b = make_2d(N, C, H, W, k, s, pad, Co, 75)
-    assert gb.dwsep2d_select_path(N, C, H, W, k, k, s, pad, 1, Co, "NHWC", wl.BF16) == 21
-    assert_close(to_f64(run_2d(x, w_dw, w_pw, b, k, s, pad, wl.BF16)),
+    assert gb.dwsep2d_select_path(N, C, H, W, k, k, s, pad, 1, Co, "NHWC", wl.BF16,
+                                  gb.PATH_IGEMM) == 21
+    assert_close(to_f64(run_2d(x, w_dw, w_pw, b, k, s, pad, wl.BF16, path=gb.PATH_IGEMM)),
                  ref_2d(x, w_dw, w_pw, b, k, s, pad, wl.BF16), wl.BF16, str(case))
 
 
@@ -181,8 +182,9 @@ def test_dwsep2d_composition(layout, path):
 
 def test_dwsep2d_fp16_no_bias_and_fallbacks():
     x, w_dw, w_pw, b = make_2d(1, 64, 10, 72, 3, 2, 1, 64, 77, dtype=wl.F16, bias=False)
-    assert gb.dwsep2d_select_path(1, 64, 10, 72, 3, 3, 2, 1, 1, 64, "NHWC", wl.F16) == 21
-    assert_close(to_f64(run_2d(x, w_dw, w_pw, None, 3, 2, 1, wl.F16)),
+    assert gb.dwsep2d_select_path(1, 64, 10, 72, 3, 3, 2, 1, 1, 64, "NHWC", wl.F16,
+                                  gb.PATH_IGEMM) == 21
+    assert_close(to_f64(run_2d(x, w_dw, w_pw, None, 3, 2, 1, wl.F16, path=gb.PATH_IGEMM)),
                  ref_2d(x, w_dw, w_pw, None, 3, 2, 1, wl.F16), wl.F16, "fp16")
     # C % 64 != 0, a 7x7 kernel and outputs narrower than a 32-column tile take the
     # composition under AUTO
