@@ -30,7 +30,7 @@ KERNEL_NAMES = {1: "direct_generic", 2: "depthwise_nhwc", 3: "igemm_tc", 4: "ige
                 12: "dgrad_depthwise_nhwc", 13: "wgrad_tiled_nhwc", 14: "wgrad_dw3_tma",
                 15: "wgrad_tiled_nchw", 16: "dwsep1d_fused", 17: "dwsep_unfused",
                 18: "wgrad_tc_nhwc", 19: "wgrad_tc_nchw", 20: "conv1d_strip",
-                21: "dwsep2d_fused", 22: "dgrad_dw3s2_tma"}
+                21: "dwsep2d_fused", 22: "dgrad_dw3s2_tma", 23: "merge_max_two_pass"}
 STATUS = {0: "GCONV_OK", 1: "GCONV_ERR_INVALID_ARG", 2: "GCONV_ERR_UNSUPPORTED",
           3: "GCONV_ERR_MISALIGNED", 4: "GCONV_ERR_WORKSPACE", 5: "GCONV_ERR_CUDA",
           6: "GCONV_ERR_DEVICE_TIMEOUT"}

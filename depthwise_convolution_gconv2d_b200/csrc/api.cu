@@ -134,6 +134,20 @@ bool out_mode_is_plain(const Conv2d& p) {
   return p.out_mode == GCONV_OUT_INTERLEAVED && p.cpg_out == 1;
 }
 
+// The max merge in two passes (GCONV_KERNEL_MERGE_MAX_TWO_PASS): the plain problem, written
+// group-major to the workspace by the transposed row-strip kernel, then the maximum over
+// groups. Taken where that kernel runs the plain problem (16-bit).
+bool merge_max_two_pass_ok(const Conv2d& p) {
+  if (p.out_mode != GCONV_OUT_MERGE_MAX || p.dtype == GCONV_F32) return false;
+  Conv2d q = p;
+  q.out_mode = GCONV_OUT_GROUP_MAJOR;
+  return igemm_supported(q) && igemm_rowt_supported(q);
+}
+
+size_t merge_max_group_major_bytes(const Conv2d& p) {
+  return ((size_t)p.N * p.C_out * p.Ho * p.Wo * 2 + 255) / 256 * 256;
+}
+
 int choose_kernel_out(const Conv2d& p, int path, const void* x, const void* w, const void* y,
                       gconv_status* why) {
   if (out_mode_is_plain(p)) {
@@ -143,6 +157,9 @@ int choose_kernel_out(const Conv2d& p, int path, const void* x, const void* w, c
   }
   *why = GCONV_OK;
   const bool query = (x == nullptr && w == nullptr && y == nullptr);
+  if (merge_max_two_pass_ok(p) && (path == GCONV_PATH_AUTO || path == GCONV_PATH_IGEMM) &&
+      (query || (aligned16(x) && aligned16(y) && (p.layout == GCONV_NCHW || aligned16(w)))))
+    return GCONV_KERNEL_MERGE_MAX_TWO_PASS;
   const bool tc_ok = igemm_supported(p);
   const bool tc_al = query || (aligned16(x) && aligned16(y) &&
                                (p.layout == GCONV_NCHW || aligned16(w)));
@@ -424,6 +441,12 @@ size_t gconv2d_fwd_out_workspace_size(int N, int C_in, int H, int W, int C_out, 
     return 0;
   gconv_status why;
   const int k = choose_kernel_out(p, path, nullptr, nullptr, nullptr, &why);
+  if (k == GCONV_KERNEL_MERGE_MAX_TWO_PASS) {
+    Conv2d q = p;
+    q.out_mode = GCONV_OUT_GROUP_MAJOR;
+    return merge_max_group_major_bytes(p) +
+           (p.layout == GCONV_NCHW ? igemm_nchw_workspace(q) : 0);
+  }
   return k == GCONV_KERNEL_IGEMM_TC_NCHW ? igemm_nchw_workspace(p) : 0;
 }
 
@@ -452,6 +475,19 @@ gconv_status gconv2d_fwd_out(const void* x, const void* w, const void* bias, voi
   const int kernel = choose_kernel_out(p, path, x, w, y, &st);
   if (kernel < 0) return st;
   if (N == 0) return GCONV_OK;
+  if (kernel == GCONV_KERNEL_MERGE_MAX_TWO_PASS) {
+    Conv2d q = p;
+    q.out_mode = GCONV_OUT_GROUP_MAJOR;
+    const size_t g_bytes = merge_max_group_major_bytes(p);
+    const size_t stage = p.layout == GCONV_NCHW ? igemm_nchw_workspace(q) : 0;
+    if (workspace == nullptr || workspace_bytes < g_bytes + stage || !aligned16(workspace))
+      return GCONV_ERR_WORKSPACE;
+    const int k1 = p.layout == GCONV_NHWC ? GCONV_KERNEL_IGEMM_TC : GCONV_KERNEL_IGEMM_TC_NCHW;
+    st = launch_forward(k1, q, x, w, bias, workspace, (char*)workspace + g_bytes, stage,
+                        (cudaStream_t)stream);
+    if (st != GCONV_OK) return st;
+    return cuda_status(launch_merge_max_groups(p, workspace, y, (cudaStream_t)stream));
+  }
   if (out_mode_is_plain(p)) p.out_mode = GCONV_OUT_GROUP_MAJOR;
   return launch_forward(kernel, p, x, w, bias, y, workspace, workspace_bytes,
                         (cudaStream_t)stream);

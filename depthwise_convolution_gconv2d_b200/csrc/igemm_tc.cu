@@ -1564,6 +1564,84 @@ cudaError_t launch_nchw_typed(const Conv2d& p, const IgemmParams& P, const void*
   return launch_core<T>(p, P, xt, wt, bias, y, s);
 }
 
+namespace {
+
+// y = the maximum over groups of the group-major output g (both 16-bit): with S = cpg_out
+// (NHWC) or cpg_out * Ho * Wo (NCHW), output element e has outer index e / S and inner index
+// e % S, and reads g[outer * groups * S + j * S + inner] for each group j. VEC: 8 consecutive
+// elements per thread as 16-byte vectors (S % 8 == 0, pointers 16-byte aligned).
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(256) merge_max_groups_kernel(const T* __restrict__ g,
+                                                               T* __restrict__ y, long long n_out,
+                                                               long long S, int groups) {
+  constexpr int V = VEC ? 8 : 1;
+  const long long n_items = n_out / V;
+  for (long long it = (long long)blockIdx.x * blockDim.x + threadIdx.x; it < n_items;
+       it += (long long)gridDim.x * blockDim.x) {
+    const long long e = it * V;
+    const long long outer = e / S, inner = e - outer * S;
+    const T* src = g + outer * groups * S + inner;
+    if constexpr (VEC) {
+      float m[8];
+      uint4 u = *reinterpret_cast<const uint4*>(src);
+      const unsigned int* w = &u.x;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = unpack2<T>(w[q]);
+        m[2 * q] = f.x;
+        m[2 * q + 1] = f.y;
+      }
+      for (int j = 1; j < groups; ++j) {
+        u = *reinterpret_cast<const uint4*>(src + (long long)j * S);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = unpack2<T>(w[q]);
+          m[2 * q] = fmaxf(m[2 * q], f.x);
+          m[2 * q + 1] = fmaxf(m[2 * q + 1], f.y);
+        }
+      }
+      uint4 o;
+      o.x = pack2<T>(make_float2(m[0], m[1]));
+      o.y = pack2<T>(make_float2(m[2], m[3]));
+      o.z = pack2<T>(make_float2(m[4], m[5]));
+      o.w = pack2<T>(make_float2(m[6], m[7]));
+      *reinterpret_cast<uint4*>(y + e) = o;
+    } else {
+      float m = Elem<T>::to_f32(src[0]);
+      for (int j = 1; j < groups; ++j) m = fmaxf(m, Elem<T>::to_f32(src[(long long)j * S]));
+      y[e] = Elem<T>::from_f32(m);
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_merge_max_typed(const Conv2d& p, const void* g, void* y, cudaStream_t s) {
+  const long long S = p.layout == GCONV_NCHW ? (long long)p.cpg_out * p.Ho * p.Wo
+                                             : (long long)p.cpg_out;
+  const long long n_out = (long long)p.N * p.cpg_out * p.Ho * p.Wo;
+  const bool vec = S % 8 == 0 && aligned16(g) && aligned16(y);
+  const long long items = vec ? n_out / 8 : n_out;
+  long long blocks = (items + 255) / 256;
+  const long long cap = (long long)sm_count() * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  if (vec)
+    merge_max_groups_kernel<T, true><<<(unsigned)blocks, 256, 0, s>>>((const T*)g, (T*)y, n_out,
+                                                                       S, p.groups);
+  else
+    merge_max_groups_kernel<T, false><<<(unsigned)blocks, 256, 0, s>>>((const T*)g, (T*)y, n_out,
+                                                                        S, p.groups);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_merge_max_groups(const Conv2d& p, const void* g, void* y, cudaStream_t s) {
+  if (p.dtype == GCONV_BF16) return launch_merge_max_typed<__nv_bfloat16>(p, g, y, s);
+  if (p.dtype == GCONV_F16) return launch_merge_max_typed<__half>(p, g, y, s);
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_nchw_to_nhwc16(const void* x, void* xt, int N, int C, long long HW,
                                   cudaStream_t s) {
   if (HW > INT32_MAX || N > 65535 || (C + 63) / 64 > 65535) return cudaErrorInvalidValue;

@@ -123,6 +123,8 @@ cudaError_t launch_igemm_nchw(const Conv2d& p, const void* x, const void* w, con
 bool igemm_rowt_supported(const Conv2d& p);
 cudaError_t launch_igemm_rowt(const Conv2d& p, const void* x, const void* w, const void* bias,
                               void* y, cudaStream_t s);
+// y (p's MERGE_MAX shape) = the maximum over groups of g, p's group-major output in p.layout.
+cudaError_t launch_merge_max_groups(const Conv2d& p, const void* g, void* y, cudaStream_t s);
 
 // Grouped conv2d backward. dgrad_as_forward: stride 1, square kernel, pad <= dil*(k-1), so the
 // data gradient is the forward conv of the exchanged problem with the flipped, transposed

@@ -141,9 +141,13 @@ typedef enum {
   GCONV_KERNEL_DWSEP2D_FUSED = 21,    /* 2-D depthwise-separable block in one kernel: 16-bit
                                          NHWC, depthwise 3x3 / 5x5, stride 1 / 2, dilation 1,
                                          C % 64 == 0, C_out % 16 == 0 and <= 512 */
-  GCONV_KERNEL_DGRAD_DW3S2_TMA = 22   /* conv2d data gradient, depthwise 3x3, stride 2, pad 1,
+  GCONV_KERNEL_DGRAD_DW3S2_TMA = 22,  /* conv2d data gradient, depthwise 3x3, stride 2, pad 1,
                                          dilation 1, 16-bit NHWC, C % 8 == 0: dy staged by TMA,
                                          dx written by TMA stores */
+  GCONV_KERNEL_MERGE_MAX_TWO_PASS = 23 /* conv2d with the max merge across groups: the
+                                         group-major output in the workspace on the transposed
+                                         row-strip kernel (NCHW: through the NHWC staging), then
+                                         the maximum over groups, 16-byte vectors */
 } gconv_kernel;
 
 /* Order and merging of the output channels ("Grouped convolutions", neon issue #296, ibmua's
@@ -180,13 +184,20 @@ gconv_status gconv2d_out_shape(int N, int C_in, int H, int W, int C_out, int kH,
 /* gconv2d_fwd_path writing the output in `out_mode` (above); y has the shape
  * gconv2d_out_shape reports. The order or the merge is applied in the kernel's epilogue, on
  * the fp32 accumulators (a merge adds or compares the groups' fp32 values, then rounds once),
- * so no second pass over y is made. GROUP_MAJOR, and the modes that equal it (one filter per
- * group for INTERLEAVED, one group for the merges), run exactly as gconv2d_fwd_path. Other
- * variants: AUTO runs the tensor-core implicit GEMM for 16-bit problems it takes (the
- * transposed row-strip kernel for INTERLEAVED where that tiling applies, otherwise the tile
- * kernel; a merge covers all groups of a 16..64-filter block in one tile) and the generic
- * direct kernel otherwise; DIRECT and GENERIC run the generic direct kernel; IGEMM forces
- * the tensor cores (UNSUPPORTED / MISALIGNED as for gconv2d_fwd_path).
+ * so no second pass over y is made -- except for MERGE_MAX on problems that the transposed
+ * row-strip kernel takes (GCONV_KERNEL_MERGE_MAX_TWO_PASS): the group-major output is written
+ * to the workspace, rounded, and a second kernel takes the maximum over groups; rounding is
+ * monotonic, so the maximum of the rounded values is the rounded maximum, bit for bit the
+ * one-pass result. GROUP_MAJOR, and the modes that equal it (one filter per group for
+ * INTERLEAVED, one group for the merges), run exactly as gconv2d_fwd_path. Other variants:
+ * AUTO runs the tensor-core implicit GEMM for 16-bit problems it takes (the transposed
+ * row-strip kernel for INTERLEAVED and MERGE_AVG where that tiling applies, the two passes
+ * above for MERGE_MAX, otherwise the tile kernel; a merge there covers all groups of a
+ * 16..64-filter block in one tile) and the generic direct kernel otherwise; DIRECT and
+ * GENERIC run the generic direct kernel; IGEMM forces the tensor cores (UNSUPPORTED /
+ * MISALIGNED as for gconv2d_fwd_path). The workspace (16-byte aligned) holds the two-pass
+ * group-major output (N * C_out * Ho * Wo elements) and, for NCHW tensor-core runs, the NHWC
+ * staging; gconv2d_fwd_out_workspace_size reports it.
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
 gconv_status gconv2d_fwd_out(const void* x, const void* w, const void* bias, void* y, int N,
                              int C_in, int H, int W, int C_out, int kH, int kW, int stride,

@@ -150,6 +150,47 @@ def _sample(p, n, seed, channels):
                      r.integers(0, p.Wo, n)], 1)
 
 
+# The max merge in two passes (the transposed row-strip kernel writes the group-major output
+# to the workspace, then the maximum over groups): problems that tiling takes (64 input
+# channels a group or a multiple, 128 filters a group or a multiple, rows of >= 128 outputs).
+MAX_TWO_PASS = [
+    # N, C_in, H, W, C_out, k, pad, groups
+    (1, 128, 4, 136, 256, 3, 1, 2),
+    (2, 256, 3, 130, 512, 3, 1, 4),
+    (1, 192, 5, 128, 384, 3, 2, 3),
+]
+
+
+@pytest.mark.parametrize("case", MAX_TWO_PASS)
+@pytest.mark.parametrize("layout", [wl.NHWC, wl.NCHW])
+@pytest.mark.parametrize("dtype", [wl.BF16, wl.F16])
+def test_max_merge_two_pass(case, layout, dtype):
+    N, C_in, H, W, C_out, k, pad, g = case
+    p = wl.Conv2dProblem(N, C_in, H, W, C_out, k, k, 1, pad, 1, g, layout, dtype, True)
+    assert kernel_of(p, "max") == 23 and kernel_of(p, "max", gb.PATH_IGEMM) == 23
+    assert kernel_of(p, "max", gb.PATH_DIRECT) == 1
+    assert gb.load_library().gconv2d_fwd_out_workspace_size(
+        N, C_in, H, W, C_out, k, k, 1, pad, 1, g, layout, dtype, 3, 0) >= \
+        N * C_out * p.Ho * p.Wo * 2
+    inp = wl.make_conv2d_inputs(p, 61)
+    y = run_out(inp, "max")
+    assert gb.device_error() == 0
+    assert_close(to_f64(y), oracle_out(inp, "max"), p.dtype, f"{case} {layout}")
+
+
+def test_max_merge_two_pass_integer_bit_exact():
+    """Ternary x and sparse ternary filters (at most 255 non-zero taps): every group's sum is
+    an exact integer below 256, so the maximum over groups is exact and equals the oracle's."""
+    p = wl.Conv2dProblem(1, 128, 4, 136, 256, 3, 3, 1, 1, 1, 2, wl.NHWC, wl.BF16, False)
+    r = np.random.default_rng(62)
+    inp = wl.make_conv2d_inputs(p, 62)
+    w = r.integers(-1, 2, p.w_shape) * (r.random(p.w_shape) < 1 / 8)
+    assert np.abs(w).reshape(p.C_out, -1).sum(axis=1).max() <= 255
+    inp.x = wl.to_storage(r.integers(-1, 2, p.x_shape), wl.BF16)
+    inp.w = wl.to_storage(w, wl.BF16)
+    assert np.array_equal(to_f64(run_out(inp, "max")), oracle_out(inp, "max"))
+
+
 @pytest.mark.parametrize("mode", MODES)
 def test_variants_wide_group_layer_sampled(mode):
     """The wide-group layer x[1,512,256,256] * w[512,128,3,3], groups 4 (NHWC), in each
