@@ -990,11 +990,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // (8 consecutive channels of one pixel) are 16-byte vectors; the transposition itself is done
 // with 2-byte shared-memory accesses (row pitch 66 elements against bank conflicts).
 template <typename T, bool VEC>
-__global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const T* __restrict__ x,
-                                                           T* __restrict__ xt, int C, int HW) {
-  __shared__ unsigned short tile[64][66];   // [c][hw]
-  const int n = blockIdx.z;
-  const int c0 = blockIdx.y * 64, s0 = blockIdx.x * 64;
+__device__ __forceinline__ void nchw_to_nhwc_tile(const T* __restrict__ x, T* __restrict__ xt,
+                                                  int C, int HW, int n, int c0, int s0,
+                                                  unsigned short (*tile)[66]) {
   const unsigned short* xn = reinterpret_cast<const unsigned short*>(x) + (long long)n * C * HW;
   unsigned short* tn = reinterpret_cast<unsigned short*>(xt) + (long long)n * C * HW;
   const int tid = threadIdx.x;
@@ -1050,23 +1048,59 @@ __global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const T* __restrict__
   }
 }
 
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const T* __restrict__ x,
+                                                           T* __restrict__ xt, int C, int HW) {
+  __shared__ unsigned short tile[64][66];   // [c][hw]
+  nchw_to_nhwc_tile<T, VEC>(x, xt, C, HW, blockIdx.z, blockIdx.y * 64, blockIdx.x * 64, tile);
+}
+
 // w[co][ci][kh][kw] -> wt[co][kh][kw][ci] for filters of at most 8192 elements: one CTA per
 // filter reads it with coalesced loads into shared memory and writes it back tap-major with
 // coalesced stores.
 template <typename T>
-__global__ void __launch_bounds__(256) repack_weight_smem_kernel(const T* __restrict__ w,
-                                                                 T* __restrict__ wt, int cpg_in,
-                                                                 int taps) {
-  __shared__ unsigned short buf[8192];
+__device__ __forceinline__ void repack_filter(const T* __restrict__ w, T* __restrict__ wt,
+                                              int cpg_in, int taps, int f, unsigned short* buf) {
   const int n = cpg_in * taps;
-  const unsigned short* src = reinterpret_cast<const unsigned short*>(w) + (long long)blockIdx.x * n;
-  unsigned short* dst = reinterpret_cast<unsigned short*>(wt) + (long long)blockIdx.x * n;
+  const unsigned short* src = reinterpret_cast<const unsigned short*>(w) + (long long)f * n;
+  unsigned short* dst = reinterpret_cast<unsigned short*>(wt) + (long long)f * n;
   for (int i = threadIdx.x; i < n; i += blockDim.x) buf[i] = src[i];
   __syncthreads();
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const int tap = i / cpg_in, ci = i - tap * cpg_in;
     dst[i] = buf[ci * taps + tap];
   }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) repack_weight_smem_kernel(const T* __restrict__ w,
+                                                                 T* __restrict__ wt, int cpg_in,
+                                                                 int taps) {
+  __shared__ unsigned short buf[8192];
+  repack_filter<T>(w, wt, cpg_in, taps, blockIdx.x, buf);
+}
+
+// The NCHW staging in one launch: blocks [0, C_out) repack one filter each (as above), blocks
+// from C_out on transpose one 64 x 64 tile of x (tile b -> pixel block b % gx, channel block
+// (b / gx) % gy, image b / (gx * gy)). The repack is latency-bound (~8 us on its own for the
+// 1.2 MB of the wide-group layer's weights, measured) and now runs beside the transpose.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(256) nchw_stage_kernel(const T* __restrict__ x,
+                                                         T* __restrict__ xt, int C, int HW,
+                                                         unsigned int gx, unsigned int gy,
+                                                         const T* __restrict__ w,
+                                                         T* __restrict__ wt, int C_out,
+                                                         int cpg_in, int taps) {
+  __shared__ __align__(16) unsigned short smem[8192];   // a filter, or a [64][66] tile
+  const unsigned int b = blockIdx.x;
+  if (b < (unsigned int)C_out) {
+    repack_filter<T>(w, wt, cpg_in, taps, (int)b, smem);
+    return;
+  }
+  const unsigned int t = b - (unsigned int)C_out;
+  const unsigned int bx = t % gx, r = t / gx;
+  nchw_to_nhwc_tile<T, VEC>(x, xt, C, HW, (int)(r / gy), (int)(r % gy) * 64, (int)bx * 64,
+                            reinterpret_cast<unsigned short (*)[66]>(smem));
 }
 
 // w[co][ci][kh][kw] -> wt[co][kh][kw][ci]
@@ -1543,6 +1577,21 @@ cudaError_t launch_nchw_typed(const Conv2d& p, const IgemmParams& P, const void*
   T* wt = (T*)((char*)workspace + align256((size_t)p.N * p.H * p.W * p.C_in * 2));
   const int taps = p.kH * p.kW;
   const int per_filter = p.cpg_in * taps;
+  const int HW = p.H * p.W;
+  const unsigned int gx = (unsigned int)((HW + 63) / 64), gy = (unsigned int)((p.C_in + 63) / 64);
+  const long long stage_blocks = (long long)p.C_out + (long long)gx * gy * p.N;
+  if (per_filter <= 8192 && stage_blocks <= INT32_MAX) {
+    // weights and activations staged by one launch
+    if (HW % 8 == 0 && p.C_in % 8 == 0 && aligned16(x))
+      nchw_stage_kernel<T, true><<<(unsigned)stage_blocks, 256, 0, s>>>(
+          (const T*)x, xt, p.C_in, HW, gx, gy, (const T*)w, wt, p.C_out, p.cpg_in, taps);
+    else
+      nchw_stage_kernel<T, false><<<(unsigned)stage_blocks, 256, 0, s>>>(
+          (const T*)x, xt, p.C_in, HW, gx, gy, (const T*)w, wt, p.C_out, p.cpg_in, taps);
+    const cudaError_t e0 = cudaGetLastError();
+    if (e0 != cudaSuccess) return e0;
+    return launch_core<T>(p, P, xt, wt, bias, y, s);
+  }
   if (per_filter <= 8192) {
     repack_weight_smem_kernel<T><<<(unsigned)p.C_out, 256, 0, s>>>((const T*)w, wt, p.cpg_in,
                                                                    taps);
@@ -1553,7 +1602,6 @@ cudaError_t launch_nchw_typed(const Conv2d& p, const IgemmParams& P, const void*
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int HW = p.H * p.W;
   dim3 grid((HW + 63) / 64, (p.C_in + 63) / 64, p.N);
   if (HW % 8 == 0 && p.C_in % 8 == 0 && aligned16(x))
     nchw_to_nhwc_kernel<T, true><<<grid, 256, 0, s>>>((const T*)x, xt, p.C_in, HW);
