@@ -70,6 +70,50 @@ __global__ void __launch_bounds__(256) flip_transpose_weight_kernel(const T* __r
   }
 }
 
+// The NHWC case as a tiled transpose: w is [C_out][kH][kW][cpg_in], so per group g the
+// [cpg_out] x [kH * kW * cpg_in] block of w (row col, column e = tap * cpg_in + ci, contiguous)
+// becomes rows (ci, reversed tap) x columns col of wt; 64 x 64 tiles through shared memory, so both the loads (along e) and the
+// stores (along col) are contiguous. (The element-wise gather above, one 2-byte load per
+// output from filters 2.3 KB apart, took several microseconds for the wide-group layer's
+// 1.2 MB of weights.)
+template <typename T>
+__global__ void __launch_bounds__(256) flip_weight_nhwc_tiled_kernel(const T* __restrict__ w,
+                                                                      T* __restrict__ wt,
+                                                                      int cpg_in, int cpg_out,
+                                                                      int taps) {
+  __shared__ unsigned short tile[64][66];
+  const unsigned short* ws = reinterpret_cast<const unsigned short*>(w);
+  unsigned short* wd = reinterpret_cast<unsigned short*>(wt);
+  const int g = blockIdx.z, e0 = blockIdx.x * 64, c0 = blockIdx.y * 64;
+  const long long E = (long long)cpg_in * taps;
+  const unsigned short* src = ws + (long long)g * cpg_out * E;
+  // a thread's 16 loads are issued before any of them is stored (a load -> store chain per
+  // element left each thread waiting out 16 DRAM latencies: 12 us for 1.2 MB, measured)
+  unsigned short v[16];
+#pragma unroll
+  for (int it = 0; it < 16; ++it) {
+    const int i = threadIdx.x + 256 * it;
+    const int r = i >> 6, q = i & 63;              // r: filter col, q: e (contiguous)
+    const int col = c0 + r, e = e0 + q;
+    v[it] = (col < cpg_out && e < E) ? src[(long long)col * E + e] : (unsigned short)0;
+  }
+#pragma unroll
+  for (int it = 0; it < 16; ++it) {
+    const int i = threadIdx.x + 256 * it;
+    tile[i >> 6][i & 63] = v[it];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 64 * 64; i += 256) {
+    const int q = i >> 6, r = i & 63;              // r: filter col (contiguous in wt)
+    const int col = c0 + r, e = e0 + q;
+    if (col < cpg_out && e < E) {
+      const int tap = e / cpg_in, ci = e - tap * cpg_in;
+      const long long c = (long long)g * cpg_in + ci;
+      wd[(c * taps + (taps - 1 - tap)) * cpg_out + col] = tile[r][q];
+    }
+  }
+}
+
 // ------------------------------------------------------------------ generic data gradient
 // One thread per dx element (decoded in dx's memory order, so stores are contiguous); fp32
 // FMA over the group's output channels and the taps whose window reads this input.
@@ -898,6 +942,15 @@ unsigned grid_for(long long total, int threads) {
 template <typename T>
 cudaError_t flip_typed(const Conv2d& p, const void* w, void* wt, cudaStream_t s) {
   const long long total = (long long)p.C_out * p.cpg_in * p.kH * p.kW;
+  const long long E = (long long)p.cpg_in * p.kH * p.kW;
+  if (p.layout == GCONV_NHWC && sizeof(T) == 2 && (E + 63) / 64 <= INT32_MAX &&
+      (p.cpg_out + 63) / 64 <= 65535 && p.groups <= 65535) {
+    const dim3 grid((unsigned)((E + 63) / 64), (unsigned)((p.cpg_out + 63) / 64),
+                    (unsigned)p.groups);
+    flip_weight_nhwc_tiled_kernel<T><<<grid, 256, 0, s>>>((const T*)w, (T*)wt, p.cpg_in,
+                                                          p.cpg_out, p.kH * p.kW);
+    return cudaGetLastError();
+  }
   if (p.layout == GCONV_NHWC)
     flip_transpose_weight_kernel<T, GCONV_NHWC><<<grid_for(total, 256), 256, 0, s>>>(
         (const T*)w, (T*)wt, p, total);
