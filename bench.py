@@ -103,6 +103,8 @@ def compact_rooflines(dwm, more, bwd, extra=None):
         if k.startswith("dw1d_") and k.endswith("_cudacore"):
             continue
         out[f"{names.get(k, k)}_hbm"] = v["frac"]
+        if "frac_b2b" in v:
+            out[f"{names.get(k, k)}_b2b_hbm"] = v["frac_b2b"]
     for k, v in (more or {}).items():
         if "_direct" in k and v.get("us", 0) > 5000:
             continue
@@ -236,6 +238,36 @@ def time_launches(torch, fn, stream, reps, flush=None):
         b.synchronize()
         times.append(a.elapsed_time(b))
     return statistics.median(times), sum(times) / len(times)
+
+
+def time_graph_b2b(torch, fn, stream, n_sets, launches=32, reps=5):
+    """Per-launch CUDA-event time (ms) of `launches` back-to-back launches of `fn(i)`, i cycling
+    over `n_sets` buffer sets whose combined size exceeds 2x L2 (a launch reads inputs that 7
+    others have evicted since it last touched them), captured in one CUDA graph and replayed
+    after a spin; median over `reps` replays. A single launch after a spin also pays the idle
+    stream's launch latency (~6 us for an empty kernel on B200, against ~1 us per launch inside
+    a graph), which dominates kernels whose HBM floor is a few microseconds."""
+    with torch.cuda.stream(stream):
+        for i in range(n_sets):
+            fn(i)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(launches):
+            fn(i % n_sets)
+    times = []
+    for _ in range(reps):
+        gpu_spin(torch, stream, 400)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b) / launches)
+    del g
+    return statistics.median(times)
 
 
 # ---------------------------------------------------------------------------- workloads
@@ -372,9 +404,16 @@ def depthwise_measurements(torch, gb, device, stream, pk, reps):
     for causal in (False, True):
         p = wl.conformer_dw1d(causal)
         inp = wl.make_dwconv1d_inputs(p, 3)
-        x, w, dy = (dev_tensor(torch, a, p.dtype, device) for a in (inp.x, inp.w, inp.dy))
-        y = torch.empty((p.B, p.T_out, p.C), dtype=torch.bfloat16, device=device)
-        dx = torch.empty((p.B, p.T, p.C), dtype=torch.bfloat16, device=device)
+        # 8 buffer sets (x, dy, y, dx: 537 MB > 2x L2) for the back-to-back figure; the
+        # single-launch figure uses set 0
+        n_sets = 8
+        w = dev_tensor(torch, inp.w, p.dtype, device)
+        xs = [dev_tensor(torch, inp.x, p.dtype, device) for _ in range(n_sets)]
+        dys = [dev_tensor(torch, inp.dy, p.dtype, device) for _ in range(n_sets)]
+        ys = [torch.empty((p.B, p.T_out, p.C), dtype=torch.bfloat16, device=device)
+              for _ in range(n_sets)]
+        dxs = [torch.empty((p.B, p.T, p.C), dtype=torch.bfloat16, device=device)
+               for _ in range(n_sets)]
         dw = torch.empty((p.C, p.K), dtype=torch.bfloat16, device=device)
         need = gb.dwconv1d_bwd_weight_workspace_size(p.B, p.T, p.C, p.K, p.pad_left, p.pad_right,
                                                      p.dtype)
@@ -382,28 +421,35 @@ def depthwise_measurements(torch, gb, device, stream, pk, reps):
         sel = lambda path: gb.KERNEL_NAMES.get(gb.dwconv1d_select_path(
             p.B, p.T, p.C, p.K, p.pad_left, p.pad_right, p.dtype, path), "?")
         ops = {
-            "fwd": (lambda i: gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right, out=y,
+            "fwd": (lambda i: gb.dwconv1d_fwd(xs[i], w, p.pad_left, p.pad_right, out=ys[i],
                                               stream=stream), sel(gb.PATH_AUTO)),
-            "dgrad": (lambda i: gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right, out=dx,
-                                                     stream=stream), sel(gb.PATH_AUTO)),
-            "wgrad": (lambda i: gb.dwconv1d_bwd_weight(x, dy, p.K, p.pad_left, p.pad_right,
-                                                       out=dw, workspace=ws, stream=stream),
+            "dgrad": (lambda i: gb.dwconv1d_bwd_data(dys[i], w, p.T, p.pad_left, p.pad_right,
+                                                     out=dxs[i], stream=stream),
+                      sel(gb.PATH_AUTO)),
+            "wgrad": (lambda i: gb.dwconv1d_bwd_weight(xs[i], dys[i], p.K, p.pad_left,
+                                                       p.pad_right, out=dw, workspace=ws,
+                                                       stream=stream),
                       "conv1d_wgrad"),
-            # the CUDA-core ring kernel on the same problem, for comparison
-            "fwd_cudacore": (lambda i: gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right, out=y,
-                                                       stream=stream, path=gb.PATH_DIRECT),
-                             "conv1d_ring"),
+            # the CUDA-core kernel of the DIRECT family on the same problem, for comparison
+            "fwd_cudacore": (lambda i: gb.dwconv1d_fwd(xs[i], w, p.pad_left, p.pad_right,
+                                                       out=ys[i], stream=stream,
+                                                       path=gb.PATH_DIRECT),
+                             sel(gb.PATH_DIRECT)),
         }
         tag = "causal" if causal else "same"
         for op, (fn, kname) in ops.items():
             for _ in range(3):
                 fn(0)
-            med, mean = time_launches(torch, fn, stream, reps, flush)
+            med, mean = time_launches(torch, lambda i: fn(0), stream, reps, flush)
+            b2b = time_graph_b2b(torch, fn, stream, n_sets)
             ab = p.bytes(op.split("_")[0])
             gbs = ab / (med * 1e-3) / 1e9
+            gbs_b2b = ab / (b2b * 1e-3) / 1e9
             out[f"dw1d_{tag}_{op}"] = {"kernel": kname, "us": round(med * 1e3, 2),
                                        "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 3),
-                                       "alg_bytes": ab}
+                                       "us_b2b": round(b2b * 1e3, 2),
+                                       "frac_b2b": round(gbs_b2b / hbm, 3), "alg_bytes": ab}
+        del xs, dys, ys, dxs
     return out
 
 
@@ -606,7 +652,7 @@ def config_dict(p, args):
 # ---------------------------------------------------------------------------- main
 
 PROFILE_WORKLOADS = ("wide_group_nhwc", "wide_group_nchw", "ensemble_g64", "depthwise56_s1",
-                     "depthwise56_s2", "dw1d_same", "sweep56_g64", "sweep56_g16",
+                     "depthwise56_s2", "dw1d_same", "dw1d_same_direct", "sweep56_g64", "sweep56_g16",
                      "depthwise56_bwd", "depthwise56_s2_bwd", "wide_group_dgrad",
                      "wide_group_wgrad", "dwsep1d", "grouped_linear", "wide_group_avg")
 
@@ -618,7 +664,14 @@ def run_profile(name: str, reps: int, batch: int = 0) -> int:
 
     from depthwise_convolution_gconv2d_b200 import binding as gb
     device = torch.device("cuda", 0)
-    if name == "dw1d_same":
+    if name == "dw1d_same_direct":
+        # the forward on the CUDA-core 128-byte-row kernel (the DIRECT family)
+        p = wl.conformer_dw1d(False)
+        inp = wl.make_dwconv1d_inputs(p, 3)
+        x, w = (dev_tensor(torch, a, p.dtype, device) for a in (inp.x, inp.w))
+        for _ in range(reps):
+            gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right, path=gb.PATH_DIRECT)
+    elif name == "dw1d_same":
         p = wl.conformer_dw1d(False)
         inp = wl.make_dwconv1d_inputs(p, 3)
         x, w, dy = (dev_tensor(torch, a, p.dtype, device) for a in (inp.x, inp.w, inp.dy))

@@ -601,6 +601,8 @@ gconv_status gconv2d_bwd_data_path(const void* dy, const void* w, void* dx, int 
     return cuda_status(launch_dgrad_depthwise(p, dy, w, dx, s));
   if (kernel == GCONV_KERNEL_DGRAD_DW3S2_TMA)
     return cuda_status(launch_dgrad_dw3s2_tma(p, dy, w, dx, s));
+  if (kernel == GCONV_KERNEL_DEPTHWISE_NHWC && depthwise_nhwc_flipped_supported(q))
+    return cuda_status(launch_depthwise_nhwc_flipped(q, dy, w, dx, s));
   st = cuda_status(launch_flip_transpose_weight(p, w, workspace, s));
   if (st != GCONV_OK) return st;
   const size_t off = round_up(weight_bytes(p), 256);

@@ -943,8 +943,11 @@ template <typename T>
 cudaError_t flip_typed(const Conv2d& p, const void* w, void* wt, cudaStream_t s) {
   const long long total = (long long)p.C_out * p.cpg_in * p.kH * p.kW;
   const long long E = (long long)p.cpg_in * p.kH * p.kW;
-  if (p.layout == GCONV_NHWC && sizeof(T) == 2 && (E + 63) / 64 <= INT32_MAX &&
-      (p.cpg_out + 63) / 64 <= 65535 && p.groups <= 65535) {
+  // the tiled transpose where its 64 x 64 tiles are mostly full (wide groups); narrow groups
+  // (a depthwise filter is 9 elements) keep the element-wise kernel, which launches no
+  // mostly idle tiles
+  if (p.layout == GCONV_NHWC && sizeof(T) == 2 && p.cpg_out >= 32 && E >= 32 &&
+      (E + 63) / 64 <= INT32_MAX && (p.cpg_out + 63) / 64 <= 65535 && p.groups <= 65535) {
     const dim3 grid((unsigned)((E + 63) / 64), (unsigned)((p.cpg_out + 63) / 64),
                     (unsigned)p.groups);
     flip_weight_nhwc_tiled_kernel<T><<<grid, 256, 0, s>>>((const T*)w, (T*)wt, p.cpg_in,

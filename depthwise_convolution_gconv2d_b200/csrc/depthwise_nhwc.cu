@@ -153,6 +153,7 @@ struct Dw3Params {
   int BW, IW, IH;                          // output tile columns; input box columns and rows
   int n_ct, n_wt, n_ht, num_tiles, stages;
   unsigned int stage_bytes, tx_bytes;
+  int flip;   // 1: read each 3x3 filter rotated by 180 degrees (the data gradient)
 };
 
 // Tile coordinates, channel tile slowest: tw -> th -> n -> ct. A CTA walks a contiguous chunk
@@ -271,10 +272,12 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
 #pragma unroll
         for (int kh = 0; kh < 3; ++kh)
 #pragma unroll
-          for (int kw = 0; kw < 3; ++kw)
-            wv[kh][kw] = ch_ok ? make_float2(Elem<T>::to_f32(w[ch * 9 + kh * 3 + kw]),
-                                             Elem<T>::to_f32(w[(ch + 1) * 9 + kh * 3 + kw]))
+          for (int kw = 0; kw < 3; ++kw) {
+            const int tp = P.flip ? 8 - (kh * 3 + kw) : kh * 3 + kw;
+            wv[kh][kw] = ch_ok ? make_float2(Elem<T>::to_f32(w[ch * 9 + tp]),
+                                             Elem<T>::to_f32(w[(ch + 1) * 9 + tp]))
                                : make_float2(0.f, 0.f);
+          }
         bv = (bias && ch_ok) ? make_float2(Elem<T>::to_f32(bias[ch]), Elem<T>::to_f32(bias[ch + 1]))
                              : make_float2(0.f, 0.f);
       }
@@ -336,8 +339,9 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
 
 template <typename T, int S, int BH>
 cudaError_t launch_dw3_tma(const Conv2d& p, const void* x, const void* w, const void* bias,
-                           void* y, cudaStream_t s) {
+                           void* y, cudaStream_t s, bool flip = false) {
   Dw3Params P;
+  P.flip = flip ? 1 : 0;
   P.N = p.N; P.H = p.H; P.W = p.W; P.C = p.C_in; P.Ho = p.Ho; P.Wo = p.Wo; P.pad = p.pad;
   P.BW = DW3_BW;
   P.IW = DW3_IW<S>();
@@ -479,6 +483,17 @@ cudaError_t launch_depthwise_nhwc(const Conv2d& p, const void* x, const void* w,
                                   const void* bias, void* y, cudaStream_t s) {
   if (p.dtype == GCONV_F16) return launch_typed<__half>(p, x, w, bias, y, s);
   return launch_typed<__nv_bfloat16>(p, x, w, bias, y, s);
+}
+
+bool depthwise_nhwc_flipped_supported(const Conv2d& p) {
+  return depthwise_nhwc_supported(p) && dw3_tma_eligible(p) && p.stride == 1;
+}
+
+cudaError_t launch_depthwise_nhwc_flipped(const Conv2d& p, const void* x, const void* w, void* y,
+                                          cudaStream_t s) {
+  if (!depthwise_nhwc_flipped_supported(p)) return cudaErrorInvalidValue;
+  if (p.dtype == GCONV_F16) return launch_dw3_tma<__half, 1, 8>(p, x, w, nullptr, y, s, true);
+  return launch_dw3_tma<__nv_bfloat16, 1, 8>(p, x, w, nullptr, y, s, true);
 }
 
 }  // namespace gconv

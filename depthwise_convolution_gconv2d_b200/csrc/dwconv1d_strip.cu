@@ -96,18 +96,22 @@ __global__ void __launch_bounds__(SP_THREADS, 2)
     prefetch_tmap(&tmx);
     prefetch_tmap(&tmy);
   }
-  // the block's taps, read once with coalesced loads and kept as fp32 pairs [tap][pair]
-  // (reversed for the data gradient), so a lane's K pairs are conflict-free 8-byte loads
-  {
+  __syncthreads();
+  if (warp != 0) {
+    // the compute warps lay out the block's taps as fp32 pairs [tap][pair] (reversed for the
+    // data gradient) while the producer already streams the first tiles; consecutive threads
+    // write consecutive channels, so the table is written without bank conflicts (a
+    // channel-major walk of w wrote 32 threads into one bank and held every CTA ~3 us before
+    // its first load was issued, measured)
     const T* wb = w + (long long)run.cb * SP_CB * K;
     float* wf = reinterpret_cast<float*>(wsm);
-    for (int e = threadIdx.x; e < SP_CB * K; e += SP_THREADS) {
-      const int c = e / K, k = e - c * K;
+    for (int e = threadIdx.x - 32; e < SP_CB * K; e += SP_THREADS - 32) {
+      const int k = e / SP_CB, c = e - k * SP_CB;
       const int kk = FLIP ? K - 1 - k : k;
-      wf[(kk * 32 + (c >> 1)) * 2 + (c & 1)] = Elem<T>::to_f32(wb[e]);
+      wf[(kk * 32 + (c >> 1)) * 2 + (c & 1)] = Elem<T>::to_f32(wb[c * K + k]);
     }
+    named_sync(1, SP_THREADS - 32);
   }
-  __syncthreads();
 
   if (warp == 0) {
     if (lane == 0) {

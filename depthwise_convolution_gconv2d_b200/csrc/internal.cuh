@@ -105,6 +105,12 @@ cudaError_t launch_direct_generic(const Conv2d& p, const void* x, const void* w,
 bool depthwise_nhwc_supported(const Conv2d& p);
 cudaError_t launch_depthwise_nhwc(const Conv2d& p, const void* x, const void* w,
                                   const void* bias, void* y, cudaStream_t s);
+// The stride-1 3x3 depthwise kernel reading each filter rotated by 180 degrees: the data
+// gradient of a stride-1 depthwise layer as a forward pass over dy, with no flipped copy of
+// the filter.
+bool depthwise_nhwc_flipped_supported(const Conv2d& p);
+cudaError_t launch_depthwise_nhwc_flipped(const Conv2d& p, const void* x, const void* w, void* y,
+                                          cudaStream_t s);
 
 // Narrow groups (2 / 4 / 8 channels per group), 3x3, NHWC, 16-bit, C % 8 == 0, aligned x, y.
 bool grouped_nhwc_supported(const Conv2d& p);
