@@ -825,8 +825,9 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    # one launch per step and no events between the steps (an event recorded between two
+    # launches kept the next one from starting until the first had fully drained: ~5 us a
+    # launch, measured), so the kernel's average launch duration is the region's time / K
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
@@ -834,21 +835,19 @@ def main():
         gpu_spin(torch, stream, 500)
         t_start.record(stream)
         for i in range(args.steps):
-            ev[i][0].record(stream)
             step(i)
-            ev[i][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
         time.sleep(0.25)
     total_ms = t_start.elapsed_time(t_end)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    local_ms = total_ms
     if world > 1:
         total_ms = max_over_ranks(torch, dist, total_ms, device)
         dist.barrier()
 
     flops = p.flops()
     value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
-    avg_launch_ms = sum(launch_ms) / len(launch_ms)
+    avg_launch_ms = local_ms / args.steps
     achieved = flops / (avg_launch_ms * 1e-3) / 1e12
     clocks = clk.summary()
     tensor_peak, which = tensor_peak_for(pk, total_ms * 1e-3, clocks)

@@ -218,6 +218,9 @@ __global__ void __launch_bounds__(DW3_THREADS, 2)
     prefetch_tmap(&tmy);
   }
   __syncthreads();
+  // the setup above may overlap the previous kernel in the stream (launch_pdl)
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -407,9 +410,8 @@ cudaError_t launch_dw3_tma(const Conv2d& p, const void* x, const void* w, const 
   if (fit > per_sm) fit = per_sm;
   long long grid = (long long)sm_count() * fit;
   if (grid > P.num_tiles) grid = P.num_tiles;
-  dw3x3_tma_kernel<T, S, BH><<<(unsigned)grid, threads, smem, s>>>(
-      tm, tmy, (const T*)w, (const T*)bias, P, device_error_word());
-  return cudaGetLastError();
+  return launch_pdl(dw3x3_tma_kernel<T, S, BH>, (unsigned)grid, (unsigned)threads, smem, s, tm,
+                    tmy, (const T*)w, (const T*)bias, P, device_error_word());
 }
 
 bool dw3_tma_eligible(const Conv2d& p) {

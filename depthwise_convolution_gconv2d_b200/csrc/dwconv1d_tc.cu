@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const unsigned int tmem_base = *tmem_slot;
+  // the setup above may overlap the previous kernel in the stream (launch_pdl)
+  pdl_wait();
+  pdl_launch_dependents();
 
   unsigned char* xs = smem;
   unsigned char* ws = smem + L.ws_off;
@@ -416,9 +419,8 @@ cudaError_t launch_tc(const Conv1d& p, const void* x, const void* w, void* y, in
   if (e != cudaSuccess) return e;
   long long grid = sm_count();
   if (grid > P.num_tiles) grid = P.num_tiles;
-  dwconv1d_tc_kernel<T, KS, FLIP><<<(unsigned)grid, TC_THREADS, smem, s>>>(
-      tmx, tmy, (const T*)w, P, device_error_word());
-  return cudaGetLastError();
+  return launch_pdl(dwconv1d_tc_kernel<T, KS, FLIP>, (unsigned)grid, TC_THREADS, smem, s, tmx,
+                    tmy, (const T*)w, P, device_error_word());
 }
 
 template <typename T, bool FLIP>

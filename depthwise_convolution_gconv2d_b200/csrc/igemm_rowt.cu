@@ -110,6 +110,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const unsigned int tmem_base = *tmem_slot;
+  // the setup above may overlap the previous kernel in the stream (launch_pdl)
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -344,6 +347,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const unsigned int tmem_base = *tmem_slot;
+  // the setup above may overlap the previous kernel in the stream (launch_pdl)
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -634,12 +640,10 @@ cudaError_t launch_rowt(const Conv2d& p, const RowTParams& R, const void* x, con
   int grid = sm_count();
   if (grid > R.num_tiles) grid = R.num_tiles;
   if (avg)
-    igemm_rowt_avg_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, txh, tw, (const T*)bias, (T*)y,
-                                                             R, device_error_word());
-  else
-    igemm_rowt_kernel<T><<<grid, NUM_THREADS, smem, s>>>(tx, txh, tw, (const T*)bias, (T*)y, R,
-                                                         device_error_word());
-  return cudaGetLastError();
+    return launch_pdl(igemm_rowt_avg_kernel<T>, (unsigned)grid, NUM_THREADS, smem, s, tx, txh,
+                      tw, (const T*)bias, (T*)y, R, device_error_word());
+  return launch_pdl(igemm_rowt_kernel<T>, (unsigned)grid, NUM_THREADS, smem, s, tx, txh, tw,
+                    (const T*)bias, (T*)y, R, device_error_word());
 }
 
 }  // namespace

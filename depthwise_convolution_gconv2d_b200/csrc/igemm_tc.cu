@@ -521,6 +521,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const unsigned int tmem_base = *tmem_slot;
+  // the setup above may overlap the previous kernel in the stream (launch_pdl)
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -1457,12 +1460,10 @@ cudaError_t launch_halo(const Conv2d& p, const HaloParams& H, const void* x, con
   int grid = sm_count();
   if (grid > H.num_tiles) grid = H.num_tiles;
   if (H.gp > 1)
-    igemm_halo_kernel<T, true><<<grid, NUM_THREADS, smem, s>>>(tx, tw, ty, (const T*)bias,
-                                                               (T*)y, H, device_error_word());
-  else
-    igemm_halo_kernel<T, false><<<grid, NUM_THREADS, smem, s>>>(tx, tw, ty, (const T*)bias,
-                                                                (T*)y, H, device_error_word());
-  return cudaGetLastError();
+    return launch_pdl(igemm_halo_kernel<T, true>, (unsigned)grid, NUM_THREADS, smem, s, tx, tw,
+                      ty, (const T*)bias, (T*)y, H, device_error_word());
+  return launch_pdl(igemm_halo_kernel<T, false>, (unsigned)grid, NUM_THREADS, smem, s, tx, tw, ty,
+                    (const T*)bias, (T*)y, H, device_error_word());
 }
 
 // A 1x1, stride-1, unpadded convolution is one GEMM over all pixels. With NHWC pixels (or one

@@ -225,6 +225,25 @@ int sm_count();                       // SMs of the current device (cached)
 // tile kernel's producer declares to its barrier; 0 unless a test set it.
 unsigned int debug_tx_surplus();
 
+// Launch with programmatic stream serialization: the kernel may start before the previous
+// kernel in the stream has finished (its setup overlapping that kernel's tail) and must call
+// ptx::pdl_wait() before its first global-memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned int grid, unsigned int block,
+                       size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Device error word (set by kernels whose bounded waits give up).
 cudaError_t read_and_clear_device_error(cudaStream_t s, int* code);
 unsigned int* device_error_word();

@@ -272,5 +272,13 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned i
       : "memory");
 }
 
+// Programmatic dependent launch (kernels launched by launch_pdl): wait until the previous
+// kernel in the stream has completed and its memory is visible -- call before the first access
+// to global memory -- and let the next kernel's CTAs be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace ptx
 }  // namespace gconv
