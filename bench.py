@@ -109,12 +109,16 @@ def compact_rooflines(dwm, more, bwd, extra=None):
         if "_direct" in k and v.get("us", 0) > 5000:
             continue
         out[f"{k}_{v['bound']}"] = v["frac"]
+        if "frac_b2b" in v:
+            out[f"{k}_b2b_{v['bound']}"] = v["frac_b2b"]
         if "ffma_frac" in v:
             out[f"{k}_ffma"] = v["ffma_frac"]
         if "tensor_frac" in v:
             out[f"{k}_tensor"] = v["tensor_frac"]
     for k, v in (bwd or {}).items():
         out[f"bwd_{k}_{v['bound']}"] = v["frac"]
+        if "frac_b2b" in v:
+            out[f"bwd_{k}_b2b_{v['bound']}"] = v["frac_b2b"]
     for k, v in (extra or {}).items():
         out[f"{k}_{v['bound']}"] = v["frac"]
     return out
@@ -240,6 +244,11 @@ def time_launches(torch, fn, stream, reps, flush=None):
     return statistics.median(times), sum(times) / len(times)
 
 
+def sets_for(set_bytes: int) -> int:
+    """Buffer sets for a back-to-back figure: at least 2, and together more than 2x L2."""
+    return max(2, -(-2 * L2_BYTES // max(1, set_bytes)) + 1)
+
+
 def time_graph_b2b(torch, fn, stream, n_sets, launches=32, reps=5):
     """Per-launch CUDA-event time (ms) of `launches` back-to-back launches of `fn(i)`, i cycling
     over `n_sets` buffer sets whose combined size exceeds 2x L2 (a launch reads inputs that 7
@@ -297,18 +306,22 @@ KERNEL_SOURCE = {1: "direct_generic.cu", 2: "depthwise_nhwc.cu", 3: "igemm_rowt.
 
 def conv2d_measurement(torch, gb, device, stream, pk, p, workload, path, reps, flush):
     inp = wl.make_conv2d_inputs(p, workload)
-    x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
-    y = torch.empty(p.y_shape, dtype=torch.bfloat16, device=device)
+    w = dev_tensor(torch, inp.w, p.dtype, device)
+    n_sets = sets_for(p.bytes())
+    xs = [dev_tensor(torch, inp.x, p.dtype, device) for _ in range(n_sets)]
+    ys = [torch.empty(p.y_shape, dtype=torch.bfloat16, device=device) for _ in range(n_sets)]
     need = gb.gconv2d_fwd_workspace_size(p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride,
                                          p.pad, p.dilation, p.groups, p.layout, p.dtype, path)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
     kcode = gb.gconv2d_select_path(p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride, p.pad,
                                    p.dilation, p.groups, p.layout, p.dtype, path)
-    fn = lambda i: gb.gconv2d_fwd(x, w, None, p.stride, p.pad, p.dilation, p.groups, p.layout,
-                                  out=y, workspace=ws, path=path, stream=stream)
+    fn = lambda i: gb.gconv2d_fwd(xs[i], w, None, p.stride, p.pad, p.dilation, p.groups,
+                                  p.layout, out=ys[i], workspace=ws, path=path, stream=stream)
     for _ in range(2):
         fn(0)
-    med, mean = time_launches(torch, fn, stream, reps, flush)
+    med, mean = time_launches(torch, lambda i: fn(0), stream, reps, flush)
+    # back to back in a graph, except for the slow generic fallbacks (milliseconds a launch)
+    b2b = time_graph_b2b(torch, fn, stream, n_sets) if med < 5.0 else None
     tf = p.flops() / (med * 1e-3) / 1e12
     gbs = p.bytes() / (med * 1e-3) / 1e9
     t_hbm = p.bytes() / (pk["hbm_gbs"] * 1e9)
@@ -324,6 +337,9 @@ def conv2d_measurement(torch, gb, device, stream, pk, p, workload, path, reps, f
         bound, t_roof = ("tensor", t_tensor) if t_tensor >= t_hbm else ("hbm", t_hbm)
     rec.update({"bound": bound, "frac": round(t_roof / (med * 1e-3), 3),
                 "alg_flops": p.flops(), "alg_bytes": p.bytes()})
+    if b2b is not None:
+        rec.update({"us_b2b": round(b2b * 1e3, 2), "frac_b2b": round(t_roof / (b2b * 1e-3), 3)})
+    del xs, ys, ws
     return rec
 
 
@@ -332,23 +348,32 @@ def variant_measurement(torch, gb, device, stream, pk, p, workload, mode, reps, 
     (gconv2d_fwd_out): same FLOPs as the layer; bytes x + w + y, y with C_out / groups channels
     for the merges."""
     inp = wl.make_conv2d_inputs(p, workload)
-    x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
-    y = gb.gconv2d_fwd_out(x, w, None, p.stride, p.pad, p.dilation, p.groups, p.layout, mode)
+    w = dev_tensor(torch, inp.w, p.dtype, device)
+    x0 = dev_tensor(torch, inp.x, p.dtype, device)
+    y0 = gb.gconv2d_fwd_out(x0, w, None, p.stride, p.pad, p.dilation, p.groups, p.layout, mode)
+    nbytes = (x0.numel() + w.numel() + y0.numel()) * 2
+    n_sets = sets_for(nbytes)
+    xs = [x0] + [dev_tensor(torch, inp.x, p.dtype, device) for _ in range(n_sets - 1)]
+    ys = [y0] + [torch.empty_like(y0) for _ in range(n_sets - 1)]
     kcode = gb.gconv2d_fwd_out_select_path(p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride,
                                            p.pad, p.dilation, p.groups, p.layout, p.dtype, mode)
-    fn = lambda i: gb.gconv2d_fwd_out(x, w, None, p.stride, p.pad, p.dilation, p.groups,
-                                      p.layout, mode, out=y, stream=stream)
+    fn = lambda i: gb.gconv2d_fwd_out(xs[i], w, None, p.stride, p.pad, p.dilation, p.groups,
+                                      p.layout, mode, out=ys[i], stream=stream)
     for _ in range(2):
         fn(0)
-    med, mean = time_launches(torch, fn, stream, reps, flush)
-    nbytes = (x.numel() + w.numel() + y.numel()) * 2
+    med, mean = time_launches(torch, lambda i: fn(0), stream, reps, flush)
+    b2b = time_graph_b2b(torch, fn, stream, n_sets)
     t_tensor = p.flops() / (pk["bf16_tflops"] * 1e12)
     t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
     bound, t_roof = ("tensor", t_tensor) if t_tensor >= t_hbm else ("hbm", t_hbm)
-    return {"kernel": kernel_name(kcode), "us": round(med * 1e3, 2),
-            "TFLOP/s": round(p.flops() / (med * 1e-3) / 1e12, 1),
-            "GB/s": round(nbytes / (med * 1e-3) / 1e9, 1), "bound": bound,
-            "frac": round(t_roof / (med * 1e-3), 3), "alg_flops": p.flops(), "alg_bytes": nbytes}
+    rec = {"kernel": kernel_name(kcode), "us": round(med * 1e3, 2),
+           "TFLOP/s": round(p.flops() / (med * 1e-3) / 1e12, 1),
+           "GB/s": round(nbytes / (med * 1e-3) / 1e9, 1), "bound": bound,
+           "frac": round(t_roof / (med * 1e-3), 3), "us_b2b": round(b2b * 1e3, 2),
+           "frac_b2b": round(t_roof / (b2b * 1e-3), 3), "alg_flops": p.flops(),
+           "alg_bytes": nbytes}
+    del xs, ys
+    return rec
 
 
 def more_conv2d_measurements(torch, gb, device, stream, pk, reps):
@@ -390,17 +415,24 @@ def depthwise_measurements(torch, gb, device, stream, pk, reps):
     for stride in (1, 2):
         p = wl.depthwise_56(stride)
         inp = wl.make_conv2d_inputs(p, 5)
-        x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
-        y = torch.empty(p.y_shape, dtype=torch.bfloat16, device=device)
-        fn = lambda i: gb.gconv2d_fwd(x, w, None, p.stride, p.pad, p.dilation, p.groups,
-                                      p.layout, out=y, stream=stream)
+        w = dev_tensor(torch, inp.w, p.dtype, device)
+        n_sets = sets_for(p.bytes())
+        xs = [dev_tensor(torch, inp.x, p.dtype, device) for _ in range(n_sets)]
+        ys = [torch.empty(p.y_shape, dtype=torch.bfloat16, device=device) for _ in range(n_sets)]
+        fn = lambda i: gb.gconv2d_fwd(xs[i], w, None, p.stride, p.pad, p.dilation, p.groups,
+                                      p.layout, out=ys[i], stream=stream)
         for _ in range(3):
             fn(0)
-        med, mean = time_launches(torch, fn, stream, reps, flush)
+        med, mean = time_launches(torch, lambda i: fn(0), stream, reps, flush)
+        b2b = time_graph_b2b(torch, fn, stream, n_sets)
         gbs = p.bytes() / (med * 1e-3) / 1e9
+        gbs_b2b = p.bytes() / (b2b * 1e-3) / 1e9
         out[f"depthwise56_s{stride}"] = {"us": round(med * 1e3, 2), "GB/s": round(gbs, 1),
-                                         "frac": round(gbs / hbm, 3), "alg_bytes": p.bytes()}
-        del x, w, y
+                                         "frac": round(gbs / hbm, 3),
+                                         "us_b2b": round(b2b * 1e3, 2),
+                                         "frac_b2b": round(gbs_b2b / hbm, 3),
+                                         "alg_bytes": p.bytes()}
+        del xs, w, ys
     for causal in (False, True):
         p = wl.conformer_dw1d(causal)
         inp = wl.make_dwconv1d_inputs(p, 3)
@@ -463,10 +495,12 @@ def dwsep_measurements(torch, gb, device, stream, pk, reps):
     p = wl.conformer_dw1d(False)
     C_out = 512
     inp = wl.make_dwsep1d_inputs(p, C_out, 7)
-    x, wdw, wpw, b = (dev_tensor(torch, a, p.dtype, device)
-                      for a in (inp.x, inp.w_dw, inp.w_pw, inp.bias))
-    z = torch.empty((p.B, p.T_out, C_out), dtype=torch.bfloat16, device=device)
-    nbytes = (x.numel() + wdw.numel() + wpw.numel() + b.numel() + z.numel()) * 2
+    wdw, wpw, b = (dev_tensor(torch, a, p.dtype, device) for a in (inp.w_dw, inp.w_pw, inp.bias))
+    nbytes = (inp.x.size + wdw.numel() + wpw.numel() + b.numel() + p.B * p.T_out * C_out) * 2
+    n_sets = sets_for(nbytes)
+    xs = [dev_tensor(torch, inp.x, p.dtype, device) for _ in range(n_sets)]
+    zs = [torch.empty((p.B, p.T_out, C_out), dtype=torch.bfloat16, device=device)
+          for _ in range(n_sets)]
     flops = 2 * p.B * p.T_out * p.C * (p.K + C_out)
     out = {}
     for name, path in (("dwsep1d_fused", gb.PATH_AUTO), ("dwsep1d_two_launches", gb.PATH_DIRECT)):
@@ -475,16 +509,18 @@ def dwsep_measurements(torch, gb, device, stream, pk, reps):
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
         kname = gb.KERNEL_NAMES.get(gb.dwsep1d_select_path(p.B, p.T, p.C, p.K, p.pad_left,
                                                            p.pad_right, C_out, p.dtype, path))
-        fn = lambda i: gb.dwsep1d_fwd(x, wdw, wpw, b, p.pad_left, p.pad_right, out=z,
+        fn = lambda i: gb.dwsep1d_fwd(xs[i], wdw, wpw, b, p.pad_left, p.pad_right, out=zs[i],
                                       workspace=ws, path=path, stream=stream)
         for _ in range(3):
             fn(0)
-        med, mean = time_launches(torch, fn, stream, reps, flush)
+        med, mean = time_launches(torch, lambda i: fn(0), stream, reps, flush)
+        b2b = time_graph_b2b(torch, fn, stream, n_sets)
         t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
         out[name] = {"kernel": kname, "us": round(med * 1e3, 2),
                      "TFLOP/s": round(flops / (med * 1e-3) / 1e12, 1),
                      "GB/s": round(nbytes / (med * 1e-3) / 1e9, 1), "bound": "hbm",
                      "frac": round(t_hbm / (med * 1e-3), 3),
+                     "us_b2b": round(b2b * 1e3, 2), "frac_b2b": round(t_hbm / (b2b * 1e-3), 3),
                      "tensor_frac": round(2 * p.B * p.T_out * p.C * C_out / (med * 1e-3) /
                                           (pk["bf16_tflops"] * 1e12), 3),
                      "alg_bytes": nbytes, "alg_flops": flops}
@@ -492,6 +528,7 @@ def dwsep_measurements(torch, gb, device, stream, pk, reps):
     # strided 2-D blocks: a Fast Conformer downsampler layer, x[8, 512, 40, 256] NHWC (frames x
     # frequency bins; 20 output columns, narrower than the fused kernel's 32-column tiles, so
     # AUTO runs the two launches there), and the same layer on 128 bins (64 output columns)
+    del xs, zs
     for tag, W in (("", 40), ("_w128", 128)):
         out.update(dwsep2d_measurement(torch, gb, device, stream, pk, reps, flush, W, tag))
     return out
@@ -502,12 +539,14 @@ def dwsep2d_measurement(torch, gb, device, stream, pk, reps, flush, W, tag):
     N, H, C, k, st, pad, Co = 8, 512, 256, 3, 2, 1, 256
     p2 = wl.Dwconv1dProblem(N, H * W, C, k * k, 0, 0, wl.BF16)
     inp2 = wl.make_dwsep1d_inputs(p2, Co, 8)
-    x2 = dev_tensor(torch, inp2.x.reshape(N, H, W, C), wl.BF16, device)
     wdw2 = dev_tensor(torch, inp2.w_dw.reshape(C, k, k, 1), wl.BF16, device)
     wpw2, b2 = (dev_tensor(torch, a, wl.BF16, device) for a in (inp2.w_pw, inp2.bias))
     Ho, Wo = gb.out_shape(N, C, H, W, C, k, k, st, pad, 1, C, "NHWC", wl.BF16)
-    z2 = torch.empty((N, Ho, Wo, Co), dtype=torch.bfloat16, device=device)
-    nbytes2 = (x2.numel() + wdw2.numel() + wpw2.numel() + b2.numel() + z2.numel()) * 2
+    nbytes2 = (N * H * W * C + wdw2.numel() + wpw2.numel() + b2.numel() + N * Ho * Wo * Co) * 2
+    n_sets = sets_for(nbytes2)
+    x2s = [dev_tensor(torch, inp2.x.reshape(N, H, W, C), wl.BF16, device) for _ in range(n_sets)]
+    z2s = [torch.empty((N, Ho, Wo, Co), dtype=torch.bfloat16, device=device)
+           for _ in range(n_sets)]
     flops2 = 2 * N * Ho * Wo * C * (k * k + Co)
     for name, path in ((f"dwsep2d{tag}_auto", gb.PATH_AUTO),
                        (f"dwsep2d{tag}_two_launches", gb.PATH_DIRECT)):
@@ -516,17 +555,21 @@ def dwsep2d_measurement(torch, gb, device, stream, pk, reps, flush, W, tag):
         need = gb.load_library().dwsep2d_fwd_workspace_size(N, C, H, W, k, k, st, pad, 1, Co,
                                                             wl.NHWC, wl.BF16, path)
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
-        fn = lambda i: gb.dwsep2d_fwd(x2, wdw2, wpw2, b2, st, pad, 1, "NHWC", out=z2,
+        fn = lambda i: gb.dwsep2d_fwd(x2s[i], wdw2, wpw2, b2, st, pad, 1, "NHWC", out=z2s[i],
                                       workspace=ws, path=path, stream=stream)
         for _ in range(3):
             fn(0)
-        med, mean = time_launches(torch, fn, stream, reps, flush)
+        med, mean = time_launches(torch, lambda i: fn(0), stream, reps, flush)
+        b2b = time_graph_b2b(torch, fn, stream, n_sets)
+        t_hbm = nbytes2 / (pk["hbm_gbs"] * 1e9)
         out[name] = {"kernel": kname, "us": round(med * 1e3, 2),
                      "TFLOP/s": round(flops2 / (med * 1e-3) / 1e12, 1),
                      "GB/s": round(nbytes2 / (med * 1e-3) / 1e9, 1), "bound": "hbm",
-                     "frac": round(nbytes2 / (pk["hbm_gbs"] * 1e9) / (med * 1e-3), 3),
+                     "frac": round(t_hbm / (med * 1e-3), 3),
+                     "us_b2b": round(b2b * 1e3, 2), "frac_b2b": round(t_hbm / (b2b * 1e-3), 3),
                      "alg_bytes": nbytes2, "alg_flops": flops2}
         del ws
+    del x2s, z2s
     return out
 
 
@@ -542,9 +585,12 @@ def backward_measurements(torch, gb, device, stream, pk, reps):
              ("wide_group_nchw", wl.wide_group(wl.NCHW), reps)]
     for tag, p, r in cases:
         inp = wl.make_conv2d_inputs(p, 5)
-        x, w = dev_tensor(torch, inp.x, p.dtype, device), dev_tensor(torch, inp.w, p.dtype, device)
-        dy = dev_tensor(torch, wl.make_conv2d_dy(p, 5), p.dtype, device)
-        dx = torch.empty(p.x_shape, dtype=torch.bfloat16, device=device)
+        w = dev_tensor(torch, inp.w, p.dtype, device)
+        dy_host = wl.make_conv2d_dy(p, 5)
+        n_sets = sets_for(p.bytes())
+        xs = [dev_tensor(torch, inp.x, p.dtype, device) for _ in range(n_sets)]
+        dys = [dev_tensor(torch, dy_host, p.dtype, device) for _ in range(n_sets)]
+        dxs = [torch.empty(p.x_shape, dtype=torch.bfloat16, device=device) for _ in range(n_sets)]
         dw = torch.empty(p.w_shape, dtype=torch.bfloat16, device=device)
         dims = (p.N, p.C_in, p.H, p.W, p.C_out, p.kH, p.kW, p.stride, p.pad, p.dilation,
                 p.groups, p.layout, p.dtype, gb.PATH_AUTO)
@@ -553,20 +599,21 @@ def backward_measurements(torch, gb, device, stream, pk, reps):
         wsw_n = gb.gconv2d_bwd_weight_workspace_size(*dims)
         wsw = torch.empty(max(wsw_n, 16), dtype=torch.uint8, device=device)
         ops = {
-            "dgrad": (lambda i: gb.gconv2d_bwd_data(dy, w, (p.H, p.W), p.stride, p.pad,
-                                                    p.dilation, p.groups, p.layout, out=dx,
+            "dgrad": (lambda i: gb.gconv2d_bwd_data(dys[i], w, (p.H, p.W), p.stride, p.pad,
+                                                    p.dilation, p.groups, p.layout, out=dxs[i],
                                                     workspace=wsd, stream=stream),
                       gb.KERNEL_NAMES.get(gb.gconv2d_bwd_data_select_path(*dims))),
-            "wgrad": (lambda i: gb.gconv2d_bwd_weight(x, dy, (p.kH, p.kW), p.stride, p.pad,
-                                                      p.dilation, p.groups, p.layout, out=dw,
-                                                      workspace=wsw, stream=stream),
+            "wgrad": (lambda i: gb.gconv2d_bwd_weight(xs[i], dys[i], (p.kH, p.kW), p.stride,
+                                                      p.pad, p.dilation, p.groups, p.layout,
+                                                      out=dw, workspace=wsw, stream=stream),
                       gb.KERNEL_NAMES.get(gb.gconv2d_bwd_weight_select_path(*dims))),
         }
         for op, (fn, kname) in ops.items():
             fn(0)
             torch.cuda.synchronize()
             n = r if not (tag.startswith("wide") and op == "wgrad") else 3
-            med, mean = time_launches(torch, fn, stream, n, flush)
+            med, mean = time_launches(torch, lambda i: fn(0), stream, n, flush)
+            b2b = time_graph_b2b(torch, fn, stream, n_sets)
             t_tensor = p.flops() / (pk["bf16_tflops"] * 1e12)
             t_hbm = p.bytes() / (pk["hbm_gbs"] * 1e9)
             bound = "tensor" if t_tensor >= t_hbm else "hbm"
@@ -574,11 +621,13 @@ def backward_measurements(torch, gb, device, stream, pk, reps):
                    "TFLOP/s": round(p.flops() / (med * 1e-3) / 1e12, 1),
                    "GB/s": round(p.bytes() / (med * 1e-3) / 1e9, 1), "bound": bound,
                    "frac": round(max(t_tensor, t_hbm) / (med * 1e-3), 3),
+                   "us_b2b": round(b2b * 1e3, 2),
+                   "frac_b2b": round(max(t_tensor, t_hbm) / (b2b * 1e-3), 3),
                    "alg_bytes": p.bytes(), "alg_flops": p.flops()}
             if op == "wgrad":
                 rec["workspace_bytes"] = wsw_n
             out[f"{tag}_{op}"] = rec
-        del x, w, dy, dx, dw, wsd, wsw
+        del xs, w, dys, dxs, dw, wsd, wsw
     return out
 
 
