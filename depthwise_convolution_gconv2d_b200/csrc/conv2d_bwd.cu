@@ -319,6 +319,7 @@ __global__ void __launch_bounds__(DWW_THREADS, 2)
                          const __grid_constant__ CUtensorMap tmd, float* __restrict__ ws,
                          const DwwParams P, unsigned int* err) {
   using namespace ptx;
+  pdl_launch_dependents();   // the slice sum may be scheduled as this grid's CTAs finish
   constexpr int BH = dww_bh<S>();
   constexpr int IW = dww_iw<S>();
   extern __shared__ unsigned char smem_raw[];
@@ -903,6 +904,7 @@ template <typename T, int MODE>
 __global__ void __launch_bounds__(256) wgrad_sum_kernel(const float* __restrict__ ws,
                                                          T* __restrict__ dw, long long E,
                                                          int S, int taps, int cpg_in, int kW) {
+  ptx::pdl_wait();   // the partials of the kernel before (launch_pdl)
   __shared__ float part[8][33];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long q = (long long)blockIdx.x * 32 + lane;
@@ -1116,9 +1118,8 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
       cudaError_t e = p.stride == 1 ? launch_dww<T, 1>(p, x, dy, (float*)ws, P, s)
                                     : launch_dww<T, 2>(p, x, dy, (float*)ws, P, s);
       if (e != cudaSuccess) return e;
-      wgrad_sum_kernel<T, SUM_TAP_MAJOR><<<sum_grid(E), 256, 0, s>>>((const float*)ws, (T*)dw,
-                                                                     E, P.slices, 9, 1, 3);
-      return cudaGetLastError();
+      return launch_pdl(wgrad_sum_kernel<T, SUM_TAP_MAJOR>, (unsigned)sum_grid(E), 256u, 0, s,
+                        (const float*)ws, (T*)dw, E, P.slices, 9, 1, 3);
     }
     const bool tc = kernel == GCONV_KERNEL_WGRAD_TC_NHWC || kernel == GCONV_KERNEL_WGRAD_TC_NCHW;
     const bool to_nchw = kernel == GCONV_KERNEL_WGRAD_TILED_NCHW ||
@@ -1159,11 +1160,10 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
       }
       if (e != cudaSuccess) return e;
       if (to_nchw)
-        wgrad_sum_kernel<T, SUM_TO_NCHW><<<sum_grid(E), 256, 0, s>>>(
-            part, (T*)dw, E, S, p.kH * p.kW, p.cpg_in, p.kW);
-      else
-        wgrad_sum_kernel<T, SUM_SAME><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S, 1, 1, 1);
-      return cudaGetLastError();
+        return launch_pdl(wgrad_sum_kernel<T, SUM_TO_NCHW>, (unsigned)sum_grid(E), 256u, 0, s,
+                          part, (T*)dw, E, S, p.kH * p.kW, p.cpg_in, p.kW);
+      return launch_pdl(wgrad_sum_kernel<T, SUM_SAME>, (unsigned)sum_grid(E), 256u, 0, s, part,
+                        (T*)dw, E, S, 1, 1, 1);
     }
   }
   int S, rows;
@@ -1185,9 +1185,8 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
       wgrad_depthwise_nhwc_kernel<T, 5, 2, 2><<<grid, 128, 0, s>>>(xt, dt, part, p, rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wgrad_sum_kernel<T, SUM_TAP_MAJOR><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S,
-                                                                   p.kH * p.kW, 1, p.kW);
-    return cudaGetLastError();
+    return launch_pdl(wgrad_sum_kernel<T, SUM_TAP_MAJOR>, (unsigned)sum_grid(E), 256u, 0, s,
+                      part, (T*)dw, E, S, p.kH * p.kW, 1, p.kW);
    }
   }
   if (p.layout == GCONV_NHWC)
@@ -1198,8 +1197,8 @@ cudaError_t wgrad_typed(const Conv2d& p, const void* x, const void* dy, void* dw
                                                             E, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  wgrad_sum_kernel<T, SUM_SAME><<<sum_grid(E), 256, 0, s>>>(part, (T*)dw, E, S, 1, 1, 1);
-  return cudaGetLastError();
+  return launch_pdl(wgrad_sum_kernel<T, SUM_SAME>, (unsigned)sum_grid(E), 256u, 0, s, part,
+                    (T*)dw, E, S, 1, 1, 1);
 }
 
 }  // namespace

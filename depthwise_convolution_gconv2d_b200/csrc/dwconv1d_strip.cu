@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(SP_THREADS, 2)
     dwconv1d_wgrad_strip_kernel(const __grid_constant__ CUtensorMap tmx,
                                 const __grid_constant__ CUtensorMap tmd,
                                 float* __restrict__ part, const SpParams P, unsigned int* err) {
+  pdl_launch_dependents();   // the run sum may be scheduled as this grid's CTAs finish
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = align_smem(smem_raw, 1024u);
   unsigned char* ring = smem;
@@ -320,6 +321,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) dwconv1d_wgrad_strip_sum(const float* __restrict__ part,
                                                                 T* __restrict__ dw, int C, int K,
                                                                 int runs) {
+  pdl_wait();   // the partials of the kernel before (launch_pdl)
   __shared__ float acc8[8][33];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int e = blockIdx.x * 32 + lane;
@@ -425,8 +427,8 @@ cudaError_t launch_wgrad_k(const SpParams& P, const CUtensorMap& tx, const CUten
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int E = P.C * K;
-  dwconv1d_wgrad_strip_sum<T><<<(E + 31) / 32, 256, 0, s>>>(part, (T*)dw, P.C, K, P.runs);
-  return cudaGetLastError();
+  return launch_pdl(dwconv1d_wgrad_strip_sum<T>, (unsigned)((E + 31) / 32), 256u, 0, s, part,
+                    (T*)dw, P.C, K, P.runs);
 }
 
 template <typename T>

@@ -1637,6 +1637,7 @@ template <typename T, bool VEC>
 __global__ void __launch_bounds__(256) merge_max_groups_kernel(const T* __restrict__ g,
                                                                T* __restrict__ y, long long n_out,
                                                                long long S, int groups) {
+  pdl_wait();   // the group-major output of the kernel before (launch_pdl)
   constexpr int V = VEC ? 8 : 1;
   const long long n_items = n_out / V;
   for (long long it = (long long)blockIdx.x * blockDim.x + threadIdx.x; it < n_items;
@@ -1689,12 +1690,10 @@ cudaError_t launch_merge_max_typed(const Conv2d& p, const void* g, void* y, cuda
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   if (vec)
-    merge_max_groups_kernel<T, true><<<(unsigned)blocks, 256, 0, s>>>((const T*)g, (T*)y, n_out,
-                                                                       S, p.groups);
-  else
-    merge_max_groups_kernel<T, false><<<(unsigned)blocks, 256, 0, s>>>((const T*)g, (T*)y, n_out,
-                                                                        S, p.groups);
-  return cudaGetLastError();
+    return launch_pdl(merge_max_groups_kernel<T, true>, (unsigned)blocks, 256u, 0, s,
+                      (const T*)g, (T*)y, n_out, S, p.groups);
+  return launch_pdl(merge_max_groups_kernel<T, false>, (unsigned)blocks, 256u, 0, s, (const T*)g,
+                    (T*)y, n_out, S, p.groups);
 }
 
 }  // namespace

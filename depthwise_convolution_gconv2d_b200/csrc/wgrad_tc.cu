@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(WT_THREADS, 1)
                     const __grid_constant__ CUtensorMap tx,
                     const __grid_constant__ CUtensorMap txh, float* __restrict__ part,
                     const WtParams P, unsigned int* err) {
+  pdl_launch_dependents();   // the slice sum may be scheduled as this grid's CTAs finish
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = align_smem(smem_raw, 1024u);
   unsigned long long* bars =
