@@ -54,6 +54,13 @@
  * state apart from the device error word read by gconv_get_device_error() and the fixed
  * scratch of dwconv1d_bwd_weight_noalloc, so calls on different streams may be made from
  * different threads (that one entry point excepted, see its comment).
+ *
+ * Stream order: the tensor-core kernels, the depthwise 3x3 kernel and the second kernel of
+ * two-kernel calls are launched with programmatic stream serialization. Their setup (barrier
+ * initialisation, tensor-memory allocation) may overlap the tail of the previous kernel in
+ * the stream, whoever launched it, but they wait for that kernel to complete before their
+ * first global-memory access, so stream order holds for every byte they read or write. Calls
+ * may be captured into CUDA graphs.
  */
 #ifndef GCONV_H_
 #define GCONV_H_
