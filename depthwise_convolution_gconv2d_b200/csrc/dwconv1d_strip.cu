@@ -41,6 +41,12 @@ constexpr int SP_WARPS = 7;           // compute warps; 16 steps each
 constexpr int SP_TS = 16 * SP_WARPS;  // output steps per tile
 constexpr int SP_THREADS = 32 * (SP_WARPS + 1);
 constexpr int SP_STAGES = 3;
+// The weight gradient runs 8 compute warps and no producer warp (thread 0 issues the copies):
+// a 7 + 1 warp CTA left one SM sub-partition with half the FMA work of the others, and
+// 128-step tiles divide T = 2048 with no ragged tile.
+constexpr int SPW_WARPS = 8;
+constexpr int SPW_TS = 16 * SPW_WARPS;
+constexpr int SPW_THREADS = 32 * SPW_WARPS;
 constexpr int SP_TARGET_CTAS = 296;   // runs of tiles are sized for about this many CTAs
 constexpr unsigned int ERR_SP = 1u << 20;
 
@@ -51,9 +57,12 @@ struct SpParams {
   unsigned int x_bytes, dy_bytes, stage_bytes;
 };
 
+__host__ __device__ inline int sp_tile_steps(bool wgrad) { return wgrad ? SPW_TS : SP_TS; }
+
 __host__ __device__ inline unsigned int sp_stage_bytes(int K, bool wgrad) {
-  const unsigned int x = (unsigned int)(SP_TS + K - 1) * 128u;
-  const unsigned int d = wgrad ? (unsigned int)SP_TS * 128u : 0u;
+  const int ts = sp_tile_steps(wgrad);
+  const unsigned int x = (unsigned int)(ts + K - 1) * 128u;
+  const unsigned int d = wgrad ? (unsigned int)ts * 128u : 0u;
   return (x + d + 1023u) & ~1023u;
 }
 
@@ -197,7 +206,7 @@ __global__ void __launch_bounds__(SP_THREADS, 2)
 
 // Weight gradient: fp32 partials part[cb][run][64 channels][K] (channel-major within a block).
 template <typename T, int K>
-__global__ void __launch_bounds__(SP_THREADS, 2)
+__global__ void __launch_bounds__(SPW_THREADS, 2)
     dwconv1d_wgrad_strip_kernel(const __grid_constant__ CUtensorMap tmx,
                                 const __grid_constant__ CUtensorMap tmd,
                                 float* __restrict__ part, const SpParams P, unsigned int* err) {
@@ -213,10 +222,12 @@ __global__ void __launch_bounds__(SP_THREADS, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Run run(P);
-  if (threadIdx.x == 0) {
+  const int n = run.t_end - run.t_begin;
+  const bool producer = threadIdx.x == 0;
+  if (producer) {
     for (int s = 0; s < SP_STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], SP_WARPS);
+      mbar_init(&empty[s], SPW_WARPS);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -225,84 +236,88 @@ __global__ void __launch_bounds__(SP_THREADS, 2)
   }
   __syncthreads();
 
+  // thread 0 fills the ring at the start and refills stage s with tile i + SP_STAGES once
+  // every warp has released tile i
+  int issued = 0, consumed = 0;
+  auto issue = [&](int i) {
+    const int s = i % SP_STAGES;
+    const int t = run.t_begin + i;
+    const int b = t / P.n_tb, tb = t - b * P.n_tb;
+    unsigned char* st = ring + (size_t)s * P.stage_bytes;
+    mbar_arrive_expect_tx(&full[s], P.x_bytes + P.dy_bytes);
+    tma_load_3d(st, &tmx, &full[s], run.cb * SP_CB, tb * SPW_TS - P.pl, b);
+    tma_load_3d(st + P.x_bytes, &tmd, &full[s], run.cb * SP_CB, tb * SPW_TS, b);
+  };
+  if (producer) {
+    for (int q = 0; q < SP_STAGES && q < n; ++q) issue(q);
+    issued = n < SP_STAGES ? n : SP_STAGES;
+  }
+
   float2 acc[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) acc[k] = make_float2(0.0f, 0.0f);
   bool ok = true;
-  if (warp == 0) {
-    if (lane == 0) {
-      int s = 0;
-      unsigned int ph = 0;
-      long long issued = 0;
-      for (int t = run.t_begin; t < run.t_end; ++t) {
-        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, err, ERR_SP | 4u)) break;
-        const int b = t / P.n_tb, tb = t - b * P.n_tb;
-        unsigned char* st = ring + (size_t)s * P.stage_bytes;
-        mbar_arrive_expect_tx(&full[s], P.x_bytes + P.dy_bytes);
-        tma_load_3d(st, &tmx, &full[s], run.cb * SP_CB, tb * SP_TS - P.pl, b);
-        tma_load_3d(st + P.x_bytes, &tmd, &full[s], run.cb * SP_CB, tb * SP_TS, b);
-        ++issued;
-        if (++s == SP_STAGES) {
-          s = 0;
-          ph ^= 1u;
-        }
-      }
-      const unsigned long long dl = drain_deadline();
-      for (long long q = (issued > SP_STAGES ? issued - SP_STAGES : 0); q < issued; ++q)
-        mbar_wait_until(&full[q % SP_STAGES], (unsigned int)((q / SP_STAGES) & 1), dl, err,
-                        ERR_DRAIN);
+  for (int i = 0; i < n; ++i) {
+    const int s = i % SP_STAGES;
+    const unsigned int ph = (unsigned int)(i / SP_STAGES) & 1u;
+    bool got = mbar_try_wait(&full[s], ph);
+    if (!got) got = mbar_wait(&full[s], ph, abort_flag, err, ERR_SP | 8u);
+    if (!__all_sync(0xffffffffu, got)) {
+      ok = false;
+      break;
     }
-  } else {
-    const int w2 = warp - 1;
-    int s = 0;
-    unsigned int ph = 0;
-    for (int t = run.t_begin; t < run.t_end; ++t) {
-      bool got = mbar_try_wait(&full[s], ph);
-      if (!got) got = mbar_wait(&full[s], ph, abort_flag, err, ERR_SP | 8u);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      const unsigned char* st = ring + (size_t)s * P.stage_bytes;
-      const uint32_t* xr = reinterpret_cast<const uint32_t*>(st) + w2 * 16 * 32 + lane;
-      const uint32_t* dr = reinterpret_cast<const uint32_t*>(st + P.x_bytes) + w2 * 16 * 32 +
-                           lane;
-      float2 g[16];
+    if (producer) consumed = i + 1;
+    const unsigned char* st = ring + (size_t)s * P.stage_bytes;
+    const uint32_t* xr = reinterpret_cast<const uint32_t*>(st) + warp * 16 * 32 + lane;
+    const uint32_t* dr = reinterpret_cast<const uint32_t*>(st + P.x_bytes) + warp * 16 * 32 +
+                         lane;
+    float2 g[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) g[j] = unpack2<T>(dr[j * 32]);
-      // dy rows past T_out read as zeros (TMA fill), so they add nothing
+    for (int j = 0; j < 16; ++j) g[j] = unpack2<T>(dr[j * 32]);
+    // dy rows past T_out read as zeros (TMA fill), so they add nothing
 #pragma unroll
-      for (int i = 0; i < 16 + K - 1; ++i) {
-        const float2 xv = unpack2<T>(xr[i * 32]);
+    for (int r = 0; r < 16 + K - 1; ++r) {
+      const float2 xv = unpack2<T>(xr[r * 32]);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int k = i - j;
-          if (k >= 0 && k < K) acc[k] = ffma2(g[j], xv, acc[k]);
-        }
+      for (int j = 0; j < 16; ++j) {
+        const int k = r - j;
+        if (k >= 0 && k < K) acc[k] = ffma2(g[j], xv, acc[k]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      if (++s == SP_STAGES) {
-        s = 0;
-        ph ^= 1u;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    bool refill_ok = true;
+    if (producer && i + SP_STAGES < n) {
+      refill_ok = mbar_wait(&empty[s], ph, abort_flag, err, ERR_SP | 4u);
+      if (refill_ok) {
+        issue(i + SP_STAGES);
+        issued = i + SP_STAGES + 1;
       }
+    }
+    if (!__all_sync(0xffffffffu, refill_ok)) {
+      ok = false;
+      break;
     }
   }
-  // the 7 warps' sums, added in warp order through the (now idle) ring
+  if (producer) {
+    const unsigned long long dl = drain_deadline();
+    for (int q = consumed; q < issued; ++q)
+      mbar_wait_until(&full[q % SP_STAGES], (unsigned int)((q / SP_STAGES) & 1), dl, err,
+                      ERR_DRAIN);
+  }
+  // the 8 warps' sums, added in warp order through the (now idle) ring
   ok = __syncthreads_and(ok ? 1 : 0) != 0 && !*abort_flag;
   if (!ok) return;
   float2* red = reinterpret_cast<float2*>(ring);      // [warp][k][lane]
-  if (warp >= 1) {
 #pragma unroll
-    for (int k = 0; k < K; ++k) red[((warp - 1) * K + k) * 32 + lane] = acc[k];
-  }
+  for (int k = 0; k < K; ++k) red[(warp * K + k) * 32 + lane] = acc[k];
   __syncthreads();
   float* out = part + ((long long)blockIdx.x) * SP_CB * K;   // [cb][run] blocks of 64 x K
-  for (int e = threadIdx.x; e < 32 * K; e += SP_THREADS) {
+  for (int e = threadIdx.x; e < 32 * K; e += SPW_THREADS) {
     const int k = e / 32, l = e - k * 32;
     float2 v = red[k * 32 + l];
 #pragma unroll
-    for (int wv = 1; wv < SP_WARPS; ++wv) {
+    for (int wv = 1; wv < SPW_WARPS; ++wv) {
       const float2 u = red[(wv * K + k) * 32 + l];
       v.x += u.x;
       v.y += u.y;
@@ -359,10 +374,11 @@ bool sp_k_supported(int K) {
 // Parameters of a pass over T_in input steps producing T_out output steps (pl: left pad).
 bool make_sp_params(const Conv1d& p, int T_in, int T_out, int pl, bool wgrad, SpParams* P) {
   if (p.dtype != GCONV_BF16 && p.dtype != GCONV_F16) return false;
-  if (p.C % SP_CB != 0 || !sp_k_supported(p.K) || SP_TS + p.K - 1 > 256) return false;
+  const int ts = sp_tile_steps(wgrad);
+  if (p.C % SP_CB != 0 || !sp_k_supported(p.K) || ts + p.K - 1 > 256) return false;
   P->B = p.B; P->T_in = T_in; P->T_out = T_out; P->C = p.C; P->pl = pl;
   P->n_cb = p.C / SP_CB;
-  P->n_tb = (T_out + SP_TS - 1) / SP_TS;
+  P->n_tb = (T_out + ts - 1) / ts;
   const long long tpc = (long long)p.B * P->n_tb;
   if (tpc > INT32_MAX || tpc < 1) return false;
   P->tiles_per_cb = (int)tpc;
@@ -370,8 +386,8 @@ bool make_sp_params(const Conv1d& p, int T_in, int T_out, int pl, bool wgrad, Sp
   if (runs > tpc) runs = tpc;
   if ((long long)P->n_cb * runs > INT32_MAX) return false;
   P->runs = (int)runs;
-  P->x_bytes = (unsigned int)(SP_TS + p.K - 1) * 128u;
-  P->dy_bytes = wgrad ? (unsigned int)SP_TS * 128u : 0u;
+  P->x_bytes = (unsigned int)(ts + p.K - 1) * 128u;
+  P->dy_bytes = wgrad ? (unsigned int)ts * 128u : 0u;
   P->stage_bytes = sp_stage_bytes(p.K, wgrad);
   return true;
 }
@@ -422,7 +438,7 @@ cudaError_t launch_wgrad_k(const SpParams& P, const CUtensorMap& tx, const CUten
   const size_t smem = sp_smem(P, K, true);
   cudaError_t e = set_max_dynamic_smem((const void*)dwconv1d_wgrad_strip_kernel<T, K>, smem, conf);
   if (e != cudaSuccess) return e;
-  dwconv1d_wgrad_strip_kernel<T, K><<<(unsigned)(P.n_cb * P.runs), SP_THREADS, smem, s>>>(
+  dwconv1d_wgrad_strip_kernel<T, K><<<(unsigned)(P.n_cb * P.runs), SPW_THREADS, smem, s>>>(
       tx, td, part, P, device_error_word());
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -496,8 +512,8 @@ cudaError_t launch_dwconv1d_wgrad_strip(const Conv1d& p, const void* x, const vo
   EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap tx, td;
-  if (!encode_rows(enc, &tx, p.dtype, x, p.C, p.T, p.B, SP_TS + p.K - 1, false) ||
-      !encode_rows(enc, &td, p.dtype, dy, p.C, p.T_out, p.B, SP_TS, false))
+  if (!encode_rows(enc, &tx, p.dtype, x, p.C, p.T, p.B, SPW_TS + p.K - 1, false) ||
+      !encode_rows(enc, &td, p.dtype, dy, p.C, p.T_out, p.B, SPW_TS, false))
     return cudaErrorInvalidValue;
   if (p.dtype == GCONV_BF16)
     return dispatch_wgrad<__nv_bfloat16>(P, p.K, tx, td, (float*)workspace, dw, s);
