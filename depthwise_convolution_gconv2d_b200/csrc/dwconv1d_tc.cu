@@ -31,11 +31,14 @@
 //               and, by a bulk copy, the 16 channels' filter taps
 //   warp 1      TMEM owner and MMA issuer (per sub-tile 8 channels x KS MMAs, one commit)
 //   warps 2-5   epilogue: TMEM -> registers -> transposed output in the A buffer ->
-//               ldmatrix.trans / stmatrix into the output buffer as [steps][16 ch] -> TMA store
+//               ldmatrix.trans / stmatrix into the tile's buffer as [steps][16 ch] -> TMA store
 //   warps 6-9   transpose of the input box into the A layout; filter copies
-// The input buffer is released once both halves are transposed; operands and accumulators go
-// through a ring of 2 sub-tiles (released once the epilogue has read them); the output buffer
-// is reused once the previous tile's TMA store has read it.
+// Two tile buffers alternate between a CTA's tiles. A tile's buffer first takes its input rows;
+// the epilogue then stages the tile's output rows in the same buffer (output half h overwrites
+// only the bytes of input half h, which the transpose of half h consumed before the sub-tile's
+// MMAs could start), and the buffer goes back to the producer once the tile's TMA store has read
+// it. The next tile's input is therefore loaded while this one is computed. Operands and
+// accumulators go through a ring of 2 sub-tiles (released once the epilogue has read them).
 #include <type_traits>
 
 #include "internal.cuh"
@@ -49,6 +52,7 @@ constexpr int TC_CH = 8;              // channels per sub-tile (MMA chains per c
 constexpr int TC_BLOCKS = 128;        // MMA rows: blocks of 16 steps
 constexpr int TC_STEPS = 16 * TC_BLOCKS;
 constexpr int TC_ASTAGES = 2;         // operand / accumulator stages (sub-tiles)
+constexpr int TC_XBUFS = 2;           // tile buffers: input rows, then the tile's output rows
 constexpr int TC_THREADS = 320;
 constexpr int TC_TMEM_COLS = 256;     // 2 stages x 8 channels x 16 columns
 constexpr int TC_MAX_KS = 4;          // K <= 49
@@ -62,7 +66,8 @@ struct TcLayout {
   int cstride;       // bytes between channels in the A buffer (odd multiple of 16)
   int bstride;       // bytes between channels in the filter copies
   int xs_bytes, as_bytes, bs_bytes;
-  int ws_off, as_off, astage, os_off, total;
+  int xbuf;          // bytes per tile buffer: the input boxes or the 2048 x 32-byte output rows
+  int ws_off, as_off, astage, total;
 };
 
 __host__ __device__ constexpr TcLayout tc_layout(int KS) {
@@ -76,11 +81,11 @@ __host__ __device__ constexpr TcLayout tc_layout(int KS) {
   L.xs_bytes = L.n_boxes * L.box_h * 32; // rows past `rows` are loaded but not used
   L.as_bytes = ((TC_CH * L.cstride + 1023) / 1024) * 1024;
   L.bs_bytes = ((TC_CH * L.bstride + 1023) / 1024) * 1024;
-  L.ws_off = L.xs_bytes;
-  L.as_off = ((L.ws_off + TC_WS_BYTES + 1023) / 1024) * 1024;
+  L.xbuf = ((L.xs_bytes > TC_STEPS * 32 ? L.xs_bytes : TC_STEPS * 32) + 127) / 128 * 128;
+  L.ws_off = TC_XBUFS * L.xbuf;
+  L.as_off = ((L.ws_off + TC_XBUFS * TC_WS_BYTES + 1023) / 1024) * 1024;
   L.astage = L.as_bytes + L.bs_bytes;
-  L.os_off = L.as_off + TC_ASTAGES * L.astage;
-  L.total = L.os_off + TC_STEPS * 32;
+  L.total = L.as_off + TC_ASTAGES * L.astage;
   return L;
 }
 
@@ -132,9 +137,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = ptx::align_smem(smem_raw, 1024u);
   unsigned long long* bars = reinterpret_cast<unsigned long long*>(smem + L.total);
-  unsigned long long* xs_full = bars;                          // producer: tx bytes
-  unsigned long long* xs_empty = bars + 1;                     // 4 transposer warps
-  unsigned long long* as_full = bars + 2;                      // 4 transposer warps
+  unsigned long long* xs_full = bars;                          // [2] producer: tx bytes
+  unsigned long long* x_free = bars + TC_XBUFS;                // [2] epilogue store thread
+  unsigned long long* as_full = bars + 2 * TC_XBUFS;           // 4 transposer warps
   unsigned long long* as_empty = as_full + TC_ASTAGES;         // epilogue store thread
   unsigned long long* tm_full = as_empty + TC_ASTAGES;         // MMA commit
   unsigned int* tmem_slot = reinterpret_cast<unsigned int*>(tm_full + TC_ASTAGES);
@@ -145,8 +150,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int t_end = (int)((long long)P.num_tiles * (blockIdx.x + 1) / gridDim.x);
 
   if (threadIdx.x == 0) {
-    mbar_init(xs_full, 1);
-    mbar_init(xs_empty, 4);
+    for (int k = 0; k < TC_XBUFS; ++k) {
+      mbar_init(&xs_full[k], 1);
+      mbar_init(&x_free[k], 1);
+    }
     for (int s = 0; s < TC_ASTAGES; ++s) {
       mbar_init(&as_full[s], 4);
       mbar_init(&as_empty[s], 1);
@@ -169,11 +176,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   pdl_wait();
   pdl_launch_dependents();
 
-  unsigned char* xs = smem;
-  unsigned char* ws = smem + L.ws_off;
+  auto xb = [&](int k) { return smem + (size_t)k * L.xbuf; };              // tile buffers
+  auto wsb = [&](int k) { return smem + L.ws_off + (size_t)k * TC_WS_BYTES; };
   auto as = [&](int s) { return smem + L.as_off + (size_t)s * L.astage; };
   auto bs = [&](int s) { return as(s) + L.as_bytes; };
-  unsigned char* os = smem + L.os_off;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -181,23 +187,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const unsigned int wbytes = (unsigned int)(TC_TCH * P.K * 2);
       int n = 0;
       for (int t = t_begin; t < t_end; ++t, ++n) {
-        if (!mbar_wait(xs_empty, ((unsigned int)n & 1u) ^ 1u, abort_flag, err, 256u)) break;
+        const int k = n % TC_XBUFS;
+        // buffer k is free again once the TMA store of tile n - 2 has read it
+        const unsigned int fph = (unsigned int)(n / TC_XBUFS - 1) & 1u;
+        if (n >= TC_XBUFS && !mbar_wait(&x_free[k], fph, abort_flag, err, 256u)) break;
         TileCoord c;
         c.set(P, t);
         const int r0 = c.row0(P);
         unsigned int nbytes = wbytes;
         for (int i = 0; i < L.n_boxes; ++i)
           if (!box_outside(P, r0, i, L.box_h)) nbytes += (unsigned int)L.box_h * 32;
-        mbar_arrive_expect_tx(xs_full, nbytes);
-        bulk_load(ws, w + (size_t)c.ct * TC_TCH * P.K, wbytes, xs_full);
+        mbar_arrive_expect_tx(&xs_full[k], nbytes);
+        bulk_load(wsb(k), w + (size_t)c.ct * TC_TCH * P.K, wbytes, &xs_full[k]);
         for (int i = 0; i < L.n_boxes; ++i)
           if (!box_outside(P, r0, i, L.box_h))
-            tma_load_3d(xs + (size_t)i * L.box_h * 32, &tmx, xs_full, c.ct * TC_TCH,
+            tma_load_3d(xb(k) + (size_t)i * L.box_h * 32, &tmx, &xs_full[k], c.ct * TC_TCH,
                         r0 + L.box_h * i, c.b);
       }
-      // copies in flight must land before the CTA exits
-      if (n > 0)
-        mbar_wait_until(xs_full, (unsigned int)(n - 1) & 1u, drain_deadline(), err, ERR_DRAIN);
+      // copies in flight must land before the CTA exits: the last load into each buffer
+      const unsigned long long dl = drain_deadline();
+      for (int q = (n > TC_XBUFS ? n - TC_XBUFS : 0); q < n; ++q)
+        mbar_wait_until(&xs_full[q % TC_XBUFS], (unsigned int)(q / TC_XBUFS) & 1u, dl, err,
+                        ERR_DRAIN);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -233,13 +244,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // ------------------------------------------------------------ transposes + filter copies
     const int tw = warp - 6, tid = threadIdx.x - 192;
     constexpr int NBLK = L.rows / 8;                 // 8x8 blocks per sub-tile
-    const unsigned short* wt = reinterpret_cast<const unsigned short*>(ws);
-    const unsigned int xsa = smem_u32(xs);
     int n = 0;
     bool ok = true;
     for (int t = t_begin; t < t_end && ok; ++t, ++n) {
-      bool got = mbar_try_wait(xs_full, (unsigned int)n & 1u);
-      if (!got) got = mbar_wait(xs_full, (unsigned int)n & 1u, abort_flag, err, 1024u);
+      const int k = n % TC_XBUFS;
+      const unsigned int xph = (unsigned int)(n / TC_XBUFS) & 1u;
+      const unsigned short* wt = reinterpret_cast<const unsigned short*>(wsb(k));
+      const unsigned int xsa = smem_u32(xb(k));
+      bool got = mbar_try_wait(&xs_full[k], xph);
+      if (!got) got = mbar_wait(&xs_full[k], xph, abort_flag, err, 1024u);
       if (!__all_sync(0xffffffffu, got)) break;
       TileCoord c;
       c.set(P, t);
@@ -300,8 +313,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&as_full[s]);
       }
-      __syncwarp();
-      if (ok && lane == 0) mbar_arrive(xs_empty);
+      // the tile buffer now belongs to the epilogue, which stages the tile's output in it
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-5)
@@ -343,11 +355,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       tc_fence_before();
-      if (h == 0 && store_thread) bulk_wait_read0(); // the previous tile's store has read `os`
+      const int n = u >> 1, k = n % TC_XBUFS;
+      if (h == 0 && n > 0 && store_thread) {
+        bulk_wait_read0();                           // tile n - 1's store has read its buffer
+        mbar_arrive(&x_free[(n - 1) % TC_XBUFS]);    // ... which may take tile n + 1's input
+      }
       named_sync(1, 128);
-      // transposed output -> half h of the [steps][16 ch] rows of the output buffer
+      // transposed output -> half h of the [steps][16 ch] rows in the tile's own buffer, whose
+      // input half h the transpose consumed before this sub-tile's MMAs
       const unsigned int ya = smem_u32(ybuf) + (unsigned int)((lane & 7) * TC_YSTRIDE);
-      const unsigned int oa = smem_u32(os) + (unsigned int)((lane & 7) * 32 + 16 * h);
+      const unsigned int oa = smem_u32(xb(k)) + (unsigned int)((lane & 7) * 32 + 16 * h);
 #pragma unroll 4
       for (int q0 = 4 * ew; q0 < TC_STEPS / 8; q0 += 16) {
         const int q = q0 + (lane >> 3);
@@ -365,7 +382,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const int t0 = c.tc * TC_STEPS;
           for (int i = 0; i < TC_STEPS / 256; ++i)
             if (t0 + 256 * i < P.T_out)
-              tma_store_3d(&tmy, os + (size_t)i * 256 * 32, c.ct * TC_TCH, t0 + 256 * i, c.b);
+              tma_store_3d(&tmy, xb(k) + (size_t)i * 256 * 32, c.ct * TC_TCH, t0 + 256 * i,
+                           c.b);
           bulk_commit();
         }
       }
@@ -412,7 +430,7 @@ cudaError_t launch_tc(const Conv1d& p, const void* x, const void* w, void* y, in
   if (!make_map_rows8(&tmx, p.dtype, x, p.C, T_in, p.B, L.box_h) ||
       !make_map_rows8(&tmy, p.dtype, y, p.C, T_out, p.B, 256))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + (size_t)L.total + 8 * (2 + 3 * TC_ASTAGES) + 16;
+  const size_t smem = 1024 + (size_t)L.total + 8 * (2 * TC_XBUFS + 3 * TC_ASTAGES) + 16;
   static std::atomic<unsigned int> configured{0};
   cudaError_t e = set_max_dynamic_smem((const void*)dwconv1d_tc_kernel<T, KS, FLIP>, smem,
                                        configured);

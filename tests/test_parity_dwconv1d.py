@@ -167,6 +167,24 @@ def test_tensor_core_64ch_integer_bit_exact(case):
     assert np.array_equal(dx, rdx)
 
 
+def test_tensor_core_tile_buffers_reused_bit_exact():
+    """More than two tiles per CTA (4 batches x 3 step chunks x 32 channel tiles = 384 tiles on
+    at most 148 CTAs), so each of a CTA's two tile buffers takes a third tile's input after the
+    store of its first tile has read it. Integer-valued data: fwd and dgrad bit for bit."""
+    p = wl.Dwconv1dProblem(4, 6100, 512, 31, 15, 15, wl.BF16)
+    assert kernel_of(p) == 7
+    inp = wl.make_dwconv1d_inputs(p, 37, "int")
+    inp.w = wl.to_storage(np.random.default_rng(7).integers(-2, 3, (p.C, p.K)), wl.BF16)
+    x, w, dy = (to_dev(a, p.dtype) for a in (inp.x, inp.w, inp.dy))
+    y = gb.dwconv1d_fwd(x, w, p.pad_left, p.pad_right, path=gb.PATH_IGEMM)
+    dx = gb.dwconv1d_bwd_data(dy, w, p.T, p.pad_left, p.pad_right, path=gb.PATH_IGEMM)
+    torch.cuda.synchronize()
+    xf, wf, dyf = (wl.widen(a, p.dtype) for a in (inp.x, inp.w, inp.dy))
+    assert np.array_equal(to_f64(y), oracle.dwconv1d_fwd(xf, wf, p.pad_left, p.pad_right))
+    assert np.array_equal(to_f64(dx),
+                          oracle.dwconv1d_bwd_data(dyf, wf, p.T, p.pad_left, p.pad_right))
+
+
 @pytest.mark.parametrize("case", TC_CASES[:4])
 def test_ring_and_generic_paths_agree_with_oracle(case):
     """The same problems forced onto the CUDA-core kernels (ring where instantiated, generic
